@@ -1,0 +1,7 @@
+"""CPU oracle of the Hadamard-rotated quantized linear layer (test infrastructure only).
+
+Only the test-suite, the smoke check and the benchmark's CPU-baseline leg may
+import this package; the product path never does.
+"""
+from .qs_oracle import *  # noqa: F401,F403
+from .qs_oracle import QMAX, HADAMARD_BLOCK, WEIGHT_SCALE_FOLD  # noqa: F401
