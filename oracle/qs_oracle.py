@@ -258,10 +258,12 @@ def gemm_rows(qa_rows: np.ndarray, qw: np.ndarray) -> np.ndarray:
 
 def gelu_erf_bf16(x_bits: np.ndarray) -> np.ndarray:
     """GELU with the exact erf form, x * Phi(x), evaluated in binary64 and
-    rounded to bf16 (the chain's activation between ffn-up and ffn-down)."""
+    rounded to bf16 (the chain's activation between ffn-up and ffn-down).
+    Phi(x) = erfc(-x / sqrt(2)) / 2, the same function as (1 + erf(x/sqrt(2)))/2
+    without its cancellation for x << 0."""
     x = bf16_bits_to_f32(x_bits).astype(np.float64)
-    erf = np.vectorize(math.erf, otypes=[np.float64])
-    y = 0.5 * x * (1.0 + erf(x / math.sqrt(2.0)))
+    erfc = np.vectorize(math.erfc, otypes=[np.float64])
+    y = 0.5 * x * erfc(-x / math.sqrt(2.0))
     return f32_to_bf16_bits(y.astype(np.float32))
 
 

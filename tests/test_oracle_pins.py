@@ -333,6 +333,14 @@ def pin_gelu(o=O):
     want = torch.nn.functional.gelu(xt, approximate="none").float().to(torch.bfloat16).float().numpy()
     ulp = np.abs(got - want) / np.maximum(np.abs(want), 1e-30)
     assert np.all((got == want) | (ulp <= 2.0 ** -7))
+    # deep negative tail: x*Phi(x) = -phi(x) * (1 - 1/x^2 + 3/x^4 - ...) (Mills ratio
+    # asymptotic series), nonzero and accurate to bf16 where 1 + erf cancels.
+    xt = np.array([-8.0, -10.0, -12.0], np.float32)
+    yt = O.bf16_bits_to_f32(o.gelu_erf_bf16(_bf16(xt))).astype(np.float64)
+    x64 = xt.astype(np.float64)
+    phi = np.exp(-x64 ** 2 / 2) / math.sqrt(2 * math.pi)
+    series = -phi * (1 - 1 / x64 ** 2 + 3 / x64 ** 4 - 15 / x64 ** 6)
+    assert np.all(np.abs(yt - series) <= 2.0 ** -7 * np.abs(series))
 
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
