@@ -1,0 +1,349 @@
+"""Benchmark of the Hadamard-rotated W4A4 quantized linear layer on B200.
+
+One step = one pass of the hot path over one batch: the fused rotate-quantize
+kernel on the bf16 activations (qs_quant_act) followed by the tcgen05 integer
+GEMM with the dequantizing epilogue (qs_qlinear).  The weights are packed once
+beforehand (qs_pack_weights is offline preparation, not part of a step).
+
+Workload: the Wan2.1-14B-like FFN up-projection, M = 32760 tokens,
+K = 5120, N = 13824, W4A4, clip ratio 0.9, seed 2 (synthetic inputs, see
+bit_quantized_linear_hadamard_b200/inputs.py).  The activations (335 MB bf16)
+and the output (906 MB bf16) are larger than the 126 MB L2, so no L2 flush
+is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 it is launched by torchrun, one process per GPU; every rank runs the
+same single-GPU workload (replicas: the layer shards by tokens with no
+collective), the time is the max over ranks, and `value` counts the work of
+all ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A4 qlinear TOPS and tokens/s at Wan-14B FFN shape; % of INT8 peak / HBM"
+UNIT = "TOPS"
+PROFILES = os.path.join(ROOT, "profiles")
+# The dense int8 tensor peak is taken as the measured dense bf16 GEMM peak times
+# the nominal int8:bf16 dense ratio of B200 (4.5 / 2.25 = 2).
+INT8_PER_BF16 = 2.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--tokens", type=int, default=None,
+                   help="override M (profiling captures of a smaller case of the same shape)")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_quantized_linear_hadamard_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, or None if the
+    kernels changed since the counters were taken."""
+    path = os.path.join(PROFILES, "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    k = d.get("kernels", {}).get(kernel)
+    return None if k is None else k.get("dram_bytes_per_launch_full")
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [l.split(", ") for l in out.strip().splitlines() if l.strip()]
+        sm = [float(r[1]) for r in rows if len(r) >= 9 and r[1].replace(".", "").isdigit()]
+        if not sm:
+            return None
+        mx = max(float(r[2]) for r in rows if len(r) >= 9 and r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows if len(r) >= 9 for i in range(4)
+                          if r[5 + i].strip() == "Active"})
+        loaded = [v for v in sm if v > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(sm), "power_w_max": max(float(r[3]) for r in rows
+                                                       if len(r) >= 9 and _isnum(r[3]))}
+
+
+def _isnum(s):
+    try:
+        float(s)
+        return True
+    except ValueError:
+        return False
+
+
+def cpu_baseline(d, bits, alpha, rows: int = 64):
+    """The oracle as it stands, on the host cores, on a bounded sample of the
+    workload: the first `rows` tokens through quant_act + int GEMM + epilogue
+    against the full weight (weight packing is offline and not timed)."""
+    import numpy as np  # noqa: F401
+    from bit_quantized_linear_hadamard_b200 import inputs as I
+    from oracle import qs_oracle as O
+
+    xb = I.bf16_bits(d["x"][:rows])
+    wb = I.bf16_bits(d["w"])
+    bb = I.bf16_bits(d["bias"])
+    qw, sw = O.pack_weights(wb, bits)
+    t0 = time.perf_counter()
+    qa, sa = O.quant_act(xb, bits, alpha)
+    acc = O.int_gemm(qa, qw)
+    O.epilogue(acc, sa, sw, bb)
+    dt = time.perf_counter() - t0
+    K, N = d["x"].shape[1], d["w"].shape[0]
+    ops = 2.0 * rows * N * K
+    return {"value": ops / dt / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"first {rows} of {d['x'].shape[0]} tokens, full K={K}, N={N} "
+                      f"(quant_act + int GEMM + epilogue; numpy, single thread), {dt:.2f} s",
+            "seconds": dt, "tokens_per_s": rows / dt}
+
+
+def run_reference(args, rank, world):
+    """The CPU oracle timed as a bounded sample per step (rank 0 only)."""
+    if rank != 0:
+        return
+    from bit_quantized_linear_hadamard_b200 import inputs as I
+    cfg = I.WAN_FFN
+    d = I.make_layer(cfg, M=256)
+    rows = 16
+    for _ in range(args.warmup):
+        cpu_baseline(d, cfg.bits, cfg.alpha, rows=4)
+    res = [cpu_baseline(d, cfg.bits, cfg.alpha, rows=rows) for _ in range(args.steps)]
+    secs = sum(r["seconds"] for r in res)
+    value = 2.0 * rows * cfg.N * cfg.K * args.steps / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "bits": cfg.bits,
+                   "alpha": cfg.alpha, "seed": cfg.seed, "sample_rows_per_step": rows},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{rows} tokens per step of the {cfg.M}-token workload, full "
+                                   f"K and N, numpy oracle on one host thread"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import bit_quantized_linear_hadamard_b200 as qs
+    from bit_quantized_linear_hadamard_b200 import inputs as I
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    qs.load()
+
+    cfg = I.WAN_FFN
+    d = I.make_layer(cfg, M=args.tokens)
+    M, K, N, bits, alpha = d["x"].shape[0], cfg.K, cfg.N, cfg.bits, cfg.alpha
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        x = d["x"].to(dev)
+        w = d["w"].to(dev)
+        bias = d["bias"].to(dev)
+        wp, ws = qs.pack_weights(w, bits, stream=stream)
+        xp = torch.empty((M, K * bits // 8), dtype=torch.uint8, device=dev)
+        xs = torch.empty((M,), dtype=torch.float32, device=dev)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    stream.synchronize()
+    del w
+
+    def step():
+        qs.qs_quant_act(x, M, K, bits, alpha, 0, xp, xs, stream)
+        qs.qs_qlinear(xp, xs, wp, ws, bias, M, N, K, bits, out, stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    stream.synchronize()
+    if qs.qs_device_error(stream) != 0:
+        raise SystemExit("kernel wait timed out during warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        qs.qs_quant_act(x, M, K, bits, alpha, 0, xp, xs, stream)
+        ev[i][1].record(stream)
+        qs.qs_qlinear(xp, xs, wp, ws, bias, M, N, K, bits, out, stream)
+        ev[i][2].record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        dist.barrier()
+    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    quant_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    gemm_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    if qs.qs_device_error(stream) != 0:
+        raise SystemExit("kernel wait timed out in the timed region")
+
+    t = torch.tensor([total_ms, quant_ms, gemm_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, quant_ms, gemm_ms = t.tolist()
+    ms_per_step = total_ms / args.steps
+    ops_per_step = 2.0 * M * N * K
+    value = ops_per_step * world / (ms_per_step * 1e-3) / 1e12
+
+    # ---- end to end through the same C ABI calls, inputs and result in pinned host memory
+    x_host = d["x"].pin_memory()
+    out_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(1, args.e2e_steps)
+
+    def e2e_step():
+        x.copy_(x_host, non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_step()
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        stream.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+
+    if rank == 0:
+        pk, src = peaks()
+        int8_peak = pk["bf16_tflops"] * INT8_PER_BF16
+        gemm_tops = ops_per_step / (gemm_ms * 1e-3) / 1e12
+        quant_bytes = M * (2 * K + K * bits // 8 + 4)
+        quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT,
+            "tokens_per_s": M * world / (ms_per_step * 1e-3),
+            "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int4", "data": "synthetic",
+            "config": {"workload": cfg.name, "M": M, "K": K, "N": N, "bits": bits, "alpha": alpha,
+                       "seed": cfg.seed, "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (x 335 MB, out 906 MB bf16); no flush"},
+            "roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak,
+                         "unit": UNIT, "frac": gemm_tops / int8_peak,
+                         "traffic": ncu_traffic("qgemm_kernel"),
+                         "kernel": "qgemm_kernel<4,false> (tcgen05 kind::i8)",
+                         "peak_source": f"{src}: bf16_tflops (burst) x {INT8_PER_BF16} "
+                                        f"nominal int8:bf16"},
+            "roofline_quant": {"bound": "hbm", "achieved": quant_gbs, "peak": pk["hbm_gbs"],
+                               "unit": "GB/s", "frac": quant_gbs / pk["hbm_gbs"],
+                               "traffic": ncu_traffic("rotate_quant_kernel"),
+                               "algorithmic_bytes": quant_bytes,
+                               "peak_source": f"{src}: hbm_gbs"},
+            "kernels_ms": {"quant": quant_ms, "gemm": gemm_ms},
+            "gpu_launches": 2 * args.steps,
+            "e2e": {"value": ops_per_step * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                    "h2d_bytes_per_step": x_host.numel() * 2,
+                    "d2h_bytes_per_step": out_host.numel() * 2,
+                    "ms_per_step": e2e_ms, "steps": e2e_steps},
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(d, bits, alpha)
+            line["cpu_baseline"].pop("seconds", None)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,211 @@
+"""ctypes binding of libqs.so.
+
+The functions named like the C entry points (``qs_pack_weights``,
+``qs_quant_act``, ``qs_qlinear``, ``qs_qgemm_s32``, ``qs_gelu_bf16``) take torch
+CUDA tensors and only marshal their pointers, sizes and the stream into the C
+call; every step of the computation runs in the library's kernels.  The
+lower-case helpers (``pack_weights``, ``quant_act``, ``qlinear``, ...) allocate
+the output tensors with torch and call those.
+
+There is no fallback: if libqs.so has not been built, or a call returns an
+error status, a ``QSError`` is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqs.so")
+
+QS_FLAG_NO_ROTATE = 1
+QS_MAX_K = 65536
+STATUS = {0: "QS_OK", 1: "QS_ERR_NULL", 2: "QS_ERR_SHAPE", 3: "QS_ERR_BITS", 4: "QS_ERR_ALIGN",
+          5: "QS_ERR_RANGE", 6: "QS_ERR_CUDA", 7: "QS_ERR_TIMEOUT", 8: "QS_ERR_PTR"}
+EXPORTS = ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qgemm_s32", "qs_gelu_bf16",
+           "qs_device_error", "qs_status_str", "qs_version")
+
+
+class QSError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({_status_str(status)})")
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Loads libqs.so (once) and declares the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is not built; run `python -m bit_quantized_linear_hadamard_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, u32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint, ctypes.c_float
+    L.qs_pack_weights.argtypes = [vp, i64, i64, i32, u32, vp, vp, vp]
+    L.qs_quant_act.argtypes = [vp, i64, i64, i32, f32, u32, vp, vp, vp]
+    L.qs_qlinear.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp, vp]
+    L.qs_qgemm_s32.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp]
+    L.qs_gelu_bf16.argtypes = [vp, i64, vp, vp]
+    L.qs_device_error.argtypes = [vp]
+    L.qs_status_str.argtypes = [i32]
+    L.qs_status_str.restype = ctypes.c_char_p
+    L.qs_version.restype = ctypes.c_char_p
+    for name in ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qgemm_s32",
+                 "qs_gelu_bf16", "qs_device_error"):
+        getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _status_str(status: int) -> str:
+    try:
+        return load().qs_status_str(status).decode()
+    except Exception:  # noqa: BLE001 - only used to decorate an error message
+        return "?"
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise QSError(status, where)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _cuda(t, dtype, name):
+    if t is None:
+        return
+    if not (isinstance(t, torch.Tensor) and t.is_cuda):
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# --------------------------------------------------------------------------- C mirrors
+
+def qs_pack_weights(w, N, K, bits, flags, w_packed, w_scale, stream=None):
+    _cuda(w, torch.bfloat16, "w")
+    _cuda(w_packed, torch.uint8, "w_packed")
+    _cuda(w_scale, torch.float32, "w_scale")
+    _check(load().qs_pack_weights(_p(w), N, K, bits, flags, _p(w_packed), _p(w_scale), _s(stream)),
+           "qs_pack_weights")
+
+
+def qs_quant_act(x, M, K, bits, alpha, flags, x_packed, x_scale, stream=None):
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(x_packed, torch.uint8, "x_packed")
+    _cuda(x_scale, torch.float32, "x_scale")
+    _check(load().qs_quant_act(_p(x), M, K, bits, float(alpha), flags, _p(x_packed), _p(x_scale),
+                               _s(stream)), "qs_quant_act")
+
+
+def qs_qlinear(x_packed, x_scale, w_packed, w_scale, bias, M, N, K, bits, out, stream=None):
+    _cuda(x_packed, torch.uint8, "x_packed")
+    _cuda(w_packed, torch.uint8, "w_packed")
+    _cuda(x_scale, torch.float32, "x_scale")
+    _cuda(w_scale, torch.float32, "w_scale")
+    _cuda(bias, torch.bfloat16, "bias")
+    _cuda(out, torch.bfloat16, "out")
+    _check(load().qs_qlinear(_p(x_packed), _p(x_scale), _p(w_packed), _p(w_scale), _p(bias),
+                             M, N, K, bits, _p(out), _s(stream)), "qs_qlinear")
+
+
+def qs_qgemm_s32(x_packed, w_packed, M, N, K, bits, acc, stream=None):
+    _cuda(x_packed, torch.uint8, "x_packed")
+    _cuda(w_packed, torch.uint8, "w_packed")
+    _cuda(acc, torch.int32, "acc")
+    _check(load().qs_qgemm_s32(_p(x_packed), _p(w_packed), M, N, K, bits, _p(acc), _s(stream)),
+           "qs_qgemm_s32")
+
+
+def qs_gelu_bf16(x, n, y, stream=None):
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(y, torch.bfloat16, "y")
+    _check(load().qs_gelu_bf16(_p(x), n, _p(y), _s(stream)), "qs_gelu_bf16")
+
+
+def qs_device_error(stream=None) -> int:
+    return int(load().qs_device_error(_s(stream)))
+
+
+def qs_version() -> str:
+    return load().qs_version().decode()
+
+
+# --------------------------------------------------------------------------- helpers
+
+def pack_weights(w: torch.Tensor, bits: int, flags: int = 0, stream=None):
+    """w bf16 [N, K] -> (w_packed uint8 [N, K*bits/8], w_scale float32 [N])."""
+    N, K = w.shape
+    wp = torch.empty((N, K * bits // 8), dtype=torch.uint8, device=w.device)
+    ws = torch.empty((N,), dtype=torch.float32, device=w.device)
+    qs_pack_weights(w, N, K, bits, flags, wp, ws, stream)
+    return wp, ws
+
+
+def quant_act(x: torch.Tensor, bits: int, alpha: float = 1.0, flags: int = 0, stream=None,
+              out=None):
+    """x bf16 [M, K] -> (x_packed uint8 [M, K*bits/8], x_scale float32 [M])."""
+    M, K = x.shape
+    if out is None:
+        xp = torch.empty((M, K * bits // 8), dtype=torch.uint8, device=x.device)
+        xs = torch.empty((M,), dtype=torch.float32, device=x.device)
+    else:
+        xp, xs = out
+    qs_quant_act(x, M, K, bits, alpha, flags, xp, xs, stream)
+    return xp, xs
+
+
+def qlinear(x_packed, x_scale, w_packed, w_scale, bias, bits: int, K: int, stream=None, out=None):
+    """Packed activations and weights -> bf16 [M, N]."""
+    M, N = x_packed.shape[0], w_packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x_packed.device)
+    qs_qlinear(x_packed, x_scale, w_packed, w_scale, bias, M, N, K, bits, out, stream)
+    return out
+
+
+def qgemm_s32(x_packed, w_packed, bits: int, K: int, stream=None):
+    M, N = x_packed.shape[0], w_packed.shape[0]
+    acc = torch.empty((M, N), dtype=torch.int32, device=x_packed.device)
+    qs_qgemm_s32(x_packed, w_packed, M, N, K, bits, acc, stream)
+    return acc
+
+
+def gelu(x: torch.Tensor, stream=None, out=None):
+    y = torch.empty_like(x) if out is None else out
+    qs_gelu_bf16(x, x.numel(), y, stream)
+    return y
+
+
+class QuantLinear:
+    """A Hadamard-rotated W4A4 / W8A8 linear layer: weights packed once, each
+    call quantizes the activations (one kernel) and runs the GEMM (one kernel)."""
+
+    def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None, bits: int,
+                 alpha: float = 1.0):
+        self.N, self.K = weight.shape
+        self.bits, self.alpha = bits, alpha
+        self.w_packed, self.w_scale = pack_weights(weight, bits)
+        self.bias = bias
+
+    def __call__(self, x: torch.Tensor, stream=None, out=None) -> torch.Tensor:
+        xp, xs = quant_act(x, self.bits, self.alpha, stream=stream)
+        return qlinear(xp, xs, self.w_packed, self.w_scale, self.bias, self.bits, self.K,
+                       stream=stream, out=out)

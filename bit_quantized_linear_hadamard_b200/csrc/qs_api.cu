@@ -1,0 +1,257 @@
+// libqs.so — C ABI entry points: argument validation, tensor-map set-up and
+// launches of the rotate-quantize kernel, the tcgen05 GEMM and the GELU glue.
+// See include/qs.h for the contract of every function.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "qs.h"
+#include "qs_gemm.cuh"
+#include "qs_glue.cuh"
+#include "qs_quant.cuh"
+
+namespace {
+
+constexpr unsigned kKnownFlags = QS_FLAG_NO_ROTATE;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The pointer must be device (or managed) memory usable by the current device.
+qs_status check_device_ptr(const void* p) {
+  cudaPointerAttributes a;
+  const cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QS_ERR_PTR;
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return QS_ERR_PTR;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QS_ERR_CUDA;
+  if (a.type == cudaMemoryTypeDevice && a.device != dev) return QS_ERR_PTR;
+  return QS_OK;
+}
+
+qs_status check_rows_k(int64_t rows, int64_t K) {
+  if (rows <= 0 || K <= 0 || K % 128 != 0) return QS_ERR_SHAPE;
+  if (K > QS_MAX_K || rows > QS_MAX_ROWS) return QS_ERR_RANGE;
+  return QS_OK;
+}
+
+qs_status check_bits(int bits) { return (bits == 4 || bits == 8) ? QS_OK : QS_ERR_BITS; }
+
+#define QS_TRY(expr)               \
+  do {                             \
+    const qs_status _s = (expr);   \
+    if (_s != QS_OK) return _s;    \
+  } while (0)
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D byte tensor [rows][row_bytes] (row-major), box [box_rows][box_bytes].
+bool make_tensor_map(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows,
+                     uint32_t box_bytes, uint32_t box_rows, bool swizzle128) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_bytes, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 0 || dev >= 64) return 0;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <int BITS, bool OUT_S32>
+qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, const float* sw,
+                       const void* bias, int64_t M, int64_t N, int64_t K, void* out,
+                       cudaStream_t stream) {
+  using C = qs::gemm::Cfg<BITS>;
+  const uint64_t row_bytes = static_cast<uint64_t>(K) * BITS / 8;
+  const uint32_t box_bytes = qs::gemm::BK * BITS / 8;
+  CUtensorMap ta, tb;
+  if (!make_tensor_map(&ta, xp, row_bytes, static_cast<uint64_t>(M), box_bytes, qs::gemm::BM,
+                       BITS == 8) ||
+      !make_tensor_map(&tb, wp, row_bytes, static_cast<uint64_t>(N), box_bytes, qs::gemm::BN,
+                       BITS == 8))
+    return QS_ERR_CUDA;
+  auto kern = qs::gemm::qgemm_kernel<BITS, OUT_S32>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+      cudaSuccess)
+    return QS_ERR_CUDA;
+  const int sms = sm_count();
+  if (sms <= 0) return QS_ERR_CUDA;
+  const int64_t tiles = ((M + qs::gemm::BM - 1) / qs::gemm::BM) *
+                        ((N + qs::gemm::BN - 1) / qs::gemm::BN);
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(
+      ta, tb, sa, sw, static_cast<const uint16_t*>(bias), out, static_cast<int>(M),
+      static_cast<int>(N), static_cast<int>(K));
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status check_gemm_args(const void* xp, const void* wp, const void* out, int64_t M, int64_t N,
+                          int64_t K, int bits) {
+  if (!xp || !wp || !out) return QS_ERR_NULL;
+  QS_TRY(check_bits(bits));
+  QS_TRY(check_rows_k(M, K));
+  QS_TRY(check_rows_k(N, K));
+  if (N % 16 != 0) return QS_ERR_SHAPE;
+  if (M > INT32_MAX || N > INT32_MAX) return QS_ERR_RANGE;
+  if (!aligned16(xp) || !aligned16(wp) || !aligned16(out)) return QS_ERR_ALIGN;
+  return QS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+qs_status qs_pack_weights(const void* w_bf16, int64_t N, int64_t K, int bits, unsigned flags,
+                          void* w_packed, float* w_scale, void* stream) {
+  if (!w_bf16 || !w_packed || !w_scale) return QS_ERR_NULL;
+  QS_TRY(check_bits(bits));
+  QS_TRY(check_rows_k(N, K));
+  if (flags & ~kKnownFlags) return QS_ERR_RANGE;
+  if (!aligned16(w_bf16) || !aligned16(w_packed) || !aligned16(w_scale)) return QS_ERR_ALIGN;
+  QS_TRY(check_device_ptr(w_bf16));
+  QS_TRY(check_device_ptr(w_packed));
+  QS_TRY(check_device_ptr(w_scale));
+  const bool rotate = !(flags & QS_FLAG_NO_ROTATE);
+  // (1/sqrt(128))^2 of the two rotations, exact in binary32.
+  const float scale_mul = rotate ? 0.0078125f : 1.0f;
+  const cudaError_t e = qs::launch_rotate_quant(
+      static_cast<const uint16_t*>(w_bf16), N, static_cast<int>(K), bits, 1.0f, scale_mul,
+      rotate ? 1 : 0, static_cast<uint8_t*>(w_packed), w_scale, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status qs_quant_act(const void* x_bf16, int64_t M, int64_t K, int bits, float alpha,
+                       unsigned flags, void* x_packed, float* x_scale, void* stream) {
+  if (!x_bf16 || !x_packed || !x_scale) return QS_ERR_NULL;
+  QS_TRY(check_bits(bits));
+  QS_TRY(check_rows_k(M, K));
+  if (!(alpha > 0.0f && alpha <= 1.0f)) return QS_ERR_RANGE;
+  if (flags & ~kKnownFlags) return QS_ERR_RANGE;
+  if (!aligned16(x_bf16) || !aligned16(x_packed) || !aligned16(x_scale)) return QS_ERR_ALIGN;
+  QS_TRY(check_device_ptr(x_bf16));
+  QS_TRY(check_device_ptr(x_packed));
+  QS_TRY(check_device_ptr(x_scale));
+  const bool rotate = !(flags & QS_FLAG_NO_ROTATE);
+  const cudaError_t e = qs::launch_rotate_quant(
+      static_cast<const uint16_t*>(x_bf16), M, static_cast<int>(K), bits, alpha, 1.0f,
+      rotate ? 1 : 0, static_cast<uint8_t*>(x_packed), x_scale, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status qs_qlinear(const void* x_packed, const float* x_scale, const void* w_packed,
+                     const float* w_scale, const void* bias_bf16, int64_t M, int64_t N,
+                     int64_t K, int bits, void* out_bf16, void* stream) {
+  QS_TRY(check_gemm_args(x_packed, w_packed, out_bf16, M, N, K, bits));
+  if (!x_scale || !w_scale) return QS_ERR_NULL;
+  if (!aligned16(x_scale) || !aligned16(w_scale) || (bias_bf16 && !aligned16(bias_bf16)))
+    return QS_ERR_ALIGN;
+  QS_TRY(check_device_ptr(x_packed));
+  QS_TRY(check_device_ptr(w_packed));
+  QS_TRY(check_device_ptr(x_scale));
+  QS_TRY(check_device_ptr(w_scale));
+  QS_TRY(check_device_ptr(out_bf16));
+  if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return bits == 4 ? launch_qgemm<4, false>(x_packed, x_scale, w_packed, w_scale, bias_bf16, M, N,
+                                             K, out_bf16, s)
+                   : launch_qgemm<8, false>(x_packed, x_scale, w_packed, w_scale, bias_bf16, M, N,
+                                             K, out_bf16, s);
+}
+
+qs_status qs_qgemm_s32(const void* x_packed, const void* w_packed, int64_t M, int64_t N,
+                       int64_t K, int bits, int32_t* acc, void* stream) {
+  QS_TRY(check_gemm_args(x_packed, w_packed, acc, M, N, K, bits));
+  QS_TRY(check_device_ptr(x_packed));
+  QS_TRY(check_device_ptr(w_packed));
+  QS_TRY(check_device_ptr(acc));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return bits == 4 ? launch_qgemm<4, true>(x_packed, nullptr, w_packed, nullptr, nullptr, M, N, K,
+                                            acc, s)
+                   : launch_qgemm<8, true>(x_packed, nullptr, w_packed, nullptr, nullptr, M, N, K,
+                                            acc, s);
+}
+
+qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream) {
+  if (!x_bf16 || !y_bf16) return QS_ERR_NULL;
+  if (n <= 0) return QS_ERR_SHAPE;
+  if (!aligned16(x_bf16) || !aligned16(y_bf16)) return QS_ERR_ALIGN;
+  QS_TRY(check_device_ptr(x_bf16));
+  QS_TRY(check_device_ptr(y_bf16));
+  const int sms = sm_count();
+  if (sms <= 0) return QS_ERR_CUDA;
+  const int64_t nvec = n / 8;
+  int64_t blocks = (nvec + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  qs::gelu_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(x_bf16), n, static_cast<uint16_t*>(y_bf16));
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status qs_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QS_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, qs::g_error_word, sizeof(word)) != cudaSuccess)
+    return QS_ERR_CUDA;
+  if (word) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(qs::g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+      return QS_ERR_CUDA;
+    return QS_ERR_TIMEOUT;
+  }
+  return QS_OK;
+}
+
+const char* qs_status_str(int status) {
+  switch (status) {
+    case QS_OK: return "ok";
+    case QS_ERR_NULL: return "a required pointer is NULL";
+    case QS_ERR_SHAPE: return "bad shape (need M,N,K > 0, K % 128 == 0, N % 16 == 0)";
+    case QS_ERR_BITS: return "bits must be 4 or 8";
+    case QS_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case QS_ERR_RANGE: return "value out of range (alpha, flags or a size limit)";
+    case QS_ERR_CUDA: return "CUDA call or launch failed";
+    case QS_ERR_TIMEOUT: return "a kernel wait exceeded its bound";
+    case QS_ERR_PTR: return "pointer is not device memory of the current device";
+    default: return "unknown status";
+  }
+}
+
+const char* qs_version(void) { return "qs 0.1.0 sm_100a"; }
+
+}  // extern "C"

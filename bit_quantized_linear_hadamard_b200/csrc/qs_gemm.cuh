@@ -1,0 +1,357 @@
+// Integer tensor-core GEMM with the dequantizing epilogue (tcgen05, sm_100a).
+//
+// The low-bit product of the rotated layer (DVD-Quant "Resumen técnico" §1 and
+// §4: W4A4; §2.C: the 8-bit branch):
+//   acc[m][n] = sum_k q_a[m][k] * q_w[n][k]                       (int32, exact)
+//   out[m][n] = bf16(fl(fl(fl(s_a[m] * s_w[n]) * float(acc)) + bias[n]))
+//
+// Structure: a persistent kernel, one CTA per SM, each CTA walking output
+// tiles of 128 x 256 (n fastest, so the whole packed weight stays in L2 while
+// activation tiles stream once).  Warp roles:
+//   warp 0      TMA producer: packed tiles of x (128 x 128 K) and W (256 x 128 K)
+//   warp 1      TMEM owner and single-thread tcgen05.mma (kind::i8) issuer
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator, scale, bias, bf16 store
+//   warps 6-9   (4-bit only) unpack packed nibbles into the 8-bit operand tiles
+// Two 256-column int32 accumulators in TMEM (all 512 columns) let the epilogue
+// of one tile run under the main loop of the next.
+//
+// 4-bit operands: tcgen05 has no 4-bit integer kind, so each packed 16-byte
+// chunk (32 nibbles = 32 consecutive K elements) is widened in shared memory to
+// 32 bytes: the low nibbles (even elements) as one 16-byte chunk and the high
+// nibbles (odd elements) as the next, each nibble placed in the HIGH half of
+// its byte.  That byte, read as int8, is 16*q exactly, so the tensor core
+// accumulates 256*acc; the epilogue shifts it back (exact).  Both operands get
+// the same K permutation, so every dot product is unchanged.  The widening is
+// one shift and one mask per 4 output bytes.  |16 q| <= 112 keeps 256*acc
+// inside int32 for K <= 65536.
+//
+// 8-bit operands go from global memory to the 128-byte-swizzled operand tiles
+// directly by TMA.
+#pragma once
+
+#include "qs_ptx.cuh"
+
+namespace qs {
+namespace gemm {
+
+constexpr int BM = 128;  // tile rows (tokens)
+constexpr int BN = 256;  // tile columns (output channels)
+constexpr int BK = 128;  // K elements per pipeline stage (= 128 bytes of 8-bit operand)
+constexpr int kTmemCols = 2 * BN;
+
+template <int BITS>
+struct Cfg {
+  static constexpr bool kPacked = BITS == 4;
+  static constexpr int kPkBytesA = BM * BK / 2;  // packed 4-bit tile of x
+  static constexpr int kPkBytesB = BN * BK / 2;  // packed 4-bit tile of W
+  static constexpr int kOpBytesA = BM * BK;      // 8-bit operand tile of x
+  static constexpr int kOpBytesB = BN * BK;      // 8-bit operand tile of W
+  static constexpr int kPkStages = kPacked ? 4 : 0;
+  static constexpr int kOpStages = kPacked ? 2 : 4;
+  static constexpr int kEpiWarps = 4;
+  static constexpr int kUnpackWarps = kPacked ? 4 : 0;
+  static constexpr int kThreads = 32 * (2 + kEpiWarps + kUnpackWarps);
+  static constexpr int kOffOp = 0;
+  static constexpr int kOffPk = kOffOp + kOpStages * (kOpBytesA + kOpBytesB);
+  static constexpr int kOffBar = kOffPk + kPkStages * (kPkBytesA + kPkBytesB);
+  static constexpr int kNumBars = 2 * kPkStages + 2 * kOpStages + 4;
+  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
+  static constexpr int kUnpackChunks = (kPkBytesA + kPkBytesB) / 16;
+  static constexpr int kUnpackThreads = kPacked ? 32 * kUnpackWarps : 1;
+  static constexpr int kChunksPerThread = kPacked ? kUnpackChunks / kUnpackThreads : 0;
+  static_assert(kUnpackChunks % kUnpackThreads == 0, "unpack split");
+};
+
+struct Smem {
+  uint32_t base;  // shared-window address of the 1024-aligned layout
+  uint8_t* ptr;
+  int P, U;
+  __device__ uint32_t pk_full(int s) const { return bar(s); }
+  __device__ uint32_t pk_empty(int s) const { return bar(P + s); }
+  __device__ uint32_t op_full(int s) const { return bar(2 * P + s); }
+  __device__ uint32_t op_empty(int s) const { return bar(2 * P + U + s); }
+  __device__ uint32_t acc_full(int b) const { return bar(2 * P + 2 * U + b); }
+  __device__ uint32_t acc_empty(int b) const { return bar(2 * P + 2 * U + 2 + b); }
+  uint32_t off_bar;
+  __device__ uint32_t bar(int i) const { return base + off_bar + 8u * i; }
+};
+
+struct Problem {
+  int M, N, K;
+  int n_tiles, num_tiles, kblocks;
+  __device__ void tile_origin(int t, int& m0, int& n0) const {
+    m0 = (t / n_tiles) * BM;
+    n0 = (t % n_tiles) * BN;
+  }
+};
+
+template <int BITS>
+__device__ __forceinline__ void producer_role(const Smem& sm, const Problem& pb,
+                                              const CUtensorMap* tmA, const CUtensorMap* tmB,
+                                              volatile int* abort_flag) {
+  using C = Cfg<BITS>;
+  int s = 0;
+  uint32_t ph = 0;
+  for (int t = blockIdx.x; t < pb.num_tiles; t += gridDim.x) {
+    int m0, n0;
+    pb.tile_origin(t, m0, n0);
+    for (int kb = 0; kb < pb.kblocks; ++kb) {
+      if (C::kPacked) {
+        if (!mbar_wait_bounded(sm.pk_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer)) return;
+        const uint32_t dst = sm.base + C::kOffPk + s * (C::kPkBytesA + C::kPkBytesB);
+        mbar_arrive_expect_tx(sm.pk_full(s), C::kPkBytesA + C::kPkBytesB);
+        tma_load_2d(dst, tmA, kb * (BK / 2), m0, sm.pk_full(s));
+        tma_load_2d(dst + C::kPkBytesA, tmB, kb * (BK / 2), n0, sm.pk_full(s));
+        if (++s == C::kPkStages) { s = 0; ph ^= 1u; }
+      } else {
+        if (!mbar_wait_bounded(sm.op_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer)) return;
+        const uint32_t dst = sm.base + C::kOffOp + s * (C::kOpBytesA + C::kOpBytesB);
+        mbar_arrive_expect_tx(sm.op_full(s), C::kOpBytesA + C::kOpBytesB);
+        tma_load_2d(dst, tmA, kb * BK, m0, sm.op_full(s));
+        tma_load_2d(dst + C::kOpBytesA, tmB, kb * BK, n0, sm.op_full(s));
+        if (++s == C::kOpStages) { s = 0; ph ^= 1u; }
+      }
+    }
+  }
+}
+
+// Widens packed 4-bit tiles into 8-bit operand tiles (see the file comment).
+// Packed stage: [x tile 128 rows x 64 B][W tile 256 rows x 64 B], plain rows.
+// Operand stage: [x tile 128 rows x 128 B][W tile 256 rows x 128 B], rows of
+// 128 B with 16-byte chunk c stored at chunk c ^ (row & 7) (128-byte swizzle).
+template <int BITS>
+__device__ __forceinline__ void unpack_role(const Smem& sm, const Problem& pb, int ut,
+                                            volatile int* abort_flag) {
+  using C = Cfg<BITS>;
+  const int lane = ut & 31;
+  int sp = 0, su = 0;
+  uint32_t php = 0, phu = 0;
+  for (int t = blockIdx.x; t < pb.num_tiles; t += gridDim.x) {
+    for (int kb = 0; kb < pb.kblocks; ++kb) {
+      if (!mbar_wait_bounded(sm.pk_full(sp), php, abort_flag, kErrWaitUnpack)) return;
+      if (!mbar_wait_bounded(sm.op_empty(su), phu ^ 1u, abort_flag, kErrWaitUnpack)) return;
+      const uint8_t* pk = sm.ptr + C::kOffPk + sp * (C::kPkBytesA + C::kPkBytesB);
+      uint8_t* op = sm.ptr + C::kOffOp + su * (C::kOpBytesA + C::kOpBytesB);
+#pragma unroll
+      for (int i = 0; i < C::kChunksPerThread; ++i) {
+        const int c = ut + i * C::kUnpackThreads;
+        const uint4 w = *reinterpret_cast<const uint4*>(pk + c * 16);
+        const int r = c >> 2;  // operand row (x rows 0..127, then W rows)
+        const int j = c & 3;   // packed 16-byte chunk within the row's 64 bytes
+        uint4 lo, hi;
+        lo.x = (w.x << 4) & 0xF0F0F0F0u;
+        lo.y = (w.y << 4) & 0xF0F0F0F0u;
+        lo.z = (w.z << 4) & 0xF0F0F0F0u;
+        lo.w = (w.w << 4) & 0xF0F0F0F0u;
+        hi.x = w.x & 0xF0F0F0F0u;
+        hi.y = w.y & 0xF0F0F0F0u;
+        hi.z = w.z & 0xF0F0F0F0u;
+        hi.w = w.w & 0xF0F0F0F0u;
+        uint8_t* rowp = op + r * 128;
+        *reinterpret_cast<uint4*>(rowp + (((2 * j) ^ (r & 7)) << 4)) = lo;
+        *reinterpret_cast<uint4*>(rowp + (((2 * j + 1) ^ (r & 7)) << 4)) = hi;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(sm.op_full(su));
+        mbar_arrive(sm.pk_empty(sp));
+      }
+      if (++sp == C::kPkStages) { sp = 0; php ^= 1u; }
+      if (++su == C::kOpStages) { su = 0; phu ^= 1u; }
+    }
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void mma_role(const Smem& sm, const Problem& pb, uint32_t tmem_base,
+                                         volatile int* abort_flag) {
+  using C = Cfg<BITS>;
+  constexpr uint32_t idesc = idesc_i8(BM, BN);
+  int s = 0;
+  uint32_t ph = 0;
+  int it = 0;
+  for (int t = blockIdx.x; t < pb.num_tiles; t += gridDim.x, ++it) {
+    const int buf = it & 1;
+    const uint32_t aph = (it >> 1) & 1;
+    if (!mbar_wait_bounded(sm.acc_empty(buf), aph ^ 1u, abort_flag, kErrWaitMma)) return;
+    tc_fence_after();
+    const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+    for (int kb = 0; kb < pb.kblocks; ++kb) {
+      if (!mbar_wait_bounded(sm.op_full(s), ph, abort_flag, kErrWaitMma)) return;
+      tc_fence_after();
+      const uint32_t a0 = sm.base + C::kOffOp + s * (C::kOpBytesA + C::kOpBytesB);
+      const uint32_t b0 = a0 + C::kOpBytesA;
+#pragma unroll
+      for (int kk = 0; kk < BK / 32; ++kk)
+        mma_i8(d, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc,
+               (kb | kk) != 0);
+      mma_commit(sm.op_empty(s));
+      if (++s == C::kOpStages) { s = 0; ph ^= 1u; }
+    }
+    mma_commit(sm.acc_full(buf));
+  }
+}
+
+template <int BITS, bool OUT_S32>
+__device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
+                                              uint32_t tmem_base, int quad, int lane,
+                                              const float* __restrict__ sa,
+                                              const float* __restrict__ sw,
+                                              const uint16_t* __restrict__ bias, void* out,
+                                              volatile int* abort_flag) {
+  int it = 0;
+  for (int t = blockIdx.x; t < pb.num_tiles; t += gridDim.x, ++it) {
+    const int buf = it & 1;
+    const uint32_t aph = (it >> 1) & 1;
+    if (!mbar_wait_bounded(sm.acc_full(buf), aph, abort_flag, kErrWaitEpilogue)) return;
+    tc_fence_after();
+    int m0, n0;
+    pb.tile_origin(t, m0, n0);
+    const int row = m0 + 32 * quad + lane;
+    const bool row_ok = row < pb.M;
+    float s_a = 0.f;
+    if (!OUT_S32 && row_ok) s_a = sa[row];
+    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quad) << 16) +
+                           static_cast<uint32_t>(buf * BN);
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int n = n0 + 32 * c;
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(taddr + 32 * c, r);
+      tmem_wait_ld();
+      if (n >= pb.N) continue;  // warp-uniform: whole 32-column chunk past N
+      int32_t acc[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        acc[i] = BITS == 4 ? (static_cast<int32_t>(r[i]) >> 8) : static_cast<int32_t>(r[i]);
+      if (OUT_S32) {
+        int32_t* dst = static_cast<int32_t*>(out) + static_cast<int64_t>(row) * pb.N + n;
+        if (row_ok) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            if (n + 4 * v + 4 <= pb.N)
+              *reinterpret_cast<int4*>(dst + 4 * v) =
+                  make_int4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+        }
+      } else {
+        uint16_t* dst = static_cast<uint16_t*>(out) + static_cast<int64_t>(row) * pb.N + n;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int nv = n + 8 * v;
+          if (nv + 8 > pb.N) break;  // N % 16 == 0: only whole 8-column groups exist
+          const float4 w0 = __ldg(reinterpret_cast<const float4*>(sw + nv));
+          const float4 w1 = __ldg(reinterpret_cast<const float4*>(sw + nv + 4));
+          const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+          uint4 braw = make_uint4(0u, 0u, 0u, 0u);
+          if (bias) braw = __ldg(reinterpret_cast<const uint4*>(bias + nv));
+          const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
+          uint32_t packed[4];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            float y[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float sab = __fmul_rn(s_a, wv[e + h]);
+              const float p = __fmul_rn(sab, __int2float_rn(acc[8 * v + e + h]));
+              const uint32_t bb = h == 0 ? (bw[e >> 1] << 16) : (bw[e >> 1] & 0xFFFF0000u);
+              y[h] = __fadd_rn(p, __uint_as_float(bb));
+            }
+            const __nv_bfloat162 y2 = __floats2bfloat162_rn(y[0], y[1]);
+            packed[e >> 1] = *reinterpret_cast<const uint32_t*>(&y2);
+          }
+          if (row_ok)
+            *reinterpret_cast<uint4*>(dst + 8 * v) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.acc_empty(buf));
+  }
+}
+
+template <int BITS, bool OUT_S32>
+__global__ void __launch_bounds__(Cfg<BITS>::kThreads, 1)
+    qgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const float* __restrict__ sa, const float* __restrict__ sw,
+                 const uint16_t* __restrict__ bias, void* out, int M, int N, int K) {
+  using C = Cfg<BITS>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+  Smem sm;
+  sm.ptr = smem_raw + pad;
+  sm.base = raw + pad;
+  sm.P = C::kPkStages;
+  sm.U = C::kOpStages;
+  sm.off_bar = C::kOffBar;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm.ptr + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm.ptr + C::kOffMisc + 4);
+
+  Problem pb;
+  pb.M = M;
+  pb.N = N;
+  pb.K = K;
+  pb.n_tiles = (N + BN - 1) / BN;
+  pb.num_tiles = ((M + BM - 1) / BM) * pb.n_tiles;
+  pb.kblocks = K / BK;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kPkStages; ++s) {
+      mbar_init(sm.pk_full(s), 1);
+      mbar_init(sm.pk_empty(s), C::kUnpackWarps);
+    }
+    for (int s = 0; s < C::kOpStages; ++s) {
+      mbar_init(sm.op_full(s), C::kPacked ? C::kUnpackWarps : 1);
+      mbar_init(sm.op_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(sm.acc_full(b), 1);
+      mbar_init(sm.acc_empty(b), C::kEpiWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) producer_role<BITS>(sm, pb, &tmA, &tmB, abort_flag);
+  } else if (warp == 1) {
+    if (lane == 0) mma_role<BITS>(sm, pb, tmem_base, abort_flag);
+  } else if (warp < 2 + C::kEpiWarps) {
+    epilogue_role<BITS, OUT_S32>(sm, pb, tmem_base, warp & 3, lane, sa, sw, bias, out, abort_flag);
+  } else {
+    if (C::kPacked) unpack_role<BITS>(sm, pb, threadIdx.x - 32 * (2 + C::kEpiWarps), abort_flag);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    // A wait gave up: give copies and MMAs already in flight time to land
+    // before the tensor memory is released.
+    const unsigned long long t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace gemm
+}  // namespace qs

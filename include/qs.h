@@ -1,0 +1,153 @@
+/*
+ * qs.h — C ABI of libqs.so: the Hadamard-rotated W4A4 / W8A8 quantized linear
+ * layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer follows DVD-Quant ("Data-free Video Diffusion Transformers
+ * Quantization"), "Resumen técnico" §2.B, Auto-scaling Rotated Quantization:
+ * a Hadamard rotation is applied to both activations and weights, and the
+ * quantization scales are computed at run time from the rotated activations
+ * (no calibration data).  The bit widths are W4A4 (§1, §4) or the 8-bit branch
+ * of δ-GBS (§2.C).  Quantities the pages leave open are fixed here as follows:
+ *   - rotation: Sylvester Hadamard of order 128 in natural order,
+ *     H[i][j] = (-1)^popcount(i&j), on consecutive blocks of 128 along K,
+ *     computed as the binary32 butterfly with stages h = 1,2,4,...,64;
+ *   - the 1/sqrt(128) of each rotation is folded into the weight scale
+ *     (both together are the exact factor 2^-7);
+ *   - activations: one scale per token (row) over all of K, clip ratio alpha;
+ *     weights: one scale per output channel (row of W), alpha = 1;
+ *   - s = fl(fl(alpha * amax) / qmax), qmax = 7 (4 bits) or 127 (8 bits);
+ *     q = clamp(round_half_even(fl(u / s)), -qmax, qmax); amax == 0 -> s = 0, q = 0;
+ *   - out = bf16_rne(fl(fl(fl(s_a[m] * s_w[n]) * float(acc[m][n])) + bias[n])),
+ *     acc = sum_k q_a[m][k] * q_w[n][k] exact in int32.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *     16-byte aligned, owned and allocated by the caller.  The library
+ *     allocates no memory and keeps no per-call state.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream); every
+ *     call only enqueues work on it and returns without synchronising.
+ *   - Arguments are validated before anything is launched; a call that
+ *     returns anything but QS_OK has launched nothing.
+ *   - No C++ exception crosses this interface.
+ *
+ * Packed formats (row-major, rows of K*bits/8 bytes)
+ *   - 8 bits: one two's complement byte per element.
+ *   - 4 bits: two's complement nibbles; byte j of a row holds element 2j in
+ *     its low nibble and element 2j+1 in its high nibble.
+ *   Codes are always in [-qmax, qmax].
+ */
+#ifndef QS_H_
+#define QS_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QS_API __attribute__((visibility("default")))
+#else
+#define QS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QS_OK = 0,
+  QS_ERR_NULL = 1,     /* a required pointer is NULL */
+  QS_ERR_SHAPE = 2,    /* M, N or K <= 0, K % 128 != 0, or N % 16 != 0 */
+  QS_ERR_BITS = 3,     /* bits not 4 or 8 */
+  QS_ERR_ALIGN = 4,    /* a pointer is not 16-byte aligned */
+  QS_ERR_RANGE = 5,    /* alpha outside (0, 1], unknown flag bits, or a size above its limit */
+  QS_ERR_CUDA = 6,     /* a CUDA runtime/driver call or a launch failed */
+  QS_ERR_TIMEOUT = 7,  /* a kernel wait exceeded its bound (reported by qs_device_error) */
+  QS_ERR_PTR = 8       /* a pointer is not device memory of the current device */
+} qs_status;
+
+/* Test-only flag: skip the Hadamard rotation (the codes are then taken from the
+ * input values themselves, which makes rounding ties easy to construct). */
+#define QS_FLAG_NO_ROTATE 1u
+
+/* Largest K accepted.  With |q| <= 127 the int32 accumulator cannot overflow
+ * (127^2 * 65536 < 2^31), and the rotate-quantize kernel keeps a whole row in
+ * registers in one pass up to this length. */
+#define QS_MAX_K 65536
+/* Largest M or N accepted (tensor-map coordinates are 32-bit). */
+#define QS_MAX_ROWS 2147483647LL
+
+/*
+ * qs_pack_weights — offline weight preparation.
+ * DVD-Quant §2.B: the Hadamard rotation is applied to the weights as well as
+ * to the activations.  Rotates every row of W along K, quantizes it with its
+ * own scale (one per output channel, alpha = 1) and packs it.
+ *   w_bf16   [N, K] bf16, row-major (torch.nn.Linear layout; y = x W^T + b)
+ *   bits     4 or 8
+ *   flags    0 or QS_FLAG_NO_ROTATE
+ *   w_packed [N, K*bits/8] bytes, written
+ *   w_scale  [N] float, written: s * 2^-7 (or s with QS_FLAG_NO_ROTATE)
+ */
+QS_API qs_status qs_pack_weights(const void* w_bf16, int64_t N, int64_t K, int bits, unsigned flags,
+                          void* w_packed, float* w_scale, void* stream);
+
+/*
+ * qs_quant_act — the fused activation kernel of the hot path.
+ * DVD-Quant §2.B: rotate the activations with the Hadamard matrix, then scale
+ * them with factors computed at run time from the rotated values.  Per token:
+ * 128-point block Walsh-Hadamard transform along K, absmax, scale with clip
+ * ratio alpha, round-half-even, pack.
+ *   x_bf16   [M, K] bf16, row-major
+ *   alpha    clip ratio in (0, 1]
+ *   flags    0 or QS_FLAG_NO_ROTATE
+ *   x_packed [M, K*bits/8] bytes, written
+ *   x_scale  [M] float, written (the per-token scale s_a)
+ */
+QS_API qs_status qs_quant_act(const void* x_bf16, int64_t M, int64_t K, int bits, float alpha,
+                       unsigned flags, void* x_packed, float* x_scale, void* stream);
+
+/*
+ * qs_qlinear — integer tensor-core GEMM with the dequantizing epilogue.
+ * The low-bit product of DVD-Quant's W4A4 (§1, §4) / 8-bit (§2.C) layers:
+ * out[m][n] = bf16(s_a[m] * s_w[n] * sum_k q_a[m][k] q_w[n][k] + bias[n]).
+ *   x_packed, x_scale  from qs_quant_act (same K and bits)
+ *   w_packed, w_scale  from qs_pack_weights (same K and bits)
+ *   bias_bf16          [N] bf16 or NULL (NULL adds +0.0)
+ *   N % 16 == 0 is required; M is arbitrary.
+ *   out_bf16           [M, N] bf16, row-major, written
+ */
+QS_API qs_status qs_qlinear(const void* x_packed, const float* x_scale, const void* w_packed,
+                     const float* w_scale, const void* bias_bf16, int64_t M, int64_t N,
+                     int64_t K, int bits, void* out_bf16, void* stream);
+
+/*
+ * qs_qgemm_s32 — the same GEMM main loop with an int32 epilogue: writes the
+ * exact accumulators acc[m][n] = sum_k q_a[m][k] q_w[n][k] (parity checks).
+ *   acc [M, N] int32, row-major, written.  N % 16 == 0.
+ */
+QS_API qs_status qs_qgemm_s32(const void* x_packed, const void* w_packed, int64_t M, int64_t N,
+                       int64_t K, int bits, int32_t* acc, void* stream);
+
+/*
+ * qs_gelu_bf16 — elementwise GELU (exact erf form, binary32 arithmetic,
+ * bf16 in and out) used between the ffn-up and ffn-down linears of a
+ * transformer block chain.  n elements; x and y may alias.
+ */
+QS_API qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream);
+
+/*
+ * qs_device_error — synchronises `stream`, then returns and clears the
+ * library's device-side error word: QS_OK, QS_ERR_TIMEOUT if a kernel gave up
+ * a bounded wait (its outputs are then undefined), or QS_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+QS_API qs_status qs_device_error(void* stream);
+
+/* Static description of a status code. */
+QS_API const char* qs_status_str(int status);
+
+/* Library version string. */
+QS_API const char* qs_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QS_H_ */

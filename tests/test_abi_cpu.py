@@ -1,0 +1,121 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header
+declares, and rejects bad arguments with the documented status before touching
+the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_quantized_linear_hadamard_b200 import build as qs_build
+from bit_quantized_linear_hadamard_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qs.h")
+
+OK, NULL, SHAPE, BITS, ALIGN, RANGE, CUDA, TIMEOUT, PTR = range(9)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    qs_build.build()
+    return binding.load()
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"QS_API\s+[\w\s\*]+?\b(qs_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert _declared() == sorted(binding.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version(lib):
+    for code in range(9):
+        assert lib.qs_status_str(code)
+    assert b"unknown" in lib.qs_status_str(99)
+    assert b"sm_100a" in lib.qs_version()
+
+
+A = ctypes.c_void_p(0x10000)      # 16-byte aligned fake device addresses:
+B = ctypes.c_void_p(0x20000)      # validation must reject before any use
+C = ctypes.c_void_p(0x30000)
+D = ctypes.c_void_p(0x40000)
+MIS = ctypes.c_void_p(0x10008)    # 8-byte aligned only
+NUL = None
+
+
+def test_pack_weights_validation(lib):
+    f = lib.qs_pack_weights
+    assert f(NUL, 256, 512, 4, 0, B, C, NUL) == NULL
+    assert f(A, 256, 512, 4, 0, NUL, C, NUL) == NULL
+    assert f(A, 256, 512, 4, 0, B, NUL, NUL) == NULL
+    assert f(A, 256, 512, 5, 0, B, C, NUL) == BITS
+    assert f(A, 256, 500, 4, 0, B, C, NUL) == SHAPE
+    assert f(A, 0, 512, 4, 0, B, C, NUL) == SHAPE
+    assert f(A, -3, 512, 4, 0, B, C, NUL) == SHAPE
+    assert f(A, 256, 0, 4, 0, B, C, NUL) == SHAPE
+    assert f(A, 256, 65536 + 128, 4, 0, B, C, NUL) == RANGE
+    assert f(A, 256, 512, 4, 2, B, C, NUL) == RANGE
+    assert f(MIS, 256, 512, 4, 0, B, C, NUL) == ALIGN
+
+
+def test_quant_act_validation(lib):
+    f = lib.qs_quant_act
+    assert f(NUL, 8, 128, 4, 1.0, 0, B, C, NUL) == NULL
+    assert f(A, 8, 128, 3, 1.0, 0, B, C, NUL) == BITS
+    assert f(A, 8, 130, 4, 1.0, 0, B, C, NUL) == SHAPE
+    for alpha in (0.0, -0.5, 1.5, float("nan"), float("inf")):
+        assert f(A, 8, 128, 4, alpha, 0, B, C, NUL) == RANGE, alpha
+    assert f(A, 8, 128, 8, 1.0, 0x10, B, C, NUL) == RANGE
+    assert f(A, 8, 128, 8, 1.0, 0, MIS, C, NUL) == ALIGN
+    assert f(A, 8, 128, 8, 1.0, 0, B, ctypes.c_void_p(0x30004), NUL) == ALIGN
+
+
+def test_qlinear_validation(lib):
+    f = lib.qs_qlinear
+    assert f(NUL, B, C, D, NUL, 8, 256, 128, 4, A, NUL) == NULL
+    assert f(A, NUL, C, D, NUL, 8, 256, 128, 4, B, NUL) == NULL
+    assert f(A, B, C, NUL, NUL, 8, 256, 128, 4, B, NUL) == NULL
+    assert f(A, B, C, D, NUL, 8, 256, 128, 4, NUL, NUL) == NULL
+    assert f(A, B, C, D, NUL, 8, 264, 128, 4, A, NUL) == SHAPE   # N % 16
+    assert f(A, B, C, D, NUL, 8, 256, 192, 4, A, NUL) == SHAPE   # K % 128
+    assert f(A, B, C, D, NUL, 0, 256, 128, 4, A, NUL) == SHAPE
+    assert f(A, B, C, D, NUL, 8, 256, 128, 6, A, NUL) == BITS
+    assert f(A, B, C, D, NUL, 8, 256, 2 * 65536, 8, A, NUL) == RANGE
+    assert f(A, B, C, D, MIS, 8, 256, 128, 4, A, NUL) == ALIGN   # bias
+    assert f(MIS, B, C, D, NUL, 8, 256, 128, 4, A, NUL) == ALIGN
+
+
+def test_qgemm_and_gelu_validation(lib):
+    assert lib.qs_qgemm_s32(NUL, B, 8, 256, 128, 4, C, NUL) == NULL
+    assert lib.qs_qgemm_s32(A, B, 8, 250, 128, 4, C, NUL) == SHAPE
+    assert lib.qs_qgemm_s32(A, B, 8, 256, 128, 2, C, NUL) == BITS
+    assert lib.qs_qgemm_s32(A, B, 8, 256, 128, 4, MIS, NUL) == ALIGN
+    assert lib.qs_gelu_bf16(NUL, 16, B, NUL) == NULL
+    assert lib.qs_gelu_bf16(A, 0, B, NUL) == SHAPE
+    assert lib.qs_gelu_bf16(A, 16, MIS, NUL) == ALIGN
+
+
+def test_host_memory_is_rejected(lib):
+    # Well-formed arguments pointing at host memory: rejected as QS_ERR_PTR (on a
+    # machine without a GPU the pointer query fails the same way).
+    buf = ctypes.create_string_buffer(4096 + 16)
+    base = (ctypes.addressof(buf) + 15) // 16 * 16
+    p = ctypes.c_void_p(base)
+    st = lib.qs_quant_act(p, 1, 128, 4, 1.0, 0, ctypes.c_void_p(base + 1024),
+                          ctypes.c_void_p(base + 2048), NUL)
+    assert st == PTR
+
+
+def test_binding_raises_without_cuda_tensors():
+    import torch
+    with pytest.raises(TypeError):
+        binding.quant_act(torch.zeros(4, 128, dtype=torch.bfloat16), 4)

@@ -1,0 +1,280 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Bar (stated by the layer's targets): packed codes, scales and int32
+accumulators bit-identical; bf16 outputs within 1 bf16 ulp (ordered bit
+patterns).  Inputs are the seeded synthetic tensors; no expected value comes
+from the CUDA path.  Full-size configurations run in the benchmark's launch
+configuration and are checked on sampled rows and columns.
+"""
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import bit_quantized_linear_hadamard_b200 as qs
+from bit_quantized_linear_hadamard_b200 import build as qs_build
+from bit_quantized_linear_hadamard_b200 import inputs as I
+from oracle import qs_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    qs_build.build()
+    qs.load()
+    yield
+    assert qs.qs_device_error() == 0, "a kernel reported a bounded-wait timeout"
+
+
+def bits16(t):
+    return I.bf16_bits(t.cpu())
+
+
+def ordered(b):
+    b = np.asarray(b, dtype=np.int32)
+    mag = b & 0x7FFF
+    return np.where(b & 0x8000, -mag, mag)
+
+
+def assert_within_1ulp(got_bits, want_bits, what=""):
+    d = np.abs(ordered(got_bits) - ordered(want_bits))
+    assert d.max(initial=0) <= 1, f"{what}: max bf16 ulp distance {d.max()} at {np.argmax(d)}"
+    return float((d == 0).mean()) if d.size else 1.0
+
+
+def gpu_quant(x, bits, alpha, flags=0):
+    xp, xs = qs.quant_act(x.cuda(), bits, alpha, flags)
+    torch.cuda.synchronize()
+    return xp.cpu().numpy(), xs.cpu().numpy()
+
+
+def gpu_pack(w, bits, flags=0):
+    wp, ws = qs.pack_weights(w.cuda(), bits, flags)
+    torch.cuda.synchronize()
+    return wp.cpu().numpy(), ws.cpu().numpy()
+
+
+def check_quant(x, bits, alpha, flags=0):
+    xp, xs = gpu_quant(x, bits, alpha, flags)
+    q, s = O.quant_act(bits16(x), bits, alpha, rotate=not (flags & qs.QS_FLAG_NO_ROTATE))
+    assert np.array_equal(xs.view(np.uint32), s.view(np.uint32)), "scales differ"
+    want = O.pack(q, bits)
+    if not np.array_equal(xp, want):
+        bad = np.argwhere(xp != want)
+        raise AssertionError(f"packed codes differ at {len(bad)} bytes, first {bad[:5].tolist()}")
+
+
+# --------------------------------------------------------------------------- rotate-quantize
+
+QUANT_SHAPES = [(1, 128), (3, 256), (129, 640), (64, 3072), (33, 5120), (17, 13824),
+                (5, 16384), (3, 16512), (2, 65536)]
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,K", QUANT_SHAPES)
+def test_quant_act_bit_exact(M, K, bits):
+    d = I.make_shape(seed=100 + M + K, M=M, K=K, N=16, bits=bits, outlier_factor=50.0)
+    for alpha in (1.0, 0.9):
+        check_quant(d["x"], bits, alpha)
+
+
+def test_quant_act_tiny_config():
+    d = I.make_layer(I.TINY)
+    check_quant(d["x"], 4, 1.0)
+
+
+def test_quant_ties_without_rotation():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "rne_ties_w4.txt"))
+            if l.strip() and not l.startswith("#")]
+    x = torch.zeros(2, 128)
+    want = np.zeros((2, 128), np.int8)
+    for r, c, v, q in rows:
+        x[int(r), int(c)] = float(v)
+        want[int(r), int(c)] = int(q)
+    xp, xs = gpu_quant(x.to(torch.bfloat16), 4, 1.0, qs.QS_FLAG_NO_ROTATE)
+    assert xs.tolist() == [1.0, 0.5]
+    assert np.array_equal(O.unpack(xp, 4), want)
+
+
+def test_quant_zero_tiny_and_constant_rows():
+    x = torch.zeros(6, 512)
+    x[1] = 1e-38            # binary32 subnormal range after rotation
+    x[2, 7] = -3.0
+    x[3] = 2.5              # constant row: one nonzero per Hadamard block
+    x[4, ::3] = 1e30
+    x[5] = torch.linspace(-4, 4, 512)
+    xb = x.to(torch.bfloat16)
+    for bits in (4, 8):
+        for alpha in (1.0, 0.5, 1e-3):
+            check_quant(xb, bits, alpha)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_pack_weights_bit_exact(bits):
+    d = I.make_layer(I.TINY)
+    wp, ws = gpu_pack(d["w"], bits)
+    q, s = O.pack_weights(bits16(d["w"]), bits)
+    assert np.array_equal(ws.view(np.uint32), s.view(np.uint32))
+    assert np.array_equal(wp, O.pack(q, bits))
+    wp, ws = gpu_pack(d["w"], bits, qs.QS_FLAG_NO_ROTATE)
+    q, s = O.pack_weights(bits16(d["w"]), bits, rotate=False)
+    assert np.array_equal(ws.view(np.uint32), s.view(np.uint32))
+    assert np.array_equal(wp, O.pack(q, bits))
+
+
+# --------------------------------------------------------------------------- integer GEMM
+
+GEMM_SHAPES = [(256, 512, 512), (1, 16, 128), (127, 272, 256), (129, 256, 384),
+               (300, 768, 640), (64, 16, 1024), (513, 528, 1152), (200, 1040, 128)]
+
+
+def _codes(rng, shape, bits):
+    qm = O.QMAX[bits]
+    return rng.integers(-qm, qm + 1, size=shape).astype(np.int8)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_qgemm_s32_bit_exact_on_oracle_codes(M, N, K, bits):
+    rng = np.random.default_rng(M * 7 + N * 3 + K + bits)
+    qa, qw = _codes(rng, (M, K), bits), _codes(rng, (N, K), bits)
+    xp = torch.from_numpy(O.pack(qa, bits)).cuda()
+    wp = torch.from_numpy(O.pack(qw, bits)).cuda()
+    acc = qs.qgemm_s32(xp, wp, bits, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.int_gemm(qa, qw))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_qgemm_s32_extreme_codes_at_max_k(bits):
+    K, qm = 65536, O.QMAX[bits]
+    qa = np.full((3, K), qm, np.int8)
+    qa[1] = -qm
+    qa[2, ::2] = -qm
+    qw = np.full((16, K), -qm, np.int8)
+    qw[5] = qm
+    acc = qs.qgemm_s32(torch.from_numpy(O.pack(qa, bits)).cuda(),
+                       torch.from_numpy(O.pack(qw, bits)).cuda(), bits, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.int_gemm(qa, qw))
+
+
+# --------------------------------------------------------------------------- whole layer
+
+def run_layer(d, bits, alpha, bias=True):
+    x, w, b = d["x"].cuda(), d["w"].cuda(), d["bias"].cuda() if bias else None
+    wp, ws = qs.pack_weights(w, bits)
+    xp, xs = qs.quant_act(x, bits, alpha)
+    out = qs.qlinear(xp, xs, wp, ws, b, bits, x.shape[1])
+    acc = qs.qgemm_s32(xp, wp, bits, x.shape[1])
+    torch.cuda.synchronize()
+    return {"out": out, "acc": acc, "xp": xp, "xs": xs, "wp": wp, "ws": ws}
+
+
+@pytest.mark.parametrize("bits,alpha", [(4, 1.0), (4, 0.9), (8, 1.0)])
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_qlinear_matches_oracle(M, N, K, bits, alpha):
+    d = I.make_shape(seed=M + N + K, M=M, K=K, N=N, bits=bits, alpha=alpha, outlier_factor=50.0)
+    g = run_layer(d, bits, alpha)
+    r = O.qlinear(bits16(d["x"]), bits16(d["w"]), bits16(d["bias"]), bits, alpha)
+    assert np.array_equal(g["xp"].cpu().numpy(), r["xp"])
+    assert np.array_equal(g["wp"].cpu().numpy(), r["wp"])
+    assert np.array_equal(g["acc"].cpu().numpy().astype(np.int64), r["acc"])
+    got = g["out"].view(torch.int16).cpu().numpy().view(np.uint16)
+    exact = assert_within_1ulp(got, r["out"], f"{M}x{N}x{K} w{bits}")
+    assert exact == 1.0, f"only {exact:.6f} of outputs bit-identical"
+
+
+def test_qlinear_null_bias_and_zero_rows():
+    d = I.make_shape(seed=5, M=130, K=256, N=272, bits=4)
+    d["x"][3] = 0
+    d["x"][129] = 0
+    g = run_layer(d, 4, 1.0, bias=False)
+    r = O.qlinear(bits16(d["x"]), bits16(d["w"]), None, 4, 1.0)
+    got = g["out"].view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, r["out"])
+    assert not got[3].any() and not got[129].any()
+
+
+def test_tiny_config_full_parity():
+    d = I.make_layer(I.TINY)
+    g = run_layer(d, 4, 1.0)
+    r = O.qlinear(bits16(d["x"]), bits16(d["w"]), bits16(d["bias"]), 4, 1.0)
+    assert np.array_equal(g["acc"].cpu().numpy().astype(np.int64), r["acc"])
+    got = g["out"].view(torch.int16).cpu().numpy().view(np.uint16)
+    assert assert_within_1ulp(got, r["out"], "tiny") == 1.0
+
+
+def test_gelu_matches_oracle():
+    x = (torch.randn(4097, generator=torch.Generator().manual_seed(9)) * 3).to(torch.bfloat16)
+    y = qs.gelu(x.cuda())
+    torch.cuda.synchronize()
+    got = y.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert_within_1ulp(got, O.gelu_erf_bf16(bits16(x)), "gelu")
+
+
+# --------------------------------------------------------------------------- full-size configs
+
+def _sampled_parity(d, bits, alpha, rows, cols):
+    g = run_layer(d, bits, alpha)
+    xb, wb, bb = bits16(d["x"][rows]), bits16(d["w"][cols]), bits16(d["bias"][cols])
+    qa, sa = O.quant_act(xb, bits, alpha)
+    qw, sw = O.pack_weights(wb, bits)
+    assert np.array_equal(g["xs"].cpu().numpy()[rows].view(np.uint32), sa.view(np.uint32))
+    assert np.array_equal(g["xp"].cpu().numpy()[rows], O.pack(qa, bits))
+    assert np.array_equal(g["ws"].cpu().numpy()[cols].view(np.uint32), sw.view(np.uint32))
+    assert np.array_equal(g["wp"].cpu().numpy()[cols], O.pack(qw, bits))
+    acc = O.int_gemm(qa, qw)
+    gacc = g["acc"].cpu().numpy()[np.ix_(rows, cols)].astype(np.int64)
+    assert np.array_equal(gacc, acc)
+    out = O.epilogue(acc, sa, sw, bb)
+    got = g["out"].view(torch.int16).cpu().numpy().view(np.uint16)[np.ix_(rows, cols)]
+    assert assert_within_1ulp(got, out, "sampled") == 1.0
+    return g
+
+
+def _samples(M, N, seed):
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, 1, M // 2, M - 129, M - 2, M - 1],
+                                     rng.choice(M, 90, replace=False)]))
+    cols = np.unique(np.concatenate([[0, 255, 256, N - 257, N - 1], rng.choice(N, 120, replace=False)]))
+    return rows, cols
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg", [I.HY_QKV, I.WAN_FFN, I.WAN_FFN_W8], ids=lambda c: c.name)
+def test_full_size_config_sampled(cfg):
+    d = I.make_layer(cfg)
+    rows, cols = _samples(cfg.M, cfg.N, cfg.seed)
+    _sampled_parity(d, cfg.bits, cfg.alpha, rows, cols)
+
+
+@pytest.mark.slow
+def test_block_chain_full_size_sampled():
+    ch = I.make_chain(I.WAN_CHAIN)
+    alpha = ch["alpha"]
+    up_out = None
+    for i, L in enumerate(ch["layers"]):
+        bits = L["bits"]
+        if i < 3:
+            x = L["x"]
+        else:
+            xg = qs.gelu(up_out)
+            torch.cuda.synchronize()
+            rows = np.random.default_rng(7).choice(xg.shape[0], 64, replace=False)
+            gb = xg.view(torch.int16).cpu().numpy().view(np.uint16)
+            ub = up_out.view(torch.int16).cpu().numpy().view(np.uint16)
+            assert_within_1ulp(gb[rows], O.gelu_erf_bf16(ub[rows]), "gelu")
+            x = xg.cpu()
+        d = {"x": x, "w": L["w"], "bias": L["bias"]}
+        rows, cols = _samples(x.shape[0], L["N"], 40 + i)
+        g = _sampled_parity(d, bits, alpha, rows, cols)
+        if L["name"] == "ffn_up":
+            up_out = g["out"]
