@@ -28,10 +28,13 @@ The pages leave the details open; the readings taken here are:
 * Scale granularity: one scale per token (row of x) over the whole K row for
   activations, one per output channel (row of W) for weights.  A per-K-channel
   activation scale could not be factored out of an integer dot product over K.
-* Scale: s = fl(fl(alpha * amax) / qmax), qmax = 2^(b-1) - 1 (7 or 127),
-  symmetric range [-qmax, qmax] (-8 / -128 never produced).  amax == 0, or a
-  scale that underflows to 0, gives s = 0 and all-zero codes.
-* Quantise: q = clamp(rint_half_even(fl(u / s)), -qmax, qmax), IEEE division.
+* Scale: with t = fl(alpha * amax), the dequantisation scale is
+  s = fl(t / qmax) and the quantisation multiplier is inv = fl(qmax / t), both
+  computed once per row by IEEE division; qmax = 2^(b-1) - 1 (7 or 127),
+  symmetric range [-qmax, qmax] (-8 / -128 never produced).  A row with
+  t < 2^-120 (all-zero, or so small that qmax / t would overflow binary32) is
+  a zero row: s = 0 and all codes 0.
+* Quantise: q = clamp(rint_half_even(fl(u * inv)), -qmax, qmax).
 * Pack: row-major, int8 as two's complement bytes; int4 as two's complement
   nibbles, element 2j in the low nibble and element 2j+1 in the high nibble of
   byte j.
@@ -117,25 +120,33 @@ def fwht128_blocks(x: np.ndarray) -> np.ndarray:
 # Online per-token scaling and quantisation (ARQ scales from rotated values)
 # ---------------------------------------------------------------------------
 
-def row_scales(u: np.ndarray, bits: int, alpha: float) -> np.ndarray:
-    """s = fl(fl(alpha * amax) / qmax) per row of the rotated values u."""
+# Rows whose clipped absmax t is below this are zero rows (qmax / t must stay finite).
+ZERO_ROW_T = np.float32(2.0 ** -120)
+
+
+def row_scales(u: np.ndarray, bits: int, alpha: float) -> tuple[np.ndarray, np.ndarray]:
+    """Per row of the rotated values u: (s, inv) with t = fl(alpha * amax),
+    s = fl(t / qmax) (dequantisation) and inv = fl(qmax / t) (quantisation).
+    Zero rows (t < 2^-120) get s = 0 and inv = 0."""
     if bits not in QMAX:
         raise ValueError("bits must be 4 or 8")
-    amax = np.max(np.abs(u), axis=1).astype(np.float32)
-    t = np.float32(alpha) * amax
-    return (t / np.float32(QMAX[bits])).astype(np.float32)
-
-
-def quantize_with_scale(u: np.ndarray, s: np.ndarray, bits: int) -> np.ndarray:
-    """q = clamp(rint_half_even(fl(u / s)), -qmax, qmax); s == 0 rows give 0."""
     qmax = np.float32(QMAX[bits])
-    s = np.asarray(s, dtype=np.float32)
-    zero = s == 0
-    safe = np.where(zero, np.float32(1), s).astype(np.float32)
-    r = u / safe[:, None]
+    amax = np.max(np.abs(u), axis=1).astype(np.float32)
+    t = (np.float32(alpha) * amax).astype(np.float32)
+    zero = t < ZERO_ROW_T
+    safe_t = np.where(zero, np.float32(1), t).astype(np.float32)
+    s = np.where(zero, np.float32(0), t / qmax).astype(np.float32)
+    inv = np.where(zero, np.float32(0), qmax / safe_t).astype(np.float32)
+    return s, inv
+
+
+def quantize_with_scale(u: np.ndarray, inv: np.ndarray, bits: int) -> np.ndarray:
+    """q = clamp(rint_half_even(fl(u * inv)), -qmax, qmax); zero rows (inv == 0) give 0."""
+    qmax = np.float32(QMAX[bits])
+    inv = np.asarray(inv, dtype=np.float32)
+    r = u * inv[:, None]
     q = np.rint(r)
     q = np.minimum(np.maximum(q, -qmax), qmax)
-    q[zero, :] = 0
     return q.astype(np.int8)
 
 
@@ -152,8 +163,8 @@ def quantize_rows(x_bits: np.ndarray, bits: int, alpha: float,
     if not (0.0 < alpha <= 1.0):
         raise ValueError("alpha must be in (0, 1]")
     u = fwht128_blocks(x) if rotate else x.copy()
-    s = row_scales(u, bits, alpha)
-    return quantize_with_scale(u, s, bits), s
+    s, inv = row_scales(u, bits, alpha)
+    return quantize_with_scale(u, inv, bits), s
 
 
 def quant_act(x_bits, bits: int, alpha: float, rotate: bool = True):

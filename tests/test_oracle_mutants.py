@@ -29,15 +29,11 @@ def _fwht_with(stage_fn, stages=(1, 2, 4, 8, 16, 32, 64)):
 
 
 def _quantize_with(round_fn=np.rint, lo_extra=0):
-    def f(u, s, bits):
+    def f(u, inv, bits):
         qmax = np.float32(O.QMAX[bits])
-        s = np.asarray(s, dtype=np.float32)
-        zero = s == 0
-        safe = np.where(zero, np.float32(1), s).astype(np.float32)
-        r = u / safe[:, None]
+        r = u * np.asarray(inv, dtype=np.float32)[:, None]
         q = round_fn(r)
         q = np.minimum(np.maximum(q, -qmax - lo_extra), qmax)
-        q[zero, :] = 0
         return q.astype(np.int8)
     return f
 
@@ -45,9 +41,12 @@ def _quantize_with(round_fn=np.rint, lo_extra=0):
 def _scales_with(alpha_used=True, div=None):
     def f(u, bits, alpha):
         amax = np.max(np.abs(u), axis=1).astype(np.float32)
-        t = (np.float32(alpha) if alpha_used else np.float32(1)) * amax
+        t = ((np.float32(alpha) if alpha_used else np.float32(1)) * amax).astype(np.float32)
         d = np.float32(O.QMAX[bits] if div is None else div(bits))
-        return (t / d).astype(np.float32)
+        zero = t == 0
+        safe = np.where(zero, np.float32(1), t)
+        return (np.where(zero, 0, t / d).astype(np.float32),
+                np.where(zero, 0, d / safe).astype(np.float32))
     return f
 
 
@@ -56,8 +55,8 @@ def _per_block_quantize_rows(x_bits, bits, alpha, rotate=True):
     u = O.fwht128_blocks(x) if rotate else x.copy()
     R, K = u.shape
     ub = u.reshape(R * (K // 128), 128)
-    s = O.row_scales(ub, bits, alpha)
-    q = O.quantize_with_scale(ub, s, bits).reshape(R, K)
+    s, inv = O.row_scales(ub, bits, alpha)
+    q = O.quantize_with_scale(ub, inv, bits).reshape(R, K)
     return q, s.reshape(R, K // 128)[:, 0].copy()
 
 

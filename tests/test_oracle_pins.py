@@ -109,7 +109,9 @@ def pin_quant_error_bound(o=O):
             deq = q.astype(np.float64) * s64
             unclipped = np.abs(u) <= qmax * s64
             err = np.abs(u - deq)
-            bound = s64 / 2 + s64 * 2.0 ** -20
+            # r = fl(u * fl(qmax / t)) carries 3 roundings relative to u / s, each
+            # at most 2^-24 relative, and |u / s| <= qmax / alpha (plus rounding).
+            bound = s64 / 2 + s64 * (qmax / alpha + 1) * 2.0 ** -22
             assert np.all(err[unclipped] <= np.broadcast_to(bound, err.shape)[unclipped]), (bits, alpha)
             clipped = ~unclipped
             assert np.all(np.abs(q[clipped]) == qmax), "clipped values saturate"
@@ -151,6 +153,14 @@ def pin_zero_row(o=O):
     r = o.qlinear(x, w, b, 4, 1.0)
     assert r["sa"][0] == 0 and not r["qa"][0].any()
     assert np.array_equal(r["out"][0], b), "a zero token gives exactly the bias"
+    # below the zero-row threshold (alpha*amax < 2^-120) codes are 0; just above it
+    # the single nonzero input spreads to +-amax everywhere and every code is +-qmax
+    tiny = np.zeros((2, 128), np.float32)
+    tiny[0, 3] = 2.0 ** -125
+    tiny[1, 3] = 2.0 ** -110
+    q, s = o.quant_act(_bf16(tiny), 4, 1.0)
+    assert s[0] == 0 and not q[0].any()
+    assert s[1] > 0 and np.all(np.abs(q[1]) == 7)
 
 
 # --------------------------------------------------------------------------- packing
@@ -256,12 +266,14 @@ def pin_scalar_loop_tiny(o=O):
                 h *= 2
             v[blk * 128:(blk + 1) * 128] = seg
         amax = max(abs(t) for t in v)
-        s = _fp32(_fp32(_fp32(a) * amax) / qmax)
-        if s == 0:
+        tt = _fp32(_fp32(a) * amax)
+        if tt < 2.0 ** -120:
             return [0] * K, 0.0
+        s = _fp32(tt / qmax)
+        inv = _fp32(qmax / tt)
         qs = []
         for t in v:
-            r = _fp32(t / s)
+            r = _fp32(t * inv)
             qi = round(r)  # Python round is half-to-even
             qs.append(max(-qmax, min(qmax, qi)))
         return qs, _fp32(s * fold)
