@@ -138,29 +138,37 @@ def _isnum(s):
         return False
 
 
-def cpu_baseline(d, bits, alpha, rows: int = 64):
+class OracleSample:
     """The oracle as it stands, on the host cores, on a bounded sample of the
-    workload: the first `rows` tokens through quant_act + int GEMM + epilogue
-    against the full weight (weight packing is offline and not timed)."""
-    import numpy as np  # noqa: F401
-    from bit_quantized_linear_hadamard_b200 import inputs as I
-    from oracle import qs_oracle as O
+    workload: `rows` tokens through quant_act + int GEMM + epilogue against
+    the full weight (weight packing is offline, done once and not timed)."""
 
-    xb = I.bf16_bits(d["x"][:rows])
-    wb = I.bf16_bits(d["w"])
-    bb = I.bf16_bits(d["bias"])
-    qw, sw = O.pack_weights(wb, bits)
-    t0 = time.perf_counter()
-    qa, sa = O.quant_act(xb, bits, alpha)
-    acc = O.int_gemm(qa, qw)
-    O.epilogue(acc, sa, sw, bb)
-    dt = time.perf_counter() - t0
-    K, N = d["x"].shape[1], d["w"].shape[0]
-    ops = 2.0 * rows * N * K
-    return {"value": ops / dt / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"first {rows} of {d['x'].shape[0]} tokens, full K={K}, N={N} "
-                      f"(quant_act + int GEMM + epilogue; numpy, single thread), {dt:.2f} s",
-            "seconds": dt, "tokens_per_s": rows / dt}
+    def __init__(self, d, bits, alpha):
+        from bit_quantized_linear_hadamard_b200 import inputs as I
+        from oracle import qs_oracle as O
+        self.O, self.bits, self.alpha = O, bits, alpha
+        self.x = d["x"]
+        self.qw, self.sw = O.pack_weights(I.bf16_bits(d["w"]), bits)
+        self.bb = I.bf16_bits(d["bias"])
+        self.bf16_bits = I.bf16_bits
+        self.K, self.N = d["x"].shape[1], d["w"].shape[0]
+
+    def run(self, rows: int) -> float:
+        xb = self.bf16_bits(self.x[:rows])
+        t0 = time.perf_counter()
+        qa, sa = self.O.quant_act(xb, self.bits, self.alpha)
+        acc = self.O.int_gemm(qa, self.qw)
+        self.O.epilogue(acc, sa, self.sw, self.bb)
+        return time.perf_counter() - t0
+
+    def baseline(self, rows: int = 128) -> dict:
+        dt = self.run(rows)
+        ops = 2.0 * rows * self.N * self.K
+        return {"value": ops / dt / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+                "sample": f"first {rows} of {self.x.shape[0]} tokens, full K={self.K}, "
+                          f"N={self.N} (quant_act + int GEMM + epilogue; numpy, one host "
+                          f"thread), {dt:.2f} s",
+                "tokens_per_s": rows / dt}
 
 
 def run_reference(args, rank, world):
@@ -170,11 +178,11 @@ def run_reference(args, rank, world):
     from bit_quantized_linear_hadamard_b200 import inputs as I
     cfg = I.WAN_FFN
     d = I.make_layer(cfg, M=256)
-    rows = 16
+    sample = OracleSample(d, cfg.bits, cfg.alpha)
+    rows = 8
     for _ in range(args.warmup):
-        cpu_baseline(d, cfg.bits, cfg.alpha, rows=4)
-    res = [cpu_baseline(d, cfg.bits, cfg.alpha, rows=rows) for _ in range(args.steps)]
-    secs = sum(r["seconds"] for r in res)
+        sample.run(2)
+    secs = sum(sample.run(rows) for _ in range(args.steps))
     value = 2.0 * rows * cfg.N * cfg.K * args.steps / secs / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
@@ -337,8 +345,7 @@ def main():
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(d, bits, alpha)
-            line["cpu_baseline"].pop("seconds", None)
+            line["cpu_baseline"] = OracleSample(d, bits, alpha).baseline()
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -55,7 +55,8 @@ struct Cfg {
   static constexpr int kOffPk = kOffOp + kOpStages * (kOpBytesA + kOpBytesB);
   static constexpr int kOffBar = kOffPk + kPkStages * (kPkBytesA + kPkBytesB);
   static constexpr int kNumBars = 2 * kPkStages + 2 * kOpStages + 4;
-  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+  static constexpr int kOffEpi = (kOffBar + 8 * kNumBars + 15) / 16 * 16;  // s_w, bias of a tile
+  static constexpr int kOffMisc = kOffEpi + 2 * BN * 4;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
   static constexpr int kUnpackChunks = (kPkBytesA + kPkBytesB) / 16;
   static constexpr int kUnpackThreads = kPacked ? 32 * kUnpackWarps : 1;
@@ -133,10 +134,15 @@ __device__ __forceinline__ void unpack_role(const Smem& sm, const Problem& pb, i
       if (!mbar_wait_bounded(sm.op_empty(su), phu ^ 1u, abort_flag, kErrWaitUnpack)) return;
       const uint8_t* pk = sm.ptr + C::kOffPk + sp * (C::kPkBytesA + C::kPkBytesB);
       uint8_t* op = sm.ptr + C::kOffOp + su * (C::kOpBytesA + C::kOpBytesB);
+      // all loads first: they are independent of the stores that follow
+      uint4 wv[C::kChunksPerThread > 0 ? C::kChunksPerThread : 1];
+#pragma unroll
+      for (int i = 0; i < C::kChunksPerThread; ++i)
+        wv[i] = *reinterpret_cast<const uint4*>(pk + (ut + i * C::kUnpackThreads) * 16);
 #pragma unroll
       for (int i = 0; i < C::kChunksPerThread; ++i) {
         const int c = ut + i * C::kUnpackThreads;
-        const uint4 w = *reinterpret_cast<const uint4*>(pk + c * 16);
+        const uint4 w = wv[i];
         const int r = c >> 2;  // operand row (x rows 0..127, then W rows)
         const int j = c & 3;   // packed 16-byte chunk within the row's 64 bytes
         uint4 lo, hi;
@@ -194,78 +200,109 @@ __device__ __forceinline__ void mma_role(const Smem& sm, const Problem& pb, uint
   }
 }
 
+__device__ __forceinline__ void epi_bar_sync() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");  // the 4 epilogue warps only
+}
+
+__device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Converts one 32-column chunk of accumulators (one row per thread) and stores it.
+template <int BITS, bool OUT_S32>
+__device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row, bool row_ok,
+                                               int n, int N, float s_a, const float* epi_sw,
+                                               const float* epi_b, void* out) {
+  if (n >= N || !row_ok) return;
+  int32_t acc[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    acc[i] = BITS == 4 ? (static_cast<int32_t>(r[i]) >> 8) : static_cast<int32_t>(r[i]);
+  if (OUT_S32) {
+    int32_t* dst = static_cast<int32_t*>(out) + static_cast<int64_t>(row) * N + n;
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+      if (n + 4 * v + 4 <= N)
+        st_stream_v4(dst + 4 * v, make_uint4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2],
+                                             acc[4 * v + 3]));
+  } else {
+    uint16_t* dst = static_cast<uint16_t*>(out) + static_cast<int64_t>(row) * N + n;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      if (n + 8 * v + 8 > N) break;  // N % 16 == 0: only whole 8-column groups exist
+      const float4 w0 = *reinterpret_cast<const float4*>(epi_sw + 8 * v);
+      const float4 w1 = *reinterpret_cast<const float4*>(epi_sw + 8 * v + 4);
+      const float4 b0 = *reinterpret_cast<const float4*>(epi_b + 8 * v);
+      const float4 b1 = *reinterpret_cast<const float4*>(epi_b + 8 * v + 4);
+      const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      uint32_t packed[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        float y[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float sab = __fmul_rn(s_a, wv[e + h]);
+          const float p = __fmul_rn(sab, __int2float_rn(acc[8 * v + e + h]));
+          y[h] = __fadd_rn(p, bv[e + h]);
+        }
+        const __nv_bfloat162 y2 = __floats2bfloat162_rn(y[0], y[1]);
+        packed[e >> 1] = *reinterpret_cast<const uint32_t*>(&y2);
+      }
+      st_stream_v4(dst + 8 * v, make_uint4(packed[0], packed[1], packed[2], packed[3]));
+    }
+  }
+}
+
 template <int BITS, bool OUT_S32>
 __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
-                                              uint32_t tmem_base, int quad, int lane,
+                                              uint32_t tmem_base, int quad, int lane, int et,
                                               const float* __restrict__ sa,
                                               const float* __restrict__ sw,
                                               const uint16_t* __restrict__ bias, void* out,
+                                              float* epi_sw, float* epi_b,
                                               volatile int* abort_flag) {
   int it = 0;
   for (int t = blockIdx.x; t < pb.num_tiles; t += gridDim.x, ++it) {
     const int buf = it & 1;
     const uint32_t aph = (it >> 1) & 1;
-    if (!mbar_wait_bounded(sm.acc_full(buf), aph, abort_flag, kErrWaitEpilogue)) return;
-    tc_fence_after();
     int m0, n0;
     pb.tile_origin(t, m0, n0);
+    if (!OUT_S32) {
+      // Stage the tile's channel scales and bias while its main loop runs.
+      epi_bar_sync();  // every epilogue warp is done with the previous tile's copy
+      for (int i = et; i < BN; i += 128) {
+        const int n = n0 + i;
+        const bool ok = n < pb.N;
+        epi_sw[i] = ok ? sw[n] : 0.f;
+        epi_b[i] = (ok && bias) ? __uint_as_float(static_cast<uint32_t>(bias[n]) << 16) : 0.f;
+      }
+      epi_bar_sync();
+    }
     const int row = m0 + 32 * quad + lane;
     const bool row_ok = row < pb.M;
-    float s_a = 0.f;
-    if (!OUT_S32 && row_ok) s_a = sa[row];
+    const float s_a = (!OUT_S32 && row_ok) ? sa[row] : 0.f;
+    if (!mbar_wait_bounded(sm.acc_full(buf), aph, abort_flag, kErrWaitEpilogue)) return;
+    tc_fence_after();
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quad) << 16) +
                            static_cast<uint32_t>(buf * BN);
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      const int n = n0 + 32 * c;
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(taddr + 32 * c, r);
+    // Two register sets: the TMEM load of chunk c+1 is in flight while chunk c
+    // is converted and stored.
+    uint32_t ra[32], rb[32];
+    tmem_ld_32x32b_x32(taddr, ra);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < BN / 32; c += 2) {
+      tmem_ld_32x32b_x32(taddr + 32 * (c + 1), rb);
+      epilogue_chunk<BITS, OUT_S32>(ra, row, row_ok, n0 + 32 * c, pb.N, s_a, epi_sw + 32 * c,
+                                    epi_b + 32 * c, out);
       tmem_wait_ld();
-      if (n >= pb.N) continue;  // warp-uniform: whole 32-column chunk past N
-      int32_t acc[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        acc[i] = BITS == 4 ? (static_cast<int32_t>(r[i]) >> 8) : static_cast<int32_t>(r[i]);
-      if (OUT_S32) {
-        int32_t* dst = static_cast<int32_t*>(out) + static_cast<int64_t>(row) * pb.N + n;
-        if (row_ok) {
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            if (n + 4 * v + 4 <= pb.N)
-              *reinterpret_cast<int4*>(dst + 4 * v) =
-                  make_int4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
-        }
-      } else {
-        uint16_t* dst = static_cast<uint16_t*>(out) + static_cast<int64_t>(row) * pb.N + n;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int nv = n + 8 * v;
-          if (nv + 8 > pb.N) break;  // N % 16 == 0: only whole 8-column groups exist
-          const float4 w0 = __ldg(reinterpret_cast<const float4*>(sw + nv));
-          const float4 w1 = __ldg(reinterpret_cast<const float4*>(sw + nv + 4));
-          const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-          uint4 braw = make_uint4(0u, 0u, 0u, 0u);
-          if (bias) braw = __ldg(reinterpret_cast<const uint4*>(bias + nv));
-          const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
-          uint32_t packed[4];
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            float y[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const float sab = __fmul_rn(s_a, wv[e + h]);
-              const float p = __fmul_rn(sab, __int2float_rn(acc[8 * v + e + h]));
-              const uint32_t bb = h == 0 ? (bw[e >> 1] << 16) : (bw[e >> 1] & 0xFFFF0000u);
-              y[h] = __fadd_rn(p, __uint_as_float(bb));
-            }
-            const __nv_bfloat162 y2 = __floats2bfloat162_rn(y[0], y[1]);
-            packed[e >> 1] = *reinterpret_cast<const uint32_t*>(&y2);
-          }
-          if (row_ok)
-            *reinterpret_cast<uint4*>(dst + 8 * v) =
-                make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        }
-      }
+      if (c + 2 < BN / 32) tmem_ld_32x32b_x32(taddr + 32 * (c + 2), ra);
+      epilogue_chunk<BITS, OUT_S32>(rb, row, row_ok, n0 + 32 * (c + 1), pb.N, s_a,
+                                    epi_sw + 32 * (c + 1), epi_b + 32 * (c + 1), out);
+      tmem_wait_ld();
     }
     tc_fence_before();
     __syncwarp();
@@ -334,7 +371,9 @@ __global__ void __launch_bounds__(Cfg<BITS>::kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) mma_role<BITS>(sm, pb, tmem_base, abort_flag);
   } else if (warp < 2 + C::kEpiWarps) {
-    epilogue_role<BITS, OUT_S32>(sm, pb, tmem_base, warp & 3, lane, sa, sw, bias, out, abort_flag);
+    float* epi_sw = reinterpret_cast<float*>(sm.ptr + C::kOffEpi);
+    epilogue_role<BITS, OUT_S32>(sm, pb, tmem_base, warp & 3, lane, threadIdx.x - 64, sa, sw,
+                                 bias, out, epi_sw, epi_sw + BN, abort_flag);
   } else {
     if (C::kPacked) unpack_role<BITS>(sm, pb, threadIdx.x - 32 * (2 + C::kEpiWarps), abort_flag);
   }

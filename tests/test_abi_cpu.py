@@ -24,7 +24,8 @@ def lib():
 
 
 def _declared():
-    src = open(HEADER).read()
+    with open(HEADER) as f:
+        src = f.read()
     return sorted(set(re.findall(r"QS_API\s+[\w\s\*]+?\b(qs_\w+)\s*\(", src)))
 
 

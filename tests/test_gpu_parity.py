@@ -91,8 +91,8 @@ def test_quant_act_tiny_config():
 
 
 def test_quant_ties_without_rotation():
-    rows = [l.split() for l in open(os.path.join(GOLDEN, "rne_ties_w4.txt"))
-            if l.strip() and not l.startswith("#")]
+    with open(os.path.join(GOLDEN, "rne_ties_w4.txt")) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
     x = torch.zeros(2, 128)
     want = np.zeros((2, 128), np.int8)
     for r, c, v, q in rows:
