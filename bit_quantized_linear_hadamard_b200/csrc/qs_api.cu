@@ -99,9 +99,10 @@ qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, const fl
   const uint64_t row_bytes = static_cast<uint64_t>(K) * BITS / 8;
   const uint32_t box_bytes = qs::gemm::BK * BITS / 8;
   CUtensorMap ta, tb;
-  if (!make_tensor_map(&ta, xp, row_bytes, static_cast<uint64_t>(M), box_bytes, qs::gemm::BM,
+  // each CTA of a pair loads 128 rows of x and 128 rows of W per stage
+  if (!make_tensor_map(&ta, xp, row_bytes, static_cast<uint64_t>(M), box_bytes, qs::gemm::HM,
                        BITS == 8) ||
-      !make_tensor_map(&tb, wp, row_bytes, static_cast<uint64_t>(N), box_bytes, qs::gemm::BN,
+      !make_tensor_map(&tb, wp, row_bytes, static_cast<uint64_t>(N), box_bytes, qs::gemm::HN,
                        BITS == 8))
     return QS_ERR_CUDA;
   auto kern = qs::gemm::qgemm_kernel<BITS, OUT_S32>;
@@ -110,9 +111,12 @@ qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, const fl
     return QS_ERR_CUDA;
   const int sms = sm_count();
   if (sms <= 0) return QS_ERR_CUDA;
+  // persistent clusters of two CTAs, at most one CTA per SM
   const int64_t tiles = ((M + qs::gemm::BM - 1) / qs::gemm::BM) *
                         ((N + qs::gemm::BN - 1) / qs::gemm::BN);
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
+  if (pairs < 1) return QS_ERR_CUDA;
+  const int grid = static_cast<int>(2 * pairs);
   kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(
       ta, tb, sa, sw, static_cast<const uint16_t*>(bias), out, static_cast<int>(M),
       static_cast<int>(N), static_cast<int>(K));

@@ -5,15 +5,38 @@
 //   acc[m][n] = sum_k q_a[m][k] * q_w[n][k]                       (int32, exact)
 //   out[m][n] = bf16(fl(fl(fl(s_a[m] * s_w[n]) * float(acc)) + bias[n]))
 //
-// Structure: a persistent kernel, one CTA per SM, each CTA walking output
-// tiles of 128 x 256 (n fastest, so the whole packed weight stays in L2 while
-// activation tiles stream once).  Warp roles:
-//   warp 0      TMA producer: packed tiles of x (128 x 128 K) and W (256 x 128 K)
-//   warp 1      TMEM owner and single-thread tcgen05.mma (kind::i8) issuer
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator, scale, bias, bf16 store
-//   warps 6-9   (4-bit only) unpack packed nibbles into the 8-bit operand tiles
-// Two 256-column int32 accumulators in TMEM (all 512 columns) let the epilogue
-// of one tile run under the main loop of the next.
+// Structure: a persistent kernel launched as clusters of two CTAs on the two
+// SMs of a TPC.  Each pair walks output tiles of 256 x 256 (n fastest, so the
+// whole packed weight stays in L2 while activation tiles stream once).  CTA r
+// of the pair holds rows [128r, 128r+128) of the x tile and rows
+// [128r, 128r+128) of the W tile; the leader (r = 0) issues one
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 32) per 32-deep K step, which
+// reads the x rows and W rows of both CTAs and accumulates each CTA's 128 x 256
+// result in that CTA's tensor memory.  Per SM this halves the W operand traffic
+// of a 128 x 256 single-CTA tile at the same MMA work.
+//
+// Warp roles (both CTAs):
+//   warp 0      TMA producer
+//   warp 1      TMEM allocation; in the leader the single-thread MMA issuer;
+//               in the other CTA (4-bit only) the relay that tells the leader
+//               that this CTA's operand tiles are ready
+//   warps 2-5   epilogue: tcgen05.ld of this CTA's accumulator rows, scale,
+//               bias, bf16 store
+//   warps 6-9   (4-bit only) widen packed nibbles into the 8-bit operand tiles
+// Two 256-column int32 accumulators (all 512 TMEM columns) let the epilogue of
+// one tile run under the main loop of the next.
+//
+// Synchronisation across the pair: 8-bit operand stages are "full" on the
+// leader's barrier when the TMA loads of both CTAs have landed.  4-bit operand
+// stages are "unpacked" on a local barrier of each CTA; the other CTA's relay
+// thread forwards its local completion to the leader's "full" barrier as a
+// 16-byte shared-to-shared bulk copy whose transaction bytes complete that
+// barrier.  (A software cluster-scope release per stage instead stalls the
+// arriving thread for a memory-barrier round trip every stage, which measured
+// as the limit of the whole main loop.)  The leader's MMA
+// completion is committed to the "empty" barrier of each CTA; accumulator
+// readiness is committed to both CTAs; the epilogue warps of both CTAs arrive
+// on the leader's "accumulator free" barrier.
 //
 // 4-bit operands: tcgen05 has no 4-bit integer kind, so each packed 16-byte
 // chunk (32 nibbles = 32 consecutive K elements) is widened in shared memory to
@@ -29,58 +52,72 @@
 // directly by TMA.
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include "qs_ptx.cuh"
 
 namespace qs {
 namespace gemm {
 
-constexpr int BM = 128;  // tile rows (tokens)
-constexpr int BN = 256;  // tile columns (output channels)
+constexpr int BM = 256;  // tile rows (tokens), 128 per CTA
+constexpr int BN = 256;  // tile columns (output channels), 128 W rows per CTA
+constexpr int HM = 128;  // x rows per CTA
+constexpr int HN = 128;  // W rows per CTA
 constexpr int BK = 128;  // K elements per pipeline stage (= 128 bytes of 8-bit operand)
 constexpr int kTmemCols = 2 * BN;
 
 template <int BITS>
 struct Cfg {
   static constexpr bool kPacked = BITS == 4;
-  static constexpr int kPkBytesA = BM * BK / 2;  // packed 4-bit tile of x
-  static constexpr int kPkBytesB = BN * BK / 2;  // packed 4-bit tile of W
-  static constexpr int kOpBytesA = BM * BK;      // 8-bit operand tile of x
-  static constexpr int kOpBytesB = BN * BK;      // 8-bit operand tile of W
+  static constexpr int kPkBytesA = HM * BK / 2;  // packed 4-bit tile of x (this CTA)
+  static constexpr int kPkBytesB = HN * BK / 2;  // packed 4-bit tile of W (this CTA)
+  static constexpr int kOpBytesA = HM * BK;      // 8-bit operand tile of x
+  static constexpr int kOpBytesB = HN * BK;      // 8-bit operand tile of W
+  static constexpr int kPkStage = kPkBytesA + kPkBytesB;
+  static constexpr int kOpStage = kOpBytesA + kOpBytesB;
   static constexpr int kPkStages = kPacked ? 4 : 0;
-  static constexpr int kOpStages = kPacked ? 2 : 4;
+  static constexpr int kOpStages = kPacked ? 4 : 6;
   static constexpr int kEpiWarps = 4;
   static constexpr int kUnpackWarps = kPacked ? 4 : 0;
   static constexpr int kThreads = 32 * (2 + kEpiWarps + kUnpackWarps);
   static constexpr int kOffOp = 0;
-  static constexpr int kOffPk = kOffOp + kOpStages * (kOpBytesA + kOpBytesB);
-  static constexpr int kOffBar = kOffPk + kPkStages * (kPkBytesA + kPkBytesB);
-  static constexpr int kNumBars = 2 * kPkStages + 2 * kOpStages + 4;
+  static constexpr int kOffPk = kOffOp + kOpStages * kOpStage;
+  static constexpr int kOffBar = kOffPk + kPkStages * kPkStage;
+  static constexpr int kNumBars = 2 * kPkStages + 3 * kOpStages + 4;
   static constexpr int kOffEpi = (kOffBar + 8 * kNumBars + 15) / 16 * 16;  // s_w, bias of a tile
-  static constexpr int kOffMisc = kOffEpi + 2 * BN * 4;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
-  static constexpr int kUnpackChunks = (kPkBytesA + kPkBytesB) / 16;
+  static constexpr int kOffMisc = kOffEpi + 2 * BN * 4;  // TMEM address, abort flag
+  static constexpr int kOffSignal = kOffMisc + 16;        // 16 bytes per operand stage
+  static constexpr int kSmemBytes = kOffSignal + 16 * kOpStages + 1024;  // + alignment slack
   static constexpr int kUnpackThreads = kPacked ? 32 * kUnpackWarps : 1;
-  static constexpr int kChunksPerThread = kPacked ? kUnpackChunks / kUnpackThreads : 0;
-  static_assert(kUnpackChunks % kUnpackThreads == 0, "unpack split");
+  static constexpr int kChunksPerThread = kPacked ? (kPkStage / 16) / kUnpackThreads : 0;
+  static_assert((kPkStage / 16) % kUnpackThreads == 0, "unpack split");
+  // arrivals completing one "operand full" phase on the leader: its MMA
+  // thread arming the relay's 16 bytes (4-bit) or its producer arming both
+  // CTAs' TMA bytes (8-bit)
+  static constexpr int kOpFullCount = 1;
+  static constexpr int kAccEmptyCount = 2 * kEpiWarps;
 };
 
 struct Smem {
-  uint32_t base;  // shared-window address of the 1024-aligned layout
+  uint32_t base;  // shared-window address of the 1024-aligned layout (this CTA)
   uint8_t* ptr;
   int P, U;
+  uint32_t off_bar;
+  __device__ uint32_t bar(int i) const { return base + off_bar + 8u * i; }
   __device__ uint32_t pk_full(int s) const { return bar(s); }
   __device__ uint32_t pk_empty(int s) const { return bar(P + s); }
   __device__ uint32_t op_full(int s) const { return bar(2 * P + s); }
   __device__ uint32_t op_empty(int s) const { return bar(2 * P + U + s); }
   __device__ uint32_t acc_full(int b) const { return bar(2 * P + 2 * U + b); }
   __device__ uint32_t acc_empty(int b) const { return bar(2 * P + 2 * U + 2 + b); }
-  uint32_t off_bar;
-  __device__ uint32_t bar(int i) const { return base + off_bar + 8u * i; }
+  __device__ uint32_t unpacked(int s) const { return bar(2 * P + 2 * U + 4 + s); }
 };
 
 struct Problem {
   int M, N, K;
   int n_tiles, num_tiles, kblocks;
+  int pair, num_pairs;  // this pair's index and the number of pairs
+  uint32_t rank;        // 0 = leader
   __device__ void tile_origin(int t, int& m0, int& n0) const {
     m0 = (t / n_tiles) * BM;
     n0 = (t % n_tiles) * BN;
@@ -94,32 +131,43 @@ __device__ __forceinline__ void producer_role(const Smem& sm, const Problem& pb,
   using C = Cfg<BITS>;
   int s = 0;
   uint32_t ph = 0;
-  for (int t = blockIdx.x; t < pb.num_tiles; t += gridDim.x) {
+  const int roff = static_cast<int>(pb.rank) * HM;
+  for (int t = pb.pair; t < pb.num_tiles; t += pb.num_pairs) {
     int m0, n0;
     pb.tile_origin(t, m0, n0);
     for (int kb = 0; kb < pb.kblocks; ++kb) {
       if (C::kPacked) {
+        // packed tiles stay in this CTA: ordinary loads on a local barrier
         if (!mbar_wait_bounded(sm.pk_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer)) return;
-        const uint32_t dst = sm.base + C::kOffPk + s * (C::kPkBytesA + C::kPkBytesB);
-        mbar_arrive_expect_tx(sm.pk_full(s), C::kPkBytesA + C::kPkBytesB);
-        tma_load_2d(dst, tmA, kb * (BK / 2), m0, sm.pk_full(s));
-        tma_load_2d(dst + C::kPkBytesA, tmB, kb * (BK / 2), n0, sm.pk_full(s));
+        const uint32_t dst = sm.base + C::kOffPk + s * C::kPkStage;
+        mbar_arrive_expect_tx(sm.pk_full(s), C::kPkStage);
+        tma_load_2d(dst, tmA, kb * (BK / 2), m0 + roff, sm.pk_full(s));
+        tma_load_2d(dst + C::kPkBytesA, tmB, kb * (BK / 2), n0 + roff, sm.pk_full(s));
         if (++s == C::kPkStages) { s = 0; ph ^= 1u; }
       } else {
+        // operand tiles of both CTAs complete on the leader's barrier
         if (!mbar_wait_bounded(sm.op_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer)) return;
-        const uint32_t dst = sm.base + C::kOffOp + s * (C::kOpBytesA + C::kOpBytesB);
-        mbar_arrive_expect_tx(sm.op_full(s), C::kOpBytesA + C::kOpBytesB);
-        tma_load_2d(dst, tmA, kb * BK, m0, sm.op_full(s));
-        tma_load_2d(dst + C::kOpBytesA, tmB, kb * BK, n0, sm.op_full(s));
+        const uint32_t dst = sm.base + C::kOffOp + s * C::kOpStage;
+        const uint32_t full_leader = map_to_rank(sm.op_full(s), 0);
+        if (pb.rank == 0) mbar_arrive_expect_tx(sm.op_full(s), 2 * C::kOpStage);
+        tma_load_2d_pair(dst, tmA, kb * BK, m0 + roff, full_leader);
+        tma_load_2d_pair(dst + C::kOpBytesA, tmB, kb * BK, n0 + roff, full_leader);
         if (++s == C::kOpStages) { s = 0; ph ^= 1u; }
       }
+    }
+  }
+  if (!C::kPacked) {
+    // drain: every stage's last release has arrived before the CTA may exit
+    for (int i = 0; i < C::kOpStages; ++i) {
+      if (!mbar_wait_bounded(sm.op_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer)) return;
+      if (++s == C::kOpStages) { s = 0; ph ^= 1u; }
     }
   }
 }
 
 // Widens packed 4-bit tiles into 8-bit operand tiles (see the file comment).
-// Packed stage: [x tile 128 rows x 64 B][W tile 256 rows x 64 B], plain rows.
-// Operand stage: [x tile 128 rows x 128 B][W tile 256 rows x 128 B], rows of
+// Packed stage: [x tile 128 rows x 64 B][W tile 128 rows x 64 B], plain rows.
+// Operand stage: [x tile 128 rows x 128 B][W tile 128 rows x 128 B], rows of
 // 128 B with 16-byte chunk c stored at chunk c ^ (row & 7) (128-byte swizzle).
 template <int BITS>
 __device__ __forceinline__ void unpack_role(const Smem& sm, const Problem& pb, int ut,
@@ -128,12 +176,12 @@ __device__ __forceinline__ void unpack_role(const Smem& sm, const Problem& pb, i
   const int lane = ut & 31;
   int sp = 0, su = 0;
   uint32_t php = 0, phu = 0;
-  for (int t = blockIdx.x; t < pb.num_tiles; t += gridDim.x) {
+  for (int t = pb.pair; t < pb.num_tiles; t += pb.num_pairs) {
     for (int kb = 0; kb < pb.kblocks; ++kb) {
       if (!mbar_wait_bounded(sm.pk_full(sp), php, abort_flag, kErrWaitUnpack)) return;
       if (!mbar_wait_bounded(sm.op_empty(su), phu ^ 1u, abort_flag, kErrWaitUnpack)) return;
-      const uint8_t* pk = sm.ptr + C::kOffPk + sp * (C::kPkBytesA + C::kPkBytesB);
-      uint8_t* op = sm.ptr + C::kOffOp + su * (C::kOpBytesA + C::kOpBytesB);
+      const uint8_t* pk = sm.ptr + C::kOffPk + sp * C::kPkStage;
+      uint8_t* op = sm.ptr + C::kOffOp + su * C::kOpStage;
       // all loads first: they are independent of the stores that follow
       uint4 wv[C::kChunksPerThread > 0 ? C::kChunksPerThread : 1];
 #pragma unroll
@@ -161,15 +209,42 @@ __device__ __forceinline__ void unpack_role(const Smem& sm, const Problem& pb, i
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(sm.op_full(su));
+        mbar_arrive(sm.unpacked(su));
         mbar_arrive(sm.pk_empty(sp));
       }
       if (++sp == C::kPkStages) { sp = 0; php ^= 1u; }
       if (++su == C::kOpStages) { su = 0; phu ^= 1u; }
     }
   }
+  // drain: every operand stage's last release has arrived before the CTA may exit
+  if (lane == 0) {
+    for (int i = 0; i < C::kOpStages; ++i) {
+      if (!mbar_wait_bounded(sm.op_empty(su), phu ^ 1u, abort_flag, kErrWaitUnpack)) return;
+      if (++su == C::kOpStages) { su = 0; phu ^= 1u; }
+    }
+  }
 }
 
+// 4-bit, non-leader CTA only: forwards "this CTA's operand stage is unpacked"
+// to the leader's "full" barrier with one 16-byte signalling bulk copy per
+// stage (the leader's MMA thread arms that barrier with the 16 bytes).
+template <int BITS>
+__device__ __forceinline__ void relay_role(const Smem& sm, const Problem& pb,
+                                           volatile int* abort_flag) {
+  using C = Cfg<BITS>;
+  int s = 0;
+  uint32_t ph = 0;
+  for (int t = pb.pair; t < pb.num_tiles; t += pb.num_pairs) {
+    for (int kb = 0; kb < pb.kblocks; ++kb) {
+      if (!mbar_wait_bounded(sm.unpacked(s), ph, abort_flag, kErrWaitUnpack)) return;
+      const uint32_t slot = sm.base + C::kOffSignal + 16 * s;
+      bulk_signal(map_to_rank(slot, 0), slot, map_to_rank(sm.op_full(s), 0));
+      if (++s == C::kOpStages) { s = 0; ph ^= 1u; }
+    }
+  }
+}
+
+// Leader CTA only.
 template <int BITS>
 __device__ __forceinline__ void mma_role(const Smem& sm, const Problem& pb, uint32_t tmem_base,
                                          volatile int* abort_flag) {
@@ -178,25 +253,29 @@ __device__ __forceinline__ void mma_role(const Smem& sm, const Problem& pb, uint
   int s = 0;
   uint32_t ph = 0;
   int it = 0;
-  for (int t = blockIdx.x; t < pb.num_tiles; t += gridDim.x, ++it) {
+  for (int t = pb.pair; t < pb.num_tiles; t += pb.num_pairs, ++it) {
     const int buf = it & 1;
     const uint32_t aph = (it >> 1) & 1;
-    if (!mbar_wait_bounded(sm.acc_empty(buf), aph ^ 1u, abort_flag, kErrWaitMma)) return;
+    if (!mbar_wait_cluster_bounded(sm.acc_empty(buf), aph ^ 1u, abort_flag, kErrWaitMma)) return;
     tc_fence_after();
     const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
     for (int kb = 0; kb < pb.kblocks; ++kb) {
-      if (!mbar_wait_bounded(sm.op_full(s), ph, abort_flag, kErrWaitMma)) return;
+      if (C::kPacked) mbar_arrive_expect_tx(sm.op_full(s), 16);  // the relay's signal
+      if (C::kPacked && !mbar_wait_bounded(sm.unpacked(s), ph, abort_flag, kErrWaitMma)) return;
+      if (!mbar_wait_cluster_bounded(sm.op_full(s), ph, abort_flag, kErrWaitMma)) return;
       tc_fence_after();
-      const uint32_t a0 = sm.base + C::kOffOp + s * (C::kOpBytesA + C::kOpBytesB);
+      const uint32_t a0 = sm.base + C::kOffOp + s * C::kOpStage;
       const uint32_t b0 = a0 + C::kOpBytesA;
 #pragma unroll
       for (int kk = 0; kk < BK / 32; ++kk)
-        mma_i8(d, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc,
-               (kb | kk) != 0);
-      mma_commit(sm.op_empty(s));
+        mma_i8_pair(d, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc,
+                    (kb | kk) != 0);
+      mma_commit_pair(map_to_rank(sm.op_empty(s), 0));
+      mma_commit_pair(map_to_rank(sm.op_empty(s), 1));
       if (++s == C::kOpStages) { s = 0; ph ^= 1u; }
     }
-    mma_commit(sm.acc_full(buf));
+    mma_commit_pair(map_to_rank(sm.acc_full(buf), 0));
+    mma_commit_pair(map_to_rank(sm.acc_full(buf), 1));
   }
 }
 
@@ -265,7 +344,7 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
                                               float* epi_sw, float* epi_b,
                                               volatile int* abort_flag) {
   int it = 0;
-  for (int t = blockIdx.x; t < pb.num_tiles; t += gridDim.x, ++it) {
+  for (int t = pb.pair; t < pb.num_tiles; t += pb.num_pairs, ++it) {
     const int buf = it & 1;
     const uint32_t aph = (it >> 1) & 1;
     int m0, n0;
@@ -281,7 +360,7 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
       }
       epi_bar_sync();
     }
-    const int row = m0 + 32 * quad + lane;
+    const int row = m0 + static_cast<int>(pb.rank) * HM + 32 * quad + lane;
     const bool row_ok = row < pb.M;
     const float s_a = (!OUT_S32 && row_ok) ? sa[row] : 0.f;
     if (!mbar_wait_bounded(sm.acc_full(buf), aph, abort_flag, kErrWaitEpilogue)) return;
@@ -306,17 +385,24 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(sm.acc_empty(buf));
+    if (lane == 0) {
+      if (pb.rank == 0)
+        mbar_arrive(sm.acc_empty(buf));
+      else
+        mbar_arrive_cluster(map_to_rank(sm.acc_empty(buf), 0));
+    }
   }
 }
 
 template <int BITS, bool OUT_S32>
-__global__ void __launch_bounds__(Cfg<BITS>::kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<BITS>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const float* __restrict__ sa, const float* __restrict__ sw,
                  const uint16_t* __restrict__ bias, void* out, int M, int N, int K) {
   using C = Cfg<BITS>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The padding is identical in both CTAs (same kernel, same static layout),
+  // so every shared object has the same offset in the two CTAs of a pair.
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
   Smem sm;
@@ -335,6 +421,9 @@ __global__ void __launch_bounds__(Cfg<BITS>::kThreads, 1)
   pb.n_tiles = (N + BN - 1) / BN;
   pb.num_tiles = ((M + BM - 1) / BM) * pb.n_tiles;
   pb.kblocks = K / BK;
+  pb.rank = cluster_ctarank();
+  pb.pair = blockIdx.x >> 1;
+  pb.num_pairs = gridDim.x >> 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -345,31 +434,34 @@ __global__ void __launch_bounds__(Cfg<BITS>::kThreads, 1)
       mbar_init(sm.pk_empty(s), C::kUnpackWarps);
     }
     for (int s = 0; s < C::kOpStages; ++s) {
-      mbar_init(sm.op_full(s), C::kPacked ? C::kUnpackWarps : 1);
+      mbar_init(sm.op_full(s), C::kOpFullCount);
       mbar_init(sm.op_empty(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(sm.acc_full(b), 1);
-      mbar_init(sm.acc_empty(b), C::kEpiWarps);
+      mbar_init(sm.acc_empty(b), C::kAccEmptyCount);
     }
+    if (C::kPacked)
+      for (int s = 0; s < C::kOpStages; ++s) mbar_init(sm.unpacked(s), C::kUnpackWarps);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
     if (lane == 0) producer_role<BITS>(sm, pb, &tmA, &tmB, abort_flag);
   } else if (warp == 1) {
-    if (lane == 0) mma_role<BITS>(sm, pb, tmem_base, abort_flag);
+    if (lane == 0 && pb.rank == 0) mma_role<BITS>(sm, pb, tmem_base, abort_flag);
+    if (lane == 0 && pb.rank != 0 && C::kPacked) relay_role<BITS>(sm, pb, abort_flag);
   } else if (warp < 2 + C::kEpiWarps) {
     float* epi_sw = reinterpret_cast<float*>(sm.ptr + C::kOffEpi);
     epilogue_role<BITS, OUT_S32>(sm, pb, tmem_base, warp & 3, lane, threadIdx.x - 64, sa, sw,
@@ -380,6 +472,7 @@ __global__ void __launch_bounds__(Cfg<BITS>::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its partner may still signal it
   if (*abort_flag) {
     // A wait gave up: give copies and MMAs already in flight time to land
     // before the tensor memory is released.
@@ -388,7 +481,7 @@ __global__ void __launch_bounds__(Cfg<BITS>::kThreads, 1)
   }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 

@@ -185,6 +185,20 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       : "memory");
 }
 
+// 16-byte bulk copy from this CTA's shared memory to a shared location of
+// another CTA of the cluster, completing as 16 transaction bytes on an mbarrier
+// of that CTA (`dst` and `bar` are cluster-window addresses).  Used as a
+// hardware-tracked "ready" signal: it is ordered after this CTA's earlier
+// async-proxy-visible writes and needs no cluster-scope fence in the issuing
+// thread.
+__device__ __forceinline__ void bulk_signal(uint32_t dst, uint32_t src, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], 16, [%2];" ::
+          "r"(dst),
+      "r"(src), "r"(bar)
+      : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
