@@ -11,6 +11,7 @@
 
 #include "qs.h"
 #include "qs_gemm.cuh"
+#include "qs_host.cuh"
 #include "qs_glue.cuh"
 #include "qs_quant.cuh"
 
@@ -49,48 +50,6 @@ qs_status check_bits(int bits) { return (bits == 4 || bits == 8) ? QS_OK : QS_ER
     if (_s != QS_OK) return _s;    \
   } while (0)
 
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// 2-D byte tensor [rows][row_bytes] (row-major), box [box_rows][box_bytes].
-bool make_tensor_map(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows,
-                     uint32_t box_bytes, uint32_t box_rows, bool swizzle128) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {row_bytes, rows};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_bytes, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
-                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-int sm_count() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev < 0 || dev >= 64) return 0;
-  if (!cached[dev]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    cached[dev] = n;
-  }
-  return cached[dev];
-}
-
 template <int BITS, bool OUT_S32>
 qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, const float* sw,
                        const void* bias, int64_t M, int64_t N, int64_t K, void* out,
@@ -100,16 +59,16 @@ qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, const fl
   const uint32_t box_bytes = qs::gemm::BK * BITS / 8;
   CUtensorMap ta, tb;
   // each CTA of a pair loads 128 rows of x and 128 rows of W per stage
-  if (!make_tensor_map(&ta, xp, row_bytes, static_cast<uint64_t>(M), box_bytes, qs::gemm::HM,
+  if (!qs::make_tensor_map_2d(&ta, xp, row_bytes, static_cast<uint64_t>(M), box_bytes, qs::gemm::HM,
                        BITS == 8) ||
-      !make_tensor_map(&tb, wp, row_bytes, static_cast<uint64_t>(N), box_bytes, qs::gemm::HN,
+      !qs::make_tensor_map_2d(&tb, wp, row_bytes, static_cast<uint64_t>(N), box_bytes, qs::gemm::HN,
                        BITS == 8))
     return QS_ERR_CUDA;
   auto kern = qs::gemm::qgemm_kernel<BITS, OUT_S32>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
       cudaSuccess)
     return QS_ERR_CUDA;
-  const int sms = sm_count();
+  const int sms = qs::sm_count();
   if (sms <= 0) return QS_ERR_CUDA;
   // persistent clusters of two CTAs, at most one CTA per SM
   const int64_t tiles = ((M + qs::gemm::BM - 1) / qs::gemm::BM) *
@@ -215,7 +174,7 @@ qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream
   if (!aligned16(x_bf16) || !aligned16(y_bf16)) return QS_ERR_ALIGN;
   QS_TRY(check_device_ptr(x_bf16));
   QS_TRY(check_device_ptr(y_bf16));
-  const int sms = sm_count();
+  const int sms = qs::sm_count();
   if (sms <= 0) return QS_ERR_CUDA;
   const int64_t nvec = n / 8;
   int64_t blocks = (nvec + 255) / 256;

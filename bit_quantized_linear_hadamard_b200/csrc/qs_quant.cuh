@@ -13,10 +13,10 @@
 // rows of t < 2^-120 treated as zero rows.
 //
 // Two kernels compute exactly that:
-//  * rotate_quant_half_kernel (K <= 16384): half a 128-element Hadamard block
+//  * rotate_quant_tma_kernel (K <= 16384): half a 128-element Hadamard block
 //    per thread, stages h = 1..32 in registers (packed f32x2 arithmetic), stage
-//    64 with the partner thread; a CTA holds whole rows (double-buffered in
-//    shared memory) and reduces their absmax through shared memory.
+//    64 with the partner thread; row groups stream into a multi-stage
+//    shared-memory ring by TMA; the row absmax is reduced through shared memory.
 //  * rotate_quant_group_kernel (longer rows): 8 elements per thread, stages
 //    h = 1, 2, 4 in registers and h = 8..64 by xor-shuffles, one row per CTA.
 // Rounding to the nearest integer, ties to even, is done by adding 1.5*2^23:
@@ -25,6 +25,7 @@
 // the low mantissa bits (two's complement in the low byte).
 #pragma once
 
+#include "qs_host.cuh"
 #include "qs_ptx.cuh"
 
 namespace qs {
@@ -100,126 +101,91 @@ __device__ __forceinline__ uint32_t pack4_int8(uint32_t c0, uint32_t c1, uint32_
 // Rows of up to 128 Hadamard blocks: half a block per thread.
 //
 // A persistent CTA walks groups of `rpc` consecutive rows.  A group is one
-// contiguous span of x; it is copied into shared memory by coalesced 16-byte
-// cp.async, two groups in flight (double buffer).  Chunk i (16 bytes) of block
-// tb of the group (block b of row r, tb = r * nblk + b) is stored at chunk
-// i ^ (tb & 15), which keeps the copy free of bank conflicts.
+// contiguous span of x, viewed as rows of 64 bf16 (128 bytes); thread 0 loads
+// it with one 2-D TMA copy (128-byte swizzle) into a stage of a `stages`-deep
+// shared-memory ring and the copy completes on that stage's mbarrier, so the
+// next groups are in flight while the current one is computed.
 //
-// Threads 2tb and 2tb+1 own the low and high 64 elements of block tb.  A half
-// lives in registers as 32 pairs (v[j], v[j + 32]): butterfly stages h = 1..16
-// pair (j, j + h) and (j + 32, j + 32 + h) alike, so two butterflies are one
-// packed add.rn.f32x2 and one sub.rn.f32x2 (independent IEEE binary32
-// operations); stage 32 works inside the pairs; stage 64 pairs the two threads:
-// each takes its partner's value p by an xor-shuffle and forms fl(p + sg * own)
-// with sg = +1 (low half: a + b) or -1 (high half: a - b) in one packed
-// fma.rn.f32x2 -- sg * own is exact, so the single rounding is that of the
-// butterfly's add or subtract.
+// Threads 2tb and 2tb+1 own the low and high 64 elements of block tb of the
+// group = 128-byte row R = 2tb + up of the stage, whose 16-byte chunk i sits at
+// chunk i ^ (R & 7): eight consecutive threads read eight different chunk
+// positions, free of bank conflicts.  A half lives in registers as 32 pairs
+// (v[j], v[j + 32]): butterfly stages h = 1..16 pair (j, j + h) and
+// (j + 32, j + 32 + h) alike, so two butterflies are one packed add.rn.f32x2
+// and one sub.rn.f32x2 (independent IEEE binary32 operations); stage 32 works
+// inside the pairs; stage 64 pairs the two threads: each takes its partner's
+// value p by an xor-shuffle and forms fl(p + sg * own) with sg = +1 (low
+// half: a + b) or -1 (high half: a - b) in one packed fma -- sg * own is exact,
+// so the single rounding is that of the butterfly's add or subtract.  Packed
+// subtraction a - b is likewise fma(b, -1, a).
+//
+// One __syncthreads per group: the row absmax (pair shuffle, then a
+// shared-memory atomicMax of the bit patterns, triple-buffered so that no
+// second barrier is needed) is complete after it, and every thread has read the
+// stage, which thread 0 then refills.
 // --------------------------------------------------------------------------
 
-__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-
-__device__ __forceinline__ void unpack_f2(uint64_t p, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
-}
-
-__device__ __forceinline__ uint64_t add_f2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
-__device__ __forceinline__ uint64_t sub_f2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
-__device__ __forceinline__ uint64_t mul_f2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
-__device__ __forceinline__ uint64_t fma_f2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_1() {
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
-}
-
-// Copies the rows of group g (those below `rows`) into a shared-memory stage.
-__device__ __forceinline__ void copy_group(const uint16_t* __restrict__ x, int64_t rows, int K,
-                                           int rpc, int64_t g, uint32_t stage) {
-  const int64_t row0 = g * rpc;
-  int64_t nrows = rows - row0;
-  if (nrows > rpc) nrows = rpc;
-  const int chunks = static_cast<int>(nrows) * (K / 8);  // 16-byte chunks
-  const char* src = reinterpret_cast<const char*>(x + row0 * static_cast<int64_t>(K));
-  for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
-    const int tb = c >> 4, i = c & 15;
-    cp_async16(stage + tb * 256 + ((i ^ (tb & 15)) << 4), src + static_cast<int64_t>(c) * 16);
-  }
-}
-
 template <int BITS>
-__global__ void __launch_bounds__(256) rotate_quant_half_kernel(
-    const uint16_t* __restrict__ x, int64_t rows, int K, int nblk, int rpc, int64_t num_groups,
-    float alpha, float scale_mul, int rotate, uint8_t* __restrict__ out,
-    float* __restrict__ scale_out) {
+__global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
+    const __grid_constant__ CUtensorMap tmx, int64_t rows, int K, int nblk, int rpc,
+    int64_t num_groups, int stages, float alpha, float scale_mul, int rotate,
+    uint8_t* __restrict__ out, float* __restrict__ scale_out) {
   constexpr int kQmax = BITS == 4 ? 7 : 127;
   constexpr int kOutBytes = 64 * BITS / 8;  // packed bytes per half block
-  extern __shared__ __align__(16) uint8_t qsmem[];
-  __shared__ unsigned int row_amax[2][128];
+  extern __shared__ __align__(1024) uint8_t qsmem_raw[];
+  __shared__ unsigned int row_amax[3][128];
+  __shared__ int abort_flag;
+
+  const uint32_t raw = smem_u32(qsmem_raw);
+  const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+  uint8_t* base = qsmem_raw + pad;
+  const uint32_t sbase = raw + pad;
+  const int stage_bytes = rpc * K * 2;                    // one group = the TMA box
+  const int stage_stride = (stage_bytes + 1023) / 1024 * 1024;
+  const uint32_t bars = sbase + stages * stage_stride;    // full[s] mbarriers
+  const int box_rows = rpc * K / 64;
 
   const int tid = threadIdx.x;
-  const int tb = tid >> 1;       // block within the group
-  const int up = tid & 1;        // which half of the block
+  const int tb = tid >> 1;  // block within the group
+  const int up = tid & 1;   // which half of the block
   const int rl = tb / nblk;
   const int blk = tb - rl * nblk;
   const bool worker = rl < rpc;
-  const int stage_bytes = rpc * K * 2;
-  const uint32_t stage0 = smem_u32(qsmem);
-  const uint64_t sg2 = pack_f2(up ? -1.f : 1.f, up ? -1.f : 1.f);
-
+  if (tid == 0) {
+    for (int i = 0; i < stages; ++i) mbar_init(bars + 8 * i, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
   if (tid < rpc) row_amax[0][tid] = 0u;
-  copy_group(x, rows, K, rpc, blockIdx.x, stage0);
-  cp_async_commit();
+  __syncthreads();
+  if (tid == 0) {
+    tma_prefetch_desc(&tmx);
+    for (int i = 0; i < stages; ++i) {
+      const int64_t g = blockIdx.x + static_cast<int64_t>(i) * gridDim.x;
+      if (g >= num_groups) break;
+      mbar_arrive_expect_tx(bars + 8 * i, stage_bytes);
+      tma_load_2d(sbase + i * stage_stride, &tmx, 0, static_cast<int>(g * box_rows), bars + 8 * i);
+    }
+  }
 
   int it = 0;
   for (int64_t g = blockIdx.x; g < num_groups; g += gridDim.x, ++it) {
-    const int par = it & 1;
-    const int64_t gn = g + gridDim.x;
-    if (gn < num_groups) copy_group(x, rows, K, rpc, gn, stage0 + (par ^ 1) * stage_bytes);
-    cp_async_commit();
-    cp_async_wait_1();
-    __syncthreads();  // the current stage is complete; row_amax[par ^ 1] is free
-    if (tid < rpc) row_amax[par ^ 1][tid] = 0u;
+    const int s = it % stages;
+    const uint32_t ph = static_cast<uint32_t>(it / stages) & 1u;
+    const int rb = it % 3;
+    if (tid < rpc) row_amax[(it + 1) % 3][tid] = 0u;  // last read two groups ago
+    mbar_wait_bounded(bars + 8 * s, ph, &abort_flag, kErrWaitTma);
 
     const int64_t row = g * rpc + rl;
     const bool active = worker && row < rows;
-    uint64_t p[32];  // (v[j], v[j + 32]) of this half block
+    float2 p[32];  // (v[j], v[j + 32]) of this half block
     if (active) {
-      const uint8_t* blkp = qsmem + par * stage_bytes + tb * 256;
+      const int R = 2 * tb + up;
+      const uint8_t* rowp = base + s * stage_stride + R * 128;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int c0 = 8 * up + i, c1 = 8 * up + i + 4;
-        const uint4 lo = *reinterpret_cast<const uint4*>(blkp + ((c0 ^ (tb & 15)) << 4));
-        const uint4 hi = *reinterpret_cast<const uint4*>(blkp + ((c1 ^ (tb & 15)) << 4));
+        const uint4 lo = *reinterpret_cast<const uint4*>(rowp + ((i ^ (R & 7)) << 4));
+        const uint4 hi = *reinterpret_cast<const uint4*>(rowp + (((i + 4) ^ (R & 7)) << 4));
         const uint32_t lw[4] = {lo.x, lo.y, lo.z, lo.w};
         const uint32_t hw[4] = {hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
@@ -227,38 +193,37 @@ __global__ void __launch_bounds__(256) rotate_quant_half_kernel(
           float a0, a1, b0, b1;
           bf16x2_to_f32(lw[k], a0, a1);
           bf16x2_to_f32(hw[k], b0, b1);
-          p[8 * i + 2 * k] = pack_f2(a0, b0);
-          p[8 * i + 2 * k + 1] = pack_f2(a1, b1);
+          p[8 * i + 2 * k] = make_float2(a0, b0);
+          p[8 * i + 2 * k + 1] = make_float2(a1, b1);
         }
       }
     } else {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) p[j] = 0ull;
+      for (int j = 0; j < 32; ++j) p[j] = make_float2(0.f, 0.f);
     }
 
     if (rotate) {
+      const float2 neg1 = make_float2(-1.f, -1.f);
 #pragma unroll
       for (int h = 1; h < 32; h <<= 1)
 #pragma unroll
         for (int j = 0; j < 32; ++j)
           if ((j & h) == 0) {
-            const uint64_t a = p[j], b = p[j + h];
-            p[j] = add_f2(a, b);
-            p[j + h] = sub_f2(a, b);
+            const float2 a = p[j], b = p[j + h];
+            p[j] = __fadd2_rn(a, b);
+            p[j + h] = __ffma2_rn(b, neg1, a);  // a - b, one rounding
           }
 #pragma unroll
       for (int j = 0; j < 32; ++j) {  // h = 32: (v[j], v[j + 32])
-        float a, b;
-        unpack_f2(p[j], a, b);
-        p[j] = pack_f2(__fadd_rn(a, b), __fsub_rn(a, b));
+        const float a = p[j].x, b = p[j].y;
+        p[j] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
       }
+      const float2 sg2 = make_float2(up ? -1.f : 1.f, up ? -1.f : 1.f);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {  // h = 64: the partner thread holds the other half
-        float a, b;
-        unpack_f2(p[j], a, b);
-        const float pa = __shfl_xor_sync(0xffffffffu, a, 1);
-        const float pb = __shfl_xor_sync(0xffffffffu, b, 1);
-        p[j] = fma_f2(sg2, p[j], pack_f2(pa, pb));
+        const float pa = __shfl_xor_sync(0xffffffffu, p[j].x, 1);
+        const float pb = __shfl_xor_sync(0xffffffffu, p[j].y, 1);
+        p[j] = __ffma2_rn(sg2, p[j], make_float2(pa, pb));
       }
     }
 
@@ -266,63 +231,74 @@ __global__ void __launch_bounds__(256) rotate_quant_half_kernel(
 #pragma unroll
     for (int k = 0; k < 4; ++k) m[k] = 0.f;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      float a, b;
-      unpack_f2(p[j], a, b);
-      m[j & 3] = fmaxf(m[j & 3], fmaxf(fabsf(a), fabsf(b)));
-    }
+    for (int j = 0; j < 32; ++j) m[j & 3] = fmaxf(m[j & 3], fmaxf(fabsf(p[j].x), fabsf(p[j].y)));
     float amax = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     // non-negative binary32 values order like their bit patterns
-    if (active && up == 0) atomicMax(&row_amax[par][rl], __float_as_uint(amax));
-    __syncthreads();  // row maxima complete; every thread is done reading the stage
+    if (active && up == 0) atomicMax(&row_amax[rb][rl], __float_as_uint(amax));
+    __syncthreads();  // row maxima complete; every thread has read stage s
+    if (abort_flag) break;
+    if (tid == 0) {
+      const int64_t gn = g + static_cast<int64_t>(stages) * gridDim.x;
+      if (gn < num_groups) {
+        mbar_arrive_expect_tx(bars + 8 * s, stage_bytes);
+        tma_load_2d(sbase + s * stage_stride, &tmx, 0, static_cast<int>(gn * box_rows),
+                    bars + 8 * s);
+      }
+    }
     if (!active) continue;
 
-    float s, inv;
-    row_factors<kQmax>(__uint_as_float(row_amax[par][rl]), alpha, s, inv);
-    if (blk == 0 && up == 0) scale_out[row] = __fmul_rn(s, scale_mul);
+    // every thread needs the multiplier; one thread per row stores the scale
+    const float t_row = __fmul_rn(alpha, __uint_as_float(row_amax[rb][rl]));
+    const bool zero_row = !(t_row >= kZeroRowT);
+    const float inv = zero_row ? 0.f : __fdiv_rn(static_cast<float>(kQmax), t_row);
+    if (blk == 0 && up == 0)
+      scale_out[row] = zero_row ? 0.f : __fmul_rn(__fdiv_rn(t_row, static_cast<float>(kQmax)), scale_mul);
 
-    const uint64_t inv2 = pack_f2(inv, inv);
-    const uint64_t magic2 = pack_f2(kRoundMagic, kRoundMagic);
-    uint32_t c[64];
+    const float2 inv2 = make_float2(inv, inv);
+    const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
+    constexpr float kQ = static_cast<float>(kQmax);
+    // Codes of 8 consecutive pairs = elements 8k..8k+7 (low halves) and
+    // 32+8k..32+8k+7 (high halves) of this half block.
+    uint32_t wlo[BITS == 4 ? 4 : 8], whi[BITS == 4 ? 4 : 8];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      float a, b;
-      unpack_f2(mul_f2(p[j], inv2), a, b);
-      a = fminf(fmaxf(a, -static_cast<float>(kQmax)), static_cast<float>(kQmax));
-      b = fminf(fmaxf(b, -static_cast<float>(kQmax)), static_cast<float>(kQmax));
-      float ca, cb;
-      unpack_f2(add_f2(pack_f2(a, b), magic2), ca, cb);
-      c[j] = __float_as_uint(ca);
-      c[j + 32] = __float_as_uint(cb);
+    for (int k = 0; k < 4; ++k) {
+      uint32_t clo[8], chi[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float2 r = __fmul2_rn(p[8 * k + e], inv2);
+        r.x = fminf(fmaxf(r.x, -kQ), kQ);
+        r.y = fminf(fmaxf(r.y, -kQ), kQ);
+        const float2 cb = __fadd2_rn(r, magic2);
+        clo[e] = __float_as_uint(cb.x);
+        chi[e] = __float_as_uint(cb.y);
+      }
+      if (BITS == 4) {
+        wlo[k] = pack8_int4(clo);
+        whi[k] = pack8_int4(chi);
+      } else {
+        wlo[2 * k] = pack4_int8(clo[0], clo[1], clo[2], clo[3]);
+        wlo[2 * k + 1] = pack4_int8(clo[4], clo[5], clo[6], clo[7]);
+        whi[2 * k] = pack4_int8(chi[0], chi[1], chi[2], chi[3]);
+        whi[2 * k + 1] = pack4_int8(chi[4], chi[5], chi[6], chi[7]);
+      }
     }
     uint8_t* dst =
         out + row * static_cast<int64_t>(K * BITS / 8) + blk * (2 * kOutBytes) + up * kOutBytes;
-    if (BITS == 4) {
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t w[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int e = 32 * q + 8 * k;
-          const uint32_t cc[8] = {c[e], c[e + 1], c[e + 2], c[e + 3],
-                                  c[e + 4], c[e + 5], c[e + 6], c[e + 7]};
-          w[k] = pack8_int4(cc);
-        }
-        *reinterpret_cast<uint4*>(dst + 16 * q) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
+    if (BITS == 4) {  // 16 bytes of elements 0..31, then 16 bytes of 32..63
+      *reinterpret_cast<uint4*>(dst) = make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
+      *reinterpret_cast<uint4*>(dst + 16) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
     } else {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t w[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int e = 16 * q + 4 * k;
-          w[k] = pack4_int8(c[e], c[e + 1], c[e + 2], c[e + 3]);
-        }
-        *reinterpret_cast<uint4*>(dst + 16 * q) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
+      *reinterpret_cast<uint4*>(dst) = make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
+      *reinterpret_cast<uint4*>(dst + 16) = make_uint4(wlo[4], wlo[5], wlo[6], wlo[7]);
+      *reinterpret_cast<uint4*>(dst + 32) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
+      *reinterpret_cast<uint4*>(dst + 48) = make_uint4(whi[4], whi[5], whi[6], whi[7]);
     }
+  }
+  if (abort_flag) {
+    // a wait gave up: let copies already in flight land before the CTA exits
+    const unsigned long long t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
   }
 }
 
@@ -460,19 +436,27 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
                                             float scale_mul, int rotate, uint8_t* out,
                                             float* scale, cudaStream_t stream) {
   const int nblk = K / 128;
-  if (nblk <= 128) {
-    const int rpc = choose_rows_per_cta(nblk);
+  const int rpc = nblk <= 128 ? choose_rows_per_cta(nblk) : 0;
+  const int64_t groups = rpc ? (rows + rpc - 1) / rpc : 0;
+  // TMA row coordinates are 32-bit: groups * (rpc * K / 64) must stay below 2^31
+  if (nblk <= 128 && groups * (static_cast<int64_t>(rpc) * K / 64) < (int64_t{1} << 31)) {
     const int threads = (rpc * 2 * nblk + 31) / 32 * 32;
-    const int64_t groups = (rows + rpc - 1) / rpc;
-    const int smem = 2 * rpc * K * 2;  // two stages of rpc rows
-    auto kern = rotate_quant_half_kernel<BITS>;
+    const int stage_stride = (rpc * K * 2 + 1023) / 1024 * 1024;
+    // Two stages: measured faster than three or four, which cost resident CTAs
+    // (the kernel is latency-bound and more warps per SM win).
+    const int stages = 2;
+    const int smem = stages * stage_stride + 8 * stages + 1024;
+    CUtensorMap tmx;
+    if (!make_tensor_map_2d(&tmx, x, 64, static_cast<uint64_t>(rows) * K / 64, 64, rpc * K / 64,
+                            true, 2))
+      return cudaErrorInvalidValue;
+    auto kern = rotate_quant_tma_kernel<BITS>;
     cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    int per_sm = 0, dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-      return e;
+    int per_sm = 0;
+    const int sms = sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
     if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem)) !=
         cudaSuccess)
       return e;
@@ -480,7 +464,7 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
     int64_t grid = static_cast<int64_t>(sms) * per_sm;
     if (grid > groups) grid = groups;
     kern<<<static_cast<unsigned>(grid), threads, smem, stream>>>(
-        x, rows, K, nblk, rpc, groups, alpha, scale_mul, rotate, out, scale);
+        tmx, rows, K, nblk, rpc, groups, stages, alpha, scale_mul, rotate, out, scale);
     return cudaGetLastError();
   }
   // Rows up to 2048 groups run with at most 256 threads so each thread keeps
