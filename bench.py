@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extras", action="store_true",
+                   help="skip the per-config table and the quality report")
     p.add_argument("--tokens", type=int, default=None,
                    help="override M (profiling captures of a smaller case of the same shape)")
     return p.parse_args()
@@ -171,6 +173,94 @@ class OracleSample:
                 "tokens_per_s": rows / dt}
 
 
+def time_layer(qs, torch, x, wp, ws, bias, bits, alpha, stream, steps=5, warmup=2):
+    """Mean CUDA-event times (ms) of the activation kernel and the GEMM for one layer."""
+    M, K = x.shape
+    N = wp.shape[0]
+    dev = x.device
+    xp = torch.empty((M, K * bits // 8), dtype=torch.uint8, device=dev)
+    xs = torch.empty((M,), dtype=torch.float32, device=dev)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    for _ in range(warmup):
+        qs.qs_quant_act(x, M, K, bits, alpha, 0, xp, xs, stream)
+        qs.qs_qlinear(xp, xs, wp, ws, bias, M, N, K, bits, out, stream)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for e in ev:
+        e[0].record(stream)
+        qs.qs_quant_act(x, M, K, bits, alpha, 0, xp, xs, stream)
+        e[1].record(stream)
+        qs.qs_qlinear(xp, xs, wp, ws, bias, M, N, K, bits, out, stream)
+        e[2].record(stream)
+    stream.synchronize()
+    q = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+    g = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+    return q, g, out
+
+
+def all_configs(qs, torch, I, dev, stream):
+    """Per-configuration throughput on one GPU (every seeded synthetic shape)."""
+    res = {}
+    for cfg in I.LAYER_CONFIGS:
+        d = I.make_layer(cfg)
+        with torch.cuda.stream(stream):
+            x, w, b = d["x"].to(dev), d["w"].to(dev), d["bias"].to(dev)
+            wp, ws = qs.pack_weights(w, cfg.bits, stream=stream)
+        q, g, _ = time_layer(qs, torch, x, wp, ws, b, cfg.bits, cfg.alpha, stream)
+        res[cfg.name] = {"bits": cfg.bits, "quant_ms": q, "gemm_ms": g,
+                         "TOPS": cfg.ops / ((q + g) * 1e-3) / 1e12,
+                         "gemm_TOPS": cfg.ops / (g * 1e-3) / 1e12,
+                         "tokens_per_s": cfg.M / ((q + g) * 1e-3)}
+        del x, w, b, wp, ws
+    ch = I.make_chain(I.WAN_CHAIN)
+    M = I.WAN_CHAIN.M
+    layers, total, gelu_ms, ops, up_out = {}, 0.0, 0.0, 0, None
+    for L in ch["layers"]:
+        with torch.cuda.stream(stream):
+            w, b = L["w"].to(dev), L["bias"].to(dev)
+            wp, ws = qs.pack_weights(w, L["bits"], stream=stream)
+            if L["x"] is not None:
+                x = L["x"].to(dev)
+            else:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                x = torch.empty_like(up_out)
+                qs.gelu(up_out, stream=stream, out=x)
+                e0.record(stream)
+                for _ in range(5):
+                    qs.gelu(up_out, stream=stream, out=x)
+                e1.record(stream)
+                stream.synchronize()
+                gelu_ms = e0.elapsed_time(e1) / 5
+        q, g, out = time_layer(qs, torch, x, wp, ws, b, L["bits"], ch["alpha"], stream)
+        if L["name"] == "ffn_up":
+            up_out = out
+        lops = 2 * M * L["K"] * L["N"]
+        ops += lops
+        total += q + g
+        layers[L["name"]] = {"bits": L["bits"], "K": L["K"], "N": L["N"], "quant_ms": q,
+                             "gemm_ms": g, "TOPS": lops / ((q + g) * 1e-3) / 1e12}
+    res[I.WAN_CHAIN.name] = {"bits_mask": ch["bits"], "layers": layers,
+                             "tokens_per_s": M / (total * 1e-3),
+                             "tokens_per_s_with_gelu": M / ((total + gelu_ms) * 1e-3),
+                             "gelu_ms": gelu_ms, "TOPS": ops / (total * 1e-3) / 1e12}
+    return res
+
+
+def quality(qs, torch, x, w, bias, bits, alpha, stream, rows=256):
+    """Relative Frobenius error and SQNR of the layer against the unquantised
+    binary64 product, with and without the Hadamard rotation (first `rows` tokens)."""
+    xs_, ws_, b = x[:rows].contiguous(), w, bias
+    ref = xs_.double() @ ws_.double().t() + b.double()
+    out = {}
+    for name, flags in (("rotated", 0), ("unrotated", qs.QS_FLAG_NO_ROTATE)):
+        wp, wsc = qs.pack_weights(ws_, bits, flags, stream=stream)
+        xp, xsc = qs.quant_act(xs_, bits, alpha, flags, stream=stream)
+        y = qs.qlinear(xp, xsc, wp, wsc, b, bits, x.shape[1], stream=stream).double()
+        stream.synchronize()
+        err = (y - ref).norm() / ref.norm()
+        out[name] = {"rel_fro_err": float(err), "sqnr_db": float(-20 * torch.log10(err))}
+    return out
+
+
 def run_reference(args, rank, world):
     """The CPU oracle timed as a bounded sample per step (rank 0 only)."""
     if rank != 0:
@@ -288,9 +378,12 @@ def main():
     out_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
     e2e_steps = max(1, args.e2e_steps)
 
-    def e2e_step():
+    ws_bytes = qs.qs_linear_workspace_bytes(M, K, bits)
+    workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+
+    def e2e_step():  # one C call for the layer, host buffers in and out
         x.copy_(x_host, non_blocking=True)
-        step()
+        qs.qs_linear(x, M, K, alpha, wp, ws, bias, N, bits, workspace, ws_bytes, out, stream)
         out_host.copy_(out, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -310,6 +403,10 @@ def main():
         dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
     e2e_ms = float(e2e_ms.item())
 
+    extra = {}
+    if world == 1 and not args.no_extras:
+        extra["quality"] = quality(qs, torch, x, d["w"].to(dev), bias, bits, alpha, stream)
+        extra["configs"] = all_configs(qs, torch, I, dev, stream)
     if rank == 0:
         pk, src = peaks()
         int8_peak = pk["bf16_tflops"] * INT8_PER_BF16
@@ -341,9 +438,11 @@ def main():
             "e2e": {"value": ops_per_step * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": x_host.numel() * 2,
                     "d2h_bytes_per_step": out_host.numel() * 2,
-                    "ms_per_step": e2e_ms, "steps": e2e_steps},
+                    "ms_per_step": e2e_ms, "steps": e2e_steps,
+                    "call": "qs_linear (C ABI), pinned host x in, bf16 output back"},
             "clocks": clocks,
         }
+        line.update(extra)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = OracleSample(d, bits, alpha).baseline()
         print(json.dumps(line), flush=True)

@@ -5,7 +5,8 @@ this package holds its build script, a ctypes binding and the seeded synthetic
 inputs used by the tests and the benchmark.
 """
 from .binding import (  # noqa: F401
-    EXPORTS, QS_FLAG_NO_ROTATE, QS_MAX_K, QSError, QuantLinear, gelu, load, pack_weights, qgemm_s32,
-    qlinear, qs_device_error, qs_gelu_bf16, qs_pack_weights, qs_qgemm_s32, qs_qlinear, qs_quant_act,
-    qs_version, quant_act,
+    EXPORTS, QS_FLAG_NO_ROTATE, QS_MAX_K, QSError, QuantLinear, gelu, linear, load, pack_weights,
+    qgemm_s32, qlinear, qs_device_error, qs_gelu_bf16, qs_linear, qs_linear_workspace_bytes,
+    qs_pack_weights, qs_qgemm_s32, qs_qlinear, qs_quant_act, qs_selftest_timeout, qs_version,
+    quant_act,
 )

@@ -26,7 +26,8 @@ QS_MAX_K = 65536
 STATUS = {0: "QS_OK", 1: "QS_ERR_NULL", 2: "QS_ERR_SHAPE", 3: "QS_ERR_BITS", 4: "QS_ERR_ALIGN",
           5: "QS_ERR_RANGE", 6: "QS_ERR_CUDA", 7: "QS_ERR_TIMEOUT", 8: "QS_ERR_PTR"}
 EXPORTS = ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qgemm_s32", "qs_gelu_bf16",
-           "qs_device_error", "qs_status_str", "qs_version")
+           "qs_linear_workspace_bytes", "qs_linear", "qs_selftest_timeout", "qs_device_error",
+           "qs_status_str", "qs_version")
 
 
 class QSError(RuntimeError):
@@ -53,12 +54,16 @@ def load() -> ctypes.CDLL:
     L.qs_qlinear.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp, vp]
     L.qs_qgemm_s32.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp]
     L.qs_gelu_bf16.argtypes = [vp, i64, vp, vp]
+    L.qs_linear_workspace_bytes.argtypes = [i64, i64, i32]
+    L.qs_linear_workspace_bytes.restype = i64
+    L.qs_linear.argtypes = [vp, i64, i64, f32, vp, vp, vp, i64, i32, vp, i64, vp, vp]
+    L.qs_selftest_timeout.argtypes = [i64, vp]
     L.qs_device_error.argtypes = [vp]
     L.qs_status_str.argtypes = [i32]
     L.qs_status_str.restype = ctypes.c_char_p
     L.qs_version.restype = ctypes.c_char_p
     for name in ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qgemm_s32",
-                 "qs_gelu_bf16", "qs_device_error"):
+                 "qs_gelu_bf16", "qs_linear", "qs_selftest_timeout", "qs_device_error"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -140,6 +145,26 @@ def qs_gelu_bf16(x, n, y, stream=None):
     _check(load().qs_gelu_bf16(_p(x), n, _p(y), _s(stream)), "qs_gelu_bf16")
 
 
+def qs_linear_workspace_bytes(M, K, bits) -> int:
+    return int(load().qs_linear_workspace_bytes(M, K, bits))
+
+
+def qs_linear(x, M, K, alpha, w_packed, w_scale, bias, N, bits, workspace, workspace_bytes, out,
+              stream=None):
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(w_packed, torch.uint8, "w_packed")
+    _cuda(w_scale, torch.float32, "w_scale")
+    _cuda(bias, torch.bfloat16, "bias")
+    _cuda(workspace, torch.uint8, "workspace")
+    _cuda(out, torch.bfloat16, "out")
+    _check(load().qs_linear(_p(x), M, K, float(alpha), _p(w_packed), _p(w_scale), _p(bias), N, bits,
+                            _p(workspace), workspace_bytes, _p(out), _s(stream)), "qs_linear")
+
+
+def qs_selftest_timeout(timeout_us: int, stream=None) -> None:
+    _check(load().qs_selftest_timeout(timeout_us, _s(stream)), "qs_selftest_timeout")
+
+
 def qs_device_error(stream=None) -> int:
     return int(load().qs_device_error(_s(stream)))
 
@@ -194,9 +219,27 @@ def gelu(x: torch.Tensor, stream=None, out=None):
     return y
 
 
+def linear(x, w_packed, w_scale, bias, bits: int, alpha: float = 1.0, workspace=None,
+           stream=None, out=None):
+    """bf16 activations [M, K] -> bf16 [M, N] through qs_linear (one C call)."""
+    M, K = x.shape
+    N = w_packed.shape[0]
+    need = qs_linear_workspace_bytes(M, K, bits)
+    if need < 0:
+        raise QSError(2, "qs_linear_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    qs_linear(x, M, K, alpha, w_packed, w_scale, bias, N, bits, workspace, workspace.numel(), out,
+              stream)
+    return out
+
+
 class QuantLinear:
-    """A Hadamard-rotated W4A4 / W8A8 linear layer: weights packed once, each
-    call quantizes the activations (one kernel) and runs the GEMM (one kernel)."""
+    """A Hadamard-rotated W4A4 / W8A8 linear layer: weights packed once; each
+    call runs qs_linear (the activation kernel, then the GEMM) on a workspace
+    the layer keeps and grows as needed."""
 
     def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None, bits: int,
                  alpha: float = 1.0):
@@ -204,8 +247,11 @@ class QuantLinear:
         self.bits, self.alpha = bits, alpha
         self.w_packed, self.w_scale = pack_weights(weight, bits)
         self.bias = bias
+        self.workspace = None
 
     def __call__(self, x: torch.Tensor, stream=None, out=None) -> torch.Tensor:
-        xp, xs = quant_act(x, self.bits, self.alpha, stream=stream)
-        return qlinear(xp, xs, self.w_packed, self.w_scale, self.bias, self.bits, self.K,
-                       stream=stream, out=out)
+        need = qs_linear_workspace_bytes(x.shape[0], self.K, self.bits)
+        if self.workspace is None or self.workspace.numel() < need:
+            self.workspace = torch.empty((max(need, 0),), dtype=torch.uint8, device=x.device)
+        return linear(x, self.w_packed, self.w_scale, self.bias, self.bits, self.alpha,
+                      self.workspace, stream=stream, out=out)

@@ -168,6 +168,36 @@ qs_status qs_qgemm_s32(const void* x_packed, const void* w_packed, int64_t M, in
                                             acc, s);
 }
 
+int64_t qs_linear_workspace_bytes(int64_t M, int64_t K, int bits) {
+  if (check_bits(bits) != QS_OK || check_rows_k(M, K) != QS_OK) return -1;
+  const int64_t packed = (M * K * bits / 8 + 255) / 256 * 256;
+  return packed + 4 * M;
+}
+
+qs_status qs_linear(const void* x_bf16, int64_t M, int64_t K, float alpha, const void* w_packed,
+                    const float* w_scale, const void* bias_bf16, int64_t N, int bits,
+                    void* workspace, int64_t workspace_bytes, void* out_bf16, void* stream) {
+  if (!x_bf16 || !w_packed || !w_scale || !workspace || !out_bf16) return QS_ERR_NULL;
+  QS_TRY(check_gemm_args(workspace, w_packed, out_bf16, M, N, K, bits));
+  if (!(alpha > 0.0f && alpha <= 1.0f)) return QS_ERR_RANGE;
+  const int64_t need = qs_linear_workspace_bytes(M, K, bits);
+  if (need < 0) return QS_ERR_SHAPE;
+  if (workspace_bytes < need) return QS_ERR_RANGE;
+  // everything both launches will check, before the first one
+  if (!aligned16(x_bf16) || !aligned16(w_scale) || (bias_bf16 && !aligned16(bias_bf16)))
+    return QS_ERR_ALIGN;
+  QS_TRY(check_device_ptr(x_bf16));
+  QS_TRY(check_device_ptr(w_packed));
+  QS_TRY(check_device_ptr(w_scale));
+  QS_TRY(check_device_ptr(workspace));
+  QS_TRY(check_device_ptr(out_bf16));
+  if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
+  uint8_t* xp = static_cast<uint8_t*>(workspace);
+  float* xs = reinterpret_cast<float*>(xp + (M * K * bits / 8 + 255) / 256 * 256);
+  QS_TRY(qs_quant_act(x_bf16, M, K, bits, alpha, 0u, xp, xs, stream));
+  return qs_qlinear(xp, xs, w_packed, w_scale, bias_bf16, M, N, K, bits, out_bf16, stream);
+}
+
 qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream) {
   if (!x_bf16 || !y_bf16) return QS_ERR_NULL;
   if (n <= 0) return QS_ERR_SHAPE;
@@ -183,6 +213,13 @@ qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream
   if (blocks < 1) blocks = 1;
   qs::gelu_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint16_t*>(x_bf16), n, static_cast<uint16_t*>(y_bf16));
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status qs_selftest_timeout(int64_t timeout_us, void* stream) {
+  if (timeout_us < 1 || timeout_us > 1000000) return QS_ERR_RANGE;
+  qs::selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(timeout_us) * 1000ull);
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 

@@ -41,4 +41,18 @@ __global__ void __launch_bounds__(256) gelu_bf16_kernel(const uint16_t* x, int64
   }
 }
 
+// Diagnostic: waits on an mbarrier that nothing ever arrives on, with a
+// bounded wait; the wait gives up after `limit_ns` and records the timeout in
+// the library's device error word.  Exercises the failure path of the bounded
+// waits without faulting or hanging the GPU.
+__global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    fence_mbar_init();
+    mbar_wait_limit(b, 0, limit_ns, kErrSelfTest);
+  }
+}
+
 }  // namespace qs

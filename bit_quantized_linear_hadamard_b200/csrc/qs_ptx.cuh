@@ -70,6 +70,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+enum : unsigned int { kErrSelfTest = 1u << 5 };
+
+// Bounded wait with an explicit limit, for the diagnostic self-test.
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity,
+                                                unsigned long long limit_ns, unsigned int err) {
+  const unsigned long long t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > limit_ns) {
+      atomicOr(&g_error_word, err);
+      return false;
+    }
+  }
+  return true;
+}
+
 // Waits for the phase of parity `parity` of the barrier to complete.  Gives up
 // (returns false, records `err` in the device error word and raises the
 // CTA-wide abort flag) after kWaitTimeoutNs, or as soon as another role of the

@@ -126,11 +126,47 @@ QS_API qs_status qs_qgemm_s32(const void* x_packed, const void* w_packed, int64_
                        int64_t K, int bits, int32_t* acc, void* stream);
 
 /*
+ * qs_linear_workspace_bytes — bytes of device scratch that qs_linear needs for
+ * M tokens of K inputs at `bits`: the packed activations (M*K*bits/8 bytes,
+ * rounded up to 256) followed by the per-token scales (4*M bytes).  Returns
+ * -1 for arguments qs_linear would reject.
+ */
+QS_API int64_t qs_linear_workspace_bytes(int64_t M, int64_t K, int bits);
+
+/*
+ * qs_linear — the whole layer in one call: qs_quant_act into the caller's
+ * workspace, then qs_qlinear (DVD-Quant §2.B: rotate and scale the
+ * activations at run time, then the low-bit product).  Results are identical
+ * to calling the two entry points in sequence.
+ *   x_bf16             [M, K] bf16
+ *   alpha              clip ratio in (0, 1]
+ *   w_packed, w_scale  from qs_pack_weights (same K and bits)
+ *   bias_bf16          [N] bf16 or NULL
+ *   workspace          device scratch of at least qs_linear_workspace_bytes(M, K, bits)
+ *                      bytes, 16-byte aligned; overwritten; must not overlap other arguments
+ *   out_bf16           [M, N] bf16, written
+ */
+QS_API qs_status qs_linear(const void* x_bf16, int64_t M, int64_t K, float alpha,
+                           const void* w_packed, const float* w_scale, const void* bias_bf16,
+                           int64_t N, int bits, void* workspace, int64_t workspace_bytes,
+                           void* out_bf16, void* stream);
+
+/*
  * qs_gelu_bf16 — elementwise GELU (exact erf form, binary32 arithmetic,
  * bf16 in and out) used between the ffn-up and ffn-down linears of a
  * transformer block chain.  n elements; x and y may alias.
  */
 QS_API qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream);
+
+/*
+ * qs_selftest_timeout — diagnostic of the failure path: enqueues one tiny
+ * kernel whose bounded mbarrier wait can never complete (nothing arrives); the
+ * wait gives up after `timeout_us` microseconds (1 .. 1000000), records the
+ * timeout in the device error word and the kernel returns.  A following
+ * qs_device_error() then reports QS_ERR_TIMEOUT and the context stays usable.
+ * No counterpart on the pages.
+ */
+QS_API qs_status qs_selftest_timeout(int64_t timeout_us, void* stream);
 
 /*
  * qs_device_error — synchronises `stream`, then returns and clears the

@@ -120,3 +120,25 @@ def test_binding_raises_without_cuda_tensors():
     import torch
     with pytest.raises(TypeError):
         binding.quant_act(torch.zeros(4, 128, dtype=torch.bfloat16), 4)
+
+
+def test_linear_validation_and_workspace(lib):
+    assert lib.qs_linear_workspace_bytes(256, 512, 4) == 256 * 256 + 4 * 256
+    assert lib.qs_linear_workspace_bytes(3, 128, 4) == 256 + 12          # packed part rounded to 256
+    assert lib.qs_linear_workspace_bytes(3, 128, 8) == 512 + 12
+    assert lib.qs_linear_workspace_bytes(3, 100, 4) == -1
+    assert lib.qs_linear_workspace_bytes(3, 128, 5) == -1
+    need = lib.qs_linear_workspace_bytes(8, 128, 4)
+    f = lib.qs_linear
+    assert f(NUL, 8, 128, 1.0, B, C, NUL, 256, 4, D, need, A, NUL) == NULL
+    assert f(A, 8, 128, 1.0, B, C, NUL, 256, 4, NUL, need, D, NUL) == NULL
+    assert f(A, 8, 128, 1.0, B, C, NUL, 250, 4, D, need, A, NUL) == SHAPE
+    assert f(A, 8, 128, 1.5, B, C, NUL, 256, 4, D, need, A, NUL) == RANGE
+    assert f(A, 8, 128, 1.0, B, C, NUL, 256, 4, D, need - 1, A, NUL) == RANGE
+    assert f(MIS, 8, 128, 1.0, B, C, NUL, 256, 4, D, need, A, NUL) == ALIGN
+    assert f(A, 8, 128, 1.0, B, C, MIS, 256, 4, D, need, A, NUL) == ALIGN
+
+
+def test_selftest_timeout_validation(lib):
+    assert lib.qs_selftest_timeout(0, NUL) == RANGE
+    assert lib.qs_selftest_timeout(1000001, NUL) == RANGE

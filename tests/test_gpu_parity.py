@@ -203,6 +203,21 @@ def test_qlinear_null_bias_and_zero_rows():
     assert not got[3].any() and not got[129].any()
 
 
+@pytest.mark.parametrize("bits,alpha", [(4, 0.9), (8, 1.0)])
+@pytest.mark.parametrize("M,N,K", [(300, 768, 640), (1, 16, 128), (513, 528, 1152)])
+def test_linear_one_call_matches_two_calls_and_oracle(M, N, K, bits, alpha):
+    d = I.make_shape(seed=7 * M + K, M=M, K=K, N=N, bits=bits, alpha=alpha, outlier_factor=50.0)
+    g = run_layer(d, bits, alpha)
+    need = qs.qs_linear_workspace_bytes(M, K, bits)
+    ws = torch.full((need,), 0xA5, dtype=torch.uint8, device="cuda")  # dirty scratch
+    out = qs.linear(d["x"].cuda(), g["wp"], g["ws"], d["bias"].cuda(), bits, alpha, workspace=ws)
+    torch.cuda.synchronize()
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, g["out"].view(torch.int16).cpu().numpy().view(np.uint16))
+    r = O.qlinear(bits16(d["x"]), bits16(d["w"]), bits16(d["bias"]), bits, alpha)
+    assert np.array_equal(got, r["out"])
+
+
 def test_tiny_config_full_parity():
     d = I.make_layer(I.TINY)
     g = run_layer(d, 4, 1.0)
