@@ -26,8 +26,9 @@ QS_MAX_K = 65536
 STATUS = {0: "QS_OK", 1: "QS_ERR_NULL", 2: "QS_ERR_SHAPE", 3: "QS_ERR_BITS", 4: "QS_ERR_ALIGN",
           5: "QS_ERR_RANGE", 6: "QS_ERR_CUDA", 7: "QS_ERR_TIMEOUT", 8: "QS_ERR_PTR"}
 EXPORTS = ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qgemm_s32", "qs_gelu_bf16",
-           "qs_linear_workspace_bytes", "qs_linear", "qs_selftest_timeout", "qs_device_error",
-           "qs_status_str", "qs_version")
+           "qs_linear_workspace_bytes", "qs_linear", "qs_linear_noalloc", "qs_selftest_timeout",
+           "qs_device_error", "qs_status_str", "qs_version")
+QS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class QSError(RuntimeError):
@@ -57,13 +58,15 @@ def load() -> ctypes.CDLL:
     L.qs_linear_workspace_bytes.argtypes = [i64, i64, i32]
     L.qs_linear_workspace_bytes.restype = i64
     L.qs_linear.argtypes = [vp, i64, i64, f32, vp, vp, vp, i64, i32, vp, i64, vp, vp]
+    L.qs_linear_noalloc.argtypes = [vp, i64, i64, f32, vp, vp, vp, i64, i32, vp, vp]
     L.qs_selftest_timeout.argtypes = [i64, vp]
     L.qs_device_error.argtypes = [vp]
     L.qs_status_str.argtypes = [i32]
     L.qs_status_str.restype = ctypes.c_char_p
     L.qs_version.restype = ctypes.c_char_p
     for name in ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qgemm_s32",
-                 "qs_gelu_bf16", "qs_linear", "qs_selftest_timeout", "qs_device_error"):
+                 "qs_gelu_bf16", "qs_linear", "qs_linear_noalloc", "qs_selftest_timeout",
+                 "qs_device_error"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -159,6 +162,18 @@ def qs_linear(x, M, K, alpha, w_packed, w_scale, bias, N, bits, workspace, works
     _cuda(out, torch.bfloat16, "out")
     _check(load().qs_linear(_p(x), M, K, float(alpha), _p(w_packed), _p(w_scale), _p(bias), N, bits,
                             _p(workspace), workspace_bytes, _p(out), _s(stream)), "qs_linear")
+
+
+def qs_linear_noalloc(x, M, K, alpha, w_packed, w_scale, bias, N, bits, out, stream=None):
+    """qs_linear on the library's own fixed scratch buffer (for callers that
+    cannot allocate device memory when they run the layer); nothing is allocated."""
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(w_packed, torch.uint8, "w_packed")
+    _cuda(w_scale, torch.float32, "w_scale")
+    _cuda(bias, torch.bfloat16, "bias")
+    _cuda(out, torch.bfloat16, "out")
+    _check(load().qs_linear_noalloc(_p(x), M, K, float(alpha), _p(w_packed), _p(w_scale), _p(bias),
+                                    N, bits, _p(out), _s(stream)), "qs_linear_noalloc")
 
 
 def qs_selftest_timeout(timeout_us: int, stream=None) -> None:

@@ -8,6 +8,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "qs.h"
 #include "qs_gemm.cuh"
@@ -92,6 +93,31 @@ qs_status check_gemm_args(const void* xp, const void* wp, const void* out, int64
   if (M > INT32_MAX || N > INT32_MAX) return QS_ERR_RANGE;
   if (!aligned16(xp) || !aligned16(wp) || !aligned16(out)) return QS_ERR_ALIGN;
   return QS_OK;
+}
+
+// Scratch of qs_linear_noalloc: one fixed buffer per device, in the module's
+// global memory (no allocation).  Host code only names the symbol; its device
+// address is looked up once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[QS_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[64] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device (looked up on the
+// first call for that device), or nullptr if the lookup failed.
+void* noalloc_scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_noalloc_addr[dev] = p;
+  }
+  return g_noalloc_addr[dev];
 }
 
 }  // namespace
@@ -214,6 +240,18 @@ qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream
   qs::gelu_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint16_t*>(x_bf16), n, static_cast<uint16_t*>(y_bf16));
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status qs_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, float alpha,
+                            const void* w_packed, const float* w_scale, const void* bias_bf16,
+                            int64_t N, int bits, void* out_bf16, void* stream) {
+  const int64_t need = qs_linear_workspace_bytes(M, K, bits);
+  if (need < 0) return check_bits(bits) != QS_OK ? QS_ERR_BITS : QS_ERR_SHAPE;
+  if (need > static_cast<int64_t>(QS_NOALLOC_SCRATCH_BYTES)) return QS_ERR_RANGE;
+  void* scratch = noalloc_scratch_address();
+  if (!scratch) return QS_ERR_CUDA;
+  return qs_linear(x_bf16, M, K, alpha, w_packed, w_scale, bias_bf16, N, bits, scratch,
+                   static_cast<int64_t>(QS_NOALLOC_SCRATCH_BYTES), out_bf16, stream);
 }
 
 qs_status qs_selftest_timeout(int64_t timeout_us, void* stream) {

@@ -159,6 +159,34 @@ QS_API qs_status qs_linear(const void* x_bf16, int64_t M, int64_t K, float alpha
 QS_API qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream);
 
 /*
+ * qs_linear_noalloc — qs_linear for callers that cannot allocate device memory
+ * when they run the layer: a host runtime that owns the whole device memory
+ * pool and forbids other allocations, a plugin interface that hands over only
+ * inputs and outputs with no workspace, or a latency-critical loop that cannot
+ * afford an allocation (and the synchronisation cudaMalloc implies) per call.
+ * The scratch qs_linear would take from the caller comes instead from a
+ * buffer of QS_NOALLOC_SCRATCH_BYTES that the library keeps in device memory
+ * (every GPU that loads libqs.so holds it until the process exits).  Nothing
+ * is allocated by this call.
+ *   Arguments as qs_linear, minus the workspace.  Calls needing more scratch
+ *   than the buffer, i.e. qs_linear_workspace_bytes(M, K, bits) >
+ *   QS_NOALLOC_SCRATCH_BYTES, are rejected with QS_ERR_RANGE (W4, K = 5120:
+ *   up to 3271 tokens per call).
+ *   The first call on a device looks up the buffer's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls share the one buffer, which keeps the previous call's contents
+ *   (every byte the layer reads from it is written earlier in the same call,
+ *   so nothing needs clearing); calls that may overlap on the GPU -- on
+ *   different streams, or from different host threads -- race on it.
+ * The pages have no counterpart: this is a deployment variant of qs_linear.
+ */
+#define QS_NOALLOC_SCRATCH_BYTES (8u << 20)
+QS_API qs_status qs_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, float alpha,
+                                   const void* w_packed, const float* w_scale,
+                                   const void* bias_bf16, int64_t N, int bits, void* out_bf16,
+                                   void* stream);
+
+/*
  * qs_selftest_timeout — diagnostic of the failure path: enqueues one tiny
  * kernel whose bounded mbarrier wait can never complete (nothing arrives); the
  * wait gives up after `timeout_us` microseconds (1 .. 1000000), records the
