@@ -34,7 +34,10 @@ The pages leave the details open; the readings taken here are:
   symmetric range [-qmax, qmax] (-8 / -128 never produced).  A row with
   t < 2^-120 (all-zero, or so small that qmax / t would overflow binary32) is
   a zero row: s = 0 and all codes 0.
-* Quantise: q = clamp(rint_half_even(fl(u * inv)), -qmax, qmax).
+* Quantise: q = clamp(rint_half_even(u * inv), -qmax, qmax) with the product
+  u * inv taken exactly (it is exact in binary64 for binary32 operands) and
+  rounded once, to the nearest integer.  The clip ratio is limited to
+  alpha >= 2^-14, so |u * inv| <= qmax / alpha < 2^22.
 * Pack: row-major, int8 as two's complement bytes; int4 as two's complement
   nibbles, element 2j in the low nibble and element 2j+1 in the high nibble of
   byte j.
@@ -141,10 +144,11 @@ def row_scales(u: np.ndarray, bits: int, alpha: float) -> tuple[np.ndarray, np.n
 
 
 def quantize_with_scale(u: np.ndarray, inv: np.ndarray, bits: int) -> np.ndarray:
-    """q = clamp(rint_half_even(fl(u * inv)), -qmax, qmax); zero rows (inv == 0) give 0."""
-    qmax = np.float32(QMAX[bits])
-    inv = np.asarray(inv, dtype=np.float32)
-    r = u * inv[:, None]
+    """q = clamp(rint_half_even(u * inv), -qmax, qmax), the product exact (binary64
+    holds the product of two binary32 values exactly); zero rows (inv == 0) give 0."""
+    qmax = float(QMAX[bits])
+    inv = np.asarray(inv, dtype=np.float32).astype(np.float64)
+    r = np.asarray(u, dtype=np.float32).astype(np.float64) * inv[:, None]
     q = np.rint(r)
     q = np.minimum(np.maximum(q, -qmax), qmax)
     return q.astype(np.int8)
@@ -160,8 +164,8 @@ def quantize_rows(x_bits: np.ndarray, bits: int, alpha: float,
     x = bf16_bits_to_f32(np.asarray(x_bits))
     if x.ndim != 2:
         raise ValueError("expected a 2-D array")
-    if not (0.0 < alpha <= 1.0):
-        raise ValueError("alpha must be in (0, 1]")
+    if not (2.0 ** -14 <= alpha <= 1.0):
+        raise ValueError("alpha must be in [2^-14, 1]")
     u = fwht128_blocks(x) if rotate else x.copy()
     s, inv = row_scales(u, bits, alpha)
     return quantize_with_scale(u, inv, bits), s

@@ -31,7 +31,7 @@ def _fwht_with(stage_fn, stages=(1, 2, 4, 8, 16, 32, 64)):
 def _quantize_with(round_fn=np.rint, lo_extra=0):
     def f(u, inv, bits):
         qmax = np.float32(O.QMAX[bits])
-        r = u * np.asarray(inv, dtype=np.float32)[:, None]
+        r = u.astype(np.float64) * np.asarray(inv, dtype=np.float32).astype(np.float64)[:, None]
         q = round_fn(r)
         q = np.minimum(np.maximum(q, -qmax - lo_extra), qmax)
         return q.astype(np.int8)
@@ -100,7 +100,14 @@ def _pack_weights_no_fold(w_bits, bits, rotate=True):
     return O.quantize_rows(w_bits, bits, 1.0, rotate)
 
 
+def _quantize_double_rounding(u, inv, bits):
+    qmax = np.float32(O.QMAX[bits])
+    r = (np.asarray(u, np.float32) * np.asarray(inv, np.float32)[:, None]).astype(np.float32)
+    return np.minimum(np.maximum(np.rint(r), -qmax), qmax).astype(np.int8)
+
+
 MUTANTS = {
+    "product_rounded_to_binary32_first": ("quantize_with_scale", _quantize_double_rounding),
     "fwht_sign_flipped": ("fwht128_blocks", _fwht_with(lambda a, b: (a + b, b - a))),
     "fwht_stage_dropped": ("fwht128_blocks", _fwht_with(lambda a, b: (a + b, a - b), (1, 2, 4, 8, 16, 32))),
     "fwht_halves_swapped": ("fwht128_blocks", _fwht_with(lambda a, b: (a - b, a + b))),

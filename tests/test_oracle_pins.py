@@ -109,8 +109,8 @@ def pin_quant_error_bound(o=O):
             deq = q.astype(np.float64) * s64
             unclipped = np.abs(u) <= qmax * s64
             err = np.abs(u - deq)
-            # r = fl(u * fl(qmax / t)) carries 3 roundings relative to u / s, each
-            # at most 2^-24 relative, and |u / s| <= qmax / alpha (plus rounding).
+            # r = u * fl(qmax / t) (exact product) carries 2 roundings relative to
+            # u / s, each at most 2^-24 relative, and |u / s| <= qmax / alpha.
             bound = s64 / 2 + s64 * (qmax / alpha + 1) * 2.0 ** -22
             assert np.all(err[unclipped] <= np.broadcast_to(bound, err.shape)[unclipped]), (bits, alpha)
             clipped = ~unclipped
@@ -131,6 +131,32 @@ def pin_rne_ties(o=O):
     q, s = o.quantize_rows(_bf16(x), 4, 1.0, rotate=False)
     assert s.tolist() == [1.0, 0.5]
     assert np.array_equal(q.astype(np.int64), want)
+
+
+def pin_exact_product_rounding(o=O):
+    """The code rounds the exact product u*inv once.  Hand-picked values where
+    fl(u*inv) lands on a .5 tie but the exact product does not (no rotation,
+    alpha = 1, qmax = 127, so inv = fl(127 / 165))."""
+    inv = np.float32(127.0) / np.float32(165.0)
+    hits = []
+    for k in range(1, 2000):
+        u = np.float32(k) * np.float32(0.125)
+        if u > 165:
+            break
+        if O.bf16_bits_to_f32(_bf16([u]))[0] != u:
+            continue  # only values the bf16 input can hold exactly
+        r32 = u * inv
+        exact = float(u) * float(inv)
+        if r32 == np.floor(r32) + np.float32(0.5) and exact != float(r32):
+            hits.append((u, exact))
+    assert hits, "the search must find double-rounding cases"
+    x = np.zeros((1, 128), np.float32)
+    x[0, 0] = 165.0
+    for i, (u, _) in enumerate(hits[:100]):
+        x[0, 1 + i] = u
+    q, _ = o.quant_act(_bf16(x), 8, 1.0, rotate=False)
+    for i, (u, exact) in enumerate(hits[:100]):
+        assert q[0, 1 + i] == int(np.rint(exact)), (u, exact)
 
 
 def pin_absmax_maps_to_qmax(o=O):
@@ -273,7 +299,7 @@ def pin_scalar_loop_tiny(o=O):
         inv = _fp32(qmax / tt)
         qs = []
         for t in v:
-            r = _fp32(t * inv)
+            r = t * inv  # binary64 product of two binary32 values: exact
             qi = round(r)  # Python round is half-to-even
             qs.append(max(-qmax, min(qmax, qi)))
         return qs, _fp32(s * fold)
