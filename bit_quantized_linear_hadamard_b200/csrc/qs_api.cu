@@ -19,6 +19,7 @@
 namespace {
 
 constexpr unsigned kKnownFlags = QS_FLAG_NO_ROTATE;
+constexpr float kMinAlpha = 1.0f / 16384.0f;  // keeps |u * inv| < 2^22
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -148,7 +149,7 @@ qs_status qs_quant_act(const void* x_bf16, int64_t M, int64_t K, int bits, float
   if (!x_bf16 || !x_packed || !x_scale) return QS_ERR_NULL;
   QS_TRY(check_bits(bits));
   QS_TRY(check_rows_k(M, K));
-  if (!(alpha > 0.0f && alpha <= 1.0f)) return QS_ERR_RANGE;
+  if (!(alpha >= kMinAlpha && alpha <= 1.0f)) return QS_ERR_RANGE;
   if (flags & ~kKnownFlags) return QS_ERR_RANGE;
   if (!aligned16(x_bf16) || !aligned16(x_packed) || !aligned16(x_scale)) return QS_ERR_ALIGN;
   QS_TRY(check_device_ptr(x_bf16));
@@ -205,7 +206,7 @@ qs_status qs_linear(const void* x_bf16, int64_t M, int64_t K, float alpha, const
                     void* workspace, int64_t workspace_bytes, void* out_bf16, void* stream) {
   if (!x_bf16 || !w_packed || !w_scale || !workspace || !out_bf16) return QS_ERR_NULL;
   QS_TRY(check_gemm_args(workspace, w_packed, out_bf16, M, N, K, bits));
-  if (!(alpha > 0.0f && alpha <= 1.0f)) return QS_ERR_RANGE;
+  if (!(alpha >= kMinAlpha && alpha <= 1.0f)) return QS_ERR_RANGE;
   const int64_t need = qs_linear_workspace_bytes(M, K, bits);
   if (need < 0) return QS_ERR_SHAPE;
   if (workspace_bytes < need) return QS_ERR_RANGE;

@@ -9,8 +9,8 @@
 //
 // Per row: u = block Walsh-Hadamard transform of the bf16 row (binary32
 // butterfly, stages h = 1, 2, 4, ..., 64 in that order), t = fl(alpha*amax),
-// s = fl(t/qmax) (stored), inv = fl(qmax/t), q = clamp(rint(fl(u*inv))) with
-// rows of t < 2^-120 treated as zero rows.
+// s = fl(t/qmax) (stored), inv = fl(qmax/t), q = clamp(rint(u*inv)) with the
+// product exact and rounded once, and rows of t < 2^-120 treated as zero rows.
 //
 // Two kernels compute exactly that:
 //  * rotate_quant_tma_kernel (K <= 16384): half a 128-element Hadamard block
@@ -19,10 +19,12 @@
 //    shared-memory ring by TMA; the row absmax is reduced through shared memory.
 //  * rotate_quant_group_kernel (longer rows): 8 elements per thread, stages
 //    h = 1, 2, 4 in registers and h = 8..64 by xor-shuffles, one row per CTA.
-// Rounding to the nearest integer, ties to even, is done by adding 1.5*2^23:
-// for |r| < 2^22 the sum is exactly representable only at integers, so the IEEE
-// round-to-nearest-even addition performs the rounding and the integer lands in
-// the low mantissa bits (two's complement in the low byte).
+// Rounding to the nearest integer, ties to even, is one fused multiply-add
+// fl(u*inv + 1.5*2^23): for |u*inv| < 2^22 (alpha >= 2^-14) the sum lies in
+// [2^23, 2^24), where binary32 holds exactly the integers, so the single
+// round-to-nearest-even of the exact u*inv + 1.5*2^23 is 1.5*2^23 +
+// rint_half_even(u*inv) (1.5*2^23 is even), and the integer lands in the low
+// mantissa bits (two's complement in the low 16 bits).
 #pragma once
 
 #include "qs_host.cuh"
@@ -74,14 +76,13 @@ __device__ __forceinline__ void row_factors(float amax, float alpha, float& s, f
   }
 }
 
-// Bits of fl(clamp(fl(u*inv)) + 1.5*2^23): the low byte is the two's complement
-// code rint_half_even(clamp(fl(u*inv))) (clamping to integer bounds commutes
-// with rounding, so this equals clamp(rint(fl(u*inv)))).
+// Bits of clamp(fl(u*inv + 1.5*2^23), 1.5*2^23 -+ qmax): the low byte is the
+// two's complement code clamp(rint_half_even(u*inv), -qmax, qmax).
 template <int QMAX>
 __device__ __forceinline__ uint32_t code_bits(float u, float inv) {
-  float r = __fmul_rn(u, inv);
-  r = fminf(fmaxf(r, -static_cast<float>(QMAX)), static_cast<float>(QMAX));
-  return __float_as_uint(__fadd_rn(r, kRoundMagic));
+  const float f = __fmaf_rn(u, inv, kRoundMagic);
+  return __float_as_uint(fminf(fmaxf(f, kRoundMagic - static_cast<float>(QMAX)),
+                               kRoundMagic + static_cast<float>(QMAX)));
 }
 
 // 8 codes (low byte/nibble of c[0..7]) -> packed bytes.
@@ -95,6 +96,34 @@ __device__ __forceinline__ uint32_t pack8_int4(const uint32_t (&c)[8]) {
 __device__ __forceinline__ uint32_t pack4_int8(uint32_t c0, uint32_t c1, uint32_t c2,
                                                uint32_t c3) {
   return __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
+}
+
+// Clamping and packing of 8 codes on packed 16-bit lanes.  Input: bits of
+// fl(u*inv + 1.5*2^23) without a clamp; their low 16 bits are the unclamped
+// code q as int16 whenever |q| < 2^15, which holds for alpha >= 1/256
+// (|q| <= qmax/alpha + 1 <= 32513).
+__device__ __forceinline__ uint32_t s16x2_clamp(uint32_t w, uint32_t hi, uint32_t lo) {
+  uint32_t r;
+  asm("min.s16x2 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(hi));
+  asm("max.s16x2 %0, %1, %2;" : "=r"(r) : "r"(r), "r"(lo));
+  return r;
+}
+
+// Clamped codes c[4h..4h+3] as 4 int8 bytes (h = 0 or 1).
+template <int QMAX>
+__device__ __forceinline__ uint32_t simd_bytes4(const uint32_t (&c)[8], int h) {
+  constexpr uint32_t hi = (static_cast<uint32_t>(QMAX) << 16) | static_cast<uint32_t>(QMAX);
+  constexpr uint32_t lo = ((0x10000u - QMAX) << 16) | (0x10000u - QMAX);
+  const uint32_t w01 = s16x2_clamp(__byte_perm(c[4 * h], c[4 * h + 1], 0x5410), hi, lo);
+  const uint32_t w23 = s16x2_clamp(__byte_perm(c[4 * h + 2], c[4 * h + 3], 0x5410), hi, lo);
+  return __byte_perm(w01, w23, 0x6420);
+}
+
+// Clamped codes c[0..7] as 8 int4 nibbles (element 2j in the low nibble of byte j).
+__device__ __forceinline__ uint32_t simd_nibbles8(const uint32_t (&c)[8]) {
+  const uint32_t n0 = simd_bytes4<7>(c, 0) & 0x0F0F0F0Fu;
+  const uint32_t n1 = simd_bytes4<7>(c, 1) & 0x0F0F0F0Fu;
+  return __byte_perm(n0 | (n0 >> 4), n1 | (n1 >> 4), 0x6420);  // bytes 0, 2 of each
 }
 
 // --------------------------------------------------------------------------
@@ -125,7 +154,7 @@ __device__ __forceinline__ uint32_t pack4_int8(uint32_t c0, uint32_t c1, uint32_
 // stage, which thread 0 then refills.
 // --------------------------------------------------------------------------
 
-template <int BITS>
+template <int BITS, bool SIMD_CLAMP>
 __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
     const __grid_constant__ CUtensorMap tmx, int64_t rows, int K, int nblk, int rpc,
     int64_t num_groups, int stages, float alpha, float scale_mul, int rotate,
@@ -257,7 +286,7 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
 
     const float2 inv2 = make_float2(inv, inv);
     const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
-    constexpr float kQ = static_cast<float>(kQmax);
+    [[maybe_unused]] constexpr float kQ = static_cast<float>(kQmax);
     // Codes of 8 consecutive pairs = elements 8k..8k+7 (low halves) and
     // 32+8k..32+8k+7 (high halves) of this half block.
     uint32_t wlo[BITS == 4 ? 4 : 8], whi[BITS == 4 ? 4 : 8];
@@ -266,14 +295,25 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
       uint32_t clo[8], chi[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        float2 r = __fmul2_rn(p[8 * k + e], inv2);
-        r.x = fminf(fmaxf(r.x, -kQ), kQ);
-        r.y = fminf(fmaxf(r.y, -kQ), kQ);
-        const float2 cb = __fadd2_rn(r, magic2);
+        float2 cb = __ffma2_rn(p[8 * k + e], inv2, magic2);  // magic + rint(u * inv)
+        if (!SIMD_CLAMP) {
+          cb.x = fminf(fmaxf(cb.x, kRoundMagic - kQ), kRoundMagic + kQ);
+          cb.y = fminf(fmaxf(cb.y, kRoundMagic - kQ), kRoundMagic + kQ);
+        }
         clo[e] = __float_as_uint(cb.x);
         chi[e] = __float_as_uint(cb.y);
       }
-      if (BITS == 4) {
+      if (SIMD_CLAMP) {
+        if (BITS == 4) {
+          wlo[k] = simd_nibbles8(clo);
+          whi[k] = simd_nibbles8(chi);
+        } else {
+          wlo[2 * k] = simd_bytes4<kQmax>(clo, 0);
+          wlo[2 * k + 1] = simd_bytes4<kQmax>(clo, 1);
+          whi[2 * k] = simd_bytes4<kQmax>(chi, 0);
+          whi[2 * k + 1] = simd_bytes4<kQmax>(chi, 1);
+        }
+      } else if (BITS == 4) {
         wlo[k] = pack8_int4(clo);
         whi[k] = pack8_int4(chi);
       } else {
@@ -450,7 +490,9 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
     if (!make_tensor_map_2d(&tmx, x, 64, static_cast<uint64_t>(rows) * K / 64, 64, rpc * K / 64,
                             true, 2))
       return cudaErrorInvalidValue;
-    auto kern = rotate_quant_tma_kernel<BITS>;
+    // codes clamp on packed int16 lanes when the unclamped code fits int16
+    auto kern = alpha >= 1.0f / 256.0f ? rotate_quant_tma_kernel<BITS, true>
+                                       : rotate_quant_tma_kernel<BITS, false>;
     cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;

@@ -15,8 +15,10 @@
  *     (both together are the exact factor 2^-7);
  *   - activations: one scale per token (row) over all of K, clip ratio alpha;
  *     weights: one scale per output channel (row of W), alpha = 1;
- *   - s = fl(fl(alpha * amax) / qmax), qmax = 7 (4 bits) or 127 (8 bits);
- *     q = clamp(round_half_even(fl(u / s)), -qmax, qmax); amax == 0 -> s = 0, q = 0;
+ *   - t = fl(alpha * amax); stored scale s = fl(t / qmax); multiplier
+ *     inv = fl(qmax / t); qmax = 7 (4 bits) or 127 (8 bits);
+ *     q = clamp(round_half_even(u * inv), -qmax, qmax), the product exact and
+ *     rounded once; rows with t < 2^-120 (amax == 0 included): s = 0, q = 0;
  *   - out = bf16_rne(fl(fl(fl(s_a[m] * s_w[n]) * float(acc[m][n])) + bias[n])),
  *     acc = sum_k q_a[m][k] * q_w[n][k] exact in int32.
  *
@@ -57,7 +59,7 @@ typedef enum {
   QS_ERR_SHAPE = 2,    /* M, N or K <= 0, K % 128 != 0, or N % 16 != 0 */
   QS_ERR_BITS = 3,     /* bits not 4 or 8 */
   QS_ERR_ALIGN = 4,    /* a pointer is not 16-byte aligned */
-  QS_ERR_RANGE = 5,    /* alpha outside (0, 1], unknown flag bits, or a size above its limit */
+  QS_ERR_RANGE = 5,    /* alpha outside [2^-14, 1], unknown flag bits, or a size above its limit */
   QS_ERR_CUDA = 6,     /* a CUDA runtime/driver call or a launch failed */
   QS_ERR_TIMEOUT = 7,  /* a kernel wait exceeded its bound (reported by qs_device_error) */
   QS_ERR_PTR = 8       /* a pointer is not device memory of the current device */
@@ -95,7 +97,7 @@ QS_API qs_status qs_pack_weights(const void* w_bf16, int64_t N, int64_t K, int b
  * 128-point block Walsh-Hadamard transform along K, absmax, scale with clip
  * ratio alpha, round-half-even, pack.
  *   x_bf16   [M, K] bf16, row-major
- *   alpha    clip ratio in (0, 1]
+ *   alpha    clip ratio in [2^-14, 1]
  *   flags    0 or QS_FLAG_NO_ROTATE
  *   x_packed [M, K*bits/8] bytes, written
  *   x_scale  [M] float, written (the per-token scale s_a)
@@ -139,7 +141,7 @@ QS_API int64_t qs_linear_workspace_bytes(int64_t M, int64_t K, int bits);
  * activations at run time, then the low-bit product).  Results are identical
  * to calling the two entry points in sequence.
  *   x_bf16             [M, K] bf16
- *   alpha              clip ratio in (0, 1]
+ *   alpha              clip ratio in [2^-14, 1]
  *   w_packed, w_scale  from qs_pack_weights (same K and bits)
  *   bias_bf16          [N] bf16 or NULL
  *   workspace          device scratch of at least qs_linear_workspace_bytes(M, K, bits)

@@ -73,7 +73,7 @@ def test_quant_act_validation(lib):
     assert f(NUL, 8, 128, 4, 1.0, 0, B, C, NUL) == NULL
     assert f(A, 8, 128, 3, 1.0, 0, B, C, NUL) == BITS
     assert f(A, 8, 130, 4, 1.0, 0, B, C, NUL) == SHAPE
-    for alpha in (0.0, -0.5, 1.5, float("nan"), float("inf")):
+    for alpha in (0.0, -0.5, 1.5, 2.0 ** -15, float("nan"), float("inf")):
         assert f(A, 8, 128, 4, alpha, 0, B, C, NUL) == RANGE, alpha
     assert f(A, 8, 128, 8, 1.0, 0x10, B, C, NUL) == RANGE
     assert f(A, 8, 128, 8, 1.0, 0, MIS, C, NUL) == ALIGN

@@ -103,6 +103,17 @@ def test_quant_ties_without_rotation():
     assert np.array_equal(O.unpack(xp, 4), want)
 
 
+def test_quant_rounds_the_exact_product():
+    # rows where fl(u*inv) is a .5 tie but the exact u*inv is not (see the oracle
+    # pin): the kernel's single rounding must follow the exact product
+    from test_oracle_pins import double_rounding_rows
+    rows = double_rounding_rows()
+    x = torch.zeros(len(rows), 128)
+    for i, (A, v, _) in enumerate(rows):
+        x[i, 0], x[i, 1] = float(A), float(v)
+    check_quant(x.to(torch.bfloat16), 8, 1.0, qs.QS_FLAG_NO_ROTATE)
+
+
 def test_quant_zero_tiny_and_constant_rows():
     x = torch.zeros(6, 512)
     x[1] = 1e-38            # binary32 subnormal range after rotation
@@ -114,6 +125,15 @@ def test_quant_zero_tiny_and_constant_rows():
     for bits in (4, 8):
         for alpha in (1.0, 0.5, 1e-3):
             check_quant(xb, bits, alpha)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("alpha", [1.0 / 256, 1.0 / 256 * 0.999, 0.02])
+def test_quant_small_alpha_heavy_clipping(bits, alpha):
+    # most codes clip; 1/256 is the smallest alpha whose unclamped codes still
+    # fit 16 bits (qmax/alpha <= 32512), just below it the float clamp is used
+    d = I.make_shape(seed=77, M=40, K=1024, N=16, bits=bits, outlier_factor=100.0)
+    check_quant(d["x"], bits, alpha)
 
 
 @pytest.mark.parametrize("bits", [4, 8])

@@ -133,30 +133,31 @@ def pin_rne_ties(o=O):
     assert np.array_equal(q.astype(np.int64), want)
 
 
-def pin_exact_product_rounding(o=O):
-    """The code rounds the exact product u*inv once.  Hand-picked values where
-    fl(u*inv) lands on a .5 tie but the exact product does not (no rotation,
-    alpha = 1, qmax = 127, so inv = fl(127 / 165))."""
-    inv = np.float32(127.0) / np.float32(165.0)
-    hits = []
-    for k in range(1, 2000):
-        u = np.float32(k) * np.float32(0.125)
-        if u > 165:
-            break
-        if O.bf16_bits_to_f32(_bf16([u]))[0] != u:
-            continue  # only values the bf16 input can hold exactly
+def double_rounding_rows():
+    """Rows (bf16 values, no rotation, int8, alpha = 1) that each hold an amax A in
+    [128, 256) and one value u < A for which fl(u * inv) is a .5 tie while the
+    exact product u * inv = u * fl(127 / A) is not: the two roundings disagree."""
+    us = O.bf16_bits_to_f32(np.arange(0x3F80, 0x4380, dtype=np.uint16))
+    rows = []
+    for A in O.bf16_bits_to_f32(np.arange(0x4300, 0x4380, dtype=np.uint16)):
+        inv = np.float32(127.0) / np.float32(A)
+        u = us[us < A]
         r32 = u * inv
-        exact = float(u) * float(inv)
-        if r32 == np.floor(r32) + np.float32(0.5) and exact != float(r32):
-            hits.append((u, exact))
-    assert hits, "the search must find double-rounding cases"
-    x = np.zeros((1, 128), np.float32)
-    x[0, 0] = 165.0
-    for i, (u, _) in enumerate(hits[:100]):
-        x[0, 1 + i] = u
+        tie = (r32 == np.floor(r32) + np.float32(0.5)) & (u.astype(np.float64) * float(inv) != r32)
+        for v in u[tie]:
+            rows.append((A, v, int(np.rint(float(v) * float(inv)))))
+    return rows
+
+
+def pin_exact_product_rounding(o=O):
+    """The code rounds the exact product u*inv once (not fl(u*inv) then rint)."""
+    rows = double_rounding_rows()
+    assert len(rows) > 10, "the search must find double-rounding cases"
+    x = np.zeros((len(rows), 128), np.float32)
+    for i, (A, v, _) in enumerate(rows):
+        x[i, 0], x[i, 1] = A, v
     q, _ = o.quant_act(_bf16(x), 8, 1.0, rotate=False)
-    for i, (u, exact) in enumerate(hits[:100]):
-        assert q[0, 1 + i] == int(np.rint(exact)), (u, exact)
+    assert [int(t) for t in q[:, 1]] == [want for _, _, want in rows]
 
 
 def pin_absmax_maps_to_qmax(o=O):
