@@ -173,6 +173,21 @@ class OracleSample:
                 "tokens_per_s": rows / dt}
 
 
+def combine_ranks(times_ms, steps, ops_per_step, world, device="cpu"):
+    """Replicas: every rank ran the same single-GPU workload.  The job's time is
+    the max over ranks of each timing; the value counts all ranks' work."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(list(times_ms), dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    times = t.tolist()
+    ms_per_step = times[0] / steps
+    return {"times_ms": times, "ms_per_step": ms_per_step,
+            "value": ops_per_step * world / (ms_per_step * 1e-3) / 1e12}
+
+
 def time_layer(qs, torch, x, wp, ws, bias, bits, alpha, stream, steps=5, warmup=2):
     """Mean CUDA-event times (ms) of the activation kernel and the GEMM for one layer."""
     M, K = x.shape
@@ -365,13 +380,10 @@ def main():
     if qs.qs_device_error(stream) != 0:
         raise SystemExit("kernel wait timed out in the timed region")
 
-    t = torch.tensor([total_ms, quant_ms, gemm_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, quant_ms, gemm_ms = t.tolist()
-    ms_per_step = total_ms / args.steps
     ops_per_step = 2.0 * M * N * K
-    value = ops_per_step * world / (ms_per_step * 1e-3) / 1e12
+    comb = combine_ranks([total_ms, quant_ms, gemm_ms], args.steps, ops_per_step, world, dev)
+    total_ms, quant_ms, gemm_ms = comb["times_ms"]
+    ms_per_step, value = comb["ms_per_step"], comb["value"]
 
     # ---- end to end through the same C ABI calls, inputs and result in pinned host memory
     x_host = d["x"].pin_memory()
@@ -398,10 +410,8 @@ def main():
             e2e_step()
         e1.record(stream)
         stream.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms = combine_ranks([e0.elapsed_time(e1) / e2e_steps], 1, ops_per_step, world,
+                           dev)["times_ms"][0]
 
     extra = {}
     if world == 1 and not args.no_extras:
