@@ -40,7 +40,7 @@ The pages leave the details open; the readings taken here are:
   alpha >= 2^-14, so |u * inv| <= qmax / alpha < 2^22.
 * Pack: row-major, int8 as two's complement bytes; int4 as two's complement
   nibbles, element 2j in the low nibble and element 2j+1 in the high nibble of
-  byte j.
+  byte j; 6-bit codes (qmax 31, the pages' W4A6 activations) as int8 bytes.
 * Integer GEMM: acc[m, n] = sum_k qa[m, k] * qw[n, k], exact (int64 here,
   checked to fit int32).
 * Dequantising epilogue: out = bf16_rne(fl(fl(fl(s_a * s_w) * float(acc)) + bias)),
@@ -57,7 +57,10 @@ import math
 
 import numpy as np
 
-QMAX = {4: 7, 8: 127}
+QMAX = {4: 7, 6: 31, 8: 127}
+# bytes of storage per code: 4-bit codes are packed two per byte; 6- and 8-bit
+# codes take one byte each (6-bit codes ride in int8 containers).
+STORAGE_BITS = {4: 4, 6: 8, 8: 8}
 HADAMARD_BLOCK = 128
 # (1/sqrt(128))^2: exact power of two carried by the weight scale.
 WEIGHT_SCALE_FOLD = np.float32(2.0 ** -7)
@@ -132,7 +135,7 @@ def row_scales(u: np.ndarray, bits: int, alpha: float) -> tuple[np.ndarray, np.n
     s = fl(t / qmax) (dequantisation) and inv = fl(qmax / t) (quantisation).
     Zero rows (t < 2^-120) get s = 0 and inv = 0."""
     if bits not in QMAX:
-        raise ValueError("bits must be 4 or 8")
+        raise ValueError("bits must be 4, 6 or 8")
     qmax = np.float32(QMAX[bits])
     amax = np.max(np.abs(u), axis=1).astype(np.float32)
     t = (np.float32(alpha) * amax).astype(np.float32)
@@ -189,12 +192,12 @@ def pack_weights(w_bits, bits: int, rotate: bool = True):
 # ---------------------------------------------------------------------------
 
 def pack(q: np.ndarray, bits: int) -> np.ndarray:
-    """Pack int8 codes [R, K] to the byte layout [R, K*bits/8] (uint8)."""
+    """Pack int8 codes [R, K] to the byte layout [R, K*storage/8] (uint8)."""
     q = np.asarray(q, dtype=np.int8)
-    if bits == 8:
+    if bits in (6, 8):
         return q.view(np.uint8).copy()
     if bits != 4:
-        raise ValueError("bits must be 4 or 8")
+        raise ValueError("bits must be 4, 6 or 8")
     nib = q.astype(np.uint8) & np.uint8(0x0F)
     lo = nib[:, 0::2]
     hi = nib[:, 1::2]
@@ -204,10 +207,10 @@ def pack(q: np.ndarray, bits: int) -> np.ndarray:
 def unpack(p: np.ndarray, bits: int) -> np.ndarray:
     """Inverse of :func:`pack`: bytes [R, K*bits/8] -> int8 codes [R, K]."""
     p = np.asarray(p, dtype=np.uint8)
-    if bits == 8:
+    if bits in (6, 8):
         return p.view(np.int8).copy()
     if bits != 4:
-        raise ValueError("bits must be 4 or 8")
+        raise ValueError("bits must be 4, 6 or 8")
     lo = (p & np.uint8(0x0F)).astype(np.int16)
     hi = (p >> np.uint8(4)).astype(np.int16)
     lo = np.where(lo >= 8, lo - 16, lo)
@@ -260,6 +263,19 @@ def qlinear(x_bits, w_bits, bias_bits, bits: int, alpha: float,
     out = epilogue(acc, sa, sw, bias_bits)
     return {"qa": qa, "sa": sa, "qw": qw, "sw": sw,
             "xp": pack(qa, bits), "wp": pack(qw, bits), "acc": acc, "out": out}
+
+
+def qlinear_mixed(x_bits, w_bits, bias_bits, bits_x: int, bits_w: int, alpha: float,
+                  rotate: bool = True):
+    """The layer with different code widths for activations and weights
+    (QuantSparse's W4A8, DVD-Quant's W4A6): each side is quantised at its own
+    width, the integer product and the epilogue are unchanged."""
+    qa, sa = quant_act(x_bits, bits_x, alpha, rotate)
+    qw, sw = pack_weights(w_bits, bits_w, rotate)
+    acc = int_gemm(qa, qw)
+    out = epilogue(acc, sa, sw, bias_bits)
+    return {"qa": qa, "sa": sa, "qw": qw, "sw": sw,
+            "xp": pack(qa, bits_x), "wp": pack(qw, bits_w), "acc": acc, "out": out}
 
 
 def gemm_rows(qa_rows: np.ndarray, qw: np.ndarray) -> np.ndarray:

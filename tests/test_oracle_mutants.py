@@ -106,6 +106,12 @@ def _quantize_double_rounding(u, inv, bits):
     return np.minimum(np.maximum(np.rint(r), -qmax), qmax).astype(np.int8)
 
 
+def _pack_six_as_nibbles(q, bits):
+    return _REAL_PACK(q, 4 if bits == 6 else bits)
+
+
+_REAL_PACK = O.pack
+
 MUTANTS = {
     "product_rounded_to_binary32_first": ("quantize_with_scale", _quantize_double_rounding),
     "fwht_sign_flipped": ("fwht128_blocks", _fwht_with(lambda a, b: (a + b, b - a))),
@@ -124,6 +130,8 @@ MUTANTS = {
     "bias_dropped": ("epilogue", _epilogue_with(drop_bias=True)),
     "bf16_truncation": ("f32_to_bf16_bits", _bf16_truncate),
     "weight_scale_not_folded": ("pack_weights", _pack_weights_no_fold),
+    "six_bit_qmax_is_2^5": ("QMAX", {4: 7, 6: 32, 8: 127}),
+    "six_bit_codes_as_nibbles": ("pack", _pack_six_as_nibbles),
 }
 
 

@@ -100,7 +100,7 @@ def pin_rotation_invariance(o=O):
 def pin_quant_error_bound(o=O):
     rng = np.random.default_rng(14)
     x = _bf16(rng.standard_normal((32, 640)) * np.where(rng.random(640) < 0.01, 50.0, 1.0))
-    for bits in (4, 8):
+    for bits in (4, 6, 8):
         for alpha in (1.0, 0.9, 0.5):
             q, s = o.quant_act(x, bits, alpha)
             u = O.fwht128_blocks(O.bf16_bits_to_f32(x)).astype(np.float64)
@@ -164,7 +164,7 @@ def pin_absmax_maps_to_qmax(o=O):
     rng = np.random.default_rng(15)
     x = _bf16(rng.standard_normal((16, 256)))
     u = O.fwht128_blocks(O.bf16_bits_to_f32(x))
-    for bits in (4, 8):
+    for bits in (4, 6, 8):
         q, _ = o.quant_act(x, bits, 1.0)
         idx = np.abs(u).argmax(1)
         got = q[np.arange(16), idx].astype(np.int64)
@@ -213,6 +213,28 @@ def pin_pack_roundtrip(o=O):
 
 
 # --------------------------------------------------------------------------- integer GEMM
+
+def pin_mixed_widths(o=O):
+    """W4A8 / W4A6: the mixed layer equals quantising each side at its own width
+    (qmax 7, 31 or 127; 6-bit codes in int8 bytes) and the exact integer product."""
+    rng = np.random.default_rng(23)
+    x = _bf16(rng.standard_normal((6, 256)) * np.where(rng.random(256) < 0.02, 30.0, 1.0))
+    w = _bf16(rng.standard_normal((5, 256)) * 0.02)
+    for bx, bw in ((8, 4), (6, 4), (4, 8)):
+        r = o.qlinear_mixed(x, w, None, bx, bw, 0.9)
+        # symmetric b-bit grid: qmax = 2^(b-1) - 1; clipping (alpha < 1) saturates
+        # every activation row and each weight row's absmax lands on qmax
+        qmax = {4: 7, 6: 31, 8: 127}
+        assert (np.abs(r["qa"]).max(axis=1) == qmax[bx]).all()
+        assert (np.abs(r["qw"]).max(axis=1) == qmax[bw]).all()
+        assert r["xp"].shape[1] == (128 if bx == 4 else 256)
+        assert r["wp"].shape[1] == (128 if bw == 4 else 256)
+        brute = [[sum(int(r["qa"][m, k]) * int(r["qw"][n, k]) for k in range(256))
+                  for n in range(5)] for m in range(6)]
+        assert r["acc"].tolist() == brute
+    q6 = np.array([[-31, -1, 0, 1, 31]], np.int8)
+    assert o.pack(q6, 6).tolist() == [[0xE1, 0xFF, 0, 1, 0x1F]]
+
 
 def pin_int_gemm_bruteforce(o=O):
     rng = np.random.default_rng(18)
