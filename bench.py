@@ -188,23 +188,25 @@ def combine_ranks(times_ms, steps, ops_per_step, world, device="cpu"):
             "value": ops_per_step * world / (ms_per_step * 1e-3) / 1e12}
 
 
-def time_layer(qs, torch, x, wp, ws, bias, bits, alpha, stream, steps=5, warmup=2):
-    """Mean CUDA-event times (ms) of the activation kernel and the GEMM for one layer."""
+def time_layer(qs, torch, x, wp, ws, bias, bits, alpha, stream, steps=5, warmup=2, bits_x=None):
+    """Mean CUDA-event times (ms) of the activation kernel and the GEMM for one
+    layer; ``bits`` is the weights' code width, ``bits_x`` the activations'."""
+    bx = bits if bits_x is None else bits_x
     M, K = x.shape
     N = wp.shape[0]
     dev = x.device
-    xp = torch.empty((M, K * bits // 8), dtype=torch.uint8, device=dev)
+    xp = torch.empty((M, qs.packed_cols(K, bx)), dtype=torch.uint8, device=dev)
     xs = torch.empty((M,), dtype=torch.float32, device=dev)
     out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     for _ in range(warmup):
-        qs.qs_quant_act(x, M, K, bits, alpha, 0, xp, xs, stream)
-        qs.qs_qlinear(xp, xs, wp, ws, bias, M, N, K, bits, out, stream)
+        qs.qs_quant_act(x, M, K, bx, alpha, 0, xp, xs, stream)
+        qs.qs_qlinear_mixed(xp, xs, bx, wp, ws, bits, bias, M, N, K, out, stream)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     for e in ev:
         e[0].record(stream)
-        qs.qs_quant_act(x, M, K, bits, alpha, 0, xp, xs, stream)
+        qs.qs_quant_act(x, M, K, bx, alpha, 0, xp, xs, stream)
         e[1].record(stream)
-        qs.qs_qlinear(xp, xs, wp, ws, bias, M, N, K, bits, out, stream)
+        qs.qs_qlinear_mixed(xp, xs, bx, wp, ws, bits, bias, M, N, K, out, stream)
         e[2].record(stream)
     stream.synchronize()
     q = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
@@ -215,13 +217,14 @@ def time_layer(qs, torch, x, wp, ws, bias, bits, alpha, stream, steps=5, warmup=
 def all_configs(qs, torch, I, dev, stream):
     """Per-configuration throughput on one GPU (every seeded synthetic shape)."""
     res = {}
-    for cfg in I.LAYER_CONFIGS:
+    for cfg in (*I.LAYER_CONFIGS, *I.MIXED_CONFIGS):
         d = I.make_layer(cfg)
         with torch.cuda.stream(stream):
             x, w, b = d["x"].to(dev), d["w"].to(dev), d["bias"].to(dev)
             wp, ws = qs.pack_weights(w, cfg.bits, stream=stream)
-        q, g, _ = time_layer(qs, torch, x, wp, ws, b, cfg.bits, cfg.alpha, stream)
-        res[cfg.name] = {"bits": cfg.bits, "quant_ms": q, "gemm_ms": g,
+        q, g, _ = time_layer(qs, torch, x, wp, ws, b, cfg.bits, cfg.alpha, stream,
+                             bits_x=cfg.act_bits)
+        res[cfg.name] = {"bits_w": cfg.bits, "bits_x": cfg.act_bits, "quant_ms": q, "gemm_ms": g,
                          "TOPS": cfg.ops / ((q + g) * 1e-3) / 1e12,
                          "gemm_TOPS": cfg.ops / (g * 1e-3) / 1e12,
                          "tokens_per_s": cfg.M / ((q + g) * 1e-3)}

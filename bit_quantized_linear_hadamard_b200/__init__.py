@@ -1,12 +1,13 @@
-"""Hadamard-rotated W4A4 / W8A8 quantized linear layer for NVIDIA B200 (sm_100a).
+"""Hadamard-rotated quantized linear layer (W4A4, W8A8, and the mixed W4A8 /
+W4A6) for NVIDIA B200 (sm_100a).
 
 The computation runs in libqs.so (CUDA kernels behind a C ABI, see include/qs.h);
 this package holds its build script, a ctypes binding and the seeded synthetic
 inputs used by the tests and the benchmark.
 """
 from .binding import (  # noqa: F401
-    EXPORTS, QS_FLAG_NO_ROTATE, QS_MAX_K, QSError, QuantLinear, gelu, linear, load, pack_weights,
-    qgemm_s32, qlinear, qs_device_error, qs_gelu_bf16, qs_linear, qs_linear_workspace_bytes,
-    qs_pack_weights, qs_qgemm_s32, qs_qlinear, qs_quant_act, qs_selftest_timeout, qs_version,
-    quant_act,
+    BITS, EXPORTS, QS_FLAG_NO_ROTATE, QS_MAX_K, QSError, QuantLinear, gelu, linear, load,
+    pack_weights, packed_cols, qgemm_s32, qlinear, qs_device_error, qs_gelu_bf16, qs_linear,
+    qs_linear_mixed, qs_linear_workspace_bytes, qs_pack_weights, qs_qgemm_s32, qs_qgemm_s32_mixed,
+    qs_qlinear, qs_qlinear_mixed, qs_quant_act, qs_selftest_timeout, qs_version, quant_act,
 )

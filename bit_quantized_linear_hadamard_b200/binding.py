@@ -1,7 +1,8 @@
 """ctypes binding of libqs.so.
 
 The functions named like the C entry points (``qs_pack_weights``,
-``qs_quant_act``, ``qs_qlinear``, ``qs_qgemm_s32``, ``qs_gelu_bf16``) take torch
+``qs_quant_act``, ``qs_qlinear``, ``qs_qlinear_mixed``, ``qs_qgemm_s32``,
+``qs_gelu_bf16``, ...) take torch
 CUDA tensors and only marshal their pointers, sizes and the stream into the C
 call; every step of the computation runs in the library's kernels.  The
 lower-case helpers (``pack_weights``, ``quant_act``, ``qlinear``, ...) allocate
@@ -25,9 +26,11 @@ QS_FLAG_NO_ROTATE = 1
 QS_MAX_K = 65536
 STATUS = {0: "QS_OK", 1: "QS_ERR_NULL", 2: "QS_ERR_SHAPE", 3: "QS_ERR_BITS", 4: "QS_ERR_ALIGN",
           5: "QS_ERR_RANGE", 6: "QS_ERR_CUDA", 7: "QS_ERR_TIMEOUT", 8: "QS_ERR_PTR"}
-EXPORTS = ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qgemm_s32", "qs_gelu_bf16",
-           "qs_linear_workspace_bytes", "qs_linear", "qs_linear_noalloc", "qs_selftest_timeout",
-           "qs_device_error", "qs_status_str", "qs_version")
+EXPORTS = ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qlinear_mixed", "qs_qgemm_s32",
+           "qs_qgemm_s32_mixed", "qs_gelu_bf16", "qs_linear_workspace_bytes", "qs_linear",
+           "qs_linear_mixed", "qs_linear_noalloc", "qs_selftest_timeout", "qs_device_error",
+           "qs_status_str", "qs_version")
+BITS = (4, 6, 8)
 QS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -53,20 +56,23 @@ def load() -> ctypes.CDLL:
     L.qs_pack_weights.argtypes = [vp, i64, i64, i32, u32, vp, vp, vp]
     L.qs_quant_act.argtypes = [vp, i64, i64, i32, f32, u32, vp, vp, vp]
     L.qs_qlinear.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp, vp]
+    L.qs_qlinear_mixed.argtypes = [vp, vp, i32, vp, vp, i32, vp, i64, i64, i64, vp, vp]
     L.qs_qgemm_s32.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp]
+    L.qs_qgemm_s32_mixed.argtypes = [vp, i32, vp, i32, i64, i64, i64, vp, vp]
     L.qs_gelu_bf16.argtypes = [vp, i64, vp, vp]
     L.qs_linear_workspace_bytes.argtypes = [i64, i64, i32]
     L.qs_linear_workspace_bytes.restype = i64
     L.qs_linear.argtypes = [vp, i64, i64, f32, vp, vp, vp, i64, i32, vp, i64, vp, vp]
+    L.qs_linear_mixed.argtypes = [vp, i64, i64, f32, i32, vp, vp, i32, vp, i64, vp, i64, vp, vp]
     L.qs_linear_noalloc.argtypes = [vp, i64, i64, f32, vp, vp, vp, i64, i32, vp, vp]
     L.qs_selftest_timeout.argtypes = [i64, vp]
     L.qs_device_error.argtypes = [vp]
     L.qs_status_str.argtypes = [i32]
     L.qs_status_str.restype = ctypes.c_char_p
     L.qs_version.restype = ctypes.c_char_p
-    for name in ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qgemm_s32",
-                 "qs_gelu_bf16", "qs_linear", "qs_linear_noalloc", "qs_selftest_timeout",
-                 "qs_device_error"):
+    for name in ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qlinear_mixed",
+                 "qs_qgemm_s32", "qs_qgemm_s32_mixed", "qs_gelu_bf16", "qs_linear",
+                 "qs_linear_mixed", "qs_linear_noalloc", "qs_selftest_timeout", "qs_device_error"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -134,6 +140,27 @@ def qs_qlinear(x_packed, x_scale, w_packed, w_scale, bias, M, N, K, bits, out, s
                              M, N, K, bits, _p(out), _s(stream)), "qs_qlinear")
 
 
+def qs_qlinear_mixed(x_packed, x_scale, bits_x, w_packed, w_scale, bits_w, bias, M, N, K, out,
+                     stream=None):
+    _cuda(x_packed, torch.uint8, "x_packed")
+    _cuda(w_packed, torch.uint8, "w_packed")
+    _cuda(x_scale, torch.float32, "x_scale")
+    _cuda(w_scale, torch.float32, "w_scale")
+    _cuda(bias, torch.bfloat16, "bias")
+    _cuda(out, torch.bfloat16, "out")
+    _check(load().qs_qlinear_mixed(_p(x_packed), _p(x_scale), bits_x, _p(w_packed), _p(w_scale),
+                                   bits_w, _p(bias), M, N, K, _p(out), _s(stream)),
+           "qs_qlinear_mixed")
+
+
+def qs_qgemm_s32_mixed(x_packed, bits_x, w_packed, bits_w, M, N, K, acc, stream=None):
+    _cuda(x_packed, torch.uint8, "x_packed")
+    _cuda(w_packed, torch.uint8, "w_packed")
+    _cuda(acc, torch.int32, "acc")
+    _check(load().qs_qgemm_s32_mixed(_p(x_packed), bits_x, _p(w_packed), bits_w, M, N, K, _p(acc),
+                                     _s(stream)), "qs_qgemm_s32_mixed")
+
+
 def qs_qgemm_s32(x_packed, w_packed, M, N, K, bits, acc, stream=None):
     _cuda(x_packed, torch.uint8, "x_packed")
     _cuda(w_packed, torch.uint8, "w_packed")
@@ -164,6 +191,19 @@ def qs_linear(x, M, K, alpha, w_packed, w_scale, bias, N, bits, workspace, works
                             _p(workspace), workspace_bytes, _p(out), _s(stream)), "qs_linear")
 
 
+def qs_linear_mixed(x, M, K, alpha, bits_x, w_packed, w_scale, bits_w, bias, N, workspace,
+                    workspace_bytes, out, stream=None):
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(w_packed, torch.uint8, "w_packed")
+    _cuda(w_scale, torch.float32, "w_scale")
+    _cuda(bias, torch.bfloat16, "bias")
+    _cuda(workspace, torch.uint8, "workspace")
+    _cuda(out, torch.bfloat16, "out")
+    _check(load().qs_linear_mixed(_p(x), M, K, float(alpha), bits_x, _p(w_packed), _p(w_scale),
+                                  bits_w, _p(bias), N, _p(workspace), workspace_bytes, _p(out),
+                                  _s(stream)), "qs_linear_mixed")
+
+
 def qs_linear_noalloc(x, M, K, alpha, w_packed, w_scale, bias, N, bits, out, stream=None):
     """qs_linear on the library's own fixed scratch buffer (for callers that
     cannot allocate device memory when they run the layer); nothing is allocated."""
@@ -190,10 +230,15 @@ def qs_version() -> str:
 
 # --------------------------------------------------------------------------- helpers
 
+def packed_cols(K: int, bits: int) -> int:
+    """Bytes of one packed row of K codes: nibbles for 4 bits, bytes for 6 and 8."""
+    return K // 2 if bits == 4 else K
+
+
 def pack_weights(w: torch.Tensor, bits: int, flags: int = 0, stream=None):
-    """w bf16 [N, K] -> (w_packed uint8 [N, K*bits/8], w_scale float32 [N])."""
+    """w bf16 [N, K] -> (w_packed uint8 [N, packed_cols(K, bits)], w_scale float32 [N])."""
     N, K = w.shape
-    wp = torch.empty((N, K * bits // 8), dtype=torch.uint8, device=w.device)
+    wp = torch.empty((N, packed_cols(K, bits)), dtype=torch.uint8, device=w.device)
     ws = torch.empty((N,), dtype=torch.float32, device=w.device)
     qs_pack_weights(w, N, K, bits, flags, wp, ws, stream)
     return wp, ws
@@ -201,10 +246,10 @@ def pack_weights(w: torch.Tensor, bits: int, flags: int = 0, stream=None):
 
 def quant_act(x: torch.Tensor, bits: int, alpha: float = 1.0, flags: int = 0, stream=None,
               out=None):
-    """x bf16 [M, K] -> (x_packed uint8 [M, K*bits/8], x_scale float32 [M])."""
+    """x bf16 [M, K] -> (x_packed uint8 [M, packed_cols(K, bits)], x_scale float32 [M])."""
     M, K = x.shape
     if out is None:
-        xp = torch.empty((M, K * bits // 8), dtype=torch.uint8, device=x.device)
+        xp = torch.empty((M, packed_cols(K, bits)), dtype=torch.uint8, device=x.device)
         xs = torch.empty((M,), dtype=torch.float32, device=x.device)
     else:
         xp, xs = out
@@ -212,19 +257,27 @@ def quant_act(x: torch.Tensor, bits: int, alpha: float = 1.0, flags: int = 0, st
     return xp, xs
 
 
-def qlinear(x_packed, x_scale, w_packed, w_scale, bias, bits: int, K: int, stream=None, out=None):
-    """Packed activations and weights -> bf16 [M, N]."""
+def qlinear(x_packed, x_scale, w_packed, w_scale, bias, bits: int, K: int, stream=None, out=None,
+            bits_w: int | None = None):
+    """Packed activations (``bits``) and weights (``bits_w``, default ``bits``) -> bf16 [M, N]."""
     M, N = x_packed.shape[0], w_packed.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x_packed.device)
-    qs_qlinear(x_packed, x_scale, w_packed, w_scale, bias, M, N, K, bits, out, stream)
+    if bits_w is None or bits_w == bits:
+        qs_qlinear(x_packed, x_scale, w_packed, w_scale, bias, M, N, K, bits, out, stream)
+    else:
+        qs_qlinear_mixed(x_packed, x_scale, bits, w_packed, w_scale, bits_w, bias, M, N, K, out,
+                         stream)
     return out
 
 
-def qgemm_s32(x_packed, w_packed, bits: int, K: int, stream=None):
+def qgemm_s32(x_packed, w_packed, bits: int, K: int, stream=None, bits_w: int | None = None):
     M, N = x_packed.shape[0], w_packed.shape[0]
     acc = torch.empty((M, N), dtype=torch.int32, device=x_packed.device)
-    qs_qgemm_s32(x_packed, w_packed, M, N, K, bits, acc, stream)
+    if bits_w is None or bits_w == bits:
+        qs_qgemm_s32(x_packed, w_packed, M, N, K, bits, acc, stream)
+    else:
+        qs_qgemm_s32_mixed(x_packed, bits, w_packed, bits_w, M, N, K, acc, stream)
     return acc
 
 
@@ -235,8 +288,9 @@ def gelu(x: torch.Tensor, stream=None, out=None):
 
 
 def linear(x, w_packed, w_scale, bias, bits: int, alpha: float = 1.0, workspace=None,
-           stream=None, out=None):
-    """bf16 activations [M, K] -> bf16 [M, N] through qs_linear (one C call)."""
+           stream=None, out=None, bits_w: int | None = None):
+    """bf16 activations [M, K] -> bf16 [M, N] through qs_linear (one C call);
+    ``bits`` is the activation width, ``bits_w`` the weights' (default ``bits``)."""
     M, K = x.shape
     N = w_packed.shape[0]
     need = qs_linear_workspace_bytes(M, K, bits)
@@ -246,27 +300,34 @@ def linear(x, w_packed, w_scale, bias, bits: int, alpha: float = 1.0, workspace=
         workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    qs_linear(x, M, K, alpha, w_packed, w_scale, bias, N, bits, workspace, workspace.numel(), out,
-              stream)
+    if bits_w is None or bits_w == bits:
+        qs_linear(x, M, K, alpha, w_packed, w_scale, bias, N, bits, workspace, workspace.numel(),
+                  out, stream)
+    else:
+        qs_linear_mixed(x, M, K, alpha, bits, w_packed, w_scale, bits_w, bias, N, workspace,
+                        workspace.numel(), out, stream)
     return out
 
 
 class QuantLinear:
-    """A Hadamard-rotated W4A4 / W8A8 linear layer: weights packed once; each
-    call runs qs_linear (the activation kernel, then the GEMM) on a workspace
-    the layer keeps and grows as needed."""
+    """A Hadamard-rotated quantized linear layer (W4A4, W8A8, or mixed such as
+    W4A8 / W4A6 with ``bits_x``): weights packed once; each call runs the
+    one-call layer (the activation kernel, then the GEMM) on a workspace the
+    layer keeps and grows as needed."""
 
     def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None, bits: int,
-                 alpha: float = 1.0):
+                 alpha: float = 1.0, bits_x: int | None = None):
         self.N, self.K = weight.shape
-        self.bits, self.alpha = bits, alpha
+        self.bits = bits
+        self.bits_x = bits if bits_x is None else bits_x
+        self.alpha = alpha
         self.w_packed, self.w_scale = pack_weights(weight, bits)
         self.bias = bias
         self.workspace = None
 
     def __call__(self, x: torch.Tensor, stream=None, out=None) -> torch.Tensor:
-        need = qs_linear_workspace_bytes(x.shape[0], self.K, self.bits)
+        need = qs_linear_workspace_bytes(x.shape[0], self.K, self.bits_x)
         if self.workspace is None or self.workspace.numel() < need:
             self.workspace = torch.empty((max(need, 0),), dtype=torch.uint8, device=x.device)
-        return linear(x, self.w_packed, self.w_scale, self.bias, self.bits, self.alpha,
-                      self.workspace, stream=stream, out=out)
+        return linear(x, self.w_packed, self.w_scale, self.bias, self.bits_x, self.alpha,
+                      self.workspace, stream=stream, out=out, bits_w=self.bits)

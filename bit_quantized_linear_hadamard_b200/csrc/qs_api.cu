@@ -44,7 +44,12 @@ qs_status check_rows_k(int64_t rows, int64_t K) {
   return QS_OK;
 }
 
-qs_status check_bits(int bits) { return (bits == 4 || bits == 8) ? QS_OK : QS_ERR_BITS; }
+qs_status check_bits(int bits) {
+  return (bits == 4 || bits == 6 || bits == 8) ? QS_OK : QS_ERR_BITS;
+}
+
+// Bytes of one packed row of K codes.
+int64_t packed_row_bytes(int64_t K, int bits) { return K * qs::code_storage_bits(bits) / 8; }
 
 #define QS_TRY(expr)               \
   do {                             \
@@ -52,21 +57,21 @@ qs_status check_bits(int bits) { return (bits == 4 || bits == 8) ? QS_OK : QS_ER
     if (_s != QS_OK) return _s;    \
   } while (0)
 
-template <int BITS, bool OUT_S32>
+// SA, SB: storage bits (4 or 8) of the x and W codes.
+template <int SA, int SB, bool OUT_S32>
 qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, const float* sw,
                        const void* bias, int64_t M, int64_t N, int64_t K, void* out,
                        cudaStream_t stream) {
-  using C = qs::gemm::Cfg<BITS>;
-  const uint64_t row_bytes = static_cast<uint64_t>(K) * BITS / 8;
-  const uint32_t box_bytes = qs::gemm::BK * BITS / 8;
+  using C = qs::gemm::Cfg<SA, SB>;
   CUtensorMap ta, tb;
-  // each CTA of a pair loads 128 rows of x and 128 rows of W per stage
-  if (!qs::make_tensor_map_2d(&ta, xp, row_bytes, static_cast<uint64_t>(M), box_bytes, qs::gemm::HM,
-                       BITS == 8) ||
-      !qs::make_tensor_map_2d(&tb, wp, row_bytes, static_cast<uint64_t>(N), box_bytes, qs::gemm::HN,
-                       BITS == 8))
+  // each CTA of a pair loads 128 rows of x and 128 rows of W per stage; 8-bit
+  // tiles land 128-byte swizzled in the operand stage, 4-bit ones as plain rows
+  if (!qs::make_tensor_map_2d(&ta, xp, static_cast<uint64_t>(K) * SA / 8, static_cast<uint64_t>(M),
+                              qs::gemm::BK * SA / 8, qs::gemm::HM, SA == 8) ||
+      !qs::make_tensor_map_2d(&tb, wp, static_cast<uint64_t>(K) * SB / 8, static_cast<uint64_t>(N),
+                              qs::gemm::BK * SB / 8, qs::gemm::HN, SB == 8))
     return QS_ERR_CUDA;
-  auto kern = qs::gemm::qgemm_kernel<BITS, OUT_S32>;
+  auto kern = qs::gemm::qgemm_kernel<SA, SB, OUT_S32>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
       cudaSuccess)
     return QS_ERR_CUDA;
@@ -84,10 +89,25 @@ qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, const fl
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
+template <bool OUT_S32>
+qs_status dispatch_qgemm(int bits_x, int bits_w, const void* xp, const float* sa, const void* wp,
+                         const float* sw, const void* bias, int64_t M, int64_t N, int64_t K,
+                         void* out, cudaStream_t stream) {
+  const int sx = qs::code_storage_bits(bits_x), sww = qs::code_storage_bits(bits_w);
+  if (sx == 4 && sww == 4)
+    return launch_qgemm<4, 4, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
+  if (sx == 8 && sww == 8)
+    return launch_qgemm<8, 8, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
+  if (sx == 8 && sww == 4)
+    return launch_qgemm<8, 4, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
+  return launch_qgemm<4, 8, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
+}
+
 qs_status check_gemm_args(const void* xp, const void* wp, const void* out, int64_t M, int64_t N,
-                          int64_t K, int bits) {
+                          int64_t K, int bits_x, int bits_w) {
   if (!xp || !wp || !out) return QS_ERR_NULL;
-  QS_TRY(check_bits(bits));
+  QS_TRY(check_bits(bits_x));
+  QS_TRY(check_bits(bits_w));
   QS_TRY(check_rows_k(M, K));
   QS_TRY(check_rows_k(N, K));
   if (N % 16 != 0) return QS_ERR_SHAPE;
@@ -162,10 +182,11 @@ qs_status qs_quant_act(const void* x_bf16, int64_t M, int64_t K, int bits, float
   return e == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
-qs_status qs_qlinear(const void* x_packed, const float* x_scale, const void* w_packed,
-                     const float* w_scale, const void* bias_bf16, int64_t M, int64_t N,
-                     int64_t K, int bits, void* out_bf16, void* stream) {
-  QS_TRY(check_gemm_args(x_packed, w_packed, out_bf16, M, N, K, bits));
+qs_status qs_qlinear_mixed(const void* x_packed, const float* x_scale, int bits_x,
+                           const void* w_packed, const float* w_scale, int bits_w,
+                           const void* bias_bf16, int64_t M, int64_t N, int64_t K,
+                           void* out_bf16, void* stream) {
+  QS_TRY(check_gemm_args(x_packed, w_packed, out_bf16, M, N, K, bits_x, bits_w));
   if (!x_scale || !w_scale) return QS_ERR_NULL;
   if (!aligned16(x_scale) || !aligned16(w_scale) || (bias_bf16 && !aligned16(bias_bf16)))
     return QS_ERR_ALIGN;
@@ -175,39 +196,46 @@ qs_status qs_qlinear(const void* x_packed, const float* x_scale, const void* w_p
   QS_TRY(check_device_ptr(w_scale));
   QS_TRY(check_device_ptr(out_bf16));
   if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return bits == 4 ? launch_qgemm<4, false>(x_packed, x_scale, w_packed, w_scale, bias_bf16, M, N,
-                                             K, out_bf16, s)
-                   : launch_qgemm<8, false>(x_packed, x_scale, w_packed, w_scale, bias_bf16, M, N,
-                                             K, out_bf16, s);
+  return dispatch_qgemm<false>(bits_x, bits_w, x_packed, x_scale, w_packed, w_scale, bias_bf16, M,
+                               N, K, out_bf16, static_cast<cudaStream_t>(stream));
+}
+
+qs_status qs_qlinear(const void* x_packed, const float* x_scale, const void* w_packed,
+                     const float* w_scale, const void* bias_bf16, int64_t M, int64_t N,
+                     int64_t K, int bits, void* out_bf16, void* stream) {
+  return qs_qlinear_mixed(x_packed, x_scale, bits, w_packed, w_scale, bits, bias_bf16, M, N, K,
+                          out_bf16, stream);
+}
+
+qs_status qs_qgemm_s32_mixed(const void* x_packed, int bits_x, const void* w_packed, int bits_w,
+                             int64_t M, int64_t N, int64_t K, int32_t* acc, void* stream) {
+  QS_TRY(check_gemm_args(x_packed, w_packed, acc, M, N, K, bits_x, bits_w));
+  QS_TRY(check_device_ptr(x_packed));
+  QS_TRY(check_device_ptr(w_packed));
+  QS_TRY(check_device_ptr(acc));
+  return dispatch_qgemm<true>(bits_x, bits_w, x_packed, nullptr, w_packed, nullptr, nullptr, M, N,
+                              K, acc, static_cast<cudaStream_t>(stream));
 }
 
 qs_status qs_qgemm_s32(const void* x_packed, const void* w_packed, int64_t M, int64_t N,
                        int64_t K, int bits, int32_t* acc, void* stream) {
-  QS_TRY(check_gemm_args(x_packed, w_packed, acc, M, N, K, bits));
-  QS_TRY(check_device_ptr(x_packed));
-  QS_TRY(check_device_ptr(w_packed));
-  QS_TRY(check_device_ptr(acc));
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return bits == 4 ? launch_qgemm<4, true>(x_packed, nullptr, w_packed, nullptr, nullptr, M, N, K,
-                                            acc, s)
-                   : launch_qgemm<8, true>(x_packed, nullptr, w_packed, nullptr, nullptr, M, N, K,
-                                            acc, s);
+  return qs_qgemm_s32_mixed(x_packed, bits, w_packed, bits, M, N, K, acc, stream);
 }
 
 int64_t qs_linear_workspace_bytes(int64_t M, int64_t K, int bits) {
   if (check_bits(bits) != QS_OK || check_rows_k(M, K) != QS_OK) return -1;
-  const int64_t packed = (M * K * bits / 8 + 255) / 256 * 256;
+  const int64_t packed = (M * packed_row_bytes(K, bits) + 255) / 256 * 256;
   return packed + 4 * M;
 }
 
-qs_status qs_linear(const void* x_bf16, int64_t M, int64_t K, float alpha, const void* w_packed,
-                    const float* w_scale, const void* bias_bf16, int64_t N, int bits,
-                    void* workspace, int64_t workspace_bytes, void* out_bf16, void* stream) {
+qs_status qs_linear_mixed(const void* x_bf16, int64_t M, int64_t K, float alpha, int bits_x,
+                          const void* w_packed, const float* w_scale, int bits_w,
+                          const void* bias_bf16, int64_t N, void* workspace,
+                          int64_t workspace_bytes, void* out_bf16, void* stream) {
   if (!x_bf16 || !w_packed || !w_scale || !workspace || !out_bf16) return QS_ERR_NULL;
-  QS_TRY(check_gemm_args(workspace, w_packed, out_bf16, M, N, K, bits));
+  QS_TRY(check_gemm_args(workspace, w_packed, out_bf16, M, N, K, bits_x, bits_w));
   if (!(alpha >= kMinAlpha && alpha <= 1.0f)) return QS_ERR_RANGE;
-  const int64_t need = qs_linear_workspace_bytes(M, K, bits);
+  const int64_t need = qs_linear_workspace_bytes(M, K, bits_x);
   if (need < 0) return QS_ERR_SHAPE;
   if (workspace_bytes < need) return QS_ERR_RANGE;
   // everything both launches will check, before the first one
@@ -220,9 +248,17 @@ qs_status qs_linear(const void* x_bf16, int64_t M, int64_t K, float alpha, const
   QS_TRY(check_device_ptr(out_bf16));
   if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
   uint8_t* xp = static_cast<uint8_t*>(workspace);
-  float* xs = reinterpret_cast<float*>(xp + (M * K * bits / 8 + 255) / 256 * 256);
-  QS_TRY(qs_quant_act(x_bf16, M, K, bits, alpha, 0u, xp, xs, stream));
-  return qs_qlinear(xp, xs, w_packed, w_scale, bias_bf16, M, N, K, bits, out_bf16, stream);
+  float* xs = reinterpret_cast<float*>(xp + (M * packed_row_bytes(K, bits_x) + 255) / 256 * 256);
+  QS_TRY(qs_quant_act(x_bf16, M, K, bits_x, alpha, 0u, xp, xs, stream));
+  return qs_qlinear_mixed(xp, xs, bits_x, w_packed, w_scale, bits_w, bias_bf16, M, N, K, out_bf16,
+                          stream);
+}
+
+qs_status qs_linear(const void* x_bf16, int64_t M, int64_t K, float alpha, const void* w_packed,
+                    const float* w_scale, const void* bias_bf16, int64_t N, int bits,
+                    void* workspace, int64_t workspace_bytes, void* out_bf16, void* stream) {
+  return qs_linear_mixed(x_bf16, M, K, alpha, bits, w_packed, w_scale, bits, bias_bf16, N,
+                         workspace, workspace_bytes, out_bf16, stream);
 }
 
 qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream) {
@@ -281,7 +317,7 @@ const char* qs_status_str(int status) {
     case QS_OK: return "ok";
     case QS_ERR_NULL: return "a required pointer is NULL";
     case QS_ERR_SHAPE: return "bad shape (need M,N,K > 0, K % 128 == 0, N % 16 == 0)";
-    case QS_ERR_BITS: return "bits must be 4 or 8";
+    case QS_ERR_BITS: return "bits must be 4, 6 or 8";
     case QS_ERR_ALIGN: return "pointer not 16-byte aligned";
     case QS_ERR_RANGE: return "value out of range (alpha, flags or a size limit)";
     case QS_ERR_CUDA: return "CUDA call or launch failed";
@@ -291,6 +327,6 @@ const char* qs_status_str(int status) {
   }
 }
 
-const char* qs_version(void) { return "qs 0.1.0 sm_100a"; }
+const char* qs_version(void) { return "qs 0.2.0 sm_100a"; }
 
 }  // extern "C"

@@ -45,11 +45,21 @@
 // its byte.  That byte, read as int8, is 16*q exactly, so the tensor core
 // accumulates 256*acc; the epilogue shifts it back (exact).  Both operands get
 // the same K permutation, so every dot product is unchanged.  The widening is
-// one shift and one mask per 4 output bytes.  |16 q| <= 112 keeps 256*acc
-// inside int32 for K <= 65536.
+// one shift and one mask per 4 output bytes.  When only one operand is 4-bit
+// the other is in natural K order, so the widened bytes are interleaved back
+// into natural order (two byte permutes more per 8 output bytes).
+// |16 q| <= 112 keeps 256*acc inside int32 for K <= 65536.
 //
 // 8-bit operands go from global memory to the 128-byte-swizzled operand tiles
-// directly by TMA.
+// directly by TMA.  (6-bit codes are stored as int8 and take this path.)
+//
+// Mixed widths (W4A8 of QuantSparse, W4A6 of DVD-Quant, both "Resumen
+// técnico" §4; 8-bit storage for x, 4-bit for W): the 8-bit operand is loaded
+// by TMA straight into its half of the operand stage and the 4-bit one is
+// widened into the other half.  The leader's producer arms its "full" barrier
+// with the direct bytes of both CTAs plus the relay's 16 bytes; the MMA
+// additionally waits for its own CTA's widening.  Only the widened operand carries the factor 16, so the epilogue
+// shifts by 4 bits per 4-bit operand.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -66,19 +76,32 @@ constexpr int HN = 128;  // W rows per CTA
 constexpr int BK = 128;  // K elements per pipeline stage (= 128 bytes of 8-bit operand)
 constexpr int kTmemCols = 2 * BN;
 
-template <int BITS>
+// SA, SB: storage bits of the x and W codes (4 = two per byte, 8 = one byte).
+template <int SA, int SB>
 struct Cfg {
-  static constexpr bool kPacked = BITS == 4;
-  static constexpr int kPkBytesA = HM * BK / 2;  // packed 4-bit tile of x (this CTA)
-  static constexpr int kPkBytesB = HN * BK / 2;  // packed 4-bit tile of W (this CTA)
+  static_assert((SA == 4 || SA == 8) && (SB == 4 || SB == 8), "storage is 4 or 8 bits");
+  static constexpr bool kPackedA = SA == 4;
+  static constexpr bool kPackedB = SB == 4;
+  static constexpr bool kPacked = kPackedA || kPackedB;   // some operand is widened
+  static constexpr bool kAllPacked = kPackedA && kPackedB;
+  static constexpr bool kDirect = !kAllPacked;            // some operand goes by TMA directly
+  static constexpr int kPkBytesA = kPackedA ? HM * BK / 2 : 0;  // packed tile of x (this CTA)
+  static constexpr int kPkBytesB = kPackedB ? HN * BK / 2 : 0;  // packed tile of W (this CTA)
   static constexpr int kOpBytesA = HM * BK;      // 8-bit operand tile of x
   static constexpr int kOpBytesB = HN * BK;      // 8-bit operand tile of W
   static constexpr int kPkStage = kPkBytesA + kPkBytesB;
   static constexpr int kOpStage = kOpBytesA + kOpBytesB;
-  static constexpr int kPkStages = kPacked ? 4 : 0;
-  static constexpr int kOpStages = kPacked ? 4 : 6;
+  // bytes the TMA writes straight into one operand stage of this CTA
+  static constexpr int kDirectBytes = (kPackedA ? 0 : kOpBytesA) + (kPackedB ? 0 : kOpBytesB);
+  // 4/4 and 8/8 sized by measurement; mixed: as many stages as fit
+  static constexpr int kOpStages = kAllPacked ? 4 : (kPacked ? 5 : 6);
+  static constexpr int kPkStages = kPacked ? kOpStages : 0;  // one ring index drives both
   static constexpr int kEpiWarps = 4;
   static constexpr int kUnpackWarps = kPacked ? 4 : 0;
+  // operand-tile row that packed row 0 widens into (W rows follow the 128 x rows)
+  static constexpr int kUnpackRow0 = kPackedA ? 0 : HM;
+  // the tensor core sees 16 q for every widened operand
+  static constexpr int kAccShift = 4 * (static_cast<int>(kPackedA) + static_cast<int>(kPackedB));
   static constexpr int kThreads = 32 * (2 + kEpiWarps + kUnpackWarps);
   static constexpr int kOffOp = 0;
   static constexpr int kOffPk = kOffOp + kOpStages * kOpStage;
@@ -92,9 +115,11 @@ struct Cfg {
   static constexpr int kChunksPerThread = kPacked ? (kPkStage / 16) / kUnpackThreads : 0;
   static_assert((kPkStage / 16) % kUnpackThreads == 0, "unpack split");
   // arrivals completing one "operand full" phase on the leader: its MMA
-  // thread arming the relay's 16 bytes (4-bit) or its producer arming both
-  // CTAs' TMA bytes (8-bit)
+  // thread arming the relay's 16 bytes (both operands 4-bit) or its producer
+  // arming both CTAs' direct TMA bytes (+ the relay's 16 bytes when mixed)
   static constexpr int kOpFullCount = 1;
+  static constexpr int kOpFullTx = 2 * kDirectBytes + (kPacked ? 16 : 0);
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
   static constexpr int kAccEmptyCount = 2 * kEpiWarps;
 };
 
@@ -124,11 +149,11 @@ struct Problem {
   }
 };
 
-template <int BITS>
+template <int SA, int SB>
 __device__ __forceinline__ void producer_role(const Smem& sm, const Problem& pb,
                                               const CUtensorMap* tmA, const CUtensorMap* tmB,
                                               volatile int* abort_flag) {
-  using C = Cfg<BITS>;
+  using C = Cfg<SA, SB>;
   int s = 0;
   uint32_t ph = 0;
   const int roff = static_cast<int>(pb.rank) * HM;
@@ -141,19 +166,21 @@ __device__ __forceinline__ void producer_role(const Smem& sm, const Problem& pb,
         if (!mbar_wait_bounded(sm.pk_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer)) return;
         const uint32_t dst = sm.base + C::kOffPk + s * C::kPkStage;
         mbar_arrive_expect_tx(sm.pk_full(s), C::kPkStage);
-        tma_load_2d(dst, tmA, kb * (BK / 2), m0 + roff, sm.pk_full(s));
-        tma_load_2d(dst + C::kPkBytesA, tmB, kb * (BK / 2), n0 + roff, sm.pk_full(s));
-        if (++s == C::kPkStages) { s = 0; ph ^= 1u; }
-      } else {
-        // operand tiles of both CTAs complete on the leader's barrier
+        if (C::kPackedA) tma_load_2d(dst, tmA, kb * (BK / 2), m0 + roff, sm.pk_full(s));
+        if (C::kPackedB)
+          tma_load_2d(dst + C::kPkBytesA, tmB, kb * (BK / 2), n0 + roff, sm.pk_full(s));
+      }
+      if (C::kDirect) {
+        // direct operand tiles of both CTAs complete on the leader's barrier
         if (!mbar_wait_bounded(sm.op_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer)) return;
         const uint32_t dst = sm.base + C::kOffOp + s * C::kOpStage;
         const uint32_t full_leader = map_to_rank(sm.op_full(s), 0);
-        if (pb.rank == 0) mbar_arrive_expect_tx(sm.op_full(s), 2 * C::kOpStage);
-        tma_load_2d_pair(dst, tmA, kb * BK, m0 + roff, full_leader);
-        tma_load_2d_pair(dst + C::kOpBytesA, tmB, kb * BK, n0 + roff, full_leader);
-        if (++s == C::kOpStages) { s = 0; ph ^= 1u; }
+        if (pb.rank == 0) mbar_arrive_expect_tx(sm.op_full(s), C::kOpFullTx);
+        if (!C::kPackedA) tma_load_2d_pair(dst, tmA, kb * BK, m0 + roff, full_leader);
+        if (!C::kPackedB)
+          tma_load_2d_pair(dst + C::kOpBytesA, tmB, kb * BK, n0 + roff, full_leader);
       }
+      if (++s == C::kOpStages) { s = 0; ph ^= 1u; }
     }
   }
   if (!C::kPacked) {
@@ -166,13 +193,14 @@ __device__ __forceinline__ void producer_role(const Smem& sm, const Problem& pb,
 }
 
 // Widens packed 4-bit tiles into 8-bit operand tiles (see the file comment).
-// Packed stage: [x tile 128 rows x 64 B][W tile 128 rows x 64 B], plain rows.
-// Operand stage: [x tile 128 rows x 128 B][W tile 128 rows x 128 B], rows of
-// 128 B with 16-byte chunk c stored at chunk c ^ (row & 7) (128-byte swizzle).
-template <int BITS>
+// Packed stage: the 4-bit tiles among [x tile 128 rows x 64 B][W tile 128 rows
+// x 64 B], plain rows.  Operand stage: [x tile 128 rows x 128 B][W tile 128
+// rows x 128 B], rows of 128 B with 16-byte chunk c stored at chunk c ^ (row & 7)
+// (128-byte swizzle).
+template <int SA, int SB>
 __device__ __forceinline__ void unpack_role(const Smem& sm, const Problem& pb, int ut,
                                             volatile int* abort_flag) {
-  using C = Cfg<BITS>;
+  using C = Cfg<SA, SB>;
   const int lane = ut & 31;
   int sp = 0, su = 0;
   uint32_t php = 0, phu = 0;
@@ -191,7 +219,7 @@ __device__ __forceinline__ void unpack_role(const Smem& sm, const Problem& pb, i
       for (int i = 0; i < C::kChunksPerThread; ++i) {
         const int c = ut + i * C::kUnpackThreads;
         const uint4 w = wv[i];
-        const int r = c >> 2;  // operand row (x rows 0..127, then W rows)
+        const int r = C::kUnpackRow0 + (c >> 2);  // operand row (x rows 0..127, then W rows)
         const int j = c & 3;   // packed 16-byte chunk within the row's 64 bytes
         uint4 lo, hi;
         lo.x = (w.x << 4) & 0xF0F0F0F0u;
@@ -202,6 +230,15 @@ __device__ __forceinline__ void unpack_role(const Smem& sm, const Problem& pb, i
         hi.y = w.y & 0xF0F0F0F0u;
         hi.z = w.z & 0xF0F0F0F0u;
         hi.w = w.w & 0xF0F0F0F0u;
+        if (!C::kAllPacked) {
+          // the other operand is in natural K order: interleave the low-nibble
+          // (even) and high-nibble (odd) bytes back to elements 0..15, 16..31
+          const uint4 l = lo, h = hi;
+          lo = make_uint4(__byte_perm(l.x, h.x, 0x5140), __byte_perm(l.x, h.x, 0x7362),
+                          __byte_perm(l.y, h.y, 0x5140), __byte_perm(l.y, h.y, 0x7362));
+          hi = make_uint4(__byte_perm(l.z, h.z, 0x5140), __byte_perm(l.z, h.z, 0x7362),
+                          __byte_perm(l.w, h.w, 0x5140), __byte_perm(l.w, h.w, 0x7362));
+        }
         uint8_t* rowp = op + r * 128;
         *reinterpret_cast<uint4*>(rowp + (((2 * j) ^ (r & 7)) << 4)) = lo;
         *reinterpret_cast<uint4*>(rowp + (((2 * j + 1) ^ (r & 7)) << 4)) = hi;
@@ -225,13 +262,13 @@ __device__ __forceinline__ void unpack_role(const Smem& sm, const Problem& pb, i
   }
 }
 
-// 4-bit, non-leader CTA only: forwards "this CTA's operand stage is unpacked"
+// A 4-bit operand, non-leader CTA only: forwards "this CTA's operand stage is unpacked"
 // to the leader's "full" barrier with one 16-byte signalling bulk copy per
 // stage (the leader's MMA thread arms that barrier with the 16 bytes).
-template <int BITS>
+template <int SA, int SB>
 __device__ __forceinline__ void relay_role(const Smem& sm, const Problem& pb,
                                            volatile int* abort_flag) {
-  using C = Cfg<BITS>;
+  using C = Cfg<SA, SB>;
   int s = 0;
   uint32_t ph = 0;
   for (int t = pb.pair; t < pb.num_tiles; t += pb.num_pairs) {
@@ -245,10 +282,10 @@ __device__ __forceinline__ void relay_role(const Smem& sm, const Problem& pb,
 }
 
 // Leader CTA only.
-template <int BITS>
+template <int SA, int SB>
 __device__ __forceinline__ void mma_role(const Smem& sm, const Problem& pb, uint32_t tmem_base,
                                          volatile int* abort_flag) {
-  using C = Cfg<BITS>;
+  using C = Cfg<SA, SB>;
   constexpr uint32_t idesc = idesc_i8(BM, BN);
   int s = 0;
   uint32_t ph = 0;
@@ -260,7 +297,7 @@ __device__ __forceinline__ void mma_role(const Smem& sm, const Problem& pb, uint
     tc_fence_after();
     const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
     for (int kb = 0; kb < pb.kblocks; ++kb) {
-      if (C::kPacked) mbar_arrive_expect_tx(sm.op_full(s), 16);  // the relay's signal
+      if (C::kAllPacked) mbar_arrive_expect_tx(sm.op_full(s), 16);  // the relay's signal
       if (C::kPacked && !mbar_wait_bounded(sm.unpacked(s), ph, abort_flag, kErrWaitMma)) return;
       if (!mbar_wait_cluster_bounded(sm.op_full(s), ph, abort_flag, kErrWaitMma)) return;
       tc_fence_after();
@@ -290,7 +327,7 @@ __device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
 }
 
 // Converts one 32-column chunk of accumulators (one row per thread) and stores it.
-template <int BITS, bool OUT_S32>
+template <int SHIFT, bool OUT_S32>
 __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row, bool row_ok,
                                                int n, int N, float s_a, const float* epi_sw,
                                                const float* epi_b, void* out) {
@@ -298,7 +335,7 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row,
   int32_t acc[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i)
-    acc[i] = BITS == 4 ? (static_cast<int32_t>(r[i]) >> 8) : static_cast<int32_t>(r[i]);
+    acc[i] = static_cast<int32_t>(r[i]) >> SHIFT;
   if (OUT_S32) {
     int32_t* dst = static_cast<int32_t*>(out) + static_cast<int64_t>(row) * N + n;
 #pragma unroll
@@ -335,7 +372,7 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row,
   }
 }
 
-template <int BITS, bool OUT_S32>
+template <int SHIFT, bool OUT_S32>
 __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
                                               uint32_t tmem_base, int quad, int lane, int et,
                                               const float* __restrict__ sa,
@@ -375,11 +412,11 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
 #pragma unroll
     for (int c = 0; c < BN / 32; c += 2) {
       tmem_ld_32x32b_x32(taddr + 32 * (c + 1), rb);
-      epilogue_chunk<BITS, OUT_S32>(ra, row, row_ok, n0 + 32 * c, pb.N, s_a, epi_sw + 32 * c,
+      epilogue_chunk<SHIFT, OUT_S32>(ra, row, row_ok, n0 + 32 * c, pb.N, s_a, epi_sw + 32 * c,
                                     epi_b + 32 * c, out);
       tmem_wait_ld();
       if (c + 2 < BN / 32) tmem_ld_32x32b_x32(taddr + 32 * (c + 2), ra);
-      epilogue_chunk<BITS, OUT_S32>(rb, row, row_ok, n0 + 32 * (c + 1), pb.N, s_a,
+      epilogue_chunk<SHIFT, OUT_S32>(rb, row, row_ok, n0 + 32 * (c + 1), pb.N, s_a,
                                     epi_sw + 32 * (c + 1), epi_b + 32 * (c + 1), out);
       tmem_wait_ld();
     }
@@ -394,12 +431,12 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
   }
 }
 
-template <int BITS, bool OUT_S32>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<BITS>::kThreads, 1)
+template <int SA, int SB, bool OUT_S32>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<SA, SB>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const float* __restrict__ sa, const float* __restrict__ sw,
                  const uint16_t* __restrict__ bias, void* out, int M, int N, int K) {
-  using C = Cfg<BITS>;
+  using C = Cfg<SA, SB>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The padding is identical in both CTAs (same kernel, same static layout),
   // so every shared object has the same offset in the two CTAs of a pair.
@@ -458,16 +495,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<BITS>::kThreads,
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) producer_role<BITS>(sm, pb, &tmA, &tmB, abort_flag);
+    if (lane == 0) producer_role<SA, SB>(sm, pb, &tmA, &tmB, abort_flag);
   } else if (warp == 1) {
-    if (lane == 0 && pb.rank == 0) mma_role<BITS>(sm, pb, tmem_base, abort_flag);
-    if (lane == 0 && pb.rank != 0 && C::kPacked) relay_role<BITS>(sm, pb, abort_flag);
+    if (lane == 0 && pb.rank == 0) mma_role<SA, SB>(sm, pb, tmem_base, abort_flag);
+    if (lane == 0 && pb.rank != 0 && C::kPacked) relay_role<SA, SB>(sm, pb, abort_flag);
   } else if (warp < 2 + C::kEpiWarps) {
     float* epi_sw = reinterpret_cast<float*>(sm.ptr + C::kOffEpi);
-    epilogue_role<BITS, OUT_S32>(sm, pb, tmem_base, warp & 3, lane, threadIdx.x - 64, sa, sw,
+    epilogue_role<C::kAccShift, OUT_S32>(sm, pb, tmem_base, warp & 3, lane, threadIdx.x - 64, sa, sw,
                                  bias, out, epi_sw, epi_sw + BN, abort_flag);
   } else {
-    if (C::kPacked) unpack_role<BITS>(sm, pb, threadIdx.x - 32 * (2 + C::kEpiWarps), abort_flag);
+    if (C::kPacked) unpack_role<SA, SB>(sm, pb, threadIdx.x - 32 * (2 + C::kEpiWarps), abort_flag);
   }
 
   tc_fence_before();

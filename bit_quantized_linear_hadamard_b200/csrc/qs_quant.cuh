@@ -25,12 +25,21 @@
 // round-to-nearest-even of the exact u*inv + 1.5*2^23 is 1.5*2^23 +
 // rint_half_even(u*inv) (1.5*2^23 is even), and the integer lands in the low
 // mantissa bits (two's complement in the low 16 bits).
+//
+// Code widths: 4 bits (qmax 7, two codes per byte), 6 bits (qmax 31, the
+// W4A6 activations of DVD-Quant, one int8 byte per code) and 8 bits (qmax 127).
 #pragma once
 
 #include "qs_host.cuh"
 #include "qs_ptx.cuh"
 
 namespace qs {
+
+// Largest code magnitude of a b-bit symmetric grid, 2^(b-1) - 1.
+__host__ __device__ constexpr int code_qmax(int bits) { return (1 << (bits - 1)) - 1; }
+// Bits of storage per code: 4-bit codes are packed in nibbles, wider codes
+// take one byte.
+__host__ __device__ constexpr int code_storage_bits(int bits) { return bits == 4 ? 4 : 8; }
 
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr float kZeroRowT = 0x1p-120f;
@@ -159,8 +168,8 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
     const __grid_constant__ CUtensorMap tmx, int64_t rows, int K, int nblk, int rpc,
     int64_t num_groups, int stages, float alpha, float scale_mul, int rotate,
     uint8_t* __restrict__ out, float* __restrict__ scale_out) {
-  constexpr int kQmax = BITS == 4 ? 7 : 127;
-  constexpr int kOutBytes = 64 * BITS / 8;  // packed bytes per half block
+  constexpr int kQmax = code_qmax(BITS);
+  constexpr int kOutBytes = 64 * code_storage_bits(BITS) / 8;  // packed bytes per half block
   extern __shared__ __align__(1024) uint8_t qsmem_raw[];
   __shared__ unsigned int row_amax[3][128];
   __shared__ int abort_flag;
@@ -324,7 +333,8 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
       }
     }
     uint8_t* dst =
-        out + row * static_cast<int64_t>(K * BITS / 8) + blk * (2 * kOutBytes) + up * kOutBytes;
+        out + row * static_cast<int64_t>(K * code_storage_bits(BITS) / 8) + blk * (2 * kOutBytes) +
+        up * kOutBytes;
     if (BITS == 4) {  // 16 bytes of elements 0..31, then 16 bytes of 32..63
       *reinterpret_cast<uint4*>(dst) = make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
       *reinterpret_cast<uint4*>(dst + 16) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
@@ -355,7 +365,7 @@ __global__ void __launch_bounds__(MAXT) rotate_quant_group_kernel(const uint16_t
                                                                   float scale_mul, int rotate,
                                                                   uint8_t* __restrict__ out,
                                                                   float* __restrict__ scale_out) {
-  constexpr int kQmax = BITS == 4 ? 7 : 127;
+  constexpr int kQmax = code_qmax(BITS);
   __shared__ float warp_max[32];
 
   const int64_t row = blockIdx.x;
@@ -544,10 +554,16 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
 inline cudaError_t launch_rotate_quant(const uint16_t* x, int64_t rows, int K, int bits, float alpha,
                                        float scale_mul, int rotate, uint8_t* out, float* scale,
                                        cudaStream_t stream) {
-  return bits == 4 ? launch_rotate_quant_bits<4>(x, rows, K, alpha, scale_mul, rotate, out, scale,
-                                                 stream)
-                   : launch_rotate_quant_bits<8>(x, rows, K, alpha, scale_mul, rotate, out, scale,
-                                                 stream);
+  switch (bits) {
+    case 4:
+      return launch_rotate_quant_bits<4>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream);
+    case 6:
+      return launch_rotate_quant_bits<6>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream);
+    case 8:
+      return launch_rotate_quant_bits<8>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream);
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace qs

@@ -42,6 +42,11 @@ class LayerConfig:
     outlier_factor: float
     sigma_w: float
     alpha: float
+    bits_x: int = 0  # activation code width; 0 = the same as `bits` (the weights')
+
+    @property
+    def act_bits(self) -> int:
+        return self.bits_x or self.bits
 
     @property
     def n_outliers(self) -> int:
@@ -75,7 +80,13 @@ WAN_CHAIN = ChainConfig(
     (("qkv", 5120, 15360), ("out", 5120, 5120), ("ffn_up", 5120, 13824), ("ffn_down", 13824, 5120)),
 )
 
+# Mixed widths at the same FFN shape: QuantSparse's W4A8 and DVD-Quant's W4A6
+# (both "Resumen técnico" §4).
+WAN_FFN_W4A8 = LayerConfig("w4a8_wan14b_ffn_up_M32760_K5120_N13824", 5, 4, 32760, 5120, 13824, 0.005, 100.0, 0.015, 1.0, 8)
+WAN_FFN_W4A6 = LayerConfig("w4a6_wan14b_ffn_up_M32760_K5120_N13824", 6, 4, 32760, 5120, 13824, 0.005, 100.0, 0.015, 0.9, 6)
+
 LAYER_CONFIGS = (TINY, HY_QKV, WAN_FFN, WAN_FFN_W8)
+MIXED_CONFIGS = (WAN_FFN_W4A8, WAN_FFN_W4A6)
 
 
 def _bf16(t: torch.Tensor) -> torch.Tensor:
@@ -107,9 +118,10 @@ def make_layer(cfg: LayerConfig, M: int | None = None) -> dict:
 
 def make_shape(seed: int, M: int, K: int, N: int, bits: int, alpha: float = 1.0,
                outlier_frac: float = 0.01, outlier_factor: float = 20.0,
-               sigma_w: float = 0.02) -> dict:
+               sigma_w: float = 0.02, bits_x: int = 0) -> dict:
     """Same recipe at an arbitrary shape (parity cases and edge shapes)."""
-    cfg = LayerConfig("custom", seed, bits, M, K, N, outlier_frac, outlier_factor, sigma_w, alpha)
+    cfg = LayerConfig("custom", seed, bits, M, K, N, outlier_frac, outlier_factor, sigma_w, alpha,
+                      bits_x)
     return make_layer(cfg)
 
 

@@ -1,13 +1,15 @@
 /*
  * qs.h — C ABI of libqs.so: the Hadamard-rotated W4A4 / W8A8 quantized linear
- * layer on NVIDIA B200 (sm_100a).
+ * layer, and its mixed-width forms W4A8 / W4A6, on NVIDIA B200 (sm_100a).
  *
  * The layer follows DVD-Quant ("Data-free Video Diffusion Transformers
  * Quantization"), "Resumen técnico" §2.B, Auto-scaling Rotated Quantization:
  * a Hadamard rotation is applied to both activations and weights, and the
  * quantization scales are computed at run time from the rotated activations
- * (no calibration data).  The bit widths are W4A4 (§1, §4) or the 8-bit branch
- * of δ-GBS (§2.C).  Quantities the pages leave open are fixed here as follows:
+ * (no calibration data).  The bit widths are W4A4 (§1, §4), the 8-bit branch
+ * of δ-GBS (§2.C), W4A6 (DVD-Quant §4, the 6-bit activation setting) and
+ * W4A8 (QuantSparse, "Resumen técnico" §4: 4-bit weights, 8-bit
+ * activations).  Quantities the pages leave open are fixed here as follows:
  *   - rotation: Sylvester Hadamard of order 128 in natural order,
  *     H[i][j] = (-1)^popcount(i&j), on consecutive blocks of 128 along K,
  *     computed as the binary32 butterfly with stages h = 1,2,4,...,64;
@@ -16,7 +18,7 @@
  *   - activations: one scale per token (row) over all of K, clip ratio alpha;
  *     weights: one scale per output channel (row of W), alpha = 1;
  *   - t = fl(alpha * amax); stored scale s = fl(t / qmax); multiplier
- *     inv = fl(qmax / t); qmax = 7 (4 bits) or 127 (8 bits);
+ *     inv = fl(qmax / t); qmax = 2^(bits-1) - 1: 7, 31 or 127 for 4, 6, 8 bits;
  *     q = clamp(round_half_even(u * inv), -qmax, qmax), the product exact and
  *     rounded once; rows with t < 2^-120 (amax == 0 included): s = 0, q = 0;
  *   - out = bf16_rne(fl(fl(fl(s_a[m] * s_w[n]) * float(acc[m][n])) + bias[n])),
@@ -32,11 +34,11 @@
  *     returns anything but QS_OK has launched nothing.
  *   - No C++ exception crosses this interface.
  *
- * Packed formats (row-major, rows of K*bits/8 bytes)
- *   - 8 bits: one two's complement byte per element.
+ * Packed formats (row-major; rows of K/2 bytes for 4 bits, K bytes otherwise)
+ *   - 8 and 6 bits: one two's complement byte per element.
  *   - 4 bits: two's complement nibbles; byte j of a row holds element 2j in
  *     its low nibble and element 2j+1 in its high nibble.
- *   Codes are always in [-qmax, qmax].
+ *   Codes are always in [-qmax, qmax].  `bits` arguments take 4, 6 or 8.
  */
 #ifndef QS_H_
 #define QS_H_
@@ -57,7 +59,7 @@ typedef enum {
   QS_OK = 0,
   QS_ERR_NULL = 1,     /* a required pointer is NULL */
   QS_ERR_SHAPE = 2,    /* M, N or K <= 0, K % 128 != 0, or N % 16 != 0 */
-  QS_ERR_BITS = 3,     /* bits not 4 or 8 */
+  QS_ERR_BITS = 3,     /* bits not 4, 6 or 8 */
   QS_ERR_ALIGN = 4,    /* a pointer is not 16-byte aligned */
   QS_ERR_RANGE = 5,    /* alpha outside [2^-14, 1], unknown flag bits, or a size above its limit */
   QS_ERR_CUDA = 6,     /* a CUDA runtime/driver call or a launch failed */
@@ -82,9 +84,9 @@ typedef enum {
  * to the activations.  Rotates every row of W along K, quantizes it with its
  * own scale (one per output channel, alpha = 1) and packs it.
  *   w_bf16   [N, K] bf16, row-major (torch.nn.Linear layout; y = x W^T + b)
- *   bits     4 or 8
+ *   bits     4, 6 or 8
  *   flags    0 or QS_FLAG_NO_ROTATE
- *   w_packed [N, K*bits/8] bytes, written
+ *   w_packed [N, K/2] bytes (4 bits) or [N, K] bytes, written
  *   w_scale  [N] float, written: s * 2^-7 (or s with QS_FLAG_NO_ROTATE)
  */
 QS_API qs_status qs_pack_weights(const void* w_bf16, int64_t N, int64_t K, int bits, unsigned flags,
@@ -97,9 +99,10 @@ QS_API qs_status qs_pack_weights(const void* w_bf16, int64_t N, int64_t K, int b
  * 128-point block Walsh-Hadamard transform along K, absmax, scale with clip
  * ratio alpha, round-half-even, pack.
  *   x_bf16   [M, K] bf16, row-major
+ *   bits     4, 6 or 8
  *   alpha    clip ratio in [2^-14, 1]
  *   flags    0 or QS_FLAG_NO_ROTATE
- *   x_packed [M, K*bits/8] bytes, written
+ *   x_packed [M, K/2] bytes (4 bits) or [M, K] bytes, written
  *   x_scale  [M] float, written (the per-token scale s_a)
  */
 QS_API qs_status qs_quant_act(const void* x_bf16, int64_t M, int64_t K, int bits, float alpha,
@@ -120,6 +123,21 @@ QS_API qs_status qs_qlinear(const void* x_packed, const float* x_scale, const vo
                      int64_t K, int bits, void* out_bf16, void* stream);
 
 /*
+ * qs_qlinear_mixed — qs_qlinear with the activation codes at `bits_x` and the
+ * weight codes at `bits_w` (each 4, 6 or 8): W4A8 is bits_x = 8, bits_w = 4
+ * (QuantSparse §4), W4A6 is bits_x = 6, bits_w = 4 (DVD-Quant §4).  Same
+ * arithmetic and output as qs_qlinear; qs_qlinear(..., bits, ...) is this
+ * call with bits_x = bits_w = bits.
+ *   x_packed, x_scale  from qs_quant_act at bits_x
+ *   w_packed, w_scale  from qs_pack_weights at bits_w
+ *   other arguments as qs_qlinear
+ */
+QS_API qs_status qs_qlinear_mixed(const void* x_packed, const float* x_scale, int bits_x,
+                                  const void* w_packed, const float* w_scale, int bits_w,
+                                  const void* bias_bf16, int64_t M, int64_t N, int64_t K,
+                                  void* out_bf16, void* stream);
+
+/*
  * qs_qgemm_s32 — the same GEMM main loop with an int32 epilogue: writes the
  * exact accumulators acc[m][n] = sum_k q_a[m][k] q_w[n][k] (parity checks).
  *   acc [M, N] int32, row-major, written.  N % 16 == 0.
@@ -127,11 +145,17 @@ QS_API qs_status qs_qlinear(const void* x_packed, const float* x_scale, const vo
 QS_API qs_status qs_qgemm_s32(const void* x_packed, const void* w_packed, int64_t M, int64_t N,
                        int64_t K, int bits, int32_t* acc, void* stream);
 
+/* qs_qgemm_s32_mixed — qs_qgemm_s32 with separate code widths (as qs_qlinear_mixed). */
+QS_API qs_status qs_qgemm_s32_mixed(const void* x_packed, int bits_x, const void* w_packed,
+                                    int bits_w, int64_t M, int64_t N, int64_t K, int32_t* acc,
+                                    void* stream);
+
 /*
  * qs_linear_workspace_bytes — bytes of device scratch that qs_linear needs for
- * M tokens of K inputs at `bits`: the packed activations (M*K*bits/8 bytes,
- * rounded up to 256) followed by the per-token scales (4*M bytes).  Returns
- * -1 for arguments qs_linear would reject.
+ * M tokens of K inputs with activation codes of `bits`: the packed activations
+ * (M*K/2 bytes for 4 bits, M*K otherwise, rounded up to 256) followed by the
+ * per-token scales (4*M bytes).  Returns -1 for arguments qs_linear would
+ * reject.
  */
 QS_API int64_t qs_linear_workspace_bytes(int64_t M, int64_t K, int bits);
 
@@ -152,6 +176,16 @@ QS_API qs_status qs_linear(const void* x_bf16, int64_t M, int64_t K, float alpha
                            const void* w_packed, const float* w_scale, const void* bias_bf16,
                            int64_t N, int bits, void* workspace, int64_t workspace_bytes,
                            void* out_bf16, void* stream);
+
+/*
+ * qs_linear_mixed — qs_linear with the activations quantized at `bits_x` and
+ * weights packed at `bits_w` (W4A8: 8 and 4; W4A6: 6 and 4).  The workspace
+ * is qs_linear_workspace_bytes(M, K, bits_x).
+ */
+QS_API qs_status qs_linear_mixed(const void* x_bf16, int64_t M, int64_t K, float alpha,
+                                 int bits_x, const void* w_packed, const float* w_scale,
+                                 int bits_w, const void* bias_bf16, int64_t N, void* workspace,
+                                 int64_t workspace_bytes, void* out_bf16, void* stream);
 
 /*
  * qs_gelu_bf16 — elementwise GELU (exact erf form, binary32 arithmetic,

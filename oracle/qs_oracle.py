@@ -268,7 +268,7 @@ def qlinear(x_bits, w_bits, bias_bits, bits: int, alpha: float,
 def qlinear_mixed(x_bits, w_bits, bias_bits, bits_x: int, bits_w: int, alpha: float,
                   rotate: bool = True):
     """The layer with different code widths for activations and weights
-    (QuantSparse's W4A8, DVD-Quant's W4A6): each side is quantised at its own
+    (QuantSparse "Resumen técnico" §4: W4A8; DVD-Quant "Resumen técnico" §4: W4A6): each side is quantised at its own
     width, the integer product and the epilogue are unchanged."""
     qa, sa = quant_act(x_bits, bits_x, alpha, rotate)
     qw, sw = pack_weights(w_bits, bits_w, rotate)

@@ -89,10 +89,31 @@ def test_qlinear_validation(lib):
     assert f(A, B, C, D, NUL, 8, 264, 128, 4, A, NUL) == SHAPE   # N % 16
     assert f(A, B, C, D, NUL, 8, 256, 192, 4, A, NUL) == SHAPE   # K % 128
     assert f(A, B, C, D, NUL, 0, 256, 128, 4, A, NUL) == SHAPE
-    assert f(A, B, C, D, NUL, 8, 256, 128, 6, A, NUL) == BITS
+    assert f(A, B, C, D, NUL, 8, 256, 128, 5, A, NUL) == BITS
+    assert f(A, B, C, D, NUL, 8, 256, 128, 16, A, NUL) == BITS
     assert f(A, B, C, D, NUL, 8, 256, 2 * 65536, 8, A, NUL) == RANGE
     assert f(A, B, C, D, MIS, 8, 256, 128, 4, A, NUL) == ALIGN   # bias
     assert f(MIS, B, C, D, NUL, 8, 256, 128, 4, A, NUL) == ALIGN
+
+
+def test_mixed_validation(lib):
+    f = lib.qs_qlinear_mixed
+    assert f(NUL, B, 8, C, D, 4, NUL, 8, 256, 128, A, NUL) == NULL
+    assert f(A, B, 8, C, NUL, 4, NUL, 8, 256, 128, A, NUL) == NULL
+    assert f(A, B, 7, C, D, 4, NUL, 8, 256, 128, A, NUL) == BITS
+    assert f(A, B, 8, C, D, 2, NUL, 8, 256, 128, A, NUL) == BITS
+    assert f(A, B, 8, C, D, 4, NUL, 8, 264, 128, A, NUL) == SHAPE
+    assert f(A, B, 6, C, D, 4, MIS, 8, 256, 128, A, NUL) == ALIGN
+    g = lib.qs_qgemm_s32_mixed
+    assert g(A, 8, NUL, 4, 8, 256, 128, C, NUL) == NULL
+    assert g(A, 8, B, 3, 8, 256, 128, C, NUL) == BITS
+    assert g(A, 6, B, 4, 8, 256, 192, C, NUL) == SHAPE
+    h = lib.qs_linear_mixed
+    need = lib.qs_linear_workspace_bytes(8, 128, 8)
+    assert h(A, 8, 128, 1.0, 8, B, C, 4, NUL, 256, D, need, A, NUL) == PTR  # fake addresses
+    assert h(A, 8, 128, 1.0, 8, B, C, 4, NUL, 256, D, need - 1, A, NUL) == RANGE
+    assert h(A, 8, 128, 1.0, 9, B, C, 4, NUL, 256, D, need, A, NUL) == BITS
+    assert h(A, 8, 128, 0.0, 8, B, C, 4, NUL, 256, D, need, A, NUL) == RANGE
 
 
 def test_qgemm_and_gelu_validation(lib):
@@ -126,6 +147,7 @@ def test_linear_validation_and_workspace(lib):
     assert lib.qs_linear_workspace_bytes(256, 512, 4) == 256 * 256 + 4 * 256
     assert lib.qs_linear_workspace_bytes(3, 128, 4) == 256 + 12          # packed part rounded to 256
     assert lib.qs_linear_workspace_bytes(3, 128, 8) == 512 + 12
+    assert lib.qs_linear_workspace_bytes(3, 128, 6) == 512 + 12          # 6-bit codes take a byte
     assert lib.qs_linear_workspace_bytes(3, 100, 4) == -1
     assert lib.qs_linear_workspace_bytes(3, 128, 5) == -1
     need = lib.qs_linear_workspace_bytes(8, 128, 4)

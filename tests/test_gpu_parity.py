@@ -77,7 +77,7 @@ QUANT_SHAPES = [(1, 128), (3, 256), (129, 640), (64, 3072), (33, 5120), (17, 138
                 (5, 16384), (3, 16512), (2, 65536)]
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", [4, 6, 8])
 @pytest.mark.parametrize("M,K", QUANT_SHAPES)
 def test_quant_act_bit_exact(M, K, bits):
     d = I.make_shape(seed=100 + M + K, M=M, K=K, N=16, bits=bits, outlier_factor=50.0)
@@ -122,12 +122,12 @@ def test_quant_zero_tiny_and_constant_rows():
     x[4, ::3] = 1e30
     x[5] = torch.linspace(-4, 4, 512)
     xb = x.to(torch.bfloat16)
-    for bits in (4, 8):
+    for bits in (4, 6, 8):
         for alpha in (1.0, 0.5, 1e-3):
             check_quant(xb, bits, alpha)
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", [4, 6, 8])
 @pytest.mark.parametrize("alpha", [1.0 / 256, 1.0 / 256 * 0.999, 0.02])
 def test_quant_small_alpha_heavy_clipping(bits, alpha):
     # most codes clip; 1/256 is the smallest alpha whose unclamped codes still
@@ -136,7 +136,7 @@ def test_quant_small_alpha_heavy_clipping(bits, alpha):
     check_quant(d["x"], bits, alpha)
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", [4, 6, 8])
 def test_pack_weights_bit_exact(bits):
     d = I.make_layer(I.TINY)
     wp, ws = gpu_pack(d["w"], bits)
@@ -186,14 +186,48 @@ def test_qgemm_s32_extreme_codes_at_max_k(bits):
     assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.int_gemm(qa, qw))
 
 
+# mixed code widths (x, W): W4A8, W4A6, and the other pairings the kernel serves
+MIXED = [(8, 4), (6, 4), (4, 8), (6, 6), (6, 8)]
+
+
+@pytest.mark.parametrize("bx,bw", MIXED)
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_qgemm_s32_mixed_bit_exact_on_oracle_codes(M, N, K, bx, bw):
+    rng = np.random.default_rng(M * 5 + N * 11 + K + 10 * bx + bw)
+    qa, qw = _codes(rng, (M, K), bx), _codes(rng, (N, K), bw)
+    xp = torch.from_numpy(O.pack(qa, bx)).cuda()
+    wp = torch.from_numpy(O.pack(qw, bw)).cuda()
+    acc = qs.qgemm_s32(xp, wp, bx, K, bits_w=bw)
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.int_gemm(qa, qw))
+
+
+@pytest.mark.parametrize("bx,bw", [(8, 4), (4, 8)])
+def test_qgemm_s32_mixed_extreme_codes_at_max_k(bx, bw):
+    # 127 * 7 * 65536 with the 4-bit side widened to 16 q: the hardware sum
+    # 16 * 127 * 7 * 65536 still fits int32
+    K = 65536
+    qa = np.full((3, K), O.QMAX[bx], np.int8)
+    qa[1] = -O.QMAX[bx]
+    qa[2, ::2] = -O.QMAX[bx]
+    qw = np.full((16, K), -O.QMAX[bw], np.int8)
+    qw[5] = O.QMAX[bw]
+    acc = qs.qgemm_s32(torch.from_numpy(O.pack(qa, bx)).cuda(),
+                       torch.from_numpy(O.pack(qw, bw)).cuda(), bx, K, bits_w=bw)
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.int_gemm(qa, qw))
+
+
 # --------------------------------------------------------------------------- whole layer
 
-def run_layer(d, bits, alpha, bias=True):
+def run_layer(d, bits, alpha, bias=True, bits_x=None):
+    """bits: the weights' code width; bits_x: the activations' (default bits)."""
+    bx = bits if bits_x is None else bits_x
     x, w, b = d["x"].cuda(), d["w"].cuda(), d["bias"].cuda() if bias else None
     wp, ws = qs.pack_weights(w, bits)
-    xp, xs = qs.quant_act(x, bits, alpha)
-    out = qs.qlinear(xp, xs, wp, ws, b, bits, x.shape[1])
-    acc = qs.qgemm_s32(xp, wp, bits, x.shape[1])
+    xp, xs = qs.quant_act(x, bx, alpha)
+    out = qs.qlinear(xp, xs, wp, ws, b, bx, x.shape[1], bits_w=bits)
+    acc = qs.qgemm_s32(xp, wp, bx, x.shape[1], bits_w=bits)
     torch.cuda.synchronize()
     return {"out": out, "acc": acc, "xp": xp, "xs": xs, "wp": wp, "ws": ws}
 
@@ -210,6 +244,42 @@ def test_qlinear_matches_oracle(M, N, K, bits, alpha):
     got = g["out"].view(torch.int16).cpu().numpy().view(np.uint16)
     exact = assert_within_1ulp(got, r["out"], f"{M}x{N}x{K} w{bits}")
     assert exact == 1.0, f"only {exact:.6f} of outputs bit-identical"
+
+
+@pytest.mark.parametrize("bx,bw,alpha", [(8, 4, 1.0), (8, 4, 0.9), (6, 4, 0.9), (4, 8, 1.0),
+                                         (6, 6, 1.0)])
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_qlinear_mixed_matches_oracle(M, N, K, bx, bw, alpha):
+    d = I.make_shape(seed=M + 2 * N + K, M=M, K=K, N=N, bits=bw, alpha=alpha, outlier_factor=50.0,
+                     bits_x=bx)
+    g = run_layer(d, bw, alpha, bits_x=bx)
+    r = O.qlinear_mixed(bits16(d["x"]), bits16(d["w"]), bits16(d["bias"]), bx, bw, alpha)
+    assert np.array_equal(g["xp"].cpu().numpy(), r["xp"])
+    assert np.array_equal(g["wp"].cpu().numpy(), r["wp"])
+    assert np.array_equal(g["acc"].cpu().numpy().astype(np.int64), r["acc"])
+    got = g["out"].view(torch.int16).cpu().numpy().view(np.uint16)
+    exact = assert_within_1ulp(got, r["out"], f"{M}x{N}x{K} a{bx}w{bw}")
+    assert exact == 1.0, f"only {exact:.6f} of outputs bit-identical"
+
+
+@pytest.mark.parametrize("bx,bw", [(8, 4), (6, 4)])
+def test_linear_mixed_one_call(bx, bw):
+    M, N, K, alpha = 300, 768, 640, 0.9
+    d = I.make_shape(seed=31 + bx, M=M, K=K, N=N, bits=bw, alpha=alpha, outlier_factor=50.0,
+                     bits_x=bx)
+    g = run_layer(d, bw, alpha, bits_x=bx)
+    need = qs.qs_linear_workspace_bytes(M, K, bx)
+    ws = torch.full((need,), 0x5A, dtype=torch.uint8, device="cuda")
+    out = qs.linear(d["x"].cuda(), g["wp"], g["ws"], d["bias"].cuda(), bx, alpha, workspace=ws,
+                    bits_w=bw)
+    layer = qs.QuantLinear(d["w"].cuda(), d["bias"].cuda(), bw, alpha, bits_x=bx)
+    out2 = layer(d["x"].cuda())
+    torch.cuda.synchronize()
+    want = g["out"].view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), want)
+    assert np.array_equal(out2.view(torch.int16).cpu().numpy().view(np.uint16), want)
+    r = O.qlinear_mixed(bits16(d["x"]), bits16(d["w"]), bits16(d["bias"]), bx, bw, alpha)
+    assert np.array_equal(want, r["out"])
 
 
 def test_qlinear_null_bias_and_zero_rows():
@@ -257,13 +327,14 @@ def test_gelu_matches_oracle():
 
 # --------------------------------------------------------------------------- full-size configs
 
-def _sampled_parity(d, bits, alpha, rows, cols):
-    g = run_layer(d, bits, alpha)
+def _sampled_parity(d, bits, alpha, rows, cols, bits_x=None):
+    bx = bits if bits_x is None else bits_x
+    g = run_layer(d, bits, alpha, bits_x=bx)
     xb, wb, bb = bits16(d["x"][rows]), bits16(d["w"][cols]), bits16(d["bias"][cols])
-    qa, sa = O.quant_act(xb, bits, alpha)
+    qa, sa = O.quant_act(xb, bx, alpha)
     qw, sw = O.pack_weights(wb, bits)
     assert np.array_equal(g["xs"].cpu().numpy()[rows].view(np.uint32), sa.view(np.uint32))
-    assert np.array_equal(g["xp"].cpu().numpy()[rows], O.pack(qa, bits))
+    assert np.array_equal(g["xp"].cpu().numpy()[rows], O.pack(qa, bx))
     assert np.array_equal(g["ws"].cpu().numpy()[cols].view(np.uint32), sw.view(np.uint32))
     assert np.array_equal(g["wp"].cpu().numpy()[cols], O.pack(qw, bits))
     acc = O.int_gemm(qa, qw)
@@ -284,11 +355,12 @@ def _samples(M, N, seed):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("cfg", [I.HY_QKV, I.WAN_FFN, I.WAN_FFN_W8], ids=lambda c: c.name)
+@pytest.mark.parametrize("cfg", [I.HY_QKV, I.WAN_FFN, I.WAN_FFN_W8, *I.MIXED_CONFIGS],
+                         ids=lambda c: c.name)
 def test_full_size_config_sampled(cfg):
     d = I.make_layer(cfg)
     rows, cols = _samples(cfg.M, cfg.N, cfg.seed)
-    _sampled_parity(d, cfg.bits, cfg.alpha, rows, cols)
+    _sampled_parity(d, cfg.bits, cfg.alpha, rows, cols, bits_x=cfg.act_bits)
 
 
 @pytest.mark.slow
