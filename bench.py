@@ -54,6 +54,8 @@ def parse():
                    help="skip the per-config table and the quality report")
     p.add_argument("--tokens", type=int, default=None,
                    help="override M (profiling captures of a smaller case of the same shape)")
+    p.add_argument("--workload", default=None,
+                   help="the Wan FFN variant to time: w4a4 (default), w8a8, w4a8 or w4a6")
     return p.parse_args()
 
 
@@ -75,9 +77,10 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, or None if the
-    kernels changed since the counters were taken."""
+def ncu_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of `kernel` in `workload` from the committed ncu
+    summary, or None if there is none or the kernels changed since the
+    counters were taken."""
     path = os.path.join(PROFILES, "ncu_traffic.json")
     if not os.path.exists(path):
         return None
@@ -85,8 +88,20 @@ def ncu_traffic(kernel: str):
         d = json.load(f)
     if d.get("source_hash") != kernel_source_hash():
         return None
-    k = d.get("kernels", {}).get(kernel)
+    k = d.get("workloads", {}).get(workload, {}).get(kernel)
     return None if k is None else k.get("dram_bytes_per_launch_full")
+
+
+def workload_config(I, name):
+    """The Wan-14B FFN up-projection config the step runs (W4A4 by default)."""
+    table = {"w4a4": I.WAN_FFN, "w8a8": I.WAN_FFN_W8, "w4a8": I.WAN_FFN_W4A8,
+             "w4a6": I.WAN_FFN_W4A6}
+    if name is None:
+        return I.WAN_FFN
+    for key, cfg in table.items():
+        if name in (key, cfg.name):
+            return cfg
+    raise SystemExit(f"unknown workload {name!r}; choose one of {sorted(table)}")
 
 
 class ClockSampler:
@@ -145,10 +160,11 @@ class OracleSample:
     workload: `rows` tokens through quant_act + int GEMM + epilogue against
     the full weight (weight packing is offline, done once and not timed)."""
 
-    def __init__(self, d, bits, alpha):
+    def __init__(self, d, bits, alpha, bits_x=None):
         from bit_quantized_linear_hadamard_b200 import inputs as I
         from oracle import qs_oracle as O
         self.O, self.bits, self.alpha = O, bits, alpha
+        self.bits_x = bits if bits_x is None else bits_x
         self.x = d["x"]
         self.qw, self.sw = O.pack_weights(I.bf16_bits(d["w"]), bits)
         self.bb = I.bf16_bits(d["bias"])
@@ -158,7 +174,7 @@ class OracleSample:
     def run(self, rows: int) -> float:
         xb = self.bf16_bits(self.x[:rows])
         t0 = time.perf_counter()
-        qa, sa = self.O.quant_act(xb, self.bits, self.alpha)
+        qa, sa = self.O.quant_act(xb, self.bits_x, self.alpha)
         acc = self.O.int_gemm(qa, self.qw)
         self.O.epilogue(acc, sa, self.sw, self.bb)
         return time.perf_counter() - t0
@@ -284,9 +300,9 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     from bit_quantized_linear_hadamard_b200 import inputs as I
-    cfg = I.WAN_FFN
+    cfg = workload_config(I, args.workload)
     d = I.make_layer(cfg, M=256)
-    sample = OracleSample(d, cfg.bits, cfg.alpha)
+    sample = OracleSample(d, cfg.bits, cfg.alpha, cfg.act_bits)
     rows = 8
     for _ in range(args.warmup):
         sample.run(2)
@@ -295,10 +311,12 @@ def run_reference(args, rank, world):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4" if cfg.act_bits == cfg.bits == 4 else f"int{cfg.bits}w-int{cfg.act_bits}a",
         "data": "synthetic",
-        "config": {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "bits": cfg.bits,
-                   "alpha": cfg.alpha, "seed": cfg.seed, "sample_rows_per_step": rows},
+        "config": {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "bits_w": cfg.bits,
+                   "bits_x": cfg.act_bits, "alpha": cfg.alpha, "seed": cfg.seed,
+                   "sample_rows_per_step": rows},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": f"{rows} tokens per step of the {cfg.M}-token workload, full "
                                    f"K and N, numpy oracle on one host thread"},
@@ -333,24 +351,31 @@ def main():
                                 device_id=dev)
     qs.load()
 
-    cfg = I.WAN_FFN
+    cfg = workload_config(I, args.workload)
     d = I.make_layer(cfg, M=args.tokens)
-    M, K, N, bits, alpha = d["x"].shape[0], cfg.K, cfg.N, cfg.bits, cfg.alpha
+    M, K, N, alpha = d["x"].shape[0], cfg.K, cfg.N, cfg.alpha
+    bits, bx = cfg.bits, cfg.act_bits  # weight and activation code widths
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
         x = d["x"].to(dev)
         w = d["w"].to(dev)
         bias = d["bias"].to(dev)
         wp, ws = qs.pack_weights(w, bits, stream=stream)
-        xp = torch.empty((M, K * bits // 8), dtype=torch.uint8, device=dev)
+        xp = torch.empty((M, qs.packed_cols(K, bx)), dtype=torch.uint8, device=dev)
         xs = torch.empty((M,), dtype=torch.float32, device=dev)
         out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     stream.synchronize()
     del w
 
+    def gemm():
+        if bx == bits:
+            qs.qs_qlinear(xp, xs, wp, ws, bias, M, N, K, bits, out, stream)
+        else:
+            qs.qs_qlinear_mixed(xp, xs, bx, wp, ws, bits, bias, M, N, K, out, stream)
+
     def step():
-        qs.qs_quant_act(x, M, K, bits, alpha, 0, xp, xs, stream)
-        qs.qs_qlinear(xp, xs, wp, ws, bias, M, N, K, bits, out, stream)
+        qs.qs_quant_act(x, M, K, bx, alpha, 0, xp, xs, stream)
+        gemm()
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -368,9 +393,9 @@ def main():
         time.sleep(0.3)
     for i in range(args.steps):
         ev[i][0].record(stream)
-        qs.qs_quant_act(x, M, K, bits, alpha, 0, xp, xs, stream)
+        qs.qs_quant_act(x, M, K, bx, alpha, 0, xp, xs, stream)
         ev[i][1].record(stream)
-        qs.qs_qlinear(xp, xs, wp, ws, bias, M, N, K, bits, out, stream)
+        gemm()
         ev[i][2].record(stream)
     stream.synchronize()
     torch.cuda.synchronize()
@@ -393,12 +418,13 @@ def main():
     out_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
     e2e_steps = max(1, args.e2e_steps)
 
-    ws_bytes = qs.qs_linear_workspace_bytes(M, K, bits)
+    ws_bytes = qs.qs_linear_workspace_bytes(M, K, bx)
     workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
 
     def e2e_step():  # one C call for the layer, host buffers in and out
         x.copy_(x_host, non_blocking=True)
-        qs.qs_linear(x, M, K, alpha, wp, ws, bias, N, bits, workspace, ws_bytes, out, stream)
+        qs.qs_linear_mixed(x, M, K, alpha, bx, wp, ws, bits, bias, N, workspace, ws_bytes, out,
+                           stream)
         out_host.copy_(out, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -418,32 +444,36 @@ def main():
 
     extra = {}
     if world == 1 and not args.no_extras:
-        extra["quality"] = quality(qs, torch, x, d["w"].to(dev), bias, bits, alpha, stream)
+        if bx == bits:
+            extra["quality"] = quality(qs, torch, x, d["w"].to(dev), bias, bits, alpha, stream)
         extra["configs"] = all_configs(qs, torch, I, dev, stream)
     if rank == 0:
         pk, src = peaks()
         int8_peak = pk["bf16_tflops"] * INT8_PER_BF16
         gemm_tops = ops_per_step / (gemm_ms * 1e-3) / 1e12
-        quant_bytes = M * (2 * K + K * bits // 8 + 4)
+        quant_bytes = M * (2 * K + qs.packed_cols(K, bx) + 4)
         quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
         line = {
             "metric": METRIC, "value": value, "unit": UNIT,
             "tokens_per_s": M * world / (ms_per_step * 1e-3),
             "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "int4", "data": "synthetic",
-            "config": {"workload": cfg.name, "M": M, "K": K, "N": N, "bits": bits, "alpha": alpha,
+            "vs_baseline": None, "data": "synthetic",
+            "dtype": "int4" if bx == bits == 4 else f"int{bits}w-int{bx}a",
+            "config": {"workload": cfg.name, "M": M, "K": K, "N": N, "bits_w": bits,
+                       "bits_x": bx, "alpha": alpha,
                        "seed": cfg.seed, "parallelism": f"replicas{world}",
                        "l2": "inputs larger than L2 (x 335 MB, out 906 MB bf16); no flush"},
             "roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak,
                          "unit": UNIT, "frac": gemm_tops / int8_peak,
-                         "traffic": ncu_traffic("qgemm_kernel"),
-                         "kernel": "qgemm_kernel<4,false> (tcgen05 kind::i8)",
+                         "traffic": ncu_traffic(cfg.name, "qgemm_kernel"),
+                         "kernel": f"qgemm_kernel<{4 if bx == 4 else 8},{4 if bits == 4 else 8},"
+                                   f"false> (tcgen05 kind::i8)",
                          "peak_source": f"{src}: bf16_tflops (burst) x {INT8_PER_BF16} "
                                         f"nominal int8:bf16"},
             "roofline_quant": {"bound": "hbm", "achieved": quant_gbs, "peak": pk["hbm_gbs"],
                                "unit": "GB/s", "frac": quant_gbs / pk["hbm_gbs"],
-                               "traffic": ncu_traffic("rotate_quant_kernel"),
+                               "traffic": ncu_traffic(cfg.name, "rotate_quant_kernel"),
                                "algorithmic_bytes": quant_bytes,
                                "peak_source": f"{src}: hbm_gbs"},
             "kernels_ms": {"quant": quant_ms, "gemm": gemm_ms},
@@ -452,12 +482,13 @@ def main():
                     "h2d_bytes_per_step": x_host.numel() * 2,
                     "d2h_bytes_per_step": out_host.numel() * 2,
                     "ms_per_step": e2e_ms, "steps": e2e_steps,
-                    "call": "qs_linear (C ABI), pinned host x in, bf16 output back"},
+                    "call": "qs_linear_mixed (C ABI; = qs_linear at equal widths), pinned host x "
+                            "in, bf16 output back"},
             "clocks": clocks,
         }
         line.update(extra)
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = OracleSample(d, bits, alpha).baseline()
+            line["cpu_baseline"] = OracleSample(d, bits, alpha, bx).baseline()
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
