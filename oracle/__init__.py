@@ -5,3 +5,6 @@ import this package; the product path never does.
 """
 from .qs_oracle import *  # noqa: F401,F403
 from .qs_oracle import QMAX, HADAMARD_BLOCK, WEIGHT_SCALE_FOLD  # noqa: F401
+from .gbs_oracle import (  # noqa: F401
+    GBS_HIGH_BITS, GBS_LOW_BITS, GbsState, gbs_run, gbs_schedule, gbs_update, l1_distance, l1_terms,
+)
