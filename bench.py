@@ -279,6 +279,54 @@ def all_configs(qs, torch, I, dev, stream):
     return res
 
 
+def gbs_sequence(qs, torch, I, dev, stream, steps=8, delta=0.3):
+    """δ-guided bit switching over consecutive steps of the Wan FFN layer:
+    each step is the gated one-call layer plus the on-device distance update.
+    The inputs drift by a seeded amount per step (synthetic stand-in for the
+    denoising trajectory).  Returns per-step widths and times and the update
+    kernel's time against HBM."""
+    cfg = I.WAN_FFN
+    d = I.make_layer(cfg)
+    with torch.cuda.stream(stream):
+        x = d["x"].to(dev)
+        layer = qs.GbsLinear(d["w"].to(dev), d["bias"].to(dev), delta, cfg.alpha, stream=stream)
+        g = torch.Generator(device=dev).manual_seed(cfg.seed)
+        sigmas = [0.0, 0.01, 0.01, 0.3, 0.01, 0.02, 0.02, 0.2, 0.01, 0.01][:steps]
+        widths, step_ms, upd_ms = [], [], []
+        for t in range(steps):
+            if t:
+                x = (x.float() + sigmas[t] * torch.randn(x.shape, generator=g, device=dev,
+                                                         dtype=torch.float32)).to(torch.bfloat16)
+            stream.synchronize()
+            widths.append(qs.gbs_state_host(layer.state)["bits"])
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            M = x.shape[0]
+            if layer.workspace is None:
+                layer.workspace = torch.empty((qs.qs_linear_workspace_bytes(M, cfg.K, 8),),
+                                              dtype=torch.uint8, device=dev)
+            out = torch.empty((M, cfg.N), dtype=torch.bfloat16, device=dev)
+            e[0].record(stream)
+            qs.qs_linear_gbs(x, M, cfg.K, cfg.alpha, layer.w4, layer.s4, layer.w8, layer.s8,
+                             layer.bias, cfg.N, layer.state, layer.workspace,
+                             layer.workspace.numel(), out, stream)
+            e[1].record(stream)
+            qs.qs_gbs_update(out, layer.prev, out.numel(), delta, layer.state, stream)
+            e[2].record(stream)
+            layer.prev = out
+            stream.synchronize()
+            step_ms.append(e[0].elapsed_time(e[2]))
+            if t:
+                upd_ms.append(e[1].elapsed_time(e[2]))
+    n = cfg.M * cfg.N
+    upd = sum(upd_ms) / len(upd_ms)
+    pk, _ = peaks()
+    return {"workload": cfg.name, "delta": delta, "sigmas": sigmas, "widths": widths,
+            "step_ms": step_ms, "update_ms": upd,
+            "update_GBps": 4.0 * n / (upd * 1e-3) / 1e9,
+            "update_frac_hbm": 4.0 * n / (upd * 1e-3) / 1e9 / pk["hbm_gbs"],
+            "update_bytes": 4 * n}
+
+
 def quality(qs, torch, x, w, bias, bits, alpha, stream, rows=256):
     """Relative Frobenius error and SQNR of the layer against the unquantised
     binary64 product, with and without the Hadamard rotation (first `rows` tokens)."""
@@ -447,6 +495,7 @@ def main():
         if bx == bits:
             extra["quality"] = quality(qs, torch, x, d["w"].to(dev), bias, bits, alpha, stream)
         extra["configs"] = all_configs(qs, torch, I, dev, stream)
+        extra["gbs"] = gbs_sequence(qs, torch, I, dev, stream)
     if rank == 0:
         pk, src = peaks()
         int8_peak = pk["bf16_tflops"] * INT8_PER_BF16

@@ -28,9 +28,13 @@ STATUS = {0: "QS_OK", 1: "QS_ERR_NULL", 2: "QS_ERR_SHAPE", 3: "QS_ERR_BITS", 4: 
           5: "QS_ERR_RANGE", 6: "QS_ERR_CUDA", 7: "QS_ERR_TIMEOUT", 8: "QS_ERR_PTR"}
 EXPORTS = ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qlinear_mixed", "qs_qgemm_s32",
            "qs_qgemm_s32_mixed", "qs_gelu_bf16", "qs_linear_workspace_bytes", "qs_linear",
-           "qs_linear_mixed", "qs_linear_noalloc", "qs_selftest_timeout", "qs_device_error",
-           "qs_status_str", "qs_version")
+           "qs_linear_mixed", "qs_linear_noalloc", "qs_gbs_reset", "qs_gbs_update",
+           "qs_linear_gbs", "qs_selftest_timeout", "qs_device_error", "qs_status_str",
+           "qs_version")
 BITS = (4, 6, 8)
+QS_GBS_MAX_BLOCKS = 1024
+# sizeof(qs_gbs_state): acc, last_d (f64), bits, step, blocks_done, reserved (i32), partials
+QS_GBS_STATE_BYTES = 8 + 8 + 4 * 4 + 2 * QS_GBS_MAX_BLOCKS * 8
 QS_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -65,6 +69,10 @@ def load() -> ctypes.CDLL:
     L.qs_linear.argtypes = [vp, i64, i64, f32, vp, vp, vp, i64, i32, vp, i64, vp, vp]
     L.qs_linear_mixed.argtypes = [vp, i64, i64, f32, i32, vp, vp, i32, vp, i64, vp, i64, vp, vp]
     L.qs_linear_noalloc.argtypes = [vp, i64, i64, f32, vp, vp, vp, i64, i32, vp, vp]
+    f64 = ctypes.c_double
+    L.qs_gbs_reset.argtypes = [vp, vp]
+    L.qs_gbs_update.argtypes = [vp, vp, i64, f64, vp, vp]
+    L.qs_linear_gbs.argtypes = [vp, i64, i64, f32, vp, vp, vp, vp, vp, i64, vp, vp, i64, vp, vp]
     L.qs_selftest_timeout.argtypes = [i64, vp]
     L.qs_device_error.argtypes = [vp]
     L.qs_status_str.argtypes = [i32]
@@ -72,7 +80,8 @@ def load() -> ctypes.CDLL:
     L.qs_version.restype = ctypes.c_char_p
     for name in ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qlinear_mixed",
                  "qs_qgemm_s32", "qs_qgemm_s32_mixed", "qs_gelu_bf16", "qs_linear",
-                 "qs_linear_mixed", "qs_linear_noalloc", "qs_selftest_timeout", "qs_device_error"):
+                 "qs_linear_mixed", "qs_linear_noalloc", "qs_gbs_reset", "qs_gbs_update",
+                 "qs_linear_gbs", "qs_selftest_timeout", "qs_device_error"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -216,6 +225,35 @@ def qs_linear_noalloc(x, M, K, alpha, w_packed, w_scale, bias, N, bits, out, str
                                     N, bits, _p(out), _s(stream)), "qs_linear_noalloc")
 
 
+def qs_gbs_reset(state, stream=None):
+    _cuda(state, torch.uint8, "state")
+    _check(load().qs_gbs_reset(_p(state), _s(stream)), "qs_gbs_reset")
+
+
+def qs_gbs_update(y_cur, y_prev, n, delta, state, stream=None):
+    _cuda(y_cur, torch.bfloat16, "y_cur")
+    _cuda(y_prev, torch.bfloat16, "y_prev")
+    _cuda(state, torch.uint8, "state")
+    _check(load().qs_gbs_update(_p(y_cur), _p(y_prev), n, float(delta), _p(state), _s(stream)),
+           "qs_gbs_update")
+
+
+def qs_linear_gbs(x, M, K, alpha, w4_packed, w4_scale, w8_packed, w8_scale, bias, N, state,
+                  workspace, workspace_bytes, out, stream=None):
+    _cuda(x, torch.bfloat16, "x")
+    for t, name in ((w4_packed, "w4_packed"), (w8_packed, "w8_packed"), (state, "state"),
+                    (workspace, "workspace")):
+        _cuda(t, torch.uint8, name)
+    _cuda(w4_scale, torch.float32, "w4_scale")
+    _cuda(w8_scale, torch.float32, "w8_scale")
+    _cuda(bias, torch.bfloat16, "bias")
+    _cuda(out, torch.bfloat16, "out")
+    _check(load().qs_linear_gbs(_p(x), M, K, float(alpha), _p(w4_packed), _p(w4_scale),
+                                _p(w8_packed), _p(w8_scale), _p(bias), N, _p(state),
+                                _p(workspace), workspace_bytes, _p(out), _s(stream)),
+           "qs_linear_gbs")
+
+
 def qs_selftest_timeout(timeout_us: int, stream=None) -> None:
     _check(load().qs_selftest_timeout(timeout_us, _s(stream)), "qs_selftest_timeout")
 
@@ -331,3 +369,51 @@ class QuantLinear:
             self.workspace = torch.empty((max(need, 0),), dtype=torch.uint8, device=x.device)
         return linear(x, self.w_packed, self.w_scale, self.bias, self.bits_x, self.alpha,
                       self.workspace, stream=stream, out=out, bits_w=self.bits)
+
+
+def gbs_state_host(state) -> dict:
+    """Copies the header of a qs_gbs_state to the host (synchronises)."""
+    import struct
+    raw = bytes(state[:32].cpu().numpy().tobytes())
+    acc, last_d, bits, step, blocks_done, _ = struct.unpack("<ddiiII", raw)
+    return {"acc": acc, "last_d": last_d, "bits": bits, "step": step, "blocks_done": blocks_done}
+
+
+class GbsLinear:
+    """A layer under δ-guided bit switching: weights packed at 4 and 8 bits,
+    one device-side state; each call runs the layer at the width the state
+    holds and then measures the change of its output against the previous
+    call's, choosing the next width on the device (no host synchronisation)."""
+
+    def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None, delta: float,
+                 alpha: float = 1.0, stream=None):
+        self.N, self.K = weight.shape
+        self.delta, self.alpha = float(delta), alpha
+        self.w4, self.s4 = pack_weights(weight, 4, stream=stream)
+        self.w8, self.s8 = pack_weights(weight, 8, stream=stream)
+        self.bias = bias
+        self.state = torch.zeros((QS_GBS_STATE_BYTES,), dtype=torch.uint8, device=weight.device)
+        qs_gbs_reset(self.state, stream)
+        self.workspace = None
+        self.prev = None
+        self.buffers = []  # two outputs used in turn when the caller passes none
+
+    def __call__(self, x: torch.Tensor, stream=None, out=None) -> torch.Tensor:
+        M = x.shape[0]
+        need = qs_linear_workspace_bytes(M, self.K, 8)
+        if self.workspace is None or self.workspace.numel() < need:
+            self.workspace = torch.empty((max(need, 0),), dtype=torch.uint8, device=x.device)
+        if out is None:
+            if not self.buffers or self.buffers[0].shape != (M, self.N):
+                self.buffers = [torch.empty((M, self.N), dtype=torch.bfloat16, device=x.device)
+                                for _ in range(2)]
+            self.buffers.reverse()
+            out = self.buffers[0]
+        if self.prev is not None and out.data_ptr() == self.prev.data_ptr():
+            raise ValueError("out must not be the previous step's output")
+        qs_linear_gbs(x, M, self.K, self.alpha, self.w4, self.s4, self.w8, self.s8, self.bias,
+                      self.N, self.state, self.workspace, self.workspace.numel(), out, stream)
+        prev = self.prev if self.prev is not None and self.prev.shape == out.shape else None
+        qs_gbs_update(out, prev, out.numel(), self.delta, self.state, stream)
+        self.prev = out
+        return out

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "qs.h"
+#include "qs_gbs.cuh"
 #include "qs_gemm.cuh"
 #include "qs_host.cuh"
 #include "qs_glue.cuh"
@@ -61,7 +62,7 @@ int64_t packed_row_bytes(int64_t K, int bits) { return K * qs::code_storage_bits
 template <int SA, int SB, bool OUT_S32>
 qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, const float* sw,
                        const void* bias, int64_t M, int64_t N, int64_t K, void* out,
-                       cudaStream_t stream) {
+                       cudaStream_t stream, const int* gate = nullptr, int gate_want = 0) {
   using C = qs::gemm::Cfg<SA, SB>;
   CUtensorMap ta, tb;
   // each CTA of a pair loads 128 rows of x and 128 rows of W per stage; 8-bit
@@ -85,7 +86,7 @@ qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, const fl
   const int grid = static_cast<int>(2 * pairs);
   kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(
       ta, tb, sa, sw, static_cast<const uint16_t*>(bias), out, static_cast<int>(M),
-      static_cast<int>(N), static_cast<int>(K));
+      static_cast<int>(N), static_cast<int>(K), gate, gate_want);
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
@@ -259,6 +260,86 @@ qs_status qs_linear(const void* x_bf16, int64_t M, int64_t K, float alpha, const
                     void* workspace, int64_t workspace_bytes, void* out_bf16, void* stream) {
   return qs_linear_mixed(x_bf16, M, K, alpha, bits, w_packed, w_scale, bits, bias_bf16, N,
                          workspace, workspace_bytes, out_bf16, stream);
+}
+
+qs_status qs_gbs_reset(void* state, void* stream) {
+  if (!state) return QS_ERR_NULL;
+  if (!aligned16(state)) return QS_ERR_ALIGN;
+  QS_TRY(check_device_ptr(state));
+  qs::gbs::gbs_reset_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<qs_gbs_state*>(state));
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status qs_gbs_update(const void* y_cur_bf16, const void* y_prev_bf16, int64_t n, double delta,
+                        void* state, void* stream) {
+  if (!y_cur_bf16 || !state) return QS_ERR_NULL;
+  if (n <= 0) return QS_ERR_SHAPE;
+  if (!(delta >= 0.0 && delta <= 1.7976931348623157e308)) return QS_ERR_RANGE;
+  if (!aligned16(y_cur_bf16) || !aligned16(state) || (y_prev_bf16 && !aligned16(y_prev_bf16)))
+    return QS_ERR_ALIGN;
+  QS_TRY(check_device_ptr(y_cur_bf16));
+  QS_TRY(check_device_ptr(state));
+  if (y_prev_bf16) QS_TRY(check_device_ptr(y_prev_bf16));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  qs_gbs_state* st = static_cast<qs_gbs_state*>(state);
+  if (!y_prev_bf16) {
+    qs::gbs::gbs_first_kernel<<<1, 1, 0, s>>>(delta, st);
+    return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+  }
+  const int sms = qs::sm_count();
+  if (sms <= 0) return QS_ERR_CUDA;
+  // a fixed grid per device and size keeps the summation order fixed
+  const int64_t nvec = n / 8;
+  int64_t blocks = (nvec + qs::gbs::kThreads - 1) / qs::gbs::kThreads;
+  const int64_t cap = static_cast<int64_t>(sms) * 4 < qs::gbs::kMaxBlocks
+                          ? static_cast<int64_t>(sms) * 4
+                          : qs::gbs::kMaxBlocks;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  qs::gbs::gbs_update_kernel<<<static_cast<unsigned>(blocks), qs::gbs::kThreads, 0, s>>>(
+      static_cast<const uint16_t*>(y_cur_bf16), static_cast<const uint16_t*>(y_prev_bf16), n,
+      delta, st);
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status qs_linear_gbs(const void* x_bf16, int64_t M, int64_t K, float alpha,
+                        const void* w4_packed, const float* w4_scale, const void* w8_packed,
+                        const float* w8_scale, const void* bias_bf16, int64_t N,
+                        const void* state, void* workspace, int64_t workspace_bytes,
+                        void* out_bf16, void* stream) {
+  if (!x_bf16 || !w4_packed || !w4_scale || !w8_packed || !w8_scale || !state || !workspace ||
+      !out_bf16)
+    return QS_ERR_NULL;
+  QS_TRY(check_gemm_args(workspace, w4_packed, out_bf16, M, N, K, 4, 4));
+  QS_TRY(check_gemm_args(workspace, w8_packed, out_bf16, M, N, K, 8, 8));
+  if (!(alpha >= kMinAlpha && alpha <= 1.0f)) return QS_ERR_RANGE;
+  const int64_t need = qs_linear_workspace_bytes(M, K, 8);
+  if (need < 0) return QS_ERR_SHAPE;
+  if (workspace_bytes < need) return QS_ERR_RANGE;
+  if (!aligned16(x_bf16) || !aligned16(w4_scale) || !aligned16(w8_scale) || !aligned16(state) ||
+      (bias_bf16 && !aligned16(bias_bf16)))
+    return QS_ERR_ALIGN;
+  for (const void* p : {x_bf16, w4_packed, static_cast<const void*>(w4_scale), w8_packed,
+                        static_cast<const void*>(w8_scale), state,
+                        static_cast<const void*>(workspace), static_cast<const void*>(out_bf16)})
+    QS_TRY(check_device_ptr(p));
+  if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the width word of the state, read by every gated kernel when it starts
+  const int* gate = &static_cast<const qs_gbs_state*>(state)->bits;
+  uint8_t* xp = static_cast<uint8_t*>(workspace);
+  float* xs = reinterpret_cast<float*>(xp + (M * K + 255) / 256 * 256);
+  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+  for (int bits : {4, 8})
+    if (qs::launch_rotate_quant(x, M, static_cast<int>(K), bits, alpha, 1.0f, 1, xp, xs, s, gate,
+                                bits) != cudaSuccess)
+      return QS_ERR_CUDA;
+  const qs_status st4 = launch_qgemm<4, 4, false>(xp, xs, w4_packed, w4_scale, bias_bf16, M, N, K,
+                                                  out_bf16, s, gate, 4);
+  if (st4 != QS_OK) return st4;
+  return launch_qgemm<8, 8, false>(xp, xs, w8_packed, w8_scale, bias_bf16, M, N, K, out_bf16, s,
+                                   gate, 8);
 }
 
 qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream) {

@@ -435,8 +435,12 @@ template <int SA, int SB, bool OUT_S32>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<SA, SB>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const float* __restrict__ sa, const float* __restrict__ sw,
-                 const uint16_t* __restrict__ bias, void* out, int M, int N, int K) {
+                 const uint16_t* __restrict__ bias, void* out, int M, int N, int K,
+                 const int* gate, int gate_want) {
   using C = Cfg<SA, SB>;
+  // a launch gated on a device-side width (δ-GBS) returns unless selected;
+  // both CTAs of a pair read the same word, before any cluster or TMEM step
+  if (gate != nullptr && *gate != gate_want) return;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The padding is identical in both CTAs (same kernel, same static layout),
   // so every shared object has the same offset in the two CTAs of a pair.

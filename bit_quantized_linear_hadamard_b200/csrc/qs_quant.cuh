@@ -167,7 +167,9 @@ template <int BITS, bool SIMD_CLAMP>
 __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
     const __grid_constant__ CUtensorMap tmx, int64_t rows, int K, int nblk, int rpc,
     int64_t num_groups, int stages, float alpha, float scale_mul, int rotate,
-    uint8_t* __restrict__ out, float* __restrict__ scale_out) {
+    uint8_t* __restrict__ out, float* __restrict__ scale_out, const int* gate, int gate_want) {
+  // a launch gated on a device-side width (δ-GBS) returns unless selected
+  if (gate != nullptr && *gate != gate_want) return;
   constexpr int kQmax = code_qmax(BITS);
   constexpr int kOutBytes = 64 * code_storage_bits(BITS) / 8;  // packed bytes per half block
   extern __shared__ __align__(1024) uint8_t qsmem_raw[];
@@ -364,7 +366,9 @@ __global__ void __launch_bounds__(MAXT) rotate_quant_group_kernel(const uint16_t
                                                                   int K, float alpha,
                                                                   float scale_mul, int rotate,
                                                                   uint8_t* __restrict__ out,
-                                                                  float* __restrict__ scale_out) {
+                                                                  float* __restrict__ scale_out,
+                                                                  const int* gate, int gate_want) {
+  if (gate != nullptr && *gate != gate_want) return;
   constexpr int kQmax = code_qmax(BITS);
   __shared__ float warp_max[32];
 
@@ -482,9 +486,12 @@ inline int choose_rows_per_cta(int nblk) {
 }
 
 template <int BITS>
+// gate / gate_want: when gate is not null the kernels return at once unless
+// *gate == gate_want (read on the device when they start).
 inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int K, float alpha,
                                             float scale_mul, int rotate, uint8_t* out,
-                                            float* scale, cudaStream_t stream) {
+                                            float* scale, cudaStream_t stream,
+                                            const int* gate = nullptr, int gate_want = 0) {
   const int nblk = K / 128;
   const int rpc = nblk <= 128 ? choose_rows_per_cta(nblk) : 0;
   const int64_t groups = rpc ? (rows + rpc - 1) / rpc : 0;
@@ -516,7 +523,8 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
     int64_t grid = static_cast<int64_t>(sms) * per_sm;
     if (grid > groups) grid = groups;
     kern<<<static_cast<unsigned>(grid), threads, smem, stream>>>(
-        tmx, rows, K, nblk, rpc, groups, stages, alpha, scale_mul, rotate, out, scale);
+        tmx, rows, K, nblk, rpc, groups, stages, alpha, scale_mul, rotate, out, scale, gate,
+        gate_want);
     return cudaGetLastError();
   }
   // Rows up to 2048 groups run with at most 256 threads so each thread keeps
@@ -530,10 +538,12 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
   case GG:                                                                                  \
     if (wide)                                                                               \
       rotate_quant_group_kernel<GG, BITS, 1024>                                             \
-          <<<grid, block, 0, stream>>>(x, K, alpha, scale_mul, rotate, out, scale);         \
+          <<<grid, block, 0, stream>>>(x, K, alpha, scale_mul, rotate, out, scale, gate,     \
+                                       gate_want);                                          \
     else                                                                                    \
       rotate_quant_group_kernel<GG, BITS, 256>                                              \
-          <<<grid, block, 0, stream>>>(x, K, alpha, scale_mul, rotate, out, scale);         \
+          <<<grid, block, 0, stream>>>(x, K, alpha, scale_mul, rotate, out, scale, gate,     \
+                                       gate_want);                                          \
     break;
   switch (G) {
     QS_QUANT_CASE(1)
@@ -553,14 +563,18 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
 
 inline cudaError_t launch_rotate_quant(const uint16_t* x, int64_t rows, int K, int bits, float alpha,
                                        float scale_mul, int rotate, uint8_t* out, float* scale,
-                                       cudaStream_t stream) {
+                                       cudaStream_t stream, const int* gate = nullptr,
+                                       int gate_want = 0) {
   switch (bits) {
     case 4:
-      return launch_rotate_quant_bits<4>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream);
+      return launch_rotate_quant_bits<4>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream,
+                                           gate, gate_want);
     case 6:
-      return launch_rotate_quant_bits<6>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream);
+      return launch_rotate_quant_bits<6>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream,
+                                           gate, gate_want);
     case 8:
-      return launch_rotate_quant_bits<8>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream);
+      return launch_rotate_quant_bits<8>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream,
+                                           gate, gate_want);
     default:
       return cudaErrorInvalidValue;
   }

@@ -188,6 +188,69 @@ QS_API qs_status qs_linear_mixed(const void* x_bf16, int64_t M, int64_t K, float
                                  int64_t workspace_bytes, void* out_bf16, void* stream);
 
 /*
+ * δ-guided bit switching (DVD-Quant "Resumen técnico" §2.C): per layer, the
+ * normalised L1 change between consecutive outputs is accumulated, and the
+ * layer's next step runs at 4 bits while the accumulated change is below
+ * delta, otherwise at 8 bits with the accumulator reset.  The state lives in
+ * caller-owned device memory and is read and written only by the library's
+ * kernels, so choosing the width needs no host synchronisation.  Readings:
+ * d = sum|y_cur - y_prev| / sum|y_prev| over all elements (binary64 terms and
+ * sums; a zero denominator gives 0 if the outputs are equal, else +inf);
+ * "below delta" is strict; the first step runs at 8 bits.
+ *
+ * qs_gbs_state — layout of the state (copy it to the host to inspect it).
+ *   acc     accumulated change since the last switch to 8 bits
+ *   last_d  distance measured by the last update (-1 after a reset or a first step)
+ *   bits    width of the layer's next step: 4 or 8
+ *   step    updates since the reset
+ *   blocks_done, partial: scratch of the update kernel (must stay as the
+ *           library leaves it: zero between calls)
+ */
+#define QS_GBS_MAX_BLOCKS 1024
+typedef struct {
+  double acc;
+  double last_d;
+  int32_t bits;
+  int32_t step;
+  uint32_t blocks_done;
+  uint32_t reserved_;
+  double partial[2][QS_GBS_MAX_BLOCKS];
+} qs_gbs_state;
+
+/* qs_gbs_reset — enqueues: acc = 0, last_d = -1, bits = 8, step = 0.
+ *   state  device pointer to a qs_gbs_state, 16-byte aligned */
+QS_API qs_status qs_gbs_reset(void* state, void* stream);
+
+/*
+ * qs_gbs_update — after a step of the layer: measures the change between its
+ * output and the previous step's and decides the next step's width.
+ *   y_cur_bf16   this step's output, n bf16 values
+ *   y_prev_bf16  the previous step's output (same n), or NULL after the first
+ *                step (no distance; only the step count advances)
+ *   delta        threshold, finite and >= 0
+ *   state        as for qs_gbs_reset; updates on one state must not overlap
+ */
+QS_API qs_status qs_gbs_update(const void* y_cur_bf16, const void* y_prev_bf16, int64_t n,
+                               double delta, void* state, void* stream);
+
+/*
+ * qs_linear_gbs — the one-call layer (as qs_linear) at the width the state
+ * holds: the 4-bit and the 8-bit kernels are both enqueued and each returns at
+ * once unless the state selects its width.  Weights are prepared at both
+ * widths (qs_pack_weights with bits 4 and 8).
+ *   w4_packed, w4_scale  weights at 4 bits; w8_packed, w8_scale  at 8 bits
+ *   state                a qs_gbs_state (read only)
+ *   workspace            at least qs_linear_workspace_bytes(M, K, 8) bytes
+ *   other arguments as qs_linear
+ */
+QS_API qs_status qs_linear_gbs(const void* x_bf16, int64_t M, int64_t K, float alpha,
+                               const void* w4_packed, const float* w4_scale,
+                               const void* w8_packed, const float* w8_scale,
+                               const void* bias_bf16, int64_t N, const void* state,
+                               void* workspace, int64_t workspace_bytes, void* out_bf16,
+                               void* stream);
+
+/*
  * qs_gelu_bf16 — elementwise GELU (exact erf form, binary32 arithmetic,
  * bf16 in and out) used between the ffn-up and ffn-down linears of a
  * transformer block chain.  n elements; x and y may alias.

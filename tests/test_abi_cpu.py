@@ -164,3 +164,48 @@ def test_linear_validation_and_workspace(lib):
 def test_selftest_timeout_validation(lib):
     assert lib.qs_selftest_timeout(0, NUL) == RANGE
     assert lib.qs_selftest_timeout(1000001, NUL) == RANGE
+
+
+def test_gbs_validation(lib):
+    assert lib.qs_gbs_reset(NUL, NUL) == NULL
+    assert lib.qs_gbs_reset(MIS, NUL) == ALIGN
+    up = lib.qs_gbs_update
+    assert up(NUL, B, 64, 0.5, C, NUL) == NULL
+    assert up(A, B, 64, 0.5, NUL, NUL) == NULL
+    assert up(A, B, 0, 0.5, C, NUL) == SHAPE
+    for delta in (-0.5, float("nan"), float("inf")):
+        assert up(A, B, 64, delta, C, NUL) == RANGE, delta
+    assert up(A, MIS, 64, 0.5, C, NUL) == ALIGN
+    assert up(A, B, 64, 0.5, ctypes.c_void_p(0x30008), NUL) == ALIGN
+    f = lib.qs_linear_gbs
+    need = lib.qs_linear_workspace_bytes(8, 128, 8)
+    args = [A, 8, 128, 1.0, B, C, B, C, NUL, 256, D, A, need, A, NUL]
+    bad = list(args); bad[6] = NUL
+    assert f(*bad) == NULL                                  # no 8-bit weights
+    bad = list(args); bad[9] = 250
+    assert f(*bad) == SHAPE
+    bad = list(args); bad[12] = need - 1
+    assert f(*bad) == RANGE                                 # workspace sized for 8 bits
+    bad = list(args); bad[10] = ctypes.c_void_p(0x40008)
+    assert f(*bad) == ALIGN                                 # state
+    assert f(*args) == PTR                                  # fake addresses
+
+
+def test_gbs_state_layout_matches_the_header(tmp_path):
+    """sizeof and offsets of qs_gbs_state as a C compiler lays it out."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stddef.h>\n#include <stdio.h>\n#include "qs.h"\n'
+        'int main(void) { printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(qs_gbs_state), '
+        'offsetof(qs_gbs_state, acc), offsetof(qs_gbs_state, last_d), '
+        'offsetof(qs_gbs_state, bits), offsetof(qs_gbs_state, step), '
+        'offsetof(qs_gbs_state, partial)); return 0; }\n')
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert [int(v) for v in out] == [binding.QS_GBS_STATE_BYTES, 0, 8, 16, 20, 32]
