@@ -327,6 +327,51 @@ def gbs_sequence(qs, torch, I, dev, stream, steps=8, delta=0.3):
             "update_bytes": 4 * n}
 
 
+def bgr_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
+    """The Wan FFN layer with weights on BGR grids (asymmetric, per channel):
+    offline pack time, per-step times of the activation kernel (with code sums)
+    and the asymmetric GEMM, and the output error against the symmetric weights
+    on the first `rows` tokens."""
+    cfg = I.WAN_FFN
+    d = I.make_layer(cfg)
+    M, K, N, bits, alpha = cfg.M, cfg.K, cfg.N, cfg.bits, cfg.alpha
+    with torch.cuda.stream(stream):
+        x, w, b = d["x"].to(dev), d["w"].to(dev), d["bias"].to(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        wp, ws, wo = qs.pack_weights_bgr(w, bits, 64, 8, stream=stream)
+        e1.record(stream)
+        stream.synchronize()
+        pack_ms = e0.elapsed_time(e1)
+        xp = torch.empty((M, qs.packed_cols(K, bits)), dtype=torch.uint8, device=dev)
+        xs = torch.empty((M,), dtype=torch.float32, device=dev)
+        xr = torch.empty((M,), dtype=torch.int32, device=dev)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        for _ in range(warmup):
+            qs.qs_quant_act_rowsum(x, M, K, bits, alpha, 0, xp, xs, xr, stream)
+            qs.qs_qlinear_asym(xp, xs, xr, wp, ws, wo, b, M, N, K, bits, out, stream)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for e in ev:
+            e[0].record(stream)
+            qs.qs_quant_act_rowsum(x, M, K, bits, alpha, 0, xp, xs, xr, stream)
+            e[1].record(stream)
+            qs.qs_qlinear_asym(xp, xs, xr, wp, ws, wo, b, M, N, K, bits, out, stream)
+            e[2].record(stream)
+        stream.synchronize()
+        q = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+        g = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+        ref = x[:rows].double() @ w.double().t() + b.double()
+        wsp, wss = qs.pack_weights(w, bits, stream=stream)
+        ysym = qs.qlinear(xp[:rows], xs[:rows], wsp, wss, b, bits, K, stream=stream).double()
+        stream.synchronize()
+    err = lambda y: float((y - ref).norm() / ref.norm())  # noqa: E731
+    return {"workload": cfg.name + "_bgr", "candidates": 64, "iterations": 8,
+            "pack_ms": pack_ms, "quant_rowsum_ms": q, "gemm_asym_ms": g,
+            "TOPS": cfg.ops / ((q + g) * 1e-3) / 1e12, "gemm_TOPS": cfg.ops / (g * 1e-3) / 1e12,
+            "rel_err_bgr": err(out[:rows].double()), "rel_err_symmetric": err(ysym),
+            "error_rows": rows}
+
+
 def quality(qs, torch, x, w, bias, bits, alpha, stream, rows=256):
     """Relative Frobenius error and SQNR of the layer against the unquantised
     binary64 product, with and without the Hadamard rotation (first `rows` tokens)."""
@@ -496,6 +541,7 @@ def main():
             extra["quality"] = quality(qs, torch, x, d["w"].to(dev), bias, bits, alpha, stream)
         extra["configs"] = all_configs(qs, torch, I, dev, stream)
         extra["gbs"] = gbs_sequence(qs, torch, I, dev, stream)
+        extra["bgr"] = bgr_layer(qs, torch, I, dev, stream)
     if rank == 0:
         pk, src = peaks()
         int8_peak = pk["bf16_tflops"] * INT8_PER_BF16

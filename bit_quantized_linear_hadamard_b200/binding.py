@@ -28,9 +28,10 @@ STATUS = {0: "QS_OK", 1: "QS_ERR_NULL", 2: "QS_ERR_SHAPE", 3: "QS_ERR_BITS", 4: 
           5: "QS_ERR_RANGE", 6: "QS_ERR_CUDA", 7: "QS_ERR_TIMEOUT", 8: "QS_ERR_PTR"}
 EXPORTS = ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qlinear_mixed", "qs_qgemm_s32",
            "qs_qgemm_s32_mixed", "qs_gelu_bf16", "qs_linear_workspace_bytes", "qs_linear",
-           "qs_linear_mixed", "qs_linear_noalloc", "qs_gbs_reset", "qs_gbs_update",
-           "qs_linear_gbs", "qs_selftest_timeout", "qs_device_error", "qs_status_str",
-           "qs_version")
+           "qs_linear_mixed", "qs_linear_noalloc", "qs_pack_weights_bgr", "qs_quant_act_rowsum",
+           "qs_qlinear_asym", "qs_qgemm_s32_asym", "qs_linear_bgr_workspace_bytes",
+           "qs_linear_bgr", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
+           "qs_selftest_timeout", "qs_device_error", "qs_status_str", "qs_version")
 BITS = (4, 6, 8)
 QS_GBS_MAX_BLOCKS = 1024
 # sizeof(qs_gbs_state): acc, last_d (f64), bits, step, blocks_done, reserved (i32), partials
@@ -70,6 +71,13 @@ def load() -> ctypes.CDLL:
     L.qs_linear_mixed.argtypes = [vp, i64, i64, f32, i32, vp, vp, i32, vp, i64, vp, i64, vp, vp]
     L.qs_linear_noalloc.argtypes = [vp, i64, i64, f32, vp, vp, vp, i64, i32, vp, vp]
     f64 = ctypes.c_double
+    L.qs_pack_weights_bgr.argtypes = [vp, i64, i64, i32, u32, i32, i32, vp, vp, vp, vp]
+    L.qs_quant_act_rowsum.argtypes = [vp, i64, i64, i32, f32, u32, vp, vp, vp, vp]
+    L.qs_qlinear_asym.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, vp, vp]
+    L.qs_qgemm_s32_asym.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp]
+    L.qs_linear_bgr_workspace_bytes.argtypes = [i64, i64, i32]
+    L.qs_linear_bgr_workspace_bytes.restype = i64
+    L.qs_linear_bgr.argtypes = [vp, i64, i64, f32, vp, vp, vp, vp, i64, i32, vp, i64, vp, vp]
     L.qs_gbs_reset.argtypes = [vp, vp]
     L.qs_gbs_update.argtypes = [vp, vp, i64, f64, vp, vp]
     L.qs_linear_gbs.argtypes = [vp, i64, i64, f32, vp, vp, vp, vp, vp, i64, vp, vp, i64, vp, vp]
@@ -80,8 +88,10 @@ def load() -> ctypes.CDLL:
     L.qs_version.restype = ctypes.c_char_p
     for name in ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qlinear_mixed",
                  "qs_qgemm_s32", "qs_qgemm_s32_mixed", "qs_gelu_bf16", "qs_linear",
-                 "qs_linear_mixed", "qs_linear_noalloc", "qs_gbs_reset", "qs_gbs_update",
-                 "qs_linear_gbs", "qs_selftest_timeout", "qs_device_error"):
+                 "qs_linear_mixed", "qs_linear_noalloc", "qs_pack_weights_bgr",
+                 "qs_quant_act_rowsum", "qs_qlinear_asym", "qs_qgemm_s32_asym", "qs_linear_bgr",
+                 "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs", "qs_selftest_timeout",
+                 "qs_device_error"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -225,6 +235,64 @@ def qs_linear_noalloc(x, M, K, alpha, w_packed, w_scale, bias, N, bits, out, str
                                     N, bits, _p(out), _s(stream)), "qs_linear_noalloc")
 
 
+def qs_pack_weights_bgr(w, N, K, bits, flags, candidates, iterations, w_packed, w_scale,
+                        w_offset, stream=None):
+    _cuda(w, torch.bfloat16, "w")
+    _cuda(w_packed, torch.uint8, "w_packed")
+    _cuda(w_scale, torch.float32, "w_scale")
+    _cuda(w_offset, torch.int32, "w_offset")
+    _check(load().qs_pack_weights_bgr(_p(w), N, K, bits, flags, candidates, iterations,
+                                      _p(w_packed), _p(w_scale), _p(w_offset), _s(stream)),
+           "qs_pack_weights_bgr")
+
+
+def qs_quant_act_rowsum(x, M, K, bits, alpha, flags, x_packed, x_scale, x_rowsum, stream=None):
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(x_packed, torch.uint8, "x_packed")
+    _cuda(x_scale, torch.float32, "x_scale")
+    _cuda(x_rowsum, torch.int32, "x_rowsum")
+    _check(load().qs_quant_act_rowsum(_p(x), M, K, bits, float(alpha), flags, _p(x_packed),
+                                      _p(x_scale), _p(x_rowsum), _s(stream)),
+           "qs_quant_act_rowsum")
+
+
+def qs_qlinear_asym(x_packed, x_scale, x_rowsum, w_packed, w_scale, w_offset, bias, M, N, K,
+                    bits, out, stream=None):
+    for t, name, dt in ((x_packed, "x_packed", torch.uint8), (w_packed, "w_packed", torch.uint8),
+                        (x_scale, "x_scale", torch.float32), (w_scale, "w_scale", torch.float32),
+                        (x_rowsum, "x_rowsum", torch.int32), (w_offset, "w_offset", torch.int32),
+                        (bias, "bias", torch.bfloat16), (out, "out", torch.bfloat16)):
+        _cuda(t, dt, name)
+    _check(load().qs_qlinear_asym(_p(x_packed), _p(x_scale), _p(x_rowsum), _p(w_packed),
+                                  _p(w_scale), _p(w_offset), _p(bias), M, N, K, bits, _p(out),
+                                  _s(stream)), "qs_qlinear_asym")
+
+
+def qs_qgemm_s32_asym(x_packed, x_rowsum, w_packed, w_offset, M, N, K, bits, acc, stream=None):
+    for t, name, dt in ((x_packed, "x_packed", torch.uint8), (w_packed, "w_packed", torch.uint8),
+                        (x_rowsum, "x_rowsum", torch.int32), (w_offset, "w_offset", torch.int32),
+                        (acc, "acc", torch.int32)):
+        _cuda(t, dt, name)
+    _check(load().qs_qgemm_s32_asym(_p(x_packed), _p(x_rowsum), _p(w_packed), _p(w_offset), M, N,
+                                    K, bits, _p(acc), _s(stream)), "qs_qgemm_s32_asym")
+
+
+def qs_linear_bgr_workspace_bytes(M, K, bits) -> int:
+    return int(load().qs_linear_bgr_workspace_bytes(M, K, bits))
+
+
+def qs_linear_bgr(x, M, K, alpha, w_packed, w_scale, w_offset, bias, N, bits, workspace,
+                  workspace_bytes, out, stream=None):
+    for t, name, dt in ((x, "x", torch.bfloat16), (w_packed, "w_packed", torch.uint8),
+                        (w_scale, "w_scale", torch.float32), (w_offset, "w_offset", torch.int32),
+                        (bias, "bias", torch.bfloat16), (workspace, "workspace", torch.uint8),
+                        (out, "out", torch.bfloat16)):
+        _cuda(t, dt, name)
+    _check(load().qs_linear_bgr(_p(x), M, K, float(alpha), _p(w_packed), _p(w_scale),
+                                _p(w_offset), _p(bias), N, bits, _p(workspace), workspace_bytes,
+                                _p(out), _s(stream)), "qs_linear_bgr")
+
+
 def qs_gbs_reset(state, stream=None):
     _cuda(state, torch.uint8, "state")
     _check(load().qs_gbs_reset(_p(state), _s(stream)), "qs_gbs_reset")
@@ -280,6 +348,28 @@ def pack_weights(w: torch.Tensor, bits: int, flags: int = 0, stream=None):
     ws = torch.empty((N,), dtype=torch.float32, device=w.device)
     qs_pack_weights(w, N, K, bits, flags, wp, ws, stream)
     return wp, ws
+
+
+def pack_weights_bgr(w: torch.Tensor, bits: int, candidates: int = 64, iterations: int = 8,
+                     flags: int = 0, stream=None):
+    """w bf16 [N, K] -> (signed codes on BGR grids, scales float32 [N], offsets int32 [N])."""
+    N, K = w.shape
+    wp = torch.empty((N, packed_cols(K, bits)), dtype=torch.uint8, device=w.device)
+    ws = torch.empty((N,), dtype=torch.float32, device=w.device)
+    wo = torch.empty((N,), dtype=torch.int32, device=w.device)
+    qs_pack_weights_bgr(w, N, K, bits, flags, candidates, iterations, wp, ws, wo, stream)
+    return wp, ws, wo
+
+
+def quant_act_rowsum(x: torch.Tensor, bits: int, alpha: float = 1.0, flags: int = 0,
+                     stream=None):
+    """x bf16 [M, K] -> (packed codes, scales, per-token code sums int32 [M])."""
+    M, K = x.shape
+    xp = torch.empty((M, packed_cols(K, bits)), dtype=torch.uint8, device=x.device)
+    xs = torch.empty((M,), dtype=torch.float32, device=x.device)
+    xr = torch.empty((M,), dtype=torch.int32, device=x.device)
+    qs_quant_act_rowsum(x, M, K, bits, alpha, flags, xp, xs, xr, stream)
+    return xp, xs, xr
 
 
 def quant_act(x: torch.Tensor, bits: int, alpha: float = 1.0, flags: int = 0, stream=None,

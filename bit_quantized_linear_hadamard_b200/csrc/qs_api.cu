@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "qs.h"
+#include "qs_bgr.cuh"
 #include "qs_gbs.cuh"
 #include "qs_gemm.cuh"
 #include "qs_host.cuh"
@@ -58,11 +59,13 @@ int64_t packed_row_bytes(int64_t K, int bits) { return K * qs::code_storage_bits
     if (_s != QS_OK) return _s;    \
   } while (0)
 
-// SA, SB: storage bits (4 or 8) of the x and W codes.
-template <int SA, int SB, bool OUT_S32>
+// SA, SB: storage bits (4 or 8) of the x and W codes.  ASYM: weights on an
+// asymmetric grid (per-token code sums `rowsum`, per-channel `offset`).
+template <int SA, int SB, bool OUT_S32, bool ASYM = false>
 qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, const float* sw,
                        const void* bias, int64_t M, int64_t N, int64_t K, void* out,
-                       cudaStream_t stream, const int* gate = nullptr, int gate_want = 0) {
+                       cudaStream_t stream, const int* gate = nullptr, int gate_want = 0,
+                       const int* rowsum = nullptr, const int* offset = nullptr) {
   using C = qs::gemm::Cfg<SA, SB>;
   CUtensorMap ta, tb;
   // each CTA of a pair loads 128 rows of x and 128 rows of W per stage; 8-bit
@@ -72,7 +75,7 @@ qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, const fl
       !qs::make_tensor_map_2d(&tb, wp, static_cast<uint64_t>(K) * SB / 8, static_cast<uint64_t>(N),
                               qs::gemm::BK * SB / 8, qs::gemm::HN, SB == 8))
     return QS_ERR_CUDA;
-  auto kern = qs::gemm::qgemm_kernel<SA, SB, OUT_S32>;
+  auto kern = qs::gemm::qgemm_kernel<SA, SB, OUT_S32, ASYM>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
       cudaSuccess)
     return QS_ERR_CUDA;
@@ -86,7 +89,7 @@ qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, const fl
   const int grid = static_cast<int>(2 * pairs);
   kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(
       ta, tb, sa, sw, static_cast<const uint16_t*>(bias), out, static_cast<int>(M),
-      static_cast<int>(N), static_cast<int>(K), gate, gate_want);
+      static_cast<int>(N), static_cast<int>(K), gate, gate_want, rowsum, offset);
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
@@ -340,6 +343,135 @@ qs_status qs_linear_gbs(const void* x_bf16, int64_t M, int64_t K, float alpha,
   if (st4 != QS_OK) return st4;
   return launch_qgemm<8, 8, false>(xp, xs, w8_packed, w8_scale, bias_bf16, M, N, K, out_bf16, s,
                                    gate, 8);
+}
+
+qs_status qs_pack_weights_bgr(const void* w_bf16, int64_t N, int64_t K, int bits, unsigned flags,
+                              int candidates, int iterations, void* w_packed, float* w_scale,
+                              int32_t* w_offset, void* stream) {
+  if (!w_bf16 || !w_packed || !w_scale || !w_offset) return QS_ERR_NULL;
+  if (bits != 4 && bits != 8) return QS_ERR_BITS;
+  QS_TRY(check_rows_k(N, K));
+  if (K > qs::bgr::kMaxK || candidates < 1 || candidates > qs::bgr::kMaxCandidates ||
+      iterations < 0 || iterations > 64 || (flags & ~kKnownFlags))
+    return QS_ERR_RANGE;
+  if (N > INT32_MAX) return QS_ERR_RANGE;
+  if (!aligned16(w_bf16) || !aligned16(w_packed) || !aligned16(w_scale) || !aligned16(w_offset))
+    return QS_ERR_ALIGN;
+  QS_TRY(check_device_ptr(w_bf16));
+  QS_TRY(check_device_ptr(w_packed));
+  QS_TRY(check_device_ptr(w_scale));
+  QS_TRY(check_device_ptr(w_offset));
+  const bool rotate = !(flags & QS_FLAG_NO_ROTATE);
+  const int smem = static_cast<int>(K) * 4;
+  auto kern = bits == 4 ? qs::bgr::bgr_pack_kernel<4> : qs::bgr::bgr_pack_kernel<8>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return QS_ERR_CUDA;
+  kern<<<static_cast<unsigned>(N), qs::bgr::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(w_bf16), static_cast<int>(K), rotate ? 1 : 0, candidates,
+      iterations, rotate ? 0.0078125f : 1.0f, static_cast<uint8_t*>(w_packed), w_scale, w_offset);
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status qs_quant_act_rowsum(const void* x_bf16, int64_t M, int64_t K, int bits, float alpha,
+                              unsigned flags, void* x_packed, float* x_scale, int32_t* x_rowsum,
+                              void* stream) {
+  if (!x_rowsum) return QS_ERR_NULL;
+  if (!aligned16(x_rowsum)) return QS_ERR_ALIGN;
+  if (!x_bf16 || !x_packed || !x_scale) return QS_ERR_NULL;
+  QS_TRY(check_bits(bits));
+  QS_TRY(check_rows_k(M, K));
+  if (!(alpha >= kMinAlpha && alpha <= 1.0f)) return QS_ERR_RANGE;
+  if (flags & ~kKnownFlags) return QS_ERR_RANGE;
+  if (!aligned16(x_bf16) || !aligned16(x_packed) || !aligned16(x_scale)) return QS_ERR_ALIGN;
+  for (const void* p : {x_bf16, static_cast<const void*>(x_packed),
+                        static_cast<const void*>(x_scale), static_cast<const void*>(x_rowsum)})
+    QS_TRY(check_device_ptr(p));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(x_rowsum, 0, static_cast<size_t>(M) * 4, s) != cudaSuccess)
+    return QS_ERR_CUDA;
+  const bool rotate = !(flags & QS_FLAG_NO_ROTATE);
+  const cudaError_t e = qs::launch_rotate_quant(
+      static_cast<const uint16_t*>(x_bf16), M, static_cast<int>(K), bits, alpha, 1.0f,
+      rotate ? 1 : 0, static_cast<uint8_t*>(x_packed), x_scale, s, nullptr, 0, x_rowsum);
+  return e == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status qs_qlinear_asym(const void* x_packed, const float* x_scale, const int32_t* x_rowsum,
+                          const void* w_packed, const float* w_scale, const int32_t* w_offset,
+                          const void* bias_bf16, int64_t M, int64_t N, int64_t K, int bits,
+                          void* out_bf16, void* stream) {
+  if (bits != 4 && bits != 8) return QS_ERR_BITS;
+  QS_TRY(check_gemm_args(x_packed, w_packed, out_bf16, M, N, K, bits, bits));
+  if (!x_scale || !w_scale || !x_rowsum || !w_offset) return QS_ERR_NULL;
+  if (!aligned16(x_scale) || !aligned16(w_scale) || !aligned16(x_rowsum) ||
+      !aligned16(w_offset) || (bias_bf16 && !aligned16(bias_bf16)))
+    return QS_ERR_ALIGN;
+  for (const void* p : {x_packed, static_cast<const void*>(x_scale),
+                        static_cast<const void*>(x_rowsum), w_packed,
+                        static_cast<const void*>(w_scale), static_cast<const void*>(w_offset),
+                        static_cast<const void*>(out_bf16)})
+    QS_TRY(check_device_ptr(p));
+  if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return bits == 4 ? launch_qgemm<4, 4, false, true>(x_packed, x_scale, w_packed, w_scale,
+                                                      bias_bf16, M, N, K, out_bf16, s, nullptr, 0,
+                                                      x_rowsum, w_offset)
+                   : launch_qgemm<8, 8, false, true>(x_packed, x_scale, w_packed, w_scale,
+                                                      bias_bf16, M, N, K, out_bf16, s, nullptr, 0,
+                                                      x_rowsum, w_offset);
+}
+
+qs_status qs_qgemm_s32_asym(const void* x_packed, const int32_t* x_rowsum, const void* w_packed,
+                            const int32_t* w_offset, int64_t M, int64_t N, int64_t K, int bits,
+                            int32_t* acc, void* stream) {
+  if (bits != 4 && bits != 8) return QS_ERR_BITS;
+  QS_TRY(check_gemm_args(x_packed, w_packed, acc, M, N, K, bits, bits));
+  if (!x_rowsum || !w_offset) return QS_ERR_NULL;
+  if (!aligned16(x_rowsum) || !aligned16(w_offset)) return QS_ERR_ALIGN;
+  for (const void* p : {x_packed, static_cast<const void*>(x_rowsum), w_packed,
+                        static_cast<const void*>(w_offset), static_cast<const void*>(acc)})
+    QS_TRY(check_device_ptr(p));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return bits == 4 ? launch_qgemm<4, 4, true, true>(x_packed, nullptr, w_packed, nullptr, nullptr,
+                                                     M, N, K, acc, s, nullptr, 0, x_rowsum,
+                                                     w_offset)
+                   : launch_qgemm<8, 8, true, true>(x_packed, nullptr, w_packed, nullptr, nullptr,
+                                                     M, N, K, acc, s, nullptr, 0, x_rowsum,
+                                                     w_offset);
+}
+
+int64_t qs_linear_bgr_workspace_bytes(int64_t M, int64_t K, int bits) {
+  if ((bits != 4 && bits != 8) || check_rows_k(M, K) != QS_OK) return -1;
+  return (M * packed_row_bytes(K, bits) + 255) / 256 * 256 + (4 * M + 255) / 256 * 256 + 4 * M;
+}
+
+qs_status qs_linear_bgr(const void* x_bf16, int64_t M, int64_t K, float alpha,
+                        const void* w_packed, const float* w_scale, const int32_t* w_offset,
+                        const void* bias_bf16, int64_t N, int bits, void* workspace,
+                        int64_t workspace_bytes, void* out_bf16, void* stream) {
+  if (!x_bf16 || !w_packed || !w_scale || !w_offset || !workspace || !out_bf16)
+    return QS_ERR_NULL;
+  if (bits != 4 && bits != 8) return QS_ERR_BITS;
+  QS_TRY(check_gemm_args(workspace, w_packed, out_bf16, M, N, K, bits, bits));
+  if (!(alpha >= kMinAlpha && alpha <= 1.0f)) return QS_ERR_RANGE;
+  const int64_t need = qs_linear_bgr_workspace_bytes(M, K, bits);
+  if (need < 0) return QS_ERR_SHAPE;
+  if (workspace_bytes < need) return QS_ERR_RANGE;
+  if (!aligned16(x_bf16) || !aligned16(w_scale) || !aligned16(w_offset) ||
+      (bias_bf16 && !aligned16(bias_bf16)))
+    return QS_ERR_ALIGN;
+  for (const void* p : {x_bf16, w_packed, static_cast<const void*>(w_scale),
+                        static_cast<const void*>(w_offset), static_cast<const void*>(workspace),
+                        static_cast<const void*>(out_bf16)})
+    QS_TRY(check_device_ptr(p));
+  if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
+  uint8_t* xp = static_cast<uint8_t*>(workspace);
+  float* xs = reinterpret_cast<float*>(xp + (M * packed_row_bytes(K, bits) + 255) / 256 * 256);
+  int32_t* xr = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(xs) + (4 * M + 255) / 256 * 256);
+  QS_TRY(qs_quant_act_rowsum(x_bf16, M, K, bits, alpha, 0u, xp, xs, xr, stream));
+  return qs_qlinear_asym(xp, xs, xr, w_packed, w_scale, w_offset, bias_bf16, M, N, K, bits,
+                         out_bf16, stream);
 }
 
 qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream) {

@@ -107,8 +107,9 @@ struct Cfg {
   static constexpr int kOffPk = kOffOp + kOpStages * kOpStage;
   static constexpr int kOffBar = kOffPk + kPkStages * kPkStage;
   static constexpr int kNumBars = 2 * kPkStages + 3 * kOpStages + 4;
-  static constexpr int kOffEpi = (kOffBar + 8 * kNumBars + 15) / 16 * 16;  // s_w, bias of a tile
-  static constexpr int kOffMisc = kOffEpi + 2 * BN * 4;  // TMEM address, abort flag
+  // s_w, bias and (asymmetric weights) channel offsets of a tile
+  static constexpr int kOffEpi = (kOffBar + 8 * kNumBars + 15) / 16 * 16;
+  static constexpr int kOffMisc = kOffEpi + 3 * BN * 4;  // TMEM address, abort flag
   static constexpr int kOffSignal = kOffMisc + 16;        // 16 bytes per operand stage
   static constexpr int kSmemBytes = kOffSignal + 16 * kOpStages + 1024;  // + alignment slack
   static constexpr int kUnpackThreads = kPacked ? 32 * kUnpackWarps : 1;
@@ -327,15 +328,20 @@ __device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
 }
 
 // Converts one 32-column chunk of accumulators (one row per thread) and stores it.
-template <int SHIFT, bool OUT_S32>
+// ASYM (weights on an asymmetric grid, signed codes s = q - 2^(b-1)): the
+// exact accumulator is sum q_a s + o[n] * sum_k q_a[m,k].
+template <int SHIFT, bool OUT_S32, bool ASYM>
 __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row, bool row_ok,
                                                int n, int N, float s_a, const float* epi_sw,
-                                               const float* epi_b, void* out) {
+                                               const float* epi_b, const int* epi_off,
+                                               int rsum, void* out) {
   if (n >= N || !row_ok) return;
   int32_t acc[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i)
+  for (int i = 0; i < 32; ++i) {
     acc[i] = static_cast<int32_t>(r[i]) >> SHIFT;
+    if (ASYM) acc[i] += epi_off[i] * rsum;
+  }
   if (OUT_S32) {
     int32_t* dst = static_cast<int32_t*>(out) + static_cast<int64_t>(row) * N + n;
 #pragma unroll
@@ -372,13 +378,15 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row,
   }
 }
 
-template <int SHIFT, bool OUT_S32>
+template <int SHIFT, bool OUT_S32, bool ASYM>
 __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
                                               uint32_t tmem_base, int quad, int lane, int et,
                                               const float* __restrict__ sa,
                                               const float* __restrict__ sw,
-                                              const uint16_t* __restrict__ bias, void* out,
-                                              float* epi_sw, float* epi_b,
+                                              const uint16_t* __restrict__ bias,
+                                              const int* __restrict__ rowsum,
+                                              const int* __restrict__ offset, void* out,
+                                              float* epi_sw, float* epi_b, int* epi_off,
                                               volatile int* abort_flag) {
   int it = 0;
   for (int t = pb.pair; t < pb.num_tiles; t += pb.num_pairs, ++it) {
@@ -386,20 +394,24 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
     const uint32_t aph = (it >> 1) & 1;
     int m0, n0;
     pb.tile_origin(t, m0, n0);
-    if (!OUT_S32) {
-      // Stage the tile's channel scales and bias while its main loop runs.
+    if (!OUT_S32 || ASYM) {
+      // Stage the tile's channel scales, bias and offsets while its main loop runs.
       epi_bar_sync();  // every epilogue warp is done with the previous tile's copy
       for (int i = et; i < BN; i += 128) {
         const int n = n0 + i;
         const bool ok = n < pb.N;
-        epi_sw[i] = ok ? sw[n] : 0.f;
-        epi_b[i] = (ok && bias) ? __uint_as_float(static_cast<uint32_t>(bias[n]) << 16) : 0.f;
+        if (!OUT_S32) {
+          epi_sw[i] = ok ? sw[n] : 0.f;
+          epi_b[i] = (ok && bias) ? __uint_as_float(static_cast<uint32_t>(bias[n]) << 16) : 0.f;
+        }
+        if (ASYM) epi_off[i] = ok ? offset[n] : 0;
       }
       epi_bar_sync();
     }
     const int row = m0 + static_cast<int>(pb.rank) * HM + 32 * quad + lane;
     const bool row_ok = row < pb.M;
     const float s_a = (!OUT_S32 && row_ok) ? sa[row] : 0.f;
+    const int rsum = (ASYM && row_ok) ? rowsum[row] : 0;
     if (!mbar_wait_bounded(sm.acc_full(buf), aph, abort_flag, kErrWaitEpilogue)) return;
     tc_fence_after();
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quad) << 16) +
@@ -412,12 +424,14 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
 #pragma unroll
     for (int c = 0; c < BN / 32; c += 2) {
       tmem_ld_32x32b_x32(taddr + 32 * (c + 1), rb);
-      epilogue_chunk<SHIFT, OUT_S32>(ra, row, row_ok, n0 + 32 * c, pb.N, s_a, epi_sw + 32 * c,
-                                    epi_b + 32 * c, out);
+      epilogue_chunk<SHIFT, OUT_S32, ASYM>(ra, row, row_ok, n0 + 32 * c, pb.N, s_a,
+                                          epi_sw + 32 * c, epi_b + 32 * c, epi_off + 32 * c,
+                                          rsum, out);
       tmem_wait_ld();
       if (c + 2 < BN / 32) tmem_ld_32x32b_x32(taddr + 32 * (c + 2), ra);
-      epilogue_chunk<SHIFT, OUT_S32>(rb, row, row_ok, n0 + 32 * (c + 1), pb.N, s_a,
-                                    epi_sw + 32 * (c + 1), epi_b + 32 * (c + 1), out);
+      epilogue_chunk<SHIFT, OUT_S32, ASYM>(rb, row, row_ok, n0 + 32 * (c + 1), pb.N, s_a,
+                                          epi_sw + 32 * (c + 1), epi_b + 32 * (c + 1),
+                                          epi_off + 32 * (c + 1), rsum, out);
       tmem_wait_ld();
     }
     tc_fence_before();
@@ -431,12 +445,13 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
   }
 }
 
-template <int SA, int SB, bool OUT_S32>
+template <int SA, int SB, bool OUT_S32, bool ASYM>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<SA, SB>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const float* __restrict__ sa, const float* __restrict__ sw,
                  const uint16_t* __restrict__ bias, void* out, int M, int N, int K,
-                 const int* gate, int gate_want) {
+                 const int* gate, int gate_want, const int* __restrict__ rowsum,
+                 const int* __restrict__ offset) {
   using C = Cfg<SA, SB>;
   // a launch gated on a device-side width (δ-GBS) returns unless selected;
   // both CTAs of a pair read the same word, before any cluster or TMEM step
@@ -505,8 +520,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<SA, SB>::kThread
     if (lane == 0 && pb.rank != 0 && C::kPacked) relay_role<SA, SB>(sm, pb, abort_flag);
   } else if (warp < 2 + C::kEpiWarps) {
     float* epi_sw = reinterpret_cast<float*>(sm.ptr + C::kOffEpi);
-    epilogue_role<C::kAccShift, OUT_S32>(sm, pb, tmem_base, warp & 3, lane, threadIdx.x - 64, sa, sw,
-                                 bias, out, epi_sw, epi_sw + BN, abort_flag);
+    epilogue_role<C::kAccShift, OUT_S32, ASYM>(
+        sm, pb, tmem_base, warp & 3, lane, threadIdx.x - 64, sa, sw, bias, rowsum, offset, out,
+        epi_sw, epi_sw + BN, reinterpret_cast<int*>(epi_sw + 2 * BN), abort_flag);
   } else {
     if (C::kPacked) unpack_role<SA, SB>(sm, pb, threadIdx.x - 32 * (2 + C::kEpiWarps), abort_flag);
   }

@@ -135,6 +135,33 @@ __device__ __forceinline__ uint32_t simd_nibbles8(const uint32_t (&c)[8]) {
   return __byte_perm(n0 | (n0 >> 4), n1 | (n1 >> 4), 0x6420);  // bytes 0, 2 of each
 }
 
+// Sum of the signed codes held in packed words: 8 nibbles per word (4-bit) or
+// 4 bytes per word.  Nibbles are moved to the high half of a byte (16 q, exact)
+// and summed with dp4a, so the total is 16 x the code sum.
+template <int BITS, int NW>
+__device__ __forceinline__ int packed_code_sum(const uint32_t (&w)[NW]) {
+  int acc = 0;
+#pragma unroll
+  for (int i = 0; i < NW; ++i) {
+    if (BITS == 4) {
+      acc = __dp4a(static_cast<int>((w[i] << 4) & 0xF0F0F0F0u), 0x01010101, acc);
+      acc = __dp4a(static_cast<int>(w[i] & 0xF0F0F0F0u), 0x01010101, acc);
+    } else {
+      acc = __dp4a(static_cast<int>(w[i]), 0x01010101, acc);
+    }
+  }
+  return BITS == 4 ? acc >> 4 : acc;
+}
+
+// Adds a per-thread code sum to rowsum[row]: the threads of one row that run
+// together add within the warp first, their lowest lane does the atomic.
+__device__ __forceinline__ void add_row_sum(int* rowsum, int64_t row, int part, int row_key) {
+  const unsigned act = __activemask();
+  const unsigned same = __match_any_sync(act, row_key);
+  const int tot = __reduce_add_sync(same, part);
+  if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(rowsum + row, tot);
+}
+
 // --------------------------------------------------------------------------
 // Rows of up to 128 Hadamard blocks: half a block per thread.
 //
@@ -163,13 +190,19 @@ __device__ __forceinline__ uint32_t simd_nibbles8(const uint32_t (&c)[8]) {
 // stage, which thread 0 then refills.
 // --------------------------------------------------------------------------
 
-template <int BITS, bool SIMD_CLAMP>
+// Launch modes of the activation kernel: the plain hot path; gated on a
+// device-side width (δ-GBS: returns at once unless *gate == gate_want); or
+// also adding every row's code sum to rowsum[row] (zeroed by the caller).
+// Separate instantiations keep the plain path free of either.
+enum QuantMode { kPlain = 0, kGated = 1, kRowsum = 2 };
+
+template <int BITS, bool SIMD_CLAMP, int MODE>
 __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
     const __grid_constant__ CUtensorMap tmx, int64_t rows, int K, int nblk, int rpc,
     int64_t num_groups, int stages, float alpha, float scale_mul, int rotate,
-    uint8_t* __restrict__ out, float* __restrict__ scale_out, const int* gate, int gate_want) {
-  // a launch gated on a device-side width (δ-GBS) returns unless selected
-  if (gate != nullptr && *gate != gate_want) return;
+    uint8_t* __restrict__ out, float* __restrict__ scale_out, const int* gate, int gate_want,
+    int* __restrict__ rowsum) {
+  if (MODE == kGated && *gate != gate_want) return;
   constexpr int kQmax = code_qmax(BITS);
   constexpr int kOutBytes = 64 * code_storage_bits(BITS) / 8;  // packed bytes per half block
   extern __shared__ __align__(1024) uint8_t qsmem_raw[];
@@ -346,6 +379,8 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
       *reinterpret_cast<uint4*>(dst + 32) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
       *reinterpret_cast<uint4*>(dst + 48) = make_uint4(whi[4], whi[5], whi[6], whi[7]);
     }
+    if (MODE == kRowsum)
+      add_row_sum(rowsum, row, packed_code_sum<BITS>(wlo) + packed_code_sum<BITS>(whi), rl);
   }
   if (abort_flag) {
     // a wait gave up: let copies already in flight land before the CTA exits
@@ -367,8 +402,11 @@ __global__ void __launch_bounds__(MAXT) rotate_quant_group_kernel(const uint16_t
                                                                   float scale_mul, int rotate,
                                                                   uint8_t* __restrict__ out,
                                                                   float* __restrict__ scale_out,
-                                                                  const int* gate, int gate_want) {
+                                                                  const int* gate, int gate_want,
+                                                                  int* __restrict__ rowsum) {
   if (gate != nullptr && *gate != gate_want) return;
+  __shared__ int s_rowsum;
+  if (threadIdx.x == 0) s_rowsum = 0;
   constexpr int kQmax = code_qmax(BITS);
   __shared__ float warp_max[32];
 
@@ -427,6 +465,7 @@ __global__ void __launch_bounds__(MAXT) rotate_quant_group_kernel(const uint16_t
   row_factors<kQmax>(amax, alpha, s, inv);
   if (tid == 0) scale_out[row] = __fmul_rn(s, scale_mul);
 
+  int rsum = 0;
 #pragma unroll
   for (int j = 0; j < G; ++j) {
     const int g = tid + j * T;
@@ -435,12 +474,20 @@ __global__ void __launch_bounds__(MAXT) rotate_quant_group_kernel(const uint16_t
 #pragma unroll
     for (int e = 0; e < 8; ++e) c[e] = code_bits<kQmax>(v[j][e], inv);
     if (BITS == 4) {
-      *reinterpret_cast<uint32_t*>(out + row * static_cast<int64_t>(K >> 1) + g * 4) =
-          pack8_int4(c);
+      const uint32_t pw[1] = {pack8_int4(c)};
+      *reinterpret_cast<uint32_t*>(out + row * static_cast<int64_t>(K >> 1) + g * 4) = pw[0];
+      if (rowsum) rsum += packed_code_sum<BITS>(pw);
     } else {
+      const uint32_t pw[2] = {pack4_int8(c[0], c[1], c[2], c[3]), pack4_int8(c[4], c[5], c[6], c[7])};
       *reinterpret_cast<uint2*>(out + row * static_cast<int64_t>(K) + g * 8) =
-          make_uint2(pack4_int8(c[0], c[1], c[2], c[3]), pack4_int8(c[4], c[5], c[6], c[7]));
+          make_uint2(pw[0], pw[1]);
+      if (rowsum) rsum += packed_code_sum<BITS>(pw);
     }
+  }
+  if (rowsum) {  // one row per CTA: block total, one store
+    atomicAdd(&s_rowsum, rsum);
+    __syncthreads();
+    if (tid == 0) rowsum[row] = s_rowsum;
   }
 }
 
@@ -487,11 +534,13 @@ inline int choose_rows_per_cta(int nblk) {
 
 template <int BITS>
 // gate / gate_want: when gate is not null the kernels return at once unless
-// *gate == gate_want (read on the device when they start).
+// *gate == gate_want (read on the device when they start).  rowsum: when not
+// null, every row's code sum is added to rowsum[row] (zeroed by the caller).
 inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int K, float alpha,
                                             float scale_mul, int rotate, uint8_t* out,
                                             float* scale, cudaStream_t stream,
-                                            const int* gate = nullptr, int gate_want = 0) {
+                                            const int* gate = nullptr, int gate_want = 0,
+                                            int* rowsum = nullptr) {
   const int nblk = K / 128;
   const int rpc = nblk <= 128 ? choose_rows_per_cta(nblk) : 0;
   const int64_t groups = rpc ? (rows + rpc - 1) / rpc : 0;
@@ -508,8 +557,15 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
                             true, 2))
       return cudaErrorInvalidValue;
     // codes clamp on packed int16 lanes when the unclamped code fits int16
-    auto kern = alpha >= 1.0f / 256.0f ? rotate_quant_tma_kernel<BITS, true>
-                                       : rotate_quant_tma_kernel<BITS, false>;
+    const bool simd = alpha >= 1.0f / 256.0f;
+    auto kern = simd ? rotate_quant_tma_kernel<BITS, true, kPlain>
+                     : rotate_quant_tma_kernel<BITS, false, kPlain>;
+    if (gate)
+      kern = simd ? rotate_quant_tma_kernel<BITS, true, kGated>
+                  : rotate_quant_tma_kernel<BITS, false, kGated>;
+    else if (rowsum)
+      kern = simd ? rotate_quant_tma_kernel<BITS, true, kRowsum>
+                  : rotate_quant_tma_kernel<BITS, false, kRowsum>;
     cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -524,7 +580,7 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
     if (grid > groups) grid = groups;
     kern<<<static_cast<unsigned>(grid), threads, smem, stream>>>(
         tmx, rows, K, nblk, rpc, groups, stages, alpha, scale_mul, rotate, out, scale, gate,
-        gate_want);
+        gate_want, rowsum);
     return cudaGetLastError();
   }
   // Rows up to 2048 groups run with at most 256 threads so each thread keeps
@@ -539,11 +595,11 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
     if (wide)                                                                               \
       rotate_quant_group_kernel<GG, BITS, 1024>                                             \
           <<<grid, block, 0, stream>>>(x, K, alpha, scale_mul, rotate, out, scale, gate,     \
-                                       gate_want);                                          \
+                                       gate_want, rowsum);                                  \
     else                                                                                    \
       rotate_quant_group_kernel<GG, BITS, 256>                                              \
           <<<grid, block, 0, stream>>>(x, K, alpha, scale_mul, rotate, out, scale, gate,     \
-                                       gate_want);                                          \
+                                       gate_want, rowsum);                                  \
     break;
   switch (G) {
     QS_QUANT_CASE(1)
@@ -564,17 +620,17 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
 inline cudaError_t launch_rotate_quant(const uint16_t* x, int64_t rows, int K, int bits, float alpha,
                                        float scale_mul, int rotate, uint8_t* out, float* scale,
                                        cudaStream_t stream, const int* gate = nullptr,
-                                       int gate_want = 0) {
+                                       int gate_want = 0, int* rowsum = nullptr) {
   switch (bits) {
     case 4:
       return launch_rotate_quant_bits<4>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream,
-                                           gate, gate_want);
+                                           gate, gate_want, rowsum);
     case 6:
       return launch_rotate_quant_bits<6>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream,
-                                           gate, gate_want);
+                                           gate, gate_want, rowsum);
     case 8:
       return launch_rotate_quant_bits<8>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream,
-                                           gate, gate_want);
+                                           gate, gate_want, rowsum);
     default:
       return cudaErrorInvalidValue;
   }

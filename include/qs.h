@@ -188,6 +188,76 @@ QS_API qs_status qs_linear_mixed(const void* x_bf16, int64_t M, int64_t K, float
                                  int64_t workspace_bytes, void* out_bf16, void* stream);
 
 /*
+ * Bounded-init grid refinement of the weights (DVD-Quant "Resumen técnico"
+ * §2.A): per output channel an asymmetric b-bit grid (step Δ, integer zero
+ * point z, levels 0..2^b-1) for the rotated weight row u, found offline by a
+ * bound search that progressively excludes outliers followed by closed-form
+ * least-squares refits of Δ and z.  Readings (the pages give no formula or
+ * count): candidate bounds r_j [min u, max u], r_j = 1 - j/(2J), j < J, each
+ * giving Δ = (hi - lo)/(2^b - 1) and z = clamp(rint(-lo/Δ)); the smallest
+ * squared error wins; then T refits: least squares u ≈ Δ q + c on the current
+ * codes, z = clamp(rint(-c/Δ)), Δ refit for that z, keep the best grid.  Codes
+ * q = clamp(rint(u * fl(1/Δ)) + z, 0, 2^b - 1); every sum in index order in
+ * binary64.  Stored: signed codes s = q - 2^(b-1) (same packing as the
+ * symmetric path: nibbles or bytes), scale fl32(Δ) * 2^-7 (the rotations'
+ * normalisation, as in qs_pack_weights) and offset o = 2^(b-1) - z, so that
+ * Δ (q - z) = Δ (s + o).  The layer's accumulator is then
+ * sum_k q_a s + o[n] * sum_k q_a[m,k] (exact in int32).
+ */
+
+/*
+ * qs_pack_weights_bgr — offline: rotate every row of W (unless
+ * QS_FLAG_NO_ROTATE), choose its grid as above and pack it.
+ *   w_bf16      [N, K] bf16; K <= 32768 (the row is held on chip)
+ *   bits        4 or 8
+ *   candidates  J in 1..256;  iterations  T in 0..64  (64 and 8 are typical)
+ *   w_packed    [N, K/2] (4 bits) or [N, K] bytes, written
+ *   w_scale     [N] float, written;  w_offset  [N] int32, written
+ */
+QS_API qs_status qs_pack_weights_bgr(const void* w_bf16, int64_t N, int64_t K, int bits,
+                                     unsigned flags, int candidates, int iterations,
+                                     void* w_packed, float* w_scale, int32_t* w_offset,
+                                     void* stream);
+
+/*
+ * qs_quant_act_rowsum — qs_quant_act that also writes every token's code sum
+ * x_rowsum[m] = sum_k q_a[m,k] (int32 [M]; zeroed and filled by the call),
+ * which the asymmetric weight grid needs.
+ */
+QS_API qs_status qs_quant_act_rowsum(const void* x_bf16, int64_t M, int64_t K, int bits,
+                                     float alpha, unsigned flags, void* x_packed,
+                                     float* x_scale, int32_t* x_rowsum, void* stream);
+
+/*
+ * qs_qlinear_asym — qs_qlinear for weights from qs_pack_weights_bgr:
+ * out = bf16(fl(fl(fl(s_a s_w) * float(acc)) + bias)) with
+ * acc = sum_k q_a s + o[n] * x_rowsum[m].  bits 4 or 8 (both operands).
+ */
+QS_API qs_status qs_qlinear_asym(const void* x_packed, const float* x_scale,
+                                 const int32_t* x_rowsum, const void* w_packed,
+                                 const float* w_scale, const int32_t* w_offset,
+                                 const void* bias_bf16, int64_t M, int64_t N, int64_t K,
+                                 int bits, void* out_bf16, void* stream);
+
+/* qs_qgemm_s32_asym — the exact accumulators of qs_qlinear_asym (parity checks). */
+QS_API qs_status qs_qgemm_s32_asym(const void* x_packed, const int32_t* x_rowsum,
+                                   const void* w_packed, const int32_t* w_offset, int64_t M,
+                                   int64_t N, int64_t K, int bits, int32_t* acc, void* stream);
+
+/*
+ * qs_linear_bgr — the one-call layer for BGR weights: qs_quant_act_rowsum into
+ * the workspace, then qs_qlinear_asym.  The workspace holds the packed
+ * activations, the scales and the code sums:
+ * qs_linear_bgr_workspace_bytes(M, K, bits) bytes (-1 for rejected arguments).
+ */
+QS_API int64_t qs_linear_bgr_workspace_bytes(int64_t M, int64_t K, int bits);
+QS_API qs_status qs_linear_bgr(const void* x_bf16, int64_t M, int64_t K, float alpha,
+                               const void* w_packed, const float* w_scale,
+                               const int32_t* w_offset, const void* bias_bf16, int64_t N,
+                               int bits, void* workspace, int64_t workspace_bytes,
+                               void* out_bf16, void* stream);
+
+/*
  * δ-guided bit switching (DVD-Quant "Resumen técnico" §2.C): per layer, the
  * normalised L1 change between consecutive outputs is accumulated, and the
  * layer's next step runs at 4 bits while the accumulated change is below

@@ -209,3 +209,30 @@ def test_gbs_state_layout_matches_the_header(tmp_path):
     subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
     assert [int(v) for v in out] == [binding.QS_GBS_STATE_BYTES, 0, 8, 16, 20, 32]
+
+
+def test_bgr_validation(lib):
+    f = lib.qs_pack_weights_bgr
+    assert f(NUL, 16, 128, 4, 0, 64, 8, B, C, D, NUL) == NULL
+    assert f(A, 16, 128, 4, 0, 64, 8, B, C, NUL, NUL) == NULL
+    assert f(A, 16, 128, 6, 0, 64, 8, B, C, D, NUL) == BITS      # BGR grids: 4 or 8 bits
+    assert f(A, 16, 130, 4, 0, 64, 8, B, C, D, NUL) == SHAPE
+    assert f(A, 16, 32768 + 128, 4, 0, 64, 8, B, C, D, NUL) == RANGE  # row held on chip
+    for cand, iters in ((0, 8), (257, 8), (64, -1), (64, 65)):
+        assert f(A, 16, 128, 4, 0, cand, iters, B, C, D, NUL) == RANGE, (cand, iters)
+    assert f(A, 16, 128, 4, 0, 64, 8, B, C, ctypes.c_void_p(0x40004), NUL) == ALIGN
+    g = lib.qs_quant_act_rowsum
+    assert g(A, 8, 128, 4, 1.0, 0, B, C, NUL, NUL) == NULL
+    assert g(A, 8, 128, 4, 1.0, 0, B, C, ctypes.c_void_p(0x40004), NUL) == ALIGN
+    assert g(A, 8, 128, 5, 1.0, 0, B, C, D, NUL) == BITS
+    h = lib.qs_qlinear_asym
+    assert h(A, B, C, D, A, B, NUL, 8, 256, 128, 6, C, NUL) == BITS
+    assert h(A, B, NUL, D, A, B, NUL, 8, 256, 128, 4, C, NUL) == NULL
+    assert h(A, B, C, D, A, B, NUL, 8, 264, 128, 4, C, NUL) == SHAPE
+    assert lib.qs_qgemm_s32_asym(A, B, C, NUL, 8, 256, 128, 4, D, NUL) == NULL
+    assert lib.qs_linear_bgr_workspace_bytes(3, 128, 4) == 256 + 256 + 12
+    assert lib.qs_linear_bgr_workspace_bytes(3, 128, 6) == -1
+    need = lib.qs_linear_bgr_workspace_bytes(8, 128, 4)
+    k = lib.qs_linear_bgr
+    assert k(A, 8, 128, 1.0, B, C, D, NUL, 256, 4, A, need - 1, B, NUL) == RANGE
+    assert k(A, 8, 128, 1.0, B, C, NUL, NUL, 256, 4, A, need, B, NUL) == NULL
