@@ -56,6 +56,9 @@ def parse():
                    help="override M (profiling captures of a smaller case of the same shape)")
     p.add_argument("--workload", default=None,
                    help="the Wan FFN variant to time: w4a4 (default), w8a8, w4a8 or w4a6")
+    p.add_argument("--act-codes", choices=["bytes", "packed"], default="bytes",
+                   help="storage of 4-bit activation codes: one per byte (the GEMM loads them "
+                        "by TMA, only the weights are widened) or two per byte")
     return p.parse_args()
 
 
@@ -204,25 +207,28 @@ def combine_ranks(times_ms, steps, ops_per_step, world, device="cpu"):
             "value": ops_per_step * world / (ms_per_step * 1e-3) / 1e12}
 
 
-def time_layer(qs, torch, x, wp, ws, bias, bits, alpha, stream, steps=5, warmup=2, bits_x=None):
+def time_layer(qs, torch, x, wp, ws, bias, bits, alpha, stream, steps=5, warmup=2, bits_x=None,
+               x_flags=0):
     """Mean CUDA-event times (ms) of the activation kernel and the GEMM for one
-    layer; ``bits`` is the weights' code width, ``bits_x`` the activations'."""
+    layer; ``bits`` is the weights' code width, ``bits_x`` the activations',
+    ``x_flags`` their quantisation flags (storage)."""
     bx = bits if bits_x is None else bits_x
+    sx = qs.storage_bits(bx, x_flags)
     M, K = x.shape
     N = wp.shape[0]
     dev = x.device
-    xp = torch.empty((M, qs.packed_cols(K, bx)), dtype=torch.uint8, device=dev)
+    xp = torch.empty((M, qs.packed_cols(K, bx, x_flags)), dtype=torch.uint8, device=dev)
     xs = torch.empty((M,), dtype=torch.float32, device=dev)
     out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     for _ in range(warmup):
-        qs.qs_quant_act(x, M, K, bx, alpha, 0, xp, xs, stream)
-        qs.qs_qlinear_mixed(xp, xs, bx, wp, ws, bits, bias, M, N, K, out, stream)
+        qs.qs_quant_act(x, M, K, bx, alpha, x_flags, xp, xs, stream)
+        qs.qs_qlinear_mixed(xp, xs, sx, wp, ws, bits, bias, M, N, K, out, stream)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     for e in ev:
         e[0].record(stream)
-        qs.qs_quant_act(x, M, K, bx, alpha, 0, xp, xs, stream)
+        qs.qs_quant_act(x, M, K, bx, alpha, x_flags, xp, xs, stream)
         e[1].record(stream)
-        qs.qs_qlinear_mixed(xp, xs, bx, wp, ws, bits, bias, M, N, K, out, stream)
+        qs.qs_qlinear_mixed(xp, xs, sx, wp, ws, bits, bias, M, N, K, out, stream)
         e[2].record(stream)
     stream.synchronize()
     q = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
@@ -233,14 +239,17 @@ def time_layer(qs, torch, x, wp, ws, bias, bits, alpha, stream, steps=5, warmup=
 def all_configs(qs, torch, I, dev, stream):
     """Per-configuration throughput on one GPU (every seeded synthetic shape)."""
     res = {}
-    for cfg in (*I.LAYER_CONFIGS, *I.MIXED_CONFIGS):
+    runs = [(cfg, 0) for cfg in (*I.LAYER_CONFIGS, *I.MIXED_CONFIGS)]
+    runs += [(cfg, qs.QS_FLAG_BYTE_CODES) for cfg in (I.HY_QKV, I.WAN_FFN)]
+    for cfg, flags in runs:
         d = I.make_layer(cfg)
         with torch.cuda.stream(stream):
             x, w, b = d["x"].to(dev), d["w"].to(dev), d["bias"].to(dev)
             wp, ws = qs.pack_weights(w, cfg.bits, stream=stream)
         q, g, _ = time_layer(qs, torch, x, wp, ws, b, cfg.bits, cfg.alpha, stream,
-                             bits_x=cfg.act_bits)
-        res[cfg.name] = {"bits_w": cfg.bits, "bits_x": cfg.act_bits, "quant_ms": q, "gemm_ms": g,
+                             bits_x=cfg.act_bits, x_flags=flags)
+        name = cfg.name + ("_act_codes_in_bytes" if flags else "")
+        res[name] = {"bits_w": cfg.bits, "bits_x": cfg.act_bits, "quant_ms": q, "gemm_ms": g,
                          "TOPS": cfg.ops / ((q + g) * 1e-3) / 1e12,
                          "gemm_TOPS": cfg.ops / (g * 1e-3) / 1e12,
                          "tokens_per_s": cfg.M / ((q + g) * 1e-3)}
@@ -448,26 +457,28 @@ def main():
     d = I.make_layer(cfg, M=args.tokens)
     M, K, N, alpha = d["x"].shape[0], cfg.K, cfg.N, cfg.alpha
     bits, bx = cfg.bits, cfg.act_bits  # weight and activation code widths
+    x_flags = qs.QS_FLAG_BYTE_CODES if (args.act_codes == "bytes" and bx == 4) else 0
+    sx = qs.storage_bits(bx, x_flags)  # storage width the GEMM reads
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
         x = d["x"].to(dev)
         w = d["w"].to(dev)
         bias = d["bias"].to(dev)
         wp, ws = qs.pack_weights(w, bits, stream=stream)
-        xp = torch.empty((M, qs.packed_cols(K, bx)), dtype=torch.uint8, device=dev)
+        xp = torch.empty((M, qs.packed_cols(K, bx, x_flags)), dtype=torch.uint8, device=dev)
         xs = torch.empty((M,), dtype=torch.float32, device=dev)
         out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     stream.synchronize()
     del w
 
     def gemm():
-        if bx == bits:
+        if sx == bits:
             qs.qs_qlinear(xp, xs, wp, ws, bias, M, N, K, bits, out, stream)
         else:
-            qs.qs_qlinear_mixed(xp, xs, bx, wp, ws, bits, bias, M, N, K, out, stream)
+            qs.qs_qlinear_mixed(xp, xs, sx, wp, ws, bits, bias, M, N, K, out, stream)
 
     def step():
-        qs.qs_quant_act(x, M, K, bx, alpha, 0, xp, xs, stream)
+        qs.qs_quant_act(x, M, K, bx, alpha, x_flags, xp, xs, stream)
         gemm()
 
     for _ in range(max(3, args.warmup)):
@@ -486,7 +497,7 @@ def main():
         time.sleep(0.3)
     for i in range(args.steps):
         ev[i][0].record(stream)
-        qs.qs_quant_act(x, M, K, bx, alpha, 0, xp, xs, stream)
+        qs.qs_quant_act(x, M, K, bx, alpha, x_flags, xp, xs, stream)
         ev[i][1].record(stream)
         gemm()
         ev[i][2].record(stream)
@@ -511,13 +522,13 @@ def main():
     out_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
     e2e_steps = max(1, args.e2e_steps)
 
-    ws_bytes = qs.qs_linear_workspace_bytes(M, K, bx)
+    ws_bytes = qs.qs_linear_workspace_bytes(M, K, sx)
     workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
 
     def e2e_step():  # one C call for the layer, host buffers in and out
         x.copy_(x_host, non_blocking=True)
-        qs.qs_linear_mixed(x, M, K, alpha, bx, wp, ws, bits, bias, N, workspace, ws_bytes, out,
-                           stream)
+        qs.qs_linear_ex(x, M, K, alpha, bx, x_flags, wp, ws, bits, bias, N, workspace, ws_bytes,
+                        out, stream)
         out_host.copy_(out, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -546,7 +557,8 @@ def main():
         pk, src = peaks()
         int8_peak = pk["bf16_tflops"] * INT8_PER_BF16
         gemm_tops = ops_per_step / (gemm_ms * 1e-3) / 1e12
-        quant_bytes = M * (2 * K + qs.packed_cols(K, bx) + 4)
+        quant_bytes = M * (2 * K + qs.packed_cols(K, bx, x_flags) + 4)
+        traffic_key = cfg.name + ("_act_codes_in_bytes" if x_flags else "")
         quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
         line = {
             "metric": METRIC, "value": value, "unit": UNIT,
@@ -557,18 +569,19 @@ def main():
             "dtype": "int4" if bx == bits == 4 else f"int{bits}w-int{bx}a",
             "config": {"workload": cfg.name, "M": M, "K": K, "N": N, "bits_w": bits,
                        "bits_x": bx, "alpha": alpha,
+                       "act_codes": "bytes" if x_flags else "packed",
                        "seed": cfg.seed, "parallelism": f"replicas{world}",
                        "l2": "inputs larger than L2 (x 335 MB, out 906 MB bf16); no flush"},
             "roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak,
                          "unit": UNIT, "frac": gemm_tops / int8_peak,
-                         "traffic": ncu_traffic(cfg.name, "qgemm_kernel"),
-                         "kernel": f"qgemm_kernel<{4 if bx == 4 else 8},{4 if bits == 4 else 8},"
-                                   f"false> (tcgen05 kind::i8)",
+                         "traffic": ncu_traffic(traffic_key, "qgemm_kernel"),
+                         "kernel": f"qgemm_kernel<{4 if sx == 4 else 8},{4 if bits == 4 else 8},"
+                                   f"false,false> (tcgen05 kind::i8)",
                          "peak_source": f"{src}: bf16_tflops (burst) x {INT8_PER_BF16} "
                                         f"nominal int8:bf16"},
             "roofline_quant": {"bound": "hbm", "achieved": quant_gbs, "peak": pk["hbm_gbs"],
                                "unit": "GB/s", "frac": quant_gbs / pk["hbm_gbs"],
-                               "traffic": ncu_traffic(cfg.name, "rotate_quant_kernel"),
+                               "traffic": ncu_traffic(traffic_key, "rotate_quant_kernel"),
                                "algorithmic_bytes": quant_bytes,
                                "peak_source": f"{src}: hbm_gbs"},
             "kernels_ms": {"quant": quant_ms, "gemm": gemm_ms},
@@ -577,8 +590,8 @@ def main():
                     "h2d_bytes_per_step": x_host.numel() * 2,
                     "d2h_bytes_per_step": out_host.numel() * 2,
                     "ms_per_step": e2e_ms, "steps": e2e_steps,
-                    "call": "qs_linear_mixed (C ABI; = qs_linear at equal widths), pinned host x "
-                            "in, bf16 output back"},
+                    "call": "qs_linear_ex (C ABI: activation kernel + GEMM), pinned host x in, "
+                            "bf16 output back"},
             "clocks": clocks,
         }
         line.update(extra)

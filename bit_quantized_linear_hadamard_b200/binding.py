@@ -23,12 +23,14 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqs.so")
 
 QS_FLAG_NO_ROTATE = 1
+QS_FLAG_BYTE_CODES = 2
 QS_MAX_K = 65536
 STATUS = {0: "QS_OK", 1: "QS_ERR_NULL", 2: "QS_ERR_SHAPE", 3: "QS_ERR_BITS", 4: "QS_ERR_ALIGN",
           5: "QS_ERR_RANGE", 6: "QS_ERR_CUDA", 7: "QS_ERR_TIMEOUT", 8: "QS_ERR_PTR"}
 EXPORTS = ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qlinear_mixed", "qs_qgemm_s32",
            "qs_qgemm_s32_mixed", "qs_gelu_bf16", "qs_linear_workspace_bytes", "qs_linear",
-           "qs_linear_mixed", "qs_linear_noalloc", "qs_pack_weights_bgr", "qs_quant_act_rowsum",
+           "qs_linear_mixed", "qs_linear_ex", "qs_linear_noalloc", "qs_pack_weights_bgr",
+           "qs_quant_act_rowsum",
            "qs_qlinear_asym", "qs_qgemm_s32_asym", "qs_linear_bgr_workspace_bytes",
            "qs_linear_bgr", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
            "qs_selftest_timeout", "qs_device_error", "qs_status_str", "qs_version")
@@ -69,6 +71,7 @@ def load() -> ctypes.CDLL:
     L.qs_linear_workspace_bytes.restype = i64
     L.qs_linear.argtypes = [vp, i64, i64, f32, vp, vp, vp, i64, i32, vp, i64, vp, vp]
     L.qs_linear_mixed.argtypes = [vp, i64, i64, f32, i32, vp, vp, i32, vp, i64, vp, i64, vp, vp]
+    L.qs_linear_ex.argtypes = [vp, i64, i64, f32, i32, u32, vp, vp, i32, vp, i64, vp, i64, vp, vp]
     L.qs_linear_noalloc.argtypes = [vp, i64, i64, f32, vp, vp, vp, i64, i32, vp, vp]
     f64 = ctypes.c_double
     L.qs_pack_weights_bgr.argtypes = [vp, i64, i64, i32, u32, i32, i32, vp, vp, vp, vp]
@@ -88,7 +91,7 @@ def load() -> ctypes.CDLL:
     L.qs_version.restype = ctypes.c_char_p
     for name in ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qlinear_mixed",
                  "qs_qgemm_s32", "qs_qgemm_s32_mixed", "qs_gelu_bf16", "qs_linear",
-                 "qs_linear_mixed", "qs_linear_noalloc", "qs_pack_weights_bgr",
+                 "qs_linear_mixed", "qs_linear_ex", "qs_linear_noalloc", "qs_pack_weights_bgr",
                  "qs_quant_act_rowsum", "qs_qlinear_asym", "qs_qgemm_s32_asym", "qs_linear_bgr",
                  "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs", "qs_selftest_timeout",
                  "qs_device_error"):
@@ -223,6 +226,19 @@ def qs_linear_mixed(x, M, K, alpha, bits_x, w_packed, w_scale, bits_w, bias, N, 
                                   _s(stream)), "qs_linear_mixed")
 
 
+def qs_linear_ex(x, M, K, alpha, bits_x, x_flags, w_packed, w_scale, bits_w, bias, N, workspace,
+                 workspace_bytes, out, stream=None):
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(w_packed, torch.uint8, "w_packed")
+    _cuda(w_scale, torch.float32, "w_scale")
+    _cuda(bias, torch.bfloat16, "bias")
+    _cuda(workspace, torch.uint8, "workspace")
+    _cuda(out, torch.bfloat16, "out")
+    _check(load().qs_linear_ex(_p(x), M, K, float(alpha), bits_x, x_flags, _p(w_packed),
+                               _p(w_scale), bits_w, _p(bias), N, _p(workspace), workspace_bytes,
+                               _p(out), _s(stream)), "qs_linear_ex")
+
+
 def qs_linear_noalloc(x, M, K, alpha, w_packed, w_scale, bias, N, bits, out, stream=None):
     """qs_linear on the library's own fixed scratch buffer (for callers that
     cannot allocate device memory when they run the layer); nothing is allocated."""
@@ -336,15 +352,21 @@ def qs_version() -> str:
 
 # --------------------------------------------------------------------------- helpers
 
-def packed_cols(K: int, bits: int) -> int:
-    """Bytes of one packed row of K codes: nibbles for 4 bits, bytes for 6 and 8."""
-    return K // 2 if bits == 4 else K
+def packed_cols(K: int, bits: int, flags: int = 0) -> int:
+    """Bytes of one packed row of K codes: nibbles for 4 bits (bytes with
+    QS_FLAG_BYTE_CODES), bytes for 6 and 8."""
+    return K // 2 if bits == 4 and not (flags & QS_FLAG_BYTE_CODES) else K
+
+
+def storage_bits(bits: int, flags: int = 0) -> int:
+    """The width the GEMM calls take for codes of `bits` written with `flags`."""
+    return 8 if (flags & QS_FLAG_BYTE_CODES) else bits
 
 
 def pack_weights(w: torch.Tensor, bits: int, flags: int = 0, stream=None):
     """w bf16 [N, K] -> (w_packed uint8 [N, packed_cols(K, bits)], w_scale float32 [N])."""
     N, K = w.shape
-    wp = torch.empty((N, packed_cols(K, bits)), dtype=torch.uint8, device=w.device)
+    wp = torch.empty((N, packed_cols(K, bits, flags)), dtype=torch.uint8, device=w.device)
     ws = torch.empty((N,), dtype=torch.float32, device=w.device)
     qs_pack_weights(w, N, K, bits, flags, wp, ws, stream)
     return wp, ws
@@ -377,7 +399,7 @@ def quant_act(x: torch.Tensor, bits: int, alpha: float = 1.0, flags: int = 0, st
     """x bf16 [M, K] -> (x_packed uint8 [M, packed_cols(K, bits)], x_scale float32 [M])."""
     M, K = x.shape
     if out is None:
-        xp = torch.empty((M, packed_cols(K, bits)), dtype=torch.uint8, device=x.device)
+        xp = torch.empty((M, packed_cols(K, bits, flags)), dtype=torch.uint8, device=x.device)
         xs = torch.empty((M,), dtype=torch.float32, device=x.device)
     else:
         xp, xs = out
@@ -416,19 +438,24 @@ def gelu(x: torch.Tensor, stream=None, out=None):
 
 
 def linear(x, w_packed, w_scale, bias, bits: int, alpha: float = 1.0, workspace=None,
-           stream=None, out=None, bits_w: int | None = None):
-    """bf16 activations [M, K] -> bf16 [M, N] through qs_linear (one C call);
-    ``bits`` is the activation width, ``bits_w`` the weights' (default ``bits``)."""
+           stream=None, out=None, bits_w: int | None = None, x_flags: int = 0):
+    """bf16 activations [M, K] -> bf16 [M, N] through one C call; ``bits`` is
+    the activation width, ``bits_w`` the weights' storage width (default
+    ``bits``), ``x_flags`` the activation quantisation flags."""
     M, K = x.shape
     N = w_packed.shape[0]
-    need = qs_linear_workspace_bytes(M, K, bits)
+    need = qs_linear_workspace_bytes(M, K, storage_bits(bits, x_flags))
     if need < 0:
         raise QSError(2, "qs_linear_workspace_bytes")
     if workspace is None:
         workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    if bits_w is None or bits_w == bits:
+    if x_flags:
+        qs_linear_ex(x, M, K, alpha, bits, x_flags, w_packed, w_scale,
+                     bits if bits_w is None else bits_w, bias, N, workspace, workspace.numel(),
+                     out, stream)
+    elif bits_w is None or bits_w == bits:
         qs_linear(x, M, K, alpha, w_packed, w_scale, bias, N, bits, workspace, workspace.numel(),
                   out, stream)
     else:

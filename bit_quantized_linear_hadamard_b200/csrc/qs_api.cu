@@ -20,7 +20,7 @@
 
 namespace {
 
-constexpr unsigned kKnownFlags = QS_FLAG_NO_ROTATE;
+constexpr unsigned kKnownFlags = QS_FLAG_NO_ROTATE | QS_FLAG_BYTE_CODES;
 constexpr float kMinAlpha = 1.0f / 16384.0f;  // keeps |u * inv| < 2^22
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -164,7 +164,8 @@ qs_status qs_pack_weights(const void* w_bf16, int64_t N, int64_t K, int bits, un
   const float scale_mul = rotate ? 0.0078125f : 1.0f;
   const cudaError_t e = qs::launch_rotate_quant(
       static_cast<const uint16_t*>(w_bf16), N, static_cast<int>(K), bits, 1.0f, scale_mul,
-      rotate ? 1 : 0, static_cast<uint8_t*>(w_packed), w_scale, static_cast<cudaStream_t>(stream));
+      rotate ? 1 : 0, static_cast<uint8_t*>(w_packed), w_scale, static_cast<cudaStream_t>(stream),
+      nullptr, 0, nullptr, (flags & QS_FLAG_BYTE_CODES) != 0);
   return e == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
@@ -182,7 +183,8 @@ qs_status qs_quant_act(const void* x_bf16, int64_t M, int64_t K, int bits, float
   const bool rotate = !(flags & QS_FLAG_NO_ROTATE);
   const cudaError_t e = qs::launch_rotate_quant(
       static_cast<const uint16_t*>(x_bf16), M, static_cast<int>(K), bits, alpha, 1.0f,
-      rotate ? 1 : 0, static_cast<uint8_t*>(x_packed), x_scale, static_cast<cudaStream_t>(stream));
+      rotate ? 1 : 0, static_cast<uint8_t*>(x_packed), x_scale, static_cast<cudaStream_t>(stream),
+      nullptr, 0, nullptr, (flags & QS_FLAG_BYTE_CODES) != 0);
   return e == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
@@ -232,14 +234,17 @@ int64_t qs_linear_workspace_bytes(int64_t M, int64_t K, int bits) {
   return packed + 4 * M;
 }
 
-qs_status qs_linear_mixed(const void* x_bf16, int64_t M, int64_t K, float alpha, int bits_x,
-                          const void* w_packed, const float* w_scale, int bits_w,
-                          const void* bias_bf16, int64_t N, void* workspace,
-                          int64_t workspace_bytes, void* out_bf16, void* stream) {
+qs_status qs_linear_ex(const void* x_bf16, int64_t M, int64_t K, float alpha, int bits_x,
+                       unsigned x_flags, const void* w_packed, const float* w_scale, int bits_w,
+                       const void* bias_bf16, int64_t N, void* workspace, int64_t workspace_bytes,
+                       void* out_bf16, void* stream) {
   if (!x_bf16 || !w_packed || !w_scale || !workspace || !out_bf16) return QS_ERR_NULL;
   QS_TRY(check_gemm_args(workspace, w_packed, out_bf16, M, N, K, bits_x, bits_w));
   if (!(alpha >= kMinAlpha && alpha <= 1.0f)) return QS_ERR_RANGE;
-  const int64_t need = qs_linear_workspace_bytes(M, K, bits_x);
+  if (x_flags & ~kKnownFlags) return QS_ERR_RANGE;
+  // storage width of the activation codes, which is what the GEMM reads
+  const int store_x = (x_flags & QS_FLAG_BYTE_CODES) ? 8 : bits_x;
+  const int64_t need = qs_linear_workspace_bytes(M, K, store_x);
   if (need < 0) return QS_ERR_SHAPE;
   if (workspace_bytes < need) return QS_ERR_RANGE;
   // everything both launches will check, before the first one
@@ -252,10 +257,18 @@ qs_status qs_linear_mixed(const void* x_bf16, int64_t M, int64_t K, float alpha,
   QS_TRY(check_device_ptr(out_bf16));
   if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
   uint8_t* xp = static_cast<uint8_t*>(workspace);
-  float* xs = reinterpret_cast<float*>(xp + (M * packed_row_bytes(K, bits_x) + 255) / 256 * 256);
-  QS_TRY(qs_quant_act(x_bf16, M, K, bits_x, alpha, 0u, xp, xs, stream));
-  return qs_qlinear_mixed(xp, xs, bits_x, w_packed, w_scale, bits_w, bias_bf16, M, N, K, out_bf16,
-                          stream);
+  float* xs = reinterpret_cast<float*>(xp + (M * packed_row_bytes(K, store_x) + 255) / 256 * 256);
+  QS_TRY(qs_quant_act(x_bf16, M, K, bits_x, alpha, x_flags, xp, xs, stream));
+  return qs_qlinear_mixed(xp, xs, store_x, w_packed, w_scale, bits_w, bias_bf16, M, N, K,
+                          out_bf16, stream);
+}
+
+qs_status qs_linear_mixed(const void* x_bf16, int64_t M, int64_t K, float alpha, int bits_x,
+                          const void* w_packed, const float* w_scale, int bits_w,
+                          const void* bias_bf16, int64_t N, void* workspace,
+                          int64_t workspace_bytes, void* out_bf16, void* stream) {
+  return qs_linear_ex(x_bf16, M, K, alpha, bits_x, 0u, w_packed, w_scale, bits_w, bias_bf16, N,
+                      workspace, workspace_bytes, out_bf16, stream);
 }
 
 qs_status qs_linear(const void* x_bf16, int64_t M, int64_t K, float alpha, const void* w_packed,
@@ -393,7 +406,8 @@ qs_status qs_quant_act_rowsum(const void* x_bf16, int64_t M, int64_t K, int bits
   const bool rotate = !(flags & QS_FLAG_NO_ROTATE);
   const cudaError_t e = qs::launch_rotate_quant(
       static_cast<const uint16_t*>(x_bf16), M, static_cast<int>(K), bits, alpha, 1.0f,
-      rotate ? 1 : 0, static_cast<uint8_t*>(x_packed), x_scale, s, nullptr, 0, x_rowsum);
+      rotate ? 1 : 0, static_cast<uint8_t*>(x_packed), x_scale, s, nullptr, 0, x_rowsum,
+      (flags & QS_FLAG_BYTE_CODES) != 0);
   return e == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 

@@ -138,19 +138,19 @@ __device__ __forceinline__ uint32_t simd_nibbles8(const uint32_t (&c)[8]) {
 // Sum of the signed codes held in packed words: 8 nibbles per word (4-bit) or
 // 4 bytes per word.  Nibbles are moved to the high half of a byte (16 q, exact)
 // and summed with dp4a, so the total is 16 x the code sum.
-template <int BITS, int NW>
+template <int STORE, int NW>
 __device__ __forceinline__ int packed_code_sum(const uint32_t (&w)[NW]) {
   int acc = 0;
 #pragma unroll
   for (int i = 0; i < NW; ++i) {
-    if (BITS == 4) {
+    if (STORE == 4) {
       acc = __dp4a(static_cast<int>((w[i] << 4) & 0xF0F0F0F0u), 0x01010101, acc);
       acc = __dp4a(static_cast<int>(w[i] & 0xF0F0F0F0u), 0x01010101, acc);
     } else {
       acc = __dp4a(static_cast<int>(w[i]), 0x01010101, acc);
     }
   }
-  return BITS == 4 ? acc >> 4 : acc;
+  return STORE == 4 ? acc >> 4 : acc;
 }
 
 // Adds a per-thread code sum to rowsum[row]: the threads of one row that run
@@ -196,7 +196,9 @@ __device__ __forceinline__ void add_row_sum(int* rowsum, int64_t row, int part, 
 // Separate instantiations keep the plain path free of either.
 enum QuantMode { kPlain = 0, kGated = 1, kRowsum = 2 };
 
-template <int BITS, bool SIMD_CLAMP, int MODE>
+// BITS: code width (qmax 2^(BITS-1) - 1); STORE: storage per code, 4 (two
+// codes per byte) or 8 (one byte per code, also for 4-bit codes).
+template <int BITS, int STORE, bool SIMD_CLAMP, int MODE>
 __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
     const __grid_constant__ CUtensorMap tmx, int64_t rows, int K, int nblk, int rpc,
     int64_t num_groups, int stages, float alpha, float scale_mul, int rotate,
@@ -204,7 +206,7 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
     int* __restrict__ rowsum) {
   if (MODE == kGated && *gate != gate_want) return;
   constexpr int kQmax = code_qmax(BITS);
-  constexpr int kOutBytes = 64 * code_storage_bits(BITS) / 8;  // packed bytes per half block
+  constexpr int kOutBytes = 64 * STORE / 8;  // packed bytes per half block
   extern __shared__ __align__(1024) uint8_t qsmem_raw[];
   __shared__ unsigned int row_amax[3][128];
   __shared__ int abort_flag;
@@ -333,7 +335,7 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
     [[maybe_unused]] constexpr float kQ = static_cast<float>(kQmax);
     // Codes of 8 consecutive pairs = elements 8k..8k+7 (low halves) and
     // 32+8k..32+8k+7 (high halves) of this half block.
-    uint32_t wlo[BITS == 4 ? 4 : 8], whi[BITS == 4 ? 4 : 8];
+    uint32_t wlo[STORE == 4 ? 4 : 8], whi[STORE == 4 ? 4 : 8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       uint32_t clo[8], chi[8];
@@ -348,7 +350,7 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
         chi[e] = __float_as_uint(cb.y);
       }
       if (SIMD_CLAMP) {
-        if (BITS == 4) {
+        if (STORE == 4) {
           wlo[k] = simd_nibbles8(clo);
           whi[k] = simd_nibbles8(chi);
         } else {
@@ -357,7 +359,7 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
           whi[2 * k] = simd_bytes4<kQmax>(chi, 0);
           whi[2 * k + 1] = simd_bytes4<kQmax>(chi, 1);
         }
-      } else if (BITS == 4) {
+      } else if (STORE == 4) {
         wlo[k] = pack8_int4(clo);
         whi[k] = pack8_int4(chi);
       } else {
@@ -368,9 +370,8 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
       }
     }
     uint8_t* dst =
-        out + row * static_cast<int64_t>(K * code_storage_bits(BITS) / 8) + blk * (2 * kOutBytes) +
-        up * kOutBytes;
-    if (BITS == 4) {  // 16 bytes of elements 0..31, then 16 bytes of 32..63
+        out + row * static_cast<int64_t>(K * STORE / 8) + blk * (2 * kOutBytes) + up * kOutBytes;
+    if (STORE == 4) {  // 16 bytes of elements 0..31, then 16 bytes of 32..63
       *reinterpret_cast<uint4*>(dst) = make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
       *reinterpret_cast<uint4*>(dst + 16) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
     } else {
@@ -380,7 +381,7 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
       *reinterpret_cast<uint4*>(dst + 48) = make_uint4(whi[4], whi[5], whi[6], whi[7]);
     }
     if (MODE == kRowsum)
-      add_row_sum(rowsum, row, packed_code_sum<BITS>(wlo) + packed_code_sum<BITS>(whi), rl);
+      add_row_sum(rowsum, row, packed_code_sum<STORE>(wlo) + packed_code_sum<STORE>(whi), rl);
   }
   if (abort_flag) {
     // a wait gave up: let copies already in flight land before the CTA exits
@@ -396,7 +397,7 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
 // lanes (T is a multiple of 32), so stage h = 8, 16, 32, 64 pairs lanes at
 // xor-distance 1, 2, 4, 8.
 // --------------------------------------------------------------------------
-template <int G, int BITS, int MAXT>
+template <int G, int BITS, int STORE, int MAXT>
 __global__ void __launch_bounds__(MAXT) rotate_quant_group_kernel(const uint16_t* __restrict__ x,
                                                                   int K, float alpha,
                                                                   float scale_mul, int rotate,
@@ -473,15 +474,15 @@ __global__ void __launch_bounds__(MAXT) rotate_quant_group_kernel(const uint16_t
     uint32_t c[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) c[e] = code_bits<kQmax>(v[j][e], inv);
-    if (BITS == 4) {
+    if (STORE == 4) {
       const uint32_t pw[1] = {pack8_int4(c)};
       *reinterpret_cast<uint32_t*>(out + row * static_cast<int64_t>(K >> 1) + g * 4) = pw[0];
-      if (rowsum) rsum += packed_code_sum<BITS>(pw);
+      if (rowsum) rsum += packed_code_sum<STORE>(pw);
     } else {
       const uint32_t pw[2] = {pack4_int8(c[0], c[1], c[2], c[3]), pack4_int8(c[4], c[5], c[6], c[7])};
       *reinterpret_cast<uint2*>(out + row * static_cast<int64_t>(K) + g * 8) =
           make_uint2(pw[0], pw[1]);
-      if (rowsum) rsum += packed_code_sum<BITS>(pw);
+      if (rowsum) rsum += packed_code_sum<STORE>(pw);
     }
   }
   if (rowsum) {  // one row per CTA: block total, one store
@@ -532,7 +533,7 @@ inline int choose_rows_per_cta(int nblk) {
   return best;
 }
 
-template <int BITS>
+template <int BITS, int STORE>
 // gate / gate_want: when gate is not null the kernels return at once unless
 // *gate == gate_want (read on the device when they start).  rowsum: when not
 // null, every row's code sum is added to rowsum[row] (zeroed by the caller).
@@ -558,14 +559,14 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
       return cudaErrorInvalidValue;
     // codes clamp on packed int16 lanes when the unclamped code fits int16
     const bool simd = alpha >= 1.0f / 256.0f;
-    auto kern = simd ? rotate_quant_tma_kernel<BITS, true, kPlain>
-                     : rotate_quant_tma_kernel<BITS, false, kPlain>;
+    auto kern = simd ? rotate_quant_tma_kernel<BITS, STORE, true, kPlain>
+                     : rotate_quant_tma_kernel<BITS, STORE, false, kPlain>;
     if (gate)
-      kern = simd ? rotate_quant_tma_kernel<BITS, true, kGated>
-                  : rotate_quant_tma_kernel<BITS, false, kGated>;
+      kern = simd ? rotate_quant_tma_kernel<BITS, STORE, true, kGated>
+                  : rotate_quant_tma_kernel<BITS, STORE, false, kGated>;
     else if (rowsum)
-      kern = simd ? rotate_quant_tma_kernel<BITS, true, kRowsum>
-                  : rotate_quant_tma_kernel<BITS, false, kRowsum>;
+      kern = simd ? rotate_quant_tma_kernel<BITS, STORE, true, kRowsum>
+                  : rotate_quant_tma_kernel<BITS, STORE, false, kRowsum>;
     cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -593,11 +594,11 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
 #define QS_QUANT_CASE(GG)                                                                   \
   case GG:                                                                                  \
     if (wide)                                                                               \
-      rotate_quant_group_kernel<GG, BITS, 1024>                                             \
+      rotate_quant_group_kernel<GG, BITS, STORE, 1024>                                      \
           <<<grid, block, 0, stream>>>(x, K, alpha, scale_mul, rotate, out, scale, gate,     \
                                        gate_want, rowsum);                                  \
     else                                                                                    \
-      rotate_quant_group_kernel<GG, BITS, 256>                                              \
+      rotate_quant_group_kernel<GG, BITS, STORE, 256>                                       \
           <<<grid, block, 0, stream>>>(x, K, alpha, scale_mul, rotate, out, scale, gate,     \
                                        gate_want, rowsum);                                  \
     break;
@@ -620,17 +621,22 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
 inline cudaError_t launch_rotate_quant(const uint16_t* x, int64_t rows, int K, int bits, float alpha,
                                        float scale_mul, int rotate, uint8_t* out, float* scale,
                                        cudaStream_t stream, const int* gate = nullptr,
-                                       int gate_want = 0, int* rowsum = nullptr) {
+                                       int gate_want = 0, int* rowsum = nullptr,
+                                       bool byte_codes = false) {
+  // byte_codes: 4-bit codes written one per byte (6- and 8-bit codes always are)
   switch (bits) {
     case 4:
-      return launch_rotate_quant_bits<4>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream,
-                                           gate, gate_want, rowsum);
+      return byte_codes
+                 ? launch_rotate_quant_bits<4, 8>(x, rows, K, alpha, scale_mul, rotate, out, scale,
+                                                  stream, gate, gate_want, rowsum)
+                 : launch_rotate_quant_bits<4, 4>(x, rows, K, alpha, scale_mul, rotate, out, scale,
+                                                  stream, gate, gate_want, rowsum);
     case 6:
-      return launch_rotate_quant_bits<6>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream,
-                                           gate, gate_want, rowsum);
+      return launch_rotate_quant_bits<6, 8>(x, rows, K, alpha, scale_mul, rotate, out, scale,
+                                            stream, gate, gate_want, rowsum);
     case 8:
-      return launch_rotate_quant_bits<8>(x, rows, K, alpha, scale_mul, rotate, out, scale, stream,
-                                           gate, gate_want, rowsum);
+      return launch_rotate_quant_bits<8, 8>(x, rows, K, alpha, scale_mul, rotate, out, scale,
+                                            stream, gate, gate_want, rowsum);
     default:
       return cudaErrorInvalidValue;
   }

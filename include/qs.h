@@ -70,6 +70,13 @@ typedef enum {
 /* Test-only flag: skip the Hadamard rotation (the codes are then taken from the
  * input values themselves, which makes rounding ties easy to construct). */
 #define QS_FLAG_NO_ROTATE 1u
+/* Storage flag for qs_quant_act / qs_pack_weights (and the _rowsum form):
+ * 4-bit codes are written one per byte (int8, values in [-7, 7]) instead of
+ * two per byte.  Such codes are passed to the GEMM calls with bits = 8 (the
+ * GEMM only needs the storage; the accumulator bounds hold a fortiori).  For
+ * activations this trades M*K/2 bytes of extra writes for a GEMM that loads
+ * them by TMA straight into its operand tiles; the arithmetic is unchanged. */
+#define QS_FLAG_BYTE_CODES 2u
 
 /* Largest K accepted.  With |q| <= 127 the int32 accumulator cannot overflow
  * (127^2 * 65536 < 2^31), and the rotate-quantize kernel keeps a whole row in
@@ -85,8 +92,8 @@ typedef enum {
  * own scale (one per output channel, alpha = 1) and packs it.
  *   w_bf16   [N, K] bf16, row-major (torch.nn.Linear layout; y = x W^T + b)
  *   bits     4, 6 or 8
- *   flags    0 or QS_FLAG_NO_ROTATE
- *   w_packed [N, K/2] bytes (4 bits) or [N, K] bytes, written
+ *   flags    QS_FLAG_NO_ROTATE, QS_FLAG_BYTE_CODES or both
+ *   w_packed [N, K/2] bytes (4 bits, packed) or [N, K] bytes, written
  *   w_scale  [N] float, written: s * 2^-7 (or s with QS_FLAG_NO_ROTATE)
  */
 QS_API qs_status qs_pack_weights(const void* w_bf16, int64_t N, int64_t K, int bits, unsigned flags,
@@ -101,8 +108,8 @@ QS_API qs_status qs_pack_weights(const void* w_bf16, int64_t N, int64_t K, int b
  *   x_bf16   [M, K] bf16, row-major
  *   bits     4, 6 or 8
  *   alpha    clip ratio in [2^-14, 1]
- *   flags    0 or QS_FLAG_NO_ROTATE
- *   x_packed [M, K/2] bytes (4 bits) or [M, K] bytes, written
+ *   flags    QS_FLAG_NO_ROTATE, QS_FLAG_BYTE_CODES or both
+ *   x_packed [M, K/2] bytes (4 bits, packed) or [M, K] bytes, written
  *   x_scale  [M] float, written (the per-token scale s_a)
  */
 QS_API qs_status qs_quant_act(const void* x_bf16, int64_t M, int64_t K, int bits, float alpha,
@@ -176,6 +183,17 @@ QS_API qs_status qs_linear(const void* x_bf16, int64_t M, int64_t K, float alpha
                            const void* w_packed, const float* w_scale, const void* bias_bf16,
                            int64_t N, int bits, void* workspace, int64_t workspace_bytes,
                            void* out_bf16, void* stream);
+
+/*
+ * qs_linear_ex — qs_linear_mixed with quantisation flags for the activations
+ * (0 or QS_FLAG_BYTE_CODES; the GEMM then reads 4-bit activation codes as
+ * bytes).  The workspace is qs_linear_workspace_bytes(M, K, s) with s = 8 when
+ * the activation codes are stored in bytes, else bits_x.
+ */
+QS_API qs_status qs_linear_ex(const void* x_bf16, int64_t M, int64_t K, float alpha, int bits_x,
+                              unsigned x_flags, const void* w_packed, const float* w_scale,
+                              int bits_w, const void* bias_bf16, int64_t N, void* workspace,
+                              int64_t workspace_bytes, void* out_bf16, void* stream);
 
 /*
  * qs_linear_mixed — qs_linear with the activations quantized at `bits_x` and

@@ -64,7 +64,7 @@ def test_pack_weights_validation(lib):
     assert f(A, -3, 512, 4, 0, B, C, NUL) == SHAPE
     assert f(A, 256, 0, 4, 0, B, C, NUL) == SHAPE
     assert f(A, 256, 65536 + 128, 4, 0, B, C, NUL) == RANGE
-    assert f(A, 256, 512, 4, 2, B, C, NUL) == RANGE
+    assert f(A, 256, 512, 4, 4, B, C, NUL) == RANGE          # unknown flag bit
     assert f(MIS, 256, 512, 4, 0, B, C, NUL) == ALIGN
 
 

@@ -385,3 +385,37 @@ def test_block_chain_full_size_sampled():
         g = _sampled_parity(d, bits, alpha, rows, cols)
         if L["name"] == "ffn_up":
             up_out = g["out"]
+
+
+# --------------------------------------------------------------------------- byte-stored 4-bit codes
+
+@pytest.mark.parametrize("M,K", [(1, 128), (129, 640), (33, 5120), (3, 16512)])
+def test_quant_act_byte_codes(M, K):
+    # QS_FLAG_BYTE_CODES: the same 4-bit codes, one per byte
+    d = I.make_shape(seed=2 * M + K, M=M, K=K, N=16, bits=4, outlier_factor=50.0)
+    for alpha in (1.0, 0.9, 0.003):
+        xp, xs = qs.quant_act(d["x"].cuda(), 4, alpha, qs.QS_FLAG_BYTE_CODES)
+        torch.cuda.synchronize()
+        q, s = O.quant_act(bits16(d["x"]), 4, alpha)
+        assert np.array_equal(xp.cpu().numpy().view(np.int8), q)
+        assert np.array_equal(xs.cpu().numpy().view(np.uint32), s.view(np.uint32))
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_w4a4_with_byte_activation_codes(M, N, K):
+    # W4A4 with the activation codes in bytes: the GEMM reads them as 8-bit
+    # storage; codes, accumulators and outputs equal the packed W4A4 layer's
+    alpha = 0.9
+    d = I.make_shape(seed=M + 5 * N + K, M=M, K=K, N=N, bits=4, alpha=alpha, outlier_factor=50.0)
+    x, w, b = d["x"].cuda(), d["w"].cuda(), d["bias"].cuda()
+    wp, ws = qs.pack_weights(w, 4)
+    xp, xs = qs.quant_act(x, 4, alpha, qs.QS_FLAG_BYTE_CODES)
+    out = qs.qlinear(xp, xs, wp, ws, b, 8, K, bits_w=4)
+    acc = qs.qgemm_s32(xp, wp, 8, K, bits_w=4)
+    one = qs.linear(x, wp, ws, b, 4, alpha, bits_w=4, x_flags=qs.QS_FLAG_BYTE_CODES)
+    torch.cuda.synchronize()
+    r = O.qlinear(bits16(d["x"]), bits16(d["w"]), bits16(d["bias"]), 4, alpha)
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), r["acc"])
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, r["out"])
+    assert np.array_equal(one.view(torch.int16).cpu().numpy().view(np.uint16), r["out"])
