@@ -13,3 +13,6 @@ from .bgr_oracle import (  # noqa: F401
     code_rowsums, grid_codes, grid_error, grid_from_bounds, least_squares_grid, pack_weights_bgr,
     qlinear_bgr, seq_sum,
 )
+from .sd4_oracle import (  # noqa: F401
+    SD4_BLOCK, SD4_DIALECTS, formatbook, linear_sd4, lut_tables, pack_codes, pack_meta,
+)
