@@ -32,7 +32,7 @@ EXPORTS = ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qlinear_mixed", 
            "qs_linear_mixed", "qs_linear_ex", "qs_linear_noalloc", "qs_pack_weights_bgr",
            "qs_quant_act_rowsum",
            "qs_qlinear_asym", "qs_qgemm_s32_asym", "qs_linear_bgr_workspace_bytes",
-           "qs_linear_bgr", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
+           "qs_linear_bgr", "qs_sd4_quant", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
            "qs_selftest_timeout", "qs_device_error", "qs_status_str", "qs_version")
 BITS = (4, 6, 8)
 QS_GBS_MAX_BLOCKS = 1024
@@ -81,6 +81,7 @@ def load() -> ctypes.CDLL:
     L.qs_linear_bgr_workspace_bytes.argtypes = [i64, i64, i32]
     L.qs_linear_bgr_workspace_bytes.restype = i64
     L.qs_linear_bgr.argtypes = [vp, i64, i64, f32, vp, vp, vp, vp, i64, i32, vp, i64, vp, vp]
+    L.qs_sd4_quant.argtypes = [vp, i64, i64, vp, vp, vp]
     L.qs_gbs_reset.argtypes = [vp, vp]
     L.qs_gbs_update.argtypes = [vp, vp, i64, f64, vp, vp]
     L.qs_linear_gbs.argtypes = [vp, i64, i64, f32, vp, vp, vp, vp, vp, i64, vp, vp, i64, vp, vp]
@@ -93,7 +94,8 @@ def load() -> ctypes.CDLL:
                  "qs_qgemm_s32", "qs_qgemm_s32_mixed", "qs_gelu_bf16", "qs_linear",
                  "qs_linear_mixed", "qs_linear_ex", "qs_linear_noalloc", "qs_pack_weights_bgr",
                  "qs_quant_act_rowsum", "qs_qlinear_asym", "qs_qgemm_s32_asym", "qs_linear_bgr",
-                 "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs", "qs_selftest_timeout",
+                 "qs_sd4_quant", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
+                 "qs_selftest_timeout",
                  "qs_device_error"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -307,6 +309,22 @@ def qs_linear_bgr(x, M, K, alpha, w_packed, w_scale, w_offset, bias, N, bits, wo
     _check(load().qs_linear_bgr(_p(x), M, K, float(alpha), _p(w_packed), _p(w_scale),
                                 _p(w_offset), _p(bias), N, bits, _p(workspace), workspace_bytes,
                                 _p(out), _s(stream)), "qs_linear_bgr")
+
+
+def qs_sd4_quant(x, rows, K, codes, meta, stream=None):
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(codes, torch.uint8, "codes")
+    _cuda(meta, torch.int16, "meta")
+    _check(load().qs_sd4_quant(_p(x), rows, K, _p(codes), _p(meta), _s(stream)), "qs_sd4_quant")
+
+
+def sd4_quant(x: torch.Tensor, stream=None):
+    """x bf16 [R, K] -> (codes uint8 [R, K/2], meta int16 [R, K/32]: e | d << 8)."""
+    R, K = x.shape
+    codes = torch.empty((R, K // 2), dtype=torch.uint8, device=x.device)
+    meta = torch.empty((R, K // 32), dtype=torch.int16, device=x.device)
+    qs_sd4_quant(x, R, K, codes, meta, stream)
+    return codes, meta
 
 
 def qs_gbs_reset(state, stream=None):

@@ -17,6 +17,7 @@
 #include "qs_host.cuh"
 #include "qs_glue.cuh"
 #include "qs_quant.cuh"
+#include "qs_sd4.cuh"
 
 namespace {
 
@@ -486,6 +487,27 @@ qs_status qs_linear_bgr(const void* x_bf16, int64_t M, int64_t K, float alpha,
   QS_TRY(qs_quant_act_rowsum(x_bf16, M, K, bits, alpha, 0u, xp, xs, xr, stream));
   return qs_qlinear_asym(xp, xs, xr, w_packed, w_scale, w_offset, bias_bf16, M, N, K, bits,
                          out_bf16, stream);
+}
+
+qs_status qs_sd4_quant(const void* x_bf16, int64_t rows, int64_t K, void* codes, uint16_t* meta,
+                       void* stream) {
+  if (!x_bf16 || !codes || !meta) return QS_ERR_NULL;
+  if (rows <= 0 || K <= 0 || K % 256 != 0) return QS_ERR_SHAPE;
+  if (K > QS_MAX_K || rows > QS_MAX_ROWS) return QS_ERR_RANGE;
+  if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(meta)) return QS_ERR_ALIGN;
+  QS_TRY(check_device_ptr(x_bf16));
+  QS_TRY(check_device_ptr(codes));
+  QS_TRY(check_device_ptr(meta));
+  const int sms = qs::sm_count();
+  if (sms <= 0) return QS_ERR_CUDA;
+  const int64_t chunks = rows * (K / 256);
+  int64_t grid = (chunks + qs::sd4::kWarps - 1) / qs::sd4::kWarps;
+  if (grid > static_cast<int64_t>(sms) * 4) grid = static_cast<int64_t>(sms) * 4;
+  qs::sd4::sd4_quant_kernel<<<static_cast<unsigned>(grid), qs::sd4::kThreads, 0,
+                              static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(x_bf16), rows, static_cast<int>(K),
+      static_cast<uint8_t*>(codes), meta);
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
 qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream) {

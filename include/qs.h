@@ -276,6 +276,32 @@ QS_API qs_status qs_linear_bgr(const void* x_bf16, int64_t M, int64_t K, float a
                                void* out_bf16, void* stream);
 
 /*
+ * SD4 (SemanticDialect "Resumen técnico" §2.A, mixed-format 4-bit blocks):
+ * each block of 32 consecutive elements of a row gets a power-of-two scale
+ * 2^e that normalises its magnitudes to [0, 2) and the one of 32 4-bit
+ * formats ("dialects") that fits it best, chosen through precomputed tables.
+ * The pages print no dialect values; this library's formatbook: a code is a
+ * sign bit (bit 3) and a level index i (bits 0-2); dialect d = 8a + s has the
+ * magnitudes L/8 with L0 = 0, top level t = 15 - a and, for i = 1..7,
+ * L = floor((2t(49p i + 7q i^2 + r i^3) + 2744) / 5488) made strictly
+ * increasing, (p,q,r) = shape s of (8,0,0) (6,2,0) (4,4,0) (3,5,0) (2,5,1)
+ * (0,8,0) (1,3,4) (0,3,5).  Block: e = max(floor(log2 amax), -126) (0 for a
+ * zero block); bin b = min(floor(|x| 2^(7-e)), 255); Qerror[d][b] =
+ * min_i (2b + 1 - 32 L_i)^2 and Qvalue[d][b] the minimising i; the block's
+ * dialect minimises sum Qerror (smallest d on ties); code = sign | Qvalue.
+ * Decoded value: (-1)^sign L/8 2^e (exact in bf16).
+ */
+
+/*
+ * qs_sd4_quant — SD4 codes of a bf16 matrix (activations or weights).
+ *   x_bf16  [rows, K] bf16, K % 256 == 0
+ *   codes   [rows, K/2] bytes, written: element 2j in the low nibble of byte j
+ *   meta    [rows, K/32] uint16, written: low byte e (int8), high byte d
+ */
+QS_API qs_status qs_sd4_quant(const void* x_bf16, int64_t rows, int64_t K, void* codes,
+                              uint16_t* meta, void* stream);
+
+/*
  * δ-guided bit switching (DVD-Quant "Resumen técnico" §2.C): per layer, the
  * normalised L1 change between consecutive outputs is accumulated, and the
  * layer's next step runs at 4 bits while the accumulated change is below

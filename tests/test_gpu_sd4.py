@@ -1,0 +1,57 @@
+"""GPU parity of the SD4 block format (SemanticDialect "Resumen técnico" §2.A)
+through the C ABI, against the oracle (this library's formatbook; parity
+against the pages is unpinned: they print no dialect values).
+
+Bar: codes and block words (exponent, dialect) bit-identical."""
+
+import numpy as np
+import pytest
+import torch
+
+import bit_quantized_linear_hadamard_b200 as qs
+from bit_quantized_linear_hadamard_b200 import build as qs_build
+from bit_quantized_linear_hadamard_b200 import inputs as I
+from oracle import qs_oracle as O
+from oracle import sd4_oracle as S
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    qs_build.build()
+    qs.load()
+    yield
+    assert qs.qs_device_error() == 0, "a kernel reported a bounded-wait timeout"
+
+
+def check_quant(x):
+    codes, meta = qs.sd4_quant(x.cuda())
+    torch.cuda.synchronize()
+    c, e, d = S.quantize_rows(I.bf16_bits(x))
+    got_meta = meta.cpu().numpy().view(np.uint16)
+    want_meta = S.pack_meta(e, d)
+    if not np.array_equal(got_meta, want_meta):
+        bad = np.argwhere(got_meta != want_meta)
+        raise AssertionError(f"block words differ at {len(bad)}, first {bad[:5].tolist()}")
+    assert np.array_equal(codes.cpu().numpy(), S.pack_codes(c)), "codes differ"
+
+
+@pytest.mark.parametrize("M,K", [(1, 256), (7, 512), (33, 5120), (5, 13824), (3, 16384)])
+def test_sd4_quant_bit_exact(M, K):
+    d = I.make_shape(seed=M + K, M=M, K=K, N=16, bits=4, outlier_factor=30.0)
+    check_quant(d["x"])
+    check_quant(d["w"][:M] if d["w"].shape[0] >= M else d["w"])
+
+
+def test_sd4_quant_edge_blocks():
+    x = torch.randn(6, 512, generator=torch.Generator().manual_seed(3))
+    x[0] = 0.0                                  # zero blocks
+    x[1] = -0.0                                 # negative zeros
+    x[2] = x[2] * 1e-39                         # subnormal blocks (exponent floor)
+    x[3, :32] = torch.tensor([15 / 8 * 4.0] * 32)   # one level repeated
+    x[4] = x[4] * 1e30                          # large exponents
+    x[5, ::2] = 0.0
+    check_quant(x.to(torch.bfloat16))
