@@ -510,6 +510,42 @@ qs_status qs_sd4_quant(const void* x_bf16, int64_t rows, int64_t K, void* codes,
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
+qs_status qs_sd4_linear(const void* x_codes, const uint16_t* x_meta, const void* w_codes,
+                        const uint16_t* w_meta, const void* bias_bf16, int64_t M, int64_t N,
+                        int64_t K, void* out_bf16, void* stream) {
+  namespace G = qs::sd4::gemm_sd4;
+  if (!x_codes || !x_meta || !w_codes || !w_meta || !out_bf16) return QS_ERR_NULL;
+  if (M <= 0 || N <= 0 || K <= 0 || K % 256 != 0 || N % 16 != 0) return QS_ERR_SHAPE;
+  if (K > QS_MAX_K || M > INT32_MAX || N > INT32_MAX) return QS_ERR_RANGE;
+  if (!aligned16(x_codes) || !aligned16(x_meta) || !aligned16(w_codes) || !aligned16(w_meta) ||
+      !aligned16(out_bf16) || (bias_bf16 && !aligned16(bias_bf16)))
+    return QS_ERR_ALIGN;
+  for (const void* p : {x_codes, static_cast<const void*>(x_meta), w_codes,
+                        static_cast<const void*>(w_meta), static_cast<const void*>(out_bf16)})
+    QS_TRY(check_device_ptr(p));
+  if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
+  CUtensorMap ca, cb, ma, mb;
+  const uint64_t code_row = static_cast<uint64_t>(K) / 2, meta_row = static_cast<uint64_t>(K) / 16;
+  if (!qs::make_tensor_map_2d(&ca, x_codes, code_row, static_cast<uint64_t>(M), G::BK / 2, G::BM,
+                              false) ||
+      !qs::make_tensor_map_2d(&cb, w_codes, code_row, static_cast<uint64_t>(N), G::BK / 2, G::BN,
+                              false) ||
+      !qs::make_tensor_map_2d(&ma, x_meta, meta_row, static_cast<uint64_t>(M), 16, G::BM, false) ||
+      !qs::make_tensor_map_2d(&mb, w_meta, meta_row, static_cast<uint64_t>(N), 16, G::BN, false))
+    return QS_ERR_CUDA;
+  if (cudaFuncSetAttribute(G::sd4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           G::kSmemBytes) != cudaSuccess)
+    return QS_ERR_CUDA;
+  const int sms = qs::sm_count();
+  if (sms <= 0) return QS_ERR_CUDA;
+  const int64_t tiles = ((M + G::BM - 1) / G::BM) * ((N + G::BN - 1) / G::BN);
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  G::sd4_gemm_kernel<<<grid, G::kThreads, G::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+      ca, cb, ma, mb, static_cast<const uint16_t*>(bias_bf16), static_cast<uint16_t*>(out_bf16),
+      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K));
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
 qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream) {
   if (!x_bf16 || !y_bf16) return QS_ERR_NULL;
   if (n <= 0) return QS_ERR_SHAPE;

@@ -23,7 +23,11 @@
 // (cost << 5 | d) picks the dialect; finally each lane writes its 8 codes.
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include <cstdint>
+
+#include "qs_ptx.cuh"
 
 namespace qs {
 namespace sd4 {
@@ -159,6 +163,315 @@ __global__ void __launch_bounds__(kThreads) sd4_quant_kernel(const uint16_t* __r
     __syncwarp();  // s_bins is rewritten by the next chunk
   }
 }
+
+// --------------------------------------------------------------------------
+// SD4 layer GEMM: out[m][n] = bf16(fl(sum_k x_hat[m][k] w_hat[n][k]) + bias[n])
+// with x_hat, w_hat the decoded SD4 values.  The decoded values are exact in
+// bf16, so the product runs on the tensor cores as a bf16 GEMM
+// (tcgen05.mma.kind::f16, binary32 accumulators in tensor memory): codes come
+// by TMA, 8 warps decode them into the 128-byte-swizzled operand tiles.
+//
+// Persistent, one CTA per SM, tiles of 128 x 256, 64 K elements per stage.
+// Warp roles: 0 TMA producer (codes every stage, block words every 4 stages:
+// a TMA row is at least 16 bytes = 8 block words = 256 elements); 1 TMEM
+// allocation and the MMA issuer; 2-5 epilogue; 6-13 decode.
+// --------------------------------------------------------------------------
+
+namespace gemm_sd4 {
+
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int kOpStages = 3, kPkStages = 4, kMetaSlots = 2;
+constexpr int kEpiWarps = 4, kDecWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps + kDecWarps);
+constexpr int kOpA = BM * BK * 2, kOpB = BN * BK * 2, kOpStage = kOpA + kOpB;  // bf16 tiles
+constexpr int kPkA = BM * BK / 2, kPkB = BN * BK / 2, kPkStage = kPkA + kPkB;  // code tiles
+constexpr int kMetaA = BM * 16, kMetaB = BN * 16, kMetaSlot = kMetaA + kMetaB;  // 8 words/row
+constexpr int kOffOp = 0;
+constexpr int kOffPk = kOffOp + kOpStages * kOpStage;
+constexpr int kOffMeta = kOffPk + kPkStages * kPkStage;
+constexpr int kOffBar = kOffMeta + kMetaSlots * kMetaSlot;
+constexpr int kNumBars = 2 * kPkStages + 2 * kMetaSlots + 2 * kOpStages + 4;
+constexpr int kOffEpi = (kOffBar + 8 * kNumBars + 15) / 16 * 16;  // bias of a tile
+constexpr int kOffLvl = kOffEpi + BN * 4;                            // level values
+constexpr int kOffMisc = kOffLvl + kDialects * 8 * 4;
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+constexpr int kTmemCols = 2 * BN;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+static_assert((BM + BN) * (BK / 16) % (32 * kDecWarps) == 0, "decode split");
+
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4)                                // D format: F32
+         | (1u << 7)                              // A: BF16
+         | (1u << 10)                             // B: BF16
+         | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+struct Bars {
+  uint32_t base;
+  __device__ uint32_t at(int i) const { return base + 8u * i; }
+  __device__ uint32_t pk_full(int s) const { return at(s); }
+  __device__ uint32_t pk_empty(int s) const { return at(kPkStages + s); }
+  __device__ uint32_t meta_full(int s) const { return at(2 * kPkStages + s); }
+  __device__ uint32_t meta_empty(int s) const { return at(2 * kPkStages + kMetaSlots + s); }
+  __device__ uint32_t op_full(int s) const { return at(2 * kPkStages + 2 * kMetaSlots + s); }
+  __device__ uint32_t op_empty(int s) const {
+    return at(2 * kPkStages + 2 * kMetaSlots + kOpStages + s);
+  }
+  __device__ uint32_t acc_full(int b) const {
+    return at(2 * kPkStages + 2 * kMetaSlots + 2 * kOpStages + b);
+  }
+  __device__ uint32_t acc_empty(int b) const {
+    return at(2 * kPkStages + 2 * kMetaSlots + 2 * kOpStages + 2 + b);
+  }
+};
+
+// Decodes 16 codes (8 bytes) of one block into 16 bf16 values (two 16-byte chunks).
+__device__ __forceinline__ void decode16(uint2 c, uint32_t word, const float* lvl, uint4& lo,
+                                         uint4& hi) {
+  const int e = static_cast<int8_t>(word & 0xFFu);
+  const int d = static_cast<int>(word >> 8) & 31;
+  const float sc = pow2f(e);
+  const float* L = lvl + 8 * d;
+  uint32_t out[8];
+  const uint32_t cw[2] = {c.x, c.y};
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t c0 = (cw[h] >> (8 * k)) & 0xFu, c1 = (cw[h] >> (8 * k + 4)) & 0xFu;
+      const float v0 = __fmul_rn(L[c0 & 7u], sc), v1 = __fmul_rn(L[c1 & 7u], sc);
+      const uint32_t s0 = __float_as_uint(v0) ^ ((c0 & 8u) << 28);
+      const uint32_t s1 = __float_as_uint(v1) ^ ((c1 & 8u) << 28);
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(s0), __uint_as_float(s1));
+      out[4 * h + k] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+  lo = make_uint4(out[0], out[1], out[2], out[3]);
+  hi = make_uint4(out[4], out[5], out[6], out[7]);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    sd4_gemm_kernel(const __grid_constant__ CUtensorMap tmCA, const __grid_constant__ CUtensorMap tmCB,
+                    const __grid_constant__ CUtensorMap tmMA, const __grid_constant__ CUtensorMap tmMB,
+                    const uint16_t* __restrict__ bias, uint16_t* __restrict__ out, int M, int N,
+                    int K) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+  uint8_t* sp = smem_raw + pad;
+  const uint32_t sbase = raw + pad;
+  Bars bars{sbase + kOffBar};
+  float* epi_b = reinterpret_cast<float*>(sp + kOffEpi);
+  float* lvl = reinterpret_cast<float*>(sp + kOffLvl);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sp + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = (N + BN - 1) / BN;
+  const int num_tiles = ((M + BM - 1) / BM) * n_tiles;
+  const int kblocks = K / BK;
+
+  for (int i = threadIdx.x; i < kDialects * 8; i += blockDim.x)
+    lvl[i] = static_cast<float>(level(i / 8, i % 8)) * 0.125f;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPkStages; ++s) {
+      mbar_init(bars.pk_full(s), 1);
+      mbar_init(bars.pk_empty(s), kDecWarps);
+    }
+    for (int s = 0; s < kMetaSlots; ++s) {
+      mbar_init(bars.meta_full(s), 1);
+      mbar_init(bars.meta_empty(s), kDecWarps);
+    }
+    for (int s = 0; s < kOpStages; ++s) {
+      mbar_init(bars.op_full(s), kDecWarps);
+      mbar_init(bars.op_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bars.acc_full(b), 1);
+      mbar_init(bars.acc_empty(b), kEpiWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {  // producer
+      int s = 0, ms = 0;
+      uint32_t ph = 0, mph = 0;
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if ((kb & 3) == 0) {
+            if (!mbar_wait_bounded(bars.meta_empty(ms), mph ^ 1u, abort_flag, kErrWaitProducer))
+              break;
+            const uint32_t dst = sbase + kOffMeta + ms * kMetaSlot;
+            mbar_arrive_expect_tx(bars.meta_full(ms), kMetaSlot);
+            tma_load_2d(dst, &tmMA, (kb / 4) * 16, m0, bars.meta_full(ms));
+            tma_load_2d(dst + kMetaA, &tmMB, (kb / 4) * 16, n0, bars.meta_full(ms));
+            if (++ms == kMetaSlots) { ms = 0; mph ^= 1u; }
+          }
+          if (!mbar_wait_bounded(bars.pk_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer)) break;
+          const uint32_t dst = sbase + kOffPk + s * kPkStage;
+          mbar_arrive_expect_tx(bars.pk_full(s), kPkStage);
+          tma_load_2d(dst, &tmCA, kb * (BK / 2), m0, bars.pk_full(s));
+          tma_load_2d(dst + kPkA, &tmCB, kb * (BK / 2), n0, bars.pk_full(s));
+          if (++s == kPkStages) { s = 0; ph ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // MMA issuer
+      constexpr uint32_t idesc = idesc_bf16(BM, BN);
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+        const int buf = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait_bounded(bars.acc_empty(buf), aph ^ 1u, abort_flag, kErrWaitMma)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(bars.op_full(s), ph, abort_flag, kErrWaitMma)) break;
+          tc_fence_after();
+          const uint32_t a0 = sbase + kOffOp + s * kOpStage;
+          const uint32_t b0 = a0 + kOpA;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_bf16(d, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc,
+                     (kb | kk) != 0);
+          mma_commit(bars.op_empty(s));
+          if (++s == kOpStages) { s = 0; ph ^= 1u; }
+        }
+        mma_commit(bars.acc_full(buf));
+      }
+    }
+  } else if (warp < 2 + kEpiWarps) {  // epilogue: TMEM lanes 32 * (warp & 3) ..
+    const int quad = warp & 3;
+    const int et = threadIdx.x - 64;
+    int it = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+      const int buf = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      for (int i = et; i < BN; i += 128) {
+        const int n = n0 + i;
+        epi_b[i] = (n < N && bias) ? __uint_as_float(static_cast<uint32_t>(bias[n]) << 16) : 0.f;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!mbar_wait_bounded(bars.acc_full(buf), aph, abort_flag, kErrWaitEpilogue)) break;
+      tc_fence_after();
+      const int row = m0 + 32 * quad + lane;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quad) << 16) +
+                             static_cast<uint32_t>(buf * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + 32 * c, r);
+        tmem_wait_ld();
+        const int n = n0 + 32 * c;
+        if (row < M && n < N) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float y0 = __fadd_rn(__uint_as_float(r[2 * j]), epi_b[32 * c + 2 * j]);
+            const float y1 = __fadd_rn(__uint_as_float(r[2 * j + 1]), epi_b[32 * c + 2 * j + 1]);
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
+            pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          uint16_t* dst = out + static_cast<int64_t>(row) * N + n;
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            if (n + 8 * v + 8 <= N)
+              *reinterpret_cast<uint4*>(dst + 8 * v) =
+                  make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.acc_empty(buf));
+    }
+  } else {  // decode warps
+    const int dt = threadIdx.x - 32 * (2 + kEpiWarps);  // 0 .. 255
+    int s = 0, so = 0, ms = 0;
+    uint32_t ph = 0, pho = 0, mph = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      for (int kb = 0; kb < kblocks; ++kb) {
+        if ((kb & 3) == 0 &&
+            !mbar_wait_bounded(bars.meta_full(ms), mph, abort_flag, kErrWaitUnpack))
+          break;
+        if (!mbar_wait_bounded(bars.pk_full(s), ph, abort_flag, kErrWaitUnpack)) break;
+        if (!mbar_wait_bounded(bars.op_empty(so), pho ^ 1u, abort_flag, kErrWaitUnpack)) break;
+        const uint8_t* pk = sp + kOffPk + s * kPkStage;
+        const uint8_t* mt = sp + kOffMeta + ms * kMetaSlot;
+        uint8_t* op = sp + kOffOp + so * kOpStage;
+        // tasks: (operand row r in 0..383, 16-element chunk c in 0..3)
+#pragma unroll
+        for (int j = 0; j < (BM + BN) * 4 / 256; ++j) {
+          const int task = dt + 256 * j;
+          const int r = task >> 2, c = task & 3;
+          const uint2 codes = *reinterpret_cast<const uint2*>(pk + r * (BK / 2) + c * 8);
+          // block word: block (kb % 4) * 2 + c / 2 of this row's 8-word slot row
+          const uint16_t word = *reinterpret_cast<const uint16_t*>(
+              mt + r * 16 + ((kb & 3) * 2 + (c >> 1)) * 2);
+          uint4 lo, hi;
+          decode16(codes, word, lvl, lo, hi);
+          uint8_t* rowp = op + r * 128;  // x rows 0..127, then W rows (operand B at +kOpA)
+          *reinterpret_cast<uint4*>(rowp + (((2 * c) ^ (r & 7)) << 4)) = lo;
+          *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (r & 7)) << 4)) = hi;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bars.op_full(so));
+          mbar_arrive(bars.pk_empty(s));
+          if ((kb & 3) == 3) mbar_arrive(bars.meta_empty(ms));
+        }
+        if (++s == kPkStages) { s = 0; ph ^= 1u; }
+        if (++so == kOpStages) { so = 0; pho ^= 1u; }
+        if ((kb & 3) == 3 && ++ms == kMetaSlots) { ms = 0; mph ^= 1u; }
+      }
+    }
+    // drain: the MMA's last releases of the operand stages have landed
+    if (lane == 0)
+      for (int i = 0; i < kOpStages; ++i) {
+        if (!mbar_wait_bounded(bars.op_empty(so), pho ^ 1u, abort_flag, kErrWaitUnpack)) break;
+        if (++so == kOpStages) { so = 0; pho ^= 1u; }
+      }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    const unsigned long long t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace gemm_sd4
 
 }  // namespace sd4
 }  // namespace qs

@@ -302,6 +302,19 @@ QS_API qs_status qs_sd4_quant(const void* x_bf16, int64_t rows, int64_t K, void*
                               uint16_t* meta, void* stream);
 
 /*
+ * qs_sd4_linear — the SD4 layer: out[m][n] = bf16(fl(sum_k x_hat w_hat) + bias[n])
+ * with x_hat, w_hat the decoded SD4 values of qs_sd4_quant(x) and
+ * qs_sd4_quant(W).  The decoded values are exact in bf16; the product runs on
+ * the tensor cores in bf16 with binary32 accumulation, so the sum is the exact
+ * one up to binary32 accumulation rounding (parity is checked within that
+ * bound).  K % 256 == 0, N % 16 == 0; bias NULL adds +0.0.
+ *   out_bf16  [M, N] bf16, written
+ */
+QS_API qs_status qs_sd4_linear(const void* x_codes, const uint16_t* x_meta, const void* w_codes,
+                               const uint16_t* w_meta, const void* bias_bf16, int64_t M,
+                               int64_t N, int64_t K, void* out_bf16, void* stream);
+
+/*
  * δ-guided bit switching (DVD-Quant "Resumen técnico" §2.C): per layer, the
  * normalised L1 change between consecutive outputs is accumulated, and the
  * layer's next step runs at 4 bits while the accumulated change is below

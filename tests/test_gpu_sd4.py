@@ -55,3 +55,48 @@ def test_sd4_quant_edge_blocks():
     x[4] = x[4] * 1e30                          # large exponents
     x[5, ::2] = 0.0
     check_quant(x.to(torch.bfloat16))
+
+
+def _layer(M, N, K, seed, bias=True):
+    d = I.make_shape(seed=seed, M=M, K=K, N=N, bits=4, outlier_factor=30.0)
+    x, w = d["x"].cuda(), d["w"].cuda()
+    b = d["bias"].cuda() if bias else None
+    cx, mx = qs.sd4_quant(x)
+    cw, mw = qs.sd4_quant(w)
+    out = qs.sd4_linear(cx, mx, cw, mw, b, K)
+    torch.cuda.synchronize()
+    return d, (cx, mx, cw, mw), out
+
+
+def _check_layer(d, dev, out, K, bias=True, exact=False):
+    r = S.linear_sd4(I.bf16_bits(d["x"]), I.bf16_bits(d["w"]),
+                     I.bf16_bits(d["bias"]) if bias else None, exact=exact)
+    cx, mx, cw, mw = dev
+    assert np.array_equal(cx.cpu().numpy(), S.pack_codes(r["codes_x"]))
+    assert np.array_equal(mw.cpu().numpy().view(np.uint16), S.pack_meta(r["exp_w"], r["dia_w"]))
+    got_bits = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    got = O.bf16_bits_to_f32(got_bits).astype(np.float64)
+    b = O.bf16_bits_to_f32(I.bf16_bits(d["bias"])).astype(np.float64) if bias else 0.0
+    exact_y = r["y"] + b
+    # binary32 accumulation of exact products: at most K * 2^-23 of sum |products|,
+    # plus the final bf16 rounding (one ulp of the result)
+    S_abs = np.abs(r["x_hat"]) @ np.abs(r["w_hat"]).T
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(got), 2.0 ** -126))) - 7)
+    allowed = K * 2.0 ** -23 * S_abs + ulp
+    err = np.abs(got - exact_y)
+    assert (err <= allowed).all(), f"max excess {np.max(err - allowed)}"
+    same = float((got_bits == r["out"]).mean())
+    assert same > 0.99, f"only {same:.4f} of outputs bit-identical to the oracle"
+    return same
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 16, 256), (127, 272, 256), (256, 512, 512),
+                                   (300, 768, 768), (513, 528, 1280)])
+def test_sd4_linear_matches_oracle(M, N, K):
+    d, dev, out = _layer(M, N, K, seed=M + N + K)
+    _check_layer(d, dev, out, K)
+
+
+def test_sd4_linear_exact_small_and_no_bias():
+    d, dev, out = _layer(3, 16, 256, seed=5, bias=False)
+    _check_layer(d, dev, out, 256, bias=False, exact=True)
