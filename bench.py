@@ -71,10 +71,16 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# the sources of the headline kernels and their launches (the activation
+# kernel, the GEMM, their shared helpers): counters taken on other sources
+# are not reported
+HEADLINE_SOURCES = ("qs_gemm.cuh", "qs_host.cuh", "qs_ptx.cuh", "qs_quant.cuh")
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_quantized_linear_hadamard_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in HEADLINE_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -381,6 +387,50 @@ def bgr_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
             "error_rows": rows}
 
 
+def sd4_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
+    """The Wan FFN layer in SD4 (per-32-element mixed 4-bit formats): the
+    weights quantised once, per step the activation quantiser and the
+    decode-bf16 tensor-core GEMM; the output error on the first `rows` tokens
+    against the unquantised layer, beside the W4A4 rotated layer's."""
+    cfg = I.WAN_FFN
+    d = I.make_layer(cfg)
+    M, K, N = cfg.M, cfg.K, cfg.N
+    with torch.cuda.stream(stream):
+        x, w, b = d["x"].to(dev), d["w"].to(dev), d["bias"].to(dev)
+        cw, mw = qs.sd4_quant(w, stream=stream)
+        cx = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        mx = torch.empty((M, K // 32), dtype=torch.int16, device=dev)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        for _ in range(warmup):
+            qs.qs_sd4_quant(x, M, K, cx, mx, stream)
+            qs.qs_sd4_linear(cx, mx, cw, mw, b, M, N, K, out, stream)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for e in ev:
+            e[0].record(stream)
+            qs.qs_sd4_quant(x, M, K, cx, mx, stream)
+            e[1].record(stream)
+            qs.qs_sd4_linear(cx, mx, cw, mw, b, M, N, K, out, stream)
+            e[2].record(stream)
+        stream.synchronize()
+        q = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+        g = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+        ref = x[:rows].double() @ w.double().t() + b.double()
+        wp, ws = qs.pack_weights(w, 4, stream=stream)
+        xp, xs = qs.quant_act(x[:rows].contiguous(), 4, cfg.alpha, stream=stream)
+        y4 = qs.qlinear(xp, xs, wp, ws, b, 4, K, stream=stream).double()
+        stream.synchronize()
+    err = lambda y: float((y - ref).norm() / ref.norm())  # noqa: E731
+    pk, _ = peaks()
+    gemm_tflops = cfg.ops / (g * 1e-3) / 1e12
+    quant_bytes = M * (2 * K + K // 2 + 2 * (K // 32))
+    return {"workload": cfg.name + "_sd4", "quant_ms": q, "gemm_ms": g,
+            "TOPS": cfg.ops / ((q + g) * 1e-3) / 1e12, "gemm_TFLOPS_bf16": gemm_tflops,
+            "gemm_frac_bf16_peak": gemm_tflops / pk["bf16_tflops"],
+            "quant_GBps": quant_bytes / (q * 1e-3) / 1e9,
+            "rel_err_sd4": err(out[:rows].double()), "rel_err_w4a4_rotated": err(y4),
+            "error_rows": rows}
+
+
 def quality(qs, torch, x, w, bias, bits, alpha, stream, rows=256):
     """Relative Frobenius error and SQNR of the layer against the unquantised
     binary64 product, with and without the Hadamard rotation (first `rows` tokens)."""
@@ -553,6 +603,7 @@ def main():
         extra["configs"] = all_configs(qs, torch, I, dev, stream)
         extra["gbs"] = gbs_sequence(qs, torch, I, dev, stream)
         extra["bgr"] = bgr_layer(qs, torch, I, dev, stream)
+        extra["sd4"] = sd4_layer(qs, torch, I, dev, stream)
     if rank == 0:
         pk, src = peaks()
         int8_peak = pk["bf16_tflops"] * INT8_PER_BF16

@@ -21,6 +21,9 @@
 
 namespace {
 
+using qs::gemm::dispatch_qgemm;
+using qs::gemm::launch_qgemm;
+
 constexpr unsigned kKnownFlags = QS_FLAG_NO_ROTATE | QS_FLAG_BYTE_CODES;
 constexpr float kMinAlpha = 1.0f / 16384.0f;  // keeps |u * inv| < 2^22
 
@@ -59,54 +62,6 @@ int64_t packed_row_bytes(int64_t K, int bits) { return K * qs::code_storage_bits
     const qs_status _s = (expr);   \
     if (_s != QS_OK) return _s;    \
   } while (0)
-
-// SA, SB: storage bits (4 or 8) of the x and W codes.  ASYM: weights on an
-// asymmetric grid (per-token code sums `rowsum`, per-channel `offset`).
-template <int SA, int SB, bool OUT_S32, bool ASYM = false>
-qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, const float* sw,
-                       const void* bias, int64_t M, int64_t N, int64_t K, void* out,
-                       cudaStream_t stream, const int* gate = nullptr, int gate_want = 0,
-                       const int* rowsum = nullptr, const int* offset = nullptr) {
-  using C = qs::gemm::Cfg<SA, SB>;
-  CUtensorMap ta, tb;
-  // each CTA of a pair loads 128 rows of x and 128 rows of W per stage; 8-bit
-  // tiles land 128-byte swizzled in the operand stage, 4-bit ones as plain rows
-  if (!qs::make_tensor_map_2d(&ta, xp, static_cast<uint64_t>(K) * SA / 8, static_cast<uint64_t>(M),
-                              qs::gemm::BK * SA / 8, qs::gemm::HM, SA == 8) ||
-      !qs::make_tensor_map_2d(&tb, wp, static_cast<uint64_t>(K) * SB / 8, static_cast<uint64_t>(N),
-                              qs::gemm::BK * SB / 8, qs::gemm::HN, SB == 8))
-    return QS_ERR_CUDA;
-  auto kern = qs::gemm::qgemm_kernel<SA, SB, OUT_S32, ASYM>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
-      cudaSuccess)
-    return QS_ERR_CUDA;
-  const int sms = qs::sm_count();
-  if (sms <= 0) return QS_ERR_CUDA;
-  // persistent clusters of two CTAs, at most one CTA per SM
-  const int64_t tiles = ((M + qs::gemm::BM - 1) / qs::gemm::BM) *
-                        ((N + qs::gemm::BN - 1) / qs::gemm::BN);
-  const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
-  if (pairs < 1) return QS_ERR_CUDA;
-  const int grid = static_cast<int>(2 * pairs);
-  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(
-      ta, tb, sa, sw, static_cast<const uint16_t*>(bias), out, static_cast<int>(M),
-      static_cast<int>(N), static_cast<int>(K), gate, gate_want, rowsum, offset);
-  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
-}
-
-template <bool OUT_S32>
-qs_status dispatch_qgemm(int bits_x, int bits_w, const void* xp, const float* sa, const void* wp,
-                         const float* sw, const void* bias, int64_t M, int64_t N, int64_t K,
-                         void* out, cudaStream_t stream) {
-  const int sx = qs::code_storage_bits(bits_x), sww = qs::code_storage_bits(bits_w);
-  if (sx == 4 && sww == 4)
-    return launch_qgemm<4, 4, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
-  if (sx == 8 && sww == 8)
-    return launch_qgemm<8, 8, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
-  if (sx == 8 && sww == 4)
-    return launch_qgemm<8, 4, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
-  return launch_qgemm<4, 8, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
-}
 
 qs_status check_gemm_args(const void* xp, const void* wp, const void* out, int64_t M, int64_t N,
                           int64_t K, int bits_x, int bits_w) {

@@ -64,6 +64,8 @@
 
 #include <cuda_bf16.h>
 
+#include "qs.h"
+#include "qs_host.cuh"
 #include "qs_ptx.cuh"
 
 namespace qs {
@@ -540,6 +542,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<SA, SB>::kThread
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, kTmemCols);
   }
+}
+
+// ---------------------------------------------------------------- launches
+// (host side, here with the kernel so that both are one unit of the source)
+
+// SA, SB: storage bits (4 or 8) of the x and W codes.  ASYM: weights on an
+// asymmetric grid (per-token code sums `rowsum`, per-channel `offset`).
+template <int SA, int SB, bool OUT_S32, bool ASYM = false>
+inline qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, const float* sw,
+                       const void* bias, int64_t M, int64_t N, int64_t K, void* out,
+                       cudaStream_t stream, const int* gate = nullptr, int gate_want = 0,
+                       const int* rowsum = nullptr, const int* offset = nullptr) {
+  using C = Cfg<SA, SB>;
+  CUtensorMap ta, tb;
+  // each CTA of a pair loads 128 rows of x and 128 rows of W per stage; 8-bit
+  // tiles land 128-byte swizzled in the operand stage, 4-bit ones as plain rows
+  if (!make_tensor_map_2d(&ta, xp, static_cast<uint64_t>(K) * SA / 8, static_cast<uint64_t>(M),
+                              BK * SA / 8, HM, SA == 8) ||
+      !make_tensor_map_2d(&tb, wp, static_cast<uint64_t>(K) * SB / 8, static_cast<uint64_t>(N),
+                              BK * SB / 8, HN, SB == 8))
+    return QS_ERR_CUDA;
+  auto kern = qgemm_kernel<SA, SB, OUT_S32, ASYM>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+      cudaSuccess)
+    return QS_ERR_CUDA;
+  const int sms = sm_count();
+  if (sms <= 0) return QS_ERR_CUDA;
+  // persistent clusters of two CTAs, at most one CTA per SM
+  const int64_t tiles = ((M + BM - 1) / BM) *
+                        ((N + BN - 1) / BN);
+  const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
+  if (pairs < 1) return QS_ERR_CUDA;
+  const int grid = static_cast<int>(2 * pairs);
+  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(
+      ta, tb, sa, sw, static_cast<const uint16_t*>(bias), out, static_cast<int>(M),
+      static_cast<int>(N), static_cast<int>(K), gate, gate_want, rowsum, offset);
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+template <bool OUT_S32>
+inline qs_status dispatch_qgemm(int bits_x, int bits_w, const void* xp, const float* sa,
+                                const void* wp,
+                         const float* sw, const void* bias, int64_t M, int64_t N, int64_t K,
+                         void* out, cudaStream_t stream) {
+  // storage per code: 4-bit codes in nibbles, 6- and 8-bit codes in bytes
+  const int sx = bits_x == 4 ? 4 : 8, sww = bits_w == 4 ? 4 : 8;
+  if (sx == 4 && sww == 4)
+    return launch_qgemm<4, 4, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
+  if (sx == 8 && sww == 8)
+    return launch_qgemm<8, 8, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
+  if (sx == 8 && sww == 4)
+    return launch_qgemm<8, 4, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
+  return launch_qgemm<4, 8, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
 }
 
 }  // namespace gemm

@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(kThreads) sd4_quant_kernel(const uint16_t* __r
                                                             uint8_t* __restrict__ codes,
                                                             uint16_t* __restrict__ meta) {
   __shared__ Tables tb;
-  __shared__ uint8_t s_bins[kWarps][8][kBlock];
+  __shared__ __align__(16) uint8_t s_bins[kWarps][8][kBlock];
   build_tables(&tb);
   __syncthreads();
 
@@ -136,13 +136,17 @@ __global__ void __launch_bounds__(kThreads) sd4_quant_kernel(const uint16_t* __r
         make_uint2(bins[0] | (bins[1] << 8) | (bins[2] << 16) | (static_cast<uint32_t>(bins[3]) << 24),
                    bins[4] | (bins[5] << 8) | (bins[6] << 16) | (static_cast<uint32_t>(bins[7]) << 24));
     __syncwarp();
-    // dialect choice: lane = dialect
+    // dialect choice: lane = dialect; the block's 32 bins come as two
+    // broadcast 16-byte reads, then 32 independent table reads
     int my_d = 0;
-#pragma unroll 1
+#pragma unroll 2
     for (int j = 0; j < 8; ++j) {
+      const uint4 q0 = *reinterpret_cast<const uint4*>(&s_bins[warp][j][0]);
+      const uint4 q1 = *reinterpret_cast<const uint4*>(&s_bins[warp][j][16]);
+      const uint32_t bw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
       uint32_t cost = 0;
-#pragma unroll 8
-      for (int k = 0; k < kBlock; ++k) cost += tb.qerr[s_bins[warp][j][k]][lane];
+#pragma unroll
+      for (int k = 0; k < kBlock; ++k) cost += tb.qerr[(bw[k >> 2] >> (8 * (k & 3))) & 0xFFu][lane];
       uint32_t key = (cost << 5) | static_cast<uint32_t>(lane);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) key = min(key, __shfl_xor_sync(0xffffffffu, key, off));
@@ -169,19 +173,19 @@ __global__ void __launch_bounds__(kThreads) sd4_quant_kernel(const uint16_t* __r
 // with x_hat, w_hat the decoded SD4 values.  The decoded values are exact in
 // bf16, so the product runs on the tensor cores as a bf16 GEMM
 // (tcgen05.mma.kind::f16, binary32 accumulators in tensor memory): codes come
-// by TMA, 8 warps decode them into the 128-byte-swizzled operand tiles.
+// by TMA, 12 warps decode them into the 128-byte-swizzled operand tiles.
 //
 // Persistent, one CTA per SM, tiles of 128 x 256, 64 K elements per stage.
 // Warp roles: 0 TMA producer (codes every stage, block words every 4 stages:
 // a TMA row is at least 16 bytes = 8 block words = 256 elements); 1 TMEM
-// allocation and the MMA issuer; 2-5 epilogue; 6-13 decode.
+// allocation and the MMA issuer; 2-5 epilogue; 6-17 decode.
 // --------------------------------------------------------------------------
 
 namespace gemm_sd4 {
 
 constexpr int BM = 128, BN = 256, BK = 64;
 constexpr int kOpStages = 3, kPkStages = 4, kMetaSlots = 2;
-constexpr int kEpiWarps = 4, kDecWarps = 8;
+constexpr int kEpiWarps = 4, kDecWarps = 12;
 constexpr int kThreads = 32 * (2 + kEpiWarps + kDecWarps);
 constexpr int kOpA = BM * BK * 2, kOpB = BN * BK * 2, kOpStage = kOpA + kOpB;  // bf16 tiles
 constexpr int kPkA = BM * BK / 2, kPkB = BN * BK / 2, kPkStage = kPkA + kPkB;  // code tiles
@@ -411,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(bars.acc_empty(buf));
     }
   } else {  // decode warps
-    const int dt = threadIdx.x - 32 * (2 + kEpiWarps);  // 0 .. 255
+    const int dt = threadIdx.x - 32 * (2 + kEpiWarps);  // 0 .. 32 kDecWarps - 1
     int s = 0, so = 0, ms = 0;
     uint32_t ph = 0, pho = 0, mph = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
@@ -426,8 +430,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* op = sp + kOffOp + so * kOpStage;
         // tasks: (operand row r in 0..383, 16-element chunk c in 0..3)
 #pragma unroll
-        for (int j = 0; j < (BM + BN) * 4 / 256; ++j) {
-          const int task = dt + 256 * j;
+        for (int j = 0; j < (BM + BN) * 4 / (32 * kDecWarps); ++j) {
+          const int task = dt + 32 * kDecWarps * j;
           const int r = task >> 2, c = task & 3;
           const uint2 codes = *reinterpret_cast<const uint2*>(pk + r * (BK / 2) + c * 8);
           // block word: block (kb % 4) * 2 + c / 2 of this row's 8-word slot row
