@@ -220,14 +220,16 @@ def test_qgemm_s32_mixed_extreme_codes_at_max_k(bx, bw):
 
 # --------------------------------------------------------------------------- whole layer
 
-def run_layer(d, bits, alpha, bias=True, bits_x=None):
-    """bits: the weights' code width; bits_x: the activations' (default bits)."""
+def run_layer(d, bits, alpha, bias=True, bits_x=None, x_flags=0):
+    """bits: the weights' code width; bits_x: the activations' (default bits);
+    x_flags: their storage (QS_FLAG_BYTE_CODES: 4-bit codes one per byte)."""
     bx = bits if bits_x is None else bits_x
+    sx = qs.storage_bits(bx, x_flags)
     x, w, b = d["x"].cuda(), d["w"].cuda(), d["bias"].cuda() if bias else None
     wp, ws = qs.pack_weights(w, bits)
-    xp, xs = qs.quant_act(x, bx, alpha)
-    out = qs.qlinear(xp, xs, wp, ws, b, bx, x.shape[1], bits_w=bits)
-    acc = qs.qgemm_s32(xp, wp, bx, x.shape[1], bits_w=bits)
+    xp, xs = qs.quant_act(x, bx, alpha, x_flags)
+    out = qs.qlinear(xp, xs, wp, ws, b, sx, x.shape[1], bits_w=bits)
+    acc = qs.qgemm_s32(xp, wp, sx, x.shape[1], bits_w=bits)
     torch.cuda.synchronize()
     return {"out": out, "acc": acc, "xp": xp, "xs": xs, "wp": wp, "ws": ws}
 
@@ -327,14 +329,14 @@ def test_gelu_matches_oracle():
 
 # --------------------------------------------------------------------------- full-size configs
 
-def _sampled_parity(d, bits, alpha, rows, cols, bits_x=None):
+def _sampled_parity(d, bits, alpha, rows, cols, bits_x=None, x_flags=0):
     bx = bits if bits_x is None else bits_x
-    g = run_layer(d, bits, alpha, bits_x=bx)
+    g = run_layer(d, bits, alpha, bits_x=bx, x_flags=x_flags)
     xb, wb, bb = bits16(d["x"][rows]), bits16(d["w"][cols]), bits16(d["bias"][cols])
     qa, sa = O.quant_act(xb, bx, alpha)
     qw, sw = O.pack_weights(wb, bits)
     assert np.array_equal(g["xs"].cpu().numpy()[rows].view(np.uint32), sa.view(np.uint32))
-    assert np.array_equal(g["xp"].cpu().numpy()[rows], O.pack(qa, bx))
+    assert np.array_equal(g["xp"].cpu().numpy()[rows], O.pack(qa, qs.storage_bits(bx, x_flags)))
     assert np.array_equal(g["ws"].cpu().numpy()[cols].view(np.uint32), sw.view(np.uint32))
     assert np.array_equal(g["wp"].cpu().numpy()[cols], O.pack(qw, bits))
     acc = O.int_gemm(qa, qw)
@@ -361,6 +363,16 @@ def test_full_size_config_sampled(cfg):
     d = I.make_layer(cfg)
     rows, cols = _samples(cfg.M, cfg.N, cfg.seed)
     _sampled_parity(d, cfg.bits, cfg.alpha, rows, cols, bits_x=cfg.act_bits)
+
+
+@pytest.mark.slow
+def test_full_size_wan_ffn_byte_codes_sampled():
+    # the benchmark's launch configuration: W4A4 with the activation codes one
+    # per byte, the mixed-storage GEMM
+    cfg = I.WAN_FFN
+    d = I.make_layer(cfg)
+    rows, cols = _samples(cfg.M, cfg.N, cfg.seed + 100)
+    _sampled_parity(d, cfg.bits, cfg.alpha, rows, cols, x_flags=qs.QS_FLAG_BYTE_CODES)
 
 
 @pytest.mark.slow
