@@ -49,6 +49,9 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--e2e-chunks", type=int, default=8,
+                   help="token chunks of the end-to-end step: the host->device copy, the layer "
+                        "and the device->host copy of consecutive chunks overlap on 3 streams")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extras", action="store_true",
                    help="skip the per-config table and the quality report")
@@ -567,34 +570,64 @@ def main():
     total_ms, quant_ms, gemm_ms = comb["times_ms"]
     ms_per_step, value = comb["ms_per_step"], comb["value"]
 
+    ref_rows = out[::1009].clone()  # the device step's output, to check the end-to-end one
     # ---- end to end through the same C ABI calls, inputs and result in pinned host memory
     x_host = d["x"].pin_memory()
     out_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
     e2e_steps = max(1, args.e2e_steps)
 
-    ws_bytes = qs.qs_linear_workspace_bytes(M, K, sx)
+    # chunks of tokens: chunk i's layer call (one public C call, qs_linear_ex)
+    # runs while chunk i+1 is copied in and chunk i-1 copied out
+    n_chunks = max(1, min(args.e2e_chunks, M))
+    rows_per = (M + n_chunks - 1) // n_chunks
+    spans = [(r0, min(M, r0 + rows_per)) for r0 in range(0, M, rows_per)]
+    ws_bytes = qs.qs_linear_workspace_bytes(rows_per, K, sx)
     workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
 
-    def e2e_step():  # one C call for the layer, host buffers in and out
-        x.copy_(x_host, non_blocking=True)
-        qs.qs_linear_ex(x, M, K, alpha, bx, x_flags, wp, ws, bits, bias, N, workspace, ws_bytes,
-                        out, stream)
-        out_host.copy_(out, non_blocking=True)
+    copied_out = [None] * len(spans)  # per chunk: the last copy-out of its output rows
 
-    with torch.cuda.stream(stream):
+    def e2e_step():
+        for i, (r0, r1) in enumerate(spans):
+            with torch.cuda.stream(s_in):
+                x[r0:r1].copy_(x_host[r0:r1], non_blocking=True)
+                got = torch.cuda.Event()
+                got.record(s_in)
+            stream.wait_event(got)
+            if copied_out[i] is not None:  # the previous step's rows have left the device
+                stream.wait_event(copied_out[i])
+            qs.qs_linear_ex(x[r0:r1], r1 - r0, K, alpha, bx, x_flags, wp, ws, bits, bias, N,
+                            workspace, ws_bytes, out[r0:r1], stream)
+            done = torch.cuda.Event()
+            done.record(stream)
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                out_host[r0:r1].copy_(out[r0:r1], non_blocking=True)
+                copied_out[i] = torch.cuda.Event()
+                copied_out[i].record(s_out)
+        # the next step's copies overwrite x: they wait for this step's layer calls
+        fin = torch.cuda.Event()
+        fin.record(stream)
+        s_in.wait_event(fin)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    for _ in range(e2e_steps):
         e2e_step()
-        stream.synchronize()
-        if world > 1:
-            dist.barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        stream.synchronize()
+    last = torch.cuda.Event()
+    last.record(s_out)
+    s_in.wait_event(last)   # e1 follows every copy, layer call and copy-out
+    e1.record(s_in)
+    torch.cuda.synchronize()
     e2e_ms = combine_ranks([e0.elapsed_time(e1) / e2e_steps], 1, ops_per_step, world,
                            dev)["times_ms"][0]
+    e2e_same = bool(torch.equal(out_host[::1009].to(dev).view(torch.int16),
+                                ref_rows.view(torch.int16)))
 
     extra = {}
     if world == 1 and not args.no_extras:
@@ -641,8 +674,9 @@ def main():
                     "h2d_bytes_per_step": x_host.numel() * 2,
                     "d2h_bytes_per_step": out_host.numel() * 2,
                     "ms_per_step": e2e_ms, "steps": e2e_steps,
-                    "call": "qs_linear_ex (C ABI: activation kernel + GEMM), pinned host x in, "
-                            "bf16 output back"},
+                    "call": "qs_linear_ex (C ABI: activation kernel + GEMM) per token chunk, pinned "
+                            "host x in, bf16 output back, copies overlapped with the layer",
+            "chunks": n_chunks, "output_equals_device_step": e2e_same},
             "clocks": clocks,
         }
         line.update(extra)
