@@ -470,7 +470,9 @@ def run_reference(args, rank, world):
         "dtype": "int4" if cfg.act_bits == cfg.bits == 4 else f"int{cfg.bits}w-int{cfg.act_bits}a",
         "data": "synthetic",
         "config": {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "bits_w": cfg.bits,
-                   "bits_x": cfg.act_bits, "alpha": cfg.alpha, "seed": cfg.seed,
+                   "bits_x": cfg.act_bits, "alpha": cfg.alpha,
+                   "act_codes": args.act_codes if cfg.act_bits == 4 else "packed",
+                   "seed": cfg.seed, "parallelism": f"replicas{world}",
                    "sample_rows_per_step": rows},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": f"{rows} tokens per step of the {cfg.M}-token workload, full "
