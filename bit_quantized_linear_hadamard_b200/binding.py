@@ -32,7 +32,8 @@ EXPORTS = ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qlinear_mixed", 
            "qs_linear_mixed", "qs_linear_ex", "qs_linear_noalloc", "qs_pack_weights_bgr",
            "qs_quant_act_rowsum",
            "qs_qlinear_asym", "qs_qgemm_s32_asym", "qs_linear_bgr_workspace_bytes",
-           "qs_linear_bgr", "qs_sd4_quant", "qs_sd4_linear", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
+           "qs_linear_bgr", "qs_sd4_quant", "qs_sd4_linear", "qs_sd4_decode",
+           "qs_sd4_linear_wdec", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
            "qs_selftest_timeout", "qs_device_error", "qs_status_str", "qs_version")
 BITS = (4, 6, 8)
 QS_GBS_MAX_BLOCKS = 1024
@@ -83,6 +84,8 @@ def load() -> ctypes.CDLL:
     L.qs_linear_bgr.argtypes = [vp, i64, i64, f32, vp, vp, vp, vp, i64, i32, vp, i64, vp, vp]
     L.qs_sd4_quant.argtypes = [vp, i64, i64, vp, vp, vp]
     L.qs_sd4_linear.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]
+    L.qs_sd4_decode.argtypes = [vp, vp, i64, i64, vp, vp]
+    L.qs_sd4_linear_wdec.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
     L.qs_gbs_reset.argtypes = [vp, vp]
     L.qs_gbs_update.argtypes = [vp, vp, i64, f64, vp, vp]
     L.qs_linear_gbs.argtypes = [vp, i64, i64, f32, vp, vp, vp, vp, vp, i64, vp, vp, i64, vp, vp]
@@ -95,7 +98,8 @@ def load() -> ctypes.CDLL:
                  "qs_qgemm_s32", "qs_qgemm_s32_mixed", "qs_gelu_bf16", "qs_linear",
                  "qs_linear_mixed", "qs_linear_ex", "qs_linear_noalloc", "qs_pack_weights_bgr",
                  "qs_quant_act_rowsum", "qs_qlinear_asym", "qs_qgemm_s32_asym", "qs_linear_bgr",
-                 "qs_sd4_quant", "qs_sd4_linear", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
+                 "qs_sd4_quant", "qs_sd4_linear", "qs_sd4_decode", "qs_sd4_linear_wdec",
+                 "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
                  "qs_selftest_timeout",
                  "qs_device_error"):
         getattr(L, name).restype = ctypes.c_int
@@ -333,6 +337,29 @@ def sd4_linear(x_codes, x_meta, w_codes, w_meta, bias, K: int, stream=None, out=
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x_codes.device)
     qs_sd4_linear(x_codes, x_meta, w_codes, w_meta, bias, M, N, K, out, stream)
+    return out
+
+
+def qs_sd4_decode(codes, meta, rows, K, out, stream=None):
+    _cuda(codes, torch.uint8, "codes")
+    _cuda(meta, torch.int16, "meta")
+    _cuda(out, torch.bfloat16, "out")
+    _check(load().qs_sd4_decode(_p(codes), _p(meta), rows, K, _p(out), _s(stream)), "qs_sd4_decode")
+
+
+def qs_sd4_linear_wdec(x_codes, x_meta, w, bias, M, N, K, out, stream=None):
+    for t, name, dt in ((x_codes, "x_codes", torch.uint8), (x_meta, "x_meta", torch.int16),
+                        (w, "w", torch.bfloat16), (bias, "bias", torch.bfloat16),
+                        (out, "out", torch.bfloat16)):
+        _cuda(t, dt, name)
+    _check(load().qs_sd4_linear_wdec(_p(x_codes), _p(x_meta), _p(w), _p(bias), M, N, K, _p(out),
+                                     _s(stream)), "qs_sd4_linear_wdec")
+
+
+def sd4_decode(codes, meta, stream=None):
+    R, K = codes.shape[0], codes.shape[1] * 2
+    out = torch.empty((R, K), dtype=torch.bfloat16, device=codes.device)
+    qs_sd4_decode(codes, meta, R, K, out, stream)
     return out
 
 

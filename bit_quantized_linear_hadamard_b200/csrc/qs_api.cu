@@ -101,6 +101,27 @@ void* noalloc_scratch_address() {
   return g_noalloc_addr[dev];
 }
 
+// Persistent launch of the SD4 GEMM: one CTA per SM at most.
+template <bool WDEC>
+qs_status launch_sd4_gemm(const CUtensorMap& ca, const CUtensorMap& cb, const CUtensorMap& ma,
+                          const CUtensorMap& mb, const CUtensorMap& wb, const void* bias,
+                          int64_t M, int64_t N, int64_t K, void* out, void* stream) {
+  namespace G = qs::sd4::gemm_sd4;
+  constexpr int smem = G::SCfg<WDEC>::kSmemBytes;
+  auto kern = G::sd4_gemm_kernel<WDEC>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return QS_ERR_CUDA;
+  const int sms = qs::sm_count();
+  if (sms <= 0) return QS_ERR_CUDA;
+  const int64_t tiles = ((M + G::BM - 1) / G::BM) * ((N + G::BN - 1) / G::BN);
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  kern<<<grid, G::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+      ca, cb, ma, mb, wb, static_cast<const uint16_t*>(bias), static_cast<uint16_t*>(out),
+      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K));
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -488,17 +509,52 @@ qs_status qs_sd4_linear(const void* x_codes, const uint16_t* x_meta, const void*
       !qs::make_tensor_map_2d(&ma, x_meta, meta_row, static_cast<uint64_t>(M), 16, G::BM, false) ||
       !qs::make_tensor_map_2d(&mb, w_meta, meta_row, static_cast<uint64_t>(N), 16, G::BN, false))
     return QS_ERR_CUDA;
-  if (cudaFuncSetAttribute(G::sd4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           G::kSmemBytes) != cudaSuccess)
-    return QS_ERR_CUDA;
+  return launch_sd4_gemm<false>(ca, cb, ma, mb, cb, bias_bf16, M, N, K, out_bf16, stream);
+}
+
+qs_status qs_sd4_decode(const void* codes, const uint16_t* meta, int64_t rows, int64_t K,
+                        void* out_bf16, void* stream) {
+  if (!codes || !meta || !out_bf16) return QS_ERR_NULL;
+  if (rows <= 0 || K <= 0 || K % 256 != 0) return QS_ERR_SHAPE;
+  if (K > QS_MAX_K || rows > QS_MAX_ROWS) return QS_ERR_RANGE;
+  if (!aligned16(codes) || !aligned16(meta) || !aligned16(out_bf16)) return QS_ERR_ALIGN;
+  for (const void* p : {codes, static_cast<const void*>(meta), static_cast<const void*>(out_bf16)})
+    QS_TRY(check_device_ptr(p));
   const int sms = qs::sm_count();
   if (sms <= 0) return QS_ERR_CUDA;
-  const int64_t tiles = ((M + G::BM - 1) / G::BM) * ((N + G::BN - 1) / G::BN);
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  G::sd4_gemm_kernel<<<grid, G::kThreads, G::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-      ca, cb, ma, mb, static_cast<const uint16_t*>(bias_bf16), static_cast<uint16_t*>(out_bf16),
-      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K));
+  const int64_t tasks = rows * (K / 16);
+  int64_t grid = (tasks + 255) / 256;
+  if (grid > static_cast<int64_t>(sms) * 8) grid = static_cast<int64_t>(sms) * 8;
+  qs::sd4::gemm_sd4::sd4_decode_kernel<<<static_cast<unsigned>(grid), 256, 0,
+                                         static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(codes), meta, rows, static_cast<int>(K),
+      static_cast<uint16_t*>(out_bf16));
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status qs_sd4_linear_wdec(const void* x_codes, const uint16_t* x_meta, const void* w_bf16,
+                             const void* bias_bf16, int64_t M, int64_t N, int64_t K,
+                             void* out_bf16, void* stream) {
+  namespace G = qs::sd4::gemm_sd4;
+  if (!x_codes || !x_meta || !w_bf16 || !out_bf16) return QS_ERR_NULL;
+  if (M <= 0 || N <= 0 || K <= 0 || K % 256 != 0 || N % 16 != 0) return QS_ERR_SHAPE;
+  if (K > QS_MAX_K || M > INT32_MAX || N > INT32_MAX) return QS_ERR_RANGE;
+  if (!aligned16(x_codes) || !aligned16(x_meta) || !aligned16(w_bf16) || !aligned16(out_bf16) ||
+      (bias_bf16 && !aligned16(bias_bf16)))
+    return QS_ERR_ALIGN;
+  for (const void* p : {x_codes, static_cast<const void*>(x_meta), w_bf16,
+                        static_cast<const void*>(out_bf16)})
+    QS_TRY(check_device_ptr(p));
+  if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
+  CUtensorMap ca, ma, wb;
+  if (!qs::make_tensor_map_2d(&ca, x_codes, static_cast<uint64_t>(K) / 2,
+                              static_cast<uint64_t>(M), G::BK / 2, G::BM, false) ||
+      !qs::make_tensor_map_2d(&ma, x_meta, static_cast<uint64_t>(K) / 16,
+                              static_cast<uint64_t>(M), 16, G::BM, false) ||
+      !qs::make_tensor_map_2d(&wb, w_bf16, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                              G::BK, G::BN, true, 2))
+    return QS_ERR_CUDA;
+  return launch_sd4_gemm<true>(ca, ca, ma, ma, wb, bias_bf16, M, N, K, out_bf16, stream);
 }
 
 qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream) {

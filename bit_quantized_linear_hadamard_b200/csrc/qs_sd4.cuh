@@ -184,24 +184,35 @@ __global__ void __launch_bounds__(kThreads) sd4_quant_kernel(const uint16_t* __r
 namespace gemm_sd4 {
 
 constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int kOpStages = 3, kPkStages = 4, kMetaSlots = 2;
+constexpr int kOpStages = 3, kPkStages = 3, kMetaSlots = 2;
 constexpr int kEpiWarps = 4, kDecWarps = 12;
 constexpr int kThreads = 32 * (2 + kEpiWarps + kDecWarps);
 constexpr int kOpA = BM * BK * 2, kOpB = BN * BK * 2, kOpStage = kOpA + kOpB;  // bf16 tiles
-constexpr int kPkA = BM * BK / 2, kPkB = BN * BK / 2, kPkStage = kPkA + kPkB;  // code tiles
-constexpr int kMetaA = BM * 16, kMetaB = BN * 16, kMetaSlot = kMetaA + kMetaB;  // 8 words/row
-constexpr int kOffOp = 0;
-constexpr int kOffPk = kOffOp + kOpStages * kOpStage;
-constexpr int kOffMeta = kOffPk + kPkStages * kPkStage;
-constexpr int kOffBar = kOffMeta + kMetaSlots * kMetaSlot;
+constexpr int kPkA = BM * BK / 2, kPkB = BN * BK / 2;                          // code tiles
+constexpr int kMetaA = BM * 16, kMetaB = BN * 16;                              // 8 words/row
 constexpr int kNumBars = 2 * kPkStages + 2 * kMetaSlots + 2 * kOpStages + 4;
-constexpr int kOffEpi = (kOffBar + 8 * kNumBars + 15) / 16 * 16;  // bias of a tile
-constexpr int kOffLvl = kOffEpi + BN * 4;                            // level values
-constexpr int kOffMisc = kOffLvl + kDialects * 8 * 4;
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 constexpr int kTmemCols = 2 * BN;
-static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
-static_assert((BM + BN) * (BK / 16) % (32 * kDecWarps) == 0, "decode split");
+
+// WDEC: the weights come already decoded (bf16, by qs_sd4_decode) and go by
+// TMA straight into their operand tile; only the activation rows are decoded.
+template <bool WDEC>
+struct SCfg {
+  static constexpr int kDecRows = WDEC ? BM : BM + BN;  // operand rows decoded per stage
+  static constexpr int kPkStage = WDEC ? kPkA : kPkA + kPkB;
+  static constexpr int kMetaSlot = WDEC ? kMetaA : kMetaA + kMetaB;
+  static constexpr int kOffOp = 0;
+  static constexpr int kOffPk = kOffOp + kOpStages * kOpStage;
+  static constexpr int kOffMeta = kOffPk + kPkStages * kPkStage;
+  static constexpr int kOffBar = kOffMeta + kMetaSlots * kMetaSlot;
+  static constexpr int kOffEpi = (kOffBar + 8 * kNumBars + 15) / 16 * 16;  // bias of a tile
+  static constexpr int kOffPair = kOffEpi + BN * 4;                          // pair table
+  static constexpr int kOffMisc = kOffPair + kDialects * 256 * 4;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  // arrivals completing an operand stage: the decode warps, plus the
+  // producer's arm of the weight tile's TMA bytes
+  static constexpr int kOpFullCount = kDecWarps + (WDEC ? 1 : 0);
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+};
 
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
   return (1u << 4)                                // D format: F32
@@ -240,13 +251,44 @@ struct Bars {
   }
 };
 
-// Decodes 16 codes (8 bytes) of one block into 16 bf16 values (two 16-byte chunks).
-__device__ __forceinline__ void decode16(uint2 c, uint32_t word, const float* lvl, uint4& lo,
-                                         uint4& hi) {
+// Decodes 16 codes (8 bytes) of one block into 16 bf16 values (two 16-byte
+// chunks).  Fast path: the pair table holds, for each dialect and code byte,
+// the two signed magnitudes L/8 as a bf16 pair; one bf16x2 multiply by 2^e
+// scales both exactly (a power of two, the result normal for e >= -123).
+// Blocks below that (results near the subnormal range) take the binary32 path.
+__device__ __forceinline__ void decode16_float(uint2 c, int e, const uint32_t* T, uint4& lo,
+                                               uint4& hi);
+
+__device__ __forceinline__ void decode16(uint2 c, uint32_t word, const uint32_t* pairs,
+                                         uint4& lo, uint4& hi) {
   const int e = static_cast<int8_t>(word & 0xFFu);
   const int d = static_cast<int>(word >> 8) & 31;
+  const uint32_t* T = pairs + 256 * d;
+  if (e < -123) {
+    decode16_float(c, e, T, lo, hi);
+    return;
+  }
+  const uint32_t sbits = static_cast<uint32_t>(e + 127) << 7;  // bf16 2^e
+  const uint32_t s2 = sbits | (sbits << 16);
+  const __nv_bfloat162 scale = *reinterpret_cast<const __nv_bfloat162*>(&s2);
+  uint32_t out[8];
+  const uint32_t cw[2] = {c.x, c.y};
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t v = T[(cw[h] >> (8 * k)) & 0xFFu];
+      const __nv_bfloat162 r = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&v), scale);
+      out[4 * h + k] = *reinterpret_cast<const uint32_t*>(&r);
+    }
+  lo = make_uint4(out[0], out[1], out[2], out[3]);
+  hi = make_uint4(out[4], out[5], out[6], out[7]);
+}
+
+__device__ __forceinline__ void decode16_float(uint2 c, int e, const uint32_t* T, uint4& lo,
+                                               uint4& hi) {
+  // T[code] (a byte whose high nibble is 0) holds the signed L/8 of `code` as bf16
   const float sc = pow2f(e);
-  const float* L = lvl + 8 * d;
   uint32_t out[8];
   const uint32_t cw[2] = {c.x, c.y};
 #pragma unroll
@@ -254,21 +296,25 @@ __device__ __forceinline__ void decode16(uint2 c, uint32_t word, const float* lv
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const uint32_t c0 = (cw[h] >> (8 * k)) & 0xFu, c1 = (cw[h] >> (8 * k + 4)) & 0xFu;
-      const float v0 = __fmul_rn(L[c0 & 7u], sc), v1 = __fmul_rn(L[c1 & 7u], sc);
-      const uint32_t s0 = __float_as_uint(v0) ^ ((c0 & 8u) << 28);
-      const uint32_t s1 = __float_as_uint(v1) ^ ((c1 & 8u) << 28);
-      const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(s0), __uint_as_float(s1));
+      const float v0 = __fmul_rn(__uint_as_float(T[c0] << 16), sc);
+      const float v1 = __fmul_rn(__uint_as_float(T[c1] << 16), sc);
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
       out[4 * h + k] = *reinterpret_cast<const uint32_t*>(&b2);
     }
   lo = make_uint4(out[0], out[1], out[2], out[3]);
   hi = make_uint4(out[4], out[5], out[6], out[7]);
 }
 
+template <bool WDEC>
 __global__ void __launch_bounds__(kThreads, 1)
     sd4_gemm_kernel(const __grid_constant__ CUtensorMap tmCA, const __grid_constant__ CUtensorMap tmCB,
                     const __grid_constant__ CUtensorMap tmMA, const __grid_constant__ CUtensorMap tmMB,
-                    const uint16_t* __restrict__ bias, uint16_t* __restrict__ out, int M, int N,
-                    int K) {
+                    const __grid_constant__ CUtensorMap tmWB, const uint16_t* __restrict__ bias,
+                    uint16_t* __restrict__ out, int M, int N, int K) {
+  using C = SCfg<WDEC>;
+  constexpr int kOffOp = C::kOffOp, kOffPk = C::kOffPk, kOffMeta = C::kOffMeta;
+  constexpr int kOffBar = C::kOffBar, kOffEpi = C::kOffEpi, kOffPair = C::kOffPair;
+  constexpr int kOffMisc = C::kOffMisc, kPkStage = C::kPkStage, kMetaSlot = C::kMetaSlot;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
@@ -276,7 +322,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = raw + pad;
   Bars bars{sbase + kOffBar};
   float* epi_b = reinterpret_cast<float*>(sp + kOffEpi);
-  float* lvl = reinterpret_cast<float*>(sp + kOffLvl);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sp + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + kOffMisc + 4);
 
@@ -285,8 +330,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_tiles = ((M + BM - 1) / BM) * n_tiles;
   const int kblocks = K / BK;
 
-  for (int i = threadIdx.x; i < kDialects * 8; i += blockDim.x)
-    lvl[i] = static_cast<float>(level(i / 8, i % 8)) * 0.125f;
+  uint32_t* pairs = reinterpret_cast<uint32_t*>(sp + kOffPair);
+  for (int i = threadIdx.x; i < kDialects * 256; i += blockDim.x) {
+    const int d = i / 256, b = i % 256;
+    uint32_t h[2];
+    for (int j = 0; j < 2; ++j) {
+      const int code = (b >> (4 * j)) & 15;
+      // L/8 is exact in bf16: the binary32 value's top 16 bits
+      const float v = static_cast<float>(level(d, code & 7)) * 0.125f;
+      h[j] = (__float_as_uint(v) >> 16) | ((code & 8) ? 0x8000u : 0u);
+    }
+    pairs[i] = h[0] | (h[1] << 16);
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPkStages; ++s) {
       mbar_init(bars.pk_full(s), 1);
@@ -297,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars.meta_empty(s), kDecWarps);
     }
     for (int s = 0; s < kOpStages; ++s) {
-      mbar_init(bars.op_full(s), kDecWarps);
+      mbar_init(bars.op_full(s), C::kOpFullCount);
       mbar_init(bars.op_empty(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -318,8 +373,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {  // producer
-      int s = 0, ms = 0;
-      uint32_t ph = 0, mph = 0;
+      int s = 0, ms = 0, so = 0;
+      uint32_t ph = 0, mph = 0, pho = 0;
       for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
         const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
         for (int kb = 0; kb < kblocks; ++kb) {
@@ -329,15 +384,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t dst = sbase + kOffMeta + ms * kMetaSlot;
             mbar_arrive_expect_tx(bars.meta_full(ms), kMetaSlot);
             tma_load_2d(dst, &tmMA, (kb / 4) * 16, m0, bars.meta_full(ms));
-            tma_load_2d(dst + kMetaA, &tmMB, (kb / 4) * 16, n0, bars.meta_full(ms));
+            if (!WDEC) tma_load_2d(dst + kMetaA, &tmMB, (kb / 4) * 16, n0, bars.meta_full(ms));
             if (++ms == kMetaSlots) { ms = 0; mph ^= 1u; }
           }
           if (!mbar_wait_bounded(bars.pk_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer)) break;
           const uint32_t dst = sbase + kOffPk + s * kPkStage;
           mbar_arrive_expect_tx(bars.pk_full(s), kPkStage);
           tma_load_2d(dst, &tmCA, kb * (BK / 2), m0, bars.pk_full(s));
-          tma_load_2d(dst + kPkA, &tmCB, kb * (BK / 2), n0, bars.pk_full(s));
+          if (!WDEC) tma_load_2d(dst + kPkA, &tmCB, kb * (BK / 2), n0, bars.pk_full(s));
           if (++s == kPkStages) { s = 0; ph ^= 1u; }
+          if (WDEC) {  // decoded weights: TMA into the operand stage's B tile
+            if (!mbar_wait_bounded(bars.op_empty(so), pho ^ 1u, abort_flag, kErrWaitProducer))
+              break;
+            const uint32_t ob = sbase + kOffOp + so * kOpStage + kOpA;
+            mbar_arrive_expect_tx(bars.op_full(so), kOpB);
+            tma_load_2d(ob, &tmWB, kb * BK, n0, bars.op_full(so));
+            if (++so == kOpStages) { so = 0; pho ^= 1u; }
+          }
         }
       }
     }
@@ -430,15 +493,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* op = sp + kOffOp + so * kOpStage;
         // tasks: (operand row r in 0..383, 16-element chunk c in 0..3)
 #pragma unroll
-        for (int j = 0; j < (BM + BN) * 4 / (32 * kDecWarps); ++j) {
+        for (int j = 0; j < (C::kDecRows * 4 + 32 * kDecWarps - 1) / (32 * kDecWarps); ++j) {
           const int task = dt + 32 * kDecWarps * j;
+          if (task >= C::kDecRows * 4) break;
           const int r = task >> 2, c = task & 3;
           const uint2 codes = *reinterpret_cast<const uint2*>(pk + r * (BK / 2) + c * 8);
           // block word: block (kb % 4) * 2 + c / 2 of this row's 8-word slot row
           const uint16_t word = *reinterpret_cast<const uint16_t*>(
               mt + r * 16 + ((kb & 3) * 2 + (c >> 1)) * 2);
           uint4 lo, hi;
-          decode16(codes, word, lvl, lo, hi);
+          decode16(codes, word, pairs, lo, hi);
           uint8_t* rowp = op + r * 128;  // x rows 0..127, then W rows (operand B at +kOpA)
           *reinterpret_cast<uint4*>(rowp + (((2 * c) ^ (r & 7)) << 4)) = lo;
           *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (r & 7)) << 4)) = hi;
@@ -472,6 +536,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// Decoded values of an SD4 matrix, bf16 [rows, K]: one thread per 16 elements
+// (8 code bytes and the block word) through the same pair table.
+__global__ void __launch_bounds__(256) sd4_decode_kernel(const uint8_t* __restrict__ codes,
+                                                         const uint16_t* __restrict__ meta,
+                                                         int64_t rows, int K,
+                                                         uint16_t* __restrict__ out) {
+  __shared__ uint32_t pairs[kDialects * 256];
+  for (int i = threadIdx.x; i < kDialects * 256; i += blockDim.x) {
+    const int d = i / 256, b = i % 256;
+    uint32_t h[2];
+    for (int j = 0; j < 2; ++j) {
+      const int code = (b >> (4 * j)) & 15;
+      const float v = static_cast<float>(level(d, code & 7)) * 0.125f;
+      h[j] = (__float_as_uint(v) >> 16) | ((code & 8) ? 0x8000u : 0u);
+    }
+    pairs[i] = h[0] | (h[1] << 16);
+  }
+  __syncthreads();
+  const int64_t per_row = K / 16;
+  const int64_t n = rows * per_row;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < n;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = t / per_row;
+    const int c = static_cast<int>(t % per_row);  // 16-element chunk of the row
+    const uint2 cw = *reinterpret_cast<const uint2*>(codes + row * (K / 2) + c * 8);
+    const uint32_t word = meta[row * (K / 32) + c / 2];
+    uint4 lo, hi;
+    decode16(cw, word, pairs, lo, hi);
+    uint4* dst = reinterpret_cast<uint4*>(out + row * static_cast<int64_t>(K) + c * 16);
+    dst[0] = lo;
+    dst[1] = hi;
   }
 }
 

@@ -315,6 +315,24 @@ QS_API qs_status qs_sd4_linear(const void* x_codes, const uint16_t* x_meta, cons
                                int64_t N, int64_t K, void* out_bf16, void* stream);
 
 /*
+ * qs_sd4_decode — the decoded values of an SD4 matrix, bf16 [rows, K] (exact).
+ * Offline use: decoding the weights once lets qs_sd4_linear_wdec load them by
+ * TMA straight into the GEMM's operand tiles (only the activations are then
+ * decoded per call), at 2 bytes per weight instead of half a byte.
+ */
+QS_API qs_status qs_sd4_decode(const void* codes, const uint16_t* meta, int64_t rows, int64_t K,
+                               void* out_bf16, void* stream);
+
+/*
+ * qs_sd4_linear_wdec — qs_sd4_linear with the weights given decoded
+ * (qs_sd4_decode of qs_sd4_quant(W)); the same arithmetic, bit-identical
+ * outputs.  w_bf16 [N, K].
+ */
+QS_API qs_status qs_sd4_linear_wdec(const void* x_codes, const uint16_t* x_meta,
+                                    const void* w_bf16, const void* bias_bf16, int64_t M,
+                                    int64_t N, int64_t K, void* out_bf16, void* stream);
+
+/*
  * δ-guided bit switching (DVD-Quant "Resumen técnico" §2.C): per layer, the
  * normalised L1 change between consecutive outputs is accumulated, and the
  * layer's next step runs at 4 bits while the accumulated change is below

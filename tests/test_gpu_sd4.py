@@ -100,3 +100,46 @@ def test_sd4_linear_matches_oracle(M, N, K):
 def test_sd4_linear_exact_small_and_no_bias():
     d, dev, out = _layer(3, 16, 256, seed=5, bias=False)
     _check_layer(d, dev, out, 256, bias=False, exact=True)
+
+
+def test_sd4_linear_extreme_exponents():
+    # activation blocks with exponents down to -123 (the lowest exponent the
+    # pair-table decode scales exactly) and up to +100; weights ordinary, so
+    # every product stays a normal binary32 number
+    g = torch.Generator().manual_seed(17)
+    M, N, K = 64, 272, 512
+    x = torch.randn(M, K, generator=g)
+    scales = torch.tensor([2.0 ** -122, 2.0 ** -115, 2.0 ** -60, 1.0, 2.0 ** 40, 2.0 ** 100])
+    x = x * scales[torch.arange(M) % len(scales)][:, None]
+    w = torch.randn(N, K, generator=g) * 0.5
+    d = {"x": x.to(torch.bfloat16), "w": w.to(torch.bfloat16),
+         "bias": torch.zeros(N, dtype=torch.bfloat16)}
+    cx, mx = qs.sd4_quant(d["x"].cuda())
+    cw, mw = qs.sd4_quant(d["w"].cuda())
+    out = qs.sd4_linear(cx, mx, cw, mw, None, K)
+    torch.cuda.synchronize()
+    e = (mx.cpu().numpy().view(np.uint16) & 0xFF).astype(np.int8)
+    assert e.min() >= -123 and e.min() <= -120 and e.max() >= 100
+    _check_layer(d, (cx, mx, cw, mw), out, K, bias=False)
+
+
+@pytest.mark.parametrize("R,K", [(5, 256), (129, 5120)])
+def test_sd4_decode_exact(R, K):
+    d = I.make_shape(seed=R + K, M=R, K=K, N=16, bits=4, outlier_factor=30.0)
+    codes, meta = qs.sd4_quant(d["x"].cuda())
+    dec = qs.sd4_decode(codes, meta)
+    torch.cuda.synchronize()
+    c, e, dd = S.quantize_rows(I.bf16_bits(d["x"]))
+    want = O.f32_to_bf16_bits(S.dequantize(c, e, dd).astype(np.float32))
+    assert np.array_equal(dec.view(torch.int16).cpu().numpy().view(np.uint16), want)
+
+
+@pytest.mark.parametrize("M,N,K", [(127, 272, 256), (300, 768, 768), (513, 528, 1280)])
+def test_sd4_linear_with_decoded_weights_is_identical(M, N, K):
+    d, dev, out = _layer(M, N, K, seed=3 * M + N)
+    cx, mx, cw, mw = dev
+    wdec = qs.sd4_decode(cw, mw)
+    out2 = torch.empty_like(out)
+    qs.qs_sd4_linear_wdec(cx, mx, wdec, d["bias"].cuda(), M, N, K, out2)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
