@@ -417,6 +417,18 @@ def sd4_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
         stream.synchronize()
         q = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
         g = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+        # the weights decoded once (offline): only the activations decoded per call
+        wdec = qs.sd4_decode(cw, mw, stream=stream)
+        out2 = torch.empty_like(out)
+        qs.qs_sd4_linear_wdec(cx, mx, wdec, b, M, N, K, out2, stream)
+        e2 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e2[0].record(stream)
+        for _ in range(steps):
+            qs.qs_sd4_linear_wdec(cx, mx, wdec, b, M, N, K, out2, stream)
+        e2[1].record(stream)
+        stream.synchronize()
+        g2 = e2[0].elapsed_time(e2[1]) / steps
+        same = bool(torch.equal(out.view(torch.int16), out2.view(torch.int16)))
         ref = x[:rows].double() @ w.double().t() + b.double()
         wp, ws = qs.pack_weights(w, 4, stream=stream)
         xp, xs = qs.quant_act(x[:rows].contiguous(), 4, cfg.alpha, stream=stream)
@@ -429,6 +441,9 @@ def sd4_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
     return {"workload": cfg.name + "_sd4", "quant_ms": q, "gemm_ms": g,
             "TOPS": cfg.ops / ((q + g) * 1e-3) / 1e12, "gemm_TFLOPS_bf16": gemm_tflops,
             "gemm_frac_bf16_peak": gemm_tflops / pk["bf16_tflops"],
+            "gemm_decoded_weights_ms": g2,
+            "gemm_decoded_weights_TFLOPS_bf16": cfg.ops / (g2 * 1e-3) / 1e12,
+            "decoded_weights_output_identical": same,
             "quant_GBps": quant_bytes / (q * 1e-3) / 1e9,
             "rel_err_sd4": err(out[:rows].double()), "rel_err_w4a4_rotated": err(y4),
             "error_rows": rows}
