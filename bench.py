@@ -24,6 +24,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import statistics
 import os
 import statistics
 import subprocess
@@ -195,10 +196,25 @@ class OracleSample:
         dt = self.run(rows)
         ops = 2.0 * rows * self.N * self.K
         return {"value": ops / dt / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+                "host": host_info(),
                 "sample": f"first {rows} of {self.x.shape[0]} tokens, full K={self.K}, "
                           f"N={self.N} (quant_act + int GEMM + epilogue; numpy, one host "
                           f"thread), {dt:.2f} s",
                 "tokens_per_s": rows / dt}
+
+
+def host_info() -> dict:
+    """The host the oracle ran on: its core count and CPU model."""
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
 
 
 def combine_ranks(times_ms, steps, ops_per_step, world, device="cpu"):
@@ -490,6 +506,7 @@ def run_reference(args, rank, world):
                    "seed": cfg.seed, "parallelism": f"replicas{world}",
                    "sample_rows_per_step": rows},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "host": host_info(),
                          "sample": f"{rows} tokens per step of the {cfg.M}-token workload, full "
                                    f"K and N, numpy oracle on one host thread"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -577,8 +594,10 @@ def main():
     if world > 1:
         dist.barrier()
     total_ms = ev[0][0].elapsed_time(ev[-1][2])
-    quant_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
-    gemm_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    quant_each = [e[0].elapsed_time(e[1]) for e in ev]
+    gemm_each = [e[1].elapsed_time(e[2]) for e in ev]
+    quant_ms = sum(quant_each) / args.steps
+    gemm_ms = sum(gemm_each) / args.steps
     if qs.qs_device_error(stream) != 0:
         raise SystemExit("kernel wait timed out in the timed region")
 
@@ -686,6 +705,8 @@ def main():
                                "algorithmic_bytes": quant_bytes,
                                "peak_source": f"{src}: hbm_gbs"},
             "kernels_ms": {"quant": quant_ms, "gemm": gemm_ms},
+            "kernels_ms_median": {"quant": statistics.median(quant_each),
+                                  "gemm": statistics.median(gemm_each)},
             "gpu_launches": 2 * args.steps,
             "e2e": {"value": ops_per_step * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": x_host.numel() * 2,
