@@ -14,5 +14,6 @@ from .bgr_oracle import (  # noqa: F401
     qlinear_bgr, seq_sum,
 )
 from .sd4_oracle import (  # noqa: F401
-    SD4_BLOCK, SD4_DIALECTS, formatbook, linear_sd4, lut_tables, pack_codes, pack_meta,
+    SD4_BLOCK, SD4_DIALECTS, decompose_rows, formatbook, linear_sd4, linear_sd4_decomp,
+    lut_tables, pack_codes, pack_decomp, pack_meta, quantize_values,
 )

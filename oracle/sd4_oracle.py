@@ -49,6 +49,16 @@ Readings:
 * Layer: y = sum_k x_hat[m,k] w_hat[n,k] exactly, rounded to binary64 and
   then to binary32, out = bf16_rne(fl(y + bias)).  The tensor-core path accumulates in binary32,
   so the device result is compared within a bound derived in the tests.
+
+Activation decomposition ("Resumen técnico" §2.B): a salient row A is split
+into its SD4 value Q(A) and the residual Delta = A - deq(Q(A)); Delta is
+quantised again with the same format and the layer uses A ~ Q(A) + Q(Delta).
+Readings: Delta is the exact difference (it is a binary32 number: see
+decompose_rows); its SD4 blocks are the same 32 columns as A's; the salient
+rows are given by the caller (the pages pick them from attention scores of a
+trained model, which this library does not have); their output is
+bf16_rne(fl(sum_k (x_hat + delta_hat)[m,k] w_hat[n,k] + bias)) with the exact
+sum, and the other rows are those of the plain layer.
 """
 
 from __future__ import annotations
@@ -100,7 +110,13 @@ def block_exponent(amax: float) -> int:
 def quantize_rows(x_bits: np.ndarray):
     """SD4 codes [R, K] (uint8 nibbles 0..15), exponents [R, K/32] (int),
     dialects [R, K/32] (int)."""
-    x = bf16_bits_to_f32(np.asarray(x_bits)).astype(np.float64)
+    return quantize_values(bf16_bits_to_f32(np.asarray(x_bits)).astype(np.float64))
+
+
+def quantize_values(x: np.ndarray):
+    """quantize_rows on binary64 values (each exactly a binary32 number, as the
+    residuals of the activation decomposition are)."""
+    x = np.asarray(x, np.float64)
     R, K = x.shape
     if K % SD4_BLOCK:
         raise ValueError("K must be a multiple of 32")
@@ -173,3 +189,54 @@ def linear_sd4(x_bits, w_bits, bias_bits=None, exact: bool = True):
     out = f32_to_bf16_bits((y32 + b[None, :]).astype(np.float32))
     return {"codes_x": cx, "exp_x": ex, "dia_x": dx, "codes_w": cw, "exp_w": ew, "dia_w": dw,
             "x_hat": xh, "w_hat": wh, "y": y, "out": out}
+
+
+def decompose_rows(x_bits, rows):
+    """Q(A) and Q(Delta) of the rows `rows` of x (bf16 bits [M, K]).
+
+    Delta = A - x_hat is exact in binary64 and is a binary32 number: a nonzero
+    x_hat is a multiple of 2^(e-3) with |x_hat| < 2^(e+1), and an element that
+    rounds to a nonzero level has |A| >= 2^(e-4), so A is a multiple of
+    2^(e-11) and |Delta| < 2^(e+2) spans at most 13 bits; an element that
+    rounds to level 0 has Delta = A."""
+    x = bf16_bits_to_f32(np.asarray(x_bits)).astype(np.float64)[np.asarray(rows, np.int64)]
+    cx, ex, dx = quantize_values(x)
+    x_hat = dequantize(cx, ex, dx)
+    delta = x - x_hat
+    cd, ed, dd = quantize_values(delta)
+    return {"codes_x": cx, "exp_x": ex, "dia_x": dx, "x_hat": x_hat, "delta": delta,
+            "codes_d": cd, "exp_d": ed, "dia_d": dd, "d_hat": dequantize(cd, ed, dd)}
+
+
+def pack_decomp(dec) -> tuple[np.ndarray, np.ndarray]:
+    """The decomposed rows as rows of 2K codes: [Q(A) | Q(Delta)] (codes two
+    per byte, one block word per 32 codes)."""
+    codes = np.concatenate([dec["codes_x"], dec["codes_d"]], axis=1)
+    exps = np.concatenate([dec["exp_x"], dec["exp_d"]], axis=1)
+    dias = np.concatenate([dec["dia_x"], dec["dia_d"]], axis=1)
+    return pack_codes(codes), pack_meta(exps, dias)
+
+
+def linear_sd4_decomp(x_bits, w_bits, bias_bits, rows, exact: bool = True):
+    """The SD4 layer with the salient rows `rows` decomposed: those rows use
+    x_hat + delta_hat (the element sum is exact in binary64), the others are
+    linear_sd4's."""
+    r = linear_sd4(x_bits, w_bits, bias_bits, exact=exact)
+    rows = np.asarray(rows, np.int64)
+    dec = decompose_rows(x_bits, rows)
+    xt = dec["x_hat"] + dec["d_hat"]
+    if len(rows) == 0:
+        y = np.zeros((0, r["w_hat"].shape[0]))
+    elif exact:
+        y = np.array([[float(v) for v in row] for row in exact_products(xt, r["w_hat"])])
+    else:
+        y = xt @ r["w_hat"].T
+    b = (np.zeros(r["w_hat"].shape[0], np.float32) if bias_bits is None
+         else bf16_bits_to_f32(np.asarray(bias_bits)))
+    out = r["out"].copy()
+    yrows = r["y"].copy()
+    if len(rows):
+        out[rows] = f32_to_bf16_bits((y.astype(np.float32) + b[None, :]).astype(np.float32))
+        yrows[rows] = y
+    r.update({"decomp": dec, "out": out, "y": yrows, "x_tilde": xt, "rows": rows})
+    return r

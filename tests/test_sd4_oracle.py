@@ -143,6 +143,106 @@ def pin_layer_exact_sum(s=S):
             assert r["out"][m, n] == want
 
 
+def _check_nearest_levels(s, vals, dec, exps, dias):
+    """Brute force: every block's dialect minimises the table cost over the 32
+    dialects and every value `dec` (what the layer uses) is that dialect's
+    nearest level (signed)."""
+    L = s.formatbook()
+    qerr, _ = s.lut_tables(L)
+    R, K = vals.shape
+    for r in range(R):
+        for j in range(K // 32):
+            blk = vals[r, 32 * j:32 * j + 32]
+            e, d = int(exps[r, j]), int(dias[r, j])
+            amax = float(np.max(np.abs(blk)))
+            assert amax == 0 or 1.0 <= amax * 2.0 ** -e < 2.0
+            bins = [min(int(math.floor(abs(v) * 2.0 ** -e * 128)), 255) for v in blk]
+            costs = [sum(int(qerr[dd, b]) for b in bins) for dd in range(32)]
+            assert d == costs.index(min(costs))
+            levels = [int(l) / 8 * 2.0 ** e for l in L[d]]
+            for k in range(32):
+                got = dec[r, 32 * j + k]
+                assert abs(got) in levels
+                assert abs(abs(blk[k]) - abs(got)) == min(abs(abs(blk[k]) - lv) for lv in levels)
+                assert got == 0 or (got < 0) == (blk[k] < 0)
+
+
+def _two_scale_rows(seed, R, K, d_res=13):
+    """Rows of blocks x = a + b: a in {0, +-15/8} 2^e, b = +-L/8 2^(e-4) with L
+    levels of dialect d_res (its top level in every block) where a != 0, else 0.
+    x is bf16-exact ((240 +- L) 2^(e-7)); Q(A) = a (15/8 is the nearest level in
+    every dialect whose top level is 15, and those dialects cost least);
+    Delta = b has block exponent e-4 and is exactly one dialect's levels."""
+    rng = np.random.default_rng(seed)
+    L = S.formatbook()
+    x = np.zeros((R, K))
+    a_all = np.zeros((R, K))
+    for r in range(R):
+        for j in range(K // 32):
+            e = int(rng.integers(-20, 20))
+            nz = rng.choice(32, 20, replace=False)
+            a = np.zeros(32)
+            a[nz] = rng.choice([-1.0, 1.0], 20) * 15 / 8 * 2.0 ** e
+            b = np.zeros(32)
+            idx = rng.integers(0, 8, 20)
+            idx[0] = 7
+            b[nz] = rng.choice([-1.0, 1.0], 20) * L[d_res, idx] / 8 * 2.0 ** (e - 4)
+            x[r, 32 * j:32 * j + 32] = a + b
+            a_all[r, 32 * j:32 * j + 32] = a
+    bits = _bf16(x)
+    assert np.array_equal(O.bf16_bits_to_f32(bits).astype(np.float64), x)
+    return bits, x, a_all
+
+
+def pin_decomposition_residual_is_exact_and_requantised(s=S):
+    """Delta = A - x_hat exactly (a binary32 number); Q(A) of the salient rows
+    is the plain quantisation; Q(Delta) is a nearest-level SD4 quantisation of
+    Delta (brute force); the residual step moves no element away from A (level
+    0 is in every dialect) and cuts the total error."""
+    x = _rows(11, 5, 256, outliers=4)
+    rows = [4, 0, 2, 2]
+    dec = s.decompose_rows(x, rows)
+    xf = O.bf16_bits_to_f32(x).astype(np.float64)[rows]
+    assert np.array_equal(dec["x_hat"] + dec["delta"], xf)
+    assert np.array_equal(dec["delta"].astype(np.float32).astype(np.float64), dec["delta"])
+    _check_nearest_levels(s, xf, dec["x_hat"], dec["exp_x"], dec["dia_x"])
+    _check_nearest_levels(s, dec["delta"], dec["d_hat"], dec["exp_d"], dec["dia_d"])
+    assert np.array_equal(s.dequantize(dec["codes_d"], dec["exp_d"], dec["dia_d"]), dec["d_hat"])
+    err0 = np.abs(xf - dec["x_hat"])
+    err1 = np.abs(xf - dec["x_hat"] - dec["d_hat"])
+    assert (err1 <= err0).all() and err1.sum() < 0.5 * err0.sum()
+
+
+def pin_decomposition_reconstructs_two_scale_blocks(s=S):
+    """On blocks that are a sum of levels at two scales, Q(A) is the coarse
+    part and Q(Delta) the fine part, so x_hat + delta_hat = A exactly."""
+    bits, x, a = _two_scale_rows(5, 3, 256)
+    dec = s.decompose_rows(bits, [0, 1, 2])
+    assert np.array_equal(dec["x_hat"], a)
+    assert np.array_equal(dec["x_hat"] + dec["d_hat"], x)
+
+
+def pin_decomposed_layer(s=S):
+    """No salient rows: the plain layer.  Two-scale rows (reconstructed
+    exactly) as the salient rows: their accumulators are the exact products of
+    A itself with w_hat (brute force), the other rows keep x_hat's."""
+    bits, x, _ = _two_scale_rows(9, 4, 64)
+    w = _rows(3, 3, 64)
+    b = _bf16(np.array([0.25, -1.0, 0.0]))
+    plain = s.linear_sd4(bits, w, b)
+    r0 = s.linear_sd4_decomp(bits, w, b, [])
+    assert np.array_equal(r0["out"], plain["out"])
+    r = s.linear_sd4_decomp(bits, w, b, [2, 0])
+    bf = O.bf16_bits_to_f32(b)
+    for m in range(4):
+        for n in range(3):
+            src = x[m] if m in (0, 2) else plain["x_hat"][m]
+            exact = sum(Fraction(float(src[k])) * Fraction(float(r["w_hat"][n, k]))
+                        for k in range(64))
+            assert r["y"][m, n] == float(exact)
+            assert r["out"][m, n] == O.f32_to_bf16_bits(np.float32(np.float32(float(exact)) + bf[n]))
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
@@ -174,7 +274,27 @@ def _formatbook_no_raise():
     return L
 
 
+def _decompose_with(residual):
+    def decompose(x_bits, rows):
+        x = O.bf16_bits_to_f32(np.asarray(x_bits)).astype(np.float64)[np.asarray(rows, np.int64)]
+        cx, ex, dx = S.quantize_values(x)
+        x_hat = S.dequantize(cx, ex, dx)
+        delta = residual(x, x_hat)
+        cd, ed, dd = S.quantize_values(delta)
+        d_hat = S.dequantize(cd, ed, dd) if residual is not _unquantised else delta
+        return {"codes_x": cx, "exp_x": ex, "dia_x": dx, "x_hat": x_hat, "delta": delta,
+                "codes_d": cd, "exp_d": ed, "dia_d": dd, "d_hat": d_hat}
+    return decompose
+
+
+def _unquantised(x, x_hat):
+    return x - x_hat
+
+
 MUTANTS = {
+    "residual_sign_flipped": ("decompose_rows", _decompose_with(lambda x, xh: xh - x)),
+    "residual_of_the_input": ("decompose_rows", _decompose_with(lambda x, xh: x)),
+    "residual_left_unquantised": ("decompose_rows", _decompose_with(_unquantised)),
     "lut_levels_in_sixteenths": ("lut_tables", _lut_half_scale),
     "exponent_rounded_up": ("block_exponent", _exponent_ceil),
     "levels_not_strictly_increasing": ("formatbook", _formatbook_no_raise),
