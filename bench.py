@@ -24,7 +24,6 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
-import statistics
 import os
 import statistics
 import subprocess
@@ -410,7 +409,9 @@ def sd4_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
     """The Wan FFN layer in SD4 (per-32-element mixed 4-bit formats): the
     weights quantised once, per step the activation quantiser and the
     decode-bf16 tensor-core GEMM; the output error on the first `rows` tokens
-    against the unquantised layer, beside the W4A4 rotated layer's."""
+    against the unquantised layer, beside the W4A4 rotated layer's.  Also the
+    activation decomposition of a seeded 1/16 of the tokens (their residual
+    quantiser and the 2K-long GEMM over them) and its error on those tokens."""
     cfg = I.WAN_FFN
     d = I.make_layer(cfg)
     M, K, N = cfg.M, cfg.K, cfg.N
@@ -445,6 +446,36 @@ def sd4_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
         stream.synchronize()
         g2 = e2[0].elapsed_time(e2[1]) / steps
         same = bool(torch.equal(out.view(torch.int16), out2.view(torch.int16)))
+        # activation decomposition of the salient tokens (a seeded 1/16 of them)
+        srows = I.salient_rows(M, cfg.seed)
+        S_ = len(srows)
+        rt = torch.tensor(srows, dtype=torch.int32, device=dev)
+        c2 = torch.empty((S_, K), dtype=torch.uint8, device=dev)
+        m2 = torch.empty((S_, K // 16), dtype=torch.int16, device=dev)
+        out3 = out2.clone()
+        for _ in range(warmup):
+            qs.qs_sd4_quant_decomp(x, M, K, rt, S_, c2, m2, stream)
+            qs.qs_sd4_linear_decomp(c2, m2, rt, S_, None, None, wdec, b, M, N, K, out3, stream)
+        e3 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for e in e3:
+            e[0].record(stream)
+            qs.qs_sd4_quant_decomp(x, M, K, rt, S_, c2, m2, stream)
+            e[1].record(stream)
+            qs.qs_sd4_linear_decomp(c2, m2, rt, S_, None, None, wdec, b, M, N, K, out3, stream)
+            e[2].record(stream)
+        stream.synchronize()
+        dq = sum(e[0].elapsed_time(e[1]) for e in e3) / steps
+        dg = sum(e[1].elapsed_time(e[2]) for e in e3) / steps
+        sel = rt[:rows].long()
+        ref_s = x[sel].double() @ w.double().t() + b.double()
+        err_s = lambda y: float((y - ref_s).norm() / ref_s.norm())  # noqa: E731
+        decomp = {"salient_rows": S_, "salient_fraction": S_ / M, "quant_decomp_ms": dq,
+                  "gemm_decomp_ms": dg,
+                  "gemm_decomp_TFLOPS_bf16": 2.0 * S_ * 2 * K * N / (dg * 1e-3) / 1e12,
+                  "layer_ms_decoded_weights": q + g2 + dq + dg,
+                  "rel_err_salient_plain": err_s(out2[sel].double()),
+                  "rel_err_salient_decomposed": err_s(out3[sel].double()),
+                  "error_rows": int(sel.numel())}
         ref = x[:rows].double() @ w.double().t() + b.double()
         wp, ws = qs.pack_weights(w, 4, stream=stream)
         xp, xs = qs.quant_act(x[:rows].contiguous(), 4, cfg.alpha, stream=stream)
@@ -462,7 +493,7 @@ def sd4_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
             "decoded_weights_output_identical": same,
             "quant_GBps": quant_bytes / (q * 1e-3) / 1e9,
             "rel_err_sd4": err(out[:rows].double()), "rel_err_w4a4_rotated": err(y4),
-            "error_rows": rows}
+            "error_rows": rows, "decomposition": decomp}
 
 
 def quality(qs, torch, x, w, bias, bits, alpha, stream, rows=256):

@@ -105,7 +105,9 @@ void* noalloc_scratch_address() {
 template <bool WDEC>
 qs_status launch_sd4_gemm(const CUtensorMap& ca, const CUtensorMap& cb, const CUtensorMap& ma,
                           const CUtensorMap& mb, const CUtensorMap& wb, const void* bias,
-                          int64_t M, int64_t N, int64_t K, void* out, void* stream) {
+                          int64_t M, int64_t N, int64_t K, void* out, void* stream,
+                          int64_t kb_wrap = 0, const int32_t* out_rows = nullptr,
+                          int64_t out_M = 0) {
   namespace G = qs::sd4::gemm_sd4;
   constexpr int smem = G::SCfg<WDEC>::kSmemBytes;
   auto kern = G::sd4_gemm_kernel<WDEC>;
@@ -118,7 +120,9 @@ qs_status launch_sd4_gemm(const CUtensorMap& ca, const CUtensorMap& cb, const CU
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   kern<<<grid, G::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(
       ca, cb, ma, mb, wb, static_cast<const uint16_t*>(bias), static_cast<uint16_t*>(out),
-      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K));
+      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+      static_cast<int>(kb_wrap > 0 ? kb_wrap : K / G::BK), out_rows,
+      static_cast<int>(out_rows ? out_M : M));
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
@@ -557,6 +561,76 @@ qs_status qs_sd4_linear_wdec(const void* x_codes, const uint16_t* x_meta, const 
   return launch_sd4_gemm<true>(ca, ca, ma, ma, wb, bias_bf16, M, N, K, out_bf16, stream);
 }
 
+qs_status qs_sd4_quant_decomp(const void* x_bf16, int64_t M, int64_t K, const int32_t* rows,
+                              int64_t S, void* codes2, uint16_t* meta2, void* stream) {
+  if (!x_bf16 || !rows || !codes2 || !meta2) return QS_ERR_NULL;
+  if (M <= 0 || S <= 0 || K <= 0 || K % 256 != 0) return QS_ERR_SHAPE;
+  if (2 * K > QS_MAX_K || M > INT32_MAX || S > QS_MAX_ROWS) return QS_ERR_RANGE;
+  if (!aligned16(x_bf16) || !aligned16(codes2) || !aligned16(meta2) ||
+      (reinterpret_cast<uintptr_t>(rows) & 3u))
+    return QS_ERR_ALIGN;
+  for (const void* p : {x_bf16, static_cast<const void*>(rows), static_cast<const void*>(codes2),
+                        static_cast<const void*>(meta2)})
+    QS_TRY(check_device_ptr(p));
+  const int sms = qs::sm_count();
+  if (sms <= 0) return QS_ERR_CUDA;
+  const int64_t chunks = S * (K / 256);
+  int64_t grid = (chunks + qs::sd4::kWarps - 1) / qs::sd4::kWarps;
+  if (grid > static_cast<int64_t>(sms) * 4) grid = static_cast<int64_t>(sms) * 4;
+  qs::sd4::sd4_decomp_kernel<<<static_cast<unsigned>(grid), qs::sd4::kThreads, 0,
+                               static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(x_bf16), M, static_cast<int>(K), rows, S,
+      static_cast<uint8_t*>(codes2), meta2);
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status qs_sd4_linear_decomp(const void* codes2, const uint16_t* meta2, const int32_t* rows,
+                               int64_t S, const void* w_codes, const uint16_t* w_meta,
+                               const void* w_bf16, const void* bias_bf16, int64_t M, int64_t N,
+                               int64_t K, void* out_bf16, void* stream) {
+  namespace G = qs::sd4::gemm_sd4;
+  if (!codes2 || !meta2 || !rows || !out_bf16) return QS_ERR_NULL;
+  if (!w_bf16 && (!w_codes || !w_meta)) return QS_ERR_NULL;
+  if (M <= 0 || S <= 0 || N <= 0 || K <= 0 || K % 256 != 0 || N % 16 != 0) return QS_ERR_SHAPE;
+  if (2 * K > QS_MAX_K || M > INT32_MAX || S > INT32_MAX || N > INT32_MAX) return QS_ERR_RANGE;
+  if (!aligned16(codes2) || !aligned16(meta2) || !aligned16(out_bf16) ||
+      (reinterpret_cast<uintptr_t>(rows) & 3u) || (bias_bf16 && !aligned16(bias_bf16)))
+    return QS_ERR_ALIGN;
+  if (w_bf16 ? !aligned16(w_bf16) : (!aligned16(w_codes) || !aligned16(w_meta)))
+    return QS_ERR_ALIGN;
+  for (const void* p : {codes2, static_cast<const void*>(meta2), static_cast<const void*>(rows),
+                        static_cast<const void*>(out_bf16)})
+    QS_TRY(check_device_ptr(p));
+  if (w_bf16) {
+    QS_TRY(check_device_ptr(w_bf16));
+  } else {
+    QS_TRY(check_device_ptr(w_codes));
+    QS_TRY(check_device_ptr(w_meta));
+  }
+  if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
+  // A: S rows of 2K codes; B: the weights' K, walked twice
+  const uint64_t K2 = 2 * static_cast<uint64_t>(K);
+  CUtensorMap ca, ma, cb, mb, wb;
+  if (!qs::make_tensor_map_2d(&ca, codes2, K2 / 2, static_cast<uint64_t>(S), G::BK / 2, G::BM,
+                              false) ||
+      !qs::make_tensor_map_2d(&ma, meta2, K2 / 16, static_cast<uint64_t>(S), 16, G::BM, false))
+    return QS_ERR_CUDA;
+  if (w_bf16) {
+    if (!qs::make_tensor_map_2d(&wb, w_bf16, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                                G::BK, G::BN, true, 2))
+      return QS_ERR_CUDA;
+    return launch_sd4_gemm<true>(ca, ca, ma, ma, wb, bias_bf16, S, N, K2, out_bf16, stream,
+                                 K / G::BK, rows, M);
+  }
+  if (!qs::make_tensor_map_2d(&cb, w_codes, static_cast<uint64_t>(K) / 2,
+                              static_cast<uint64_t>(N), G::BK / 2, G::BN, false) ||
+      !qs::make_tensor_map_2d(&mb, w_meta, static_cast<uint64_t>(K) / 16,
+                              static_cast<uint64_t>(N), 16, G::BN, false))
+    return QS_ERR_CUDA;
+  return launch_sd4_gemm<false>(ca, cb, ma, mb, cb, bias_bf16, S, N, K2, out_bf16, stream,
+                                K / G::BK, rows, M);
+}
+
 qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream) {
   if (!x_bf16 || !y_bf16) return QS_ERR_NULL;
   if (n <= 0) return QS_ERR_SHAPE;
@@ -603,7 +677,7 @@ qs_status qs_device_error(void* stream) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(qs::g_error_word, &zero, sizeof(zero)) != cudaSuccess)
       return QS_ERR_CUDA;
-    return QS_ERR_TIMEOUT;
+    return (word & ~static_cast<unsigned int>(qs::kErrIndex)) ? QS_ERR_TIMEOUT : QS_ERR_RANGE;
   }
   return QS_OK;
 }

@@ -18,6 +18,7 @@ enum : unsigned int {
   kErrWaitMma = 1u << 2,
   kErrWaitEpilogue = 1u << 3,
   kErrWaitProducer = 1u << 4,
+  kErrIndex = 1u << 6,  // a row index given on the device was out of range
 };
 
 // A wait that has not completed after this many nanoseconds gives up.

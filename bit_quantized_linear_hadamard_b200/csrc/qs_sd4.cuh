@@ -38,11 +38,14 @@ constexpr int kBins = 256;
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
+// (p, q, r) of the shapes, the ramp, square and cube weights (sum 8), one
+// nibble per shape (shape 0 in the low nibble): (8,0,0) (6,2,0) (4,4,0)
+// (3,5,0) (2,5,1) (0,8,0) (1,3,4) (0,3,5).  Held in registers, not in a
+// local-memory table.
+constexpr uint32_t kShapeP = 0x01023468u, kShapeQ = 0x33855420u, kShapeR = 0x54010000u;
+
 __host__ __device__ constexpr int shape_coef(int s, int k) {
-  // (p, q, r) per shape: ramp, square, cube weights (sum 8)
-  constexpr int kShapes[8][3] = {{8, 0, 0}, {6, 2, 0}, {4, 4, 0}, {3, 5, 0},
-                                 {2, 5, 1}, {0, 8, 0}, {1, 3, 4}, {0, 3, 5}};
-  return kShapes[s][k];
+  return static_cast<int>(((k == 0 ? kShapeP : (k == 1 ? kShapeQ : kShapeR)) >> (4 * s)) & 15u);
 }
 
 // Level L[d][i] of the formatbook (i = 0..7).
@@ -61,15 +64,20 @@ __host__ __device__ inline int level(int d, int i) {
 struct Tables {
   uint32_t qerr[kBins][kDialects];  // [bin][dialect]: lane d reads word d
   uint8_t qval[kDialects][kBins];
+  int lvl[kDialects][8];            // the formatbook L[d][i]
 };
 
+// Fills the tables; ends with a __syncthreads.
 __device__ void build_tables(Tables* tb) {
+  for (int idx = threadIdx.x; idx < kDialects * 8; idx += blockDim.x)
+    tb->lvl[idx / 8][idx % 8] = level(idx / 8, idx % 8);
+  __syncthreads();
   for (int idx = threadIdx.x; idx < kDialects * kBins; idx += blockDim.x) {
     const int d = idx / kBins, b = idx % kBins;
     uint32_t best = 0xFFFFFFFFu;
     int bi = 0;
     for (int i = 0; i < 8; ++i) {
-      const int diff = 2 * b + 1 - 32 * level(d, i);
+      const int diff = 2 * b + 1 - 32 * tb->lvl[d][i];
       const uint32_t sq = static_cast<uint32_t>(diff * diff);
       if (sq < best) {
         best = sq;
@@ -79,11 +87,86 @@ __device__ void build_tables(Tables* tb) {
     tb->qerr[b][d] = best;
     tb->qval[d][b] = static_cast<uint8_t>(bi);
   }
+  __syncthreads();
 }
 
 // 2^n as binary32 for n in [-127, 127] (n = -127: the subnormal 2^-127).
 __device__ __forceinline__ float pow2f(int n) {
   return n >= -126 ? __int_as_float((n + 127) << 23) : __int_as_float(0x00400000);
+}
+
+// One warp quantises 8 blocks (256 consecutive elements of a row): lane l
+// holds elements 8l .. 8l + 7 in a[] (block l / 4).  Returns the lane's 8 codes
+// (element k in nibble k) and sets e and d of the lane's block.  `bins` is the
+// warp's 8 x 32 byte scratch.
+__device__ __forceinline__ uint32_t quant_warp_chunk(const float (&a)[8], const Tables& tb,
+                                                     uint8_t (*bins_sm)[kBlock], int lane, int& e_out,
+                                                     int& d_out) {
+  const int blk = lane >> 2;
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(a[k]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  int e = 0;
+  if (amax != 0.f) {
+    const int ef = (__float_as_uint(amax) >> 23) & 0xFF;
+    e = ef == 0 ? -126 : max(ef - 127, -126);
+  }
+  const float sc = pow2f(-e);  // exact; |x| 2^-e < 2
+  uint8_t bins[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float v = __fmul_rn(__fmul_rn(fabsf(a[k]), sc), 128.f);
+    const int b = static_cast<int>(v);  // truncation = floor for v >= 0
+    bins[k] = static_cast<uint8_t>(b > 255 ? 255 : b);
+  }
+  *reinterpret_cast<uint2*>(&bins_sm[blk][8 * (lane & 3)]) =
+      make_uint2(bins[0] | (bins[1] << 8) | (bins[2] << 16) | (static_cast<uint32_t>(bins[3]) << 24),
+                 bins[4] | (bins[5] << 8) | (bins[6] << 16) | (static_cast<uint32_t>(bins[7]) << 24));
+  __syncwarp();
+  // dialect choice: lane = dialect; the block's 32 bins come as two
+  // broadcast 16-byte reads, then 32 independent table reads
+  int my_d = 0;
+#pragma unroll 2
+  for (int j = 0; j < 8; ++j) {
+    const uint4 q0 = *reinterpret_cast<const uint4*>(&bins_sm[j][0]);
+    const uint4 q1 = *reinterpret_cast<const uint4*>(&bins_sm[j][16]);
+    const uint32_t bw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    uint32_t cost = 0;
+#pragma unroll
+    for (int k = 0; k < kBlock; ++k) cost += tb.qerr[(bw[k >> 2] >> (8 * (k & 3))) & 0xFFu][lane];
+    uint32_t key = (cost << 5) | static_cast<uint32_t>(lane);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) key = min(key, __shfl_xor_sync(0xffffffffu, key, off));
+    if (j == blk) my_d = static_cast<int>(key & 31u);
+  }
+  uint32_t packed = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t code = (a[k] < 0.f ? 8u : 0u) | tb.qval[my_d][bins[k]];
+    packed |= code << (4 * k);
+  }
+  __syncwarp();  // the scratch is rewritten by the next chunk
+  e_out = e;
+  d_out = my_d;
+  return packed;
+}
+
+__device__ __forceinline__ void load_chunk8(const uint16_t* __restrict__ src, int lane,
+                                            float (&a)[8]) {
+  const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src) + lane);
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    a[2 * k] = __uint_as_float(w[k] << 16);
+    a[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint16_t block_word(int e, int d) {
+  return static_cast<uint16_t>((static_cast<uint32_t>(e) & 0xFFu) |
+                               (static_cast<uint32_t>(d) << 8));
 }
 
 __global__ void __launch_bounds__(kThreads) sd4_quant_kernel(const uint16_t* __restrict__ x,
@@ -93,7 +176,6 @@ __global__ void __launch_bounds__(kThreads) sd4_quant_kernel(const uint16_t* __r
   __shared__ Tables tb;
   __shared__ __align__(16) uint8_t s_bins[kWarps][8][kBlock];
   build_tables(&tb);
-  __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int blocks_per_row = K / kBlock;
@@ -103,68 +185,70 @@ __global__ void __launch_bounds__(kThreads) sd4_quant_kernel(const uint16_t* __r
        c += static_cast<int64_t>(gridDim.x) * kWarps) {
     const int64_t row = c / chunks_per_row;
     const int col0 = static_cast<int>(c % chunks_per_row) * 256;
-    const int blk = lane >> 2;  // block within the chunk
-    // 8 elements of block blk: elements 8 * (lane & 3) .. + 7
-    const uint4 raw =
-        __ldg(reinterpret_cast<const uint4*>(x + row * static_cast<int64_t>(K) + col0) + lane);
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
     float a[8];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      a[2 * k] = __uint_as_float(w[k] << 16);
-      a[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    load_chunk8(x + row * static_cast<int64_t>(K) + col0, lane, a);
+    int e, d;
+    const uint32_t packed = quant_warp_chunk(a, tb, s_bins[warp], lane, e, d);
+    *reinterpret_cast<uint32_t*>(codes + row * static_cast<int64_t>(K / 2) + col0 / 2 + 4 * lane) =
+        packed;
+    if ((lane & 3) == 0) meta[row * blocks_per_row + col0 / kBlock + (lane >> 2)] = block_word(e, d);
+  }
+}
+
+// Activation decomposition of the salient rows (SemanticDialect "Resumen
+// técnico" §2.B): output row i holds 2K codes, those of x[rows[i]] followed by
+// those of the residual Delta = x - x_hat, and 2K/32 block words.  x_hat =
+// (-1)^s L/8 2^e is exact in binary32 (e >= -126 keeps L 2^(e-3) a multiple
+// of 2^-149) and so is the difference: an element rounded to a nonzero level
+// has |x| >= 2^(e-4), both are multiples of 2^(e-11) and |Delta| < 2^(e+2);
+// one rounded to level 0 has Delta = x.  An index outside [0, M) gives zero
+// codes and words for the row and sets kErrIndex.
+__global__ void __launch_bounds__(kThreads) sd4_decomp_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int K, const int32_t* __restrict__ rows, int64_t S,
+    uint8_t* __restrict__ codes2, uint16_t* __restrict__ meta2) {
+  __shared__ Tables tb;
+  __shared__ __align__(16) uint8_t s_bins[kWarps][8][kBlock];
+  build_tables(&tb);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int blk = lane >> 2;
+  const int64_t chunks_per_row = K / 256;
+  const int64_t num_chunks = S * chunks_per_row;
+  for (int64_t c = static_cast<int64_t>(blockIdx.x) * kWarps + warp; c < num_chunks;
+       c += static_cast<int64_t>(gridDim.x) * kWarps) {
+    const int64_t i = c / chunks_per_row;
+    const int col0 = static_cast<int>(c % chunks_per_row) * 256;
+    uint8_t* crow = codes2 + i * static_cast<int64_t>(K);        // 2K codes
+    uint16_t* mrow = meta2 + i * static_cast<int64_t>(K / 16);   // 2K/32 words
+    const int64_t r = rows[i];
+    if (r < 0 || r >= M) {
+      *reinterpret_cast<uint32_t*>(crow + col0 / 2 + 4 * lane) = 0u;
+      *reinterpret_cast<uint32_t*>(crow + K / 2 + col0 / 2 + 4 * lane) = 0u;
+      if ((lane & 3) == 0) {
+        mrow[col0 / kBlock + blk] = 0;
+        mrow[K / kBlock + col0 / kBlock + blk] = 0;
+      }
+      if (lane == 0) atomicOr(&g_error_word, kErrIndex);
+      continue;
     }
-    float amax = 0.f;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(a[k]));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    int e = 0;
-    if (amax != 0.f) {
-      const int ef = (__float_as_uint(amax) >> 23) & 0xFF;
-      e = ef == 0 ? -126 : max(ef - 127, -126);
-    }
-    const float sc = pow2f(-e);  // exact; |x| 2^-e < 2
-    uint8_t bins[8];
+    float a[8];
+    load_chunk8(x + r * static_cast<int64_t>(K) + col0, lane, a);
+    int e, d;
+    const uint32_t pa = quant_warp_chunk(a, tb, s_bins[warp], lane, e, d);
+    *reinterpret_cast<uint32_t*>(crow + col0 / 2 + 4 * lane) = pa;
+    if ((lane & 3) == 0) mrow[col0 / kBlock + blk] = block_word(e, d);
+    const float sc = pow2f(e);
+    float delta[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const float v = __fmul_rn(__fmul_rn(fabsf(a[k]), sc), 128.f);
-      const int b = static_cast<int>(v);  // truncation = floor for v >= 0
-      bins[k] = static_cast<uint8_t>(b > 255 ? 255 : b);
+      const uint32_t code = (pa >> (4 * k)) & 15u;
+      const float xh = __fmul_rn(static_cast<float>(tb.lvl[d][code & 7u]) * 0.125f, sc);
+      delta[k] = __fsub_rn(a[k], (code & 8u) ? -xh : xh);
     }
-    *reinterpret_cast<uint2*>(&s_bins[warp][blk][8 * (lane & 3)]) =
-        make_uint2(bins[0] | (bins[1] << 8) | (bins[2] << 16) | (static_cast<uint32_t>(bins[3]) << 24),
-                   bins[4] | (bins[5] << 8) | (bins[6] << 16) | (static_cast<uint32_t>(bins[7]) << 24));
-    __syncwarp();
-    // dialect choice: lane = dialect; the block's 32 bins come as two
-    // broadcast 16-byte reads, then 32 independent table reads
-    int my_d = 0;
-#pragma unroll 2
-    for (int j = 0; j < 8; ++j) {
-      const uint4 q0 = *reinterpret_cast<const uint4*>(&s_bins[warp][j][0]);
-      const uint4 q1 = *reinterpret_cast<const uint4*>(&s_bins[warp][j][16]);
-      const uint32_t bw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-      uint32_t cost = 0;
-#pragma unroll
-      for (int k = 0; k < kBlock; ++k) cost += tb.qerr[(bw[k >> 2] >> (8 * (k & 3))) & 0xFFu][lane];
-      uint32_t key = (cost << 5) | static_cast<uint32_t>(lane);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) key = min(key, __shfl_xor_sync(0xffffffffu, key, off));
-      if (j == blk) my_d = static_cast<int>(key & 31u);
-    }
-    // codes of this lane's 8 elements
-    uint32_t packed = 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t code = (a[k] < 0.f ? 8u : 0u) | tb.qval[my_d][bins[k]];
-      packed |= code << (4 * k);
-    }
-    const int64_t code_off = row * static_cast<int64_t>(K / 2) + col0 / 2 + 4 * lane;
-    *reinterpret_cast<uint32_t*>(codes + code_off) = packed;
-    if ((lane & 3) == 0)
-      meta[row * blocks_per_row + col0 / kBlock + blk] =
-          static_cast<uint16_t>((static_cast<uint32_t>(e) & 0xFFu) | (static_cast<uint32_t>(my_d) << 8));
-    __syncwarp();  // s_bins is rewritten by the next chunk
+    int e2, d2;
+    const uint32_t pd = quant_warp_chunk(delta, tb, s_bins[warp], lane, e2, d2);
+    *reinterpret_cast<uint32_t*>(crow + K / 2 + col0 / 2 + 4 * lane) = pd;
+    if ((lane & 3) == 0) mrow[K / kBlock + col0 / kBlock + blk] = block_word(e2, d2);
   }
 }
 
@@ -310,7 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     sd4_gemm_kernel(const __grid_constant__ CUtensorMap tmCA, const __grid_constant__ CUtensorMap tmCB,
                     const __grid_constant__ CUtensorMap tmMA, const __grid_constant__ CUtensorMap tmMB,
                     const __grid_constant__ CUtensorMap tmWB, const uint16_t* __restrict__ bias,
-                    uint16_t* __restrict__ out, int M, int N, int K) {
+                    uint16_t* __restrict__ out, int M, int N, int K, int kb_wrap,
+                    const int32_t* __restrict__ out_rows, int out_M) {
   using C = SCfg<WDEC>;
   constexpr int kOffOp = C::kOffOp, kOffPk = C::kOffPk, kOffMeta = C::kOffMeta;
   constexpr int kOffBar = C::kOffBar, kOffEpi = C::kOffEpi, kOffPair = C::kOffPair;
@@ -377,28 +462,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ph = 0, mph = 0, pho = 0;
       for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
         const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = 0, kbw = 0; kb < kblocks; ++kb, kbw = (kbw + 1 == kb_wrap ? 0 : kbw + 1)) {
+          // kbw: the weights' K-block (the A rows may be longer: [x | Delta]
+          // against [w | w]); kb_wrap % 4 == 0 keeps the block words aligned
           if ((kb & 3) == 0) {
             if (!mbar_wait_bounded(bars.meta_empty(ms), mph ^ 1u, abort_flag, kErrWaitProducer))
               break;
             const uint32_t dst = sbase + kOffMeta + ms * kMetaSlot;
             mbar_arrive_expect_tx(bars.meta_full(ms), kMetaSlot);
             tma_load_2d(dst, &tmMA, (kb / 4) * 16, m0, bars.meta_full(ms));
-            if (!WDEC) tma_load_2d(dst + kMetaA, &tmMB, (kb / 4) * 16, n0, bars.meta_full(ms));
+            if (!WDEC) tma_load_2d(dst + kMetaA, &tmMB, (kbw / 4) * 16, n0, bars.meta_full(ms));
             if (++ms == kMetaSlots) { ms = 0; mph ^= 1u; }
           }
           if (!mbar_wait_bounded(bars.pk_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer)) break;
           const uint32_t dst = sbase + kOffPk + s * kPkStage;
           mbar_arrive_expect_tx(bars.pk_full(s), kPkStage);
           tma_load_2d(dst, &tmCA, kb * (BK / 2), m0, bars.pk_full(s));
-          if (!WDEC) tma_load_2d(dst + kPkA, &tmCB, kb * (BK / 2), n0, bars.pk_full(s));
+          if (!WDEC) tma_load_2d(dst + kPkA, &tmCB, kbw * (BK / 2), n0, bars.pk_full(s));
           if (++s == kPkStages) { s = 0; ph ^= 1u; }
           if (WDEC) {  // decoded weights: TMA into the operand stage's B tile
             if (!mbar_wait_bounded(bars.op_empty(so), pho ^ 1u, abort_flag, kErrWaitProducer))
               break;
             const uint32_t ob = sbase + kOffOp + so * kOpStage + kOpA;
             mbar_arrive_expect_tx(bars.op_full(so), kOpB);
-            tma_load_2d(ob, &tmWB, kb * BK, n0, bars.op_full(so));
+            tma_load_2d(ob, &tmWB, kbw * BK, n0, bars.op_full(so));
             if (++so == kOpStages) { so = 0; pho ^= 1u; }
           }
         }
@@ -448,6 +535,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_bounded(bars.acc_full(buf), aph, abort_flag, kErrWaitEpilogue)) break;
       tc_fence_after();
       const int row = m0 + 32 * quad + lane;
+      int orow = row < M ? row : -1;  // the output row this accumulator row goes to
+      if (out_rows && orow >= 0) {
+        orow = out_rows[row];
+        if (orow < 0 || orow >= out_M) {
+          atomicOr(&g_error_word, kErrIndex);
+          orow = -1;
+        }
+      }
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quad) << 16) +
                              static_cast<uint32_t>(buf * BN);
 #pragma unroll 1
@@ -456,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x32(taddr + 32 * c, r);
         tmem_wait_ld();
         const int n = n0 + 32 * c;
-        if (row < M && n < N) {
+        if (orow >= 0 && n < N) {
           uint32_t pk[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -465,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
             pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
           }
-          uint16_t* dst = out + static_cast<int64_t>(row) * N + n;
+          uint16_t* dst = out + static_cast<int64_t>(orow) * N + n;
 #pragma unroll
           for (int v = 0; v < 4; ++v)
             if (n + 8 * v + 8 <= N)

@@ -149,3 +149,16 @@ def make_chain(cfg: ChainConfig = WAN_CHAIN, M: int | None = None) -> dict:
 def bf16_bits(t: torch.Tensor):
     """uint16 numpy view of a bf16 CPU tensor (what the oracle consumes)."""
     return t.contiguous().view(torch.int16).numpy().view("uint16")
+
+
+SALIENT_FRACTION = 1 / 16
+
+
+def salient_rows(M: int, seed: int, frac: float = SALIENT_FRACTION) -> list[int]:
+    """Stand-in for the salient tokens of SemanticDialect's activation
+    decomposition (chosen there from attention scores of a trained model):
+    round(frac * M) distinct rows drawn by a generator of their own (seed +
+    7919, so the layer's tensors are unchanged), in increasing order."""
+    g = torch.Generator(device="cpu").manual_seed(seed + 7919)
+    n = max(1, round(frac * M))
+    return sorted(torch.randperm(M, generator=g)[:n].tolist())

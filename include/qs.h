@@ -61,7 +61,8 @@ typedef enum {
   QS_ERR_SHAPE = 2,    /* M, N or K <= 0, K % 128 != 0, or N % 16 != 0 */
   QS_ERR_BITS = 3,     /* bits not 4, 6 or 8 */
   QS_ERR_ALIGN = 4,    /* a pointer is not 16-byte aligned */
-  QS_ERR_RANGE = 5,    /* alpha outside [2^-14, 1], unknown flag bits, or a size above its limit */
+  QS_ERR_RANGE = 5,    /* alpha outside [2^-14, 1], unknown flag bits, a size above its limit,
+                          or (from qs_device_error) a row index out of range */
   QS_ERR_CUDA = 6,     /* a CUDA runtime/driver call or a launch failed */
   QS_ERR_TIMEOUT = 7,  /* a kernel wait exceeded its bound (reported by qs_device_error) */
   QS_ERR_PTR = 8       /* a pointer is not device memory of the current device */
@@ -333,6 +334,46 @@ QS_API qs_status qs_sd4_linear_wdec(const void* x_codes, const uint16_t* x_meta,
                                     int64_t N, int64_t K, void* out_bf16, void* stream);
 
 /*
+ * Activation decomposition (SemanticDialect "Resumen técnico" §2.B): a salient
+ * activation row A is split into its SD4 value Q(A) and the residual
+ * Delta = A - x_hat, which is quantised again with the same format, and the
+ * layer uses A ~ Q(A) + Q(Delta) for that row.  The pages choose the salient
+ * rows from attention scores; here the caller gives them as row indices.
+ *
+ * qs_sd4_quant_decomp — the decomposed rows: row i of the output holds 2K
+ * codes, the SD4 codes of x[rows[i]] (those qs_sd4_quant writes) followed by
+ * the SD4 codes of Delta (exact in binary32; blocks of the same 32 columns),
+ * and the 2K/32 block words.
+ *   x_bf16  [M, K] bf16, K % 256 == 0, K <= QS_MAX_K / 2
+ *   rows    [S] int32 (device, 4-byte aligned); indices may repeat; an index
+ *           outside [0, M) gives zero codes and words for that row and makes
+ *           qs_device_error report QS_ERR_RANGE
+ *   codes2  [S, K] bytes (2K codes, two per byte), written
+ *   meta2   [S, K/16] uint16 (2K/32 block words), written
+ */
+QS_API qs_status qs_sd4_quant_decomp(const void* x_bf16, int64_t M, int64_t K,
+                                     const int32_t* rows, int64_t S, void* codes2,
+                                     uint16_t* meta2, void* stream);
+
+/*
+ * qs_sd4_linear_decomp — the decomposed rows of the SD4 layer: for i < S,
+ *   out[rows[i]][n] = bf16(fl(sum_k (x_hat + delta_hat)[k] w_hat[n][k]) + bias[n])
+ * as one binary32 tensor-core accumulation over the 2K products of a
+ * qs_sd4_quant_decomp row with [w_hat | w_hat].  Only those rows of out are
+ * written: the layer with decomposition is qs_sd4_linear (or _wdec) over all
+ * M rows followed, on the same stream, by this call.  The weights are given
+ * either as codes (w_codes [N, K/2], w_meta [N, K/32]) or, when w_bf16 is not
+ * NULL, decoded (qs_sd4_decode, [N, K]; w_codes and w_meta are then ignored).
+ * An index outside [0, M) is skipped and reported as in qs_sd4_quant_decomp.
+ *   out_bf16  [M, N] bf16, rows rows[i] written
+ */
+QS_API qs_status qs_sd4_linear_decomp(const void* codes2, const uint16_t* meta2,
+                                      const int32_t* rows, int64_t S, const void* w_codes,
+                                      const uint16_t* w_meta, const void* w_bf16,
+                                      const void* bias_bf16, int64_t M, int64_t N, int64_t K,
+                                      void* out_bf16, void* stream);
+
+/*
  * δ-guided bit switching (DVD-Quant "Resumen técnico" §2.C): per layer, the
  * normalised L1 change between consecutive outputs is accumulated, and the
  * layer's next step runs at 4 bits while the accumulated change is below
@@ -443,8 +484,9 @@ QS_API qs_status qs_selftest_timeout(int64_t timeout_us, void* stream);
 /*
  * qs_device_error — synchronises `stream`, then returns and clears the
  * library's device-side error word: QS_OK, QS_ERR_TIMEOUT if a kernel gave up
- * a bounded wait (its outputs are then undefined), or QS_ERR_CUDA if the
- * synchronisation itself failed.
+ * a bounded wait (its outputs are then undefined), QS_ERR_RANGE if a row index
+ * read on the device was out of range (and no wait gave up), or QS_ERR_CUDA if
+ * the synchronisation itself failed.
  */
 QS_API qs_status qs_device_error(void* stream);
 

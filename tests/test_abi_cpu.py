@@ -236,3 +236,30 @@ def test_bgr_validation(lib):
     k = lib.qs_linear_bgr
     assert k(A, 8, 128, 1.0, B, C, D, NUL, 256, 4, A, need - 1, B, NUL) == RANGE
     assert k(A, 8, 128, 1.0, B, C, NUL, NUL, 256, 4, A, need, B, NUL) == NULL
+
+
+def test_sd4_validation(lib):
+    q = lib.qs_sd4_quant
+    assert q(NUL, 8, 256, B, C, NUL) == NULL
+    assert q(A, 8, 384, B, C, NUL) == SHAPE                 # K % 256
+    assert q(A, 8, 256, B, ctypes.c_void_p(0x30008), NUL) == ALIGN
+    f = lib.qs_sd4_linear
+    assert f(A, B, C, NUL, NUL, 8, 256, 256, D, NUL) == NULL
+    assert f(A, B, C, D, NUL, 8, 264, 256, D, NUL) == SHAPE  # N % 16
+    assert f(A, B, C, D, NUL, 8, 256, 65536 + 256, D, NUL) == RANGE
+    assert lib.qs_sd4_decode(A, B, 4, 128, C, NUL) == SHAPE
+    assert lib.qs_sd4_linear_wdec(A, B, NUL, NUL, 8, 256, 256, D, NUL) == NULL
+    g = lib.qs_sd4_quant_decomp
+    assert g(A, 8, 256, NUL, 4, C, D, NUL) == NULL          # rows
+    assert g(A, 8, 256, B, 0, C, D, NUL) == SHAPE           # no salient rows
+    assert g(A, 0, 256, B, 4, C, D, NUL) == SHAPE
+    assert g(A, 8, 32768 + 256, B, 4, C, D, NUL) == RANGE   # 2K codes per row
+    assert g(A, 8, 256, ctypes.c_void_p(0x20002), 4, C, D, NUL) == ALIGN
+    h = lib.qs_sd4_linear_decomp
+    assert h(A, B, C, 4, NUL, NUL, NUL, NUL, 8, 256, 256, D, NUL) == NULL   # no weights
+    assert h(A, B, C, 4, A, NUL, NUL, NUL, 8, 256, 256, D, NUL) == NULL     # codes without words
+    assert h(A, B, C, 4, NUL, NUL, D, NUL, 8, 264, 256, D, NUL) == SHAPE
+    assert h(A, B, C, 4, NUL, NUL, D, NUL, 8, 256, 384, D, NUL) == SHAPE
+    assert h(A, B, C, 4, NUL, NUL, D, NUL, 8, 256, 32768 + 256, D, NUL) == RANGE
+    assert h(A, B, C, 4, NUL, NUL, MIS, NUL, 8, 256, 256, D, NUL) == ALIGN
+    assert h(A, B, ctypes.c_void_p(0x30002), 4, A, B, NUL, NUL, 8, 256, 256, D, NUL) == ALIGN

@@ -143,3 +143,191 @@ def test_sd4_linear_with_decoded_weights_is_identical(M, N, K):
     qs.qs_sd4_linear_wdec(cx, mx, wdec, d["bias"].cuda(), M, N, K, out2)
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+
+
+# ------------------------------------------------- activation decomposition (§2.B)
+
+def _rows_tensor(rows):
+    return torch.tensor(rows, dtype=torch.int32, device="cuda")
+
+
+def check_decomp(x, rows):
+    codes2, meta2 = qs.sd4_quant_decomp(x.cuda(), _rows_tensor(rows))
+    torch.cuda.synchronize()
+    dec = S.decompose_rows(I.bf16_bits(x), rows)
+    want_c, want_m = S.pack_decomp(dec)
+    got_m = meta2.cpu().numpy().view(np.uint16)
+    if not np.array_equal(got_m, want_m):
+        bad = np.argwhere(got_m != want_m)
+        raise AssertionError(f"block words differ at {len(bad)}, first {bad[:5].tolist()}")
+    assert np.array_equal(codes2.cpu().numpy(), want_c), "codes differ"
+    return codes2, meta2, dec
+
+
+@pytest.mark.parametrize("M,K,S_", [(7, 256, 7), (33, 5120, 12), (40, 13824, 9), (3, 32768, 2)])
+def test_sd4_quant_decomp_bit_exact(M, K, S_):
+    d = I.make_shape(seed=M + K + 1, M=M, K=K, N=16, bits=4, outlier_factor=30.0)
+    rng = np.random.default_rng(M + K)
+    rows = [0, M - 1] + rng.integers(0, M, S_ - 2).tolist() if S_ > 2 else [M - 1, 0][:S_]
+    check_decomp(d["x"], rows)
+
+
+def test_sd4_quant_decomp_edge_rows():
+    g = torch.Generator().manual_seed(8)
+    x = torch.randn(6, 512, generator=g)
+    x[0] = 0.0                              # zero residual, zero blocks
+    x[1] = -0.0
+    x[2] = x[2] * 2.0 ** -118               # residuals at the exponent floor (subnormal binary32)
+    x[3] = x[3] * 1e30
+    x[2, 5] = 2.0 ** -130                   # rounds to level 0: a subnormal residual
+    x[2, 40] = -3 * 2.0 ** -131
+    x[4, ::3] = 0.0
+    k = torch.arange(32, dtype=torch.float32)
+    x[5, 64:96] = k * 2.0 ** -133 * (1 - 2 * (k % 2))   # a block of bf16 subnormals: e = -126
+    x = x.to(torch.bfloat16)
+    _, _, dec = check_decomp(x, [0, 1, 2, 3, 4, 5, 2])
+    assert dec["delta"][2, 5] == 2.0 ** -130 and dec["exp_x"][5, 2] == -126
+
+
+def test_sd4_decomp_reconstructs_two_scale_rows_exactly():
+    # blocks x = a + b (levels at two scales, built as in the oracle's pins):
+    # the device codes decode to x_hat + delta_hat = x exactly
+    rng = np.random.default_rng(2)
+    L = S.formatbook()
+    R, K = 4, 512
+    x = np.zeros((R, K))
+    for r in range(R):
+        for j in range(K // 32):
+            e = int(rng.integers(-30, 30))
+            nz = rng.choice(32, 20, replace=False)
+            idx = rng.integers(0, 8, 20)
+            idx[0] = 7
+            x[r, 32 * j + nz] = (rng.choice([-1.0, 1.0], 20) * 15 / 8 * 2.0 ** e
+                                 + rng.choice([-1.0, 1.0], 20) * L[21, idx] / 8 * 2.0 ** (e - 4))
+    xt = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16)
+    assert np.array_equal(xt.float().numpy().astype(np.float64), x)
+    codes2, meta2, _ = check_decomp(xt, [3, 1, 0, 2])
+    dec = qs.sd4_decode(codes2, meta2).float().cpu().numpy().astype(np.float64)
+    assert np.array_equal(dec[:, :K] + dec[:, K:], x[[3, 1, 0, 2]])
+
+
+def test_sd4_decomp_index_out_of_range_is_reported():
+    x = torch.randn(8, 256, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16).cuda()
+    rows = _rows_tensor([1, -1, 8, 7])
+    codes2 = torch.full((4, 256), 0x5A, dtype=torch.uint8, device="cuda")
+    meta2 = torch.full((4, 16), 0x1234, dtype=torch.int16, device="cuda")
+    qs.qs_sd4_quant_decomp(x, 8, 256, rows, 4, codes2, meta2)
+    assert qs.qs_device_error() == 5                    # QS_ERR_RANGE, then cleared
+    assert qs.qs_device_error() == 0
+    c = codes2.cpu().numpy()
+    assert not c[1].any() and not c[2].any() and not meta2.cpu().numpy()[1:3].any()
+    dec = S.decompose_rows(I.bf16_bits(x.cpu()), [1, 7])
+    want_c, _ = S.pack_decomp(dec)
+    assert np.array_equal(c[[0, 3]], want_c)
+    # the layer call skips those rows and reports them the same way
+    w = torch.randn(16, 256, generator=torch.Generator().manual_seed(2)).to(torch.bfloat16).cuda()
+    cw, mw = qs.sd4_quant(w)
+    out = torch.full((8, 16), 7, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+    qs.qs_sd4_linear_decomp(codes2, meta2, rows, 4, cw, mw, None, None, 8, 16, 256, out)
+    assert qs.qs_device_error() == 5
+    o = out.view(torch.int16).cpu().numpy()
+    assert (o[[0, 2, 3, 4, 5, 6]] == 7).all() and not (o[[1, 7]] == 7).all()
+
+
+def _decomp_layer(M, N, K, rows, seed, wdec, bias=True):
+    d = I.make_shape(seed=seed, M=M, K=K, N=N, bits=4, outlier_factor=30.0)
+    x, w = d["x"].cuda(), d["w"].cuda()
+    b = d["bias"].cuda() if bias else None
+    cx, mx = qs.sd4_quant(x)
+    cw, mw = qs.sd4_quant(w)
+    rt = _rows_tensor(rows)
+    codes2, meta2 = qs.sd4_quant_decomp(x, rt)
+    w_dec = qs.sd4_decode(cw, mw) if wdec else None
+    out = qs.sd4_linear_decomp(cx, mx, codes2, meta2, rt, cw, mw, b, K, w_dec=w_dec)
+    torch.cuda.synchronize()
+    return d, out
+
+
+def _check_decomp_layer(d, out, rows, K, bias=True):
+    xb, wb = I.bf16_bits(d["x"]), I.bf16_bits(d["w"])
+    bb = I.bf16_bits(d["bias"]) if bias else None
+    r = S.linear_sd4_decomp(xb, wb, bb, rows, exact=False)
+    got_bits = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    got = O.bf16_bits_to_f32(got_bits).astype(np.float64)
+    b = O.bf16_bits_to_f32(bb).astype(np.float64) if bias else 0.0
+    M = got.shape[0]
+    # binary32 accumulation of exact products: at most (terms) 2^-23 sum|products|
+    # (2K terms on a decomposed row: x_hat and delta_hat separately), plus one
+    # bf16 ulp of the result
+    absw = np.abs(r["w_hat"]).T
+    S_abs = np.abs(r["x_hat"]) @ absw
+    terms = np.full((M, 1), float(K))
+    rows_u = np.unique(rows)
+    dec = r["decomp"]
+    first = {int(v): i for i, v in reversed(list(enumerate(rows)))}
+    sel = np.array([first[int(m)] for m in rows_u])
+    S_abs[rows_u] = (np.abs(dec["x_hat"][sel]) @ absw) + (np.abs(dec["d_hat"][sel]) @ absw)
+    terms[rows_u] = 2.0 * K
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(got), 2.0 ** -126))) - 7)
+    allowed = terms * 2.0 ** -23 * S_abs + ulp
+    err = np.abs(got - (r["y"] + b))
+    assert (err <= allowed).all(), f"max excess {np.max(err - allowed)}"
+    same = float((got_bits == r["out"]).mean())
+    assert same > 0.99, f"only {same:.4f} of outputs bit-identical to the oracle"
+    # the decomposition moved the salient rows toward the unquantised product
+    xf = O.bf16_bits_to_f32(xb).astype(np.float64)
+    wf = O.bf16_bits_to_f32(wb).astype(np.float64)
+    ref = xf[rows_u] @ wf.T
+    plain = S.linear_sd4(xb, wb, bb, exact=False)["y"][rows_u]
+    assert np.linalg.norm(r["y"][rows_u] - ref) < np.linalg.norm(plain - ref)
+
+
+@pytest.mark.parametrize("wdec", [False, True])
+@pytest.mark.parametrize("M,N,K", [(127, 272, 256), (300, 768, 768), (513, 528, 1280)])
+def test_sd4_linear_decomp_matches_oracle(M, N, K, wdec):
+    rng = np.random.default_rng(M + N)
+    rows = sorted(set(rng.choice(M, max(1, M // 8), replace=False).tolist()) | {0, M - 1})
+    rows = rows + rows[:3]                   # repeated indices write the same values
+    rng.shuffle(rows)
+    d, out = _decomp_layer(M, N, K, rows, seed=M + 2 * N, wdec=wdec)
+    _check_decomp_layer(d, out, rows, K)
+
+
+def test_sd4_linear_decomp_single_row_no_bias_and_forms_agree():
+    rows = [5]
+    d, out = _decomp_layer(64, 272, 512, rows, seed=9, wdec=False, bias=False)
+    _check_decomp_layer(d, out, rows, 512, bias=False)
+    _, out2 = _decomp_layer(64, 272, 512, rows, seed=9, wdec=True, bias=False)
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+
+
+@pytest.mark.slow
+def test_full_size_wan_ffn_decomp_sampled():
+    """The Wan FFN layer (32760 x 5120 -> 13824) with 1/16 of the tokens
+    decomposed, in the decoded-weight form the benchmark times; sampled
+    outputs of salient and plain rows against the oracle."""
+    cfg = I.WAN_FFN
+    d = I.make_layer(cfg)
+    M, K, N = cfg.M, cfg.K, cfg.N
+    rows = I.salient_rows(M, seed=cfg.seed)
+    x, w, b = d["x"].cuda(), d["w"].cuda(), d["bias"].cuda()
+    cx, mx = qs.sd4_quant(x)
+    cw, mw = qs.sd4_quant(w)
+    wd = qs.sd4_decode(cw, mw)
+    rt = _rows_tensor(rows)
+    codes2, meta2 = qs.sd4_quant_decomp(x, rt)
+    out = qs.sd4_linear_decomp(cx, mx, codes2, meta2, rt, None, None, b, K, w_dec=wd)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(4)
+    pick_s = np.unique(np.concatenate([[0, len(rows) - 1], rng.choice(len(rows), 24, replace=False)]))
+    srows = np.asarray(rows)[pick_s]
+    others = np.setdiff1d(rng.choice(M, 40, replace=False), rows)[:16]
+    cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 40, replace=False)]))
+    wb, bb = I.bf16_bits(d["w"][cols]), I.bf16_bits(d["bias"][cols])
+    mrows = np.concatenate([srows, others])
+    xb = I.bf16_bits(d["x"][mrows])
+    sub = {"x": d["x"][mrows], "w": d["w"][cols], "bias": d["bias"][cols]}
+    got = out[torch.from_numpy(mrows).cuda()][:, torch.from_numpy(cols).cuda()]
+    _check_decomp_layer(sub, got, list(range(len(srows))), K)
+    assert np.array_equal(codes2[torch.from_numpy(pick_s).cuda()].cpu().numpy(),
+                          S.pack_decomp(S.decompose_rows(xb[:len(srows)], range(len(srows))))[0])
