@@ -434,34 +434,43 @@ def sd4_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
         stream.synchronize()
         q = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
         g = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
-        # the weights decoded once (offline): only the activations decoded per call
+        # the weights decoded once (offline): only the activations decoded per
+        # call; as bf16 (bf16 tensor cores) and as e4m3 bytes (block-scaled fp8)
         wdec = qs.sd4_decode(cw, mw, stream=stream)
+        w8 = qs.sd4_decode_e4m3(cw, mw, stream=stream)
         out2 = torch.empty_like(out)
+        out8 = torch.empty_like(out)
         qs.qs_sd4_linear_wdec(cx, mx, wdec, b, M, N, K, out2, stream)
-        e2 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        e2[0].record(stream)
-        for _ in range(steps):
-            qs.qs_sd4_linear_wdec(cx, mx, wdec, b, M, N, K, out2, stream)
-        e2[1].record(stream)
-        stream.synchronize()
-        g2 = e2[0].elapsed_time(e2[1]) / steps
-        same = bool(torch.equal(out.view(torch.int16), out2.view(torch.int16)))
+        qs.qs_sd4_linear_e4m3w(cx, mx, w8, mw, b, M, N, K, out8, stream)
+
+        def timed(fn):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            e[0].record(stream)
+            for _ in range(steps):
+                fn()
+            e[1].record(stream)
+            stream.synchronize()
+            return e[0].elapsed_time(e[1]) / steps
+
+        g2 = timed(lambda: qs.qs_sd4_linear_wdec(cx, mx, wdec, b, M, N, K, out2, stream))
+        g8 = timed(lambda: qs.qs_sd4_linear_e4m3w(cx, mx, w8, mw, b, M, N, K, out8, stream))
+        same = bool(torch.equal(out.view(torch.int16), out8.view(torch.int16)))
         # activation decomposition of the salient tokens (a seeded 1/16 of them)
         srows = I.salient_rows(M, cfg.seed)
         S_ = len(srows)
         rt = torch.tensor(srows, dtype=torch.int32, device=dev)
         c2 = torch.empty((S_, K), dtype=torch.uint8, device=dev)
         m2 = torch.empty((S_, K // 16), dtype=torch.int16, device=dev)
-        out3 = out2.clone()
+        out3 = out8.clone()
         for _ in range(warmup):
             qs.qs_sd4_quant_decomp(x, M, K, rt, S_, c2, m2, stream)
-            qs.qs_sd4_linear_decomp(c2, m2, rt, S_, None, None, wdec, b, M, N, K, out3, stream)
+            qs.qs_sd4_linear_decomp(c2, m2, rt, S_, None, mw, w8, b, M, N, K, out3, stream)
         e3 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
         for e in e3:
             e[0].record(stream)
             qs.qs_sd4_quant_decomp(x, M, K, rt, S_, c2, m2, stream)
             e[1].record(stream)
-            qs.qs_sd4_linear_decomp(c2, m2, rt, S_, None, None, wdec, b, M, N, K, out3, stream)
+            qs.qs_sd4_linear_decomp(c2, m2, rt, S_, None, mw, w8, b, M, N, K, out3, stream)
             e[2].record(stream)
         stream.synchronize()
         dq = sum(e[0].elapsed_time(e[1]) for e in e3) / steps
@@ -471,9 +480,9 @@ def sd4_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
         err_s = lambda y: float((y - ref_s).norm() / ref_s.norm())  # noqa: E731
         decomp = {"salient_rows": S_, "salient_fraction": S_ / M, "quant_decomp_ms": dq,
                   "gemm_decomp_ms": dg,
-                  "gemm_decomp_TFLOPS_bf16": 2.0 * S_ * 2 * K * N / (dg * 1e-3) / 1e12,
-                  "layer_ms_decoded_weights": q + g2 + dq + dg,
-                  "rel_err_salient_plain": err_s(out2[sel].double()),
+                  "gemm_decomp_TFLOPS": 2.0 * S_ * 2 * K * N / (dg * 1e-3) / 1e12,
+                  "layer_ms_e4m3_weights": q + g8 + dq + dg,
+                  "rel_err_salient_plain": err_s(out8[sel].double()),
                   "rel_err_salient_decomposed": err_s(out3[sel].double()),
                   "error_rows": int(sel.numel())}
         ref = x[:rows].double() @ w.double().t() + b.double()
@@ -483,14 +492,18 @@ def sd4_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
         stream.synchronize()
     err = lambda y: float((y - ref).norm() / ref.norm())  # noqa: E731
     pk, _ = peaks()
-    gemm_tflops = cfg.ops / (g * 1e-3) / 1e12
+    fp8_peak = 2.0 * pk["bf16_tflops"]  # measured bf16 x the nominal fp8:bf16 dense ratio
+    tf = lambda ms: cfg.ops / (ms * 1e-3) / 1e12  # noqa: E731
     quant_bytes = M * (2 * K + K // 2 + 2 * (K // 32))
-    return {"workload": cfg.name + "_sd4", "quant_ms": q, "gemm_ms": g,
-            "TOPS": cfg.ops / ((q + g) * 1e-3) / 1e12, "gemm_TFLOPS_bf16": gemm_tflops,
-            "gemm_frac_bf16_peak": gemm_tflops / pk["bf16_tflops"],
-            "gemm_decoded_weights_ms": g2,
-            "gemm_decoded_weights_TFLOPS_bf16": cfg.ops / (g2 * 1e-3) / 1e12,
-            "decoded_weights_output_identical": same,
+    return {"workload": cfg.name + "_sd4", "quant_ms": q,
+            "gemm_ms": g, "gemm_path": "block-scaled fp8 (e4m3 + UE8M0 per 32), codes decoded",
+            "TOPS": cfg.ops / ((q + g) * 1e-3) / 1e12, "gemm_TFLOPS": tf(g),
+            "gemm_frac_fp8_peak": tf(g) / fp8_peak,
+            "gemm_e4m3_weights_ms": g8, "gemm_e4m3_weights_TFLOPS": tf(g8),
+            "gemm_e4m3_weights_frac_fp8_peak": tf(g8) / fp8_peak,
+            "e4m3_weights_output_identical": same,
+            "gemm_bf16_weights_ms": g2, "gemm_bf16_weights_TFLOPS": tf(g2),
+            "gemm_bf16_weights_frac_bf16_peak": tf(g2) / pk["bf16_tflops"],
             "quant_GBps": quant_bytes / (q * 1e-3) / 1e9,
             "rel_err_sd4": err(out[:rows].double()), "rel_err_w4a4_rotated": err(y4),
             "error_rows": rows, "decomposition": decomp}

@@ -33,7 +33,8 @@ EXPORTS = ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qlinear_mixed", 
            "qs_quant_act_rowsum",
            "qs_qlinear_asym", "qs_qgemm_s32_asym", "qs_linear_bgr_workspace_bytes",
            "qs_linear_bgr", "qs_sd4_quant", "qs_sd4_linear", "qs_sd4_decode",
-           "qs_sd4_linear_wdec", "qs_sd4_quant_decomp", "qs_sd4_linear_decomp", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
+           "qs_sd4_linear_wdec", "qs_sd4_quant_decomp", "qs_sd4_linear_decomp",
+           "qs_sd4_decode_e4m3", "qs_sd4_linear_e4m3w", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
            "qs_selftest_timeout", "qs_device_error", "qs_status_str", "qs_version")
 BITS = (4, 6, 8)
 QS_GBS_MAX_BLOCKS = 1024
@@ -88,6 +89,8 @@ def load() -> ctypes.CDLL:
     L.qs_sd4_linear_wdec.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
     L.qs_sd4_quant_decomp.argtypes = [vp, i64, i64, vp, i64, vp, vp, vp]
     L.qs_sd4_linear_decomp.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, i64, i64, i64, vp, vp]
+    L.qs_sd4_decode_e4m3.argtypes = [vp, vp, i64, i64, vp, vp]
+    L.qs_sd4_linear_e4m3w.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]
     L.qs_gbs_reset.argtypes = [vp, vp]
     L.qs_gbs_update.argtypes = [vp, vp, i64, f64, vp, vp]
     L.qs_linear_gbs.argtypes = [vp, i64, i64, f32, vp, vp, vp, vp, vp, i64, vp, vp, i64, vp, vp]
@@ -101,7 +104,8 @@ def load() -> ctypes.CDLL:
                  "qs_linear_mixed", "qs_linear_ex", "qs_linear_noalloc", "qs_pack_weights_bgr",
                  "qs_quant_act_rowsum", "qs_qlinear_asym", "qs_qgemm_s32_asym", "qs_linear_bgr",
                  "qs_sd4_quant", "qs_sd4_linear", "qs_sd4_decode", "qs_sd4_linear_wdec",
-                 "qs_sd4_quant_decomp", "qs_sd4_linear_decomp", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
+                 "qs_sd4_quant_decomp", "qs_sd4_linear_decomp", "qs_sd4_decode_e4m3",
+           "qs_sd4_linear_e4m3w", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
                  "qs_selftest_timeout",
                  "qs_device_error"):
         getattr(L, name).restype = ctypes.c_int
@@ -383,16 +387,42 @@ def qs_sd4_quant_decomp(x, M, K, rows, S, codes2, meta2, stream=None):
                                       _s(stream)), "qs_sd4_quant_decomp")
 
 
-def qs_sd4_linear_decomp(codes2, meta2, rows, S, w_codes, w_meta, w_bf16, bias, M, N, K, out,
+def qs_sd4_linear_decomp(codes2, meta2, rows, S, w_codes, w_meta, w_e4m3, bias, M, N, K, out,
                          stream=None):
     for t, name, dt in ((codes2, "codes2", torch.uint8), (meta2, "meta2", torch.int16),
                         (rows, "rows", torch.int32), (w_codes, "w_codes", torch.uint8),
-                        (w_meta, "w_meta", torch.int16), (w_bf16, "w_bf16", torch.bfloat16),
+                        (w_meta, "w_meta", torch.int16), (w_e4m3, "w_e4m3", torch.uint8),
                         (bias, "bias", torch.bfloat16), (out, "out", torch.bfloat16)):
         _cuda(t, dt, name)
     _check(load().qs_sd4_linear_decomp(_p(codes2), _p(meta2), _p(rows), S, _p(w_codes),
-                                       _p(w_meta), _p(w_bf16), _p(bias), M, N, K, _p(out),
+                                       _p(w_meta), _p(w_e4m3), _p(bias), M, N, K, _p(out),
                                        _s(stream)), "qs_sd4_linear_decomp")
+
+
+def qs_sd4_decode_e4m3(codes, meta, rows, K, out, stream=None):
+    _cuda(codes, torch.uint8, "codes")
+    _cuda(meta, torch.int16, "meta")
+    _cuda(out, torch.uint8, "out")
+    _check(load().qs_sd4_decode_e4m3(_p(codes), _p(meta), rows, K, _p(out), _s(stream)),
+           "qs_sd4_decode_e4m3")
+
+
+def sd4_decode_e4m3(codes, meta, stream=None):
+    """SD4 codes [R, K/2] + block words -> e4m3 bytes uint8 [R, K] (the block
+    scales stay in the words)."""
+    R, K = codes.shape[0], codes.shape[1] * 2
+    out = torch.empty((R, K), dtype=torch.uint8, device=codes.device)
+    qs_sd4_decode_e4m3(codes, meta, R, K, out, stream)
+    return out
+
+
+def qs_sd4_linear_e4m3w(x_codes, x_meta, w_e4m3, w_meta, bias, M, N, K, out, stream=None):
+    for t, name, dt in ((x_codes, "x_codes", torch.uint8), (x_meta, "x_meta", torch.int16),
+                        (w_e4m3, "w_e4m3", torch.uint8), (w_meta, "w_meta", torch.int16),
+                        (bias, "bias", torch.bfloat16), (out, "out", torch.bfloat16)):
+        _cuda(t, dt, name)
+    _check(load().qs_sd4_linear_e4m3w(_p(x_codes), _p(x_meta), _p(w_e4m3), _p(w_meta), _p(bias),
+                                      M, N, K, _p(out), _s(stream)), "qs_sd4_linear_e4m3w")
 
 
 def sd4_quant_decomp(x: torch.Tensor, rows: torch.Tensor, stream=None):
@@ -407,21 +437,20 @@ def sd4_quant_decomp(x: torch.Tensor, rows: torch.Tensor, stream=None):
 
 
 def sd4_linear_decomp(x_codes, x_meta, codes2, meta2, rows, w_codes, w_meta, bias, K: int,
-                      w_dec=None, stream=None, out=None):
+                      w_e4m3=None, stream=None, out=None):
     """The SD4 layer with the salient rows decomposed: qs_sd4_linear (or the
-    decoded-weight form when w_dec is given) over all rows, then
+    e4m3-weight form when w_e4m3 is given) over all rows, then
     qs_sd4_linear_decomp over the salient ones."""
-    M, N = x_codes.shape[0], (w_dec if w_dec is not None else w_codes).shape[0]
+    M, N = x_codes.shape[0], w_meta.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x_codes.device)
-    if w_dec is not None:
-        qs_sd4_linear_wdec(x_codes, x_meta, w_dec, bias, M, N, K, out, stream)
-        qs_sd4_linear_decomp(codes2, meta2, rows, rows.shape[0], None, None, w_dec, bias, M, N, K,
-                             out, stream)
+    if w_e4m3 is not None:
+        qs_sd4_linear_e4m3w(x_codes, x_meta, w_e4m3, w_meta, bias, M, N, K, out, stream)
     else:
         qs_sd4_linear(x_codes, x_meta, w_codes, w_meta, bias, M, N, K, out, stream)
-        qs_sd4_linear_decomp(codes2, meta2, rows, rows.shape[0], w_codes, w_meta, None, bias, M,
-                             N, K, out, stream)
+    qs_sd4_linear_decomp(codes2, meta2, rows, rows.shape[0],
+                         None if w_e4m3 is not None else w_codes, w_meta, w_e4m3, bias, M, N, K,
+                         out, stream)
     return out
 
 

@@ -18,6 +18,7 @@
 #include "qs_glue.cuh"
 #include "qs_quant.cuh"
 #include "qs_sd4.cuh"
+#include "qs_sd4_mx.cuh"
 
 namespace {
 
@@ -124,6 +125,59 @@ qs_status launch_sd4_gemm(const CUtensorMap& ca, const CUtensorMap& cb, const CU
       static_cast<int>(kb_wrap > 0 ? kb_wrap : K / G::BK), out_rows,
       static_cast<int>(out_rows ? out_M : M));
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+template <bool WDEC>
+qs_status launch_sd4_mx(const CUtensorMap& ca, const CUtensorMap& cb, const CUtensorMap& ma,
+                        const CUtensorMap& mb, const CUtensorMap& wb, const void* bias, int64_t M,
+                        int64_t N, int64_t K, void* out, void* stream, int64_t kb_wrap,
+                        const int32_t* out_rows, int64_t out_M) {
+  namespace G = qs::sd4::gemm_mx;
+  constexpr int smem = G::MCfg<WDEC>::kSmemBytes;
+  auto kern = G::sd4_mx_gemm_kernel<WDEC>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return QS_ERR_CUDA;
+  const int sms = qs::sm_count();
+  if (sms <= 0) return QS_ERR_CUDA;
+  const int64_t tiles = ((M + G::BM - 1) / G::BM) * ((N + G::BN - 1) / G::BN);
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  kern<<<grid, G::MCfg<WDEC>::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+      ca, cb, ma, mb, wb, static_cast<const uint16_t*>(bias), static_cast<uint16_t*>(out),
+      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(kb_wrap),
+      out_rows, static_cast<int>(out_rows ? out_M : M));
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+// The block-scaled SD4 GEMM: A = `a_rows` rows of Ka codes (Ka = K, or 2K for
+// decomposed rows), the weights as codes + block words or, when w_e4m3 is not
+// NULL, as e4m3 bytes + block words.
+qs_status run_sd4_mx(const void* a_codes, const uint16_t* a_meta, int64_t a_rows, int64_t Ka,
+                     const void* w_codes, const uint16_t* w_meta, const void* w_e4m3,
+                     const void* bias, int64_t N, int64_t K, void* out, void* stream,
+                     const int32_t* out_rows, int64_t out_M) {
+  namespace G = qs::sd4::gemm_mx;
+  CUtensorMap ca, ma, cb, mb, wb;
+  if (!qs::make_tensor_map_2d(&ca, a_codes, static_cast<uint64_t>(Ka) / 2,
+                              static_cast<uint64_t>(a_rows), G::BK / 2, G::BM, false) ||
+      !qs::make_tensor_map_2d(&ma, a_meta, static_cast<uint64_t>(Ka) / 16,
+                              static_cast<uint64_t>(a_rows), 16, G::BM, false) ||
+      !qs::make_tensor_map_2d(&mb, w_meta, static_cast<uint64_t>(K) / 16,
+                              static_cast<uint64_t>(N), 16, G::BN, false))
+    return QS_ERR_CUDA;
+  const int64_t kb_wrap = K / G::BK;
+  if (w_e4m3) {
+    if (!qs::make_tensor_map_2d(&wb, w_e4m3, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                                G::BK, G::BN, true))
+      return QS_ERR_CUDA;
+    return launch_sd4_mx<true>(ca, ca, ma, mb, wb, bias, a_rows, N, Ka, out, stream, kb_wrap,
+                               out_rows, out_M);
+  }
+  if (!qs::make_tensor_map_2d(&cb, w_codes, static_cast<uint64_t>(K) / 2,
+                              static_cast<uint64_t>(N), G::BK / 2, G::BN, false))
+    return QS_ERR_CUDA;
+  return launch_sd4_mx<false>(ca, cb, ma, mb, cb, bias, a_rows, N, Ka, out, stream, kb_wrap,
+                              out_rows, out_M);
 }
 
 }  // namespace
@@ -493,7 +547,6 @@ qs_status qs_sd4_quant(const void* x_bf16, int64_t rows, int64_t K, void* codes,
 qs_status qs_sd4_linear(const void* x_codes, const uint16_t* x_meta, const void* w_codes,
                         const uint16_t* w_meta, const void* bias_bf16, int64_t M, int64_t N,
                         int64_t K, void* out_bf16, void* stream) {
-  namespace G = qs::sd4::gemm_sd4;
   if (!x_codes || !x_meta || !w_codes || !w_meta || !out_bf16) return QS_ERR_NULL;
   if (M <= 0 || N <= 0 || K <= 0 || K % 256 != 0 || N % 16 != 0) return QS_ERR_SHAPE;
   if (K > QS_MAX_K || M > INT32_MAX || N > INT32_MAX) return QS_ERR_RANGE;
@@ -504,16 +557,45 @@ qs_status qs_sd4_linear(const void* x_codes, const uint16_t* x_meta, const void*
                         static_cast<const void*>(w_meta), static_cast<const void*>(out_bf16)})
     QS_TRY(check_device_ptr(p));
   if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
-  CUtensorMap ca, cb, ma, mb;
-  const uint64_t code_row = static_cast<uint64_t>(K) / 2, meta_row = static_cast<uint64_t>(K) / 16;
-  if (!qs::make_tensor_map_2d(&ca, x_codes, code_row, static_cast<uint64_t>(M), G::BK / 2, G::BM,
-                              false) ||
-      !qs::make_tensor_map_2d(&cb, w_codes, code_row, static_cast<uint64_t>(N), G::BK / 2, G::BN,
-                              false) ||
-      !qs::make_tensor_map_2d(&ma, x_meta, meta_row, static_cast<uint64_t>(M), 16, G::BM, false) ||
-      !qs::make_tensor_map_2d(&mb, w_meta, meta_row, static_cast<uint64_t>(N), 16, G::BN, false))
-    return QS_ERR_CUDA;
-  return launch_sd4_gemm<false>(ca, cb, ma, mb, cb, bias_bf16, M, N, K, out_bf16, stream);
+  return run_sd4_mx(x_codes, x_meta, M, K, w_codes, w_meta, nullptr, bias_bf16, N, K, out_bf16,
+                    stream, nullptr, 0);
+}
+
+qs_status qs_sd4_decode_e4m3(const void* codes, const uint16_t* meta, int64_t rows, int64_t K,
+                             void* out_e4m3, void* stream) {
+  if (!codes || !meta || !out_e4m3) return QS_ERR_NULL;
+  if (rows <= 0 || K <= 0 || K % 256 != 0) return QS_ERR_SHAPE;
+  if (K > QS_MAX_K || rows > QS_MAX_ROWS) return QS_ERR_RANGE;
+  if (!aligned16(codes) || !aligned16(meta) || !aligned16(out_e4m3)) return QS_ERR_ALIGN;
+  for (const void* p : {codes, static_cast<const void*>(meta), static_cast<const void*>(out_e4m3)})
+    QS_TRY(check_device_ptr(p));
+  const int sms = qs::sm_count();
+  if (sms <= 0) return QS_ERR_CUDA;
+  const int64_t tasks = rows * (K / 16);
+  int64_t grid = (tasks + 255) / 256;
+  if (grid > static_cast<int64_t>(sms) * 8) grid = static_cast<int64_t>(sms) * 8;
+  qs::sd4::gemm_mx::sd4_decode_e4m3_kernel<<<static_cast<unsigned>(grid), 256, 0,
+                                             static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(codes), meta, rows, static_cast<int>(K),
+      static_cast<uint8_t*>(out_e4m3));
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status qs_sd4_linear_e4m3w(const void* x_codes, const uint16_t* x_meta, const void* w_e4m3,
+                              const uint16_t* w_meta, const void* bias_bf16, int64_t M, int64_t N,
+                              int64_t K, void* out_bf16, void* stream) {
+  if (!x_codes || !x_meta || !w_e4m3 || !w_meta || !out_bf16) return QS_ERR_NULL;
+  if (M <= 0 || N <= 0 || K <= 0 || K % 256 != 0 || N % 16 != 0) return QS_ERR_SHAPE;
+  if (K > QS_MAX_K || M > INT32_MAX || N > INT32_MAX) return QS_ERR_RANGE;
+  if (!aligned16(x_codes) || !aligned16(x_meta) || !aligned16(w_e4m3) || !aligned16(w_meta) ||
+      !aligned16(out_bf16) || (bias_bf16 && !aligned16(bias_bf16)))
+    return QS_ERR_ALIGN;
+  for (const void* p : {x_codes, static_cast<const void*>(x_meta), w_e4m3,
+                        static_cast<const void*>(w_meta), static_cast<const void*>(out_bf16)})
+    QS_TRY(check_device_ptr(p));
+  if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
+  return run_sd4_mx(x_codes, x_meta, M, K, nullptr, w_meta, w_e4m3, bias_bf16, N, K, out_bf16,
+                    stream, nullptr, 0);
 }
 
 qs_status qs_sd4_decode(const void* codes, const uint16_t* meta, int64_t rows, int64_t K,
@@ -586,49 +668,24 @@ qs_status qs_sd4_quant_decomp(const void* x_bf16, int64_t M, int64_t K, const in
 
 qs_status qs_sd4_linear_decomp(const void* codes2, const uint16_t* meta2, const int32_t* rows,
                                int64_t S, const void* w_codes, const uint16_t* w_meta,
-                               const void* w_bf16, const void* bias_bf16, int64_t M, int64_t N,
+                               const void* w_e4m3, const void* bias_bf16, int64_t M, int64_t N,
                                int64_t K, void* out_bf16, void* stream) {
-  namespace G = qs::sd4::gemm_sd4;
-  if (!codes2 || !meta2 || !rows || !out_bf16) return QS_ERR_NULL;
-  if (!w_bf16 && (!w_codes || !w_meta)) return QS_ERR_NULL;
+  if (!codes2 || !meta2 || !rows || !out_bf16 || !w_meta) return QS_ERR_NULL;
+  if (!w_e4m3 && !w_codes) return QS_ERR_NULL;
   if (M <= 0 || S <= 0 || N <= 0 || K <= 0 || K % 256 != 0 || N % 16 != 0) return QS_ERR_SHAPE;
   if (2 * K > QS_MAX_K || M > INT32_MAX || S > INT32_MAX || N > INT32_MAX) return QS_ERR_RANGE;
-  if (!aligned16(codes2) || !aligned16(meta2) || !aligned16(out_bf16) ||
+  if (!aligned16(codes2) || !aligned16(meta2) || !aligned16(out_bf16) || !aligned16(w_meta) ||
       (reinterpret_cast<uintptr_t>(rows) & 3u) || (bias_bf16 && !aligned16(bias_bf16)))
     return QS_ERR_ALIGN;
-  if (w_bf16 ? !aligned16(w_bf16) : (!aligned16(w_codes) || !aligned16(w_meta)))
-    return QS_ERR_ALIGN;
+  if (w_e4m3 ? !aligned16(w_e4m3) : !aligned16(w_codes)) return QS_ERR_ALIGN;
   for (const void* p : {codes2, static_cast<const void*>(meta2), static_cast<const void*>(rows),
-                        static_cast<const void*>(out_bf16)})
+                        static_cast<const void*>(out_bf16), static_cast<const void*>(w_meta),
+                        w_e4m3 ? w_e4m3 : w_codes})
     QS_TRY(check_device_ptr(p));
-  if (w_bf16) {
-    QS_TRY(check_device_ptr(w_bf16));
-  } else {
-    QS_TRY(check_device_ptr(w_codes));
-    QS_TRY(check_device_ptr(w_meta));
-  }
   if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
-  // A: S rows of 2K codes; B: the weights' K, walked twice
-  const uint64_t K2 = 2 * static_cast<uint64_t>(K);
-  CUtensorMap ca, ma, cb, mb, wb;
-  if (!qs::make_tensor_map_2d(&ca, codes2, K2 / 2, static_cast<uint64_t>(S), G::BK / 2, G::BM,
-                              false) ||
-      !qs::make_tensor_map_2d(&ma, meta2, K2 / 16, static_cast<uint64_t>(S), 16, G::BM, false))
-    return QS_ERR_CUDA;
-  if (w_bf16) {
-    if (!qs::make_tensor_map_2d(&wb, w_bf16, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
-                                G::BK, G::BN, true, 2))
-      return QS_ERR_CUDA;
-    return launch_sd4_gemm<true>(ca, ca, ma, ma, wb, bias_bf16, S, N, K2, out_bf16, stream,
-                                 K / G::BK, rows, M);
-  }
-  if (!qs::make_tensor_map_2d(&cb, w_codes, static_cast<uint64_t>(K) / 2,
-                              static_cast<uint64_t>(N), G::BK / 2, G::BN, false) ||
-      !qs::make_tensor_map_2d(&mb, w_meta, static_cast<uint64_t>(K) / 16,
-                              static_cast<uint64_t>(N), 16, G::BN, false))
-    return QS_ERR_CUDA;
-  return launch_sd4_gemm<false>(ca, cb, ma, mb, cb, bias_bf16, S, N, K2, out_bf16, stream,
-                                K / G::BK, rows, M);
+  // A: S rows of 2K codes; the weights' K walked twice
+  return run_sd4_mx(codes2, meta2, S, 2 * K, w_e4m3 ? nullptr : w_codes, w_meta, w_e4m3,
+                    bias_bf16, N, K, out_bf16, stream, rows, M);
 }
 
 qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream) {

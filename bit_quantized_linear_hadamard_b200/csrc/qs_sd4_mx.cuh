@@ -1,0 +1,487 @@
+// SD4 layer GEMM on the block-scaled fp8 tensor-core path.
+//
+// An SD4 value is (-1)^s L/8 2^e with L <= 15 and one power-of-two scale per
+// 32 consecutive elements of a row: L/8 is an e4m3 number exactly (at most 4
+// significant bits, exponent -3..0) and 2^e is a UE8M0 scale (e + 127,
+// e in [-126, 127]).  That is the operand format of
+// tcgen05.mma.kind::mxf8f6f4.block_scale with one scale per 32 elements along
+// K, so the products x_hat * w_hat come out of the tensor cores exactly and
+// are summed with binary32 accumulation, at the fp8 rate and with one byte
+// per operand element in shared memory (the bf16 form needs two).
+//
+// Persistent, one CTA per SM, tiles of 128 x 192 (two 192-column binary32
+// accumulators and the 12 scale columns fit the 512 TMEM columns; a 256-wide
+// pair would not), 128 K elements (four scale blocks) per stage.
+// Warp roles: 0 TMA producer (codes every stage, block words every two
+// stages, the decoded weights when given), 1 TMEM allocation and the MMA
+// issuer (per stage: three tcgen05.cp of the stage's scales into TMEM, then
+// four MMAs of K = 32 that select scale byte j = 0..3), 2-5 epilogue, then
+// the decode warps: codes -> e4m3 bytes through an 8-byte per-dialect level
+// table and `prmt`, block words -> scale bytes in the tcgen05.cp layout.
+//
+// Scale layout (the one tcgen05.cp.32x128b.warpx4 expects): 512 bytes per
+// 128 rows, row m's four scale bytes (K-blocks 0..3 of the stage) at
+// 16 (m % 32) + 4 (m / 32); the copy replicates them to the four TMEM lane
+// quarters, columns 0..3.  B's 192 rows take two such blocks (8 columns).
+#pragma once
+
+#include "qs_sd4.cuh"
+
+namespace qs {
+namespace sd4 {
+namespace gemm_mx {
+
+constexpr int BM = 128, BN = 192, BK = 128;
+constexpr int kEpiWarps = 4;
+constexpr int kTmemCols = 512;
+constexpr int kSfaCol = 2 * BN;      // 4 columns
+constexpr int kSfbCol = 2 * BN + 4;  // 8 columns
+constexpr int kOpA = BM * BK, kOpB = BN * BK;          // e4m3 tiles, 128-byte rows
+constexpr int kSfA = 512, kSfB = 1024;                 // scale bytes of a stage
+constexpr int kPkA = BM * BK / 2, kPkB = BN * BK / 2;  // code tiles, 64-byte rows
+constexpr int kMetaA = BM * 16, kMetaB = BN * 16;      // 8 block words per row = 2 stages
+static_assert(BN % 32 == 0 && BN <= 256 && 2 * BN + 12 <= kTmemCols, "tile");
+
+// WDEC: the weights come as e4m3 bytes (qs_sd4_decode_e4m3), loaded by TMA
+// straight into their operand tile; their block words still give the scales.
+template <bool WDEC>
+struct MCfg {
+  static constexpr int kDecWarps = WDEC ? 8 : 10;
+  static constexpr int kDecThreads = 32 * kDecWarps;
+  static constexpr int kThreads = 32 * (2 + kEpiWarps + kDecWarps);
+  static constexpr int kOpStages = WDEC ? 4 : 3;
+  static constexpr int kPkStages = WDEC ? 4 : 3;
+  static constexpr int kMetaSlots = 2;
+  static constexpr int kDecRows = WDEC ? BM : BM + BN;  // rows decoded per stage
+  static constexpr int kTasks = 2 * kDecRows;           // (row, half of the stage's K)
+  static constexpr int kOpStage = kOpA + kOpB;
+  static constexpr int kSfStage = kSfA + kSfB;
+  static constexpr int kPkStage = WDEC ? kPkA : kPkA + kPkB;
+  static constexpr int kMetaSlot = kMetaA + kMetaB;
+  static constexpr int kOffOp = 0;
+  static constexpr int kOffSf = kOffOp + kOpStages * kOpStage;
+  static constexpr int kOffPk = kOffSf + kOpStages * kSfStage;
+  static constexpr int kOffMeta = kOffPk + kPkStages * kPkStage;
+  static constexpr int kOffBar = kOffMeta + kMetaSlots * kMetaSlot;
+  static constexpr int kNumBars = 2 * kPkStages + 2 * kMetaSlots + 2 * kOpStages + 4;
+  static constexpr int kOffEpi = (kOffBar + 8 * kNumBars + 15) / 16 * 16;  // bias of a tile
+  static constexpr int kOffTab = kOffEpi + BN * 4;                          // e4m3 level table
+  static constexpr int kOffMisc = kOffTab + kDialects * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  // arrivals completing an operand stage: the decode warps, plus the
+  // producer's arm of the decoded weight tile's TMA bytes
+  static constexpr int kOpFullCount = kDecWarps + (WDEC ? 1 : 0);
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+  static_assert(kOffSf % 1024 == 0 && kOffPk % 128 == 0 && kOffMeta % 128 == 0, "alignment");
+  static_assert(kTasks % kDecThreads == 0, "decode split");
+};
+
+// e4m3 encoding of L/8, 0 <= L <= 15 (normal for L >= 1: exponent field
+// p + 4 with p = floor(log2 L), mantissa (L - 2^p) 2^(3-p)).
+__host__ __device__ constexpr uint32_t e4m3_eighths(int L) {
+  return L == 0 ? 0u
+                : static_cast<uint32_t>(
+                      (((L >= 8 ? 3 : L >= 4 ? 2 : L >= 2 ? 1 : 0) + 4) << 3) |
+                      ((L - (1 << (L >= 8 ? 3 : L >= 4 ? 2 : L >= 2 ? 1 : 0)))
+                       << (3 - (L >= 8 ? 3 : L >= 4 ? 2 : L >= 2 ? 1 : 0))));
+}
+
+// Instruction descriptor of kind::mxf8f6f4.block_scale: e4m3 A and B, both
+// K-major, UE8M0 scales, binary32 accumulation; scale byte j of A and B.
+__host__ __device__ constexpr uint32_t idesc_mx(int M, int N, uint32_t j) {
+  return (j << 4)                                 // B scale byte
+         | (0u << 7) | (0u << 10)                 // A, B: E4M3
+         | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
+         | (1u << 23)                             // scales: UE8M0
+         | (static_cast<uint32_t>(M >> 4) << 24)  // M / 16
+         | (j << 29);                             // A scale byte
+}
+
+__device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::
+          "r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Shared -> tensor memory: 32 rows of 16 bytes, replicated to the 4 lane quarters.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// Source descriptor of a 512-byte scale block: no swizzle, K-major, rows of
+// 16 bytes, 8-row groups 128 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sf(uint32_t addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr & 0x3FFFFu) >> 4);  // start address
+  d |= static_cast<uint64_t>(1) << 16;                  // leading byte offset (one 16-byte unit)
+  d |= static_cast<uint64_t>(128 >> 4) << 32;           // stride byte offset
+  d |= static_cast<uint64_t>(1) << 46;                  // descriptor version (sm_100)
+  return d;                                             // layout type 0: no swizzle
+}
+
+// Eight codes (element k in nibble k) -> eight e4m3 bytes.  E: the dialect's
+// magnitudes e4m3(L_i/8), byte i of the pair (lo, hi); `prmt` picks byte i for
+// each code's level index, and the code's sign bit (nibble bit 3) moves to
+// bit 7 of its byte.
+__device__ __forceinline__ uint2 decode8_e4m3(uint32_t w, uint2 E) {
+  const uint32_t v03 = __byte_perm(E.x, E.y, w & 0x7777u);
+  const uint32_t v47 = __byte_perm(E.x, E.y, (w >> 16) & 0x7777u);
+  const uint32_t s = w & 0x88888888u;
+  const uint32_t t03 = __byte_perm(s, 0u, 0x1100u);  // bytes s0 s0 s1 s1
+  const uint32_t t47 = __byte_perm(s, 0u, 0x3322u);  // bytes s2 s2 s3 s3
+  const uint32_t s03 = ((t03 << 4) & 0x00800080u) | (t03 & 0x80008000u);
+  const uint32_t s47 = ((t47 << 4) & 0x00800080u) | (t47 & 0x80008000u);
+  return make_uint2(v03 | s03, v47 | s47);
+}
+
+struct MBars {
+  uint32_t base;
+  int P, T, U;  // code stages, meta slots, operand stages
+  __device__ uint32_t at(int i) const { return base + 8u * i; }
+  __device__ uint32_t pk_full(int s) const { return at(s); }
+  __device__ uint32_t pk_empty(int s) const { return at(P + s); }
+  __device__ uint32_t meta_full(int s) const { return at(2 * P + s); }
+  __device__ uint32_t meta_empty(int s) const { return at(2 * P + T + s); }
+  __device__ uint32_t op_full(int s) const { return at(2 * P + 2 * T + s); }
+  __device__ uint32_t op_empty(int s) const { return at(2 * P + 2 * T + U + s); }
+  __device__ uint32_t acc_full(int b) const { return at(2 * P + 2 * T + 2 * U + b); }
+  __device__ uint32_t acc_empty(int b) const { return at(2 * P + 2 * T + 2 * U + 2 + b); }
+};
+
+// Scale-block offset of row m (within A's 128 rows or B's 192) in a stage.
+__device__ __forceinline__ int sf_row_offset(int m) {
+  return 512 * (m >> 7) + 16 * (m & 31) + 4 * ((m & 127) >> 5);
+}
+
+// out[orow(m)][n] = bf16(fl(sum_k x_hat[m][k] w_hat[n][k]) + bias[n]).  The A
+// rows may be longer than the weights' K (kb_wrap K-blocks, walked again):
+// the decomposed rows [Q(x) | Q(Delta)] against [w | w].  out_rows (nullable)
+// maps accumulator row m to its output row; an index outside [0, out_M) is
+// skipped and flagged.
+template <bool WDEC>
+__global__ void __launch_bounds__(MCfg<WDEC>::kThreads, 1)
+    sd4_mx_gemm_kernel(const __grid_constant__ CUtensorMap tmCA,
+                       const __grid_constant__ CUtensorMap tmCB,
+                       const __grid_constant__ CUtensorMap tmMA,
+                       const __grid_constant__ CUtensorMap tmMB,
+                       const __grid_constant__ CUtensorMap tmWB, const uint16_t* __restrict__ bias,
+                       uint16_t* __restrict__ out, int M, int N, int K, int kb_wrap,
+                       const int32_t* __restrict__ out_rows, int out_M) {
+  using C = MCfg<WDEC>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+  uint8_t* sp = smem_raw + pad;
+  const uint32_t sbase = raw + pad;
+  const MBars bars{sbase + C::kOffBar, C::kPkStages, C::kMetaSlots, C::kOpStages};
+  float* epi_b = reinterpret_cast<float*>(sp + C::kOffEpi);
+  uint2* tab = reinterpret_cast<uint2*>(sp + C::kOffTab);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sp + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = (N + BN - 1) / BN;
+  const int num_tiles = ((M + BM - 1) / BM) * n_tiles;
+  const int kblocks = K / BK;
+
+  for (int d = threadIdx.x; d < kDialects; d += blockDim.x) {
+    uint32_t lo = 0, hi = 0;
+    for (int i = 0; i < 4; ++i) {
+      lo |= e4m3_eighths(level(d, i)) << (8 * i);
+      hi |= e4m3_eighths(level(d, i + 4)) << (8 * i);
+    }
+    tab[d] = make_uint2(lo, hi);
+  }
+  // B's scale blocks hold rows 192..255 that no MMA reads but tcgen05.cp copies
+  for (int i = threadIdx.x; i < C::kOpStages * C::kSfStage / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(sp + C::kOffSf)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kPkStages; ++s) {
+      mbar_init(bars.pk_full(s), 1);
+      mbar_init(bars.pk_empty(s), C::kDecWarps);
+    }
+    for (int s = 0; s < C::kMetaSlots; ++s) {
+      mbar_init(bars.meta_full(s), 1);
+      mbar_init(bars.meta_empty(s), C::kDecWarps);
+    }
+    for (int s = 0; s < C::kOpStages; ++s) {
+      mbar_init(bars.op_full(s), C::kOpFullCount);
+      mbar_init(bars.op_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bars.acc_full(b), 1);
+      mbar_init(bars.acc_empty(b), kEpiWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {  // producer
+      int s = 0, ms = 0, so = 0;
+      uint32_t ph = 0, mph = 0, pho = 0;
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
+        for (int kb = 0, kbw = 0; kb < kblocks; ++kb, kbw = (kbw + 1 == kb_wrap ? 0 : kbw + 1)) {
+          // kbw: the weights' K-block; kb_wrap is even, so both stay in step
+          // with the two-stage block-word slots
+          if ((kb & 1) == 0) {
+            if (!mbar_wait_bounded(bars.meta_empty(ms), mph ^ 1u, abort_flag, kErrWaitProducer))
+              break;
+            const uint32_t dst = sbase + C::kOffMeta + ms * C::kMetaSlot;
+            mbar_arrive_expect_tx(bars.meta_full(ms), C::kMetaSlot);
+            tma_load_2d(dst, &tmMA, (kb / 2) * 16, m0, bars.meta_full(ms));
+            tma_load_2d(dst + kMetaA, &tmMB, (kbw / 2) * 16, n0, bars.meta_full(ms));
+            if (++ms == C::kMetaSlots) { ms = 0; mph ^= 1u; }
+          }
+          if (!mbar_wait_bounded(bars.pk_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer)) break;
+          const uint32_t dst = sbase + C::kOffPk + s * C::kPkStage;
+          mbar_arrive_expect_tx(bars.pk_full(s), C::kPkStage);
+          tma_load_2d(dst, &tmCA, kb * (BK / 2), m0, bars.pk_full(s));
+          if (!WDEC) tma_load_2d(dst + kPkA, &tmCB, kbw * (BK / 2), n0, bars.pk_full(s));
+          if (++s == C::kPkStages) { s = 0; ph ^= 1u; }
+          if (WDEC) {  // decoded weights: TMA into the operand stage's B tile
+            if (!mbar_wait_bounded(bars.op_empty(so), pho ^ 1u, abort_flag, kErrWaitProducer))
+              break;
+            const uint32_t ob = sbase + C::kOffOp + so * C::kOpStage + kOpA;
+            mbar_arrive_expect_tx(bars.op_full(so), kOpB);
+            tma_load_2d(ob, &tmWB, kbw * BK, n0, bars.op_full(so));
+            if (++so == C::kOpStages) { so = 0; pho ^= 1u; }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // MMA issuer
+      const uint32_t sfa = tmem_base + kSfaCol, sfb = tmem_base + kSfbCol;
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+        const int buf = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait_bounded(bars.acc_empty(buf), aph ^ 1u, abort_flag, kErrWaitMma)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(bars.op_full(s), ph, abort_flag, kErrWaitMma)) break;
+          tc_fence_after();
+          const uint32_t a0 = sbase + C::kOffOp + s * C::kOpStage;
+          const uint32_t b0 = a0 + kOpA;
+          const uint32_t f0 = sbase + C::kOffSf + s * C::kSfStage;
+          // the stage's scales into TMEM; the tensor pipe runs these copies
+          // and the MMAs below in issue order
+          tmem_cp_32x128b_x4(sfa, smem_desc_sf(f0));
+          tmem_cp_32x128b_x4(sfb, smem_desc_sf(f0 + kSfA));
+          tmem_cp_32x128b_x4(sfb + 4, smem_desc_sf(f0 + kSfA + 512));
+#pragma unroll
+          for (int j = 0; j < BK / 32; ++j)
+            mma_mx(d, smem_desc_sw128(a0 + j * 32), smem_desc_sw128(b0 + j * 32),
+                   idesc_mx(BM, BN, static_cast<uint32_t>(j)),
+                   sfa + (static_cast<uint32_t>(j) << 30), sfb + (static_cast<uint32_t>(j) << 30),
+                   (kb | j) != 0);
+          mma_commit(bars.op_empty(s));
+          if (++s == C::kOpStages) { s = 0; ph ^= 1u; }
+        }
+        mma_commit(bars.acc_full(buf));
+      }
+    }
+  } else if (warp < 2 + kEpiWarps) {  // epilogue: TMEM lanes 32 * (warp & 3) ..
+    const int quad = warp & 3;
+    const int et = threadIdx.x - 64;
+    int it = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+      const int buf = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      for (int i = et; i < BN; i += 128) {
+        const int n = n0 + i;
+        epi_b[i] = (n < N && bias) ? __uint_as_float(static_cast<uint32_t>(bias[n]) << 16) : 0.f;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!mbar_wait_bounded(bars.acc_full(buf), aph, abort_flag, kErrWaitEpilogue)) break;
+      tc_fence_after();
+      const int row = m0 + 32 * quad + lane;
+      int orow = row < M ? row : -1;
+      if (out_rows && orow >= 0) {
+        orow = out_rows[row];
+        if (orow < 0 || orow >= out_M) {
+          atomicOr(&g_error_word, kErrIndex);
+          orow = -1;
+        }
+      }
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quad) << 16) +
+                             static_cast<uint32_t>(buf * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + 32 * c, r);
+        tmem_wait_ld();
+        const int n = n0 + 32 * c;
+        if (orow >= 0 && n < N) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float y0 = __fadd_rn(__uint_as_float(r[2 * j]), epi_b[32 * c + 2 * j]);
+            const float y1 = __fadd_rn(__uint_as_float(r[2 * j + 1]), epi_b[32 * c + 2 * j + 1]);
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
+            pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          uint16_t* dst = out + static_cast<int64_t>(orow) * N + n;
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            if (n + 8 * v + 8 <= N)
+              *reinterpret_cast<uint4*>(dst + 8 * v) =
+                  make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.acc_empty(buf));
+    }
+  } else {  // decode warps
+    const int dt = threadIdx.x - 32 * (2 + kEpiWarps);  // 0 .. kDecThreads - 1
+    int s = 0, so = 0, ms = 0;
+    uint32_t ph = 0, pho = 0, mph = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      for (int kb = 0; kb < kblocks; ++kb) {
+        if ((kb & 1) == 0 &&
+            !mbar_wait_bounded(bars.meta_full(ms), mph, abort_flag, kErrWaitUnpack))
+          break;
+        if (!mbar_wait_bounded(bars.pk_full(s), ph, abort_flag, kErrWaitUnpack)) break;
+        if (!mbar_wait_bounded(bars.op_empty(so), pho ^ 1u, abort_flag, kErrWaitUnpack)) break;
+        const uint8_t* pk = sp + C::kOffPk + s * C::kPkStage;
+        const uint8_t* mt = sp + C::kOffMeta + ms * C::kMetaSlot;
+        uint8_t* op = sp + C::kOffOp + so * C::kOpStage;
+        uint8_t* sf = sp + C::kOffSf + so * C::kSfStage;
+        // task = (operand row r: x rows 0..127, then W rows; half h of the
+        // stage's K: scale blocks 2h, 2h + 1)
+#pragma unroll
+        for (int j = 0; j < C::kTasks / C::kDecThreads; ++j) {
+          const int task = dt + C::kDecThreads * j;
+          const int r = task >> 1, h = task & 1;
+          const bool is_b = r >= BM;
+          const int rr = is_b ? r - BM : r;
+          const uint8_t* crow = pk + (is_b ? kPkA : 0) + rr * (BK / 2) + 32 * h;
+          const uint32_t words = *reinterpret_cast<const uint32_t*>(
+              mt + (is_b ? kMetaA : 0) + rr * 16 + ((kb & 1) * 4 + 2 * h) * 2);
+          uint8_t* orow_p = op + (is_b ? kOpA : 0) + rr * 128;
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            // block bb of this half: 16 code bytes (these reads are 2-way
+            // bank conflicted; the swizzled stores below are conflict-free,
+            // and one order cannot make both free)
+            const int bb = b;
+            const uint4 cw = *reinterpret_cast<const uint4*>(crow + 16 * bb);
+            const uint32_t word = (words >> (16 * bb)) & 0xFFFFu;
+            const uint2 E = tab[(word >> 8) & 31u];
+            const uint2 o0 = decode8_e4m3(cw.x, E), o1 = decode8_e4m3(cw.y, E);
+            const uint2 o2 = decode8_e4m3(cw.z, E), o3 = decode8_e4m3(cw.w, E);
+            const int q = 4 * h + 2 * bb;  // 16-byte chunk of the 128-byte row
+            *reinterpret_cast<uint4*>(orow_p + ((q ^ (rr & 7)) << 4)) =
+                make_uint4(o0.x, o0.y, o1.x, o1.y);
+            *reinterpret_cast<uint4*>(orow_p + (((q + 1) ^ (rr & 7)) << 4)) =
+                make_uint4(o2.x, o2.y, o3.x, o3.y);
+          }
+          // the two blocks' UE8M0 scales: e + 127
+          const uint32_t e0 = static_cast<uint32_t>(static_cast<int>(static_cast<int8_t>(words & 0xFFu)) + 127);
+          const uint32_t e1 = static_cast<uint32_t>(static_cast<int>(static_cast<int8_t>((words >> 16) & 0xFFu)) + 127);
+          *reinterpret_cast<uint16_t*>(sf + (is_b ? kSfA : 0) + sf_row_offset(rr) + 2 * h) =
+              static_cast<uint16_t>(e0 | (e1 << 8));
+        }
+        if (WDEC) {  // the decoded weights' scales: one 4-byte word per row
+          for (int n = dt; n < BN; n += C::kDecThreads) {
+            const uint32_t w01 = *reinterpret_cast<const uint32_t*>(mt + kMetaA + n * 16 + (kb & 1) * 8);
+            const uint32_t w23 = *reinterpret_cast<const uint32_t*>(mt + kMetaA + n * 16 + (kb & 1) * 8 + 4);
+            uint32_t v = 0;
+            const uint32_t wv[2] = {w01, w23};
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              v |= static_cast<uint32_t>(
+                       static_cast<int>(static_cast<int8_t>((wv[k >> 1] >> (16 * (k & 1))) & 0xFFu)) + 127)
+                   << (8 * k);
+            *reinterpret_cast<uint32_t*>(sf + kSfA + sf_row_offset(n)) = v;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bars.op_full(so));
+          mbar_arrive(bars.pk_empty(s));
+          if ((kb & 1) == 1) mbar_arrive(bars.meta_empty(ms));
+        }
+        if (++s == C::kPkStages) { s = 0; ph ^= 1u; }
+        if (++so == C::kOpStages) { so = 0; pho ^= 1u; }
+        if ((kb & 1) == 1 && ++ms == C::kMetaSlots) { ms = 0; mph ^= 1u; }
+      }
+    }
+    // drain: the MMA's last releases of the operand stages have landed
+    if (lane == 0)
+      for (int i = 0; i < C::kOpStages; ++i) {
+        if (!mbar_wait_bounded(bars.op_empty(so), pho ^ 1u, abort_flag, kErrWaitUnpack)) break;
+        if (++so == C::kOpStages) { so = 0; pho ^= 1u; }
+      }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    const unsigned long long t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// e4m3 bytes of an SD4 matrix (the magnitudes L/8 with their signs; the
+// block words keep the scales): one thread per 16 elements.
+__global__ void __launch_bounds__(256) sd4_decode_e4m3_kernel(const uint8_t* __restrict__ codes,
+                                                              const uint16_t* __restrict__ meta,
+                                                              int64_t rows, int K,
+                                                              uint8_t* __restrict__ out) {
+  __shared__ uint2 tab[kDialects];
+  for (int d = threadIdx.x; d < kDialects; d += blockDim.x) {
+    uint32_t lo = 0, hi = 0;
+    for (int i = 0; i < 4; ++i) {
+      lo |= e4m3_eighths(level(d, i)) << (8 * i);
+      hi |= e4m3_eighths(level(d, i + 4)) << (8 * i);
+    }
+    tab[d] = make_uint2(lo, hi);
+  }
+  __syncthreads();
+  const int64_t per_row = K / 16;
+  const int64_t n = rows * per_row;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < n;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = t / per_row;
+    const int c = static_cast<int>(t % per_row);
+    const uint2 cw = *reinterpret_cast<const uint2*>(codes + row * (K / 2) + c * 8);
+    const uint2 E = tab[(meta[row * (K / 32) + c / 2] >> 8) & 31u];
+    const uint2 lo = decode8_e4m3(cw.x, E), hi = decode8_e4m3(cw.y, E);
+    *reinterpret_cast<uint4*>(out + row * static_cast<int64_t>(K) + c * 16) =
+        make_uint4(lo.x, lo.y, hi.x, hi.y);
+  }
+}
+
+}  // namespace gemm_mx
+}  // namespace sd4
+}  // namespace qs

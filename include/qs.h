@@ -305,10 +305,11 @@ QS_API qs_status qs_sd4_quant(const void* x_bf16, int64_t rows, int64_t K, void*
 /*
  * qs_sd4_linear — the SD4 layer: out[m][n] = bf16(fl(sum_k x_hat w_hat) + bias[n])
  * with x_hat, w_hat the decoded SD4 values of qs_sd4_quant(x) and
- * qs_sd4_quant(W).  The decoded values are exact in bf16; the product runs on
- * the tensor cores in bf16 with binary32 accumulation, so the sum is the exact
- * one up to binary32 accumulation rounding (parity is checked within that
- * bound).  K % 256 == 0, N % 16 == 0; bias NULL adds +0.0.
+ * qs_sd4_quant(W).  Each decoded value is an e4m3 number (L/8, signed) times
+ * its block's power of two, so the product runs on the block-scaled fp8
+ * tensor-core path (one UE8M0 scale per 32 elements along K): the products
+ * are exact and summed with binary32 accumulation (parity is checked within
+ * that bound).  K % 256 == 0, N % 16 == 0; bias NULL adds +0.0.
  *   out_bf16  [M, N] bf16, written
  */
 QS_API qs_status qs_sd4_linear(const void* x_codes, const uint16_t* x_meta, const void* w_codes,
@@ -325,13 +326,36 @@ QS_API qs_status qs_sd4_decode(const void* codes, const uint16_t* meta, int64_t 
                                void* out_bf16, void* stream);
 
 /*
- * qs_sd4_linear_wdec — qs_sd4_linear with the weights given decoded
- * (qs_sd4_decode of qs_sd4_quant(W)); the same arithmetic, bit-identical
- * outputs.  w_bf16 [N, K].
+ * qs_sd4_linear_wdec — the SD4 layer with the weights given decoded to bf16
+ * (qs_sd4_decode of qs_sd4_quant(W)), on the bf16 tensor-core path (the
+ * activations decoded to bf16 in the kernel).  The same exact products with
+ * binary32 accumulation as qs_sd4_linear (outputs may differ from it only by
+ * the accumulation order).  w_bf16 [N, K].
  */
 QS_API qs_status qs_sd4_linear_wdec(const void* x_codes, const uint16_t* x_meta,
                                     const void* w_bf16, const void* bias_bf16, int64_t M,
                                     int64_t N, int64_t K, void* out_bf16, void* stream);
+
+/*
+ * qs_sd4_decode_e4m3 — the e4m3 bytes of an SD4 matrix: element k of a row
+ * is the e4m3 encoding of its signed L/8 (exact); the block words keep the
+ * block scales.  Offline use for the weights: qs_sd4_linear_e4m3w then loads
+ * them by TMA straight into the GEMM's operand tiles, at one byte per weight.
+ *   codes [rows, K/2], meta [rows, K/32] (qs_sd4_quant); out_e4m3 [rows, K] bytes
+ */
+QS_API qs_status qs_sd4_decode_e4m3(const void* codes, const uint16_t* meta, int64_t rows,
+                                    int64_t K, void* out_e4m3, void* stream);
+
+/*
+ * qs_sd4_linear_e4m3w — qs_sd4_linear with the weights given as
+ * qs_sd4_decode_e4m3 bytes (w_e4m3 [N, K]) and their block words
+ * (w_meta [N, K/32]); only the activations are decoded per call.  The same
+ * arithmetic as qs_sd4_linear.
+ */
+QS_API qs_status qs_sd4_linear_e4m3w(const void* x_codes, const uint16_t* x_meta,
+                                     const void* w_e4m3, const uint16_t* w_meta,
+                                     const void* bias_bf16, int64_t M, int64_t N, int64_t K,
+                                     void* out_bf16, void* stream);
 
 /*
  * Activation decomposition (SemanticDialect "Resumen técnico" §2.B): a salient
@@ -358,18 +382,19 @@ QS_API qs_status qs_sd4_quant_decomp(const void* x_bf16, int64_t M, int64_t K,
 /*
  * qs_sd4_linear_decomp — the decomposed rows of the SD4 layer: for i < S,
  *   out[rows[i]][n] = bf16(fl(sum_k (x_hat + delta_hat)[k] w_hat[n][k]) + bias[n])
- * as one binary32 tensor-core accumulation over the 2K products of a
- * qs_sd4_quant_decomp row with [w_hat | w_hat].  Only those rows of out are
- * written: the layer with decomposition is qs_sd4_linear (or _wdec) over all
- * M rows followed, on the same stream, by this call.  The weights are given
- * either as codes (w_codes [N, K/2], w_meta [N, K/32]) or, when w_bf16 is not
- * NULL, decoded (qs_sd4_decode, [N, K]; w_codes and w_meta are then ignored).
+ * as one binary32 accumulation (block-scaled fp8 tensor cores, as
+ * qs_sd4_linear) over the 2K products of a qs_sd4_quant_decomp row with
+ * [w_hat | w_hat].  Only those rows of out are written: the layer with
+ * decomposition is qs_sd4_linear (or _e4m3w) over all M rows followed, on the
+ * same stream, by this call.  The weights: their block words w_meta
+ * [N, K/32] and either their codes (w_codes [N, K/2]) or, when w_e4m3 is not
+ * NULL, their qs_sd4_decode_e4m3 bytes ([N, K]; w_codes is then ignored).
  * An index outside [0, M) is skipped and reported as in qs_sd4_quant_decomp.
  *   out_bf16  [M, N] bf16, rows rows[i] written
  */
 QS_API qs_status qs_sd4_linear_decomp(const void* codes2, const uint16_t* meta2,
                                       const int32_t* rows, int64_t S, const void* w_codes,
-                                      const uint16_t* w_meta, const void* w_bf16,
+                                      const uint16_t* w_meta, const void* w_e4m3,
                                       const void* bias_bf16, int64_t M, int64_t N, int64_t K,
                                       void* out_bf16, void* stream);
 

@@ -256,10 +256,19 @@ def test_sd4_validation(lib):
     assert g(A, 8, 32768 + 256, B, 4, C, D, NUL) == RANGE   # 2K codes per row
     assert g(A, 8, 256, ctypes.c_void_p(0x20002), 4, C, D, NUL) == ALIGN
     h = lib.qs_sd4_linear_decomp
-    assert h(A, B, C, 4, NUL, NUL, NUL, NUL, 8, 256, 256, D, NUL) == NULL   # no weights
+    assert h(A, B, C, 4, NUL, D, NUL, NUL, 8, 256, 256, D, NUL) == NULL     # no weights
     assert h(A, B, C, 4, A, NUL, NUL, NUL, 8, 256, 256, D, NUL) == NULL     # codes without words
-    assert h(A, B, C, 4, NUL, NUL, D, NUL, 8, 264, 256, D, NUL) == SHAPE
-    assert h(A, B, C, 4, NUL, NUL, D, NUL, 8, 256, 384, D, NUL) == SHAPE
-    assert h(A, B, C, 4, NUL, NUL, D, NUL, 8, 256, 32768 + 256, D, NUL) == RANGE
-    assert h(A, B, C, 4, NUL, NUL, MIS, NUL, 8, 256, 256, D, NUL) == ALIGN
+    assert h(A, B, C, 4, NUL, NUL, D, NUL, 8, 256, 256, D, NUL) == NULL     # e4m3 without words
+    assert h(A, B, C, 4, NUL, D, D, NUL, 8, 264, 256, D, NUL) == SHAPE
+    assert h(A, B, C, 4, NUL, D, D, NUL, 8, 256, 384, D, NUL) == SHAPE
+    assert h(A, B, C, 4, NUL, D, D, NUL, 8, 256, 32768 + 256, D, NUL) == RANGE
+    assert h(A, B, C, 4, NUL, D, MIS, NUL, 8, 256, 256, D, NUL) == ALIGN
     assert h(A, B, ctypes.c_void_p(0x30002), 4, A, B, NUL, NUL, 8, 256, 256, D, NUL) == ALIGN
+    assert lib.qs_sd4_decode_e4m3(A, B, 4, 128, C, NUL) == SHAPE
+    assert lib.qs_sd4_decode_e4m3(A, NUL, 4, 256, C, NUL) == NULL
+    assert lib.qs_sd4_decode_e4m3(A, B, 4, 256, MIS, NUL) == ALIGN
+    e = lib.qs_sd4_linear_e4m3w
+    assert e(A, B, C, NUL, NUL, 8, 256, 256, D, NUL) == NULL                # block words required
+    assert e(A, B, C, D, NUL, 8, 200, 256, D, NUL) == SHAPE
+    assert e(A, B, C, D, NUL, 8, 256, 256 + 128, D, NUL) == SHAPE
+    assert e(A, B, C, D, MIS, 8, 256, 256, D, NUL) == ALIGN

@@ -135,14 +135,36 @@ def test_sd4_decode_exact(R, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(127, 272, 256), (300, 768, 768), (513, 528, 1280)])
-def test_sd4_linear_with_decoded_weights_is_identical(M, N, K):
+def test_sd4_linear_e4m3_weights_identical_and_bf16_weights_within_bound(M, N, K):
     d, dev, out = _layer(M, N, K, seed=3 * M + N)
     cx, mx, cw, mw = dev
+    # e4m3 weights: the same kernel arithmetic as the codes form
+    w8 = qs.sd4_decode_e4m3(cw, mw)
+    out8 = torch.empty_like(out)
+    qs.qs_sd4_linear_e4m3w(cx, mx, w8, mw, d["bias"].cuda(), M, N, K, out8)
+    # bf16 weights: the bf16 tensor-core kernel, its own accumulation order
     wdec = qs.sd4_decode(cw, mw)
-    out2 = torch.empty_like(out)
-    qs.qs_sd4_linear_wdec(cx, mx, wdec, d["bias"].cuda(), M, N, K, out2)
+    out16 = torch.empty_like(out)
+    qs.qs_sd4_linear_wdec(cx, mx, wdec, d["bias"].cuda(), M, N, K, out16)
     torch.cuda.synchronize()
-    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+    assert torch.equal(out.view(torch.int16), out8.view(torch.int16))
+    _check_layer(d, dev, out16, K)
+
+
+@pytest.mark.parametrize("R,K", [(5, 256), (129, 5120)])
+def test_sd4_decode_e4m3_exact(R, K):
+    d = I.make_shape(seed=R + 2 * K, M=R, K=K, N=16, bits=4, outlier_factor=30.0)
+    codes, meta = qs.sd4_quant(d["x"].cuda())
+    got = qs.sd4_decode_e4m3(codes, meta).cpu()
+    torch.cuda.synchronize()
+    c, e, dd = S.quantize_rows(I.bf16_bits(d["x"]))
+    L = S.formatbook()
+    mag = L[np.repeat(dd, 32, axis=1), c & 7] / 8.0          # L/8, exact in e4m3
+    val = np.where(c & 8, -mag, mag)
+    want = torch.from_numpy(val).to(torch.float8_e4m3fn).view(torch.uint8)
+    # torch encodes -0.0 with the sign bit, as the kernel does for a negative level-0 code
+    assert torch.equal(got, want)
+    assert np.array_equal(got.view(torch.float8_e4m3fn).double().numpy(), val)
 
 
 # ------------------------------------------------- activation decomposition (§2.B)
@@ -242,8 +264,8 @@ def _decomp_layer(M, N, K, rows, seed, wdec, bias=True):
     cw, mw = qs.sd4_quant(w)
     rt = _rows_tensor(rows)
     codes2, meta2 = qs.sd4_quant_decomp(x, rt)
-    w_dec = qs.sd4_decode(cw, mw) if wdec else None
-    out = qs.sd4_linear_decomp(cx, mx, codes2, meta2, rt, cw, mw, b, K, w_dec=w_dec)
+    w8 = qs.sd4_decode_e4m3(cw, mw) if wdec else None
+    out = qs.sd4_linear_decomp(cx, mx, codes2, meta2, rt, cw, mw, b, K, w_e4m3=w8)
     torch.cuda.synchronize()
     return d, out
 
@@ -304,8 +326,8 @@ def test_sd4_linear_decomp_single_row_no_bias_and_forms_agree():
 @pytest.mark.slow
 def test_full_size_wan_ffn_decomp_sampled():
     """The Wan FFN layer (32760 x 5120 -> 13824) with 1/16 of the tokens
-    decomposed, in the decoded-weight form the benchmark times; sampled
-    outputs of salient and plain rows against the oracle."""
+    decomposed, in the e4m3-weight form the benchmark times; sampled outputs
+    of salient and plain rows against the oracle."""
     cfg = I.WAN_FFN
     d = I.make_layer(cfg)
     M, K, N = cfg.M, cfg.K, cfg.N
@@ -313,10 +335,10 @@ def test_full_size_wan_ffn_decomp_sampled():
     x, w, b = d["x"].cuda(), d["w"].cuda(), d["bias"].cuda()
     cx, mx = qs.sd4_quant(x)
     cw, mw = qs.sd4_quant(w)
-    wd = qs.sd4_decode(cw, mw)
+    w8 = qs.sd4_decode_e4m3(cw, mw)
     rt = _rows_tensor(rows)
     codes2, meta2 = qs.sd4_quant_decomp(x, rt)
-    out = qs.sd4_linear_decomp(cx, mx, codes2, meta2, rt, None, None, b, K, w_dec=wd)
+    out = qs.sd4_linear_decomp(cx, mx, codes2, meta2, rt, None, mw, b, K, w_e4m3=w8)
     torch.cuda.synchronize()
     rng = np.random.default_rng(4)
     pick_s = np.unique(np.concatenate([[0, len(rows) - 1], rng.choice(len(rows), 24, replace=False)]))
