@@ -455,6 +455,15 @@ def sd4_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
         g2 = timed(lambda: qs.qs_sd4_linear_wdec(cx, mx, wdec, b, M, N, K, out2, stream))
         g8 = timed(lambda: qs.qs_sd4_linear_e4m3w(cx, mx, w8, mw, b, M, N, K, out8, stream))
         same = bool(torch.equal(out.view(torch.int16), out8.view(torch.int16)))
+        # activations quantised straight to e4m3 bytes: nothing decoded in the GEMM
+        x8 = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        m8 = torch.empty((M, K // 32), dtype=torch.int16, device=dev)
+        out88 = torch.empty_like(out)
+        qs.qs_sd4_quant_e4m3(x, M, K, x8, m8, stream)
+        qs.qs_sd4_linear_e4m3(x8, m8, w8, mw, b, M, N, K, out88, stream)
+        q8 = timed(lambda: qs.qs_sd4_quant_e4m3(x, M, K, x8, m8, stream))
+        g88 = timed(lambda: qs.qs_sd4_linear_e4m3(x8, m8, w8, mw, b, M, N, K, out88, stream))
+        same88 = bool(torch.equal(out.view(torch.int16), out88.view(torch.int16)))
         # activation decomposition of the salient tokens (a seeded 1/16 of them)
         srows = I.salient_rows(M, cfg.seed)
         S_ = len(srows)
@@ -502,6 +511,10 @@ def sd4_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
             "gemm_e4m3_weights_ms": g8, "gemm_e4m3_weights_TFLOPS": tf(g8),
             "gemm_e4m3_weights_frac_fp8_peak": tf(g8) / fp8_peak,
             "e4m3_weights_output_identical": same,
+            "quant_e4m3_ms": q8, "gemm_e4m3_both_ms": g88, "gemm_e4m3_both_TFLOPS": tf(g88),
+            "gemm_e4m3_both_frac_fp8_peak": tf(g88) / fp8_peak,
+            "e4m3_both_output_identical": same88,
+            "layer_e4m3_ms": q8 + g88, "layer_e4m3_TOPS": cfg.ops / ((q8 + g88) * 1e-3) / 1e12,
             "gemm_bf16_weights_ms": g2, "gemm_bf16_weights_TFLOPS": tf(g2),
             "gemm_bf16_weights_frac_bf16_peak": tf(g2) / pk["bf16_tflops"],
             "quant_GBps": quant_bytes / (q * 1e-3) / 1e9,

@@ -30,11 +30,11 @@ STATUS = {0: "QS_OK", 1: "QS_ERR_NULL", 2: "QS_ERR_SHAPE", 3: "QS_ERR_BITS", 4: 
 EXPORTS = ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qlinear_mixed", "qs_qgemm_s32",
            "qs_qgemm_s32_mixed", "qs_gelu_bf16", "qs_linear_workspace_bytes", "qs_linear",
            "qs_linear_mixed", "qs_linear_ex", "qs_linear_noalloc", "qs_pack_weights_bgr",
-           "qs_quant_act_rowsum",
-           "qs_qlinear_asym", "qs_qgemm_s32_asym", "qs_linear_bgr_workspace_bytes",
-           "qs_linear_bgr", "qs_sd4_quant", "qs_sd4_linear", "qs_sd4_decode",
-           "qs_sd4_linear_wdec", "qs_sd4_quant_decomp", "qs_sd4_linear_decomp",
-           "qs_sd4_decode_e4m3", "qs_sd4_linear_e4m3w", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
+           "qs_quant_act_rowsum", "qs_qlinear_asym", "qs_qgemm_s32_asym",
+           "qs_linear_bgr_workspace_bytes", "qs_linear_bgr", "qs_sd4_quant", "qs_sd4_quant_e4m3",
+           "qs_sd4_linear", "qs_sd4_decode", "qs_sd4_linear_wdec", "qs_sd4_decode_e4m3",
+           "qs_sd4_linear_e4m3w", "qs_sd4_linear_e4m3", "qs_sd4_quant_decomp",
+           "qs_sd4_linear_decomp", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
            "qs_selftest_timeout", "qs_device_error", "qs_status_str", "qs_version")
 BITS = (4, 6, 8)
 QS_GBS_MAX_BLOCKS = 1024
@@ -91,6 +91,8 @@ def load() -> ctypes.CDLL:
     L.qs_sd4_linear_decomp.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, i64, i64, i64, vp, vp]
     L.qs_sd4_decode_e4m3.argtypes = [vp, vp, i64, i64, vp, vp]
     L.qs_sd4_linear_e4m3w.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]
+    L.qs_sd4_quant_e4m3.argtypes = [vp, i64, i64, vp, vp, vp]
+    L.qs_sd4_linear_e4m3.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]
     L.qs_gbs_reset.argtypes = [vp, vp]
     L.qs_gbs_update.argtypes = [vp, vp, i64, f64, vp, vp]
     L.qs_linear_gbs.argtypes = [vp, i64, i64, f32, vp, vp, vp, vp, vp, i64, vp, vp, i64, vp, vp]
@@ -103,10 +105,10 @@ def load() -> ctypes.CDLL:
                  "qs_qgemm_s32", "qs_qgemm_s32_mixed", "qs_gelu_bf16", "qs_linear",
                  "qs_linear_mixed", "qs_linear_ex", "qs_linear_noalloc", "qs_pack_weights_bgr",
                  "qs_quant_act_rowsum", "qs_qlinear_asym", "qs_qgemm_s32_asym", "qs_linear_bgr",
-                 "qs_sd4_quant", "qs_sd4_linear", "qs_sd4_decode", "qs_sd4_linear_wdec",
-                 "qs_sd4_quant_decomp", "qs_sd4_linear_decomp", "qs_sd4_decode_e4m3",
-           "qs_sd4_linear_e4m3w", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
-                 "qs_selftest_timeout",
+                 "qs_sd4_quant", "qs_sd4_quant_e4m3", "qs_sd4_linear", "qs_sd4_decode",
+                 "qs_sd4_linear_wdec", "qs_sd4_decode_e4m3", "qs_sd4_linear_e4m3w",
+                 "qs_sd4_linear_e4m3", "qs_sd4_quant_decomp", "qs_sd4_linear_decomp",
+                 "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs", "qs_selftest_timeout",
                  "qs_device_error"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -452,6 +454,32 @@ def sd4_linear_decomp(x_codes, x_meta, codes2, meta2, rows, w_codes, w_meta, bia
                          None if w_e4m3 is not None else w_codes, w_meta, w_e4m3, bias, M, N, K,
                          out, stream)
     return out
+
+
+def qs_sd4_quant_e4m3(x, rows, K, out, meta, stream=None):
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(out, torch.uint8, "out")
+    _cuda(meta, torch.int16, "meta")
+    _check(load().qs_sd4_quant_e4m3(_p(x), rows, K, _p(out), _p(meta), _s(stream)),
+           "qs_sd4_quant_e4m3")
+
+
+def sd4_quant_e4m3(x: torch.Tensor, stream=None):
+    """x bf16 [R, K] -> (e4m3 bytes uint8 [R, K], meta int16 [R, K/32])."""
+    R, K = x.shape
+    out = torch.empty((R, K), dtype=torch.uint8, device=x.device)
+    meta = torch.empty((R, K // 32), dtype=torch.int16, device=x.device)
+    qs_sd4_quant_e4m3(x, R, K, out, meta, stream)
+    return out, meta
+
+
+def qs_sd4_linear_e4m3(x_e4m3, x_meta, w_e4m3, w_meta, bias, M, N, K, out, stream=None):
+    for t, name, dt in ((x_e4m3, "x_e4m3", torch.uint8), (x_meta, "x_meta", torch.int16),
+                        (w_e4m3, "w_e4m3", torch.uint8), (w_meta, "w_meta", torch.int16),
+                        (bias, "bias", torch.bfloat16), (out, "out", torch.bfloat16)):
+        _cuda(t, dt, name)
+    _check(load().qs_sd4_linear_e4m3(_p(x_e4m3), _p(x_meta), _p(w_e4m3), _p(w_meta), _p(bias),
+                                     M, N, K, _p(out), _s(stream)), "qs_sd4_linear_e4m3")
 
 
 def qs_gbs_reset(state, stream=None):

@@ -127,14 +127,15 @@ qs_status launch_sd4_gemm(const CUtensorMap& ca, const CUtensorMap& cb, const CU
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
-template <bool WDEC>
+template <bool ADEC, bool BDEC>
 qs_status launch_sd4_mx(const CUtensorMap& ca, const CUtensorMap& cb, const CUtensorMap& ma,
-                        const CUtensorMap& mb, const CUtensorMap& wb, const void* bias, int64_t M,
-                        int64_t N, int64_t K, void* out, void* stream, int64_t kb_wrap,
-                        const int32_t* out_rows, int64_t out_M) {
+                        const CUtensorMap& mb, const CUtensorMap& xa, const CUtensorMap& wb,
+                        const void* bias, int64_t M, int64_t N, int64_t K, void* out,
+                        void* stream, int64_t kb_wrap, const int32_t* out_rows, int64_t out_M) {
   namespace G = qs::sd4::gemm_mx;
-  constexpr int smem = G::MCfg<WDEC>::kSmemBytes;
-  auto kern = G::sd4_mx_gemm_kernel<WDEC>;
+  using C = G::MCfg<ADEC, BDEC>;
+  constexpr int smem = C::kSmemBytes;
+  auto kern = G::sd4_mx_gemm_kernel<ADEC, BDEC>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return QS_ERR_CUDA;
@@ -142,42 +143,49 @@ qs_status launch_sd4_mx(const CUtensorMap& ca, const CUtensorMap& cb, const CUte
   if (sms <= 0) return QS_ERR_CUDA;
   const int64_t tiles = ((M + G::BM - 1) / G::BM) * ((N + G::BN - 1) / G::BN);
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  kern<<<grid, G::MCfg<WDEC>::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(
-      ca, cb, ma, mb, wb, static_cast<const uint16_t*>(bias), static_cast<uint16_t*>(out),
+  kern<<<grid, C::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+      ca, cb, ma, mb, xa, wb, static_cast<const uint16_t*>(bias), static_cast<uint16_t*>(out),
       static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(kb_wrap),
       out_rows, static_cast<int>(out_rows ? out_M : M));
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
-// The block-scaled SD4 GEMM: A = `a_rows` rows of Ka codes (Ka = K, or 2K for
-// decomposed rows), the weights as codes + block words or, when w_e4m3 is not
-// NULL, as e4m3 bytes + block words.
-qs_status run_sd4_mx(const void* a_codes, const uint16_t* a_meta, int64_t a_rows, int64_t Ka,
-                     const void* w_codes, const uint16_t* w_meta, const void* w_e4m3,
-                     const void* bias, int64_t N, int64_t K, void* out, void* stream,
-                     const int32_t* out_rows, int64_t out_M) {
+// The block-scaled SD4 GEMM: A = `a_rows` rows of Ka elements (Ka = K, or 2K
+// for decomposed rows) as codes or, when a_e4m3 is not NULL, as e4m3 bytes;
+// the weights as codes or, when w_e4m3 is not NULL, as e4m3 bytes; block
+// words for both.
+qs_status run_sd4_mx(const void* a_codes, const void* a_e4m3, const uint16_t* a_meta,
+                     int64_t a_rows, int64_t Ka, const void* w_codes, const void* w_e4m3,
+                     const uint16_t* w_meta, const void* bias, int64_t N, int64_t K, void* out,
+                     void* stream, const int32_t* out_rows, int64_t out_M) {
   namespace G = qs::sd4::gemm_mx;
-  CUtensorMap ca, ma, cb, mb, wb;
-  if (!qs::make_tensor_map_2d(&ca, a_codes, static_cast<uint64_t>(Ka) / 2,
-                              static_cast<uint64_t>(a_rows), G::BK / 2, G::BM, false) ||
-      !qs::make_tensor_map_2d(&ma, a_meta, static_cast<uint64_t>(Ka) / 16,
+  CUtensorMap ca, ma, cb, mb, xa, wb;
+  if (!qs::make_tensor_map_2d(&ma, a_meta, static_cast<uint64_t>(Ka) / 16,
                               static_cast<uint64_t>(a_rows), 16, G::BM, false) ||
       !qs::make_tensor_map_2d(&mb, w_meta, static_cast<uint64_t>(K) / 16,
                               static_cast<uint64_t>(N), 16, G::BN, false))
     return QS_ERR_CUDA;
-  const int64_t kb_wrap = K / G::BK;
-  if (w_e4m3) {
-    if (!qs::make_tensor_map_2d(&wb, w_e4m3, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
-                                G::BK, G::BN, true))
-      return QS_ERR_CUDA;
-    return launch_sd4_mx<true>(ca, ca, ma, mb, wb, bias, a_rows, N, Ka, out, stream, kb_wrap,
-                               out_rows, out_M);
-  }
-  if (!qs::make_tensor_map_2d(&cb, w_codes, static_cast<uint64_t>(K) / 2,
-                              static_cast<uint64_t>(N), G::BK / 2, G::BN, false))
+  if (a_e4m3 ? !qs::make_tensor_map_2d(&xa, a_e4m3, static_cast<uint64_t>(Ka),
+                                       static_cast<uint64_t>(a_rows), G::BK, G::BM, true)
+             : !qs::make_tensor_map_2d(&ca, a_codes, static_cast<uint64_t>(Ka) / 2,
+                                       static_cast<uint64_t>(a_rows), G::BK / 2, G::BM, false))
     return QS_ERR_CUDA;
-  return launch_sd4_mx<false>(ca, cb, ma, mb, cb, bias, a_rows, N, Ka, out, stream, kb_wrap,
-                              out_rows, out_M);
+  if (w_e4m3 ? !qs::make_tensor_map_2d(&wb, w_e4m3, static_cast<uint64_t>(K),
+                                       static_cast<uint64_t>(N), G::BK, G::BN, true)
+             : !qs::make_tensor_map_2d(&cb, w_codes, static_cast<uint64_t>(K) / 2,
+                                       static_cast<uint64_t>(N), G::BK / 2, G::BN, false))
+    return QS_ERR_CUDA;
+  const int64_t kb_wrap = K / G::BK;
+  if (a_e4m3) {
+    if (!w_e4m3) return QS_ERR_NULL;  // e4m3 activations go with e4m3 weights
+    return launch_sd4_mx<false, false>(xa, xa, ma, mb, xa, wb, bias, a_rows, N, Ka, out, stream,
+                                       kb_wrap, out_rows, out_M);
+  }
+  if (w_e4m3)
+    return launch_sd4_mx<true, false>(ca, ca, ma, mb, ca, wb, bias, a_rows, N, Ka, out, stream,
+                                      kb_wrap, out_rows, out_M);
+  return launch_sd4_mx<true, true>(ca, cb, ma, mb, ca, cb, bias, a_rows, N, Ka, out, stream,
+                                   kb_wrap, out_rows, out_M);
 }
 
 }  // namespace
@@ -537,10 +545,31 @@ qs_status qs_sd4_quant(const void* x_bf16, int64_t rows, int64_t K, void* codes,
   const int64_t chunks = rows * (K / 256);
   int64_t grid = (chunks + qs::sd4::kWarps - 1) / qs::sd4::kWarps;
   if (grid > static_cast<int64_t>(sms) * 4) grid = static_cast<int64_t>(sms) * 4;
-  qs::sd4::sd4_quant_kernel<<<static_cast<unsigned>(grid), qs::sd4::kThreads, 0,
-                              static_cast<cudaStream_t>(stream)>>>(
+  qs::sd4::sd4_quant_kernel<false><<<static_cast<unsigned>(grid), qs::sd4::kThreads, 0,
+                                     static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint16_t*>(x_bf16), rows, static_cast<int>(K),
       static_cast<uint8_t*>(codes), meta);
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status qs_sd4_quant_e4m3(const void* x_bf16, int64_t rows, int64_t K, void* out_e4m3,
+                            uint16_t* meta, void* stream) {
+  if (!x_bf16 || !out_e4m3 || !meta) return QS_ERR_NULL;
+  if (rows <= 0 || K <= 0 || K % 256 != 0) return QS_ERR_SHAPE;
+  if (K > QS_MAX_K || rows > QS_MAX_ROWS) return QS_ERR_RANGE;
+  if (!aligned16(x_bf16) || !aligned16(out_e4m3) || !aligned16(meta)) return QS_ERR_ALIGN;
+  QS_TRY(check_device_ptr(x_bf16));
+  QS_TRY(check_device_ptr(out_e4m3));
+  QS_TRY(check_device_ptr(meta));
+  const int sms = qs::sm_count();
+  if (sms <= 0) return QS_ERR_CUDA;
+  const int64_t chunks = rows * (K / 256);
+  int64_t grid = (chunks + qs::sd4::kWarps - 1) / qs::sd4::kWarps;
+  if (grid > static_cast<int64_t>(sms) * 4) grid = static_cast<int64_t>(sms) * 4;
+  qs::sd4::sd4_quant_kernel<true><<<static_cast<unsigned>(grid), qs::sd4::kThreads, 0,
+                                    static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(x_bf16), rows, static_cast<int>(K),
+      static_cast<uint8_t*>(out_e4m3), meta);
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
@@ -557,8 +586,8 @@ qs_status qs_sd4_linear(const void* x_codes, const uint16_t* x_meta, const void*
                         static_cast<const void*>(w_meta), static_cast<const void*>(out_bf16)})
     QS_TRY(check_device_ptr(p));
   if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
-  return run_sd4_mx(x_codes, x_meta, M, K, w_codes, w_meta, nullptr, bias_bf16, N, K, out_bf16,
-                    stream, nullptr, 0);
+  return run_sd4_mx(x_codes, nullptr, x_meta, M, K, w_codes, nullptr, w_meta, bias_bf16, N, K,
+                    out_bf16, stream, nullptr, 0);
 }
 
 qs_status qs_sd4_decode_e4m3(const void* codes, const uint16_t* meta, int64_t rows, int64_t K,
@@ -594,8 +623,25 @@ qs_status qs_sd4_linear_e4m3w(const void* x_codes, const uint16_t* x_meta, const
                         static_cast<const void*>(w_meta), static_cast<const void*>(out_bf16)})
     QS_TRY(check_device_ptr(p));
   if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
-  return run_sd4_mx(x_codes, x_meta, M, K, nullptr, w_meta, w_e4m3, bias_bf16, N, K, out_bf16,
-                    stream, nullptr, 0);
+  return run_sd4_mx(x_codes, nullptr, x_meta, M, K, nullptr, w_e4m3, w_meta, bias_bf16, N, K,
+                    out_bf16, stream, nullptr, 0);
+}
+
+qs_status qs_sd4_linear_e4m3(const void* x_e4m3, const uint16_t* x_meta, const void* w_e4m3,
+                             const uint16_t* w_meta, const void* bias_bf16, int64_t M, int64_t N,
+                             int64_t K, void* out_bf16, void* stream) {
+  if (!x_e4m3 || !x_meta || !w_e4m3 || !w_meta || !out_bf16) return QS_ERR_NULL;
+  if (M <= 0 || N <= 0 || K <= 0 || K % 256 != 0 || N % 16 != 0) return QS_ERR_SHAPE;
+  if (K > QS_MAX_K || M > INT32_MAX || N > INT32_MAX) return QS_ERR_RANGE;
+  if (!aligned16(x_e4m3) || !aligned16(x_meta) || !aligned16(w_e4m3) || !aligned16(w_meta) ||
+      !aligned16(out_bf16) || (bias_bf16 && !aligned16(bias_bf16)))
+    return QS_ERR_ALIGN;
+  for (const void* p : {x_e4m3, static_cast<const void*>(x_meta), w_e4m3,
+                        static_cast<const void*>(w_meta), static_cast<const void*>(out_bf16)})
+    QS_TRY(check_device_ptr(p));
+  if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
+  return run_sd4_mx(nullptr, x_e4m3, x_meta, M, K, nullptr, w_e4m3, w_meta, bias_bf16, N, K,
+                    out_bf16, stream, nullptr, 0);
 }
 
 qs_status qs_sd4_decode(const void* codes, const uint16_t* meta, int64_t rows, int64_t K,
@@ -684,7 +730,7 @@ qs_status qs_sd4_linear_decomp(const void* codes2, const uint16_t* meta2, const 
     QS_TRY(check_device_ptr(p));
   if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
   // A: S rows of 2K codes; the weights' K walked twice
-  return run_sd4_mx(codes2, meta2, S, 2 * K, w_e4m3 ? nullptr : w_codes, w_meta, w_e4m3,
+  return run_sd4_mx(codes2, nullptr, meta2, S, 2 * K, w_e4m3 ? nullptr : w_codes, w_e4m3, w_meta,
                     bias_bf16, N, K, out_bf16, stream, rows, M);
 }
 

@@ -90,6 +90,41 @@ __device__ void build_tables(Tables* tb) {
   __syncthreads();
 }
 
+// e4m3 encoding of L/8, 0 <= L <= 15 (normal for L >= 1: exponent field
+// p + 4 with p = floor(log2 L), mantissa (L - 2^p) 2^(3-p)).
+__host__ __device__ constexpr uint32_t e4m3_eighths(int L) {
+  return L == 0 ? 0u
+                : static_cast<uint32_t>(
+                      (((L >= 8 ? 3 : L >= 4 ? 2 : L >= 2 ? 1 : 0) + 4) << 3) |
+                      ((L - (1 << (L >= 8 ? 3 : L >= 4 ? 2 : L >= 2 ? 1 : 0)))
+                       << (3 - (L >= 8 ? 3 : L >= 4 ? 2 : L >= 2 ? 1 : 0))));
+}
+
+// Eight codes (element k in nibble k) -> eight e4m3 bytes.  E: the dialect's
+// magnitudes e4m3(L_i/8), byte i of the pair (lo, hi); `prmt` picks byte i for
+// each code's level index, and the code's sign bit (nibble bit 3) moves to
+// bit 7 of its byte.
+__device__ __forceinline__ uint2 decode8_e4m3(uint32_t w, uint2 E) {
+  const uint32_t v03 = __byte_perm(E.x, E.y, w & 0x7777u);
+  const uint32_t v47 = __byte_perm(E.x, E.y, (w >> 16) & 0x7777u);
+  const uint32_t s = w & 0x88888888u;
+  const uint32_t t03 = __byte_perm(s, 0u, 0x1100u);  // bytes s0 s0 s1 s1
+  const uint32_t t47 = __byte_perm(s, 0u, 0x3322u);  // bytes s2 s2 s3 s3
+  const uint32_t s03 = ((t03 << 4) & 0x00800080u) | (t03 & 0x80008000u);
+  const uint32_t s47 = ((t47 << 4) & 0x00800080u) | (t47 & 0x80008000u);
+  return make_uint2(v03 | s03, v47 | s47);
+}
+
+// Byte i of the pair (lo, hi): e4m3(L[d][i] / 8) of dialect d.
+__device__ __forceinline__ uint2 e4m3_levels(int d) {
+  uint32_t lo = 0, hi = 0;
+  for (int i = 0; i < 4; ++i) {
+    lo |= e4m3_eighths(level(d, i)) << (8 * i);
+    hi |= e4m3_eighths(level(d, i + 4)) << (8 * i);
+  }
+  return make_uint2(lo, hi);
+}
+
 // 2^n as binary32 for n in [-127, 127] (n = -127: the subnormal 2^-127).
 __device__ __forceinline__ float pow2f(int n) {
   return n >= -126 ? __int_as_float((n + 127) << 23) : __int_as_float(0x00400000);
@@ -169,13 +204,28 @@ __device__ __forceinline__ uint16_t block_word(int e, int d) {
                                (static_cast<uint32_t>(d) << 8));
 }
 
+// E4M3: instead of packed codes, each element's value as an e4m3 byte (the
+// sign and L/8; the block words keep the scales): [rows, K] bytes.
+template <bool E4M3>
 __global__ void __launch_bounds__(kThreads) sd4_quant_kernel(const uint16_t* __restrict__ x,
                                                             int64_t rows, int K,
                                                             uint8_t* __restrict__ codes,
                                                             uint16_t* __restrict__ meta) {
   __shared__ Tables tb;
   __shared__ __align__(16) uint8_t s_bins[kWarps][8][kBlock];
+  __shared__ uint2 s_e4m3[E4M3 ? kDialects : 1];
   build_tables(&tb);
+  if (E4M3) {
+    for (int d = threadIdx.x; d < kDialects; d += blockDim.x) {
+      uint32_t lo = 0, hi = 0;
+      for (int i = 0; i < 4; ++i) {
+        lo |= e4m3_eighths(tb.lvl[d][i]) << (8 * i);
+        hi |= e4m3_eighths(tb.lvl[d][i + 4]) << (8 * i);
+      }
+      s_e4m3[d] = make_uint2(lo, hi);
+    }
+    __syncthreads();
+  }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int blocks_per_row = K / kBlock;
@@ -189,8 +239,12 @@ __global__ void __launch_bounds__(kThreads) sd4_quant_kernel(const uint16_t* __r
     load_chunk8(x + row * static_cast<int64_t>(K) + col0, lane, a);
     int e, d;
     const uint32_t packed = quant_warp_chunk(a, tb, s_bins[warp], lane, e, d);
-    *reinterpret_cast<uint32_t*>(codes + row * static_cast<int64_t>(K / 2) + col0 / 2 + 4 * lane) =
-        packed;
+    if (E4M3)
+      *reinterpret_cast<uint2*>(codes + row * static_cast<int64_t>(K) + col0 + 8 * lane) =
+          decode8_e4m3(packed, s_e4m3[d]);
+    else
+      *reinterpret_cast<uint32_t*>(codes + row * static_cast<int64_t>(K / 2) + col0 / 2 +
+                                   4 * lane) = packed;
     if ((lane & 3) == 0) meta[row * blocks_per_row + col0 / kBlock + (lane >> 2)] = block_word(e, d);
   }
 }

@@ -42,21 +42,26 @@ constexpr int kPkA = BM * BK / 2, kPkB = BN * BK / 2;  // code tiles, 64-byte ro
 constexpr int kMetaA = BM * 16, kMetaB = BN * 16;      // 8 block words per row = 2 stages
 static_assert(BN % 32 == 0 && BN <= 256 && 2 * BN + 12 <= kTmemCols, "tile");
 
-// WDEC: the weights come as e4m3 bytes (qs_sd4_decode_e4m3), loaded by TMA
-// straight into their operand tile; their block words still give the scales.
-template <bool WDEC>
+// ADEC / BDEC: the activations / weights come as SD4 codes and are decoded
+// to e4m3 in the kernel; otherwise as e4m3 bytes (qs_sd4_quant_e4m3,
+// qs_sd4_decode_e4m3) that TMA loads straight into their operand tile.  The
+// block words give the scales in every case.
+template <bool ADEC, bool BDEC>
 struct MCfg {
-  static constexpr int kDecWarps = WDEC ? 8 : 10;
+  static constexpr bool kAnyDec = ADEC || BDEC;
+  static constexpr int kDecWarps = ADEC ? (BDEC ? 10 : 8) : 4;
   static constexpr int kDecThreads = 32 * kDecWarps;
   static constexpr int kThreads = 32 * (2 + kEpiWarps + kDecWarps);
-  static constexpr int kOpStages = WDEC ? 4 : 3;
-  static constexpr int kPkStages = WDEC ? 4 : 3;
+  static constexpr int kOpStages = kAnyDec ? (BDEC ? 3 : 4) : 5;
+  static constexpr int kPkStages = kAnyDec ? kOpStages : 0;
   static constexpr int kMetaSlots = 2;
-  static constexpr int kDecRows = WDEC ? BM : BM + BN;  // rows decoded per stage
-  static constexpr int kTasks = 2 * kDecRows;           // (row, half of the stage's K)
+  static constexpr int kDecRows = (ADEC ? BM : 0) + (BDEC ? BN : 0);  // rows decoded per stage
+  static constexpr int kTasks = 2 * kDecRows;  // (row, half of the stage's K)
   static constexpr int kOpStage = kOpA + kOpB;
   static constexpr int kSfStage = kSfA + kSfB;
-  static constexpr int kPkStage = WDEC ? kPkA : kPkA + kPkB;
+  static constexpr int kPkStage = (ADEC ? kPkA : 0) + (BDEC ? kPkB : 0);
+  // operand bytes TMA writes straight into an operand stage
+  static constexpr int kDirectBytes = (ADEC ? 0 : kOpA) + (BDEC ? 0 : kOpB);
   static constexpr int kMetaSlot = kMetaA + kMetaB;
   static constexpr int kOffOp = 0;
   static constexpr int kOffSf = kOffOp + kOpStages * kOpStage;
@@ -69,22 +74,13 @@ struct MCfg {
   static constexpr int kOffMisc = kOffTab + kDialects * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   // arrivals completing an operand stage: the decode warps, plus the
-  // producer's arm of the decoded weight tile's TMA bytes
-  static constexpr int kOpFullCount = kDecWarps + (WDEC ? 1 : 0);
+  // producer's arm of the direct operands' TMA bytes
+  static constexpr int kOpFullCount = kDecWarps + (kDirectBytes ? 1 : 0);
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
   static_assert(kOffSf % 1024 == 0 && kOffPk % 128 == 0 && kOffMeta % 128 == 0, "alignment");
   static_assert(kTasks % kDecThreads == 0, "decode split");
+  static_assert(!BDEC || ADEC, "codes for W with e4m3 x is not a form of this kernel");
 };
-
-// e4m3 encoding of L/8, 0 <= L <= 15 (normal for L >= 1: exponent field
-// p + 4 with p = floor(log2 L), mantissa (L - 2^p) 2^(3-p)).
-__host__ __device__ constexpr uint32_t e4m3_eighths(int L) {
-  return L == 0 ? 0u
-                : static_cast<uint32_t>(
-                      (((L >= 8 ? 3 : L >= 4 ? 2 : L >= 2 ? 1 : 0) + 4) << 3) |
-                      ((L - (1 << (L >= 8 ? 3 : L >= 4 ? 2 : L >= 2 ? 1 : 0)))
-                       << (3 - (L >= 8 ? 3 : L >= 4 ? 2 : L >= 2 ? 1 : 0))));
-}
 
 // Instruction descriptor of kind::mxf8f6f4.block_scale: e4m3 A and B, both
 // K-major, UE8M0 scales, binary32 accumulation; scale byte j of A and B.
@@ -126,21 +122,6 @@ __device__ __forceinline__ uint64_t smem_desc_sf(uint32_t addr) {
   return d;                                             // layout type 0: no swizzle
 }
 
-// Eight codes (element k in nibble k) -> eight e4m3 bytes.  E: the dialect's
-// magnitudes e4m3(L_i/8), byte i of the pair (lo, hi); `prmt` picks byte i for
-// each code's level index, and the code's sign bit (nibble bit 3) moves to
-// bit 7 of its byte.
-__device__ __forceinline__ uint2 decode8_e4m3(uint32_t w, uint2 E) {
-  const uint32_t v03 = __byte_perm(E.x, E.y, w & 0x7777u);
-  const uint32_t v47 = __byte_perm(E.x, E.y, (w >> 16) & 0x7777u);
-  const uint32_t s = w & 0x88888888u;
-  const uint32_t t03 = __byte_perm(s, 0u, 0x1100u);  // bytes s0 s0 s1 s1
-  const uint32_t t47 = __byte_perm(s, 0u, 0x3322u);  // bytes s2 s2 s3 s3
-  const uint32_t s03 = ((t03 << 4) & 0x00800080u) | (t03 & 0x80008000u);
-  const uint32_t s47 = ((t47 << 4) & 0x00800080u) | (t47 & 0x80008000u);
-  return make_uint2(v03 | s03, v47 | s47);
-}
-
 struct MBars {
   uint32_t base;
   int P, T, U;  // code stages, meta slots, operand stages
@@ -165,16 +146,19 @@ __device__ __forceinline__ int sf_row_offset(int m) {
 // the decomposed rows [Q(x) | Q(Delta)] against [w | w].  out_rows (nullable)
 // maps accumulator row m to its output row; an index outside [0, out_M) is
 // skipped and flagged.
-template <bool WDEC>
-__global__ void __launch_bounds__(MCfg<WDEC>::kThreads, 1)
+// tmCA / tmCB: the codes (when decoded), tmXA / tmWB: the e4m3 bytes (when
+// loaded directly), tmMA / tmMB: the block words.
+template <bool ADEC, bool BDEC>
+__global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
     sd4_mx_gemm_kernel(const __grid_constant__ CUtensorMap tmCA,
                        const __grid_constant__ CUtensorMap tmCB,
                        const __grid_constant__ CUtensorMap tmMA,
                        const __grid_constant__ CUtensorMap tmMB,
+                       const __grid_constant__ CUtensorMap tmXA,
                        const __grid_constant__ CUtensorMap tmWB, const uint16_t* __restrict__ bias,
                        uint16_t* __restrict__ out, int M, int N, int K, int kb_wrap,
                        const int32_t* __restrict__ out_rows, int out_M) {
-  using C = MCfg<WDEC>;
+  using C = MCfg<ADEC, BDEC>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
@@ -250,18 +234,23 @@ __global__ void __launch_bounds__(MCfg<WDEC>::kThreads, 1)
             tma_load_2d(dst + kMetaA, &tmMB, (kbw / 2) * 16, n0, bars.meta_full(ms));
             if (++ms == C::kMetaSlots) { ms = 0; mph ^= 1u; }
           }
-          if (!mbar_wait_bounded(bars.pk_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer)) break;
-          const uint32_t dst = sbase + C::kOffPk + s * C::kPkStage;
-          mbar_arrive_expect_tx(bars.pk_full(s), C::kPkStage);
-          tma_load_2d(dst, &tmCA, kb * (BK / 2), m0, bars.pk_full(s));
-          if (!WDEC) tma_load_2d(dst + kPkA, &tmCB, kbw * (BK / 2), n0, bars.pk_full(s));
-          if (++s == C::kPkStages) { s = 0; ph ^= 1u; }
-          if (WDEC) {  // decoded weights: TMA into the operand stage's B tile
+          if (C::kAnyDec) {  // codes of the decoded operands
+            if (!mbar_wait_bounded(bars.pk_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer))
+              break;
+            const uint32_t dst = sbase + C::kOffPk + s * C::kPkStage;
+            mbar_arrive_expect_tx(bars.pk_full(s), C::kPkStage);
+            if (ADEC) tma_load_2d(dst, &tmCA, kb * (BK / 2), m0, bars.pk_full(s));
+            if (BDEC)
+              tma_load_2d(dst + (ADEC ? kPkA : 0), &tmCB, kbw * (BK / 2), n0, bars.pk_full(s));
+            if (++s == C::kPkStages) { s = 0; ph ^= 1u; }
+          }
+          if (C::kDirectBytes) {  // e4m3 operands: TMA into the operand stage
             if (!mbar_wait_bounded(bars.op_empty(so), pho ^ 1u, abort_flag, kErrWaitProducer))
               break;
-            const uint32_t ob = sbase + C::kOffOp + so * C::kOpStage + kOpA;
-            mbar_arrive_expect_tx(bars.op_full(so), kOpB);
-            tma_load_2d(ob, &tmWB, kbw * BK, n0, bars.op_full(so));
+            const uint32_t ob = sbase + C::kOffOp + so * C::kOpStage;
+            mbar_arrive_expect_tx(bars.op_full(so), C::kDirectBytes);
+            if (!ADEC) tma_load_2d(ob, &tmXA, kb * BK, m0, bars.op_full(so));
+            if (!BDEC) tma_load_2d(ob + kOpA, &tmWB, kbw * BK, n0, bars.op_full(so));
             if (++so == C::kOpStages) { so = 0; pho ^= 1u; }
           }
         }
@@ -365,7 +354,8 @@ __global__ void __launch_bounds__(MCfg<WDEC>::kThreads, 1)
         if ((kb & 1) == 0 &&
             !mbar_wait_bounded(bars.meta_full(ms), mph, abort_flag, kErrWaitUnpack))
           break;
-        if (!mbar_wait_bounded(bars.pk_full(s), ph, abort_flag, kErrWaitUnpack)) break;
+        if (C::kAnyDec && !mbar_wait_bounded(bars.pk_full(s), ph, abort_flag, kErrWaitUnpack))
+          break;
         if (!mbar_wait_bounded(bars.op_empty(so), pho ^ 1u, abort_flag, kErrWaitUnpack)) break;
         const uint8_t* pk = sp + C::kOffPk + s * C::kPkStage;
         const uint8_t* mt = sp + C::kOffMeta + ms * C::kMetaSlot;
@@ -379,7 +369,7 @@ __global__ void __launch_bounds__(MCfg<WDEC>::kThreads, 1)
           const int r = task >> 1, h = task & 1;
           const bool is_b = r >= BM;
           const int rr = is_b ? r - BM : r;
-          const uint8_t* crow = pk + (is_b ? kPkA : 0) + rr * (BK / 2) + 32 * h;
+          const uint8_t* crow = pk + (is_b && ADEC ? kPkA : 0) + rr * (BK / 2) + 32 * h;
           const uint32_t words = *reinterpret_cast<const uint32_t*>(
               mt + (is_b ? kMetaA : 0) + rr * 16 + ((kb & 1) * 4 + 2 * h) * 2);
           uint8_t* orow_p = op + (is_b ? kOpA : 0) + rr * 128;
@@ -406,28 +396,32 @@ __global__ void __launch_bounds__(MCfg<WDEC>::kThreads, 1)
           *reinterpret_cast<uint16_t*>(sf + (is_b ? kSfA : 0) + sf_row_offset(rr) + 2 * h) =
               static_cast<uint16_t>(e0 | (e1 << 8));
         }
-        if (WDEC) {  // the decoded weights' scales: one 4-byte word per row
-          for (int n = dt; n < BN; n += C::kDecThreads) {
-            const uint32_t w01 = *reinterpret_cast<const uint32_t*>(mt + kMetaA + n * 16 + (kb & 1) * 8);
-            const uint32_t w23 = *reinterpret_cast<const uint32_t*>(mt + kMetaA + n * 16 + (kb & 1) * 8 + 4);
-            uint32_t v = 0;
-            const uint32_t wv[2] = {w01, w23};
+        // the scales of the operands loaded as e4m3: one 4-byte word per row
+        // (x rows 0..127, then W rows)
+        constexpr int kDirectRows = (ADEC ? 0 : BM) + (BDEC ? 0 : BN);
+        for (int i = dt; i < kDirectRows; i += C::kDecThreads) {
+          const bool is_b = ADEC || i >= BM;
+          const int rr = ADEC ? i : (i >= BM ? i - BM : i);
+          const uint8_t* wp = mt + (is_b ? kMetaA : 0) + rr * 16 + (kb & 1) * 8;
+          const uint32_t wv[2] = {*reinterpret_cast<const uint32_t*>(wp),
+                                  *reinterpret_cast<const uint32_t*>(wp + 4)};
+          uint32_t v = 0;
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              v |= static_cast<uint32_t>(
-                       static_cast<int>(static_cast<int8_t>((wv[k >> 1] >> (16 * (k & 1))) & 0xFFu)) + 127)
-                   << (8 * k);
-            *reinterpret_cast<uint32_t*>(sf + kSfA + sf_row_offset(n)) = v;
-          }
+          for (int k = 0; k < 4; ++k)
+            v |= static_cast<uint32_t>(
+                     static_cast<int>(static_cast<int8_t>((wv[k >> 1] >> (16 * (k & 1))) & 0xFFu)) +
+                     127)
+                 << (8 * k);
+          *reinterpret_cast<uint32_t*>(sf + (is_b ? kSfA : 0) + sf_row_offset(rr)) = v;
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(bars.op_full(so));
-          mbar_arrive(bars.pk_empty(s));
+          if (C::kAnyDec) mbar_arrive(bars.pk_empty(s));
           if ((kb & 1) == 1) mbar_arrive(bars.meta_empty(ms));
         }
-        if (++s == C::kPkStages) { s = 0; ph ^= 1u; }
+        if (C::kAnyDec && ++s == C::kPkStages) { s = 0; ph ^= 1u; }
         if (++so == C::kOpStages) { so = 0; pho ^= 1u; }
         if ((kb & 1) == 1 && ++ms == C::kMetaSlots) { ms = 0; mph ^= 1u; }
       }

@@ -303,6 +303,17 @@ QS_API qs_status qs_sd4_quant(const void* x_bf16, int64_t rows, int64_t K, void*
                               uint16_t* meta, void* stream);
 
 /*
+ * qs_sd4_quant_e4m3 — qs_sd4_quant with each element written as the e4m3
+ * byte of its decoded magnitude and sign (the same values: (-1)^s L/8; the
+ * block words, identical to qs_sd4_quant's, keep the block scales).  One byte
+ * per element instead of half: the activation form that
+ * qs_sd4_linear_e4m3 loads by TMA straight into its operand tiles.
+ *   out_e4m3  [rows, K] bytes, written;  meta [rows, K/32] uint16, written
+ */
+QS_API qs_status qs_sd4_quant_e4m3(const void* x_bf16, int64_t rows, int64_t K, void* out_e4m3,
+                                   uint16_t* meta, void* stream);
+
+/*
  * qs_sd4_linear — the SD4 layer: out[m][n] = bf16(fl(sum_k x_hat w_hat) + bias[n])
  * with x_hat, w_hat the decoded SD4 values of qs_sd4_quant(x) and
  * qs_sd4_quant(W).  Each decoded value is an e4m3 number (L/8, signed) times
@@ -356,6 +367,18 @@ QS_API qs_status qs_sd4_linear_e4m3w(const void* x_codes, const uint16_t* x_meta
                                      const void* w_e4m3, const uint16_t* w_meta,
                                      const void* bias_bf16, int64_t M, int64_t N, int64_t K,
                                      void* out_bf16, void* stream);
+
+/*
+ * qs_sd4_linear_e4m3 — qs_sd4_linear with both operands as e4m3 bytes and
+ * block words (x from qs_sd4_quant_e4m3, W from qs_sd4_decode_e4m3 or
+ * qs_sd4_quant_e4m3): nothing is decoded in the GEMM.  The same arithmetic
+ * as qs_sd4_linear.
+ *   x_e4m3 [M, K], x_meta [M, K/32], w_e4m3 [N, K], w_meta [N, K/32]
+ */
+QS_API qs_status qs_sd4_linear_e4m3(const void* x_e4m3, const uint16_t* x_meta,
+                                    const void* w_e4m3, const uint16_t* w_meta,
+                                    const void* bias_bf16, int64_t M, int64_t N, int64_t K,
+                                    void* out_bf16, void* stream);
 
 /*
  * Activation decomposition (SemanticDialect "Resumen técnico" §2.B): a salient

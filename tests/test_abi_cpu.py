@@ -272,3 +272,9 @@ def test_sd4_validation(lib):
     assert e(A, B, C, D, NUL, 8, 200, 256, D, NUL) == SHAPE
     assert e(A, B, C, D, NUL, 8, 256, 256 + 128, D, NUL) == SHAPE
     assert e(A, B, C, D, MIS, 8, 256, 256, D, NUL) == ALIGN
+    assert lib.qs_sd4_quant_e4m3(A, 8, 384, B, C, NUL) == SHAPE
+    assert lib.qs_sd4_quant_e4m3(A, 8, 256, NUL, C, NUL) == NULL
+    f8 = lib.qs_sd4_linear_e4m3
+    assert f8(A, B, C, NUL, NUL, 8, 256, 256, D, NUL) == NULL
+    assert f8(A, B, C, D, NUL, 8, 248, 256, D, NUL) == SHAPE
+    assert f8(MIS, B, C, D, NUL, 8, 256, 256, D, NUL) == ALIGN

@@ -151,6 +151,39 @@ def test_sd4_linear_e4m3_weights_identical_and_bf16_weights_within_bound(M, N, K
     _check_layer(d, dev, out16, K)
 
 
+def _e4m3_of_codes(c, dd):
+    L = S.formatbook()
+    mag = L[np.repeat(dd, 32, axis=1), c & 7] / 8.0          # L/8, exact in e4m3
+    val = np.where(c & 8, -mag, mag)
+    return torch.from_numpy(val).to(torch.float8_e4m3fn).view(torch.uint8), val
+
+
+@pytest.mark.parametrize("M,K", [(7, 256), (33, 5120), (5, 13824)])
+def test_sd4_quant_e4m3_bit_exact(M, K):
+    d = I.make_shape(seed=M + 3 * K, M=M, K=K, N=16, bits=4, outlier_factor=30.0)
+    x8, meta = qs.sd4_quant_e4m3(d["x"].cuda())
+    torch.cuda.synchronize()
+    c, e, dd = S.quantize_rows(I.bf16_bits(d["x"]))
+    assert np.array_equal(meta.cpu().numpy().view(np.uint16), S.pack_meta(e, dd))
+    want, _ = _e4m3_of_codes(c, dd)
+    assert torch.equal(x8.cpu(), want)
+
+
+@pytest.mark.parametrize("M,N,K", [(127, 272, 256), (300, 768, 768), (513, 528, 1280),
+                                   (1, 16, 256)])
+def test_sd4_linear_e4m3_operands_identical(M, N, K):
+    d, dev, out = _layer(M, N, K, seed=5 * M + N)
+    cx, mx, cw, mw = dev
+    x8, mx8 = qs.sd4_quant_e4m3(d["x"].cuda())
+    w8 = qs.sd4_decode_e4m3(cw, mw)
+    out8 = torch.empty_like(out)
+    qs.qs_sd4_linear_e4m3(x8, mx8, w8, mw, d["bias"].cuda(), M, N, K, out8)
+    torch.cuda.synchronize()
+    assert torch.equal(mx8, mx)
+    assert torch.equal(out.view(torch.int16), out8.view(torch.int16))
+    _check_layer(d, dev, out8, K)
+
+
 @pytest.mark.parametrize("R,K", [(5, 256), (129, 5120)])
 def test_sd4_decode_e4m3_exact(R, K):
     d = I.make_shape(seed=R + 2 * K, M=R, K=K, N=16, bits=4, outlier_factor=30.0)
