@@ -21,6 +21,8 @@
 // bins go to shared memory; then for each block lane d sums dialect d's cost
 // (conflict-free: the table is laid out [bin][dialect]) and a warp minimum on
 // (cost << 5 | d) picks the dialect; finally each lane writes its 8 codes.
+// (Scoring runs two blocks at a time on packed 16-bit Qerror pairs: see
+// Tables.)
 #pragma once
 
 #include <cuda_bf16.h>
@@ -61,10 +63,14 @@ __host__ __device__ inline int level(int d, int i) {
   return i == 0 ? 0 : prev;
 }
 
+// Qerror is at most 16129 (< 2^14), so two dialects share a word and four
+// entries sum without carrying across the halves.  qerr2[b][w] holds
+// Qerror[2w][b] | Qerror[2w + 1][b] << 16 for w < 16 and again at w + 16, so
+// the two half-warps, scoring different blocks, read disjoint banks.
 struct Tables {
-  uint32_t qerr[kBins][kDialects];  // [bin][dialect]: lane d reads word d
+  uint32_t qerr2[kBins][32];
   uint8_t qval[kDialects][kBins];
-  int lvl[kDialects][8];            // the formatbook L[d][i]
+  int lvl[kDialects][8];  // the formatbook L[d][i]
 };
 
 // Fills the tables; ends with a __syncthreads.
@@ -84,7 +90,9 @@ __device__ void build_tables(Tables* tb) {
         bi = i;
       }
     }
-    tb->qerr[b][d] = best;
+    uint16_t* row = reinterpret_cast<uint16_t*>(tb->qerr2[b]);
+    row[d] = static_cast<uint16_t>(best);       // word d / 2, half d % 2
+    row[32 + d] = static_cast<uint16_t>(best);  // the copy for the upper half-warp
     tb->qval[d][b] = static_cast<uint8_t>(bi);
   }
   __syncthreads();
@@ -160,21 +168,34 @@ __device__ __forceinline__ uint32_t quant_warp_chunk(const float (&a)[8], const 
       make_uint2(bins[0] | (bins[1] << 8) | (bins[2] << 16) | (static_cast<uint32_t>(bins[3]) << 24),
                  bins[4] | (bins[5] << 8) | (bins[6] << 16) | (static_cast<uint32_t>(bins[7]) << 24));
   __syncwarp();
-  // dialect choice: lane = dialect; the block's 32 bins come as two
-  // broadcast 16-byte reads, then 32 independent table reads
+  // dialect choice, two blocks at a time: half-warp h scores block 2jj + h,
+  // lane w of it dialects 2w and 2w + 1 (one packed table read per bin);
+  // the block's 32 bins come as two broadcast 16-byte reads
   int my_d = 0;
+  const int half = lane >> 4, w = lane & 15;
 #pragma unroll 2
-  for (int j = 0; j < 8; ++j) {
+  for (int jj = 0; jj < 4; ++jj) {
+    const int j = 2 * jj + half;
     const uint4 q0 = *reinterpret_cast<const uint4*>(&bins_sm[j][0]);
     const uint4 q1 = *reinterpret_cast<const uint4*>(&bins_sm[j][16]);
     const uint32_t bw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-    uint32_t cost = 0;
+    uint32_t lo = 0, hi = 0;
 #pragma unroll
-    for (int k = 0; k < kBlock; ++k) cost += tb.qerr[(bw[k >> 2] >> (8 * (k & 3))) & 0xFFu][lane];
-    uint32_t key = (cost << 5) | static_cast<uint32_t>(lane);
+    for (int k4 = 0; k4 < 8; ++k4) {
+      uint32_t p = 0;  // four entries, both halves below 2^16
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) key = min(key, __shfl_xor_sync(0xffffffffu, key, off));
-    if (j == blk) my_d = static_cast<int>(key & 31u);
+      for (int k = 0; k < 4; ++k) p += tb.qerr2[(bw[k4] >> (8 * k)) & 0xFFu][lane];
+      lo += p & 0xFFFFu;
+      hi += p >> 16;
+    }
+    uint32_t key = min((lo << 5) | static_cast<uint32_t>(2 * w),
+                       (hi << 5) | static_cast<uint32_t>(2 * w + 1));
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) key = min(key, __shfl_xor_sync(0xffffffffu, key, off));
+    const uint32_t k_even = __shfl_sync(0xffffffffu, key, 0);
+    const uint32_t k_odd = __shfl_sync(0xffffffffu, key, 16);
+    if (blk == 2 * jj) my_d = static_cast<int>(k_even & 31u);
+    if (blk == 2 * jj + 1) my_d = static_cast<int>(k_odd & 31u);
   }
   uint32_t packed = 0;
 #pragma unroll
