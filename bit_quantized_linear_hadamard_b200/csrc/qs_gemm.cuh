@@ -329,14 +329,24 @@ __device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
                : "memory");
 }
 
+// 32-byte streaming store (one whole sector per lane); p 32-byte aligned.
+__device__ __forceinline__ void st_stream_v8(void* p, const uint32_t (&v)[8]) {
+  asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
 // Converts one 32-column chunk of accumulators (one row per thread) and stores it.
 // ASYM (weights on an asymmetric grid, signed codes s = q - 2^(b-1)): the
 // exact accumulator is sum q_a s + o[n] * sum_k q_a[m,k].
+// wide: `out` is 32-byte aligned, so 16 bf16 outputs go out as one 32-byte
+// store (rows are 2N bytes apart with N % 16 == 0, chunks start at multiples
+// of 32 columns); otherwise as two 16-byte stores.
 template <int SHIFT, bool OUT_S32, bool ASYM>
 __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row, bool row_ok,
                                                int n, int N, float s_a, const float* epi_sw,
                                                const float* epi_b, const int* epi_off,
-                                               int rsum, void* out) {
+                                               int rsum, void* out, bool wide) {
   if (n >= N || !row_ok) return;
   int32_t acc[32];
 #pragma unroll
@@ -354,28 +364,34 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row,
   } else {
     uint16_t* dst = static_cast<uint16_t*>(out) + static_cast<int64_t>(row) * N + n;
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      if (n + 8 * v + 8 > N) break;  // N % 16 == 0: only whole 8-column groups exist
-      const float4 w0 = *reinterpret_cast<const float4*>(epi_sw + 8 * v);
-      const float4 w1 = *reinterpret_cast<const float4*>(epi_sw + 8 * v + 4);
-      const float4 b0 = *reinterpret_cast<const float4*>(epi_b + 8 * v);
-      const float4 b1 = *reinterpret_cast<const float4*>(epi_b + 8 * v + 4);
-      const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-      uint32_t packed[4];
+    for (int v = 0; v < 2; ++v) {
+      if (n + 16 * v + 16 > N) break;  // N % 16 == 0: only whole 16-column groups exist
+      uint32_t packed[8];
 #pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        float y[2];
+      for (int q = 0; q < 4; ++q) {
+        const float4 w4 = *reinterpret_cast<const float4*>(epi_sw + 16 * v + 4 * q);
+        const float4 b4 = *reinterpret_cast<const float4*>(epi_b + 16 * v + 4 * q);
+        const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+        const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float sab = __fmul_rn(s_a, wv[e + h]);
-          const float p = __fmul_rn(sab, __int2float_rn(acc[8 * v + e + h]));
-          y[h] = __fadd_rn(p, bv[e + h]);
+        for (int e = 0; e < 4; e += 2) {
+          float y[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const float sab = __fmul_rn(s_a, wv[e + h]);
+            const float p = __fmul_rn(sab, __int2float_rn(acc[16 * v + 4 * q + e + h]));
+            y[h] = __fadd_rn(p, bv[e + h]);
+          }
+          const __nv_bfloat162 y2 = __floats2bfloat162_rn(y[0], y[1]);
+          packed[2 * q + (e >> 1)] = *reinterpret_cast<const uint32_t*>(&y2);
         }
-        const __nv_bfloat162 y2 = __floats2bfloat162_rn(y[0], y[1]);
-        packed[e >> 1] = *reinterpret_cast<const uint32_t*>(&y2);
       }
-      st_stream_v4(dst + 8 * v, make_uint4(packed[0], packed[1], packed[2], packed[3]));
+      if (wide) {
+        st_stream_v8(dst + 16 * v, packed);
+      } else {
+        st_stream_v4(dst + 16 * v, make_uint4(packed[0], packed[1], packed[2], packed[3]));
+        st_stream_v4(dst + 16 * v + 8, make_uint4(packed[4], packed[5], packed[6], packed[7]));
+      }
     }
   }
 }
@@ -420,6 +436,7 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
                            static_cast<uint32_t>(buf * BN);
     // Two register sets: the TMEM load of chunk c+1 is in flight while chunk c
     // is converted and stored.
+    const bool wide = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
     uint32_t ra[32], rb[32];
     tmem_ld_32x32b_x32(taddr, ra);
     tmem_wait_ld();
@@ -428,12 +445,12 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
       tmem_ld_32x32b_x32(taddr + 32 * (c + 1), rb);
       epilogue_chunk<SHIFT, OUT_S32, ASYM>(ra, row, row_ok, n0 + 32 * c, pb.N, s_a,
                                           epi_sw + 32 * c, epi_b + 32 * c, epi_off + 32 * c,
-                                          rsum, out);
+                                          rsum, out, wide);
       tmem_wait_ld();
       if (c + 2 < BN / 32) tmem_ld_32x32b_x32(taddr + 32 * (c + 2), ra);
       epilogue_chunk<SHIFT, OUT_S32, ASYM>(rb, row, row_ok, n0 + 32 * (c + 1), pb.N, s_a,
                                           epi_sw + 32 * (c + 1), epi_b + 32 * (c + 1),
-                                          epi_off + 32 * (c + 1), rsum, out);
+                                          epi_off + 32 * (c + 1), rsum, out, wide);
       tmem_wait_ld();
     }
     tc_fence_before();

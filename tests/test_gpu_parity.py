@@ -431,3 +431,26 @@ def test_w4a4_with_byte_activation_codes(M, N, K):
     got = out.view(torch.int16).cpu().numpy().view(np.uint16)
     assert np.array_equal(got, r["out"])
     assert np.array_equal(one.view(torch.int16).cpu().numpy().view(np.uint16), r["out"])
+
+
+@pytest.mark.parametrize("bx,bw", [(4, 4), (8, 4), (8, 8)])
+def test_qlinear_output_only_16_byte_aligned(bx, bw):
+    """An output only 16-byte aligned (the ABI's requirement) takes the 16-byte
+    store path; a 32-byte aligned one the 32-byte path: the same values."""
+    M, N, K = 300, 272, 512
+    d = I.make_shape(seed=13 + bx, M=M, K=K, N=N, bits=4, bits_x=bx if bx != bw else 0)
+    x, w, b = d["x"].cuda(), d["w"].cuda(), d["bias"].cuda()
+    wp, ws = qs.pack_weights(w, bw)
+    xp, xs = qs.quant_act(x, bx, 1.0)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    buf = torch.empty(M * N + 8, dtype=torch.bfloat16, device="cuda")
+    out16 = buf[8:].view(M, N)
+    assert out.data_ptr() % 32 == 0 and out16.data_ptr() % 32 == 16
+    for o in (out, out16):
+        qs.qs_qlinear_mixed(xp, xs, bx, wp, ws, bw, b, M, N, K, o)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), out16.view(torch.int16))
+    q, s = O.quant_act(I.bf16_bits(d["x"]), bx, 1.0)
+    qw, sw = O.pack_weights(I.bf16_bits(d["w"]), bw)
+    want = O.epilogue(O.int_gemm(q, qw), s, sw, I.bf16_bits(d["bias"]))
+    assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), want)

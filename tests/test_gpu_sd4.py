@@ -386,3 +386,58 @@ def test_full_size_wan_ffn_decomp_sampled():
     _check_decomp_layer(sub, got, list(range(len(srows))), K)
     assert np.array_equal(codes2[torch.from_numpy(pick_s).cuda()].cpu().numpy(),
                           S.pack_decomp(S.decompose_rows(xb[:len(srows)], range(len(srows))))[0])
+
+
+@pytest.mark.slow
+def test_full_size_wan_ffn_e4m3_layer_sampled():
+    """The SD4 layer the benchmark times (Wan FFN, 32760 x 5120 -> 13824): e4m3
+    activations and weights; bit-identical to the codes form everywhere, and
+    sampled outputs against the oracle."""
+    cfg = I.WAN_FFN
+    d = I.make_layer(cfg)
+    M, K, N = cfg.M, cfg.K, cfg.N
+    x, w, b = d["x"].cuda(), d["w"].cuda(), d["bias"].cuda()
+    cx, mx = qs.sd4_quant(x)
+    cw, mw = qs.sd4_quant(w)
+    x8, mx8 = qs.sd4_quant_e4m3(x)
+    w8 = qs.sd4_decode_e4m3(cw, mw)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    out8 = torch.empty_like(out)
+    qs.qs_sd4_linear(cx, mx, cw, mw, b, M, N, K, out)
+    qs.qs_sd4_linear_e4m3(x8, mx8, w8, mw, b, M, N, K, out8)
+    torch.cuda.synchronize()
+    assert torch.equal(mx8, mx)
+    assert torch.equal(out.view(torch.int16), out8.view(torch.int16))
+    rng = np.random.default_rng(6)
+    rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, 40, replace=False)]))
+    cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 40, replace=False)]))
+    sub = {"x": d["x"][rows], "w": d["w"][cols], "bias": d["bias"][cols]}
+    got = out8[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()]
+    r = S.linear_sd4(I.bf16_bits(sub["x"]), I.bf16_bits(sub["w"]), I.bf16_bits(sub["bias"]),
+                     exact=False)
+    got_bits = got.view(torch.int16).cpu().numpy().view(np.uint16)
+    gotf = O.bf16_bits_to_f32(got_bits).astype(np.float64)
+    S_abs = np.abs(r["x_hat"]) @ np.abs(r["w_hat"]).T
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(gotf), 2.0 ** -126))) - 7)
+    exact_y = r["y"] + O.bf16_bits_to_f32(I.bf16_bits(sub["bias"])).astype(np.float64)
+    assert (np.abs(gotf - exact_y) <= K * 2.0 ** -23 * S_abs + ulp).all()
+    assert float((got_bits == r["out"]).mean()) > 0.99
+
+
+def test_sd4_output_only_16_byte_aligned():
+    """16-byte (not 32-byte) aligned outputs take the 16-byte store path."""
+    M, N, K = 200, 400, 512
+    d, dev, out = _layer(M, N, K, seed=41)
+    cx, mx, cw, mw = dev
+    x8, mx8 = qs.sd4_quant_e4m3(d["x"].cuda())
+    w8 = qs.sd4_decode_e4m3(cw, mw)
+    for fn in ("codes", "e4m3"):
+        buf = torch.empty(M * N + 8, dtype=torch.bfloat16, device="cuda")
+        o = buf[8:].view(M, N)
+        assert o.data_ptr() % 32 == 16
+        if fn == "codes":
+            qs.qs_sd4_linear(cx, mx, cw, mw, d["bias"].cuda(), M, N, K, o)
+        else:
+            qs.qs_sd4_linear_e4m3(x8, mx8, w8, mw, d["bias"].cuda(), M, N, K, o)
+        torch.cuda.synchronize()
+        assert torch.equal(o.view(torch.int16), out.view(torch.int16)), fn
