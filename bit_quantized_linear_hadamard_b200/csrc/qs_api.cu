@@ -150,37 +150,6 @@ qs_status launch_sd4_mx(const CUtensorMap& ca, const CUtensorMap& cb, const CUte
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
-// e4m3 x e4m3 on pairs of CTAs (no output row map, Ka = K).
-qs_status launch_sd4_mx_pair(const void* x_e4m3, const uint16_t* x_meta, const void* w_e4m3,
-                             const uint16_t* w_meta, const void* bias, int64_t M, int64_t N,
-                             int64_t K, void* out, void* stream) {
-  namespace G = qs::sd4::gemm_mx;
-  namespace P = qs::sd4::gemm_mx::pair;
-  CUtensorMap xa, wb, ma, mb;
-  if (!qs::make_tensor_map_2d(&xa, x_e4m3, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
-                              G::BK, P::HA, true) ||
-      !qs::make_tensor_map_2d(&wb, w_e4m3, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
-                              G::BK, P::HB, true) ||
-      !qs::make_tensor_map_2d(&ma, x_meta, static_cast<uint64_t>(K) / 16,
-                              static_cast<uint64_t>(M), 16, P::HA, false) ||
-      !qs::make_tensor_map_2d(&mb, w_meta, static_cast<uint64_t>(K) / 16,
-                              static_cast<uint64_t>(N), 16, P::PN, false))
-    return QS_ERR_CUDA;
-  auto kern = P::sd4_mx2_gemm_kernel;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::kSmemBytes) !=
-      cudaSuccess)
-    return QS_ERR_CUDA;
-  const int sms = qs::sm_count();
-  if (sms <= 1) return QS_ERR_CUDA;
-  const int64_t tiles = ((M + P::PM - 1) / P::PM) * ((N + P::PN - 1) / P::PN);
-  const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
-  kern<<<static_cast<int>(2 * pairs), P::kThreads, P::kSmemBytes,
-         static_cast<cudaStream_t>(stream)>>>(xa, wb, ma, mb, static_cast<const uint16_t*>(bias),
-                                              static_cast<uint16_t*>(out), static_cast<int>(M),
-                                              static_cast<int>(N), static_cast<int>(K));
-  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
-}
-
 // The block-scaled SD4 GEMM: A = `a_rows` rows of Ka elements (Ka = K, or 2K
 // for decomposed rows) as codes or, when a_e4m3 is not NULL, as e4m3 bytes;
 // the weights as codes or, when w_e4m3 is not NULL, as e4m3 bytes; block
@@ -207,8 +176,6 @@ qs_status run_sd4_mx(const void* a_codes, const void* a_e4m3, const uint16_t* a_
                                        static_cast<uint64_t>(N), G::BK / 2, G::BN, false))
     return QS_ERR_CUDA;
   const int64_t kb_wrap = K / G::BK;
-  if (a_e4m3 && w_e4m3 && !out_rows && Ka == K)
-    return launch_sd4_mx_pair(a_e4m3, a_meta, w_e4m3, w_meta, bias, a_rows, N, K, out, stream);
   if (a_e4m3) {
     if (!w_e4m3) return QS_ERR_NULL;  // e4m3 activations go with e4m3 weights
     return launch_sd4_mx<false, false>(xa, xa, ma, mb, xa, wb, bias, a_rows, N, Ka, out, stream,

@@ -486,352 +486,6 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
   }
 }
 
-// --------------------------------------------------------------------------
-// e4m3 x e4m3 on pairs of CTAs (cta_group::2): the pair computes a 256 x 192
-// tile, each CTA holding its own 128 activation rows and half (96 rows) of
-// the weight tile, so an SM moves 28 KB per stage instead of 40 KB.  The
-// leader's MMA thread copies both CTAs' scale blocks into their tensor
-// memories (tcgen05.cp.cta_group::2: each CTA's shared memory into its own
-// TMEM) and issues M = 256 block-scaled MMAs.  A CTA's A scales cover its own
-// 128 rows, its B scales the whole 192 (both halves of the MMA use all N).
-// The other CTA's scale writes reach the leader's "full" barrier through a
-// 16-byte bulk-copy signal, as in the integer GEMM.
-namespace pair {
-
-constexpr int PM = 256, PN = 192;  // pair tile
-constexpr int HA = 128, HB = 96;   // rows of x and of W per CTA
-constexpr int kOpA = HA * BK, kOpB = HB * BK, kOpStage = kOpA + kOpB;
-constexpr int kSfStage = kSfA + kSfB;
-constexpr int kMetaSlot = kMetaA + kMetaB;  // own 128 x rows, all 192 W rows
-constexpr int kOpStages = 6, kMetaSlots = 2;
-constexpr int kSfWarps = 4;
-constexpr int kThreads = 32 * (2 + kEpiWarps + kSfWarps);
-constexpr int kOffOp = 0;
-constexpr int kOffSf = kOffOp + kOpStages * kOpStage;
-constexpr int kOffMeta = kOffSf + kOpStages * kSfStage;
-constexpr int kOffBar = kOffMeta + kMetaSlots * kMetaSlot;
-constexpr int kNumBars = 3 * kOpStages + 2 * kMetaSlots + 4;
-constexpr int kOffEpi = (kOffBar + 8 * kNumBars + 15) / 16 * 16;
-constexpr int kOffSignal = kOffEpi + PN * 4;  // 16 bytes per operand stage
-constexpr int kOffMisc = kOffSignal + 16 * kOpStages;
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;
-// the leader's "full": both CTAs' TMA bytes and the other CTA's 16-byte signal
-constexpr int kOpFullTx = 2 * kOpStage + 16;
-constexpr int kGroupN = 36;
-static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
-static_assert(kOpStage % 1024 == 0 && kOffSf % 1024 == 0 && kOffMeta % 128 == 0, "alignment");
-
-struct PBars {
-  uint32_t base;
-  __device__ uint32_t at(int i) const { return base + 8u * i; }
-  __device__ uint32_t op_full(int s) const { return at(s); }
-  __device__ uint32_t op_empty(int s) const { return at(kOpStages + s); }
-  __device__ uint32_t sf_ready(int s) const { return at(2 * kOpStages + s); }
-  __device__ uint32_t meta_full(int s) const { return at(3 * kOpStages + s); }
-  __device__ uint32_t meta_empty(int s) const { return at(3 * kOpStages + kMetaSlots + s); }
-  __device__ uint32_t acc_full(int b) const { return at(3 * kOpStages + 2 * kMetaSlots + b); }
-  __device__ uint32_t acc_empty(int b) const {
-    return at(3 * kOpStages + 2 * kMetaSlots + 2 + b);
-  }
-};
-
-__device__ __forceinline__ void mma_mx_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t sfa, uint32_t sfb,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::
-          "r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
-      : "memory");
-}
-
-// Both CTAs: 32 rows of 16 bytes of their own shared memory into their own
-// tensor memory, replicated to the 4 lane quarters.
-__device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
-}
-
-__device__ __forceinline__ void tile_origin(int t, int m_tiles, int n_tiles, int& m0, int& n0) {
-  const int per_group = kGroupN * m_tiles;
-  const int g = t / per_group, r = t - g * per_group;
-  const int gn = min(kGroupN, n_tiles - g * kGroupN);
-  m0 = (r / gn) * PM;
-  n0 = (g * kGroupN + r % gn) * PN;
-}
-
-// UE8M0 scale bytes of four consecutive blocks from their block words.
-__device__ __forceinline__ uint32_t scales4(const uint8_t* words) {
-  const uint32_t w01 = *reinterpret_cast<const uint32_t*>(words);
-  const uint32_t w23 = *reinterpret_cast<const uint32_t*>(words + 4);
-  const uint32_t wv[2] = {w01, w23};
-  uint32_t v = 0;
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-    v |= static_cast<uint32_t>(
-             static_cast<int>(static_cast<int8_t>((wv[k >> 1] >> (16 * (k & 1))) & 0xFFu)) + 127)
-         << (8 * k);
-  return v;
-}
-
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    sd4_mx2_gemm_kernel(const __grid_constant__ CUtensorMap tmXA,
-                        const __grid_constant__ CUtensorMap tmWB,
-                        const __grid_constant__ CUtensorMap tmMA,
-                        const __grid_constant__ CUtensorMap tmMB,
-                        const uint16_t* __restrict__ bias, uint16_t* __restrict__ out, int M,
-                        int N, int K) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // the padding is the same in both CTAs: every shared object has the same
-  // offset in the two CTAs of a pair
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
-  uint8_t* sp = smem_raw + pad;
-  const uint32_t sbase = raw + pad;
-  const PBars bars{sbase + kOffBar};
-  float* epi_b = reinterpret_cast<float*>(sp + kOffEpi);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sp + kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + kOffMisc + 4);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const int pair_id = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
-  const int n_tiles = (N + PN - 1) / PN;
-  const int m_tiles = (M + PM - 1) / PM;
-  const int num_tiles = m_tiles * n_tiles;
-  const int kblocks = K / BK;
-
-  // B's scale blocks hold rows 192..255 that no MMA reads but tcgen05.cp copies
-  for (int i = threadIdx.x; i < kOpStages * kSfStage / 16; i += blockDim.x)
-    reinterpret_cast<uint4*>(sp + kOffSf)[i] = make_uint4(0u, 0u, 0u, 0u);
-  fence_proxy_async_smem();
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kOpStages; ++s) {
-      mbar_init(bars.op_full(s), 1);
-      mbar_init(bars.op_empty(s), 1);
-      mbar_init(bars.sf_ready(s), kSfWarps);
-    }
-    for (int s = 0; s < kMetaSlots; ++s) {
-      mbar_init(bars.meta_full(s), 1);
-      mbar_init(bars.meta_empty(s), kSfWarps);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bars.acc_full(b), 1);
-      mbar_init(bars.acc_empty(b), 2 * kEpiWarps);
-    }
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0) {  // producer (both CTAs)
-      const uint32_t a_row = rank * HA, b_row = rank * HB;
-      int s = 0, ms = 0;
-      uint32_t ph = 0, mph = 0;
-      bool ok = true;
-      for (int t = pair_id; t < num_tiles && ok; t += num_pairs) {
-        int m0, n0;
-        tile_origin(t, m_tiles, n_tiles, m0, n0);
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if ((kb & 1) == 0) {
-            if (!mbar_wait_bounded(bars.meta_empty(ms), mph ^ 1u, abort_flag, kErrWaitProducer)) {
-              ok = false;
-              break;
-            }
-            const uint32_t dst = sbase + kOffMeta + ms * kMetaSlot;
-            mbar_arrive_expect_tx(bars.meta_full(ms), kMetaSlot);
-            tma_load_2d(dst, &tmMA, (kb / 2) * 16, m0 + static_cast<int>(a_row),
-                        bars.meta_full(ms));
-            tma_load_2d(dst + kMetaA, &tmMB, (kb / 2) * 16, n0, bars.meta_full(ms));
-            if (++ms == kMetaSlots) { ms = 0; mph ^= 1u; }
-          }
-          if (!mbar_wait_bounded(bars.op_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer)) {
-            ok = false;
-            break;
-          }
-          const uint32_t dst = sbase + kOffOp + s * kOpStage;
-          const uint32_t full_leader = map_to_rank(bars.op_full(s), 0);
-          if (rank == 0) mbar_arrive_expect_tx(bars.op_full(s), kOpFullTx);
-          tma_load_2d_pair(dst, &tmXA, kb * BK, m0 + static_cast<int>(a_row), full_leader);
-          tma_load_2d_pair(dst + kOpA, &tmWB, kb * BK, n0 + static_cast<int>(b_row), full_leader);
-          if (++s == kOpStages) { s = 0; ph ^= 1u; }
-        }
-      }
-      // drain: the leader's last releases of this CTA's stages have arrived
-      for (int i = 0; ok && i < kOpStages; ++i) {
-        if (!mbar_wait_bounded(bars.op_empty(s), ph ^ 1u, abort_flag, kErrWaitProducer)) break;
-        if (++s == kOpStages) { s = 0; ph ^= 1u; }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {  // MMA issuer
-      const uint32_t sfa = tmem_base + kSfaCol, sfb = tmem_base + kSfbCol;
-      int s = 0;
-      uint32_t ph = 0;
-      int it = 0;
-      bool ok = true;
-      for (int t = pair_id; t < num_tiles && ok; t += num_pairs, ++it) {
-        const int buf = it & 1;
-        const uint32_t aph = (it >> 1) & 1;
-        if (!mbar_wait_cluster_bounded(bars.acc_empty(buf), aph ^ 1u, abort_flag, kErrWaitMma))
-          break;
-        tc_fence_after();
-        const uint32_t d = tmem_base + static_cast<uint32_t>(buf * PN);
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_bounded(bars.sf_ready(s), ph, abort_flag, kErrWaitMma) ||
-              !mbar_wait_cluster_bounded(bars.op_full(s), ph, abort_flag, kErrWaitMma)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a0 = sbase + kOffOp + s * kOpStage;
-          const uint32_t b0 = a0 + kOpA;
-          const uint32_t f0 = sbase + kOffSf + s * kSfStage;
-          tmem_cp_32x128b_x4_pair(sfa, smem_desc_sf(f0));
-          tmem_cp_32x128b_x4_pair(sfb, smem_desc_sf(f0 + kSfA));
-          tmem_cp_32x128b_x4_pair(sfb + 4, smem_desc_sf(f0 + kSfA + 512));
-#pragma unroll
-          for (int j = 0; j < BK / 32; ++j)
-            mma_mx_pair(d, smem_desc_sw128(a0 + j * 32), smem_desc_sw128(b0 + j * 32),
-                        idesc_mx(PM, PN, static_cast<uint32_t>(j)),
-                        sfa + (static_cast<uint32_t>(j) << 30),
-                        sfb + (static_cast<uint32_t>(j) << 30), (kb | j) != 0);
-          mma_commit_pair(map_to_rank(bars.op_empty(s), 0));
-          mma_commit_pair(map_to_rank(bars.op_empty(s), 1));
-          if (++s == kOpStages) { s = 0; ph ^= 1u; }
-        }
-        if (!ok) break;
-        mma_commit_pair(map_to_rank(bars.acc_full(buf), 0));
-        mma_commit_pair(map_to_rank(bars.acc_full(buf), 1));
-      }
-    }
-    if (lane == 0 && rank != 0) {  // relay: this CTA's scales are written
-      int s = 0;
-      uint32_t ph = 0;
-      for (int t = pair_id; t < num_tiles; t += num_pairs) {
-        bool ok = true;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_bounded(bars.sf_ready(s), ph, abort_flag, kErrWaitUnpack)) {
-            ok = false;
-            break;
-          }
-          const uint32_t slot = sbase + kOffSignal + 16 * s;
-          bulk_signal(map_to_rank(slot, 0), slot, map_to_rank(bars.op_full(s), 0));
-          if (++s == kOpStages) { s = 0; ph ^= 1u; }
-        }
-        if (!ok) break;
-      }
-    }
-  } else if (warp < 2 + kEpiWarps) {  // epilogue: this CTA's 128 rows
-    const int quad = warp & 3;
-    const int et = threadIdx.x - 64;
-    int it = 0;
-    for (int t = pair_id; t < num_tiles; t += num_pairs, ++it) {
-      const int buf = it & 1;
-      const uint32_t aph = (it >> 1) & 1;
-      int m0, n0;
-      tile_origin(t, m_tiles, n_tiles, m0, n0);
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      for (int i = et; i < PN; i += 128) {
-        const int n = n0 + i;
-        epi_b[i] = (n < N && bias) ? __uint_as_float(static_cast<uint32_t>(bias[n]) << 16) : 0.f;
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (!mbar_wait_cluster_bounded(bars.acc_full(buf), aph, abort_flag, kErrWaitEpilogue)) break;
-      tc_fence_after();
-      const int row = m0 + static_cast<int>(rank) * HA + 32 * quad + lane;
-      const bool wide = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quad) << 16) +
-                             static_cast<uint32_t>(buf * PN);
-#pragma unroll 1
-      for (int c = 0; c < PN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(taddr + 32 * c, r);
-        tmem_wait_ld();
-        const int n = n0 + 32 * c;
-        if (row < M && n < N) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float y0 = __fadd_rn(__uint_as_float(r[2 * j]), epi_b[32 * c + 2 * j]);
-            const float y1 = __fadd_rn(__uint_as_float(r[2 * j + 1]), epi_b[32 * c + 2 * j + 1]);
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
-            pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
-          }
-          uint16_t* dst = out + static_cast<int64_t>(row) * N + n;
-          store_row16x2(dst, pk, N - n, wide);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (rank == 0)
-          mbar_arrive(bars.acc_empty(buf));
-        else
-          mbar_arrive_cluster(map_to_rank(bars.acc_empty(buf), 0));
-      }
-    }
-  } else {  // scale writers: own 128 x rows, all 192 W rows
-    const int dt = threadIdx.x - 32 * (2 + kEpiWarps);
-    int s = 0, ms = 0;
-    uint32_t ph = 0, mph = 0;
-    bool ok = true;
-    for (int t = pair_id; t < num_tiles && ok; t += num_pairs) {
-      for (int kb = 0; kb < kblocks; ++kb) {
-        if ((kb & 1) == 0 &&
-            !mbar_wait_bounded(bars.meta_full(ms), mph, abort_flag, kErrWaitUnpack)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait_bounded(bars.op_empty(s), ph ^ 1u, abort_flag, kErrWaitUnpack)) {
-          ok = false;
-          break;
-        }
-        const uint8_t* mt = sp + kOffMeta + ms * kMetaSlot;
-        uint8_t* sf = sp + kOffSf + s * kSfStage;
-        for (int i = dt; i < HA + PN; i += 32 * kSfWarps) {
-          const bool is_b = i >= HA;
-          const int rr = is_b ? i - HA : i;
-          const uint32_t v = scales4(mt + (is_b ? kMetaA : 0) + rr * 16 + (kb & 1) * 8);
-          *reinterpret_cast<uint32_t*>(sf + (is_b ? kSfA : 0) + sf_row_offset(rr)) = v;
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(bars.sf_ready(s));
-          if ((kb & 1) == 1) mbar_arrive(bars.meta_empty(ms));
-        }
-        if (++s == kOpStages) { s = 0; ph ^= 1u; }
-        if ((kb & 1) == 1 && ++ms == kMetaSlots) { ms = 0; mph ^= 1u; }
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();  // no CTA leaves while its partner may still signal it
-  if (*abort_flag) {
-    const unsigned long long t0 = global_timer_ns();
-    while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
-  }
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc_pair(tmem_base, kTmemCols);
-  }
-}
-
-}  // namespace pair
-
 // e4m3 bytes of an SD4 matrix (the magnitudes L/8 with their signs; the
 // block words keep the scales): one thread per 16 elements.
 __global__ void __launch_bounds__(256) sd4_decode_e4m3_kernel(const uint8_t* __restrict__ codes,
