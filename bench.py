@@ -117,16 +117,67 @@ def workload_config(I, name):
 
 
 class ClockSampler:
+    """SM clock, power and clock-event reasons of the GPU under test, read on a
+    host thread every millisecond through NVML (reads only; nvidia-smi if NVML
+    is not available).  Only the samples taken between mark_start() and
+    mark_end(), i.e. during the timed region, are reported."""
+
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.lines = []
+        self.nv = None
+        self.samples = []
+        self.t_on = self.t_off = None
+
+    def _handle(self, nv):
+        """The NVML handle of CUDA device `index` (by UUID: CUDA and NVML may
+        number the devices differently)."""
+        try:
+            import torch
+            u = str(getattr(torch.cuda.get_device_properties(self.index), "uuid", ""))
+        except Exception:  # noqa: BLE001 - no CUDA device: NVML's numbering
+            u = ""
+        for cand in ((u, "GPU-" + u) if u else ()):
+            try:
+                return nv.nvmlDeviceGetHandleByUUID(cand)
+            except Exception:  # noqa: BLE001 - try the next form
+                pass
+        return nv.nvmlDeviceGetHandleByIndex(self.index)
 
     def start(self):
+        try:
+            import threading
+            import pynvml as nv
+            nv.nvmlInit()
+            self.h = self._handle(nv)
+            self.nv = nv
+            reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.stop_flag = False
+
+            def loop():
+                while not self.stop_flag:
+                    try:
+                        self.samples.append((time.perf_counter(),
+                                             nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                             reasons(self.h),
+                                             nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0))
+                    except Exception:  # noqa: BLE001 - a failed read is skipped
+                        pass
+                    time.sleep(0.001)
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            return
+        except Exception:  # noqa: BLE001 - no NVML: nvidia-smi
+            self.nv = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
@@ -135,7 +186,30 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def mark_start(self):
+        self.t_on = time.perf_counter()
+
+    def mark_end(self):
+        self.t_off = time.perf_counter()
+
     def stop(self):
+        if self.nv is not None:
+            time.sleep(0.01)
+            self.stop_flag = True
+            self.thread.join(timeout=2)
+            nv = self.nv
+            mx = float(nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM))
+            inside = [r for r in self.samples
+                      if self.t_on is not None and self.t_on <= r[0] <= (self.t_off or r[0])]
+            rows = inside or self.samples
+            if not rows:
+                return None
+            reasons = sorted({name for r in rows for bit, name in self.REASONS.items()
+                              if r[2] & bit})
+            return {"sm_mhz": statistics.median(float(r[1]) for r in rows), "sm_max_mhz": mx,
+                    "reasons": reasons, "samples": len(rows),
+                    "power_w_max": max(r[3] for r in rows),
+                    "source": "nvml, 1 ms, " + ("timed region" if inside else "whole run")}
         if self.proc is None:
             return None
         time.sleep(0.25)
@@ -156,7 +230,8 @@ class ClockSampler:
         loaded = [v for v in sm if v > 0.5 * mx] or sm
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons,
                 "samples": len(sm), "power_w_max": max(float(r[3]) for r in rows
-                                                       if len(r) >= 9 and _isnum(r[3]))}
+                                                       if len(r) >= 9 and _isnum(r[3])),
+                "source": "nvidia-smi, 100 ms, whole run"}
 
 
 def _isnum(s):
@@ -639,6 +714,7 @@ def main():
     if sampler:
         sampler.start()
         time.sleep(0.3)
+        sampler.mark_start()
     for i in range(args.steps):
         ev[i][0].record(stream)
         qs.qs_quant_act(x, M, K, bx, alpha, x_flags, xp, xs, stream)
@@ -647,6 +723,8 @@ def main():
         ev[i][2].record(stream)
     stream.synchronize()
     torch.cuda.synchronize()
+    if sampler:
+        sampler.mark_end()
     clocks = sampler.stop() if sampler else None
     if world > 1:
         dist.barrier()

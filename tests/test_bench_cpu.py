@@ -31,3 +31,38 @@ def test_traffic_lookup_follows_the_kernel_sources():
     else:  # the kernels changed since the counters were taken: no stale number
         assert got is None
     assert bench.ncu_traffic("no such workload", "qgemm_kernel") is None
+
+
+def test_clock_sampler_reports_the_timed_region_from_nvml(monkeypatch):
+    """The clock record comes from NVML reads taken between the marks around
+    the timed region: samples before and after it (idle clocks, another
+    reason) are not reported; reason bits map to their names."""
+    import sys
+    import time
+    import types
+
+    import bench
+
+    state = {"clock": 900, "reasons": 0x1}
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=0, nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByUUID=lambda u: "h", nvmlDeviceGetHandleByIndex=lambda i: "h",
+        nvmlDeviceGetClockInfo=lambda h, c: state["clock"],
+        nvmlDeviceGetMaxClockInfo=lambda h, c: 1965,
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: state["reasons"],
+        nvmlDeviceGetPowerUsage=lambda h: 700000)
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    s = bench.ClockSampler(0)
+    s.start()
+    time.sleep(0.03)
+    state.update(clock=1965, reasons=0x4)
+    s.mark_start()
+    time.sleep(0.05)
+    s.mark_end()
+    time.sleep(0.01)
+    state.update(clock=600, reasons=0x8 | 0x40)
+    time.sleep(0.02)
+    r = s.stop()
+    assert r["source"].startswith("nvml") and "timed region" in r["source"]
+    assert r["sm_mhz"] == 1965 and r["sm_max_mhz"] == 1965 and r["power_w_max"] == 700.0
+    assert r["reasons"] == ["sw_power_cap"] and r["samples"] >= 5
