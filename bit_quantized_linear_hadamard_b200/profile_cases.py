@@ -1,0 +1,80 @@
+"""Small cases of the library's kernels, for profiler captures of one kernel.
+
+    python -m bit_quantized_linear_hadamard_b200.profile_cases CASE [--tokens M]
+
+Each case builds seeded synthetic inputs of the Wan-14B FFN up-projection
+shape (K = 5120, N = 13824) with M tokens on cuda:0, runs its kernel three
+times through the C ABI and checks the device error word.  The inputs are
+sized to exceed the 126 MB L2 at the default M while keeping a few hundred MB
+on the device.
+
+Cases:
+  sd4_gemm_e4m3   qs_sd4_linear_e4m3 (block-scaled fp8 GEMM, e4m3 x e4m3)
+  sd4_gemm_codes  qs_sd4_linear (block-scaled fp8 GEMM decoding SD4 codes)
+  sd4_quant_e4m3  qs_sd4_quant_e4m3 (SD4 activation quantiser, e4m3 bytes out)
+  gbs_update      qs_gbs_update (normalised L1 change of two layer outputs)
+"""
+
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import binding as qs
+
+K, N = 5120, 13824
+
+
+def _inputs(M: int):
+    g = torch.Generator(device="cuda").manual_seed(0)
+    x = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+    w = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+    b = (torch.randn(N, device="cuda", generator=g) * 0.01).to(torch.bfloat16)
+    return x, w, b
+
+
+def main(argv=None) -> None:
+    p = argparse.ArgumentParser()
+    p.add_argument("case", choices=["sd4_gemm_e4m3", "sd4_gemm_codes", "sd4_quant_e4m3",
+                                    "gbs_update"])
+    p.add_argument("--tokens", type=int, default=None)
+    a = p.parse_args(argv)
+    qs.load()
+    torch.cuda.init()
+    if a.case in ("sd4_gemm_e4m3", "sd4_gemm_codes"):
+        M = a.tokens or 4096
+        x, w, b = _inputs(M)
+        cw, mw = qs.sd4_quant(w)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        if a.case == "sd4_gemm_e4m3":
+            x8, mx = qs.sd4_quant_e4m3(x)
+            w8 = qs.sd4_decode_e4m3(cw, mw)
+            run = lambda: qs.qs_sd4_linear_e4m3(x8, mx, w8, mw, b, M, N, K, out)  # noqa: E731
+        else:
+            cx, mx = qs.sd4_quant(x)
+            run = lambda: qs.qs_sd4_linear(cx, mx, cw, mw, b, M, N, K, out)  # noqa: E731
+    elif a.case == "sd4_quant_e4m3":
+        M = a.tokens or 16384
+        x, _, _ = _inputs(M)
+        x8 = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+        mx = torch.empty((M, K // 32), dtype=torch.int16, device="cuda")
+        run = lambda: qs.qs_sd4_quant_e4m3(x, M, K, x8, mx)  # noqa: E731
+    else:
+        M = a.tokens or 8192
+        g = torch.Generator(device="cuda").manual_seed(1)
+        y0 = torch.randn(M, N, device="cuda", generator=g).to(torch.bfloat16)
+        y1 = (y0.float() + 0.05 * torch.randn(M, N, device="cuda", generator=g)).to(torch.bfloat16)
+        state = torch.zeros(qs.QS_GBS_STATE_BYTES, dtype=torch.uint8, device="cuda")
+        qs.qs_gbs_reset(state)
+        run = lambda: qs.qs_gbs_update(y1, y0, M * N, 0.3, state)  # noqa: E731
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    if qs.qs_device_error() != 0:
+        raise SystemExit("a kernel reported a device error")
+    print("ok")
+
+
+if __name__ == "__main__":
+    main()
