@@ -188,6 +188,26 @@ qs_status run_sd4_mx(const void* a_codes, const void* a_e4m3, const uint16_t* a_
                                    kb_wrap, out_rows, out_M);
 }
 
+// The SD4 quantiser (dialect choice on the tensor cores): codes or e4m3 bytes.
+template <bool E4M3>
+qs_status launch_sd4_quant_tc(const void* x, int64_t rows, int64_t K, void* out, uint16_t* meta,
+                              void* stream) {
+  namespace T = qs::sd4::tc;
+  auto kern = T::sd4_quant_tc_kernel<E4M3>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes) !=
+      cudaSuccess)
+    return QS_ERR_CUDA;
+  const int sms = qs::sm_count();
+  if (sms <= 0) return QS_ERR_CUDA;
+  const int64_t tiles = (rows * (K / 32) + T::kTileBlocks - 1) / T::kTileBlocks;
+  int64_t grid = static_cast<int64_t>(sms) * 4;  // four CTAs fit an SM's shared memory
+  if (grid > tiles) grid = tiles;
+  kern<<<static_cast<unsigned>(grid), T::kThreads, T::kSmemBytes,
+         static_cast<cudaStream_t>(stream)>>>(static_cast<const uint16_t*>(x), rows,
+                                              static_cast<int>(K), static_cast<uint8_t*>(out), meta);
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -540,16 +560,7 @@ qs_status qs_sd4_quant(const void* x_bf16, int64_t rows, int64_t K, void* codes,
   QS_TRY(check_device_ptr(x_bf16));
   QS_TRY(check_device_ptr(codes));
   QS_TRY(check_device_ptr(meta));
-  const int sms = qs::sm_count();
-  if (sms <= 0) return QS_ERR_CUDA;
-  const int64_t chunks = rows * (K / 256);
-  int64_t grid = (chunks + qs::sd4::kWarps - 1) / qs::sd4::kWarps;
-  if (grid > static_cast<int64_t>(sms) * 4) grid = static_cast<int64_t>(sms) * 4;
-  qs::sd4::sd4_quant_kernel<false><<<static_cast<unsigned>(grid), qs::sd4::kThreads, 0,
-                                     static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint16_t*>(x_bf16), rows, static_cast<int>(K),
-      static_cast<uint8_t*>(codes), meta);
-  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+  return launch_sd4_quant_tc<false>(x_bf16, rows, K, codes, meta, stream);
 }
 
 qs_status qs_sd4_quant_e4m3(const void* x_bf16, int64_t rows, int64_t K, void* out_e4m3,
@@ -561,16 +572,7 @@ qs_status qs_sd4_quant_e4m3(const void* x_bf16, int64_t rows, int64_t K, void* o
   QS_TRY(check_device_ptr(x_bf16));
   QS_TRY(check_device_ptr(out_e4m3));
   QS_TRY(check_device_ptr(meta));
-  const int sms = qs::sm_count();
-  if (sms <= 0) return QS_ERR_CUDA;
-  const int64_t chunks = rows * (K / 256);
-  int64_t grid = (chunks + qs::sd4::kWarps - 1) / qs::sd4::kWarps;
-  if (grid > static_cast<int64_t>(sms) * 4) grid = static_cast<int64_t>(sms) * 4;
-  qs::sd4::sd4_quant_kernel<true><<<static_cast<unsigned>(grid), qs::sd4::kThreads, 0,
-                                    static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint16_t*>(x_bf16), rows, static_cast<int>(K),
-      static_cast<uint8_t*>(out_e4m3), meta);
-  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+  return launch_sd4_quant_tc<true>(x_bf16, rows, K, out_e4m3, meta, stream);
 }
 
 qs_status qs_sd4_linear(const void* x_codes, const uint16_t* x_meta, const void* w_codes,

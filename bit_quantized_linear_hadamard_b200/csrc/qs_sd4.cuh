@@ -270,6 +270,254 @@ __global__ void __launch_bounds__(kThreads) sd4_quant_kernel(const uint16_t* __r
   }
 }
 
+// --------------------------------------------------------------------------
+// SD4 quantiser with the dialect choice on the tensor cores.  A block's cost
+// for dialect d, sum_k Qerror[d][b_k], equals sum_b count[b] Qerror[d][b]
+// with count the block's histogram over the 256 bins: an exact integer
+// product of the count matrix (128 blocks x 256 bins, unsigned bytes, at most
+// 32) with the cost table split into low and high bytes (64 x 256 unsigned
+// bytes: Qerror <= 16129 = 63 * 256 + 1), accumulated in int32 (at most
+// 32 * 255 per column: exact).  One thread per block: it loads the block,
+// takes e and the bins, builds its row of the count matrix in shared memory
+// (zeroed, then one non-returning shared add per element into a byte
+// counter), and after the MMA reads its row of the costs back from tensor
+// memory, takes the argmin (smallest d on ties) and writes the codes.
+namespace tc {
+
+constexpr int kTileBlocks = 128;  // rows of the count matrix per tile
+constexpr int kThreads = kTileBlocks;
+constexpr int kHHalf = kTileBlocks * 128;  // one K-half of the count matrix (128 bins)
+constexpr int kQHalf = 64 * 128;           // one K-half of the cost bytes (64 rows)
+constexpr int kOffH = 0;
+constexpr int kOffQ = kOffH + 2 * kHHalf;
+constexpr int kOffE4 = kOffQ + 2 * kQHalf;
+constexpr int kOffLvl = kOffE4 + kDialects * 8;
+constexpr int kOffMisc = kOffLvl + kDialects * 8 * 4;  // mbarrier, TMEM address, abort flag
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;       // + alignment slack
+constexpr int kTmemCols = 64;
+static_assert(kOffQ % 1024 == 0, "alignment");
+
+// Byte offset of (row r, byte c < 128) in a K-major tile of 128-byte rows
+// stored with the 128-byte swizzle.
+__device__ __forceinline__ int sw128(int r, int c) {
+  return r * 128 + ((((c >> 4) ^ (r & 7)) << 4) | (c & 15));
+}
+
+// Instruction descriptor: kind::i8 with unsigned A and B, int32 D, K-major.
+__host__ __device__ constexpr uint32_t idesc_u8(int M, int N) {
+  return (2u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+template <bool E4M3>
+__global__ void __launch_bounds__(kThreads) sd4_quant_tc_kernel(const uint16_t* __restrict__ x,
+                                                               int64_t rows, int K,
+                                                               uint8_t* __restrict__ out,
+                                                               uint16_t* __restrict__ meta) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+  uint8_t* sp = smem_raw + pad;
+  const uint32_t sbase = raw + pad;
+  uint8_t* H = sp + kOffH;
+  uint8_t* Q = sp + kOffQ;
+  uint2* e4 = reinterpret_cast<uint2*>(sp + kOffE4);
+  int* lvl = reinterpret_cast<int*>(sp + kOffLvl);
+  const uint32_t bar = sbase + kOffMisc;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sp + kOffMisc + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + kOffMisc + 12);
+  const int tid = threadIdx.x, warp = tid >> 5;
+
+  for (int i = tid; i < kDialects * 8; i += kThreads) lvl[i] = level(i / 8, i % 8);
+  __syncthreads();
+  for (int idx = tid; idx < kDialects * kBins; idx += kThreads) {
+    const int d = idx / kBins, b = idx % kBins;
+    uint32_t best = 0xFFFFFFFFu;
+    for (int i = 0; i < 8; ++i) {
+      const int diff = 2 * b + 1 - 32 * lvl[d * 8 + i];
+      best = min(best, static_cast<uint32_t>(diff * diff));
+    }
+    uint8_t* qh = Q + (b >> 7) * kQHalf;
+    qh[sw128(d, b & 127)] = static_cast<uint8_t>(best & 0xFFu);      // low bytes: rows 0..31
+    qh[sw128(32 + d, b & 127)] = static_cast<uint8_t>(best >> 8);    // high bytes: rows 32..63
+  }
+  for (int d = tid; d < kDialects; d += kThreads) {
+    uint32_t lo = 0, hi = 0;
+    for (int i = 0; i < 4; ++i) {
+      lo |= e4m3_eighths(lvl[d * 8 + i]) << (8 * i);
+      hi |= e4m3_eighths(lvl[d * 8 + i + 4]) << (8 * i);
+    }
+    e4[d] = make_uint2(lo, hi);
+  }
+  fence_proxy_async_smem();  // the cost bytes are read by the tensor cores
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int64_t nblocks = rows * static_cast<int64_t>(K / kBlock);
+  const int64_t ntiles = (nblocks + kTileBlocks - 1) / kTileBlocks;
+  uint32_t phase = 0;
+  uint8_t* hrow0 = H + tid * 128;
+  uint8_t* hrow1 = H + kHHalf + tid * 128;
+  // the block's 32 elements (blocks are consecutive: row-major, K % 32 == 0);
+  // the next tile's are loaded while this one is processed
+  auto load_block = [&](int64_t tt, uint4 (&r)[4]) {
+    const int64_t bb = tt * kTileBlocks + tid;
+    const uint4* src = reinterpret_cast<const uint4*>(x + bb * kBlock);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      r[q] = (tt < ntiles && bb < nblocks) ? __ldcs(src + q) : make_uint4(0u, 0u, 0u, 0u);
+  };
+  uint4 nxt[4];
+  load_block(blockIdx.x, nxt);
+  for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    const int64_t blk = t * kTileBlocks + tid;
+    const bool valid = blk < nblocks;
+    uint4 raw4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) raw4[q] = nxt[q];
+    load_block(t + gridDim.x, nxt);
+    float amax = 0.f;
+    uint32_t neg = 0;  // bit k: element k is negative
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t w[4] = {raw4[q].x, raw4[q].y, raw4[q].z, raw4[q].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float a0 = __uint_as_float(w[k] << 16), a1 = __uint_as_float(w[k] & 0xFFFF0000u);
+        amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
+        neg |= (a0 < 0.f ? 1u : 0u) << (8 * q + 2 * k);
+        neg |= (a1 < 0.f ? 1u : 0u) << (8 * q + 2 * k + 1);
+      }
+    }
+    int e = 0;
+    if (amax != 0.f) {
+      const int ef = (__float_as_uint(amax) >> 23) & 0xFF;
+      e = ef == 0 ? -126 : max(ef - 127, -126);
+    }
+    const float sc = pow2f(-e);  // exact; |x| 2^-e < 2
+    uint32_t binw[8];            // bins, 4 per word, element k in byte k % 4 of word k / 4
+    // this block's row of the count matrix: zero, then one add per element
+    // chunk order rotated by the row: the 8 lanes of a store phase hit 8
+    // different 16-byte bank groups (rows are 128 bytes apart)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      reinterpret_cast<uint4*>(hrow0)[c ^ (tid & 7)] = make_uint4(0u, 0u, 0u, 0u);
+      reinterpret_cast<uint4*>(hrow1)[c ^ (tid & 7)] = make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t w[4] = {raw4[q].x, raw4[q].y, raw4[q].z, raw4[q].w};
+      uint32_t bw0 = 0, bw1 = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t h = (k & 1) ? (w[k >> 1] & 0xFFFF0000u) : (w[k >> 1] << 16);
+        const float v = __fmul_rn(__fmul_rn(fabsf(__uint_as_float(h)), sc), 128.f);
+        const int bv = static_cast<int>(v);  // truncation = floor for v >= 0
+        const uint32_t b = static_cast<uint32_t>(bv > 255 ? 255 : bv);
+        if (k < 4)
+          bw0 |= b << (8 * k);
+        else
+          bw1 |= b << (8 * (k - 4));
+        const int off = (b >> 7) * kHHalf + sw128(tid, static_cast<int>(b & 127u));
+        atomicAdd(reinterpret_cast<uint32_t*>(H + (off & ~3)), 1u << (8 * (off & 3)));
+      }
+      binw[2 * q] = bw0;
+      binw[2 * q + 1] = bw1;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t idesc = idesc_u8(kTileBlocks, 64);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int half = j >> 2, koff = (j & 3) * 32;
+        mma_i8(tmem_base, smem_desc_sw128(sbase + kOffH + half * kHHalf + koff),
+               smem_desc_sw128(sbase + kOffQ + half * kQHalf + koff), idesc, j != 0);
+      }
+      mma_commit(bar);
+      if (!mbar_wait_bounded(bar, phase, abort_flag, kErrWaitMma)) *abort_flag = 1;
+      tc_fence_before();
+    }
+    __syncthreads();
+    if (*abort_flag) break;  // uniform: every thread sees the flag after the barrier
+    phase ^= 1u;
+    tc_fence_after();
+    uint32_t lo[32], hi[32];
+    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * warp) << 16);
+    tmem_ld_32x32b_x32(taddr, lo);
+    tmem_ld_32x32b_x32(taddr + 32, hi);
+    tmem_wait_ld();
+    uint32_t best = 0xFFFFFFFFu;
+    int d = 0;
+#pragma unroll
+    for (int dd = 0; dd < kDialects; ++dd) {
+      const uint32_t cost = hi[dd] * 256u + lo[dd];
+      if (cost < best) {
+        best = cost;
+        d = dd;
+      }
+    }
+    // Qvalue[d][b], the nearest level, is the number of level midpoints
+    // 16 (L_i + L_i+1) below 2b + 1 (odd against even: never a tie)
+    uint32_t mid[7];
+#pragma unroll
+    for (int i = 0; i < 7; ++i) mid[i] = static_cast<uint32_t>(16 * (lvl[d * 8 + i] + lvl[d * 8 + i + 1]));
+    uint32_t cw[4];  // codes, element k in nibble k % 8 of word k / 8
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t c = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t b2 = 2u * ((binw[(8 * q + k) >> 2] >> (8 * (k & 3))) & 0xFFu) + 1u;
+        uint32_t idx = 0;
+#pragma unroll
+        for (int i = 0; i < 7; ++i) idx += b2 > mid[i] ? 1u : 0u;
+        const uint32_t code = (((neg >> (8 * q + k)) & 1u) << 3) | idx;
+        c |= code << (4 * k);
+      }
+      cw[q] = c;
+    }
+    if (valid) {
+      if (E4M3) {
+        const uint2 E = e4[d];
+        const uint2 o0 = decode8_e4m3(cw[0], E), o1 = decode8_e4m3(cw[1], E);
+        const uint2 o2 = decode8_e4m3(cw[2], E), o3 = decode8_e4m3(cw[3], E);
+        uint4* dst = reinterpret_cast<uint4*>(out + blk * kBlock);
+        dst[0] = make_uint4(o0.x, o0.y, o1.x, o1.y);
+        dst[1] = make_uint4(o2.x, o2.y, o3.x, o3.y);
+      } else {
+        *reinterpret_cast<uint4*>(out + blk * (kBlock / 2)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      }
+      meta[blk] = block_word(e, d);
+    }
+    tc_fence_before();  // this tile's tensor-memory reads precede the next MMA
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    const unsigned long long t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
+  }
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace tc
+
 // Activation decomposition of the salient rows (SemanticDialect "Resumen
 // técnico" §2.B): output row i holds 2K codes, those of x[rows[i]] followed by
 // those of the residual Delta = x - x_hat, and 2K/32 block words.  x_hat =
