@@ -15,14 +15,12 @@
 // (x < 0) << 3 | Qvalue[d][b].  Stored: codes two per byte (element 2j in the
 // low nibble), one 16-bit word per block (low byte e as int8, high byte d).
 //
-// Quantiser: persistent CTAs of 8 warps; each CTA first builds the tables in
-// shared memory.  A warp takes 8 blocks (256 elements) at a time: each lane
-// loads 8 elements (16 bytes), four lanes reduce a block's absmax, and the
-// bins go to shared memory; then for each block lane d sums dialect d's cost
-// (conflict-free: the table is laid out [bin][dialect]) and a warp minimum on
-// (cost << 5 | d) picks the dialect; finally each lane writes its 8 codes.
-// (Scoring runs two blocks at a time on packed 16-bit Qerror pairs: see
-// Tables.)
+// Quantiser (tc::sd4_quant_tc_kernel): one thread per block, the dialect
+// choice as an exact integer product on the tensor cores (see there).  The
+// activation decomposition uses a warp-level form (quant_warp_chunk): a warp
+// takes 8 blocks (256 elements), four lanes reduce a block's absmax, and the
+// half-warps score two blocks at a time on packed 16-bit Qerror pairs (see
+// Tables), a warp minimum on (cost << 5 | d) picking the dialect.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -223,51 +221,6 @@ __device__ __forceinline__ void load_chunk8(const uint16_t* __restrict__ src, in
 __device__ __forceinline__ uint16_t block_word(int e, int d) {
   return static_cast<uint16_t>((static_cast<uint32_t>(e) & 0xFFu) |
                                (static_cast<uint32_t>(d) << 8));
-}
-
-// E4M3: instead of packed codes, each element's value as an e4m3 byte (the
-// sign and L/8; the block words keep the scales): [rows, K] bytes.
-template <bool E4M3>
-__global__ void __launch_bounds__(kThreads) sd4_quant_kernel(const uint16_t* __restrict__ x,
-                                                            int64_t rows, int K,
-                                                            uint8_t* __restrict__ codes,
-                                                            uint16_t* __restrict__ meta) {
-  __shared__ Tables tb;
-  __shared__ __align__(16) uint8_t s_bins[kWarps][8][kBlock];
-  __shared__ uint2 s_e4m3[E4M3 ? kDialects : 1];
-  build_tables(&tb);
-  if (E4M3) {
-    for (int d = threadIdx.x; d < kDialects; d += blockDim.x) {
-      uint32_t lo = 0, hi = 0;
-      for (int i = 0; i < 4; ++i) {
-        lo |= e4m3_eighths(tb.lvl[d][i]) << (8 * i);
-        hi |= e4m3_eighths(tb.lvl[d][i + 4]) << (8 * i);
-      }
-      s_e4m3[d] = make_uint2(lo, hi);
-    }
-    __syncthreads();
-  }
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int blocks_per_row = K / kBlock;
-  const int64_t chunks_per_row = K / 256;  // 8 blocks per chunk (K % 256 == 0)
-  const int64_t num_chunks = rows * chunks_per_row;
-  for (int64_t c = static_cast<int64_t>(blockIdx.x) * kWarps + warp; c < num_chunks;
-       c += static_cast<int64_t>(gridDim.x) * kWarps) {
-    const int64_t row = c / chunks_per_row;
-    const int col0 = static_cast<int>(c % chunks_per_row) * 256;
-    float a[8];
-    load_chunk8(x + row * static_cast<int64_t>(K) + col0, lane, a);
-    int e, d;
-    const uint32_t packed = quant_warp_chunk(a, tb, s_bins[warp], lane, e, d);
-    if (E4M3)
-      *reinterpret_cast<uint2*>(codes + row * static_cast<int64_t>(K) + col0 + 8 * lane) =
-          decode8_e4m3(packed, s_e4m3[d]);
-    else
-      *reinterpret_cast<uint32_t*>(codes + row * static_cast<int64_t>(K / 2) + col0 / 2 +
-                                   4 * lane) = packed;
-    if ((lane & 3) == 0) meta[row * blocks_per_row + col0 / kBlock + (lane >> 2)] = block_word(e, d);
-  }
 }
 
 // --------------------------------------------------------------------------
