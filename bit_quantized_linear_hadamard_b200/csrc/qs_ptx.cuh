@@ -278,12 +278,17 @@ __device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
-// Arrive once on the mbarrier at cluster-window address `bar` (in either CTA of
-// the pair) when all tcgen05 operations issued so far by this thread are done.
-__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
+// Arrive once on the mbarrier at the shared-memory offset `bar` in BOTH CTAs of
+// the pair when all tcgen05 operations issued so far by this thread are done:
+// one commit with a CTA mask of 0b11 (each CTA's barrier sits at the same
+// offset).  It replaces a commit per CTA; the tensor pipe handles one commit
+// per k-block instead of two, which measured 3-5 % faster on the 8x4 GEMM.
+__device__ __forceinline__ void mma_commit_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
 }
 
 // Arrive once on `bar` when every tcgen05 operation issued so far by this
