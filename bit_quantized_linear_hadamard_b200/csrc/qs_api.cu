@@ -745,6 +745,17 @@ qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream
   const int sms = qs::sm_count();
   if (sms <= 0) return QS_ERR_CUDA;
   const int64_t nvec = n / 8;
+  if (n >= qs::kGeluTableMinElems) {
+    // one CTA per SM (the 128 KB table), each building its own table
+    if (cudaFuncSetAttribute(qs::gelu_bf16_table_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             qs::kGeluTableBytes) != cudaSuccess)
+      return QS_ERR_CUDA;
+    qs::gelu_bf16_table_kernel<<<static_cast<unsigned>(sms), qs::kGeluTableThreads,
+                                 qs::kGeluTableBytes, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint16_t*>(x_bf16), n, static_cast<uint16_t*>(y_bf16));
+    return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+  }
   int64_t blocks = (nvec + 255) / 256;
   const int64_t cap = static_cast<int64_t>(sms) * 8;
   if (blocks > cap) blocks = cap;

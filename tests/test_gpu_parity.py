@@ -327,6 +327,24 @@ def test_gelu_matches_oracle():
     assert_within_1ulp(got, O.gelu_erf_bf16(bits16(x)), "gelu")
 
 
+def test_gelu_table_path_covers_every_bf16_pattern():
+    """Inputs of 2^24 elements and more take the shared-memory table kernel:
+    every one of the 65536 bf16 bit patterns (tiled 256 times, plus a ragged
+    tail of 5) must give the direct kernel's bits, and every finite pattern
+    must be within 1 bf16 ulp of the oracle."""
+    pats = np.arange(65536, dtype=np.uint16)
+    direct = qs.gelu(torch.from_numpy(pats.view(np.int16)).view(torch.bfloat16).cuda())
+    big = np.concatenate([np.tile(pats, 256), pats[:5]])
+    tab = qs.gelu(torch.from_numpy(big.view(np.int16)).view(torch.bfloat16).cuda())
+    torch.cuda.synchronize()
+    d = direct.view(torch.int16).cpu().numpy().view(np.uint16)
+    t = tab.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(t[:65536 * 256].reshape(256, 65536), np.broadcast_to(d, (256, 65536)))
+    assert np.array_equal(t[65536 * 256:], d[:5])
+    finite = (pats & 0x7F80) != 0x7F80
+    assert_within_1ulp(d[finite], O.gelu_erf_bf16(pats[finite]), "gelu all patterns")
+
+
 # --------------------------------------------------------------------------- full-size configs
 
 def _sampled_parity(d, bits, alpha, rows, cols, bits_x=None, x_flags=0):
