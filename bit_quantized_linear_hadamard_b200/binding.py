@@ -641,24 +641,31 @@ class QuantLinear:
     """A Hadamard-rotated quantized linear layer (W4A4, W8A8, or mixed such as
     W4A8 / W4A6 with ``bits_x``): weights packed once; each call runs the
     one-call layer (the activation kernel, then the GEMM) on a workspace the
-    layer keeps and grows as needed."""
+    layer keeps and grows as needed.  ``act_codes`` stores 4-bit activation
+    codes one per byte ("bytes", the faster GEMM: only the weights are widened
+    in shared memory) or two per byte ("packed"); the codes, and so the
+    outputs, are the same."""
 
     def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None, bits: int,
-                 alpha: float = 1.0, bits_x: int | None = None):
+                 alpha: float = 1.0, bits_x: int | None = None, act_codes: str = "bytes"):
+        if act_codes not in ("bytes", "packed"):
+            raise ValueError("act_codes is 'bytes' or 'packed'")
         self.N, self.K = weight.shape
         self.bits = bits
         self.bits_x = bits if bits_x is None else bits_x
         self.alpha = alpha
+        self.x_flags = QS_FLAG_BYTE_CODES if (self.bits_x == 4 and act_codes == "bytes") else 0
         self.w_packed, self.w_scale = pack_weights(weight, bits)
         self.bias = bias
         self.workspace = None
 
     def __call__(self, x: torch.Tensor, stream=None, out=None) -> torch.Tensor:
-        need = qs_linear_workspace_bytes(x.shape[0], self.K, self.bits_x)
+        need = qs_linear_workspace_bytes(x.shape[0], self.K, storage_bits(self.bits_x, self.x_flags))
         if self.workspace is None or self.workspace.numel() < need:
             self.workspace = torch.empty((max(need, 0),), dtype=torch.uint8, device=x.device)
         return linear(x, self.w_packed, self.w_scale, self.bias, self.bits_x, self.alpha,
-                      self.workspace, stream=stream, out=out, bits_w=self.bits)
+                      self.workspace, stream=stream, out=out, bits_w=self.bits,
+                      x_flags=self.x_flags)
 
 
 def gbs_state_host(state) -> dict:

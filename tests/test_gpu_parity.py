@@ -284,6 +284,20 @@ def test_linear_mixed_one_call(bx, bw):
     assert np.array_equal(want, r["out"])
 
 
+@pytest.mark.parametrize("act_codes", ["bytes", "packed"])
+def test_quant_linear_layer_w4a4_both_code_layouts(act_codes):
+    M, N, K, alpha = 300, 768, 640, 0.9
+    d = I.make_shape(seed=37, M=M, K=K, N=N, bits=4, alpha=alpha, outlier_factor=50.0)
+    layer = qs.QuantLinear(d["w"].cuda(), d["bias"].cuda(), 4, alpha, act_codes=act_codes)
+    assert layer.x_flags == (qs.QS_FLAG_BYTE_CODES if act_codes == "bytes" else 0)
+    out = layer(d["x"].cuda())
+    out_again = layer(d["x"][:7].cuda())  # the workspace kept from the larger call
+    torch.cuda.synchronize()
+    r = O.qlinear(bits16(d["x"]), bits16(d["w"]), bits16(d["bias"]), 4, alpha)
+    assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), r["out"])
+    assert np.array_equal(out_again.view(torch.int16).cpu().numpy().view(np.uint16), r["out"][:7])
+
+
 def test_qlinear_null_bias_and_zero_rows():
     d = I.make_shape(seed=5, M=130, K=256, N=272, bits=4)
     d["x"][3] = 0
