@@ -143,6 +143,22 @@ def test_binding_raises_without_cuda_tensors():
         binding.quant_act(torch.zeros(4, 128, dtype=torch.bfloat16), 4)
 
 
+def test_quant_linear_rejects_an_unknown_code_layout():
+    import torch
+    with pytest.raises(ValueError):
+        binding.QuantLinear(torch.zeros((16, 128), dtype=torch.bfloat16), None, 4,
+                            act_codes="nibbles")
+
+
+def test_storage_widths():
+    assert binding.storage_bits(4) == 4
+    assert binding.storage_bits(4, binding.QS_FLAG_BYTE_CODES) == 8
+    assert binding.storage_bits(8) == 8
+    assert binding.packed_cols(5120, 4) == 2560
+    assert binding.packed_cols(5120, 4, binding.QS_FLAG_BYTE_CODES) == 5120
+    assert binding.packed_cols(5120, 6) == 5120 and binding.packed_cols(5120, 8) == 5120
+
+
 def test_linear_validation_and_workspace(lib):
     assert lib.qs_linear_workspace_bytes(256, 512, 4) == 256 * 256 + 4 * 256
     assert lib.qs_linear_workspace_bytes(3, 128, 4) == 256 + 12          # packed part rounded to 256
