@@ -59,7 +59,7 @@ __device__ __forceinline__ uint4 gelu_lookup8(const uint16_t* tab, uint4 d) {
 }
 
 __global__ void __launch_bounds__(kGeluTableThreads, 1)
-    gelu_bf16_table_kernel(const uint16_t* __restrict__ x, int64_t n, uint16_t* __restrict__ y) {
+    gelu_bf16_table_kernel(const uint16_t* x, int64_t n, uint16_t* y) {  // x and y may alias
   extern __shared__ __align__(16) uint16_t gelu_tab[];
   for (int i = threadIdx.x; i < 65536; i += blockDim.x)
     gelu_tab[i] = static_cast<uint16_t>(gelu_bf16_bits(static_cast<uint32_t>(i)));

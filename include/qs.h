@@ -487,7 +487,13 @@ QS_API qs_status qs_linear_gbs(const void* x_bf16, int64_t M, int64_t K, float a
 /*
  * qs_gelu_bf16 — elementwise GELU (exact erf form, binary32 arithmetic,
  * bf16 in and out) used between the ffn-up and ffn-down linears of a
- * transformer block chain.  n elements; x and y may alias.
+ * transformer block chain.  n elements; x and y may alias (each element is
+ * read and written by the same thread).  For n >= 2^24 each CTA first
+ * tabulates the function over all 65536 bf16 inputs in shared memory and
+ * then reads the table: the same bits as the direct evaluation.
+ * Errors: QS_ERR_NULL, QS_ERR_SHAPE (n <= 0), QS_ERR_ALIGN (x or y not
+ * 16-byte aligned), QS_ERR_PTR (not device memory of the current device),
+ * QS_ERR_CUDA.
  */
 QS_API qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream);
 
