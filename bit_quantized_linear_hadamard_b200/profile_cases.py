@@ -13,6 +13,8 @@ Cases:
   sd4_gemm_codes  qs_sd4_linear (block-scaled fp8 GEMM decoding SD4 codes)
   sd4_quant_e4m3  qs_sd4_quant_e4m3 (SD4 activation quantiser, e4m3 bytes out)
   gbs_update      qs_gbs_update (normalised L1 change of two layer outputs)
+  gelu            qs_gelu_bf16 on an up-projection output (2^24 elements and more:
+                  the shared-memory table kernel)
 """
 
 from __future__ import annotations
@@ -37,7 +39,7 @@ def _inputs(M: int):
 def main(argv=None) -> None:
     p = argparse.ArgumentParser()
     p.add_argument("case", choices=["sd4_gemm_e4m3", "sd4_gemm_codes", "sd4_quant_e4m3",
-                                    "gbs_update"])
+                                    "gbs_update", "gelu"])
     p.add_argument("--tokens", type=int, default=None)
     a = p.parse_args(argv)
     qs.load()
@@ -60,6 +62,12 @@ def main(argv=None) -> None:
         x8 = torch.empty((M, K), dtype=torch.uint8, device="cuda")
         mx = torch.empty((M, K // 32), dtype=torch.int16, device="cuda")
         run = lambda: qs.qs_sd4_quant_e4m3(x, M, K, x8, mx)  # noqa: E731
+    elif a.case == "gelu":
+        M = a.tokens or 4096
+        g = torch.Generator(device="cuda").manual_seed(2)
+        y0 = (2.0 * torch.randn(M, N, device="cuda", generator=g)).to(torch.bfloat16)
+        y1 = torch.empty_like(y0)
+        run = lambda: qs.qs_gelu_bf16(y0, M * N, y1)  # noqa: E731
     else:
         M = a.tokens or 8192
         g = torch.Generator(device="cuda").manual_seed(1)
