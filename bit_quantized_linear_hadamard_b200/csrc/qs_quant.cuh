@@ -177,12 +177,16 @@ __device__ __forceinline__ void add_row_sum(int* rowsum, int64_t row, int part, 
 // positions, free of bank conflicts.  A half lives in registers as 32 pairs
 // (v[j], v[j + 32]): butterfly stages h = 1..16 pair (j, j + h) and
 // (j + 32, j + 32 + h) alike, so two butterflies are one packed add.rn.f32x2
-// and one sub.rn.f32x2 (independent IEEE binary32 operations); stage 32 works
-// inside the pairs; stage 64 pairs the two threads: each takes its partner's
-// value p by an xor-shuffle and forms fl(p + sg * own) with sg = +1 (low
-// half: a + b) or -1 (high half: a - b) in one packed fma -- sg * own is exact,
-// so the single rounding is that of the butterfly's add or subtract.  Packed
-// subtraction a - b is likewise fma(b, -1, a).
+// and one packed fma (independent IEEE binary32 operations; a - b is
+// fma(b, -1, a): the product is exact, the one rounding is the subtraction's).
+// Stage 32 works inside the pairs, as fma(b, c, a) with c = +-1; the high
+// thread keeps its result swapped, (out[96 + j], out[64 + j]).  Stage 64 pairs
+// the two threads, and each finishes both outputs of half the butterflies:
+// it receives its partner's .y by one xor-shuffle (r) and forms
+// (keep + r, keep - r) from its own .x (keep), giving (out[j], out[64 + j])
+// in the low thread and (out[32 + j], -out[96 + j]) in the high one -- one
+// shuffle per pair of values, where exchanging whole halves takes two.  The
+// sign is exact and is undone by the quantisation multiplier of that lane.
 //
 // One __syncthreads per group: the row absmax (pair shuffle, then a
 // shared-memory atomicMax of the bit patterns, triple-buffered so that no
@@ -288,17 +292,24 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
             p[j] = __fadd2_rn(a, b);
             p[j + h] = __ffma2_rn(b, neg1, a);  // a - b, one rounding
           }
+      // h = 32 inside the pairs (the high thread's result swapped)
+      const float2 c32 = make_float2(up ? -1.f : 1.f, up ? 1.f : -1.f);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {  // h = 32: (v[j], v[j + 32])
-        const float a = p[j].x, b = p[j].y;
-        p[j] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+      for (int j = 0; j < 32; ++j)
+        p[j] = __ffma2_rn(make_float2(p[j].y, p[j].y), c32, make_float2(p[j].x, p[j].x));
+      // h = 64: (keep + r, keep - r) with r the partner's .y
+      const float2 pm = make_float2(1.f, -1.f);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float r = __shfl_xor_sync(0xffffffffu, p[j].y, 1);
+        p[j] = __ffma2_rn(make_float2(r, r), pm, make_float2(p[j].x, p[j].x));
       }
-      const float2 sg2 = make_float2(up ? -1.f : 1.f, up ? -1.f : 1.f);
+    } else {
+      // no rotation: the same element layout, low (j, 64 + j), high (32 + j, 96 + j)
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {  // h = 64: the partner thread holds the other half
-        const float pa = __shfl_xor_sync(0xffffffffu, p[j].x, 1);
-        const float pb = __shfl_xor_sync(0xffffffffu, p[j].y, 1);
-        p[j] = __ffma2_rn(sg2, p[j], make_float2(pa, pb));
+      for (int j = 0; j < 32; ++j) {
+        const float r = __shfl_xor_sync(0xffffffffu, up ? p[j].x : p[j].y, 1);
+        p[j] = up ? make_float2(r, p[j].y) : make_float2(p[j].x, r);
       }
     }
 
@@ -330,11 +341,12 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
     if (blk == 0 && up == 0)
       scale_out[row] = zero_row ? 0.f : __fmul_rn(__fdiv_rn(t_row, static_cast<float>(kQmax)), scale_mul);
 
-    const float2 inv2 = make_float2(inv, inv);
+    // the high thread's .y holds -out[96 + j] after the rotation
+    const float2 inv2 = make_float2(inv, (rotate && up) ? -inv : inv);
     const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
     [[maybe_unused]] constexpr float kQ = static_cast<float>(kQmax);
-    // Codes of 8 consecutive pairs = elements 8k..8k+7 (low halves) and
-    // 32+8k..32+8k+7 (high halves) of this half block.
+    // Codes of 8 consecutive pairs: .x = elements 32 up + 8k .. + 7 of the
+    // block, .y = elements 64 + 32 up + 8k .. + 7.
     uint32_t wlo[STORE == 4 ? 4 : 8], whi[STORE == 4 ? 4 : 8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -369,16 +381,19 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
         whi[2 * k + 1] = pack4_int8(chi[4], chi[5], chi[6], chi[7]);
       }
     }
-    uint8_t* dst =
-        out + row * static_cast<int64_t>(K * STORE / 8) + blk * (2 * kOutBytes) + up * kOutBytes;
-    if (STORE == 4) {  // 16 bytes of elements 0..31, then 16 bytes of 32..63
-      *reinterpret_cast<uint4*>(dst) = make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
-      *reinterpret_cast<uint4*>(dst + 16) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
+    // the .x codes cover elements 32 up .. 32 up + 31 of the block, the .y
+    // codes 64 + 32 up .. 64 + 32 up + 31: two 16-byte aligned pieces
+    uint8_t* dst = out + row * static_cast<int64_t>(K * STORE / 8) + blk * (2 * kOutBytes);
+    uint8_t* dlo = dst + up * (kOutBytes / 2);
+    uint8_t* dhi = dst + kOutBytes + up * (kOutBytes / 2);
+    if (STORE == 4) {
+      *reinterpret_cast<uint4*>(dlo) = make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
+      *reinterpret_cast<uint4*>(dhi) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
     } else {
-      *reinterpret_cast<uint4*>(dst) = make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
-      *reinterpret_cast<uint4*>(dst + 16) = make_uint4(wlo[4], wlo[5], wlo[6], wlo[7]);
-      *reinterpret_cast<uint4*>(dst + 32) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
-      *reinterpret_cast<uint4*>(dst + 48) = make_uint4(whi[4], whi[5], whi[6], whi[7]);
+      *reinterpret_cast<uint4*>(dlo) = make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
+      *reinterpret_cast<uint4*>(dlo + 16) = make_uint4(wlo[4], wlo[5], wlo[6], wlo[7]);
+      *reinterpret_cast<uint4*>(dhi) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
+      *reinterpret_cast<uint4*>(dhi + 16) = make_uint4(whi[4], whi[5], whi[6], whi[7]);
     }
     if (MODE == kRowsum)
       add_row_sum(rowsum, row, packed_code_sum<STORE>(wlo) + packed_code_sum<STORE>(whi), rl);
