@@ -10,8 +10,10 @@
 // per operand element in shared memory (the bf16 form needs two).
 //
 // Persistent, one CTA per SM, tiles of 128 x 192 (two 192-column binary32
-// accumulators and the 12 scale columns fit the 512 TMEM columns; a 256-wide
-// pair would not), 128 K elements (four scale blocks) per stage.
+// accumulators and the 12 scale columns fit the 512 TMEM columns; two
+// 256-column accumulators would leave none for the scales), 128 K elements
+// (four scale blocks) per stage.  Tiles on CTA pairs (cta_group::2, M = 256)
+// measured slower than this single-CTA form.
 // Warp roles: 0 TMA producer (codes every stage, block words every two
 // stages, the decoded weights when given), 1 TMEM allocation and the MMA
 // issuer (per stage: three tcgen05.cp of the stage's scales into TMEM, then
