@@ -423,20 +423,31 @@ __global__ void __launch_bounds__(kThreads) sd4_quant_tc_kernel(const uint16_t* 
       }
     }
     // Qvalue[d][b], the nearest level, is the number of level midpoints
-    // 16 (L_i + L_i+1) below 2b + 1 (odd against even: never a tie)
-    uint32_t mid[7];
+    // 16 (L_i + L_i+1) below 2b + 1 (odd against even: never a tie).  As
+    // 2b + 1 > 16 s  <=>  b >= 8 s  <=>  (b >> 3) >= s, it depends on b >> 3
+    // (0..31) alone: the block's dialect gives the count for all 32 values
+    // as three bit planes (bit v of P_j = bit j of the count at b >> 3 = v),
+    // summed from the seven masks {v >= s_i} by a bit-sliced counter.
+    uint32_t P0 = 0, P1 = 0, P2 = 0;
 #pragma unroll
-    for (int i = 0; i < 7; ++i) mid[i] = static_cast<uint32_t>(16 * (lvl[d * 8 + i] + lvl[d * 8 + i + 1]));
+    for (int i = 0; i < 7; ++i) {
+      const int si = lvl[d * 8 + i] + lvl[d * 8 + i + 1];  // 0..30
+      const uint32_t m = si >= 32 ? 0u : (0xFFFFFFFFu << si);
+      const uint32_t c0 = P0 & m;
+      P0 ^= m;
+      const uint32_t c1 = P1 & c0;
+      P1 ^= c0;
+      P2 ^= c1;  // the count is at most 7
+    }
     uint32_t cw[4];  // codes, element k in nibble k % 8 of word k / 8
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       uint32_t c = 0;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const uint32_t b2 = 2u * ((binw[(8 * q + k) >> 2] >> (8 * (k & 3))) & 0xFFu) + 1u;
-        uint32_t idx = 0;
-#pragma unroll
-        for (int i = 0; i < 7; ++i) idx += b2 > mid[i] ? 1u : 0u;
+        const uint32_t v = (binw[(8 * q + k) >> 2] >> (8 * (k & 3) + 3)) & 31u;  // b >> 3
+        const uint32_t idx =
+            ((P0 >> v) & 1u) | (((P1 >> v) & 1u) << 1) | (((P2 >> v) & 1u) << 2);
         const uint32_t code = (((neg >> (8 * q + k)) & 1u) << 3) | idx;
         c |= code << (4 * k);
       }
