@@ -15,6 +15,10 @@ Cases:
   gbs_update      qs_gbs_update (normalised L1 change of two layer outputs)
   gelu            qs_gelu_bf16 on an up-projection output (2^24 elements and more:
                   the shared-memory table kernel)
+  gemm_w8a8       qs_qlinear, 8-bit activations and weights
+  gemm_w4a8       qs_qlinear_mixed, 8-bit activations, 4-bit weights
+  gemm_bgr        qs_qlinear_asym, 4-bit activations with code sums, 4-bit weights on
+                  bounded (asymmetric) grids
 """
 
 from __future__ import annotations
@@ -39,7 +43,8 @@ def _inputs(M: int):
 def main(argv=None) -> None:
     p = argparse.ArgumentParser()
     p.add_argument("case", choices=["sd4_gemm_e4m3", "sd4_gemm_codes", "sd4_quant_e4m3",
-                                    "gbs_update", "gelu"])
+                                    "gbs_update", "gelu", "gemm_w8a8", "gemm_w4a8",
+                                    "gemm_bgr"])
     p.add_argument("--tokens", type=int, default=None)
     a = p.parse_args(argv)
     qs.load()
@@ -62,6 +67,19 @@ def main(argv=None) -> None:
         x8 = torch.empty((M, K), dtype=torch.uint8, device="cuda")
         mx = torch.empty((M, K // 32), dtype=torch.int16, device="cuda")
         run = lambda: qs.qs_sd4_quant_e4m3(x, M, K, x8, mx)  # noqa: E731
+    elif a.case in ("gemm_w8a8", "gemm_w4a8", "gemm_bgr"):
+        M = a.tokens or 16384
+        x, w, b = _inputs(M)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        if a.case == "gemm_bgr":
+            xp, xs, xr = qs.quant_act_rowsum(x, 4, 1.0)
+            wp, ws, wo = qs.pack_weights_bgr(w, 4)
+            run = lambda: qs.qs_qlinear_asym(xp, xs, xr, wp, ws, wo, b, M, N, K, 4, out)  # noqa: E731
+        else:
+            bits_w = 8 if a.case == "gemm_w8a8" else 4
+            xp, xs = qs.quant_act(x, 8)
+            wp, ws = qs.pack_weights(w, bits_w)
+            run = lambda: qs.qlinear(xp, xs, wp, ws, b, 8, K, out=out, bits_w=bits_w)  # noqa: E731
     elif a.case == "gelu":
         M = a.tokens or 4096
         g = torch.Generator(device="cuda").manual_seed(2)
