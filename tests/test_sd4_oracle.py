@@ -56,6 +56,20 @@ def pin_lut_is_the_nearest_level(s=S):
             assert qerr[d, b] == min((c - Fraction(int(l), 8)) ** 2 for l in L[d]) * 65536
 
 
+def pin_qvalue_changes_only_at_multiples_of_eight_bins(s=S):
+    """Levels are multiples of 1/8 and bins 1/128 wide, so every midpoint
+    (L_i + L_i+1)/16 between neighbouring levels falls on a multiple of 8
+    bins: Qvalue is constant on each run of 8 bins, and it steps exactly at
+    bin 8 (L_i + L_i+1) for every pair of levels of the dialect."""
+    L = s.formatbook()
+    _, qval = s.lut_tables(L)
+    for d in range(32):
+        assert np.array_equal(qval[d], np.repeat(qval[d, ::8], 8)), d
+        steps = sorted(set(int(8 * (L[d, i] + L[d, i + 1])) for i in range(7)))
+        got = [b for b in range(1, 256) if qval[d, b] != qval[d, b - 1]]
+        assert got == [t for t in steps if t < 256], (d, got, steps)
+
+
 def pin_block_scale(s=S):
     """amax normalises into [1, 2); zero blocks; the floor at 2^-126."""
     for amax in (1.0, 1.999, 2.0, 0.75, 3e-5, 6e4):
