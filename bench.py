@@ -74,31 +74,48 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-# the sources of the headline kernels and their launches (the activation
-# kernel, the GEMM, their shared helpers): counters taken on other sources
-# are not reported
+# the sources of each headline kernel and its launch (the kernel's file and
+# the shared helpers): counters taken on other sources are not reported
+KERNEL_SOURCES = {
+    "qgemm_kernel": ("qs_gemm.cuh", "qs_host.cuh", "qs_ptx.cuh"),
+    "rotate_quant_kernel": ("qs_host.cuh", "qs_ptx.cuh", "qs_quant.cuh"),
+}
 HEADLINE_SOURCES = ("qs_gemm.cuh", "qs_host.cuh", "qs_ptx.cuh", "qs_quant.cuh")
 
 
-def kernel_source_hash() -> str:
-    h = hashlib.sha256()
+def source_hash(names, read=None) -> str:
+    """sha256 over (name, contents) of the given csrc files, 16 hex digits;
+    `read(name) -> bytes` supplies the contents (default: the files here)."""
     csrc = os.path.join(ROOT, "bit_quantized_linear_hadamard_b200", "csrc")
-    for name in HEADLINE_SOURCES:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+    if read is None:
+        def read(name):
+            with open(os.path.join(csrc, name), "rb") as f:
+                return f.read()
+    h = hashlib.sha256()
+    for name in names:
+        h.update(name.encode() + read(name))
     return h.hexdigest()[:16]
+
+
+def kernel_source_hash(kernel: str | None = None) -> str:
+    """Hash of one headline kernel's sources, or of all of them."""
+    return source_hash(HEADLINE_SOURCES if kernel is None else KERNEL_SOURCES[kernel])
 
 
 def ncu_traffic(workload: str, kernel: str):
     """DRAM bytes per launch of `kernel` in `workload` from the committed ncu
-    summary, or None if there is none or the kernels changed since the
-    counters were taken."""
+    summary, or None if there is none or the kernel's sources changed since
+    the counters were taken."""
     path = os.path.join(PROFILES, "ncu_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    if d.get("source_hash") != kernel_source_hash():
+    hashes = d.get("source_hashes")
+    if hashes is not None:
+        if kernel not in KERNEL_SOURCES or hashes.get(kernel) != kernel_source_hash(kernel):
+            return None
+    elif d.get("source_hash") != kernel_source_hash():
         return None
     k = d.get("workloads", {}).get(workload, {}).get(kernel)
     return None if k is None else k.get("dram_bytes_per_launch_full")

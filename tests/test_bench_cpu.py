@@ -25,12 +25,26 @@ def test_traffic_lookup_follows_the_kernel_sources():
     path = os.path.join(bench.PROFILES, "ncu_traffic.json")
     with open(path) as f:
         d = json.load(f)
-    got = bench.ncu_traffic(I.WAN_FFN.name, "qgemm_kernel")
-    if d["source_hash"] == bench.kernel_source_hash():
-        assert got == d["workloads"][I.WAN_FFN.name]["qgemm_kernel"]["dram_bytes_per_launch_full"]
-    else:  # the kernels changed since the counters were taken: no stale number
-        assert got is None
+    for kernel in ("qgemm_kernel", "rotate_quant_kernel"):
+        got = bench.ncu_traffic(I.WAN_FFN.name, kernel)
+        if d["source_hashes"][kernel] == bench.kernel_source_hash(kernel):
+            assert got == d["workloads"][I.WAN_FFN.name][kernel]["dram_bytes_per_launch_full"]
+        else:  # the kernel changed since its counters were taken: no stale number
+            assert got is None
     assert bench.ncu_traffic("no such workload", "qgemm_kernel") is None
+    assert bench.ncu_traffic(I.WAN_FFN.name, "no such kernel") is None
+
+
+def test_traffic_of_one_kernel_survives_a_change_to_the_other(monkeypatch):
+    path = os.path.join(bench.PROFILES, "ncu_traffic.json")
+    with open(path) as f:
+        d = json.load(f)
+    rec = dict(d["source_hashes"])
+    monkeypatch.setattr(bench, "kernel_source_hash",
+                        lambda kernel=None: "changed" if kernel == "qgemm_kernel" else rec[kernel])
+    assert bench.ncu_traffic(I.WAN_FFN.name, "qgemm_kernel") is None
+    assert bench.ncu_traffic(I.WAN_FFN.name, "rotate_quant_kernel") == \
+        d["workloads"][I.WAN_FFN.name]["rotate_quant_kernel"]["dram_bytes_per_launch_full"]
 
 
 def test_clock_sampler_reports_the_timed_region_from_nvml(monkeypatch):
