@@ -7,7 +7,9 @@
 //
 // Structure: a persistent kernel launched as clusters of two CTAs on the two
 // SMs of a TPC.  Each pair walks output tiles of 256 x 256 (n fastest, so the
-// whole packed weight stays in L2 while activation tiles stream once).  CTA r
+// whole packed weight stays in L2 while activation tiles stream once; the
+// 8-bit weight of the 8x8 form is twice as large and is walked in bands of
+// N-tiles instead, see kBandN).  CTA r
 // of the pair holds rows [128r, 128r+128) of the x tile and rows
 // [128r, 128r+128) of the W tile; the leader (r = 0) issues one
 // tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 32) per 32-deep K step, which
