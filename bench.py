@@ -283,15 +283,84 @@ class OracleSample:
         self.O.epilogue(acc, sa, self.sw, self.bb)
         return time.perf_counter() - t0
 
-    def baseline(self, rows: int = 128) -> dict:
+    def baseline(self, rows: int = 128, rows_per_core: int = 64) -> dict:
+        """All host cores (one oracle process per core on its own token
+        block) as the value, the one-thread run beside it."""
         dt = self.run(rows)
         ops = 2.0 * rows * self.N * self.K
-        return {"value": ops / dt / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+        single = {"value": ops / dt / 1e12, "unit": UNIT, "cores": 1,
+                  "sample": f"first {rows} tokens, one host thread, {dt:.2f} s",
+                  "tokens_per_s": rows / dt}
+        pool = OraclePool(self)
+        try:
+            prow, pdt = pool.run(rows_per_core)
+        finally:
+            pool.close()
+        pops = 2.0 * prow * self.N * self.K
+        return {"value": pops / pdt / 1e12, "unit": UNIT, "cores": pool.procs, "kind": "oracle",
                 "host": host_info(),
-                "sample": f"first {rows} of {self.x.shape[0]} tokens, full K={self.K}, "
-                          f"N={self.N} (quant_act + int GEMM + epilogue; numpy, one host "
-                          f"thread), {dt:.2f} s",
-                "tokens_per_s": rows / dt}
+                "sample": f"{prow} of {self.x.shape[0]} tokens ({rows_per_core} per process, "
+                          f"{pool.procs} processes, one per host core, each numpy on one "
+                          f"thread), full K={self.K}, N={self.N} (quant_act + int GEMM + "
+                          f"epilogue), {pdt:.2f} s wall",
+                "tokens_per_s": prow / pdt, "single_core": single}
+
+
+def _oracle_worker_init(qw, sw, bb, bits_x, alpha):
+    global _OW
+    from oracle import qs_oracle as O
+    _OW = (O, qw, sw, bb, bits_x, alpha)
+
+
+def _oracle_worker(xb):
+    O, qw, sw, bb, bits_x, alpha = _OW
+    t0 = time.perf_counter()
+    qa, sa = O.quant_act(xb, bits_x, alpha)
+    acc = O.int_gemm(qa, qw)
+    O.epilogue(acc, sa, sw, bb)
+    return time.perf_counter() - t0
+
+
+class OraclePool:
+    """One spawned oracle process per host core (spawned, not forked: the
+    parent has a CUDA context), each with one BLAS/OpenMP thread."""
+
+    def __init__(self, sample: "OracleSample", procs: int | None = None):
+        import multiprocessing as mp
+        self.sample = sample
+        self.procs = procs or os.cpu_count() or 1
+        saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS",
+                                                  "MKL_NUM_THREADS")}
+        for k in saved:
+            os.environ[k] = "1"
+        try:
+            self.pool = mp.get_context("spawn").Pool(
+                self.procs, initializer=_oracle_worker_init,
+                initargs=(sample.qw, sample.sw, sample.bb, sample.bits_x, sample.alpha))
+        finally:
+            for k, v in saved.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+        # every worker imports numpy and the oracle before anything is timed
+        self.pool.map(_oracle_worker, [sample.bf16_bits(sample.x[:2])] * self.procs)
+
+    def run(self, rows_per_proc: int) -> tuple[int, float]:
+        """Token blocks of `rows_per_proc` rows, one per process, all at once:
+        returns (rows, wall seconds)."""
+        blocks = []
+        M = self.sample.x.shape[0]
+        for i in range(self.procs):
+            r0 = (i * rows_per_proc) % max(1, M - rows_per_proc)
+            blocks.append(self.sample.bf16_bits(self.sample.x[r0:r0 + rows_per_proc]).copy())
+        t0 = time.perf_counter()
+        self.pool.map(_oracle_worker, blocks, chunksize=1)
+        return rows_per_proc * self.procs, time.perf_counter() - t0
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
 
 
 def host_info() -> dict:
@@ -631,18 +700,27 @@ def quality(qs, torch, x, w, bias, bits, alpha, stream, rows=256):
 
 
 def run_reference(args, rank, world):
-    """The CPU oracle timed as a bounded sample per step (rank 0 only)."""
+    """The CPU oracle timed as a bounded sample per step on every host core
+    (rank 0 only; the other ranks exit without work)."""
     if rank != 0:
         return
     from bit_quantized_linear_hadamard_b200 import inputs as I
     cfg = workload_config(I, args.workload)
-    d = I.make_layer(cfg, M=256)
+    rows_per_proc = 8
+    d = I.make_layer(cfg, M=max(256, rows_per_proc * (os.cpu_count() or 1)))
     sample = OracleSample(d, cfg.bits, cfg.alpha, cfg.act_bits)
-    rows = 8
-    for _ in range(args.warmup):
-        sample.run(2)
-    secs = sum(sample.run(rows) for _ in range(args.steps))
-    value = 2.0 * rows * cfg.N * cfg.K * args.steps / secs / 1e12
+    pool = OraclePool(sample)
+    try:
+        for _ in range(args.warmup):
+            pool.run(2)
+        secs, rows = 0.0, 0
+        for _ in range(args.steps):
+            r, dt = pool.run(rows_per_proc)
+            secs += dt
+            rows += r
+    finally:
+        pool.close()
+    value = 2.0 * rows * cfg.N * cfg.K / secs / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
@@ -653,11 +731,12 @@ def run_reference(args, rank, world):
                    "bits_x": cfg.act_bits, "alpha": cfg.alpha,
                    "act_codes": args.act_codes if cfg.act_bits == 4 else "packed",
                    "seed": cfg.seed, "parallelism": f"replicas{world}",
-                   "sample_rows_per_step": rows},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                   "sample_rows_per_step": rows // args.steps},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": pool.procs, "kind": "oracle",
                          "host": host_info(),
-                         "sample": f"{rows} tokens per step of the {cfg.M}-token workload, full "
-                                   f"K and N, numpy oracle on one host thread"},
+                         "sample": f"{rows // args.steps} tokens per step ({rows_per_proc} per "
+                                   f"process, one numpy process per host core) of the "
+                                   f"{cfg.M}-token workload, full K and N"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -817,6 +896,20 @@ def main():
     e2e_same = bool(torch.equal(out_host[::1009].to(dev).view(torch.int16),
                                 ref_rows.view(torch.int16)))
 
+    # both storages of 4-bit activation codes, timed the same way (the
+    # headline's own numbers are the ones measured above)
+    layouts = {}
+    if bx == 4:
+        for name, flags in (("packed", 0), ("bytes", qs.QS_FLAG_BYTE_CODES)):
+            if flags == x_flags:
+                q_ms, g_ms = quant_ms, gemm_ms
+            else:
+                q_ms, g_ms, _ = time_layer(qs, torch, x, wp, ws, bias, bits, alpha, stream,
+                                           steps=args.steps, warmup=3, bits_x=bx, x_flags=flags)
+                q_ms, g_ms = combine_ranks([q_ms, g_ms], 1, ops_per_step, world, dev)["times_ms"]
+            layouts[name] = {"quant_ms": q_ms, "gemm_ms": g_ms, "step_ms": q_ms + g_ms,
+                             "x_flags": flags, "headline": flags == x_flags}
+
     extra = {}
     if world == 1 and not args.no_extras:
         if bx == bits:
@@ -829,9 +922,26 @@ def main():
         pk, src = peaks()
         int8_peak = pk["bf16_tflops"] * INT8_PER_BF16
         gemm_tops = ops_per_step / (gemm_ms * 1e-3) / 1e12
-        quant_bytes = M * (2 * K + qs.packed_cols(K, bx, x_flags) + 4)
+        # algorithmic bytes of the activation kernel per token: read 2K (bf16),
+        # write K*b/8 (codes at their width b) and 4 (scale), whatever the
+        # storage layout; the bytes a layout actually writes are reported beside
+        quant_bytes = M * (2 * K + K * bx // 8 + 4)
+        stored_bytes = M * (2 * K + qs.packed_cols(K, bx, x_flags) + 4)
         traffic_key = cfg.name + ("_act_codes_in_bytes" if x_flags else "")
         quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
+        for name, L in layouts.items():
+            key = cfg.name + ("_act_codes_in_bytes" if L["x_flags"] else "")
+            g_tops = ops_per_step / (L["gemm_ms"] * 1e-3) / 1e12
+            q_gbs = quant_bytes / (L["quant_ms"] * 1e-3) / 1e9
+            L.update({
+                "TOPS": ops_per_step * world / (L["step_ms"] * 1e-3) / 1e12,
+                "tokens_per_s": M * world / (L["step_ms"] * 1e-3),
+                "gemm_TOPS": g_tops, "gemm_frac_int8_peak": g_tops / int8_peak,
+                "gemm_kernel": f"qgemm_kernel<{8 if L['x_flags'] else 4},{bits},false,false>",
+                "gemm_traffic": ncu_traffic(key, "qgemm_kernel"),
+                "quant_GBps": q_gbs, "quant_frac_hbm": q_gbs / pk["hbm_gbs"],
+                "quant_stored_bytes": M * (2 * K + qs.packed_cols(K, bx, L["x_flags"]) + 4),
+                "quant_traffic": ncu_traffic(key, "rotate_quant_kernel")})
         line = {
             "metric": METRIC, "value": value, "unit": UNIT,
             "tokens_per_s": M * world / (ms_per_step * 1e-3),
@@ -855,7 +965,10 @@ def main():
                                "unit": "GB/s", "frac": quant_gbs / pk["hbm_gbs"],
                                "traffic": ncu_traffic(traffic_key, "rotate_quant_kernel"),
                                "algorithmic_bytes": quant_bytes,
+                               "algorithmic_bytes_rule": "M*(2K + K*b/8 + 4), b the code width",
+                               "stored_bytes": stored_bytes,
                                "peak_source": f"{src}: hbm_gbs"},
+            "act_code_layouts": layouts,
             "kernels_ms": {"quant": quant_ms, "gemm": gemm_ms},
             "kernels_ms_median": {"quant": statistics.median(quant_each),
                                   "gemm": statistics.median(gemm_each)},

@@ -79,27 +79,61 @@ qs_status check_gemm_args(const void* xp, const void* wp, const void* out, int64
 
 // Scratch of qs_linear_noalloc: one fixed buffer per device, in the module's
 // global memory (no allocation).  Host code only names the symbol; its device
-// address is looked up once per device.
+// address is looked up once per device and context.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[QS_NOALLOC_SCRATCH_BYTES];
 
 std::mutex g_noalloc_mutex;
 void* g_noalloc_addr[64] = {nullptr};
+unsigned long long g_noalloc_ctx[64] = {0};  // context id the address belongs to
 
-// Device address of g_noalloc_scratch on the current device (looked up on the
-// first call for that device), or nullptr if the lookup failed.
+// Unique id of the calling thread's current CUDA context (driver entry points,
+// no link-time libcuda dependency); 0 if it cannot be read.  A context created
+// after cudaDeviceReset gets a new id even if it reuses the old handle's memory.
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_noalloc_scratch on the current device, or nullptr if the
+// lookup failed.  It is looked up with that device current on the first call
+// for the device, and again whenever the calling thread's context differs from
+// the one the cached address was taken in (after a cudaDeviceReset the module
+// may load at another address), or cannot be identified.
 void* noalloc_scratch_address() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
-      cudaGetLastError();
-      return nullptr;
-    }
-    g_noalloc_addr[dev] = p;
+  if (g_noalloc_addr[dev] && ctx != 0 && g_noalloc_ctx[dev] == ctx) return g_noalloc_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
   }
-  return g_noalloc_addr[dev];
+  // the lookup has made the device's context current if it was not
+  g_noalloc_addr[dev] = p;
+  g_noalloc_ctx[dev] = current_context_id();
+  return p;
 }
 
 // Persistent launch of the SD4 GEMM: one CTA per SM at most.
@@ -410,11 +444,15 @@ qs_status qs_linear_gbs(const void* x_bf16, int64_t M, int64_t K, float alpha,
   uint8_t* xp = static_cast<uint8_t*>(workspace);
   float* xs = reinterpret_cast<float*>(xp + (M * K + 255) / 256 * 256);
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+  // The 4-bit step writes its codes one per byte and runs the GEMM form with
+  // 8-bit activation storage and packed 4-bit weights: the same codes and
+  // outputs as the packed 4x4 form, and the faster of the two W4 GEMMs, so
+  // that the low-precision step is the cheaper one.
   for (int bits : {4, 8})
     if (qs::launch_rotate_quant(x, M, static_cast<int>(K), bits, alpha, 1.0f, 1, xp, xs, s, gate,
-                                bits) != cudaSuccess)
+                                bits, nullptr, /*byte_codes=*/true) != cudaSuccess)
       return QS_ERR_CUDA;
-  const qs_status st4 = launch_qgemm<4, 4, false>(xp, xs, w4_packed, w4_scale, bias_bf16, M, N, K,
+  const qs_status st4 = launch_qgemm<8, 4, false>(xp, xs, w4_packed, w4_scale, bias_bf16, M, N, K,
                                                   out_bf16, s, gate, 4);
   if (st4 != QS_OK) return st4;
   return launch_qgemm<8, 8, false>(xp, xs, w8_packed, w8_scale, bias_bf16, M, N, K, out_bf16, s,

@@ -513,6 +513,11 @@ QS_API qs_status qs_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void*
  *   up to 3271 tokens per call).
  *   The first call on a device looks up the buffer's device address (with
  *   that device current); make that first call before any stream capture.
+ *   The address is kept per device together with the id of the CUDA context
+ *   it was taken in; a call from a different context (for instance after
+ *   cudaDeviceReset, when the library's module may load elsewhere) looks it
+ *   up again, so the first call after a reset should also come before any
+ *   capture.
  *   All calls share the one buffer, which keeps the previous call's contents
  *   (every byte the layer reads from it is written earlier in the same call,
  *   so nothing needs clearing); calls that may overlap on the GPU -- on

@@ -235,6 +235,26 @@ def int_gemm(qa: np.ndarray, qw: np.ndarray) -> np.ndarray:
     return acc
 
 
+def int_gemm_f64(qa: np.ndarray, qw: np.ndarray) -> np.ndarray:
+    """The same accumulators through a binary64 matrix product (BLAS), for
+    full-size checks where the exact int64 product is too slow.
+
+    Exact: every code is an integer with |q| <= 127, so every partial sum that
+    any summation order (or fused multiply-add) forms is an integer of
+    magnitude at most sum_k |qa[m,k]| |qw[n,k]| <= 127^2 K, below 2^53 for
+    every K < 5.5e11 -- binary64 represents all of them, and no rounding
+    happens.  Returns int64, checked to fit int32 like :func:`int_gemm`.
+    """
+    a = np.asarray(qa, dtype=np.int8)
+    w = np.asarray(qw, dtype=np.int8)
+    if a.shape[1] * 127 * 127 >= 2 ** 53:
+        raise ValueError("K too large for an exact binary64 product")
+    acc = (a.astype(np.float64) @ w.astype(np.float64).T).astype(np.int64)
+    if acc.size and (acc.max() > 2**31 - 1 or acc.min() < -2**31):
+        raise OverflowError("accumulator does not fit int32")
+    return acc
+
+
 def epilogue(acc: np.ndarray, s_a: np.ndarray, s_w: np.ndarray,
              bias_bits: np.ndarray | None) -> np.ndarray:
     """out = bf16_rne(fl(fl(fl(s_a*s_w) * float(acc)) + bias)); returns uint16 bits."""

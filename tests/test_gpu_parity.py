@@ -3,8 +3,8 @@
 Bar (stated by the layer's targets): packed codes, scales and int32
 accumulators bit-identical; bf16 outputs within 1 bf16 ulp (ordered bit
 patterns).  Inputs are the seeded synthetic tensors; no expected value comes
-from the CUDA path.  Full-size configurations run in the benchmark's launch
-configuration and are checked on sampled rows and columns.
+from the CUDA path.  The full-size configurations, in the benchmark's launch
+configuration, are compared element by element in test_gpu_full_size.py.
 """
 
 import os
@@ -359,76 +359,49 @@ def test_gelu_table_path_covers_every_bf16_pattern():
     assert_within_1ulp(d[finite], O.gelu_erf_bf16(pats[finite]), "gelu all patterns")
 
 
-# --------------------------------------------------------------------------- full-size configs
+# --------------------------------------------------------------------------- multi-tile grids, in full
 
-def _sampled_parity(d, bits, alpha, rows, cols, bits_x=None, x_flags=0):
-    bx = bits if bits_x is None else bits_x
-    g = run_layer(d, bits, alpha, bits_x=bx, x_flags=x_flags)
-    xb, wb, bb = bits16(d["x"][rows]), bits16(d["w"][cols]), bits16(d["bias"][cols])
-    qa, sa = O.quant_act(xb, bx, alpha)
-    qw, sw = O.pack_weights(wb, bits)
-    assert np.array_equal(g["xs"].cpu().numpy()[rows].view(np.uint32), sa.view(np.uint32))
-    assert np.array_equal(g["xp"].cpu().numpy()[rows], O.pack(qa, qs.storage_bits(bx, x_flags)))
-    assert np.array_equal(g["ws"].cpu().numpy()[cols].view(np.uint32), sw.view(np.uint32))
-    assert np.array_equal(g["wp"].cpu().numpy()[cols], O.pack(qw, bits))
-    acc = O.int_gemm(qa, qw)
-    gacc = g["acc"].cpu().numpy()[np.ix_(rows, cols)].astype(np.int64)
-    assert np.array_equal(gacc, acc)
-    out = O.epilogue(acc, sa, sw, bb)
-    got = g["out"].view(torch.int16).cpu().numpy().view(np.uint16)[np.ix_(rows, cols)]
-    assert assert_within_1ulp(got, out, "sampled") == 1.0
-    return g
+# (bits_x, bits_w, x_flags): packed W4A4, W4A4 with byte-stored activation
+# codes (the mixed-storage kernel), W8A8 (banded tile order) and W4A8
+MULTI_TILE_FORMS = [(4, 4, 0), (4, 4, qs.QS_FLAG_BYTE_CODES), (8, 8, 0), (8, 4, 0)]
 
 
-def _samples(M, N, seed):
-    rng = np.random.default_rng(seed)
-    rows = np.unique(np.concatenate([[0, 1, M // 2, M - 129, M - 2, M - 1],
-                                     rng.choice(M, 90, replace=False)]))
-    cols = np.unique(np.concatenate([[0, 255, 256, N - 257, N - 1], rng.choice(N, 120, replace=False)]))
-    return rows, cols
+@pytest.mark.parametrize("bx,bw,flags", MULTI_TILE_FORMS, ids=["w4a4", "w4a4_bytes", "w8a8", "w4a8"])
+def test_multi_tile_grid_every_element(bx, bw, flags):
+    """M = 4096, N = 5120, K = 5120: 16 x 20 = 320 output tiles for 74 CTA
+    pairs, so every pair runs several tiles (the persistent loop, both TMEM
+    accumulator buffers, the operand ring wrapping many times) and the 8-bit
+    x 8-bit form crosses a band edge (18 + 2 N-tiles).  Every code, scale,
+    accumulator and output is compared with the oracle."""
+    M, N, K, alpha = 4096, 5120, 5120, 0.9
+    d = I.make_shape(seed=4096 + 10 * bx + bw, M=M, K=K, N=N, bits=bw, alpha=alpha,
+                     outlier_factor=100.0, outlier_frac=0.005, sigma_w=0.015,
+                     bits_x=bx if bx != bw else 0)
+    g = run_layer(d, bw, alpha, bits_x=bx, x_flags=flags)
+    qa, sa = O.quant_act(bits16(d["x"]), bx, alpha)
+    qw, sw = O.pack_weights(bits16(d["w"]), bw)
+    assert np.array_equal(g["xs"].cpu().numpy().view(np.uint32), sa.view(np.uint32))
+    assert np.array_equal(g["xp"].cpu().numpy(), O.pack(qa, qs.storage_bits(bx, flags)))
+    assert np.array_equal(g["ws"].cpu().numpy().view(np.uint32), sw.view(np.uint32))
+    assert np.array_equal(g["wp"].cpu().numpy(), O.pack(qw, bw))
+    acc = O.int_gemm_f64(qa, qw)
+    assert np.array_equal(g["acc"].cpu().numpy().astype(np.int64), acc)
+    want = O.epilogue(acc, sa, sw, bits16(d["bias"]))
+    got = g["out"].view(torch.int16).cpu().numpy().view(np.uint16)
+    assert assert_within_1ulp(got, want, "multi-tile") == 1.0
 
 
-@pytest.mark.slow
-@pytest.mark.parametrize("cfg", [I.HY_QKV, I.WAN_FFN, I.WAN_FFN_W8, *I.MIXED_CONFIGS],
-                         ids=lambda c: c.name)
-def test_full_size_config_sampled(cfg):
-    d = I.make_layer(cfg)
-    rows, cols = _samples(cfg.M, cfg.N, cfg.seed)
-    _sampled_parity(d, cfg.bits, cfg.alpha, rows, cols, bits_x=cfg.act_bits)
-
-
-@pytest.mark.slow
-def test_full_size_wan_ffn_byte_codes_sampled():
-    # the benchmark's launch configuration: W4A4 with the activation codes one
-    # per byte, the mixed-storage GEMM
-    cfg = I.WAN_FFN
-    d = I.make_layer(cfg)
-    rows, cols = _samples(cfg.M, cfg.N, cfg.seed + 100)
-    _sampled_parity(d, cfg.bits, cfg.alpha, rows, cols, x_flags=qs.QS_FLAG_BYTE_CODES)
-
-
-@pytest.mark.slow
-def test_block_chain_full_size_sampled():
-    ch = I.make_chain(I.WAN_CHAIN)
-    alpha = ch["alpha"]
-    up_out = None
-    for i, L in enumerate(ch["layers"]):
-        bits = L["bits"]
-        if i < 3:
-            x = L["x"]
-        else:
-            xg = qs.gelu(up_out)
-            torch.cuda.synchronize()
-            rows = np.random.default_rng(7).choice(xg.shape[0], 64, replace=False)
-            gb = xg.view(torch.int16).cpu().numpy().view(np.uint16)
-            ub = up_out.view(torch.int16).cpu().numpy().view(np.uint16)
-            assert_within_1ulp(gb[rows], O.gelu_erf_bf16(ub[rows]), "gelu")
-            x = xg.cpu()
-        d = {"x": x, "w": L["w"], "bias": L["bias"]}
-        rows, cols = _samples(x.shape[0], L["N"], 40 + i)
-        g = _sampled_parity(d, bits, alpha, rows, cols)
-        if L["name"] == "ffn_up":
-            up_out = g["out"]
+def test_w8a8_band_edge_small():
+    """The 8-bit x 8-bit form walks N-tiles in bands of 18: N = 5120 has 20
+    N-tiles (a full band and a last band of 2), M = 300 a ragged second M-tile.
+    Full int32 and bf16 parity."""
+    M, N, K = 300, 5120, 256
+    d = I.make_shape(seed=3005, M=M, K=K, N=N, bits=8, outlier_factor=50.0)
+    g = run_layer(d, 8, 1.0)
+    r = O.qlinear(bits16(d["x"]), bits16(d["w"]), bits16(d["bias"]), 8, 1.0)
+    assert np.array_equal(g["acc"].cpu().numpy().astype(np.int64), r["acc"])
+    got = g["out"].view(torch.int16).cpu().numpy().view(np.uint16)
+    assert assert_within_1ulp(got, r["out"], "band edge") == 1.0
 
 
 # --------------------------------------------------------------------------- byte-stored 4-bit codes

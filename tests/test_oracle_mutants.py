@@ -132,6 +132,8 @@ MUTANTS = {
     "weight_scale_not_folded": ("pack_weights", _pack_weights_no_fold),
     "six_bit_qmax_is_2^5": ("QMAX", {4: 7, 6: 32, 8: 127}),
     "six_bit_codes_as_nibbles": ("pack", _pack_six_as_nibbles),
+    "blas_gemm_in_binary32": ("int_gemm_f64", lambda a, w: (np.asarray(a, np.float32) @ np.asarray(w, np.float32).T).astype(np.int64)),
+    "blas_gemm_operand_transposed": ("int_gemm_f64", lambda a, w: (np.asarray(a, np.float64) @ np.asarray(w, np.float64)[:, ::-1].T).astype(np.int64)),
 }
 
 

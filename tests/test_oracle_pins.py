@@ -248,6 +248,44 @@ def pin_int_gemm_bruteforce(o=O):
         assert np.array_equal(o.int_gemm(a, w).astype(np.float64), f64)
 
 
+def pin_int_gemm_f64_exact(o=O):
+    """The binary64-BLAS accumulators (used for full-size parity) equal exact
+    integer sums: brute-force Python loops on 8 x 8 x 128, and at K = 65536
+    with extreme codes, where sums reach 127^2 K ~ 1.06e9 (a binary32 product
+    would round there: 2^24 < 1.06e9)."""
+    rng = np.random.default_rng(23)
+    for bits in (4, 6, 8):
+        qm = O.QMAX[bits]
+        a = rng.integers(-qm, qm + 1, size=(8, 128)).astype(np.int8)
+        w = rng.integers(-qm, qm + 1, size=(8, 128)).astype(np.int8)
+        want = [[sum(int(a[m, k]) * int(w[n, k]) for k in range(128)) for n in range(8)]
+                for m in range(8)]
+        assert o.int_gemm_f64(a, w).tolist() == want
+    K = 65536
+    a = np.full((4, K), 127, np.int8)
+    a[1] = -127
+    a[2, ::2] = -127
+    a[3, :K // 2] = 1  # small terms first, then large ones
+    w = np.full((3, K), -127, np.int8)
+    w[1] = 127
+    w[2, 1::2] = 1
+
+    def exact(m, n):
+        # rows and columns are periodic in k with period 2, except row 3,
+        # whose halves differ: count the (a, w) value pairs and multiply out
+        s = 0
+        for half in (0, 1):
+            for par in (0, 1):
+                k = half * (K // 2) + par
+                s += (K // 4) * int(a[m, k]) * int(w[n, k])
+        return s
+
+    want = [[exact(m, n) for n in range(3)] for m in range(4)]
+    got = o.int_gemm_f64(a, w)
+    assert got.tolist() == want
+    assert np.abs(got).max() > 2 ** 24
+
+
 # --------------------------------------------------------------------------- epilogue / bf16
 
 def pin_bf16_rounding_matches_torch(o=O):
