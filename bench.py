@@ -78,9 +78,18 @@ def peaks():
 # the shared helpers): counters taken on other sources are not reported
 KERNEL_SOURCES = {
     "qgemm_kernel": ("qs_gemm.cuh", "qs_host.cuh", "qs_ptx.cuh"),
+    "qgemm_ta_kernel": ("qs_gemm.cuh", "qs_gemm_ta.cuh", "qs_host.cuh", "qs_ptx.cuh"),
     "rotate_quant_kernel": ("qs_host.cuh", "qs_ptx.cuh", "qs_quant.cuh"),
 }
-HEADLINE_SOURCES = ("qs_gemm.cuh", "qs_host.cuh", "qs_ptx.cuh", "qs_quant.cuh")
+HEADLINE_SOURCES = ("qs_gemm.cuh", "qs_gemm_ta.cuh", "qs_host.cuh", "qs_ptx.cuh", "qs_quant.cuh")
+
+
+def gemm_kernel(sx: int, sw: int) -> tuple[str, str]:
+    """(kernel family as keyed in the ncu record, instantiation) of the GEMM
+    that the storage widths sx (activations) and sw (weights) run."""
+    if sx == 4 and sw == 4:
+        return "qgemm_ta_kernel", "qgemm_ta_kernel<false,false> (tcgen05 kind::i8, A in TMEM)"
+    return "qgemm_kernel", f"qgemm_kernel<{sx},{sw},false,false> (tcgen05 kind::i8)"
 
 
 def source_hash(names, read=None) -> str:
@@ -928,17 +937,19 @@ def main():
         quant_bytes = M * (2 * K + K * bx // 8 + 4)
         stored_bytes = M * (2 * K + qs.packed_cols(K, bx, x_flags) + 4)
         traffic_key = cfg.name + ("_act_codes_in_bytes" if x_flags else "")
+        headline_fam, headline_inst = gemm_kernel(4 if sx == 4 else 8, 4 if bits == 4 else 8)
         quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
         for name, L in layouts.items():
             key = cfg.name + ("_act_codes_in_bytes" if L["x_flags"] else "")
             g_tops = ops_per_step / (L["gemm_ms"] * 1e-3) / 1e12
             q_gbs = quant_bytes / (L["quant_ms"] * 1e-3) / 1e9
+            fam, inst = gemm_kernel(8 if L["x_flags"] else 4, 4 if bits == 4 else 8)
             L.update({
                 "TOPS": ops_per_step * world / (L["step_ms"] * 1e-3) / 1e12,
                 "tokens_per_s": M * world / (L["step_ms"] * 1e-3),
                 "gemm_TOPS": g_tops, "gemm_frac_int8_peak": g_tops / int8_peak,
-                "gemm_kernel": f"qgemm_kernel<{8 if L['x_flags'] else 4},{bits},false,false>",
-                "gemm_traffic": ncu_traffic(key, "qgemm_kernel"),
+                "gemm_kernel": inst,
+                "gemm_traffic": ncu_traffic(key, fam),
                 "quant_GBps": q_gbs, "quant_frac_hbm": q_gbs / pk["hbm_gbs"],
                 "quant_stored_bytes": M * (2 * K + qs.packed_cols(K, bx, L["x_flags"]) + 4),
                 "quant_traffic": ncu_traffic(key, "rotate_quant_kernel")})
@@ -956,9 +967,8 @@ def main():
                        "l2": "inputs larger than L2 (x 335 MB, out 906 MB bf16); no flush"},
             "roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak,
                          "unit": UNIT, "frac": gemm_tops / int8_peak,
-                         "traffic": ncu_traffic(traffic_key, "qgemm_kernel"),
-                         "kernel": f"qgemm_kernel<{4 if sx == 4 else 8},{4 if bits == 4 else 8},"
-                                   f"false,false> (tcgen05 kind::i8)",
+                         "traffic": ncu_traffic(traffic_key, headline_fam),
+                         "kernel": headline_inst,
                          "peak_source": f"{src}: bf16_tflops (burst) x {INT8_PER_BF16} "
                                         f"nominal int8:bf16"},
             "roofline_quant": {"bound": "hbm", "achieved": quant_gbs, "peak": pk["hbm_gbs"],

@@ -19,6 +19,9 @@ Cases:
   gemm_w4a8       qs_qlinear_mixed, 8-bit activations, 4-bit weights
   gemm_bgr        qs_qlinear_asym, 4-bit activations with code sums, 4-bit weights on
                   bounded (asymmetric) grids
+  quant           qs_quant_act at any shape and width (--K, --bits, --alpha, --byte-codes)
+  gemm            qs_qlinear_mixed at any shape and widths (--K, --N, --bits-x, --bits-w,
+                  --byte-codes: 4-bit activation codes stored one per byte)
 """
 
 from __future__ import annotations
@@ -44,8 +47,15 @@ def main(argv=None) -> None:
     p = argparse.ArgumentParser()
     p.add_argument("case", choices=["sd4_gemm_e4m3", "sd4_gemm_codes", "sd4_quant_e4m3",
                                     "gbs_update", "gelu", "gemm_w8a8", "gemm_w4a8",
-                                    "gemm_bgr"])
+                                    "gemm_bgr", "quant", "gemm"])
     p.add_argument("--tokens", type=int, default=None)
+    p.add_argument("--K", type=int, default=K)
+    p.add_argument("--N", type=int, default=N)
+    p.add_argument("--bits", type=int, default=4)
+    p.add_argument("--bits-x", type=int, default=4)
+    p.add_argument("--bits-w", type=int, default=4)
+    p.add_argument("--alpha", type=float, default=1.0)
+    p.add_argument("--byte-codes", action="store_true")
     a = p.parse_args(argv)
     qs.load()
     torch.cuda.init()
@@ -80,6 +90,28 @@ def main(argv=None) -> None:
             xp, xs = qs.quant_act(x, 8)
             wp, ws = qs.pack_weights(w, bits_w)
             run = lambda: qs.qlinear(xp, xs, wp, ws, b, 8, K, out=out, bits_w=bits_w)  # noqa: E731
+    elif a.case == "quant":
+        M = a.tokens or 16384
+        g = torch.Generator(device="cuda").manual_seed(0)
+        x = torch.randn(M, a.K, device="cuda", generator=g).to(torch.bfloat16)
+        flags = qs.QS_FLAG_BYTE_CODES if a.byte_codes else 0
+        xp = torch.empty((M, qs.packed_cols(a.K, a.bits, flags)), dtype=torch.uint8,
+                         device="cuda")
+        xs = torch.empty((M,), dtype=torch.float32, device="cuda")
+        run = lambda: qs.qs_quant_act(x, M, a.K, a.bits, a.alpha, flags, xp, xs)  # noqa: E731
+    elif a.case == "gemm":
+        M = a.tokens or 16384
+        g = torch.Generator(device="cuda").manual_seed(0)
+        x = torch.randn(M, a.K, device="cuda", generator=g).to(torch.bfloat16)
+        w = (torch.randn(a.N, a.K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+        b = (torch.randn(a.N, device="cuda", generator=g) * 0.01).to(torch.bfloat16)
+        flags = qs.QS_FLAG_BYTE_CODES if a.byte_codes else 0
+        xp, xs = qs.quant_act(x, a.bits_x, a.alpha, flags)
+        wp, ws = qs.pack_weights(w, a.bits_w)
+        sx = qs.storage_bits(a.bits_x, flags)
+        out = torch.empty((M, a.N), dtype=torch.bfloat16, device="cuda")
+        run = lambda: qs.qs_qlinear_mixed(xp, xs, sx, wp, ws, a.bits_w, b, M, a.N, a.K,  # noqa: E731
+                                          out)
     elif a.case == "gelu":
         M = a.tokens or 4096
         g = torch.Generator(device="cuda").manual_seed(2)
