@@ -78,17 +78,14 @@ def peaks():
 # the shared helpers): counters taken on other sources are not reported
 KERNEL_SOURCES = {
     "qgemm_kernel": ("qs_gemm.cuh", "qs_host.cuh", "qs_ptx.cuh"),
-    "qgemm_ta_kernel": ("qs_gemm.cuh", "qs_gemm_ta.cuh", "qs_host.cuh", "qs_ptx.cuh"),
     "rotate_quant_kernel": ("qs_host.cuh", "qs_ptx.cuh", "qs_quant.cuh"),
 }
-HEADLINE_SOURCES = ("qs_gemm.cuh", "qs_gemm_ta.cuh", "qs_host.cuh", "qs_ptx.cuh", "qs_quant.cuh")
+HEADLINE_SOURCES = ("qs_gemm.cuh", "qs_host.cuh", "qs_ptx.cuh", "qs_quant.cuh")
 
 
 def gemm_kernel(sx: int, sw: int) -> tuple[str, str]:
     """(kernel family as keyed in the ncu record, instantiation) of the GEMM
     that the storage widths sx (activations) and sw (weights) run."""
-    if sx == 4 and sw == 4:
-        return "qgemm_ta_kernel", "qgemm_ta_kernel<false,false> (tcgen05 kind::i8, A in TMEM)"
     return "qgemm_kernel", f"qgemm_kernel<{sx},{sw},false,false> (tcgen05 kind::i8)"
 
 

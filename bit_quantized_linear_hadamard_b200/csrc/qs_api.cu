@@ -14,7 +14,6 @@
 #include "qs_bgr.cuh"
 #include "qs_gbs.cuh"
 #include "qs_gemm.cuh"
-#include "qs_gemm_ta.cuh"
 #include "qs_host.cuh"
 #include "qs_glue.cuh"
 #include "qs_quant.cuh"
@@ -530,9 +529,9 @@ qs_status qs_qlinear_asym(const void* x_packed, const float* x_scale, const int3
     QS_TRY(check_device_ptr(p));
   if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return bits == 4 ? qs::gemm_ta::launch_qgemm_ta<false, true>(
-                         x_packed, x_scale, w_packed, w_scale, bias_bf16, M, N, K, out_bf16, s,
-                         nullptr, 0, x_rowsum, w_offset)
+  return bits == 4 ? launch_qgemm<4, 4, false, true>(x_packed, x_scale, w_packed, w_scale,
+                                                      bias_bf16, M, N, K, out_bf16, s, nullptr, 0,
+                                                      x_rowsum, w_offset)
                    : launch_qgemm<8, 8, false, true>(x_packed, x_scale, w_packed, w_scale,
                                                       bias_bf16, M, N, K, out_bf16, s, nullptr, 0,
                                                       x_rowsum, w_offset);
@@ -549,9 +548,9 @@ qs_status qs_qgemm_s32_asym(const void* x_packed, const int32_t* x_rowsum, const
                         static_cast<const void*>(w_offset), static_cast<const void*>(acc)})
     QS_TRY(check_device_ptr(p));
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return bits == 4 ? qs::gemm_ta::launch_qgemm_ta<true, true>(x_packed, nullptr, w_packed,
-                                                               nullptr, nullptr, M, N, K, acc, s,
-                                                               nullptr, 0, x_rowsum, w_offset)
+  return bits == 4 ? launch_qgemm<4, 4, true, true>(x_packed, nullptr, w_packed, nullptr, nullptr,
+                                                     M, N, K, acc, s, nullptr, 0, x_rowsum,
+                                                     w_offset)
                    : launch_qgemm<8, 8, true, true>(x_packed, nullptr, w_packed, nullptr, nullptr,
                                                      M, N, K, acc, s, nullptr, 0, x_rowsum,
                                                      w_offset);

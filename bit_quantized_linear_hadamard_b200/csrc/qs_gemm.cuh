@@ -620,5 +620,21 @@ inline qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, c
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
+template <bool OUT_S32>
+inline qs_status dispatch_qgemm(int bits_x, int bits_w, const void* xp, const float* sa,
+                                const void* wp,
+                         const float* sw, const void* bias, int64_t M, int64_t N, int64_t K,
+                         void* out, cudaStream_t stream) {
+  // storage per code: 4-bit codes in nibbles, 6- and 8-bit codes in bytes
+  const int sx = bits_x == 4 ? 4 : 8, sww = bits_w == 4 ? 4 : 8;
+  if (sx == 4 && sww == 4)
+    return launch_qgemm<4, 4, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
+  if (sx == 8 && sww == 8)
+    return launch_qgemm<8, 8, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
+  if (sx == 8 && sww == 4)
+    return launch_qgemm<8, 4, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
+  return launch_qgemm<4, 8, OUT_S32>(xp, sa, wp, sw, bias, M, N, K, out, stream);
+}
+
 }  // namespace gemm
 }  // namespace qs

@@ -42,24 +42,6 @@ inline bool make_tensor_map_2d(CUtensorMap* map, const void* base, uint64_t row_
   return r == CUDA_SUCCESS;
 }
 
-// Byte tensor [rows][row_bytes] with a box of [box_rows][64 bytes] stored with
-// the 64-byte swizzle: 16-byte chunk j of box row r lands at chunk
-// j ^ ((r >> 1) & 3) of that row (the destination is 512-byte aligned).
-inline bool make_tensor_map_2d_sw64(CUtensorMap* map, const void* base, uint64_t row_bytes,
-                                    uint64_t rows, uint32_t box_rows) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {row_bytes, rows};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {64, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
-                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 inline int sm_count() {
   static int cached[64] = {0};
   int dev = 0;
