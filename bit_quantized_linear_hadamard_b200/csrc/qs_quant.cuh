@@ -42,6 +42,10 @@ __host__ __device__ constexpr int code_qmax(int bits) { return (1 << (bits - 1))
 __host__ __device__ constexpr int code_storage_bits(int bits) { return bits == 4 ? 4 : 8; }
 
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+// Depth of the activation kernel's shared-memory ring (rows of up to 128
+// Hadamard blocks): two stages measured faster than three or four, which cost
+// resident CTAs (the kernel is latency-bound and more warps per SM win).
+constexpr int kQuantStages = 2;
 constexpr float kZeroRowT = 0x1p-120f;
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
@@ -257,12 +261,33 @@ __global__ void __launch_bounds__(256) rotate_quant_tma_kernel(
     }
   }
 
+  // Stage, phase and row-maximum buffer of group number `it`.  The launcher
+  // uses a ring of two stages.  The packed (two codes per byte) instantiation
+  // advances them as counters, the others derive them from `it`: with
+  // identical outputs, each form measured the faster one for its
+  // instantiation (packed W4 at the Wan FFN shape 96.4 -> 94.4 us; the
+  // byte-code and 8-bit ones 98.6 -> 106 us with counters).
   int it = 0;
+  int s_ctr = 0, rb_ctr = 0;
+  uint32_t ph_ctr = 0;
   for (int64_t g = blockIdx.x; g < num_groups; g += gridDim.x, ++it) {
-    const int s = it % stages;
-    const uint32_t ph = static_cast<uint32_t>(it / stages) & 1u;
-    const int rb = it % 3;
-    if (tid < rpc) row_amax[(it + 1) % 3][tid] = 0u;  // last read two groups ago
+    int s, rb;
+    uint32_t ph;
+    if constexpr (STORE == 4) {
+      static_assert(kQuantStages == 2, "the counters below step a ring of two stages");
+      s = s_ctr;
+      ph = ph_ctr;
+      rb = rb_ctr;
+      ph_ctr ^= static_cast<uint32_t>(s_ctr);
+      s_ctr ^= 1;
+      rb_ctr = rb_ctr == 2 ? 0 : rb_ctr + 1;
+      if (tid < rpc) row_amax[rb_ctr][tid] = 0u;  // last read two groups ago
+    } else {
+      s = it % stages;
+      ph = static_cast<uint32_t>(it / stages) & 1u;
+      rb = it % 3;
+      if (tid < rpc) row_amax[(it + 1) % 3][tid] = 0u;  // last read two groups ago
+    }
     mbar_wait_bounded(bars + 8 * s, ph, &abort_flag, kErrWaitTma);
 
     const int64_t row = g * rpc + rl;
@@ -574,9 +599,7 @@ inline cudaError_t launch_rotate_quant_bits(const uint16_t* x, int64_t rows, int
   if (nblk <= 128 && groups * (static_cast<int64_t>(rpc) * K / 64) < (int64_t{1} << 31)) {
     const int threads = (rpc * 2 * nblk + 31) / 32 * 32;
     const int stage_stride = (rpc * K * 2 + 1023) / 1024 * 1024;
-    // Two stages: measured faster than three or four, which cost resident CTAs
-    // (the kernel is latency-bound and more warps per SM win).
-    const int stages = 2;
+    const int stages = kQuantStages;
     const int smem = stages * stage_stride + 8 * stages + 1024;
     CUtensorMap tmx;
     if (!make_tensor_map_2d(&tmx, x, 64, static_cast<uint64_t>(rows) * K / 64, 64, rpc * K / 64,
