@@ -127,6 +127,16 @@ def ncu_traffic(workload: str, kernel: str):
     return None if k is None else k.get("dram_bytes_per_launch_full")
 
 
+def workload_line_config(cfg, act_codes: str, world: int, M: int | None = None) -> dict:
+    """The `config` object of a bench line: the same keys and values for this
+    library's arm and the oracle arm of one workload."""
+    return {"workload": cfg.name, "M": cfg.M if M is None else M, "K": cfg.K, "N": cfg.N,
+            "bits_w": cfg.bits, "bits_x": cfg.act_bits, "alpha": cfg.alpha,
+            "act_codes": act_codes if cfg.act_bits == 4 else "bytes",
+            "seed": cfg.seed, "parallelism": f"replicas{world}",
+            "l2": "inputs larger than L2 (x 335 MB, out 906 MB bf16); no flush"}
+
+
 def workload_config(I, name):
     """The Wan-14B FFN up-projection config the step runs (W4A4 by default)."""
     table = {"w4a4": I.WAN_FFN, "w8a8": I.WAN_FFN_W8, "w4a8": I.WAN_FFN_W4A8,
@@ -733,11 +743,7 @@ def run_reference(args, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int4" if cfg.act_bits == cfg.bits == 4 else f"int{cfg.bits}w-int{cfg.act_bits}a",
         "data": "synthetic",
-        "config": {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "bits_w": cfg.bits,
-                   "bits_x": cfg.act_bits, "alpha": cfg.alpha,
-                   "act_codes": args.act_codes if cfg.act_bits == 4 else "packed",
-                   "seed": cfg.seed, "parallelism": f"replicas{world}",
-                   "sample_rows_per_step": rows // args.steps},
+        "config": workload_line_config(cfg, args.act_codes, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": pool.procs, "kind": "oracle",
                          "host": host_info(),
                          "sample": f"{rows // args.steps} tokens per step ({rows_per_proc} per "
@@ -957,11 +963,7 @@ def main():
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "data": "synthetic",
             "dtype": "int4" if bx == bits == 4 else f"int{bits}w-int{bx}a",
-            "config": {"workload": cfg.name, "M": M, "K": K, "N": N, "bits_w": bits,
-                       "bits_x": bx, "alpha": alpha,
-                       "act_codes": "bytes" if x_flags else "packed",
-                       "seed": cfg.seed, "parallelism": f"replicas{world}",
-                       "l2": "inputs larger than L2 (x 335 MB, out 906 MB bf16); no flush"},
+            "config": workload_line_config(cfg, "bytes" if x_flags else "packed", world, M=M),
             "roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak,
                          "unit": UNIT, "frac": gemm_tops / int8_peak,
                          "traffic": ncu_traffic(traffic_key, headline_fam),
