@@ -177,9 +177,13 @@ def code_rowsums(qa: np.ndarray) -> np.ndarray:
     return np.asarray(qa, dtype=np.int64).sum(axis=1)
 
 
-def asym_accumulators(qa: np.ndarray, s: np.ndarray, offset: np.ndarray) -> np.ndarray:
-    """acc[m, n] = sum_k q_a[m,k] s[n,k] + o[n] sum_k q_a[m,k]  (= sum q_a (q - z))."""
-    acc = int_gemm(qa, s) + code_rowsums(qa)[:, None] * np.asarray(offset, np.int64)[None, :]
+def asym_accumulators(qa: np.ndarray, s: np.ndarray, offset: np.ndarray,
+                      gemm=int_gemm) -> np.ndarray:
+    """acc[m, n] = sum_k q_a[m,k] s[n,k] + o[n] sum_k q_a[m,k]  (= sum q_a (q - z)).
+
+    `gemm`: the exact integer product (int_gemm, or int_gemm_f64 -- exact by
+    the 2^53 bound it checks -- for full-size operands)."""
+    acc = gemm(qa, s) + code_rowsums(qa)[:, None] * np.asarray(offset, np.int64)[None, :]
     if np.abs(acc).max(initial=0) >= 2 ** 31:
         raise OverflowError("accumulator exceeds int32")
     return acc

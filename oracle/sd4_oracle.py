@@ -179,16 +179,25 @@ def linear_sd4(x_bits, w_bits, bias_bits=None, exact: bool = True):
     cx, ex, dx = quantize_rows(x_bits)
     cw, ew, dw = quantize_rows(w_bits)
     xh, wh = dequantize(cx, ex, dx), dequantize(cw, ew, dw)
-    if exact:
-        y = np.array([[float(v) for v in row] for row in exact_products(xh, wh)])
-    else:
-        y = xh @ wh.T
-    y32 = y.astype(np.float32)
-    b = (np.zeros(wh.shape[0], np.float32) if bias_bits is None
-         else bf16_bits_to_f32(np.asarray(bias_bits)))
-    out = f32_to_bf16_bits((y32 + b[None, :]).astype(np.float32))
+    y, out = layer_outputs(xh, wh, bias_bits, exact)
     return {"codes_x": cx, "exp_x": ex, "dia_x": dx, "codes_w": cw, "exp_w": ew, "dia_w": dw,
             "x_hat": xh, "w_hat": wh, "y": y, "out": out}
+
+
+def layer_outputs(x_hat, w_hat, bias_bits=None, exact: bool = True):
+    """The layer's last steps on decoded operands: y = sum_k x_hat w_hat (exact
+    rationals, or binary64 when not `exact`) and out = bf16_rne(fl(fl32(y) +
+    bias)) as bf16 bits."""
+    N = w_hat.shape[0]
+    if len(x_hat) == 0:
+        y = np.zeros((0, N))
+    elif exact:
+        y = np.array([[float(v) for v in row] for row in exact_products(x_hat, w_hat)])
+    else:
+        y = x_hat @ w_hat.T
+    b = (np.zeros(N, np.float32) if bias_bits is None
+         else bf16_bits_to_f32(np.asarray(bias_bits)))
+    return y, f32_to_bf16_bits((y.astype(np.float32) + b[None, :]).astype(np.float32))
 
 
 def decompose_rows(x_bits, rows):
@@ -225,18 +234,11 @@ def linear_sd4_decomp(x_bits, w_bits, bias_bits, rows, exact: bool = True):
     rows = np.asarray(rows, np.int64)
     dec = decompose_rows(x_bits, rows)
     xt = dec["x_hat"] + dec["d_hat"]
-    if len(rows) == 0:
-        y = np.zeros((0, r["w_hat"].shape[0]))
-    elif exact:
-        y = np.array([[float(v) for v in row] for row in exact_products(xt, r["w_hat"])])
-    else:
-        y = xt @ r["w_hat"].T
-    b = (np.zeros(r["w_hat"].shape[0], np.float32) if bias_bits is None
-         else bf16_bits_to_f32(np.asarray(bias_bits)))
+    y, o = layer_outputs(xt, r["w_hat"], bias_bits, exact)
     out = r["out"].copy()
     yrows = r["y"].copy()
     if len(rows):
-        out[rows] = f32_to_bf16_bits((y.astype(np.float32) + b[None, :]).astype(np.float32))
+        out[rows] = o
         yrows[rows] = y
     r.update({"decomp": dec, "out": out, "y": yrows, "x_tilde": xt, "rows": rows})
     return r

@@ -144,25 +144,3 @@ def test_linear_bgr_one_call(bits):
                      bits, ws, need, out)
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), g["out"].view(torch.int16))
-
-
-@pytest.mark.slow
-def test_full_size_bgr_sampled():
-    cfg = I.WAN_FFN
-    d = I.make_layer(cfg)
-    g = run_bgr_layer(d, cfg.bits, cfg.alpha)
-    rng = np.random.default_rng(21)
-    rows = np.unique(np.concatenate([[0, cfg.M - 1], rng.choice(cfg.M, 40, replace=False)]))
-    cols = np.unique(np.concatenate([[0, cfg.N - 1], rng.choice(cfg.N, 40, replace=False)]))
-    xb, wb, bb = bits16(d["x"][rows]), bits16(d["w"][cols]), bits16(d["bias"][cols])
-    qa, sa = O.quant_act(xb, cfg.bits, cfg.alpha)
-    s, sw, off = B.pack_weights_bgr(wb, cfg.bits, J, T)
-    assert np.array_equal(g["wp"].cpu().numpy()[cols], O.pack(s, cfg.bits))
-    assert np.array_equal(g["ws"].cpu().numpy()[cols].view(np.uint32), sw.view(np.uint32))
-    assert np.array_equal(g["wo"].cpu().numpy()[cols], off)
-    assert np.array_equal(g["xr"].cpu().numpy()[rows].astype(np.int64), B.code_rowsums(qa))
-    acc = B.asym_accumulators(qa, s, off)
-    assert np.array_equal(g["acc"].cpu().numpy()[np.ix_(rows, cols)].astype(np.int64), acc)
-    out = O.epilogue(acc, sa, sw, bb)
-    got = g["out"].view(torch.int16).cpu().numpy().view(np.uint16)[np.ix_(rows, cols)]
-    assert np.array_equal(got, out)

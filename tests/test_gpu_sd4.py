@@ -356,74 +356,6 @@ def test_sd4_linear_decomp_single_row_no_bias_and_forms_agree():
     assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
 
 
-@pytest.mark.slow
-def test_full_size_wan_ffn_decomp_sampled():
-    """The Wan FFN layer (32760 x 5120 -> 13824) with 1/16 of the tokens
-    decomposed, in the e4m3-weight form the benchmark times; sampled outputs
-    of salient and plain rows against the oracle."""
-    cfg = I.WAN_FFN
-    d = I.make_layer(cfg)
-    M, K, N = cfg.M, cfg.K, cfg.N
-    rows = I.salient_rows(M, seed=cfg.seed)
-    x, w, b = d["x"].cuda(), d["w"].cuda(), d["bias"].cuda()
-    cx, mx = qs.sd4_quant(x)
-    cw, mw = qs.sd4_quant(w)
-    w8 = qs.sd4_decode_e4m3(cw, mw)
-    rt = _rows_tensor(rows)
-    codes2, meta2 = qs.sd4_quant_decomp(x, rt)
-    out = qs.sd4_linear_decomp(cx, mx, codes2, meta2, rt, None, mw, b, K, w_e4m3=w8)
-    torch.cuda.synchronize()
-    rng = np.random.default_rng(4)
-    pick_s = np.unique(np.concatenate([[0, len(rows) - 1], rng.choice(len(rows), 24, replace=False)]))
-    srows = np.asarray(rows)[pick_s]
-    others = np.setdiff1d(rng.choice(M, 40, replace=False), rows)[:16]
-    cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 40, replace=False)]))
-    wb, bb = I.bf16_bits(d["w"][cols]), I.bf16_bits(d["bias"][cols])
-    mrows = np.concatenate([srows, others])
-    xb = I.bf16_bits(d["x"][mrows])
-    sub = {"x": d["x"][mrows], "w": d["w"][cols], "bias": d["bias"][cols]}
-    got = out[torch.from_numpy(mrows).cuda()][:, torch.from_numpy(cols).cuda()]
-    _check_decomp_layer(sub, got, list(range(len(srows))), K)
-    assert np.array_equal(codes2[torch.from_numpy(pick_s).cuda()].cpu().numpy(),
-                          S.pack_decomp(S.decompose_rows(xb[:len(srows)], range(len(srows))))[0])
-
-
-@pytest.mark.slow
-def test_full_size_wan_ffn_e4m3_layer_sampled():
-    """The SD4 layer the benchmark times (Wan FFN, 32760 x 5120 -> 13824): e4m3
-    activations and weights; bit-identical to the codes form everywhere, and
-    sampled outputs against the oracle."""
-    cfg = I.WAN_FFN
-    d = I.make_layer(cfg)
-    M, K, N = cfg.M, cfg.K, cfg.N
-    x, w, b = d["x"].cuda(), d["w"].cuda(), d["bias"].cuda()
-    cx, mx = qs.sd4_quant(x)
-    cw, mw = qs.sd4_quant(w)
-    x8, mx8 = qs.sd4_quant_e4m3(x)
-    w8 = qs.sd4_decode_e4m3(cw, mw)
-    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    out8 = torch.empty_like(out)
-    qs.qs_sd4_linear(cx, mx, cw, mw, b, M, N, K, out)
-    qs.qs_sd4_linear_e4m3(x8, mx8, w8, mw, b, M, N, K, out8)
-    torch.cuda.synchronize()
-    assert torch.equal(mx8, mx)
-    assert torch.equal(out.view(torch.int16), out8.view(torch.int16))
-    rng = np.random.default_rng(6)
-    rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, 40, replace=False)]))
-    cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 40, replace=False)]))
-    sub = {"x": d["x"][rows], "w": d["w"][cols], "bias": d["bias"][cols]}
-    got = out8[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()]
-    r = S.linear_sd4(I.bf16_bits(sub["x"]), I.bf16_bits(sub["w"]), I.bf16_bits(sub["bias"]),
-                     exact=False)
-    got_bits = got.view(torch.int16).cpu().numpy().view(np.uint16)
-    gotf = O.bf16_bits_to_f32(got_bits).astype(np.float64)
-    S_abs = np.abs(r["x_hat"]) @ np.abs(r["w_hat"]).T
-    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(gotf), 2.0 ** -126))) - 7)
-    exact_y = r["y"] + O.bf16_bits_to_f32(I.bf16_bits(sub["bias"])).astype(np.float64)
-    assert (np.abs(gotf - exact_y) <= K * 2.0 ** -23 * S_abs + ulp).all()
-    assert float((got_bits == r["out"]).mean()) > 0.99
-
-
 def test_sd4_output_only_16_byte_aligned():
     """16-byte (not 32-byte) aligned outputs take the 16-byte store path."""
     M, N, K = 200, 400, 512
