@@ -6,27 +6,33 @@
 //   out[m][n] = bf16(fl(fl(fl(s_a[m] * s_w[n]) * float(acc)) + bias[n]))
 //
 // Structure: a persistent kernel launched as clusters of two CTAs on the two
-// SMs of a TPC.  Each pair walks output tiles of 256 x 256 (n fastest, so the
+// SMs of a TPC.  Each pair walks output tiles of 256 x 512 (n fastest, so the
 // whole packed weight stays in L2 while activation tiles stream once; the
 // 8-bit weight of the 8x8 form is twice as large and is walked in bands of
-// N-tiles instead, see kBandN).  CTA r
-// of the pair holds rows [128r, 128r+128) of the x tile and rows
-// [128r, 128r+128) of the W tile; the leader (r = 0) issues one
-// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 32) per 32-deep K step, which
-// reads the x rows and W rows of both CTAs and accumulates each CTA's 128 x 256
-// result in that CTA's tensor memory.  Per SM this halves the W operand traffic
-// of a 128 x 256 single-CTA tile at the same MMA work.
+// N-tiles instead, see kBandN).  CTA r of the pair holds rows [128r, 128r+128)
+// of the x tile and, for each N-half h of the tile, rows
+// [256h + 128r, 256h + 128r + 128) of the W tile; the leader (r = 0) issues
+// per 32-deep K step two tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 32),
+// one per N-half, both reading the same x rows of both CTAs; each CTA's
+// 128 x 512 result accumulates in that CTA's tensor memory.  Per SM this
+// halves the W operand traffic of a single-CTA tile at the same MMA work, and
+// the two N-halves share one x tile: one widening of a 4-bit x tile, one set
+// of stage barriers and one TMA load of x serve twice the multiply-adds of a
+// 256 x 256 tile.  (Measured: with the operand traffic of a 256 x 256 tile,
+// issuing twice the MMAs per stage took 1.33x the time, at the tensor pipe's
+// full rate; the smaller tile left it idle a third of its cycles.)
 //
 // Warp roles (both CTAs):
 //   warp 0      TMA producer
 //   warp 1      TMEM allocation; in the leader the single-thread MMA issuer;
 //               in the other CTA (4-bit only) the relay that tells the leader
 //               that this CTA's operand tiles are ready
-//   warps 2-5   epilogue: tcgen05.ld of this CTA's accumulator rows, scale,
-//               bias, bf16 store
-//   warps 6-9   (4-bit only) widen packed nibbles into the 8-bit operand tiles
-// Two 256-column int32 accumulators (all 512 TMEM columns) let the epilogue of
-// one tile run under the main loop of the next.
+//   warps 2-9   epilogue: tcgen05.ld of this CTA's accumulator rows, scale,
+//               bias, bf16 store; warps 2-5 the first N-half, 6-9 the second
+//   warps 10-13 (4-bit only) widen packed nibbles into the 8-bit operand tiles
+// The 128 x 512 int32 accumulator fills the 512 TMEM columns, so the MMA of
+// the next tile waits for the epilogue to drain it; the operand ring keeps
+// filling meanwhile.
 //
 // Synchronisation across the pair: 8-bit operand stages are "full" on the
 // leader's barrier when the TMA loads of both CTAs have landed.  4-bit operand
@@ -76,11 +82,12 @@ namespace qs {
 namespace gemm {
 
 constexpr int BM = 256;  // tile rows (tokens), 128 per CTA
-constexpr int BN = 256;  // tile columns (output channels), 128 W rows per CTA
+constexpr int BN = 512;  // tile columns (output channels): two MMA halves
+constexpr int NH = 256;  // columns of one MMA (an N-half of the tile)
 constexpr int HM = 128;  // x rows per CTA
-constexpr int HN = 128;  // W rows per CTA
+constexpr int HN = 128;  // W rows per CTA and N-half
 constexpr int BK = 128;  // K elements per pipeline stage (= 128 bytes of 8-bit operand)
-constexpr int kTmemCols = 2 * BN;
+constexpr int kTmemCols = BN;  // one 512-column int32 accumulator: all of tensor memory
 
 // SA, SB: storage bits of the x and W codes (4 = two per byte, 8 = one byte).
 template <int SA, int SB>
@@ -92,17 +99,17 @@ struct Cfg {
   static constexpr bool kAllPacked = kPackedA && kPackedB;
   static constexpr bool kDirect = !kAllPacked;            // some operand goes by TMA directly
   static constexpr int kPkBytesA = kPackedA ? HM * BK / 2 : 0;  // packed tile of x (this CTA)
-  static constexpr int kPkBytesB = kPackedB ? HN * BK / 2 : 0;  // packed tile of W (this CTA)
+  static constexpr int kPkBytesB = kPackedB ? 2 * HN * BK / 2 : 0;  // packed W, both halves
   static constexpr int kOpBytesA = HM * BK;      // 8-bit operand tile of x
-  static constexpr int kOpBytesB = HN * BK;      // 8-bit operand tile of W
+  static constexpr int kOpBytesB = 2 * HN * BK;  // 8-bit operand tiles of W, both halves
   static constexpr int kPkStage = kPkBytesA + kPkBytesB;
   static constexpr int kOpStage = kOpBytesA + kOpBytesB;
   // bytes the TMA writes straight into one operand stage of this CTA
   static constexpr int kDirectBytes = (kPackedA ? 0 : kOpBytesA) + (kPackedB ? 0 : kOpBytesB);
-  // 4/4 and 8/8 sized by measurement; mixed: as many stages as fit
-  static constexpr int kOpStages = kAllPacked ? 4 : (kPacked ? 5 : 6);
+  // as many stages as fit in shared memory
+  static constexpr int kOpStages = kPacked ? 3 : 4;
   static constexpr int kPkStages = kPacked ? kOpStages : 0;  // one ring index drives both
-  static constexpr int kEpiWarps = 4;
+  static constexpr int kEpiWarps = 8;  // two per TMEM lane quarter: one per N-half
   static constexpr int kUnpackWarps = kPacked ? 4 : 0;
   // operand-tile row that packed row 0 widens into (W rows follow the 128 x rows)
   static constexpr int kUnpackRow0 = kPackedA ? 0 : HM;
@@ -128,6 +135,7 @@ struct Cfg {
   static constexpr int kOpFullTx = 2 * kDirectBytes + (kPacked ? 16 : 0);
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
   static constexpr int kAccEmptyCount = 2 * kEpiWarps;
+  static constexpr int kEpiThreads = 32 * kEpiWarps;
 };
 
 struct Smem {
@@ -147,12 +155,12 @@ struct Smem {
 
 // Tile order of the 8-bit x 8-bit instantiation: bands of kBandN N-tiles,
 // M advancing inside a band, so that the band's slice of the 8-bit weight
-// (18 x 256 rows, 23.6 MB at K = 5120) stays in L2 while the activation tiles
+// (9 x 512 rows, 23.6 MB at K = 5120) stays in L2 while the activation tiles
 // stream.  In n-fastest order the whole 70.8 MB weight of the Wan FFN was read
-// from DRAM about 19 times per launch; banded, the launch measured 5-10 %
+// from DRAM many times per launch; banded, the launch measured 5-10 %
 // faster.  The other instantiations, whose packed 4-bit weight fits in L2,
 // keep the n-fastest order.
-constexpr int kBandN = 18;
+constexpr int kBandN = 9;
 
 struct Problem {
   int M, N, K;
@@ -194,7 +202,10 @@ __device__ __forceinline__ void producer_role(const Smem& sm, const Problem& pb,
         mbar_arrive_expect_tx(sm.pk_full(s), C::kPkStage);
         if (C::kPackedA) tma_load_2d(dst, tmA, kb * (BK / 2), m0 + roff, sm.pk_full(s));
         if (C::kPackedB)
-          tma_load_2d(dst + C::kPkBytesA, tmB, kb * (BK / 2), n0 + roff, sm.pk_full(s));
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d(dst + C::kPkBytesA + h * (HN * BK / 2), tmB, kb * (BK / 2),
+                        n0 + h * NH + roff, sm.pk_full(s));
       }
       if (C::kDirect) {
         // direct operand tiles of both CTAs complete on the leader's barrier
@@ -204,7 +215,10 @@ __device__ __forceinline__ void producer_role(const Smem& sm, const Problem& pb,
         if (pb.rank == 0) mbar_arrive_expect_tx(sm.op_full(s), C::kOpFullTx);
         if (!C::kPackedA) tma_load_2d_pair(dst, tmA, kb * BK, m0 + roff, full_leader);
         if (!C::kPackedB)
-          tma_load_2d_pair(dst + C::kOpBytesA, tmB, kb * BK, n0 + roff, full_leader);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d_pair(dst + C::kOpBytesA + h * (HN * BK), tmB, kb * BK,
+                             n0 + h * NH + roff, full_leader);
       }
       if (++s == C::kOpStages) { s = 0; ph ^= 1u; }
     }
@@ -219,10 +233,10 @@ __device__ __forceinline__ void producer_role(const Smem& sm, const Problem& pb,
 }
 
 // Widens packed 4-bit tiles into 8-bit operand tiles (see the file comment).
-// Packed stage: the 4-bit tiles among [x tile 128 rows x 64 B][W tile 128 rows
-// x 64 B], plain rows.  Operand stage: [x tile 128 rows x 128 B][W tile 128
-// rows x 128 B], rows of 128 B with 16-byte chunk c stored at chunk c ^ (row & 7)
-// (128-byte swizzle).
+// Packed stage: the 4-bit tiles among [x tile 128 rows x 64 B][W tiles of the
+// two N-halves, 2 x 128 rows x 64 B], plain rows.  Operand stage: [x tile 128
+// rows x 128 B][W tiles 2 x 128 rows x 128 B], rows of 128 B with 16-byte
+// chunk c stored at chunk c ^ (row & 7) (128-byte swizzle).
 template <int SA, int SB>
 __device__ __forceinline__ void unpack_role(const Smem& sm, const Problem& pb, int ut,
                                             volatile int* abort_flag) {
@@ -312,16 +326,15 @@ template <int SA, int SB>
 __device__ __forceinline__ void mma_role(const Smem& sm, const Problem& pb, uint32_t tmem_base,
                                          volatile int* abort_flag) {
   using C = Cfg<SA, SB>;
-  constexpr uint32_t idesc = idesc_i8(BM, BN);
+  constexpr uint32_t idesc = idesc_i8(BM, NH);
   int s = 0;
   uint32_t ph = 0;
   int it = 0;
   for (int t = pb.pair; t < pb.num_tiles; t += pb.num_pairs, ++it) {
-    const int buf = it & 1;
-    const uint32_t aph = (it >> 1) & 1;
-    if (!mbar_wait_cluster_bounded(sm.acc_empty(buf), aph ^ 1u, abort_flag, kErrWaitMma)) return;
+    const uint32_t aph = it & 1;
+    if (!mbar_wait_cluster_bounded(sm.acc_empty(0), aph ^ 1u, abort_flag, kErrWaitMma)) return;
     tc_fence_after();
-    const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+    const uint32_t d = tmem_base;
     for (int kb = 0; kb < pb.kblocks; ++kb) {
       if (C::kAllPacked) mbar_arrive_expect_tx(sm.op_full(s), 16);  // the relay's signal
       if (C::kPacked && !mbar_wait_bounded(sm.unpacked(s), ph, abort_flag, kErrWaitMma)) return;
@@ -329,19 +342,24 @@ __device__ __forceinline__ void mma_role(const Smem& sm, const Problem& pb, uint
       tc_fence_after();
       const uint32_t a0 = sm.base + C::kOffOp + s * C::kOpStage;
       const uint32_t b0 = a0 + C::kOpBytesA;
+      // both N-halves read the same x tile
 #pragma unroll
-      for (int kk = 0; kk < BK / 32; ++kk)
-        mma_i8_pair(d, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc,
-                    (kb | kk) != 0);
+      for (int kk = 0; kk < BK / 32; ++kk) {
+        const uint64_t adesc = smem_desc_sw128(a0 + kk * 32);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          mma_i8_pair(d + h * NH, adesc, smem_desc_sw128(b0 + h * (HN * BK) + kk * 32), idesc,
+                      (kb | kk) != 0);
+      }
       mma_commit_both(sm.op_empty(s));
       if (++s == C::kOpStages) { s = 0; ph ^= 1u; }
     }
-    mma_commit_both(sm.acc_full(buf));
+    mma_commit_both(sm.acc_full(0));
   }
 }
 
 __device__ __forceinline__ void epi_bar_sync() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");  // the 4 epilogue warps only
+  asm volatile("bar.sync 1, 256;" ::: "memory");  // the 8 epilogue warps only
 }
 
 __device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
@@ -417,9 +435,12 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row,
   }
 }
 
+// Epilogue warp (quad, ch): TMEM lanes 32 quad .. 32 quad + 31 (its rows)
+// and the accumulator columns of N-half ch; et = 0 .. 255 over the 8 warps.
 template <int SHIFT, bool OUT_S32, bool ASYM>
 __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
-                                              uint32_t tmem_base, int quad, int lane, int et,
+                                              uint32_t tmem_base, int quad, int ch, int lane,
+                                              int et,
                                               const float* __restrict__ sa,
                                               const float* __restrict__ sw,
                                               const uint16_t* __restrict__ bias,
@@ -429,14 +450,13 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
                                               volatile int* abort_flag) {
   int it = 0;
   for (int t = pb.pair; t < pb.num_tiles; t += pb.num_pairs, ++it) {
-    const int buf = it & 1;
-    const uint32_t aph = (it >> 1) & 1;
+    const uint32_t aph = it & 1;
     int m0, n0;
     pb.tile_origin(t, m0, n0);
     if (!OUT_S32 || ASYM) {
       // Stage the tile's channel scales, bias and offsets while its main loop runs.
       epi_bar_sync();  // every epilogue warp is done with the previous tile's copy
-      for (int i = et; i < BN; i += 128) {
+      for (int i = et; i < BN; i += 256) {
         const int n = n0 + i;
         const bool ok = n < pb.N;
         if (!OUT_S32) {
@@ -451,10 +471,15 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
     const bool row_ok = row < pb.M;
     const float s_a = (!OUT_S32 && row_ok) ? sa[row] : 0.f;
     const int rsum = (ASYM && row_ok) ? rowsum[row] : 0;
-    if (!mbar_wait_bounded(sm.acc_full(buf), aph, abort_flag, kErrWaitEpilogue)) return;
+    if (!mbar_wait_bounded(sm.acc_full(0), aph, abort_flag, kErrWaitEpilogue)) return;
     tc_fence_after();
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quad) << 16) +
-                           static_cast<uint32_t>(buf * BN);
+                           static_cast<uint32_t>(ch * NH);
+    // this warp's columns: n0 + ch NH .. + NH - 1
+    n0 += ch * NH;
+    const float* e_sw = epi_sw + ch * NH;
+    const float* e_b = epi_b + ch * NH;
+    const int* e_off = epi_off + ch * NH;
     // Two register sets: the TMEM load of chunk c+1 is in flight while chunk c
     // is converted and stored.
     const bool wide = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
@@ -462,25 +487,25 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
     tmem_ld_32x32b_x32(taddr, ra);
     tmem_wait_ld();
 #pragma unroll
-    for (int c = 0; c < BN / 32; c += 2) {
+    for (int c = 0; c < NH / 32; c += 2) {
       tmem_ld_32x32b_x32(taddr + 32 * (c + 1), rb);
       epilogue_chunk<SHIFT, OUT_S32, ASYM>(ra, row, row_ok, n0 + 32 * c, pb.N, s_a,
-                                          epi_sw + 32 * c, epi_b + 32 * c, epi_off + 32 * c,
+                                          e_sw + 32 * c, e_b + 32 * c, e_off + 32 * c,
                                           rsum, out, wide);
       tmem_wait_ld();
-      if (c + 2 < BN / 32) tmem_ld_32x32b_x32(taddr + 32 * (c + 2), ra);
+      if (c + 2 < NH / 32) tmem_ld_32x32b_x32(taddr + 32 * (c + 2), ra);
       epilogue_chunk<SHIFT, OUT_S32, ASYM>(rb, row, row_ok, n0 + 32 * (c + 1), pb.N, s_a,
-                                          epi_sw + 32 * (c + 1), epi_b + 32 * (c + 1),
-                                          epi_off + 32 * (c + 1), rsum, out, wide);
+                                          e_sw + 32 * (c + 1), e_b + 32 * (c + 1),
+                                          e_off + 32 * (c + 1), rsum, out, wide);
       tmem_wait_ld();
     }
     tc_fence_before();
     __syncwarp();
     if (lane == 0) {
       if (pb.rank == 0)
-        mbar_arrive(sm.acc_empty(buf));
+        mbar_arrive(sm.acc_empty(0));
       else
-        mbar_arrive_cluster(map_to_rank(sm.acc_empty(buf), 0));
+        mbar_arrive_cluster(map_to_rank(sm.acc_empty(0), 0));
     }
   }
 }
@@ -534,10 +559,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<SA, SB>::kThread
       mbar_init(sm.op_full(s), C::kOpFullCount);
       mbar_init(sm.op_empty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(sm.acc_full(b), 1);
-      mbar_init(sm.acc_empty(b), C::kAccEmptyCount);
-    }
+    mbar_init(sm.acc_full(0), 1);
+    mbar_init(sm.acc_empty(0), C::kAccEmptyCount);
     if (C::kPacked)
       for (int s = 0; s < C::kOpStages; ++s) mbar_init(sm.unpacked(s), C::kUnpackWarps);
     *abort_flag = 0;
@@ -562,8 +585,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<SA, SB>::kThread
   } else if (warp < 2 + C::kEpiWarps) {
     float* epi_sw = reinterpret_cast<float*>(sm.ptr + C::kOffEpi);
     epilogue_role<C::kAccShift, OUT_S32, ASYM>(
-        sm, pb, tmem_base, warp & 3, lane, threadIdx.x - 64, sa, sw, bias, rowsum, offset, out,
-        epi_sw, epi_sw + BN, reinterpret_cast<int*>(epi_sw + 2 * BN), abort_flag);
+        sm, pb, tmem_base, warp & 3, (warp - 2) >> 2, lane, threadIdx.x - 64, sa, sw, bias,
+        rowsum, offset, out, epi_sw, epi_sw + BN, reinterpret_cast<int*>(epi_sw + 2 * BN),
+        abort_flag);
   } else {
     if (C::kPacked) unpack_role<SA, SB>(sm, pb, threadIdx.x - 32 * (2 + C::kEpiWarps), abort_flag);
   }
