@@ -59,9 +59,10 @@ def parse():
                    help="override M (profiling captures of a smaller case of the same shape)")
     p.add_argument("--workload", default=None,
                    help="the Wan FFN variant to time: w4a4 (default), w8a8, w4a8 or w4a6")
-    p.add_argument("--act-codes", choices=["bytes", "packed"], default="bytes",
-                   help="storage of 4-bit activation codes: one per byte (the GEMM loads them "
-                        "by TMA, only the weights are widened) or two per byte")
+    p.add_argument("--act-codes", choices=["bytes", "packed"], default="packed",
+                   help="storage of 4-bit activation codes: two per byte (packed int4, "
+                        "widened in the GEMM's shared memory) or one per byte (loaded by TMA "
+                        "straight into the operand tiles)")
     return p.parse_args()
 
 

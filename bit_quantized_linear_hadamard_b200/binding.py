@@ -642,12 +642,13 @@ class QuantLinear:
     W4A8 / W4A6 with ``bits_x``): weights packed once; each call runs the
     one-call layer (the activation kernel, then the GEMM) on a workspace the
     layer keeps and grows as needed.  ``act_codes`` stores 4-bit activation
-    codes one per byte ("bytes", the faster GEMM: only the weights are widened
-    in shared memory) or two per byte ("packed"); the codes, and so the
-    outputs, are the same."""
+    codes two per byte ("packed", packed int4 widened in the GEMM's shared
+    memory; the faster form with the GEMM's 256 x 512 tiles) or one per byte
+    ("bytes", loaded by TMA straight into the operand tiles); the codes, and
+    so the outputs, are the same."""
 
     def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None, bits: int,
-                 alpha: float = 1.0, bits_x: int | None = None, act_codes: str = "bytes"):
+                 alpha: float = 1.0, bits_x: int | None = None, act_codes: str = "packed"):
         if act_codes not in ("bytes", "packed"):
             raise ValueError("act_codes is 'bytes' or 'packed'")
         self.N, self.K = weight.shape
@@ -678,8 +679,7 @@ def gbs_state_host(state) -> dict:
 
 class GbsLinear:
     """A layer under δ-guided bit switching: weights quantised at 4 bits (codes
-    stored one per byte, the form qs_linear_gbs takes) and at 8 bits, one
-    device-side state; each call runs the layer at the width the state holds
+    two per byte) and at 8 bits, one device-side state; each call runs the layer at the width the state holds
     and then measures the change of its output against the previous call's,
     choosing the next width on the device (no host synchronisation)."""
 
@@ -687,7 +687,7 @@ class GbsLinear:
                  alpha: float = 1.0, stream=None):
         self.N, self.K = weight.shape
         self.delta, self.alpha = float(delta), alpha
-        self.w4, self.s4 = pack_weights(weight, 4, QS_FLAG_BYTE_CODES, stream=stream)
+        self.w4, self.s4 = pack_weights(weight, 4, stream=stream)
         self.w8, self.s8 = pack_weights(weight, 8, stream=stream)
         self.bias = bias
         self.state = torch.zeros((QS_GBS_STATE_BYTES,), dtype=torch.uint8, device=weight.device)

@@ -6,33 +6,36 @@
 //   out[m][n] = bf16(fl(fl(fl(s_a[m] * s_w[n]) * float(acc)) + bias[n]))
 //
 // Structure: a persistent kernel launched as clusters of two CTAs on the two
-// SMs of a TPC.  Each pair walks output tiles of 256 x 512 (n fastest, so the
-// whole packed weight stays in L2 while activation tiles stream once; the
-// 8-bit weight of the 8x8 form is twice as large and is walked in bands of
-// N-tiles instead, see kBandN).  CTA r of the pair holds rows [128r, 128r+128)
-// of the x tile and, for each N-half h of the tile, rows
-// [256h + 128r, 256h + 128r + 128) of the W tile; the leader (r = 0) issues
-// per 32-deep K step two tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 32),
-// one per N-half, both reading the same x rows of both CTAs; each CTA's
-// 128 x 512 result accumulates in that CTA's tensor memory.  Per SM this
-// halves the W operand traffic of a single-CTA tile at the same MMA work, and
-// the two N-halves share one x tile: one widening of a 4-bit x tile, one set
-// of stage barriers and one TMA load of x serve twice the multiply-adds of a
-// 256 x 256 tile.  (Measured: with the operand traffic of a 256 x 256 tile,
-// issuing twice the MMAs per stage took 1.33x the time, at the tensor pipe's
-// full rate; the smaller tile left it idle a third of its cycles.)
+// SMs of a TPC.  Each pair walks output tiles of 256 x 512 (forms with a 4-bit
+// operand) or 256 x 256 (the 8x8 form), n fastest, so the whole packed weight
+// stays in L2 while activation tiles stream once (the 8-bit weight of the 8x8
+// form is twice as large and is walked in bands of N-tiles instead, see
+// kBandN).  CTA r of the pair holds rows [128r, 128r+128) of the x tile and,
+// for each N-half h of the tile, rows [256h + 128r, 256h + 128r + 128) of the
+// W tile; the leader (r = 0) issues per 32-deep K step one
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 32) per N-half, all reading
+// the same x rows of both CTAs; each CTA's 128-row result accumulates in that
+// CTA's tensor memory.  Per SM this halves the W operand traffic of a
+// single-CTA tile at the same MMA work.  With two N-halves, one widening of a
+// 4-bit x tile, one TMA load of x and one set of stage barriers serve twice
+// the multiply-adds of a 256 x 256 tile.  (Measured: with the operand traffic
+// of a 256 x 256 tile, issuing twice the MMAs per stage took 1.33x the time,
+// at the tensor pipe's full rate; the smaller tile left it idle a third of its
+// cycles.)
 //
 // Warp roles (both CTAs):
 //   warp 0      TMA producer
 //   warp 1      TMEM allocation; in the leader the single-thread MMA issuer;
 //               in the other CTA (4-bit only) the relay that tells the leader
 //               that this CTA's operand tiles are ready
-//   warps 2-9   epilogue: tcgen05.ld of this CTA's accumulator rows, scale,
-//               bias, bf16 store; warps 2-5 the first N-half, 6-9 the second
+//   warps 2-9   epilogue (2-5 in the 8x8 form): tcgen05.ld of this CTA's
+//               accumulator rows, scale, bias, bf16 store; warps 2-5 the first
+//               N-half, 6-9 the second
 //   warps 10-13 (4-bit only) widen packed nibbles into the 8-bit operand tiles
-// The 128 x 512 int32 accumulator fills the 512 TMEM columns, so the MMA of
-// the next tile waits for the epilogue to drain it; the operand ring keeps
-// filling meanwhile.
+// With 256 x 512 tiles the 128 x 512 int32 accumulator fills the 512 TMEM
+// columns, so the MMA of the next tile waits for the epilogue to drain it (the
+// operand ring keeps filling meanwhile); the 8x8 form's 256-column
+// accumulators are two, so its epilogue runs under the next tile's main loop.
 //
 // Synchronisation across the pair: 8-bit operand stages are "full" on the
 // leader's barrier when the TMA loads of both CTAs have landed.  4-bit operand
@@ -82,12 +85,11 @@ namespace qs {
 namespace gemm {
 
 constexpr int BM = 256;  // tile rows (tokens), 128 per CTA
-constexpr int BN = 512;  // tile columns (output channels): two MMA halves
-constexpr int NH = 256;  // columns of one MMA (an N-half of the tile)
+constexpr int NH = 256;  // columns of one MMA (an N-half of a tile)
 constexpr int HM = 128;  // x rows per CTA
 constexpr int HN = 128;  // W rows per CTA and N-half
 constexpr int BK = 128;  // K elements per pipeline stage (= 128 bytes of 8-bit operand)
-constexpr int kTmemCols = BN;  // one 512-column int32 accumulator: all of tensor memory
+constexpr int kTmemCols = 512;  // all of tensor memory: int32 accumulator columns
 
 // SA, SB: storage bits of the x and W codes (4 = two per byte, 8 = one byte).
 template <int SA, int SB>
@@ -98,18 +100,23 @@ struct Cfg {
   static constexpr bool kPacked = kPackedA || kPackedB;   // some operand is widened
   static constexpr bool kAllPacked = kPackedA && kPackedB;
   static constexpr bool kDirect = !kAllPacked;            // some operand goes by TMA directly
+  // N-halves per tile: 2 (tiles of 256 x 512) when an operand is widened;
+  // the 8x8 form keeps tiles of 256 x 256 with two accumulators (see kBandN)
+  static constexpr int kHalves = kPacked ? 2 : 1;
+  static constexpr int kBN = kHalves * NH;               // tile columns
+  static constexpr int kAccBufs = kTmemCols / kBN;       // accumulators in tensor memory
   static constexpr int kPkBytesA = kPackedA ? HM * BK / 2 : 0;  // packed tile of x (this CTA)
-  static constexpr int kPkBytesB = kPackedB ? 2 * HN * BK / 2 : 0;  // packed W, both halves
-  static constexpr int kOpBytesA = HM * BK;      // 8-bit operand tile of x
-  static constexpr int kOpBytesB = 2 * HN * BK;  // 8-bit operand tiles of W, both halves
+  static constexpr int kPkBytesB = kPackedB ? kHalves * HN * BK / 2 : 0;  // packed W tiles
+  static constexpr int kOpBytesA = HM * BK;            // 8-bit operand tile of x
+  static constexpr int kOpBytesB = kHalves * HN * BK;  // 8-bit operand tiles of W
   static constexpr int kPkStage = kPkBytesA + kPkBytesB;
   static constexpr int kOpStage = kOpBytesA + kOpBytesB;
   // bytes the TMA writes straight into one operand stage of this CTA
   static constexpr int kDirectBytes = (kPackedA ? 0 : kOpBytesA) + (kPackedB ? 0 : kOpBytesB);
   // as many stages as fit in shared memory
-  static constexpr int kOpStages = kPacked ? 3 : 4;
+  static constexpr int kOpStages = kPacked ? 3 : 6;
   static constexpr int kPkStages = kPacked ? kOpStages : 0;  // one ring index drives both
-  static constexpr int kEpiWarps = 8;  // two per TMEM lane quarter: one per N-half
+  static constexpr int kEpiWarps = 4 * kHalves;  // per TMEM lane quarter, one per N-half
   static constexpr int kUnpackWarps = kPacked ? 4 : 0;
   // operand-tile row that packed row 0 widens into (W rows follow the 128 x rows)
   static constexpr int kUnpackRow0 = kPackedA ? 0 : HM;
@@ -122,7 +129,7 @@ struct Cfg {
   static constexpr int kNumBars = 2 * kPkStages + 3 * kOpStages + 4;
   // s_w, bias and (asymmetric weights) channel offsets of a tile
   static constexpr int kOffEpi = (kOffBar + 8 * kNumBars + 15) / 16 * 16;
-  static constexpr int kOffMisc = kOffEpi + 3 * BN * 4;  // TMEM address, abort flag
+  static constexpr int kOffMisc = kOffEpi + 3 * kBN * 4;  // TMEM address, abort flag
   static constexpr int kOffSignal = kOffMisc + 16;        // 16 bytes per operand stage
   static constexpr int kSmemBytes = kOffSignal + 16 * kOpStages + 1024;  // + alignment slack
   static constexpr int kUnpackThreads = kPacked ? 32 * kUnpackWarps : 1;
@@ -155,15 +162,18 @@ struct Smem {
 
 // Tile order of the 8-bit x 8-bit instantiation: bands of kBandN N-tiles,
 // M advancing inside a band, so that the band's slice of the 8-bit weight
-// (9 x 512 rows, 23.6 MB at K = 5120) stays in L2 while the activation tiles
+// (18 x 256 rows, 23.6 MB at K = 5120) stays in L2 while the activation tiles
 // stream.  In n-fastest order the whole 70.8 MB weight of the Wan FFN was read
-// from DRAM many times per launch; banded, the launch measured 5-10 %
+// from DRAM about 19 times per launch; banded, the launch measured 5-10 %
 // faster.  The other instantiations, whose packed 4-bit weight fits in L2,
-// keep the n-fastest order.
-constexpr int kBandN = 9;
+// keep the n-fastest order.  (The 8x8 form keeps tiles of 256 x 256: with
+// 256 x 512 tiles it measured 1.478 against 1.395 ms at the Wan FFN shape,
+// where it runs at the board's power limit.)
+constexpr int kBandN = 18;
 
 struct Problem {
   int M, N, K;
+  int bn;               // tile columns
   int n_tiles, num_tiles, kblocks;
   int band;             // N-tiles per band, 0: n-fastest order
   int pair, num_pairs;  // this pair's index and the number of pairs
@@ -175,10 +185,10 @@ struct Problem {
       const int g = t / per_band, r = t - g * per_band;
       const int gn = min(band, n_tiles - g * band);  // the last band may be narrower
       m0 = (r / gn) * BM;
-      n0 = (g * band + r % gn) * BN;
+      n0 = (g * band + r % gn) * bn;
     } else {
       m0 = (t / n_tiles) * BM;
-      n0 = (t % n_tiles) * BN;
+      n0 = (t % n_tiles) * bn;
     }
   }
 };
@@ -203,7 +213,7 @@ __device__ __forceinline__ void producer_role(const Smem& sm, const Problem& pb,
         if (C::kPackedA) tma_load_2d(dst, tmA, kb * (BK / 2), m0 + roff, sm.pk_full(s));
         if (C::kPackedB)
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
+          for (int h = 0; h < C::kHalves; ++h)
             tma_load_2d(dst + C::kPkBytesA + h * (HN * BK / 2), tmB, kb * (BK / 2),
                         n0 + h * NH + roff, sm.pk_full(s));
       }
@@ -216,7 +226,7 @@ __device__ __forceinline__ void producer_role(const Smem& sm, const Problem& pb,
         if (!C::kPackedA) tma_load_2d_pair(dst, tmA, kb * BK, m0 + roff, full_leader);
         if (!C::kPackedB)
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
+          for (int h = 0; h < C::kHalves; ++h)
             tma_load_2d_pair(dst + C::kOpBytesA + h * (HN * BK), tmB, kb * BK,
                              n0 + h * NH + roff, full_leader);
       }
@@ -331,10 +341,11 @@ __device__ __forceinline__ void mma_role(const Smem& sm, const Problem& pb, uint
   uint32_t ph = 0;
   int it = 0;
   for (int t = pb.pair; t < pb.num_tiles; t += pb.num_pairs, ++it) {
-    const uint32_t aph = it & 1;
-    if (!mbar_wait_cluster_bounded(sm.acc_empty(0), aph ^ 1u, abort_flag, kErrWaitMma)) return;
+    const int buf = it % C::kAccBufs;
+    const uint32_t aph = (it / C::kAccBufs) & 1;
+    if (!mbar_wait_cluster_bounded(sm.acc_empty(buf), aph ^ 1u, abort_flag, kErrWaitMma)) return;
     tc_fence_after();
-    const uint32_t d = tmem_base;
+    const uint32_t d = tmem_base + static_cast<uint32_t>(buf * C::kBN);
     for (int kb = 0; kb < pb.kblocks; ++kb) {
       if (C::kAllPacked) mbar_arrive_expect_tx(sm.op_full(s), 16);  // the relay's signal
       if (C::kPacked && !mbar_wait_bounded(sm.unpacked(s), ph, abort_flag, kErrWaitMma)) return;
@@ -347,19 +358,21 @@ __device__ __forceinline__ void mma_role(const Smem& sm, const Problem& pb, uint
       for (int kk = 0; kk < BK / 32; ++kk) {
         const uint64_t adesc = smem_desc_sw128(a0 + kk * 32);
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+        for (int h = 0; h < C::kHalves; ++h)
           mma_i8_pair(d + h * NH, adesc, smem_desc_sw128(b0 + h * (HN * BK) + kk * 32), idesc,
                       (kb | kk) != 0);
       }
       mma_commit_both(sm.op_empty(s));
       if (++s == C::kOpStages) { s = 0; ph ^= 1u; }
     }
-    mma_commit_both(sm.acc_full(0));
+    mma_commit_both(sm.acc_full(buf));
   }
 }
 
+// named barrier 1 over the epilogue warps only
+template <int THREADS>
 __device__ __forceinline__ void epi_bar_sync() {
-  asm volatile("bar.sync 1, 256;" ::: "memory");  // the 8 epilogue warps only
+  asm volatile("bar.sync 1, %0;" ::"n"(THREADS) : "memory");
 }
 
 __device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
@@ -436,8 +449,8 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row,
 }
 
 // Epilogue warp (quad, ch): TMEM lanes 32 quad .. 32 quad + 31 (its rows)
-// and the accumulator columns of N-half ch; et = 0 .. 255 over the 8 warps.
-template <int SHIFT, bool OUT_S32, bool ASYM>
+// and the accumulator columns of N-half ch; et = 0 .. 32 EPI_WARPS - 1.
+template <int SHIFT, bool OUT_S32, bool ASYM, int EPI_WARPS, int ACC_BUFS>
 __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
                                               uint32_t tmem_base, int quad, int ch, int lane,
                                               int et,
@@ -450,13 +463,14 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
                                               volatile int* abort_flag) {
   int it = 0;
   for (int t = pb.pair; t < pb.num_tiles; t += pb.num_pairs, ++it) {
-    const uint32_t aph = it & 1;
+    const int buf = it % ACC_BUFS;
+    const uint32_t aph = (it / ACC_BUFS) & 1;
     int m0, n0;
     pb.tile_origin(t, m0, n0);
     if (!OUT_S32 || ASYM) {
       // Stage the tile's channel scales, bias and offsets while its main loop runs.
-      epi_bar_sync();  // every epilogue warp is done with the previous tile's copy
-      for (int i = et; i < BN; i += 256) {
+      epi_bar_sync<32 * EPI_WARPS>();  // every epilogue warp is done with the previous copy
+      for (int i = et; i < pb.bn; i += 32 * EPI_WARPS) {
         const int n = n0 + i;
         const bool ok = n < pb.N;
         if (!OUT_S32) {
@@ -465,16 +479,16 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
         }
         if (ASYM) epi_off[i] = ok ? offset[n] : 0;
       }
-      epi_bar_sync();
+      epi_bar_sync<32 * EPI_WARPS>();
     }
     const int row = m0 + static_cast<int>(pb.rank) * HM + 32 * quad + lane;
     const bool row_ok = row < pb.M;
     const float s_a = (!OUT_S32 && row_ok) ? sa[row] : 0.f;
     const int rsum = (ASYM && row_ok) ? rowsum[row] : 0;
-    if (!mbar_wait_bounded(sm.acc_full(0), aph, abort_flag, kErrWaitEpilogue)) return;
+    if (!mbar_wait_bounded(sm.acc_full(buf), aph, abort_flag, kErrWaitEpilogue)) return;
     tc_fence_after();
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quad) << 16) +
-                           static_cast<uint32_t>(ch * NH);
+                           static_cast<uint32_t>(buf * pb.bn + ch * NH);
     // this warp's columns: n0 + ch NH .. + NH - 1
     n0 += ch * NH;
     const float* e_sw = epi_sw + ch * NH;
@@ -503,9 +517,9 @@ __device__ __forceinline__ void epilogue_role(const Smem& sm, const Problem& pb,
     __syncwarp();
     if (lane == 0) {
       if (pb.rank == 0)
-        mbar_arrive(sm.acc_empty(0));
+        mbar_arrive(sm.acc_empty(buf));
       else
-        mbar_arrive_cluster(map_to_rank(sm.acc_empty(0), 0));
+        mbar_arrive_cluster(map_to_rank(sm.acc_empty(buf), 0));
     }
   }
 }
@@ -539,7 +553,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<SA, SB>::kThread
   pb.M = M;
   pb.N = N;
   pb.K = K;
-  pb.n_tiles = (N + BN - 1) / BN;
+  pb.bn = C::kBN;
+  pb.n_tiles = (N + C::kBN - 1) / C::kBN;
   pb.num_tiles = ((M + BM - 1) / BM) * pb.n_tiles;
   pb.kblocks = K / BK;
   pb.band = (SA == 8 && SB == 8) ? kBandN : 0;
@@ -559,8 +574,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<SA, SB>::kThread
       mbar_init(sm.op_full(s), C::kOpFullCount);
       mbar_init(sm.op_empty(s), 1);
     }
-    mbar_init(sm.acc_full(0), 1);
-    mbar_init(sm.acc_empty(0), C::kAccEmptyCount);
+    for (int b = 0; b < C::kAccBufs; ++b) {
+      mbar_init(sm.acc_full(b), 1);
+      mbar_init(sm.acc_empty(b), C::kAccEmptyCount);
+    }
     if (C::kPacked)
       for (int s = 0; s < C::kOpStages; ++s) mbar_init(sm.unpacked(s), C::kUnpackWarps);
     *abort_flag = 0;
@@ -584,10 +601,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<SA, SB>::kThread
     if (lane == 0 && pb.rank != 0 && C::kPacked) relay_role<SA, SB>(sm, pb, abort_flag);
   } else if (warp < 2 + C::kEpiWarps) {
     float* epi_sw = reinterpret_cast<float*>(sm.ptr + C::kOffEpi);
-    epilogue_role<C::kAccShift, OUT_S32, ASYM>(
+    epilogue_role<C::kAccShift, OUT_S32, ASYM, C::kEpiWarps, C::kAccBufs>(
         sm, pb, tmem_base, warp & 3, (warp - 2) >> 2, lane, threadIdx.x - 64, sa, sw, bias,
-        rowsum, offset, out, epi_sw, epi_sw + BN, reinterpret_cast<int*>(epi_sw + 2 * BN),
-        abort_flag);
+        rowsum, offset, out, epi_sw, epi_sw + C::kBN,
+        reinterpret_cast<int*>(epi_sw + 2 * C::kBN), abort_flag);
   } else {
     if (C::kPacked) unpack_role<SA, SB>(sm, pb, threadIdx.x - 32 * (2 + C::kEpiWarps), abort_flag);
   }
@@ -634,7 +651,7 @@ inline qs_status launch_qgemm(const void* xp, const float* sa, const void* wp, c
   if (sms <= 0) return QS_ERR_CUDA;
   // persistent clusters of two CTAs, at most one CTA per SM
   const int64_t tiles = ((M + BM - 1) / BM) *
-                        ((N + BN - 1) / BN);
+                        ((N + C::kBN - 1) / C::kBN);
   const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
   if (pairs < 1) return QS_ERR_CUDA;
   const int grid = static_cast<int>(2 * pairs);

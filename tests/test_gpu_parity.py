@@ -369,11 +369,11 @@ MULTI_TILE_FORMS = [(4, 4, 0), (4, 4, qs.QS_FLAG_BYTE_CODES), (8, 8, 0), (8, 4, 
 @pytest.mark.parametrize("bx,bw,flags", MULTI_TILE_FORMS, ids=["w4a4", "w4a4_bytes", "w8a8", "w4a8"])
 def test_multi_tile_grid_every_element(bx, bw, flags):
     """M = 4096, N = 5120, K = 5120: 16 x 10 = 160 output tiles of 256 x 512
-    for 74 CTA pairs, so every pair runs two or three tiles (the persistent
-    loop, the tensor-memory accumulator drained and reused, the operand ring
-    wrapping many times) and the 8-bit x 8-bit form crosses a band edge
-    (9 + 1 N-tiles).  Every code, scale, accumulator and output is compared
-    with the oracle."""
+    (16 x 20 = 320 of 256 x 256 in the 8-bit x 8-bit form) for 74 CTA pairs,
+    so every pair runs several tiles (the persistent loop, the tensor-memory
+    accumulators drained and reused, the operand ring wrapping many times)
+    and the 8-bit x 8-bit form crosses a band edge (18 + 2 N-tiles).  Every
+    code, scale, accumulator and output is compared with the oracle."""
     M, N, K, alpha = 4096, 5120, 5120, 0.9
     d = I.make_shape(seed=4096 + 10 * bx + bw, M=M, K=K, N=N, bits=bw, alpha=alpha,
                      outlier_factor=100.0, outlier_frac=0.005, sigma_w=0.015,
@@ -393,9 +393,9 @@ def test_multi_tile_grid_every_element(bx, bw, flags):
 
 
 def test_w8a8_band_edge_small():
-    """The 8-bit x 8-bit form walks N-tiles of 512 columns in bands of 9:
-    N = 5120 has 10 N-tiles (a full band and a last band of 1), M = 300 a
-    ragged second M-tile.  Full int32 and bf16 parity."""
+    """The 8-bit x 8-bit form walks N-tiles in bands of 18: N = 5120 has 20
+    N-tiles (a full band and a last band of 2), M = 300 a ragged second M-tile.
+    Full int32 and bf16 parity."""
     M, N, K = 300, 5120, 256
     d = I.make_shape(seed=3005, M=M, K=K, N=N, bits=8, outlier_factor=50.0)
     g = run_layer(d, 8, 1.0)
