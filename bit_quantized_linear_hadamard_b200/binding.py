@@ -679,7 +679,8 @@ def gbs_state_host(state) -> dict:
 
 class GbsLinear:
     """A layer under δ-guided bit switching: weights quantised at 4 bits (codes
-    two per byte) and at 8 bits, one device-side state; each call runs the layer at the width the state holds
+    stored one per byte, the form qs_linear_gbs takes) and at 8 bits, one
+    device-side state; each call runs the layer at the width the state holds
     and then measures the change of its output against the previous call's,
     choosing the next width on the device (no host synchronisation)."""
 
@@ -687,7 +688,7 @@ class GbsLinear:
                  alpha: float = 1.0, stream=None):
         self.N, self.K = weight.shape
         self.delta, self.alpha = float(delta), alpha
-        self.w4, self.s4 = pack_weights(weight, 4, stream=stream)
+        self.w4, self.s4 = pack_weights(weight, 4, QS_FLAG_BYTE_CODES, stream=stream)
         self.w8, self.s8 = pack_weights(weight, 8, stream=stream)
         self.bias = bias
         self.state = torch.zeros((QS_GBS_STATE_BYTES,), dtype=torch.uint8, device=weight.device)

@@ -471,9 +471,13 @@ QS_API qs_status qs_gbs_update(const void* y_cur_bf16, const void* y_prev_bf16, 
  * qs_linear_gbs — the one-call layer (as qs_linear) at the width the state
  * holds: the 4-bit and the 8-bit kernels are both enqueued and each returns at
  * once unless the state selects its width.  Weights are prepared at both
- * widths with qs_pack_weights (flags 0): the 4-bit step is the packed W4A4
- * layer, the 8-bit step the W8A8 layer.
- *   w4_packed, w4_scale  weights at 4 bits, two codes per byte ([N][K/2]);
+ * widths: qs_pack_weights with bits 8, and with bits 4 and QS_FLAG_BYTE_CODES
+ * (the 4-bit codes one per byte, [N][K] bytes).  With both operands stored in
+ * bytes the 4-bit step runs the 8-bit-storage GEMM on 4-bit codes: the int8
+ * tensor cores multiply them no faster, and that GEMM, which runs at the
+ * board's power limit, clocks higher on 4-bit values than the packed 4x4
+ * GEMM runs in the same sequence.
+ *   w4_packed, w4_scale  weights at 4 bits, one code per byte;
  *   w8_packed, w8_scale  weights at 8 bits
  *   state                a qs_gbs_state (read only)
  *   workspace            at least qs_linear_workspace_bytes(M, K, 8) bytes
