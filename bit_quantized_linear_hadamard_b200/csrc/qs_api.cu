@@ -161,21 +161,21 @@ qs_status launch_sd4_gemm(const CUtensorMap& ca, const CUtensorMap& cb, const CU
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
-template <bool ADEC, bool BDEC>
+template <bool ADEC, bool BDEC, bool WIDE = false>
 qs_status launch_sd4_mx(const CUtensorMap& ca, const CUtensorMap& cb, const CUtensorMap& ma,
                         const CUtensorMap& mb, const CUtensorMap& xa, const CUtensorMap& wb,
                         const void* bias, int64_t M, int64_t N, int64_t K, void* out,
                         void* stream, int64_t kb_wrap, const int32_t* out_rows, int64_t out_M) {
   namespace G = qs::sd4::gemm_mx;
-  using C = G::MCfg<ADEC, BDEC>;
+  using C = G::MCfg<ADEC, BDEC, WIDE>;
   constexpr int smem = C::kSmemBytes;
-  auto kern = G::sd4_mx_gemm_kernel<ADEC, BDEC>;
+  auto kern = G::sd4_mx_gemm_kernel<ADEC, BDEC, WIDE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return QS_ERR_CUDA;
   const int sms = qs::sm_count();
   if (sms <= 0) return QS_ERR_CUDA;
-  const int64_t tiles = ((M + G::BM - 1) / G::BM) * ((N + G::BN - 1) / G::BN);
+  const int64_t tiles = ((M + G::BM - 1) / G::BM) * ((N + C::kBN - 1) / C::kBN);
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   kern<<<grid, C::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(
       ca, cb, ma, mb, xa, wb, static_cast<const uint16_t*>(bias), static_cast<uint16_t*>(out),
@@ -212,8 +212,8 @@ qs_status run_sd4_mx(const void* a_codes, const void* a_e4m3, const uint16_t* a_
   const int64_t kb_wrap = K / G::BK;
   if (a_e4m3) {
     if (!w_e4m3) return QS_ERR_NULL;  // e4m3 activations go with e4m3 weights
-    return launch_sd4_mx<false, false>(xa, xa, ma, mb, xa, wb, bias, a_rows, N, Ka, out, stream,
-                                       kb_wrap, out_rows, out_M);
+    return launch_sd4_mx<false, false, true>(xa, xa, ma, mb, xa, wb, bias, a_rows, N, Ka, out,
+                                             stream, kb_wrap, out_rows, out_M);
   }
   if (w_e4m3)
     return launch_sd4_mx<true, false>(ca, ca, ma, mb, ca, wb, bias, a_rows, N, Ka, out, stream,

@@ -13,7 +13,11 @@
 // accumulators and the 12 scale columns fit the 512 TMEM columns; two
 // 256-column accumulators would leave none for the scales), 128 K elements
 // (four scale blocks) per stage.  Tiles on CTA pairs (cta_group::2, M = 256)
-// measured slower than this single-CTA form.
+// measured slower than this single-CTA form.  With e4m3 operands for both x
+// and W the tiles are 128 x 384 (WIDE): two N = 192 MMAs per K step share the
+// x tile, into one 384-column accumulator (measured: issuing every stage's
+// MMAs twice took 1.43x the time of once, so with 128 x 192 tiles the tensor
+// pipe idled between stages).
 // Warp roles: 0 TMA producer (codes every stage, block words every two
 // stages, the decoded weights when given), 1 TMEM allocation and the MMA
 // issuer (per stage: three tcgen05.cp of the stage's scales into TMEM, then
@@ -42,31 +46,46 @@ constexpr int kOpA = BM * BK, kOpB = BN * BK;          // e4m3 tiles, 128-byte r
 constexpr int kSfA = 512, kSfB = 1024;                 // scale bytes of a stage
 constexpr int kPkA = BM * BK / 2, kPkB = BN * BK / 2;  // code tiles, 64-byte rows
 constexpr int kMetaA = BM * 16, kMetaB = BN * 16;      // 8 block words per row = 2 stages
+// Bands of 36 tiles of 192 columns (6912 weight rows; e4m3 x e4m3 at the Wan
+// FFN shape: 2.35 ms against 2.53 ms in plain row-major tile order; bands of
+// 12 N-tiles 2.39 ms); wide tiles take half as many.
+constexpr int kGroupN = 36;
 static_assert(BN % 32 == 0 && BN <= 256 && 2 * BN + 12 <= kTmemCols, "tile");
 
 // ADEC / BDEC: the activations / weights come as SD4 codes and are decoded
 // to e4m3 in the kernel; otherwise as e4m3 bytes (qs_sd4_quant_e4m3,
 // qs_sd4_decode_e4m3) that TMA loads straight into their operand tile.  The
 // block words give the scales in every case.
-template <bool ADEC, bool BDEC>
+// WIDE (e4m3 x and W only): tiles of 128 x 384, two MMAs of N = 192 per K
+// step reading the same x tile, into one 384-column accumulator (the scales
+// take 4 + 16 more columns, so a second accumulator does not fit); eight
+// epilogue warps, one per TMEM lane quarter and N-half.
+template <bool ADEC, bool BDEC, bool WIDE = false>
 struct MCfg {
+  static_assert(!WIDE || (!ADEC && !BDEC), "wide tiles for e4m3 operands only");
   static constexpr bool kAnyDec = ADEC || BDEC;
+  static constexpr int kHalves = WIDE ? 2 : 1;
+  static constexpr int kBN = kHalves * BN;          // tile columns
+  static constexpr int kAccBufs = WIDE ? 1 : 2;     // accumulators in tensor memory
+  static constexpr int kEpiW = kEpiWarps * kHalves;  // epilogue warps
+  static constexpr int kGroup = kGroupN / kHalves;   // N-tiles per band (same columns)
   static constexpr int kDecWarps = ADEC ? (BDEC ? 10 : 8) : 4;
   static constexpr int kDecThreads = 32 * kDecWarps;
-  static constexpr int kThreads = 32 * (2 + kEpiWarps + kDecWarps);
+  static constexpr int kThreads = 32 * (2 + kEpiW + kDecWarps);
   // operand stages by measurement (e4m3 x e4m3 at the Wan FFN shape: 3 stages
-  // 2.72 ms, 4 stages 2.35 ms, 5 stages 2.47 ms; deeper block-word rings no gain)
-  static constexpr int kOpStages = BDEC ? 3 : 4;
+  // 2.72 ms, 4 stages 2.35 ms, 5 stages 2.47 ms; deeper block-word rings no
+  // gain); wide tiles: as many as fit
+  static constexpr int kOpStages = (BDEC || WIDE) ? 3 : 4;
   static constexpr int kPkStages = kAnyDec ? kOpStages : 0;
   static constexpr int kMetaSlots = 2;
   static constexpr int kDecRows = (ADEC ? BM : 0) + (BDEC ? BN : 0);  // rows decoded per stage
   static constexpr int kTasks = 2 * kDecRows;  // (row, half of the stage's K)
-  static constexpr int kOpStage = kOpA + kOpB;
-  static constexpr int kSfStage = kSfA + kSfB;
+  static constexpr int kOpStage = kOpA + kHalves * kOpB;
+  static constexpr int kSfStage = kSfA + kHalves * kSfB;
   static constexpr int kPkStage = (ADEC ? kPkA : 0) + (BDEC ? kPkB : 0);
   // operand bytes TMA writes straight into an operand stage
-  static constexpr int kDirectBytes = (ADEC ? 0 : kOpA) + (BDEC ? 0 : kOpB);
-  static constexpr int kMetaSlot = kMetaA + kMetaB;
+  static constexpr int kDirectBytes = (ADEC ? 0 : kOpA) + (BDEC ? 0 : kHalves * kOpB);
+  static constexpr int kMetaSlot = kMetaA + kHalves * kMetaB;
   static constexpr int kOffOp = 0;
   static constexpr int kOffSf = kOffOp + kOpStages * kOpStage;
   static constexpr int kOffPk = kOffSf + kOpStages * kSfStage;
@@ -74,7 +93,7 @@ struct MCfg {
   static constexpr int kOffBar = kOffMeta + kMetaSlots * kMetaSlot;
   static constexpr int kNumBars = 2 * kPkStages + 2 * kMetaSlots + 2 * kOpStages + 4;
   static constexpr int kOffEpi = (kOffBar + 8 * kNumBars + 15) / 16 * 16;  // bias of a tile
-  static constexpr int kOffTab = kOffEpi + BN * 4;                          // e4m3 level table
+  static constexpr int kOffTab = kOffEpi + kBN * 4;                         // e4m3 level table
   static constexpr int kOffMisc = kOffTab + kDialects * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   // arrivals completing an operand stage: the decode warps, plus the
@@ -163,19 +182,17 @@ struct MBars {
   __device__ uint32_t acc_empty(int b) const { return at(2 * P + 2 * T + 2 * U + 2 + b); }
 };
 
-// Tile order: bands of kGroupN N-tiles, every M-tile inside a band (N fastest
-// within it), so the tiles the CTAs hold at one time share a few MB of
-// activations and weights in L2 and each weight band is read from HBM once
-// (e4m3 x e4m3 at the Wan FFN shape: 2.35 ms against 2.53 ms in plain
-// row-major tile order; bands of 12 N-tiles 2.39 ms).
-constexpr int kGroupN = 36;
-
-__device__ __forceinline__ void tile_origin(int t, int m_tiles, int n_tiles, int& m0, int& n0) {
-  const int per_group = kGroupN * m_tiles;
+// Tile order: bands of `group` N-tiles of `bn` columns, every M-tile inside a
+// band (N fastest within it), so the tiles the CTAs hold at one time share a
+// few MB of activations and weights in L2 and each weight band is read from
+// HBM once (kGroupN; see its note).
+__device__ __forceinline__ void tile_origin(int t, int m_tiles, int n_tiles, int group, int bn,
+                                            int& m0, int& n0) {
+  const int per_group = group * m_tiles;
   const int g = t / per_group, r = t - g * per_group;
-  const int gn = min(kGroupN, n_tiles - g * kGroupN);  // N-tiles in this band
+  const int gn = min(group, n_tiles - g * group);  // N-tiles in this band
   m0 = (r / gn) * BM;
-  n0 = (g * kGroupN + r % gn) * BN;
+  n0 = (g * group + r % gn) * bn;
 }
 
 // Scale-block offset of row m (within A's 128 rows or B's 192) in a stage.
@@ -190,8 +207,8 @@ __device__ __forceinline__ int sf_row_offset(int m) {
 // skipped and flagged.
 // tmCA / tmCB: the codes (when decoded), tmXA / tmWB: the e4m3 bytes (when
 // loaded directly), tmMA / tmMB: the block words.
-template <bool ADEC, bool BDEC>
-__global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
+template <bool ADEC, bool BDEC, bool WIDE>
+__global__ void __launch_bounds__(MCfg<ADEC, BDEC, WIDE>::kThreads, 1)
     sd4_mx_gemm_kernel(const __grid_constant__ CUtensorMap tmCA,
                        const __grid_constant__ CUtensorMap tmCB,
                        const __grid_constant__ CUtensorMap tmMA,
@@ -200,7 +217,7 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
                        const __grid_constant__ CUtensorMap tmWB, const uint16_t* __restrict__ bias,
                        uint16_t* __restrict__ out, int M, int N, int K, int kb_wrap,
                        const int32_t* __restrict__ out_rows, int out_M) {
-  using C = MCfg<ADEC, BDEC>;
+  using C = MCfg<ADEC, BDEC, WIDE>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
@@ -213,7 +230,7 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + C::kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = (N + BN - 1) / BN;
+  const int n_tiles = (N + C::kBN - 1) / C::kBN;
   const int m_tiles = (M + BM - 1) / BM;
   const int num_tiles = m_tiles * n_tiles;
   const int kblocks = K / BK;
@@ -243,9 +260,9 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
       mbar_init(bars.op_full(s), C::kOpFullCount);
       mbar_init(bars.op_empty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(bars.acc_full(b), 1);
-      mbar_init(bars.acc_empty(b), kEpiWarps);
+      mbar_init(bars.acc_empty(b), C::kEpiW);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -265,7 +282,7 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
       uint32_t ph = 0, mph = 0, pho = 0;
       for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
         int m0, n0;
-        tile_origin(t, m_tiles, n_tiles, m0, n0);
+        tile_origin(t, m_tiles, n_tiles, C::kGroup, C::kBN, m0, n0);
         for (int kb = 0, kbw = 0; kb < kblocks; ++kb, kbw = (kbw + 1 == kb_wrap ? 0 : kbw + 1)) {
           // kbw: the weights' K-block; kb_wrap is even, so both stay in step
           // with the two-stage block-word slots
@@ -275,7 +292,10 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
             const uint32_t dst = sbase + C::kOffMeta + ms * C::kMetaSlot;
             mbar_arrive_expect_tx(bars.meta_full(ms), C::kMetaSlot);
             tma_load_2d(dst, &tmMA, (kb / 2) * 16, m0, bars.meta_full(ms));
-            tma_load_2d(dst + kMetaA, &tmMB, (kbw / 2) * 16, n0, bars.meta_full(ms));
+#pragma unroll
+            for (int h = 0; h < C::kHalves; ++h)
+              tma_load_2d(dst + kMetaA + h * kMetaB, &tmMB, (kbw / 2) * 16, n0 + h * BN,
+                          bars.meta_full(ms));
             if (++ms == C::kMetaSlots) { ms = 0; mph ^= 1u; }
           }
           if (C::kAnyDec) {  // codes of the decoded operands
@@ -294,7 +314,10 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
             const uint32_t ob = sbase + C::kOffOp + so * C::kOpStage;
             mbar_arrive_expect_tx(bars.op_full(so), C::kDirectBytes);
             if (!ADEC) tma_load_2d(ob, &tmXA, kb * BK, m0, bars.op_full(so));
-            if (!BDEC) tma_load_2d(ob + kOpA, &tmWB, kbw * BK, n0, bars.op_full(so));
+            if (!BDEC)
+#pragma unroll
+              for (int h = 0; h < C::kHalves; ++h)
+                tma_load_2d(ob + kOpA + h * kOpB, &tmWB, kbw * BK, n0 + h * BN, bars.op_full(so));
             if (++so == C::kOpStages) { so = 0; pho ^= 1u; }
           }
         }
@@ -307,8 +330,8 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
       uint32_t ph = 0;
       int it = 0;
       for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
-        const int buf = it & 1;
-        const uint32_t aph = (it >> 1) & 1;
+        const int buf = it % C::kAccBufs;
+        const uint32_t aph = (it / C::kAccBufs) & 1;
         if (!mbar_wait_bounded(bars.acc_empty(buf), aph ^ 1u, abort_flag, kErrWaitMma)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
@@ -321,35 +344,45 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
           // the stage's scales into TMEM; the tensor pipe runs these copies
           // and the MMAs below in issue order
           tmem_cp_32x128b_x4(sfa, smem_desc_sf(f0));
-          tmem_cp_32x128b_x4(sfb, smem_desc_sf(f0 + kSfA));
-          tmem_cp_32x128b_x4(sfb + 4, smem_desc_sf(f0 + kSfA + 512));
+#pragma unroll
+          for (int h = 0; h < C::kHalves; ++h) {  // N-half h: 8 scale columns of its own
+            tmem_cp_32x128b_x4(sfb + 8 * h, smem_desc_sf(f0 + kSfA + h * kSfB));
+            tmem_cp_32x128b_x4(sfb + 8 * h + 4, smem_desc_sf(f0 + kSfA + h * kSfB + 512));
+          }
 #pragma unroll
           for (int j = 0; j < BK / 32; ++j)
-            mma_mx(d, smem_desc_sw128(a0 + j * 32), smem_desc_sw128(b0 + j * 32),
-                   idesc_mx(BM, BN, static_cast<uint32_t>(j)),
-                   sfa + (static_cast<uint32_t>(j) << 30), sfb + (static_cast<uint32_t>(j) << 30),
-                   (kb | j) != 0);
+#pragma unroll
+            for (int h = 0; h < C::kHalves; ++h)
+              mma_mx(d + h * BN, smem_desc_sw128(a0 + j * 32),
+                     smem_desc_sw128(b0 + h * kOpB + j * 32),
+                     idesc_mx(BM, BN, static_cast<uint32_t>(j)),
+                     sfa + (static_cast<uint32_t>(j) << 30),
+                     sfb + 8 * h + (static_cast<uint32_t>(j) << 30), (kb | j) != 0);
           mma_commit(bars.op_empty(s));
           if (++s == C::kOpStages) { s = 0; ph ^= 1u; }
         }
         mma_commit(bars.acc_full(buf));
       }
     }
-  } else if (warp < 2 + kEpiWarps) {  // epilogue: TMEM lanes 32 * (warp & 3) ..
+  } else if (warp < 2 + C::kEpiW) {  // epilogue: TMEM lanes 32 * (warp & 3) ..
     const int quad = warp & 3;
+    const int hh = (warp - 2) >> 2;  // N-half of the tile
     const int et = threadIdx.x - 64;
+    constexpr int kEpiT = 32 * C::kEpiW;
     int it = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
-      const int buf = it & 1;
-      const uint32_t aph = (it >> 1) & 1;
+      const int buf = it % C::kAccBufs;
+      const uint32_t aph = (it / C::kAccBufs) & 1;
       int m0, n0;
-      tile_origin(t, m_tiles, n_tiles, m0, n0);
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      for (int i = et; i < BN; i += 128) {
+      tile_origin(t, m_tiles, n_tiles, C::kGroup, C::kBN, m0, n0);
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiT) : "memory");
+      for (int i = et; i < C::kBN; i += kEpiT) {
         const int n = n0 + i;
         epi_b[i] = (n < N && bias) ? __uint_as_float(static_cast<uint32_t>(bias[n]) << 16) : 0.f;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiT) : "memory");
+      n0 += hh * BN;  // this warp's columns
+      const float* e_b = epi_b + hh * BN;
       if (!mbar_wait_bounded(bars.acc_full(buf), aph, abort_flag, kErrWaitEpilogue)) break;
       tc_fence_after();
       const int row = m0 + 32 * quad + lane;
@@ -363,7 +396,7 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
         }
       }
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quad) << 16) +
-                             static_cast<uint32_t>(buf * BN);
+                             static_cast<uint32_t>(buf * BN + hh * BN);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
@@ -374,8 +407,8 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const float y0 = __fadd_rn(__uint_as_float(r[2 * j]), epi_b[32 * c + 2 * j]);
-            const float y1 = __fadd_rn(__uint_as_float(r[2 * j + 1]), epi_b[32 * c + 2 * j + 1]);
+            const float y0 = __fadd_rn(__uint_as_float(r[2 * j]), e_b[32 * c + 2 * j]);
+            const float y1 = __fadd_rn(__uint_as_float(r[2 * j + 1]), e_b[32 * c + 2 * j + 1]);
             const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
             pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
           }
@@ -388,7 +421,7 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
       if (lane == 0) mbar_arrive(bars.acc_empty(buf));
     }
   } else {  // decode warps
-    const int dt = threadIdx.x - 32 * (2 + kEpiWarps);  // 0 .. kDecThreads - 1
+    const int dt = threadIdx.x - 32 * (2 + C::kEpiW);  // 0 .. kDecThreads - 1
     int s = 0, so = 0, ms = 0;
     uint32_t ph = 0, pho = 0, mph = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
@@ -440,10 +473,10 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
         }
         // the scales of the operands loaded as e4m3: one 4-byte word per row
         // (x rows 0..127, then W rows)
-        constexpr int kDirectRows = (ADEC ? 0 : BM) + (BDEC ? 0 : BN);
+        constexpr int kDirectRows = (ADEC ? 0 : BM) + (BDEC ? 0 : C::kBN);
         for (int i = dt; i < kDirectRows; i += C::kDecThreads) {
           const bool is_b = ADEC || i >= BM;
-          const int rr = ADEC ? i : (i >= BM ? i - BM : i);
+          const int rr = ADEC ? i : (i >= BM ? i - BM : i);  // W rows of both N-halves in turn
           const uint8_t* wp = mt + (is_b ? kMetaA : 0) + rr * 16 + (kb & 1) * 8;
           const uint32_t wv[2] = {*reinterpret_cast<const uint32_t*>(wp),
                                   *reinterpret_cast<const uint32_t*>(wp + 4)};
@@ -454,7 +487,10 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC>::kThreads, 1)
                      static_cast<int>(static_cast<int8_t>((wv[k >> 1] >> (16 * (k & 1))) & 0xFFu)) +
                      127)
                  << (8 * k);
-          *reinterpret_cast<uint32_t*>(sf + (is_b ? kSfA : 0) + sf_row_offset(rr)) = v;
+          // W rows: the scale blocks of their N-half (1024 bytes each)
+          const int off = is_b ? kSfA + (rr / BN) * kSfB + sf_row_offset(rr % BN)
+                               : sf_row_offset(rr);
+          *reinterpret_cast<uint32_t*>(sf + off) = v;
         }
         fence_proxy_async_smem();
         __syncwarp();
