@@ -392,6 +392,29 @@ def test_multi_tile_grid_every_element(bx, bw, flags):
     assert assert_within_1ulp(got, want, "multi-tile") == 1.0
 
 
+@pytest.mark.parametrize("bx,bw,flags", MULTI_TILE_FORMS, ids=["w4a4", "w4a4_bytes", "w8a8", "w4a8"])
+def test_wide_tile_ragged_edges_every_element(bx, bw, flags):
+    """N = 2320 = 4 x 512 + 272: the last 256 x 512 tile has a full first
+    N-half and 16 columns of its second; M = 1000 ends in a ragged M-tile
+    (232 rows); K = 5120 as in the Wan FFN.  Every code, scale, accumulator
+    and output against the oracle."""
+    M, N, K, alpha = 1000, 2320, 5120, 0.9
+    d = I.make_shape(seed=2320 + 10 * bx + bw, M=M, K=K, N=N, bits=bw, alpha=alpha,
+                     outlier_factor=100.0, outlier_frac=0.005, sigma_w=0.015,
+                     bits_x=bx if bx != bw else 0)
+    g = run_layer(d, bw, alpha, bits_x=bx, x_flags=flags)
+    qa, sa = O.quant_act(bits16(d["x"]), bx, alpha)
+    qw, sw = O.pack_weights(bits16(d["w"]), bw)
+    assert np.array_equal(g["xs"].cpu().numpy().view(np.uint32), sa.view(np.uint32))
+    assert np.array_equal(g["xp"].cpu().numpy(), O.pack(qa, qs.storage_bits(bx, flags)))
+    assert np.array_equal(g["wp"].cpu().numpy(), O.pack(qw, bw))
+    acc = O.int_gemm_f64(qa, qw)
+    assert np.array_equal(g["acc"].cpu().numpy().astype(np.int64), acc)
+    want = O.epilogue(acc, sa, sw, bits16(d["bias"]))
+    got = g["out"].view(torch.int16).cpu().numpy().view(np.uint16)
+    assert assert_within_1ulp(got, want, "ragged wide tile") == 1.0
+
+
 def test_w8a8_band_edge_small():
     """The 8-bit x 8-bit form walks N-tiles in bands of 18: N = 5120 has 20
     N-tiles (a full band and a last band of 2), M = 300 a ragged second M-tile.
