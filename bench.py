@@ -642,6 +642,17 @@ def sd4_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
         q8 = timed(lambda: qs.qs_sd4_quant_e4m3(x, M, K, x8, m8, stream))
         g88 = timed(lambda: qs.qs_sd4_linear_e4m3(x8, m8, w8, mw, b, M, N, K, out88, stream))
         same88 = bool(torch.equal(out.view(torch.int16), out88.view(torch.int16)))
+        # the scales pre-arranged as the GEMM copies them (weights offline,
+        # activations by one small pass per call): no block-word conversion
+        # inside the GEMM
+        xt = qs.sd4_scale_tiles(m8, False, stream=stream)
+        wt = qs.sd4_scale_tiles(mw, True, stream=stream)
+        out_t = torch.empty_like(out)
+        qs.qs_sd4_linear_e4m3_tiles(x8, xt, w8, wt, b, M, N, K, out_t, stream)
+        qt = timed(lambda: qs.qs_sd4_scale_tiles(m8, M, K, 0, xt, stream))
+        gt = timed(lambda: qs.qs_sd4_linear_e4m3_tiles(x8, xt, w8, wt, b, M, N, K, out_t,
+                                                       stream))
+        same_t = bool(torch.equal(out.view(torch.int16), out_t.view(torch.int16)))
         # activation decomposition of the salient tokens (a seeded 1/16 of them)
         srows = I.salient_rows(M, cfg.seed)
         S_ = len(srows)
@@ -693,6 +704,11 @@ def sd4_layer(qs, torch, I, dev, stream, steps=5, warmup=2, rows=256):
             "gemm_e4m3_both_frac_fp8_peak": tf(g88) / fp8_peak,
             "e4m3_both_output_identical": same88,
             "layer_e4m3_ms": q8 + g88, "layer_e4m3_TOPS": cfg.ops / ((q8 + g88) * 1e-3) / 1e12,
+            "scale_tiles_ms": qt, "gemm_e4m3_tiles_ms": gt, "gemm_e4m3_tiles_TFLOPS": tf(gt),
+            "gemm_e4m3_tiles_frac_fp8_peak": tf(gt) / fp8_peak,
+            "e4m3_tiles_output_identical": same_t,
+            "layer_e4m3_tiles_ms": q8 + qt + gt,
+            "layer_e4m3_tiles_TOPS": cfg.ops / ((q8 + qt + gt) * 1e-3) / 1e12,
             "gemm_bf16_weights_ms": g2, "gemm_bf16_weights_TFLOPS": tf(g2),
             "gemm_bf16_weights_frac_bf16_peak": tf(g2) / pk["bf16_tflops"],
             "quant_GBps": quant_bytes / (q * 1e-3) / 1e9,

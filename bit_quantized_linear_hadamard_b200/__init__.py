@@ -13,7 +13,8 @@ from .binding import (  # noqa: F401
     storage_bits, qs_sd4_quant, sd4_quant, qs_sd4_linear, sd4_linear, qs_sd4_decode, sd4_decode,
     qs_sd4_linear_wdec, qs_sd4_quant_decomp, qs_sd4_linear_decomp, sd4_quant_decomp,
     sd4_linear_decomp, qs_sd4_decode_e4m3, sd4_decode_e4m3, qs_sd4_linear_e4m3w,
-    qs_sd4_quant_e4m3, sd4_quant_e4m3, qs_sd4_linear_e4m3,
+    qs_sd4_quant_e4m3, sd4_quant_e4m3, qs_sd4_linear_e4m3, qs_sd4_scale_tiles_bytes,
+    qs_sd4_scale_tiles, sd4_scale_tiles, qs_sd4_linear_e4m3_tiles,
     pack_weights, packed_cols, qgemm_s32, qlinear, qs_device_error, qs_gelu_bf16, qs_linear,
     qs_linear_mixed, qs_linear_workspace_bytes, qs_pack_weights, qs_qgemm_s32, qs_qgemm_s32_mixed,
     qs_qlinear, qs_qlinear_mixed, qs_quant_act, qs_selftest_timeout, qs_version, quant_act,

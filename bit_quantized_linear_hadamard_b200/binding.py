@@ -33,7 +33,8 @@ EXPORTS = ("qs_pack_weights", "qs_quant_act", "qs_qlinear", "qs_qlinear_mixed", 
            "qs_quant_act_rowsum", "qs_qlinear_asym", "qs_qgemm_s32_asym",
            "qs_linear_bgr_workspace_bytes", "qs_linear_bgr", "qs_sd4_quant", "qs_sd4_quant_e4m3",
            "qs_sd4_linear", "qs_sd4_decode", "qs_sd4_linear_wdec", "qs_sd4_decode_e4m3",
-           "qs_sd4_linear_e4m3w", "qs_sd4_linear_e4m3", "qs_sd4_quant_decomp",
+           "qs_sd4_linear_e4m3w", "qs_sd4_linear_e4m3", "qs_sd4_scale_tiles_bytes",
+           "qs_sd4_scale_tiles", "qs_sd4_linear_e4m3_tiles", "qs_sd4_quant_decomp",
            "qs_sd4_linear_decomp", "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs",
            "qs_selftest_timeout", "qs_device_error", "qs_status_str", "qs_version")
 BITS = (4, 6, 8)
@@ -93,6 +94,10 @@ def load() -> ctypes.CDLL:
     L.qs_sd4_linear_e4m3w.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]
     L.qs_sd4_quant_e4m3.argtypes = [vp, i64, i64, vp, vp, vp]
     L.qs_sd4_linear_e4m3.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]
+    L.qs_sd4_scale_tiles_bytes.argtypes = [i64, i64, i32]
+    L.qs_sd4_scale_tiles_bytes.restype = i64
+    L.qs_sd4_scale_tiles.argtypes = [vp, i64, i64, i32, vp, i64, vp]
+    L.qs_sd4_linear_e4m3_tiles.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]
     L.qs_gbs_reset.argtypes = [vp, vp]
     L.qs_gbs_update.argtypes = [vp, vp, i64, f64, vp, vp]
     L.qs_linear_gbs.argtypes = [vp, i64, i64, f32, vp, vp, vp, vp, vp, i64, vp, vp, i64, vp, vp]
@@ -107,7 +112,8 @@ def load() -> ctypes.CDLL:
                  "qs_quant_act_rowsum", "qs_qlinear_asym", "qs_qgemm_s32_asym", "qs_linear_bgr",
                  "qs_sd4_quant", "qs_sd4_quant_e4m3", "qs_sd4_linear", "qs_sd4_decode",
                  "qs_sd4_linear_wdec", "qs_sd4_decode_e4m3", "qs_sd4_linear_e4m3w",
-                 "qs_sd4_linear_e4m3", "qs_sd4_quant_decomp", "qs_sd4_linear_decomp",
+                 "qs_sd4_linear_e4m3", "qs_sd4_scale_tiles", "qs_sd4_linear_e4m3_tiles",
+                 "qs_sd4_quant_decomp", "qs_sd4_linear_decomp",
                  "qs_gbs_reset", "qs_gbs_update", "qs_linear_gbs", "qs_selftest_timeout",
                  "qs_device_error"):
         getattr(L, name).restype = ctypes.c_int
@@ -480,6 +486,38 @@ def qs_sd4_linear_e4m3(x_e4m3, x_meta, w_e4m3, w_meta, bias, M, N, K, out, strea
         _cuda(t, dt, name)
     _check(load().qs_sd4_linear_e4m3(_p(x_e4m3), _p(x_meta), _p(w_e4m3), _p(w_meta), _p(bias),
                                      M, N, K, _p(out), _s(stream)), "qs_sd4_linear_e4m3")
+
+
+def qs_sd4_scale_tiles_bytes(rows: int, K: int, weights: int) -> int:
+    return int(load().qs_sd4_scale_tiles_bytes(rows, K, weights))
+
+
+def qs_sd4_scale_tiles(meta, rows, K, weights, tiles, stream=None):
+    _cuda(meta, torch.int16, "meta")
+    _cuda(tiles, torch.uint8, "tiles")
+    _check(load().qs_sd4_scale_tiles(_p(meta), rows, K, weights, _p(tiles), tiles.numel(),
+                                     _s(stream)), "qs_sd4_scale_tiles")
+
+
+def sd4_scale_tiles(meta: torch.Tensor, weights: bool, stream=None) -> torch.Tensor:
+    """Block words [rows, K/32] -> the GEMM's pre-arranged scale tiles (uint8)."""
+    rows, K = meta.shape[0], meta.shape[1] * 32
+    need = qs_sd4_scale_tiles_bytes(rows, K, int(weights))
+    if need < 0:
+        raise QSError(2, f"qs_sd4_scale_tiles_bytes({rows}, {K})")
+    tiles = torch.empty((need,), dtype=torch.uint8, device=meta.device)
+    qs_sd4_scale_tiles(meta, rows, K, int(weights), tiles, stream)
+    return tiles
+
+
+def qs_sd4_linear_e4m3_tiles(x_e4m3, x_tiles, w_e4m3, w_tiles, bias, M, N, K, out, stream=None):
+    for t, name, dt in ((x_e4m3, "x_e4m3", torch.uint8), (x_tiles, "x_tiles", torch.uint8),
+                        (w_e4m3, "w_e4m3", torch.uint8), (w_tiles, "w_tiles", torch.uint8),
+                        (bias, "bias", torch.bfloat16), (out, "out", torch.bfloat16)):
+        _cuda(t, dt, name)
+    _check(load().qs_sd4_linear_e4m3_tiles(_p(x_e4m3), _p(x_tiles), _p(w_e4m3), _p(w_tiles),
+                                           _p(bias), M, N, K, _p(out), _s(stream)),
+           "qs_sd4_linear_e4m3_tiles")
 
 
 def qs_gbs_reset(state, stream=None):

@@ -161,15 +161,16 @@ qs_status launch_sd4_gemm(const CUtensorMap& ca, const CUtensorMap& cb, const CU
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
-template <bool ADEC, bool BDEC, bool WIDE = false>
+template <bool ADEC, bool BDEC, bool WIDE = false, bool TILES = false>
 qs_status launch_sd4_mx(const CUtensorMap& ca, const CUtensorMap& cb, const CUtensorMap& ma,
                         const CUtensorMap& mb, const CUtensorMap& xa, const CUtensorMap& wb,
                         const void* bias, int64_t M, int64_t N, int64_t K, void* out,
-                        void* stream, int64_t kb_wrap, const int32_t* out_rows, int64_t out_M) {
+                        void* stream, int64_t kb_wrap, const int32_t* out_rows, int64_t out_M,
+                        const void* a_tiles = nullptr, const void* b_tiles = nullptr) {
   namespace G = qs::sd4::gemm_mx;
-  using C = G::MCfg<ADEC, BDEC, WIDE>;
+  using C = G::MCfg<ADEC, BDEC, WIDE, TILES>;
   constexpr int smem = C::kSmemBytes;
-  auto kern = G::sd4_mx_gemm_kernel<ADEC, BDEC, WIDE>;
+  auto kern = G::sd4_mx_gemm_kernel<ADEC, BDEC, WIDE, TILES>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return QS_ERR_CUDA;
@@ -180,7 +181,8 @@ qs_status launch_sd4_mx(const CUtensorMap& ca, const CUtensorMap& cb, const CUte
   kern<<<grid, C::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(
       ca, cb, ma, mb, xa, wb, static_cast<const uint16_t*>(bias), static_cast<uint16_t*>(out),
       static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(kb_wrap),
-      out_rows, static_cast<int>(out_rows ? out_M : M));
+      out_rows, static_cast<int>(out_rows ? out_M : M), static_cast<const uint8_t*>(a_tiles),
+      static_cast<const uint8_t*>(b_tiles));
   return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
 }
 
@@ -685,6 +687,67 @@ qs_status qs_sd4_linear_e4m3(const void* x_e4m3, const uint16_t* x_meta, const v
   if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
   return run_sd4_mx(nullptr, x_e4m3, x_meta, M, K, nullptr, w_e4m3, w_meta, bias_bf16, N, K,
                     out_bf16, stream, nullptr, 0);
+}
+
+int64_t qs_sd4_scale_tiles_bytes(int64_t rows, int64_t K, int weights) {
+  namespace G = qs::sd4::gemm_mx;
+  if (rows <= 0 || K <= 0 || K % 256 != 0 || K > QS_MAX_K || rows > QS_MAX_ROWS) return -1;
+  const int64_t kbs = K / G::BK;
+  if (weights) {  // groups of BN rows, whole 2-group tiles: 1024 bytes per group and stage
+    const int64_t groups = 2 * ((rows + 2 * G::BN - 1) / (2 * G::BN));
+    return groups * kbs * 2 * 512;
+  }
+  return ((rows + G::BM - 1) / G::BM) * kbs * 512;  // groups of BM rows
+}
+
+qs_status qs_sd4_scale_tiles(const uint16_t* meta, int64_t rows, int64_t K, int weights,
+                             void* tiles, int64_t tiles_bytes, void* stream) {
+  namespace G = qs::sd4::gemm_mx;
+  if (!meta || !tiles) return QS_ERR_NULL;
+  if (rows <= 0 || K <= 0 || K % 256 != 0) return QS_ERR_SHAPE;
+  if (K > QS_MAX_K || rows > QS_MAX_ROWS || (weights != 0 && weights != 1)) return QS_ERR_RANGE;
+  const int64_t need = qs_sd4_scale_tiles_bytes(rows, K, weights);
+  if (tiles_bytes < need) return QS_ERR_RANGE;
+  if (!aligned16(meta) || !aligned16(tiles)) return QS_ERR_ALIGN;
+  QS_TRY(check_device_ptr(meta));
+  QS_TRY(check_device_ptr(tiles));
+  const int group = weights ? G::BN : G::BM;
+  const int slots = weights ? 256 : 128;
+  const int64_t groups = need / ((K / G::BK) * (slots / 128) * 512);
+  const int sms = qs::sm_count();
+  if (sms <= 0) return QS_ERR_CUDA;
+  const int64_t tasks = groups * (K / G::BK) * slots;
+  int64_t grid = (tasks + 255) / 256;
+  if (grid > static_cast<int64_t>(sms) * 8) grid = static_cast<int64_t>(sms) * 8;
+  G::sd4_scale_tiles_kernel<<<static_cast<unsigned>(grid), 256, 0,
+                              static_cast<cudaStream_t>(stream)>>>(
+      meta, rows, static_cast<int>(K), group, slots, groups, static_cast<uint8_t*>(tiles));
+  return cudaGetLastError() == cudaSuccess ? QS_OK : QS_ERR_CUDA;
+}
+
+qs_status qs_sd4_linear_e4m3_tiles(const void* x_e4m3, const void* x_tiles, const void* w_e4m3,
+                                   const void* w_tiles, const void* bias_bf16, int64_t M,
+                                   int64_t N, int64_t K, void* out_bf16, void* stream) {
+  namespace G = qs::sd4::gemm_mx;
+  if (!x_e4m3 || !x_tiles || !w_e4m3 || !w_tiles || !out_bf16) return QS_ERR_NULL;
+  if (M <= 0 || N <= 0 || K <= 0 || K % 256 != 0 || N % 16 != 0) return QS_ERR_SHAPE;
+  if (K > QS_MAX_K || M > INT32_MAX || N > INT32_MAX) return QS_ERR_RANGE;
+  if (!aligned16(x_e4m3) || !aligned16(x_tiles) || !aligned16(w_e4m3) || !aligned16(w_tiles) ||
+      !aligned16(out_bf16) || (bias_bf16 && !aligned16(bias_bf16)))
+    return QS_ERR_ALIGN;
+  for (const void* p : {x_e4m3, x_tiles, w_e4m3, w_tiles, static_cast<const void*>(out_bf16)})
+    QS_TRY(check_device_ptr(p));
+  if (bias_bf16) QS_TRY(check_device_ptr(bias_bf16));
+  CUtensorMap xa, wb;
+  if (!qs::make_tensor_map_2d(&xa, x_e4m3, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                              G::BK, G::BM, true) ||
+      !qs::make_tensor_map_2d(&wb, w_e4m3, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                              G::BK, G::BN, true))
+    return QS_ERR_CUDA;
+  // the block-word maps are not read with pre-arranged scales
+  return launch_sd4_mx<false, false, true, true>(xa, xa, xa, xa, xa, wb, bias_bf16, M, N, K,
+                                                 out_bf16, stream, K / G::BK, nullptr, 0,
+                                                 x_tiles, w_tiles);
 }
 
 qs_status qs_sd4_decode(const void* codes, const uint16_t* meta, int64_t rows, int64_t K,

@@ -60,9 +60,13 @@ static_assert(BN % 32 == 0 && BN <= 256 && 2 * BN + 12 <= kTmemCols, "tile");
 // step reading the same x tile, into one 384-column accumulator (the scales
 // take 4 + 16 more columns, so a second accumulator does not fit); eight
 // epilogue warps, one per TMEM lane quarter and N-half.
-template <bool ADEC, bool BDEC, bool WIDE = false>
+// TILES (wide tiles only): the scale bytes come pre-arranged in the
+// tensor-memory copy layout (qs_sd4_scale_tiles) and are bulk-copied with the
+// operands, so the kernel has no decode warps.
+template <bool ADEC, bool BDEC, bool WIDE = false, bool TILES = false>
 struct MCfg {
   static_assert(!WIDE || (!ADEC && !BDEC), "wide tiles for e4m3 operands only");
+  static_assert(!TILES || WIDE, "pre-arranged scales with wide tiles only");
   static constexpr bool kAnyDec = ADEC || BDEC;
   static constexpr int kHalves = WIDE ? 2 : 1;
   static constexpr int kBN = kHalves * BN;          // tile columns
@@ -72,7 +76,7 @@ struct MCfg {
   // decode warps (for e4m3 operands they only turn block words into scale
   // bytes; with wide tiles, 512 rows per stage: 8 warps measured 1.995
   // against 2.148 ms for 4 and 2.020 ms for 16 at the Wan FFN shape)
-  static constexpr int kDecWarps = ADEC ? (BDEC ? 10 : 8) : (WIDE ? 8 : 4);
+  static constexpr int kDecWarps = TILES ? 0 : (ADEC ? (BDEC ? 10 : 8) : (WIDE ? 8 : 4));
   static constexpr int kDecThreads = 32 * kDecWarps;
   static constexpr int kThreads = 32 * (2 + kEpiW + kDecWarps);
   // operand stages by measurement (e4m3 x e4m3 at the Wan FFN shape: 3 stages
@@ -80,7 +84,7 @@ struct MCfg {
   // gain); wide tiles: as many as fit
   static constexpr int kOpStages = (BDEC || WIDE) ? 3 : 4;
   static constexpr int kPkStages = kAnyDec ? kOpStages : 0;
-  static constexpr int kMetaSlots = 2;
+  static constexpr int kMetaSlots = TILES ? 0 : 2;
   static constexpr int kDecRows = (ADEC ? BM : 0) + (BDEC ? BN : 0);  // rows decoded per stage
   static constexpr int kTasks = 2 * kDecRows;  // (row, half of the stage's K)
   static constexpr int kOpStage = kOpA + kHalves * kOpB;
@@ -104,7 +108,10 @@ struct MCfg {
   static constexpr int kOpFullCount = kDecWarps + (kDirectBytes ? 1 : 0);
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
   static_assert(kOffSf % 1024 == 0 && kOffPk % 128 == 0 && kOffMeta % 128 == 0, "alignment");
-  static_assert(kTasks % kDecThreads == 0, "decode split");
+  static_assert(kTasks % (kDecThreads > 0 ? kDecThreads : 1) == 0, "decode split");
+  // bytes completing an operand stage by TMA: direct operands and, with
+  // TILES, the stage's scale tiles
+  static constexpr int kStageTx = kDirectBytes + (TILES ? kSfStage : 0);
   static_assert(!BDEC || ADEC, "codes for W with e4m3 x is not a form of this kernel");
 };
 
@@ -128,6 +135,16 @@ __device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_
       "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::
           "r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Global -> this CTA's shared memory, `bytes` contiguous (16-byte aligned,
+// a multiple of 16), completing as transaction bytes on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
 
@@ -209,9 +226,10 @@ __device__ __forceinline__ int sf_row_offset(int m) {
 // maps accumulator row m to its output row; an index outside [0, out_M) is
 // skipped and flagged.
 // tmCA / tmCB: the codes (when decoded), tmXA / tmWB: the e4m3 bytes (when
-// loaded directly), tmMA / tmMB: the block words.
-template <bool ADEC, bool BDEC, bool WIDE>
-__global__ void __launch_bounds__(MCfg<ADEC, BDEC, WIDE>::kThreads, 1)
+// loaded directly), tmMA / tmMB: the block words; a_tiles / b_tiles: the
+// scale tiles (TILES; qs_sd4_scale_tiles layout).
+template <bool ADEC, bool BDEC, bool WIDE, bool TILES>
+__global__ void __launch_bounds__(MCfg<ADEC, BDEC, WIDE, TILES>::kThreads, 1)
     sd4_mx_gemm_kernel(const __grid_constant__ CUtensorMap tmCA,
                        const __grid_constant__ CUtensorMap tmCB,
                        const __grid_constant__ CUtensorMap tmMA,
@@ -219,8 +237,9 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC, WIDE>::kThreads, 1)
                        const __grid_constant__ CUtensorMap tmXA,
                        const __grid_constant__ CUtensorMap tmWB, const uint16_t* __restrict__ bias,
                        uint16_t* __restrict__ out, int M, int N, int K, int kb_wrap,
-                       const int32_t* __restrict__ out_rows, int out_M) {
-  using C = MCfg<ADEC, BDEC, WIDE>;
+                       const int32_t* __restrict__ out_rows, int out_M,
+                       const uint8_t* __restrict__ a_tiles, const uint8_t* __restrict__ b_tiles) {
+  using C = MCfg<ADEC, BDEC, WIDE, TILES>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
@@ -289,7 +308,7 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC, WIDE>::kThreads, 1)
         for (int kb = 0, kbw = 0; kb < kblocks; ++kb, kbw = (kbw + 1 == kb_wrap ? 0 : kbw + 1)) {
           // kbw: the weights' K-block; kb_wrap is even, so both stay in step
           // with the two-stage block-word slots
-          if ((kb & 1) == 0) {
+          if (!TILES && (kb & 1) == 0) {
             if (!mbar_wait_bounded(bars.meta_empty(ms), mph ^ 1u, abort_flag, kErrWaitProducer))
               break;
             const uint32_t dst = sbase + C::kOffMeta + ms * C::kMetaSlot;
@@ -315,16 +334,32 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC, WIDE>::kThreads, 1)
             if (!mbar_wait_bounded(bars.op_empty(so), pho ^ 1u, abort_flag, kErrWaitProducer))
               break;
             const uint32_t ob = sbase + C::kOffOp + so * C::kOpStage;
-            mbar_arrive_expect_tx(bars.op_full(so), C::kDirectBytes);
+            mbar_arrive_expect_tx(bars.op_full(so), C::kStageTx);
             if (!ADEC) tma_load_2d(ob, &tmXA, kb * BK, m0, bars.op_full(so));
             if (!BDEC)
 #pragma unroll
               for (int h = 0; h < C::kHalves; ++h)
                 tma_load_2d(ob + kOpA + h * kOpB, &tmWB, kbw * BK, n0 + h * BN, bars.op_full(so));
+            if (TILES) {  // the stage's scale tiles: x rows m0.., W rows n0.. per N-half
+              const uint32_t f0 = sbase + C::kOffSf + so * C::kSfStage;
+              bulk_load(f0, a_tiles + (static_cast<int64_t>(m0 / BM) * kblocks + kb) * kSfA, kSfA,
+                        bars.op_full(so));
+#pragma unroll
+              for (int h = 0; h < C::kHalves; ++h)
+                bulk_load(f0 + kSfA + h * kSfB,
+                          b_tiles + (static_cast<int64_t>(n0 / BN + h) * kb_wrap + kbw) * kSfB,
+                          kSfB, bars.op_full(so));
+            }
             if (++so == C::kOpStages) { so = 0; pho ^= 1u; }
           }
         }
       }
+      if (TILES)  // no decode warps: the producer waits for the last releases
+        for (int i = 0; i < C::kOpStages; ++i) {
+          if (!mbar_wait_bounded(bars.op_empty(so), pho ^ 1u, abort_flag, kErrWaitProducer))
+            break;
+          if (++so == C::kOpStages) { so = 0; pho ^= 1u; }
+        }
     }
   } else if (warp == 1) {
     if (lane == 0) {  // MMA issuer
@@ -423,7 +458,7 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC, WIDE>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.acc_empty(buf));
     }
-  } else {  // decode warps
+  } else if constexpr (C::kDecWarps > 0) {  // decode warps
     const int dt = threadIdx.x - 32 * (2 + C::kEpiW);  // 0 .. kDecThreads - 1
     int s = 0, so = 0, ms = 0;
     uint32_t ph = 0, pho = 0, mph = 0;
@@ -554,6 +589,41 @@ __global__ void __launch_bounds__(256) sd4_decode_e4m3_kernel(const uint8_t* __r
     const uint2 lo = decode8_e4m3(cw.x, E), hi = decode8_e4m3(cw.y, E);
     *reinterpret_cast<uint4*>(out + row * static_cast<int64_t>(K) + c * 16) =
         make_uint4(lo.x, lo.y, hi.x, hi.y);
+  }
+}
+
+// Scale tiles: the UE8M0 scale bytes (e + 127) of an SD4 matrix, arranged as
+// the GEMM copies them into tensor memory, so that one stage's scales are one
+// contiguous block for a bulk copy.  Rows go in groups of `group` (BM = 128
+// for activations, BN = 192, one N-half, for weights), padded to `slots`
+// rows (128 or 256); tile (g, kb) holds slots / 128 blocks of 512 bytes, row
+// r of the group and K-block j of the stage at byte sf_row_offset(r) + j.
+// Rows past `rows` or past the group's size are zero.  One thread per row
+// slot of a tile.
+__global__ void __launch_bounds__(256) sd4_scale_tiles_kernel(const uint16_t* __restrict__ meta,
+                                                              int64_t rows, int K, int group,
+                                                              int slots, int64_t groups,
+                                                              uint8_t* __restrict__ tiles) {
+  const int kbs = K / BK;
+  const int64_t n = groups * kbs * slots;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < n;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int slot = static_cast<int>(t % slots);
+    const int64_t gk = t / slots;  // g * kbs + kb
+    const int kb = static_cast<int>(gk % kbs);
+    const int64_t row = (gk / kbs) * group + slot;
+    uint32_t v = 0;
+    if (slot < group && row < rows) {
+      const uint2 w = *reinterpret_cast<const uint2*>(meta + row * (K / 32) + kb * 4);
+      const uint32_t wv[2] = {w.x, w.y};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        v |= static_cast<uint32_t>(
+                 static_cast<int>(static_cast<int8_t>((wv[k >> 1] >> (16 * (k & 1))) & 0xFFu)) +
+                 127)
+             << (8 * k);
+    }
+    *reinterpret_cast<uint32_t*>(tiles + gk * (slots / 128) * 512 + sf_row_offset(slot)) = v;
   }
 }
 

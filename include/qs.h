@@ -381,6 +381,38 @@ QS_API qs_status qs_sd4_linear_e4m3(const void* x_e4m3, const uint16_t* x_meta,
                                     void* out_bf16, void* stream);
 
 /*
+ * qs_sd4_scale_tiles — the UE8M0 scale bytes (e + 127) of an SD4 matrix's
+ * block words, arranged as the SD4 GEMM copies them into tensor memory, so
+ * that qs_sd4_linear_e4m3_tiles loads them with the operands instead of
+ * converting block words in the kernel.  Rows go in groups of 128
+ * (weights = 0: activations) or 192 (weights = 1: one N-half of the GEMM's
+ * 384-column tile; the group count is rounded up to even), each group padded
+ * to 128 or 256 rows; per group and 128-element K step one tile of 512 or
+ * 1024 bytes: row r of the group, 32-element block j of the step at byte
+ * 512 (r / 128) + 16 (r % 32) + 4 ((r % 128) / 32) + j.  Padding rows are 0.
+ *   meta   [rows, K/32] block words (qs_sd4_quant, qs_sd4_quant_e4m3)
+ *   tiles  qs_sd4_scale_tiles_bytes(rows, K, weights) bytes, written;
+ *          tiles_bytes: its size (QS_ERR_RANGE if smaller)
+ * qs_sd4_scale_tiles_bytes returns -1 for an invalid shape.
+ */
+QS_API int64_t qs_sd4_scale_tiles_bytes(int64_t rows, int64_t K, int weights);
+QS_API qs_status qs_sd4_scale_tiles(const uint16_t* meta, int64_t rows, int64_t K, int weights,
+                                    void* tiles, int64_t tiles_bytes, void* stream);
+
+/*
+ * qs_sd4_linear_e4m3_tiles — qs_sd4_linear_e4m3 with the scales given as
+ * qs_sd4_scale_tiles of the activations (weights = 0) and of the weights
+ * (weights = 1): the GEMM copies operands and scales, nothing else.  The same
+ * arithmetic, bit-identical output.
+ *   x_e4m3 [M, K], x_tiles, w_e4m3 [N, K], w_tiles; other arguments as
+ *   qs_sd4_linear_e4m3
+ */
+QS_API qs_status qs_sd4_linear_e4m3_tiles(const void* x_e4m3, const void* x_tiles,
+                                          const void* w_e4m3, const void* w_tiles,
+                                          const void* bias_bf16, int64_t M, int64_t N, int64_t K,
+                                          void* out_bf16, void* stream);
+
+/*
  * Activation decomposition (SemanticDialect "Resumen técnico" §2.B): a salient
  * activation row A is split into its SD4 value Q(A) and the residual
  * Delta = A - x_hat, which is quantised again with the same format, and the

@@ -294,3 +294,30 @@ def test_sd4_validation(lib):
     assert f8(A, B, C, NUL, NUL, 8, 256, 256, D, NUL) == NULL
     assert f8(A, B, C, D, NUL, 8, 248, 256, D, NUL) == SHAPE
     assert f8(MIS, B, C, D, NUL, 8, 256, 256, D, NUL) == ALIGN
+
+
+def test_sd4_scale_tiles_sizes_and_validation(lib):
+    nb = lib.qs_sd4_scale_tiles_bytes
+    # activations: groups of 128 rows, 512 bytes per group and 128-element K step
+    assert nb(128, 256, 0) == 1 * 2 * 512
+    assert nb(129, 256, 0) == 2 * 2 * 512
+    assert nb(32760, 5120, 0) == 256 * 40 * 512
+    # weights: groups of 192 rows in whole pairs (one 384-column GEMM tile), 1024 bytes
+    assert nb(16, 256, 1) == 2 * 2 * 1024
+    assert nb(384, 256, 1) == 2 * 2 * 1024
+    assert nb(385, 256, 1) == 4 * 2 * 1024
+    assert nb(13824, 5120, 1) == 72 * 40 * 1024
+    assert nb(0, 256, 0) == -1 and nb(8, 384, 0) == -1 and nb(8, 256 + 65536, 1) == -1
+    t = lib.qs_sd4_scale_tiles
+    need = nb(8, 256, 0)
+    assert t(NUL, 8, 256, 0, B, need, NUL) == NULL
+    assert t(A, 8, 384, 0, B, need, NUL) == SHAPE
+    assert t(A, 8, 256, 2, B, need, NUL) == RANGE
+    assert t(A, 8, 256, 0, B, need - 16, NUL) == RANGE      # buffer too small
+    assert t(MIS, 8, 256, 0, B, need, NUL) == ALIGN
+    g = lib.qs_sd4_linear_e4m3_tiles
+    assert g(A, NUL, C, D, NUL, 8, 256, 256, D, NUL) == NULL
+    assert g(A, B, C, D, NUL, 8, 248, 256, D, NUL) == SHAPE
+    assert g(A, B, C, D, NUL, 8, 256, 384, D, NUL) == SHAPE
+    assert g(A, B, C, D, NUL, 8, 256, 65536 + 256, D, NUL) == RANGE
+    assert g(A, MIS, C, D, NUL, 8, 256, 256, D, NUL) == ALIGN

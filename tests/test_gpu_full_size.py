@@ -239,7 +239,7 @@ def test_full_size_sd4_every_element():
     decomposition of a seeded 1/16 of the tokens (§2.B): every activation and
     weight code and block word, every e4m3 byte and decoded bf16 weight
     bit-identical to the oracle; every output of the codes form (with the
-    e4m3 forms bit-identical to it) and of the bf16-weight form, and every
+    e4m3 forms, also with pre-arranged scale tiles, bit-identical to it) and of the bf16-weight form, and every
     decomposed row's codes, block words and outputs, within the
     binary32-accumulation bound of the oracle's exact-product layer, with
     more than 99 % of them bit-identical to the oracle's rounding."""
@@ -258,6 +258,9 @@ def test_full_size_sd4_every_element():
     qs.qs_sd4_linear_e4m3w(cx, mx, w8, mw, b, M, N, K, outs["e4m3w"])
     qs.qs_sd4_linear_e4m3(x8, mx8, w8, mw, b, M, N, K, outs["e4m3"])
     qs.qs_sd4_linear_wdec(cx, mx, wdec, b, M, N, K, outs["wdec"])
+    out_tiles = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    qs.qs_sd4_linear_e4m3_tiles(x8, qs.sd4_scale_tiles(mx8, False), w8,
+                                qs.sd4_scale_tiles(mw, True), b, M, N, K, out_tiles)
     rows = I.salient_rows(M, cfg.seed)
     rt = torch.tensor(rows, dtype=torch.int32, device="cuda")
     codes2, meta2 = qs.sd4_quant_decomp(x, rt)
@@ -269,6 +272,8 @@ def test_full_size_sd4_every_element():
     ref16 = outs["codes"].view(torch.int16)
     assert torch.equal(outs["e4m3w"].view(torch.int16), ref16), "e4m3-weight form"
     assert torch.equal(outs["e4m3"].view(torch.int16), ref16), "e4m3 form"
+    assert torch.equal(out_tiles.view(torch.int16), ref16), "e4m3 form with scale tiles"
+    del out_tiles
     plain = torch.ones(M, dtype=torch.bool, device="cuda")
     plain[rt.long()] = False
     assert torch.equal(outd.view(torch.int16)[plain], ref16[plain]), \

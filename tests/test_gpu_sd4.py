@@ -373,3 +373,53 @@ def test_sd4_output_only_16_byte_aligned():
             qs.qs_sd4_linear_e4m3(x8, mx8, w8, mw, d["bias"].cuda(), M, N, K, o)
         torch.cuda.synchronize()
         assert torch.equal(o.view(torch.int16), out.view(torch.int16)), fn
+
+
+def _tiles_want(e, rows, K, weights):
+    """The scale tiles from the oracle's block exponents, by the layout the
+    header states (group of 128 / 192 rows padded to 128 / 256, 512-byte
+    blocks, row r and block j at 512 (r / 128) + 16 (r % 32) + 4 ((r % 128) / 32) + j)."""
+    group, slots = (192, 256) if weights else (128, 128)
+    groups = 2 * -(-rows // 384) if weights else -(-rows // 128)
+    kbs = K // 128
+    out = np.zeros(groups * kbs * slots * 4, np.uint8)
+    for row in range(rows):
+        g, r = divmod(row, group)
+        for kb in range(kbs):
+            base = (g * kbs + kb) * slots * 4 + 512 * (r // 128) + 16 * (r % 32) + 4 * ((r % 128) // 32)
+            for j in range(4):
+                out[base + j] = (int(e[row, 4 * kb + j]) + 127) & 0xFF
+    return out
+
+
+@pytest.mark.parametrize("rows,K,weights", [(1, 256, 0), (129, 512, 0), (300, 768, 0),
+                                            (16, 256, 1), (385, 512, 1), (200, 1280, 1)])
+def test_sd4_scale_tiles_layout(rows, K, weights):
+    d = I.make_shape(seed=rows + K + weights, M=rows, K=K, N=16, bits=4, outlier_factor=30.0)
+    _, meta = qs.sd4_quant(d["x"].cuda())
+    tiles = qs.sd4_scale_tiles(meta, bool(weights))
+    torch.cuda.synchronize()
+    _, e, _ = S.quantize_rows(I.bf16_bits(d["x"]))
+    assert tiles.numel() == qs.qs_sd4_scale_tiles_bytes(rows, K, weights)
+    assert np.array_equal(tiles.cpu().numpy(), _tiles_want(e, rows, K, weights))
+
+
+@pytest.mark.parametrize("M,N,K", [(127, 272, 256), (300, 768, 768), (513, 528, 1280),
+                                   (1, 16, 256), (129, 2320, 512)])
+def test_sd4_linear_e4m3_tiles_identical(M, N, K):
+    """Scales loaded as pre-arranged tiles: bit-identical to the e4m3 GEMM
+    that converts block words in the kernel (and so to the codes form, which
+    the tests above compare with the oracle)."""
+    d = I.make_shape(seed=7 * M + N, M=M, K=K, N=N, bits=4, outlier_factor=30.0)
+    x, w, b = d["x"].cuda(), d["w"].cuda(), d["bias"].cuda()
+    x8, mx = qs.sd4_quant_e4m3(x)
+    cw, mw = qs.sd4_quant(w)
+    w8 = qs.sd4_decode_e4m3(cw, mw)
+    out8 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    qs.qs_sd4_linear_e4m3(x8, mx, w8, mw, b, M, N, K, out8)
+    outt = torch.full((M, N), 3, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+    qs.qs_sd4_linear_e4m3_tiles(x8, qs.sd4_scale_tiles(mx, False), w8,
+                                qs.sd4_scale_tiles(mw, True), b, M, N, K, outt)
+    torch.cuda.synchronize()
+    assert qs.qs_device_error() == 0
+    assert torch.equal(outt.view(torch.int16), out8.view(torch.int16))
