@@ -45,7 +45,8 @@ def _inputs(M: int):
 
 def main(argv=None) -> None:
     p = argparse.ArgumentParser()
-    p.add_argument("case", choices=["sd4_gemm_e4m3", "sd4_gemm_codes", "sd4_quant_e4m3",
+    p.add_argument("case", choices=["sd4_gemm_e4m3", "sd4_gemm_e4m3_tiles", "sd4_gemm_codes",
+                                    "sd4_quant_e4m3",
                                     "gbs_update", "gelu", "gemm_w8a8", "gemm_w4a8",
                                     "gemm_bgr", "quant", "gemm"])
     p.add_argument("--tokens", type=int, default=None)
@@ -59,7 +60,7 @@ def main(argv=None) -> None:
     a = p.parse_args(argv)
     qs.load()
     torch.cuda.init()
-    if a.case in ("sd4_gemm_e4m3", "sd4_gemm_codes"):
+    if a.case in ("sd4_gemm_e4m3", "sd4_gemm_e4m3_tiles", "sd4_gemm_codes"):
         M = a.tokens or 4096
         x, w, b = _inputs(M)
         cw, mw = qs.sd4_quant(w)
@@ -68,6 +69,11 @@ def main(argv=None) -> None:
             x8, mx = qs.sd4_quant_e4m3(x)
             w8 = qs.sd4_decode_e4m3(cw, mw)
             run = lambda: qs.qs_sd4_linear_e4m3(x8, mx, w8, mw, b, M, N, K, out)  # noqa: E731
+        elif a.case == "sd4_gemm_e4m3_tiles":
+            x8, mx = qs.sd4_quant_e4m3(x)
+            w8 = qs.sd4_decode_e4m3(cw, mw)
+            xt, wt = qs.sd4_scale_tiles(mx, False), qs.sd4_scale_tiles(mw, True)
+            run = lambda: qs.qs_sd4_linear_e4m3_tiles(x8, xt, w8, wt, b, M, N, K, out)  # noqa: E731
         else:
             cx, mx = qs.sd4_quant(x)
             run = lambda: qs.qs_sd4_linear(cx, mx, cw, mw, b, M, N, K, out)  # noqa: E731
