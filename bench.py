@@ -438,6 +438,24 @@ def time_layer(qs, torch, x, wp, ws, bias, bits, alpha, stream, steps=5, warmup=
     return q, g, out
 
 
+def time_quant_alone(qs, torch, x, bx, alpha, x_flags, stream, launches=20, warmup=3):
+    """Mean CUDA-event time (ms) of the activation kernel launched back to back
+    on its own (no GEMM between launches: none of the GEMM's output lines are
+    still being written back from L2 while it streams x)."""
+    M, K = x.shape
+    xp = torch.empty((M, qs.packed_cols(K, bx, x_flags)), dtype=torch.uint8, device=x.device)
+    xs = torch.empty((M,), dtype=torch.float32, device=x.device)
+    for _ in range(warmup):
+        qs.qs_quant_act(x, M, K, bx, alpha, x_flags, xp, xs, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(launches):
+        qs.qs_quant_act(x, M, K, bx, alpha, x_flags, xp, xs, stream)
+    e1.record(stream)
+    stream.synchronize()
+    return e0.elapsed_time(e1) / launches
+
+
 def all_configs(qs, torch, I, dev, stream):
     """Per-configuration throughput on one GPU (every seeded synthetic shape)."""
     res = {}
@@ -867,6 +885,8 @@ def main():
     ms_per_step, value = comb["ms_per_step"], comb["value"]
 
     ref_rows = out[::1009].clone()  # the device step's output, to check the end-to-end one
+    quant_alone_ms = combine_ranks([time_quant_alone(qs, torch, x, bx, alpha, x_flags, stream)],
+                                   1, ops_per_step, world, dev)["times_ms"][0]
     # ---- end to end through the same C ABI calls, inputs and result in pinned host memory
     x_host = d["x"].pin_memory()
     out_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
@@ -993,7 +1013,15 @@ def main():
                                "algorithmic_bytes": quant_bytes,
                                "algorithmic_bytes_rule": "M*(2K + K*b/8 + 4), b the code width",
                                "stored_bytes": stored_bytes,
-                               "peak_source": f"{src}: hbm_gbs"},
+                               "peak_source": f"{src}: hbm_gbs",
+                               "alone": {
+                                   "ms": quant_alone_ms,
+                                   "achieved": quant_bytes / (quant_alone_ms * 1e-3) / 1e9,
+                                   "frac": quant_bytes / (quant_alone_ms * 1e-3) / 1e9
+                                           / pk["hbm_gbs"],
+                                   "note": "the same kernel launched back to back on its own; "
+                                           "in the step it follows the GEMM, whose last output "
+                                           "lines are written back from L2 while it runs"}},
             "act_code_layouts": layouts,
             "kernels_ms": {"quant": quant_ms, "gemm": gemm_ms},
             "kernels_ms_median": {"quant": statistics.median(quant_each),
