@@ -20,10 +20,12 @@
 // pipe idled between stages).
 // Warp roles: 0 TMA producer (codes every stage, block words every two
 // stages, the decoded weights when given), 1 TMEM allocation and the MMA
-// issuer (per stage: three tcgen05.cp of the stage's scales into TMEM, then
-// four MMAs of K = 32 that select scale byte j = 0..3), 2-5 epilogue, then
-// the decode warps: codes -> e4m3 bytes through an 8-byte per-dialect level
-// table and `prmt`, block words -> scale bytes in the tcgen05.cp layout.
+// issuer (per stage: the tcgen05.cp of the stage's scales into TMEM, then
+// four MMAs of K = 32 per N-half that select scale byte j = 0..3), 2-5
+// epilogue (2-9 with wide tiles), then the decode warps: codes -> e4m3 bytes
+// through an 8-byte per-dialect level table and `prmt`, block words -> scale
+// bytes in the tcgen05.cp layout.  With pre-arranged scales (TILES) the
+// producer bulk-copies them with the operands and there are no decode warps.
 //
 // Scale layout (the one tcgen05.cp.32x128b.warpx4 expects): 512 bytes per
 // 128 rows, row m's four scale bytes (K-blocks 0..3 of the stage) at
