@@ -204,16 +204,16 @@ struct MBars {
   __device__ uint32_t acc_empty(int b) const { return at(2 * P + 2 * T + 2 * U + 2 + b); }
 };
 
-// Tile order: bands of `group` N-tiles of `bn` columns, every M-tile inside a
+// Tile order: bands of `group` N-tiles of `bn` columns (M-tiles of `bm` rows), every M-tile inside a
 // band (N fastest within it), so the tiles the CTAs hold at one time share a
 // few MB of activations and weights in L2 and each weight band is read from
 // HBM once (kGroupN; see its note).
-__device__ __forceinline__ void tile_origin(int t, int m_tiles, int n_tiles, int group, int bn,
-                                            int& m0, int& n0) {
+__device__ __forceinline__ void tile_origin(int t, int m_tiles, int n_tiles, int group, int bm,
+                                            int bn, int& m0, int& n0) {
   const int per_group = group * m_tiles;
   const int g = t / per_group, r = t - g * per_group;
   const int gn = min(group, n_tiles - g * group);  // N-tiles in this band
-  m0 = (r / gn) * BM;
+  m0 = (r / gn) * bm;
   n0 = (g * group + r % gn) * bn;
 }
 
@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC, WIDE, TILES>::kThreads, 1)
       uint32_t ph = 0, mph = 0, pho = 0;
       for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
         int m0, n0;
-        tile_origin(t, m_tiles, n_tiles, C::kGroup, C::kBN, m0, n0);
+        tile_origin(t, m_tiles, n_tiles, C::kGroup, BM, C::kBN, m0, n0);
         for (int kb = 0, kbw = 0; kb < kblocks; ++kb, kbw = (kbw + 1 == kb_wrap ? 0 : kbw + 1)) {
           // kbw: the weights' K-block; kb_wrap is even, so both stay in step
           // with the two-stage block-word slots
@@ -414,7 +414,7 @@ __global__ void __launch_bounds__(MCfg<ADEC, BDEC, WIDE, TILES>::kThreads, 1)
       const int buf = it % C::kAccBufs;
       const uint32_t aph = (it / C::kAccBufs) & 1;
       int m0, n0;
-      tile_origin(t, m_tiles, n_tiles, C::kGroup, C::kBN, m0, n0);
+      tile_origin(t, m_tiles, n_tiles, C::kGroup, BM, C::kBN, m0, n0);
       asm volatile("bar.sync 1, %0;" ::"n"(kEpiT) : "memory");
       for (int i = et; i < C::kBN; i += kEpiT) {
         const int n = n0 + i;

@@ -405,7 +405,7 @@ def test_sd4_scale_tiles_layout(rows, K, weights):
 
 
 @pytest.mark.parametrize("M,N,K", [(127, 272, 256), (300, 768, 768), (513, 528, 1280),
-                                   (1, 16, 256), (129, 2320, 512)])
+                                   (1, 16, 256), (129, 2320, 512), (4097, 2320, 256)])
 def test_sd4_linear_e4m3_tiles_identical(M, N, K):
     """Scales loaded as pre-arranged tiles: bit-identical to the e4m3 GEMM
     that converts block words in the kernel (and so to the codes form, which
