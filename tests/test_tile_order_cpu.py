@@ -28,7 +28,10 @@ def tile_origin(t, m_tiles, n_tiles, band):
     return t // n_tiles, t % n_tiles
 
 
-@pytest.mark.parametrize("band", [0, BAND_N, 9, 1])
+# 18 and 9: the integer GEMM's bands of 256- and 512-column tiles; 36 and 18
+# are also the SD4 GEMM's bands of 192- and 384-column tiles (its tile_origin
+# is the same map with the band given per form)
+@pytest.mark.parametrize("band", [0, BAND_N, 9, 36, 1])
 def test_tile_order_is_a_bijection(band):
     for m_tiles, n_tiles in itertools.product(range(1, 40), range(1, 80)):
         seen = set()
