@@ -49,7 +49,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--e2e-steps", type=int, default=3)
-    p.add_argument("--e2e-chunks", type=int, default=8,
+    p.add_argument("--e2e-chunks", type=int, default=16,
                    help="token chunks of the end-to-end step: the host->device copy, the layer "
                         "and the device->host copy of consecutive chunks overlap on 3 streams")
     p.add_argument("--no-cpu-baseline", action="store_true")
